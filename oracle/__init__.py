@@ -1,0 +1,222 @@
+"""CPU oracle for the simulated-communicator collectives -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may import this
+package. The product (the CUDA library and its Python binding) never imports, links or calls it.
+
+This module only marshals numpy arrays into ``liboracle.so`` (built from ``oracle.cpp``), where the
+definitions live. bf16 arrays are passed as ``numpy.uint16`` bit patterns.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+DTYPE_CODES = {"int32": 0, "fp32": 1, "bf16": 2}
+OP_CODES = {"sum": 0, "min": 1, "max": 2, "avg": 3}
+ACC_CODES = {"exact": 0, "rankfold": 1}
+NP_DTYPES = {"int32": np.int32, "fp32": np.float32, "bf16": np.uint16}
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        # ORACLE_LIB points at another build of oracle.cpp (the mutation tests plant mistakes in a
+        # copy and check that the pins catch them).
+        path = os.environ.get("ORACLE_LIB") or _build.build()
+        L = ctypes.CDLL(path)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        pp = ctypes.POINTER(ctypes.c_void_p)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        sigs = {
+            "oracle_allreduce": [i32, pp, pp, sz, i32, i32, i32],
+            "oracle_reduce": [i32, pp, vp, sz, i32, i32, i32, i32],
+            "oracle_broadcast": [i32, vp, pp, sz, i32, i32],
+            "oracle_reduce_scatter": [i32, pp, pp, sz, i32, i32, i32],
+            "oracle_allgather": [i32, pp, pp, sz, i32],
+            "oracle_alltoall": [i32, pp, pp, sz, i32],
+            "oracle_alltoallv": [i32, pp, pp, i64p, i32, i64p],
+            "oracle_ring_allreduce": [i32, pp, pp, sz, i32, i32],
+            "oracle_ring_reduce_scatter": [i32, pp, pp, sz, i32, i32],
+            "oracle_ring_allgather": [i32, pp, pp, sz, i32],
+            "oracle_ring_reduce": [i32, pp, vp, sz, i32, i32, i32],
+            "oracle_ring_broadcast": [i32, vp, pp, sz, i32, i32],
+            "oracle_ring_alltoall": [i32, pp, pp, sz, i32],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.oracle_float_to_bf16.argtypes = [ctypes.c_float]
+        L.oracle_float_to_bf16.restype = ctypes.c_uint16
+        L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_float.restype = ctypes.c_float
+        L.oracle_ring_segment.argtypes = [sz, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.oracle_ring_segment.restype = None
+        _LIB = L
+    return _LIB
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name}: arguments outside the oracle's definitions")
+
+
+def _arr(x, dtype):
+    a = np.ascontiguousarray(x)
+    if a.dtype != NP_DTYPES[dtype]:
+        raise TypeError(f"expected {NP_DTYPES[dtype]} for {dtype}, got {a.dtype}")
+    return a
+
+
+def _ptrs(arrays):
+    return (ctypes.c_void_p * len(arrays))(*[a.ctypes.data for a in arrays])
+
+
+def _outs(p, count, dtype):
+    return [np.zeros(count, dtype=NP_DTYPES[dtype]) for _ in range(p)]
+
+
+def allreduce(inputs, dtype, op, acc="exact"):
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    outs = _outs(len(ins), n, dtype)
+    _check(lib().oracle_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op],
+                                  ACC_CODES[acc]), "allreduce")
+    return outs
+
+
+def reduce(inputs, dtype, op, root, acc="exact", out=None):
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    res = np.zeros(n, dtype=NP_DTYPES[dtype]) if out is None else out
+    _check(lib().oracle_reduce(len(ins), _ptrs(ins), res.ctypes.data, n, DTYPE_CODES[dtype], OP_CODES[op], root,
+                               ACC_CODES[acc]), "reduce")
+    return res
+
+
+def broadcast(root_input, p, dtype, root):
+    x = _arr(root_input, dtype)
+    outs = _outs(p, x.size, dtype)
+    _check(lib().oracle_broadcast(p, x.ctypes.data, _ptrs(outs), x.size, DTYPE_CODES[dtype], root), "broadcast")
+    return outs
+
+
+def reduce_scatter(inputs, dtype, op, acc="exact"):
+    ins = [_arr(x, dtype) for x in inputs]
+    p, n = len(ins), ins[0].size
+    outs = _outs(p, n // p, dtype)
+    _check(lib().oracle_reduce_scatter(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op],
+                                       ACC_CODES[acc]), "reduce_scatter")
+    return outs
+
+
+def allgather(shards, dtype):
+    ins = [_arr(x, dtype) for x in shards]
+    p = len(ins)
+    n = p * ins[0].size
+    outs = _outs(p, n, dtype)
+    _check(lib().oracle_allgather(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype]), "allgather")
+    return outs
+
+
+def alltoall(inputs, dtype):
+    ins = [_arr(x, dtype) for x in inputs]
+    p, n = len(ins), ins[0].size
+    outs = _outs(p, n, dtype)
+    _check(lib().oracle_alltoall(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype]), "alltoall")
+    return outs
+
+
+def alltoallv(inputs, counts, dtype):
+    """counts: [p][p] int64, c[i][j] elements from source i to destination j. Returns
+    (outputs sized Σ_i c_ij per destination j, recv_counts)."""
+    ins = [_arr(x, dtype) for x in inputs]
+    p = len(ins)
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.int64).reshape(p, p))
+    recv = c.sum(axis=0)
+    outs = [np.zeros(int(recv[j]), dtype=NP_DTYPES[dtype]) for j in range(p)]
+    rc = np.zeros(p, dtype=np.int64)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    _check(lib().oracle_alltoallv(p, _ptrs(ins), _ptrs(outs), c.ctypes.data_as(i64p), DTYPE_CODES[dtype],
+                                  rc.ctypes.data_as(i64p)), "alltoallv")
+    return outs, rc
+
+
+def ring_allreduce(inputs, dtype, op):
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    outs = _outs(len(ins), n, dtype)
+    _check(lib().oracle_ring_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
+           "ring_allreduce")
+    return outs
+
+
+def ring_reduce_scatter(inputs, dtype, op):
+    ins = [_arr(x, dtype) for x in inputs]
+    p, n = len(ins), ins[0].size
+    outs = _outs(p, n // p, dtype)
+    _check(lib().oracle_ring_reduce_scatter(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
+           "ring_reduce_scatter")
+    return outs
+
+
+def ring_allgather(shards, dtype):
+    ins = [_arr(x, dtype) for x in shards]
+    p = len(ins)
+    n = p * ins[0].size
+    outs = _outs(p, n, dtype)
+    _check(lib().oracle_ring_allgather(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype]), "ring_allgather")
+    return outs
+
+
+def ring_reduce(inputs, dtype, op, root):
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    res = np.zeros(n, dtype=NP_DTYPES[dtype])
+    _check(lib().oracle_ring_reduce(len(ins), _ptrs(ins), res.ctypes.data, n, DTYPE_CODES[dtype], OP_CODES[op],
+                                    root), "ring_reduce")
+    return res
+
+
+def ring_broadcast(root_input, p, dtype, root):
+    x = _arr(root_input, dtype)
+    outs = _outs(p, x.size, dtype)
+    _check(lib().oracle_ring_broadcast(p, x.ctypes.data, _ptrs(outs), x.size, DTYPE_CODES[dtype], root),
+           "ring_broadcast")
+    return outs
+
+
+def ring_alltoall(inputs, dtype):
+    ins = [_arr(x, dtype) for x in inputs]
+    p, n = len(ins), ins[0].size
+    outs = _outs(p, n, dtype)
+    _check(lib().oracle_ring_alltoall(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype]), "ring_alltoall")
+    return outs
+
+
+def float_to_bf16(x):
+    L = lib()
+    a = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([L.oracle_float_to_bf16(float(v)) for v in a], dtype=np.uint16)
+
+
+def double_to_bf16(x):
+    L = lib()
+    a = np.asarray(x, dtype=np.float64).ravel()
+    return np.array([L.oracle_double_to_bf16(float(v)) for v in a], dtype=np.uint16)
+
+
+def bf16_to_float(h):
+    return (np.asarray(h, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def ring_segment(n, p, k):
+    b, e = ctypes.c_size_t(), ctypes.c_size_t()
+    lib().oracle_ring_segment(n, p, k, ctypes.byref(b), ctypes.byref(e))
+    return b.value, e.value

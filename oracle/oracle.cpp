@@ -1,0 +1,514 @@
+/*
+ * Oracle for the simulated-communicator collectives: a plain, slow, obviously correct CPU
+ * implementation of what every collective computes.
+ *
+ * THIS IS TEST INFRASTRUCTURE. Only the tests, the smoke check and the benchmark's CPU-baseline leg
+ * load it. It shares no code, header, table or helper with the CUDA library, and the CUDA library
+ * never calls it. Each function follows the passage cited above it.
+ *
+ * Pages cited:
+ *   [Atlas]  "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives)
+ *   [Primer] "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
+ *            (charlestar.github.io/2026/08/20/gpu-collective-communication)
+ *
+ * Conventions (our own; the pages write the data layouts only as figures):
+ *   - p ranks; rank r's buffer is in[r] / out[r], a host pointer.
+ *   - n is the per-rank full-buffer element count: the AllReduce in/out size, the ReduceScatter
+ *     input size, the AllGather output size and the All-to-All send size ([Primer] section
+ *     "先统一通信量的记号", where B is the full logical tensor).
+ *   - dtype 0 = int32, 1 = fp32, 2 = bf16 (stored as the upper 16 bits of an IEEE fp32).
+ *   - op 0 = sum, 1 = min, 2 = max, 3 = avg (sum times 1/p).
+ *   - acc 0 = EXACT: sums in double in rank order, rounded once to the output type.
+ *     acc 1 = RANKFOLD: the fp32 left fold acc = x0; acc = acc + x1; ... in rank order.
+ *
+ * Return value: 0 on success, -1 on an argument the definitions do not cover.
+ *
+ * Parity pins: every function here is pinned by a CPU test against the pages' worked example,
+ * figure layouts, identities, closed forms or brute force. The ring schedule itself (as opposed to
+ * its result) is "parity unpinned": the page's p = 4 trace is garbled, so the schedule follows the
+ * reading that makes rank r own block r.
+ */
+#include <cfenv>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+enum { DT_INT32 = 0, DT_FP32 = 1, DT_BF16 = 2 };
+enum { OP_SUM = 0, OP_MIN = 1, OP_MAX = 2, OP_AVG = 3 };
+enum { ACC_EXACT = 0, ACC_RANKFOLD = 1 };
+
+size_t elem_size(int dtype) { return dtype == DT_BF16 ? 2 : 4; }
+
+bool valid_dtype(int dtype) { return dtype == DT_INT32 || dtype == DT_FP32 || dtype == DT_BF16; }
+
+/* ---- IEEE conversions written from the definitions -------------------------------------------- */
+
+float bits_to_float(uint32_t u) {
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+uint32_t float_to_bits(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return u;
+}
+
+/* A bf16 value is the top half of an fp32 bit pattern. */
+float bf16_to_float(uint16_t h) { return bits_to_float(uint32_t(h) << 16); }
+
+/* fp32 -> bf16, round to nearest, ties to even, on the 16 dropped bits. NaN stays NaN. */
+uint16_t float_to_bf16_rne(float f) {
+    uint32_t u = float_to_bits(f);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0) return uint16_t((u >> 16) | 0x40);
+    uint32_t lower = u & 0xFFFFu;
+    uint32_t upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1;  // carry may reach inf: correct
+    return uint16_t(upper);
+}
+
+/* double -> bf16 with a single rounding (no detour through fp32): round |x| to the bf16 grid
+ * (8 significant bits for normal numbers, spacing 2^-133 below 2^-126), ties to even. */
+uint16_t double_to_bf16_rne(double x) {
+    if (std::isnan(x)) return 0x7FC0;
+    bool neg = std::signbit(x);
+    double a = std::fabs(x);
+    double r;
+    if (a == 0.0) {
+        r = 0.0;
+    } else {
+        int e;
+        std::frexp(a, &e);                 // a = m * 2^e, m in [0.5, 1)
+        int q = e - 8;                     // 8 significant bits -> quantum 2^(e-8)
+        if (q < -133) q = -133;            // subnormal spacing
+        double scaled = std::ldexp(a, -q);
+        double rounded = std::nearbyint(scaled);  // default rounding mode: ties to even
+        r = std::ldexp(rounded, q);
+    }
+    float f = float(r);                    // exact: r has at most 8 significant bits, or overflows to inf
+    if (r >= 0x1p128) f = INFINITY;
+    uint16_t h = uint16_t(float_to_bits(f) >> 16);
+    return neg ? uint16_t(h | 0x8000u) : h;
+}
+
+/* ---- element access ---------------------------------------------------------------------------- */
+
+double load_as_double(const void* buf, int dtype, size_t i) {
+    if (dtype == DT_INT32) return double(static_cast<const int32_t*>(buf)[i]);
+    if (dtype == DT_FP32) return double(static_cast<const float*>(buf)[i]);
+    return double(bf16_to_float(static_cast<const uint16_t*>(buf)[i]));
+}
+
+float load_as_float(const void* buf, int dtype, size_t i) {
+    if (dtype == DT_FP32) return static_cast<const float*>(buf)[i];
+    return bf16_to_float(static_cast<const uint16_t*>(buf)[i]);
+}
+
+void store_float(void* buf, int dtype, size_t i, float v) {
+    if (dtype == DT_FP32)
+        static_cast<float*>(buf)[i] = v;
+    else
+        static_cast<uint16_t*>(buf)[i] = float_to_bf16_rne(v);
+}
+
+void store_double_rounded_once(void* buf, int dtype, size_t i, double v) {
+    if (dtype == DT_FP32)
+        static_cast<float*>(buf)[i] = float(v);  // C conversion rounds to nearest even
+    else
+        static_cast<uint16_t*>(buf)[i] = double_to_bf16_rne(v);
+}
+
+void copy_element(const void* src, size_t si, void* dst, size_t di, int dtype) {
+    size_t d = elem_size(dtype);
+    std::memcpy(static_cast<char*>(dst) + di * d, static_cast<const char*>(src) + si * d, d);
+}
+
+/* ---- the reduction operator ⊕ ----------------------------------------------------------------- */
+
+/* min/max as a left fold: the earlier operand is kept on ties. */
+template <typename T>
+T apply_minmax(int op, T a, T b) {
+    if (op == OP_MIN) return (b < a) ? b : a;
+    return (a < b) ? b : a;
+}
+
+/* Reduce element i over the given rank order and store it to out at index oi.
+ * [Atlas] §1.3/§1.4: out[i] = in_0[i] ⊕ in_1[i] ⊕ ... ⊕ in_{p-1}[i] (⊕ = sum, min or max).
+ * AVG is sum times 1/p: [Atlas] §1.4 notes that DDP takes the mean as a sum followed by a division
+ * by the world size. */
+void reduce_element(int p, const void* const* in, const std::vector<int>& order, size_t i, int dtype,
+                    int op, int acc, void* out, size_t oi) {
+    if (dtype == DT_INT32) {
+        const int32_t* first = static_cast<const int32_t*>(in[order[0]]);
+        if (op == OP_SUM) {
+            uint32_t s = uint32_t(first[i]);  // two's-complement wraparound
+            for (int k = 1; k < p; ++k) s += uint32_t(static_cast<const int32_t*>(in[order[k]])[i]);
+            static_cast<int32_t*>(out)[oi] = int32_t(s);
+        } else {
+            int32_t v = first[i];
+            for (int k = 1; k < p; ++k) v = apply_minmax(op, v, static_cast<const int32_t*>(in[order[k]])[i]);
+            static_cast<int32_t*>(out)[oi] = v;
+        }
+        return;
+    }
+    if (op == OP_MIN || op == OP_MAX) {
+        float v = load_as_float(in[order[0]], dtype, i);
+        for (int k = 1; k < p; ++k) v = apply_minmax(op, v, load_as_float(in[order[k]], dtype, i));
+        store_float(out, dtype, oi, v);  // v is one of the inputs: exact in any precision
+        return;
+    }
+    if (acc == ACC_EXACT) {
+        double s = load_as_double(in[order[0]], dtype, i);
+        for (int k = 1; k < p; ++k) s += load_as_double(in[order[k]], dtype, i);
+        if (op == OP_AVG) s = s / double(p);
+        store_double_rounded_once(out, dtype, oi, s);
+    } else {
+        volatile float s = load_as_float(in[order[0]], dtype, i);
+        for (int k = 1; k < p; ++k) s = s + load_as_float(in[order[k]], dtype, i);
+        float v = s;
+        if (op == OP_AVG) {
+            volatile float scale = 1.0f / float(p);
+            v = v * scale;
+        }
+        store_float(out, dtype, oi, v);
+    }
+}
+
+bool valid_common(int p, int dtype) { return p >= 1 && valid_dtype(dtype); }
+
+bool valid_reduce_args(int p, int dtype, int op, int acc) {
+    if (!valid_common(p, dtype)) return false;
+    if (op < OP_SUM || op > OP_AVG) return false;
+    if (dtype == DT_INT32 && op == OP_AVG) return false;
+    return acc == ACC_EXACT || acc == ACC_RANKFOLD;
+}
+
+std::vector<int> rank_order(int p) {
+    std::vector<int> o(p);
+    for (int r = 0; r < p; ++r) o[r] = r;
+    return o;
+}
+
+int mod(long long a, int p) { return int(((a % p) + p) % p); }
+
+/* Ring segment k of an n-element buffer: p equal chunks of ceil(n/p) elements, the last ones
+ * shorter (possibly empty). [Primer] "Ring AllReduce 怎样拆成两半" assumes B splits evenly into
+ * p chunks; when it does, this is exactly that split. */
+void ring_segment(size_t n, int p, int k, size_t* begin, size_t* end) {
+    size_t seg = (n + size_t(p) - 1) / size_t(p);
+    size_t b = size_t(k) * seg, e = b + seg;
+    if (b > n) b = n;
+    if (e > n) e = n;
+    *begin = b;
+    *end = e;
+}
+
+/* Accumulator of the ring emulation: fp32 for fp32/bf16, wrapping uint32 for int32 sums, the
+ * exact int32 for int32 min/max. */
+struct RingAcc {
+    int dtype, op;
+    std::vector<float> f;
+    std::vector<int32_t> i;
+    void resize(size_t n) {
+        if (dtype == DT_INT32) i.assign(n, 0); else f.assign(n, 0.0f);
+    }
+    void load(const void* src, size_t k) {
+        if (dtype == DT_INT32) i[k] = static_cast<const int32_t*>(src)[k];
+        else f[k] = load_as_float(src, dtype, k);
+    }
+    /* this[k] = received ⊕ own, received first (it carries the earlier ranks of the chain). */
+    void combine(float received_f, int32_t received_i, const void* own, size_t k) {
+        if (dtype == DT_INT32) {
+            int32_t o = static_cast<const int32_t*>(own)[k];
+            if (op == OP_SUM) i[k] = int32_t(uint32_t(received_i) + uint32_t(o));
+            else i[k] = apply_minmax(op, received_i, o);
+        } else {
+            volatile float r = received_f;
+            float o = load_as_float(own, dtype, k);
+            if (op == OP_MIN || op == OP_MAX) f[k] = apply_minmax(op, float(r), o);
+            else { volatile float s = r + o; f[k] = s; }
+        }
+    }
+    /* Final value of a fully reduced element: AVG scales in fp32, then one rounding to dtype. */
+    void store_final(int p, void* out, size_t oi, size_t k) const {
+        if (dtype == DT_INT32) { static_cast<int32_t*>(out)[oi] = i[k]; return; }
+        float v = f[k];
+        if (op == OP_AVG) { volatile float scale = 1.0f / float(p); v = v * scale; }
+        store_float(out, dtype, oi, v);
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+/* ===================== plain definitions ======================================================= */
+
+/* [Atlas] §1.4 AllReduce: out_r[i] = ⊕_{r'} in_{r'}[i], identical on every rank r.
+ * [Primer] "AllReduce：Partial 变成 Replicated". */
+int oracle_allreduce(int p, const void* const* in, void* const* out, size_t n, int dtype, int op, int acc) {
+    if (!valid_reduce_args(p, dtype, op, acc)) return -1;
+    std::vector<int> order = rank_order(p);
+    std::vector<char> tmp(elem_size(dtype));
+    for (size_t i = 0; i < n; ++i) {
+        reduce_element(p, in, order, i, dtype, op, acc, tmp.data(), 0);
+        for (int r = 0; r < p; ++r) copy_element(tmp.data(), 0, out[r], i, dtype);
+    }
+    return 0;
+}
+
+/* [Atlas] §1.3 Reduce: out_root[i] = ⊕_r in_r[i]; only the root's buffer receives it (the other
+ * ranks' outputs are shown empty and are left untouched here). Root is a rank index ([Atlas] §0). */
+int oracle_reduce(int p, const void* const* in, void* out_root, size_t n, int dtype, int op, int root, int acc) {
+    if (!valid_reduce_args(p, dtype, op, acc) || root < 0 || root >= p) return -1;
+    std::vector<int> order = rank_order(p);
+    for (size_t i = 0; i < n; ++i) reduce_element(p, in, order, i, dtype, op, acc, out_root, i);
+    return 0;
+}
+
+/* [Atlas] §1.1 Broadcast: the root's n-element buffer is copied to every rank, root included. */
+int oracle_broadcast(int p, const void* in_root, void* const* out, size_t n, int dtype, int root) {
+    if (!valid_common(p, dtype) || root < 0 || root >= p) return -1;
+    for (int r = 0; r < p; ++r)
+        for (size_t i = 0; i < n; ++i) copy_element(in_root, i, out[r], i, dtype);
+    return 0;
+}
+
+/* [Atlas] §1.5 ReduceScatter: each rank holds [p·m] (m = n/p); the reduction of block r goes to
+ * rank r: out_r[k] = ⊕_q in_q[r·m + k]. */
+int oracle_reduce_scatter(int p, const void* const* in, void* const* out, size_t n, int dtype, int op, int acc) {
+    if (!valid_reduce_args(p, dtype, op, acc) || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p);
+    std::vector<int> order = rank_order(p);
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < m; ++k) reduce_element(p, in, order, size_t(r) * m + k, dtype, op, acc, out[r], k);
+    return 0;
+}
+
+/* [Atlas] §1.2 AllGather: p shards of m = n/p elements are concatenated in rank order and every
+ * rank receives the [p·m] result: out_r[q·m + k] = in_q[k]. */
+int oracle_allgather(int p, const void* const* in, void* const* out, size_t n, int dtype) {
+    if (!valid_common(p, dtype) || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p);
+    for (int r = 0; r < p; ++r)
+        for (int q = 0; q < p; ++q)
+            for (size_t k = 0; k < m; ++k) copy_element(in[q], k, out[r], size_t(q) * m + k, dtype);
+    return 0;
+}
+
+/* [Atlas] §1.6 AllToAll: the [src][dst] block matrix is transposed. Block j of source i lands as
+ * block i of destination j: out_j[i·m + k] = in_i[j·m + k], m = n/p. */
+int oracle_alltoall(int p, const void* const* in, void* const* out, size_t n, int dtype) {
+    if (!valid_common(p, dtype) || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p);
+    for (int i = 0; i < p; ++i)
+        for (int j = 0; j < p; ++j)
+            for (size_t k = 0; k < m; ++k) copy_element(in[i], size_t(j) * m + k, out[j], size_t(i) * m + k, dtype);
+    return 0;
+}
+
+/* [Primer] "Ragged All-to-All：MoE 的真实输入通常不等长": c_ij elements go from source i to
+ * destination j; counts -> prefix-sum offsets -> payload exchange. Source i packs its blocks in
+ * destination order, destination j stores them in source order:
+ *   sdispl_i[j] = Σ_{j'<j} c_ij',  rdispl_j[i] = Σ_{i'<i} c_i'j,
+ *   out_j[rdispl_j[i] + k] = in_i[sdispl_i[j] + k] for k < c_ij.
+ * counts is row-major [p][p]; recv_counts (may be null) gets Σ_i c_ij per destination j.
+ * Negative counts are outside the definition. */
+int oracle_alltoallv(int p, const void* const* in, void* const* out, const int64_t* counts, int dtype,
+                     int64_t* recv_counts) {
+    if (!valid_common(p, dtype)) return -1;
+    for (int a = 0; a < p * p; ++a)
+        if (counts[a] < 0) return -1;
+    for (int i = 0; i < p; ++i) {
+        for (int j = 0; j < p; ++j) {
+            int64_t sdispl = 0;
+            for (int jj = 0; jj < j; ++jj) sdispl += counts[i * p + jj];
+            int64_t rdispl = 0;
+            for (int ii = 0; ii < i; ++ii) rdispl += counts[ii * p + j];
+            for (int64_t k = 0; k < counts[i * p + j]; ++k)
+                copy_element(in[i], size_t(sdispl + k), out[j], size_t(rdispl + k), dtype);
+        }
+    }
+    if (recv_counts) {
+        for (int j = 0; j < p; ++j) {
+            int64_t s = 0;
+            for (int i = 0; i < p; ++i) s += counts[i * p + j];
+            recv_counts[j] = s;
+        }
+    }
+    return 0;
+}
+
+/* ===================== ring schedule emulation ================================================== */
+/* [Atlas] §2.2: ranks form the ring r0 -> r1 -> ... -> r_{p-1} -> r0, every buffer is cut into p
+ * chunks, a ring reduce-scatter of p-1 steps is followed by a ring all-gather of p-1 steps.
+ * Reading of the page's garbled p = 4 trace: at reduce-scatter step s (1..p-1) rank r sends its
+ * current chunk (r - s) mod p to rank r+1, which adds its own input to it; after step p-1 rank r
+ * holds the fully reduced chunk r, matching ReduceScatter's owner rule ([Atlas] §1.5). At
+ * all-gather step s (1..p-1) rank r forwards chunk (r - s + 1) mod p to rank r+1. The partials
+ * travel in fp32 for fp32 and bf16 data; an owner rounds once when its chunk is complete. */
+
+static int ring_reduce_scatter_phase(int p, const void* const* in, size_t n, int dtype, int op,
+                                     std::vector<RingAcc>& part) {
+    part.assign(p, RingAcc{dtype, op, {}, {}});
+    for (int r = 0; r < p; ++r) part[r].resize(n);
+    /* Step 1 sends raw inputs: seed every rank's partial with its own input. */
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < n; ++k) part[r].load(in[r], k);
+    /* The receiver's partial of a chunk it has not reduced yet is its raw input, so "receive and
+     * add" overwrites the chunk with received ⊕ own. */
+    for (int s = 1; s <= p - 1; ++s) {
+        /* messages of this step: rank r sends chunk (r - s) mod p to rank r+1 */
+        std::vector<std::vector<float>> msg_f(p);
+        std::vector<std::vector<int32_t>> msg_i(p);
+        std::vector<int> msg_chunk(p);
+        for (int r = 0; r < p; ++r) {
+            int c = mod(r - s, p);
+            size_t b, e;
+            ring_segment(n, p, c, &b, &e);
+            int dst = mod(r + 1, p);
+            msg_chunk[dst] = c;
+            if (dtype == DT_INT32) msg_i[dst].assign(part[r].i.begin() + b, part[r].i.begin() + e);
+            else msg_f[dst].assign(part[r].f.begin() + b, part[r].f.begin() + e);
+        }
+        for (int q = 0; q < p; ++q) {
+            int c = msg_chunk[q];
+            size_t b, e;
+            ring_segment(n, p, c, &b, &e);
+            for (size_t k = b; k < e; ++k)
+                part[q].combine(dtype == DT_INT32 ? 0.0f : msg_f[q][k - b], dtype == DT_INT32 ? msg_i[q][k - b] : 0,
+                                in[q], k);
+        }
+    }
+    return 0;
+}
+
+/* Ring AllReduce = ring ReduceScatter then ring AllGather ([Atlas] §0 second identity, §2.2). */
+int oracle_ring_allreduce(int p, const void* const* in, void* const* out, size_t n, int dtype, int op) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD)) return -1;
+    std::vector<RingAcc> part;
+    ring_reduce_scatter_phase(p, in, n, dtype, op, part);
+    /* owners round their complete chunk into their own output */
+    for (int r = 0; r < p; ++r) {
+        size_t b, e;
+        ring_segment(n, p, r, &b, &e);
+        for (size_t k = b; k < e; ++k) part[r].store_final(p, out[r], k, k);
+    }
+    /* all-gather: step s, rank r forwards chunk (r - s + 1) mod p of its output to rank r+1 */
+    size_t d = elem_size(dtype);
+    for (int s = 1; s <= p - 1; ++s) {
+        std::vector<std::vector<char>> msg(p);
+        std::vector<int> msg_chunk(p);
+        for (int r = 0; r < p; ++r) {
+            int c = mod(r - s + 1, p);
+            size_t b, e;
+            ring_segment(n, p, c, &b, &e);
+            int dst = mod(r + 1, p);
+            msg_chunk[dst] = c;
+            const char* src = static_cast<const char*>(out[r]);
+            msg[dst].assign(src + b * d, src + e * d);
+        }
+        for (int q = 0; q < p; ++q) {
+            size_t b, e;
+            ring_segment(n, p, msg_chunk[q], &b, &e);
+            if (e > b) std::memcpy(static_cast<char*>(out[q]) + b * d, msg[q].data(), (e - b) * d);
+        }
+    }
+    return 0;
+}
+
+/* Ring ReduceScatter: the reduce-scatter phase alone; rank r outputs its complete chunk r. */
+int oracle_ring_reduce_scatter(int p, const void* const* in, void* const* out, size_t n, int dtype, int op) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD) || n % size_t(p) != 0) return -1;
+    std::vector<RingAcc> part;
+    ring_reduce_scatter_phase(p, in, n, dtype, op, part);
+    size_t m = n / size_t(p);
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < m; ++k) part[r].store_final(p, out[r], k, size_t(r) * m + k);
+    return 0;
+}
+
+/* Ring AllGather: rank r starts with its shard as chunk r of its output; at step s it forwards
+ * chunk (r - s + 1) mod p to rank r+1. n is the output element count (m = n/p per shard). */
+int oracle_ring_allgather(int p, const void* const* in, void* const* out, size_t n, int dtype) {
+    if (!valid_common(p, dtype) || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p), d = elem_size(dtype);
+    for (int r = 0; r < p; ++r)
+        if (m) std::memcpy(static_cast<char*>(out[r]) + size_t(r) * m * d, in[r], m * d);
+    for (int s = 1; s <= p - 1; ++s) {
+        std::vector<std::vector<char>> msg(p);
+        std::vector<int> msg_chunk(p);
+        for (int r = 0; r < p; ++r) {
+            int c = mod(r - s + 1, p);
+            int dst = mod(r + 1, p);
+            msg_chunk[dst] = c;
+            const char* src = static_cast<const char*>(out[r]) + size_t(c) * m * d;
+            msg[dst].assign(src, src + m * d);
+        }
+        for (int q = 0; q < p; ++q)
+            if (m) std::memcpy(static_cast<char*>(out[q]) + size_t(msg_chunk[q]) * m * d, msg[q].data(), m * d);
+    }
+    return 0;
+}
+
+/* Ring Reduce (our reading: the pages define rings only for AllReduce/ReduceScatter/AllGather):
+ * a chain root+1 -> root+2 -> ... -> root. The first rank sends its raw input, each next rank adds
+ * its own input to what it received, the root rounds the complete result. */
+int oracle_ring_reduce(int p, const void* const* in, void* out_root, size_t n, int dtype, int op, int root) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD) || root < 0 || root >= p) return -1;
+    RingAcc held{dtype, op, {}, {}};
+    held.resize(n);
+    int first = mod(root + 1, p);
+    for (size_t k = 0; k < n; ++k) held.load(in[first], k);
+    for (int h = 1; h <= p - 1; ++h) {
+        int q = mod(root + 1 + h, p);
+        RingAcc received = held;  // the message from the previous rank of the chain
+        for (size_t k = 0; k < n; ++k)
+            held.combine(dtype == DT_INT32 ? 0.0f : received.f[k], dtype == DT_INT32 ? received.i[k] : 0, in[q], k);
+    }
+    for (size_t k = 0; k < n; ++k) held.store_final(p, out_root, k, k);
+    return 0;
+}
+
+/* Ring Broadcast (our reading): a chain root -> root+1 -> ... -> root-1 of p-1 hops; the root's
+ * own output receives the root's input too. */
+int oracle_ring_broadcast(int p, const void* in_root, void* const* out, size_t n, int dtype, int root) {
+    if (!valid_common(p, dtype) || root < 0 || root >= p) return -1;
+    size_t d = elem_size(dtype);
+    if (n) std::memcpy(out[root], in_root, n * d);
+    for (int h = 1; h <= p - 1; ++h) {
+        int src = mod(root + h - 1, p), dst = mod(root + h, p);
+        if (n) std::memcpy(out[dst], out[src], n * d);
+    }
+    return 0;
+}
+
+/* Ring All-to-All (our reading): the p-1 step shift exchange. Step 0 keeps the own block; at step s
+ * rank r sends its block (r+s) mod p to rank (r+s) mod p. */
+int oracle_ring_alltoall(int p, const void* const* in, void* const* out, size_t n, int dtype) {
+    if (!valid_common(p, dtype) || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p), d = elem_size(dtype);
+    for (int s = 0; s <= p - 1; ++s)
+        for (int r = 0; r < p; ++r) {
+            int j = mod(r + s, p);
+            if (m)
+                std::memcpy(static_cast<char*>(out[j]) + size_t(r) * m * d,
+                            static_cast<const char*>(in[r]) + size_t(j) * m * d, m * d);
+        }
+    return 0;
+}
+
+/* ===================== helpers the tests pin directly ============================================ */
+
+uint16_t oracle_float_to_bf16(float f) { return float_to_bf16_rne(f); }
+uint16_t oracle_double_to_bf16(double x) { return double_to_bf16_rne(x); }
+float oracle_bf16_to_float(uint16_t h) { return bf16_to_float(h); }
+
+/* The ring segment rule, exposed so a test can pin it against the page's even split. */
+void oracle_ring_segment(size_t n, int p, int k, size_t* begin, size_t* end) { ring_segment(n, p, k, begin, end); }
+
+}  // extern "C"
