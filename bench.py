@@ -1,0 +1,442 @@
+"""Benchmark: effective HBM GB/s of the simulated-communicator collectives on one B200.
+
+Workload (the DP gradient-bucket configuration): a communicator of p = 8 ranks in one GPU, each
+rank holding a 25 Mi-element bucket (26,214,400 elements; 100 MiB fp32, 50 MiB bf16) of N(0, 1e-3)
+values. One step runs every row of the hot path once on it:
+  direct AllReduce AVG fp32 and bf16, ring AllReduce AVG fp32 and bf16 (1 MiB chunks),
+  direct and ring Reduce SUM (root 2), Broadcast (root 2), ReduceScatter SUM, AllGather of the
+  bucket's shards, equal All-to-All, and All-to-Allv of the bucket as 6,400 rows of 4,096 elements
+  routed by a seeded top-2 / Zipf(1.1) router over 64 experts.
+value = Σ (minimum HBM bytes of each call: every input read once, every output written once) /
+device time of the step, summed over ranks (replicas) for N GPUs.
+
+Prints one JSON line. ``--impl reference`` times the CPU oracle on a bounded sample instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "effective HBM GB/s per collective vs ~8 TB/s peak (1×B200); oracle CPU GB/s"
+P = 8
+N_BUCKET = 26_214_400
+HIDDEN = 4096
+ROOT_RANK = 2
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="simcomm", choices=["simcomm", "reference"])
+    ap.add_argument("--n", type=int, default=N_BUCKET, help="elements per rank (default: the 25 Mi bucket)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# the step
+
+def moe_rows_counts(n, p):
+    """Rows of HIDDEN elements per (source, destination) for a bucket of n elements per rank."""
+    from collective_communication_primitives_b200 import synth as S
+    rows = n // HIDDEN
+    tokens = rows // 2
+    return S.moe_counts(p=p, tokens=tokens, experts=64, topk=2, zipf_s=1.1, hidden=1)
+
+
+class Workload:
+    def __init__(self, n, device):
+        import numpy as np
+        import torch
+
+        from collective_communication_primitives_b200 import synth as S
+        self.n, self.p = n, P
+        self.m = n // P
+        f32 = [S.normal(f"dp.fp32.rank{r}", n, 1e-3, "fp32") for r in range(P)]
+        b16 = [S.normal(f"dp.bf16.rank{r}", n, 1e-3, "bf16") for r in range(P)]
+        self.host_f32 = [torch.from_numpy(x).pin_memory() for x in f32]
+        self.host_b16 = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in b16]
+        self.x32 = [h.to(device) for h in self.host_f32]
+        self.x16 = [h.to(device) for h in self.host_b16]
+        self.ar32 = [torch.empty(n, dtype=torch.float32, device=device) for _ in range(P)]
+        self.ar16 = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.out32 = [torch.empty(n, dtype=torch.float32, device=device) for _ in range(P)]
+        self.red = [None] * P
+        self.red[ROOT_RANK] = torch.empty(n, dtype=torch.float32, device=device)
+        self.rs = [torch.empty(self.m, dtype=torch.float32, device=device) for _ in range(P)]
+        self.shards = [x[:self.m] for x in self.x32]
+        rows = moe_rows_counts(n, P)
+        self.counts_host = rows * HIDDEN
+        self.counts = torch.from_numpy(self.counts_host).to(device)
+        self.v_elems = int(self.counts_host.sum())
+        self.v_send = [x[:int(self.counts_host[i].sum())] for i, x in enumerate(self.x32)]
+        self.v_recv = [torch.empty(int(self.counts_host[:, j].sum()), dtype=torch.float32, device=device)
+                       for j in range(P)]
+        self.rows = rows
+
+
+def build_step(comm, wl):
+    """[(name, kernel, callable, effective bytes, kernel-model bytes)] for one step."""
+    from collective_communication_primitives_b200 import bytemodel as BM
+    n, p = wl.n, wl.p
+    ops = []
+
+    def add(name, kernel, fn, eff, kb):
+        ops.append((name, kernel, fn, eff, kb))
+
+    for algo in ("direct", "ring"):
+        kern = "ring" if algo == "ring" else None
+        add(f"allreduce_avg_fp32_{algo}", kern or "direct_reduce",
+            lambda a=algo: comm.allreduce(wl.x32, wl.ar32, op="avg", algo=a),
+            BM.direct_hbm_bytes("allreduce", p, n, 4),
+            BM.ring_hbm_bytes("allreduce", p, n, 4) if algo == "ring" else BM.direct_hbm_bytes("allreduce", p, n, 4))
+        add(f"allreduce_avg_bf16_{algo}", kern or "direct_reduce",
+            lambda a=algo: comm.allreduce(wl.x16, wl.ar16, op="avg", algo=a),
+            BM.direct_hbm_bytes("allreduce", p, n, 2),
+            BM.ring_hbm_bytes("allreduce", p, n, 2, 4) if algo == "ring" else BM.direct_hbm_bytes("allreduce", p, n, 2))
+        add(f"reduce_sum_fp32_{algo}", kern or "direct_reduce",
+            lambda a=algo: comm.reduce(wl.x32, wl.red, ROOT_RANK, op="sum", algo=a),
+            BM.direct_hbm_bytes("reduce", p, n, 4),
+            BM.ring_hbm_bytes("reduce", p, n, 4) if algo == "ring" else BM.direct_hbm_bytes("reduce", p, n, 4))
+        add(f"broadcast_fp32_{algo}", kern or "copy_engine",
+            lambda a=algo: comm.broadcast(wl.x32, wl.out32, ROOT_RANK, algo=a),
+            BM.direct_hbm_bytes("broadcast", p, n, 4),
+            BM.ring_hbm_bytes("broadcast", p, n, 4) if algo == "ring" else BM.direct_hbm_bytes("broadcast", p, n, 4))
+        add(f"reduce_scatter_sum_fp32_{algo}", kern or "direct_reduce",
+            lambda a=algo: comm.reduce_scatter(wl.x32, wl.rs, op="sum", algo=a),
+            BM.direct_hbm_bytes("reduce_scatter", p, n, 4),
+            BM.ring_hbm_bytes("reduce_scatter", p, n, 4) if algo == "ring"
+            else BM.direct_hbm_bytes("reduce_scatter", p, n, 4))
+        add(f"allgather_fp32_{algo}", kern or "copy_engine",
+            lambda a=algo: comm.allgather(wl.shards, wl.out32, algo=a),
+            BM.direct_hbm_bytes("allgather", p, n, 4),
+            BM.ring_hbm_bytes("allgather", p, n, 4) if algo == "ring" else BM.direct_hbm_bytes("allgather", p, n, 4))
+        add(f"alltoall_fp32_{algo}", kern or "copy_engine",
+            lambda a=algo: comm.alltoall(wl.x32, wl.out32, algo=a),
+            BM.direct_hbm_bytes("alltoall", p, n, 4), BM.direct_hbm_bytes("alltoall", p, n, 4))
+        add(f"alltoallv_fp32_{algo}", kern or "copy_engine",
+            lambda a=algo: comm.alltoallv(wl.v_send, wl.v_recv, wl.counts, algo=a),
+            BM.direct_hbm_bytes("alltoallv", p, 0, 4, moved_elems=wl.v_elems),
+            BM.direct_hbm_bytes("alltoallv", p, 0, 4, moved_elems=wl.v_elems))
+    return ops
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def time_device(ops, steps, warmup, stream):
+    """Warm up, then time exactly `steps` steps with events on the launching stream; also per-op
+    events inside the timed region."""
+    import torch
+    for _ in range(warmup):
+        for op in ops:
+            op[2]()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
+          for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for s in range(steps):
+        for i, op in enumerate(ops):
+            ev[s][i][0].record(stream)
+            op[2]()
+            ev[s][i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    per_op = [sum(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)) / steps for i in range(len(ops))]
+    return total_ms, per_op
+
+
+def time_e2e(comm, wl, ops, steps, warmup, stream):
+    """Same step through the public API with host buffers: pinned inputs copied in, the step run,
+    both AllReduce results copied out, all inside the timed region."""
+    import torch
+    out_host32 = [torch.empty(wl.n, dtype=torch.float32).pin_memory() for _ in range(P)]
+    out_host16 = [torch.empty(wl.n, dtype=torch.bfloat16).pin_memory() for _ in range(P)]
+
+    def one():
+        for r in range(P):
+            wl.x32[r].copy_(wl.host_f32[r], non_blocking=True)
+            wl.x16[r].copy_(wl.host_b16[r], non_blocking=True)
+        for op in ops:
+            op[2]()
+        for r in range(P):
+            out_host32[r].copy_(wl.ar32[r], non_blocking=True)
+            out_host16[r].copy_(wl.ar16[r], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    h2d = P * wl.n * (4 + 2)
+    d2h = P * wl.n * (4 + 2)
+    return start.elapsed_time(end), h2d, d2h
+
+
+# ---------------------------------------------------------------------------------------------
+# the oracle as a CPU baseline (and as the reference arm)
+
+def oracle_inputs(n):
+    """The step's inputs for the oracle, from the same seeded recipe, generated on the host."""
+    from collective_communication_primitives_b200 import synth as S
+    p = P
+    x32 = [S.normal(f"dp.fp32.rank{r}", n, 1e-3, "fp32") for r in range(p)]
+    x16 = [S.normal(f"dp.bf16.rank{r}", n, 1e-3, "bf16") for r in range(p)]
+    counts = moe_rows_counts(n, p) * HIDDEN
+    vsend = [x32[i][:int(counts[i].sum())] for i in range(p)]
+    return {"n": n, "x32": x32, "x16": x16, "counts": counts, "vsend": vsend}
+
+
+def oracle_step(inp):
+    """Run the oracle over every row of the step once; returns (seconds, effective bytes)."""
+    import oracle as O
+    from collective_communication_primitives_b200 import bytemodel as BM
+    p, n = P, inp["n"]
+    m = n // p
+    x32, x16, counts, vsend = inp["x32"], inp["x16"], inp["counts"], inp["vsend"]
+    t0 = time.perf_counter()
+    O.allreduce(x32, "fp32", "avg", acc="rankfold")
+    O.allreduce(x16, "bf16", "avg", acc="rankfold")
+    O.ring_allreduce(x32, "fp32", "avg")
+    O.ring_allreduce(x16, "bf16", "avg")
+    O.reduce(x32, "fp32", "sum", ROOT_RANK, acc="rankfold")
+    O.ring_reduce(x32, "fp32", "sum", ROOT_RANK)
+    O.broadcast(x32[ROOT_RANK], p, "fp32", ROOT_RANK)
+    O.ring_broadcast(x32[ROOT_RANK], p, "fp32", ROOT_RANK)
+    O.reduce_scatter(x32, "fp32", "sum", acc="rankfold")
+    O.ring_reduce_scatter(x32, "fp32", "sum")
+    O.allgather([x[:m] for x in x32], "fp32")
+    O.ring_allgather([x[:m] for x in x32], "fp32")
+    O.alltoall(x32, "fp32")
+    O.ring_alltoall(x32, "fp32")
+    O.alltoallv(vsend, counts, "fp32")
+    O.alltoallv(vsend, counts, "fp32")
+    secs = time.perf_counter() - t0
+    eff = 2 * (BM.direct_hbm_bytes("allreduce", p, n, 4) + BM.direct_hbm_bytes("allreduce", p, n, 2) +
+               BM.direct_hbm_bytes("reduce", p, n, 4) + BM.direct_hbm_bytes("broadcast", p, n, 4) +
+               BM.direct_hbm_bytes("reduce_scatter", p, n, 4) + BM.direct_hbm_bytes("allgather", p, n, 4) +
+               BM.direct_hbm_bytes("alltoall", p, n, 4) +
+               BM.direct_hbm_bytes("alltoallv", p, 0, 4, moved_elems=int(counts.sum())))
+    return secs, eff
+
+
+CPU_SAMPLE_N = N_BUCKET             # the CPU baseline: one full step (about 10-20 s of CPU work)
+REF_SAMPLE_N = N_BUCKET // 8        # one reference-arm step: 1/8 of the bucket
+
+
+def cpu_baseline():
+    secs, eff = oracle_step(oracle_inputs(CPU_SAMPLE_N))
+    return {"value": eff / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one step of every row on the full bucket (p={P}, n={CPU_SAMPLE_N} per rank), "
+                      f"single-threaded C++ oracle, {secs:.1f} s"}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = oracle_inputs(REF_SAMPLE_N)
+    for _ in range(args.warmup):
+        oracle_step(inp)
+    tot_s, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        s, b = oracle_step(inp)
+        tot_s += s
+        tot_b += b
+    v = tot_b / tot_s / 1e9
+    sample = f"each step: every row on a 1/8-size bucket (p={P}, n={REF_SAMPLE_N} per rank), single-threaded C++ oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"DP gradient bucket, p={P} ranks x {REF_SAMPLE_N} elements (1/8 sample)",
+                   "p": P, "n_per_rank": REF_SAMPLE_N},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+# ---------------------------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from collective_communication_primitives_b200 import simcomm as SC
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    device = f"cuda:{local}"
+    stream = torch.cuda.current_stream()
+
+    wl = Workload(args.n, device)
+    comm = SC.SimComm(P)
+    comm.set_option("chunk_bytes", 1 << 20)
+    ops = build_step(comm, wl)
+    eff_per_step = sum(o[3] for o in ops)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = comm.launch_count()
+    with ClockSampler(local) as clk:
+        total_ms, per_op = time_device(ops, args.steps, args.warmup, stream)
+    launches = comm.launch_count() - launches0 - args.warmup * len(ops)
+    clocks = clk.summary()
+    torch.cuda.synchronize()
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(comm, wl, ops, max(3, args.steps // 4), 1, stream)
+        e_steps = max(3, args.steps // 4)
+        if world > 1:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * eff_per_step * e_steps / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    hbm, peak_kind = peaks()
+    ms_per_step = total_ms / args.steps
+    value = world * eff_per_step / (ms_per_step / 1e3) / 1e9
+    per_op_json = {}
+    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
+        per_op_json[name] = {"ms": round(ms, 4), "effective_GBps": round(eff / (ms / 1e3) / 1e9, 1),
+                             "kernel_GBps": round(kb / (ms / 1e3) / 1e9, 1),
+                             "frac_of_measured_peak": round(kb / (ms / 1e3) / 1e9 / hbm, 4)}
+    # the dominant kernel: the kernel family with the largest share of the step's device time
+    fam = {}
+    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
+        f = fam.setdefault(kernel, [0.0, 0, 0])
+        f[0] += ms
+        f[1] += kb
+        f[2] += 1
+    dom = max(fam, key=lambda k: fam[k][0])
+    d_ms, d_bytes, d_launches = fam[dom]
+    achieved = d_bytes / (d_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
+                "traffic": None, "share_of_step": round(d_ms / sum(per_op), 4),
+                "bytes_per_launch": d_bytes // d_launches}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"DP gradient bucket, p={P} ranks x {args.n} elements per rank, every hot-path row "
+                               f"(direct and ring) per step", "p": P, "n_per_rank": args.n,
+                   "chunk_bytes": 1 << 20, "l2": "inputs larger than L2 (100 MiB per rank fp32)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "per_op": per_op_json,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if e2e:
+        out["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(out))
+    comm.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

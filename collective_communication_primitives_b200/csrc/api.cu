@@ -1,0 +1,700 @@
+// Host side of the C ABI declared in include/simcomm.h: communicator lifecycle, options,
+// argument validation, asynchronous error state and dispatch to the kernels.
+//
+// Citations name "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives)
+// as [Atlas] and "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
+// (charlestar.github.io/2026/08/20/gpu-collective-communication) as [Primer].
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "simcomm.h"
+
+using namespace simcomm;
+
+struct sim_comm {
+    int p = 0;
+    int device = 0;
+    int num_sms = 0;
+    DevState* dstate = nullptr;     // device scratch header
+    uint32_t* host_words = nullptr; // host-mapped: [0] status mirror, [1] abort flag
+    uint32_t* dev_words = nullptr;  // device alias of host_words
+    uint32_t* flags = nullptr;      // ring flags
+    size_t flags_cap = 0;           // elements
+    char* stage = nullptr;          // ring partial buffers
+    size_t stage_cap = 0;           // bytes
+    uint32_t epoch = 0;
+    long long chunk_bytes = 1 << 20;
+    long long ring_ctas = 0;
+    long long timeout_ns = 2000000000LL;
+    long long fault_skip_rank = -1;
+    unsigned long long launches = 0;
+    int ring_ctas_max = 0;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+coll_status_t fail(coll_status_t st, const std::string& msg) {
+    g_last_error = msg;
+    return st;
+}
+
+coll_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(COLL_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+size_t dtype_bytes(coll_dtype_t dt) { return dt == COLL_BF16 ? 2 : 4; }
+
+bool valid_dtype(int dt) { return dt == COLL_INT32 || dt == COLL_FP32 || dt == COLL_BF16; }
+
+coll_status_t check_reduce_args(coll_dtype_t dt, coll_op_t op) {
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if (op < COLL_SUM || op > COLL_AVG) return fail(COLL_ERR_INVALID_ARG, "unknown reduction op");
+    if (dt == COLL_INT32 && op == COLL_AVG) return fail(COLL_ERR_UNSUPPORTED, "AVG is not defined for int32");
+    return COLL_OK;
+}
+
+coll_status_t check_algo(coll_algo_t algo) {
+    if (algo != COLL_ALGO_DIRECT && algo != COLL_ALGO_RING) return fail(COLL_ERR_INVALID_ARG, "unknown algorithm");
+    return COLL_OK;
+}
+
+// The sticky state: an abort requested on the host, or an asynchronous error already reported.
+coll_status_t check_usable(sim_comm* c) {
+    if (!c) return fail(COLL_ERR_INVALID_ARG, "null communicator");
+    volatile uint32_t* hw = c->host_words;
+    if (hw[1] != 0u) return fail(COLL_ERR_ABORTED, "communicator was aborted; call sim_comm_reset");
+    if (hw[0] != 0u)
+        return fail(coll_status_t(hw[0]), "communicator has an asynchronous error; call sim_comm_reset");
+    return COLL_OK;
+}
+
+Ctl make_ctl(sim_comm* c) {
+    Ctl ctl;
+    ctl.status = &c->dstate->status;
+    ctl.host_status = c->dev_words;
+    ctl.abort_flag = c->dev_words + 1;
+    return ctl;
+}
+
+// ---- buffer validation -------------------------------------------------------------------------
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+    bool out;
+    int rank;
+};
+
+bool overlap(const Range& a, const Range& b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// Allowed in-place pairs ([Primer] "In-place 不是“任意让输入输出指向同一地址”"): an output may
+// coincide with or contain the SAME rank's input in the documented form only.
+enum InPlaceRule { INPLACE_NONE, INPLACE_SAME, INPLACE_RS, INPLACE_AG };
+
+bool allowed_pair(InPlaceRule rule, const Range& out, const Range& in, size_t shard_bytes) {
+    if (out.rank != in.rank) return false;
+    switch (rule) {
+        case INPLACE_SAME: return out.lo == in.lo && out.hi == in.hi;
+        case INPLACE_RS: return out.lo == in.lo + size_t(out.rank) * shard_bytes;  // recv = send + r*m
+        case INPLACE_AG: return in.lo == out.lo + size_t(in.rank) * shard_bytes;   // send = recv + r*m
+        default: return false;
+    }
+}
+
+coll_status_t check_ranges(const std::vector<Range>& rs, InPlaceRule rule, size_t shard_bytes) {
+    for (size_t i = 0; i < rs.size(); ++i) {
+        for (size_t j = i + 1; j < rs.size(); ++j) {
+            const Range& a = rs[i];
+            const Range& b = rs[j];
+            if (!a.out && !b.out) continue;  // inputs may share memory: they are only read
+            if (a.lo == a.hi || b.lo == b.hi || !overlap(a, b)) continue;
+            if (a.out && b.out) return fail(COLL_ERR_INVALID_ARG, "two output buffers overlap");
+            const Range& o = a.out ? a : b;
+            const Range& in = a.out ? b : a;
+            if (!allowed_pair(rule, o, in, shard_bytes))
+                return fail(COLL_ERR_INVALID_ARG, "an output overlaps an input outside the allowed in-place forms");
+        }
+    }
+    return COLL_OK;
+}
+
+coll_status_t check_ptr(const void* p, size_t bytes, size_t elem, const char* what) {
+    if (bytes == 0) return COLL_OK;
+    if (!p) return fail(COLL_ERR_INVALID_ARG, std::string("null ") + what + " pointer");
+    if (reinterpret_cast<uintptr_t>(p) % elem != 0)
+        return fail(COLL_ERR_INVALID_ARG, std::string(what) + " pointer is not element-aligned");
+    return COLL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void fill_ptrs(RankPtrs& rp, const coll_bufs_t& b, int p, bool use_send, bool use_recv) {
+    std::memset(&rp, 0, sizeof(rp));
+    for (int r = 0; r < p; ++r) {
+        rp.send[r] = (use_send && b.send) ? b.send[r] : nullptr;
+        rp.recv[r] = (use_recv && b.recv) ? b.recv[r] : nullptr;
+    }
+}
+
+// ---- scratch -----------------------------------------------------------------------------------
+
+coll_status_t ensure_flags(sim_comm* c, size_t count) {
+    if (count <= c->flags_cap) return COLL_OK;
+    if (c->flags) cudaFree(c->flags);  // synchronises the device: no kernel still uses the old flags
+    c->flags = nullptr;
+    c->flags_cap = 0;
+    cudaError_t e = cudaMalloc(&c->flags, count * sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(ring flags)");
+    e = cudaMemset(c->flags, 0, count * sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(ring flags)");
+    c->flags_cap = count;
+    return COLL_OK;
+}
+
+coll_status_t ensure_stage(sim_comm* c, size_t bytes) {
+    if (bytes <= c->stage_cap) return COLL_OK;
+    if (c->stage) cudaFree(c->stage);
+    c->stage = nullptr;
+    c->stage_cap = 0;
+    cudaError_t e = cudaMalloc(&c->stage, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(ring partial buffers)");
+    c->stage_cap = bytes;
+    return COLL_OK;
+}
+
+uint32_t next_epoch(sim_comm* c) {
+    c->epoch += 1;
+    if (c->epoch == 0) {  // wrapped: old flags could alias a future epoch, so clear them
+        if (c->flags) cudaMemset(c->flags, 0, c->flags_cap * sizeof(uint32_t));
+        c->epoch = 1;
+    }
+    return c->epoch;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- launches ----------------------------------------------------------------------------------
+
+coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                int mode, int root, cudaStream_t s) {
+    DirectReduceArgs a;
+    fill_ptrs(a.ptrs, b, c->p, true, true);
+    a.p = c->p;
+    a.mode = mode;
+    a.root = root;
+    a.n = n;
+    a.seg = (mode == MODE_REDUCE_SCATTER) ? n / size_t(c->p) : n;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(c->p) : 1.0f;
+    a.ctl = make_ctl(c);
+    const size_t d = dtype_bytes(dt);
+    bool vec = true;
+    for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.send[r]);
+    if (mode == MODE_ALLREDUCE)
+        for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.recv[r]);
+    else if (mode == MODE_REDUCE)
+        vec = vec && aligned16(a.ptrs.recv[root]);
+    else {
+        for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.recv[r]);
+        vec = vec && (a.seg * d) % 16 == 0;
+    }
+    a.vec = vec ? 1 : 0;
+    cudaError_t e = launch_direct_reduce(a, dt, op, c->num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "direct reduction launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
+coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_elems, coll_dtype_t dt, int root,
+                       bool use_send_all, cudaStream_t s, const long long* counts = nullptr,
+                       const long long* send_cap = nullptr, const long long* recv_cap = nullptr,
+                       long long* recv_counts = nullptr) {
+    CopyArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, c->p, true, true);
+    if (!use_send_all)
+        for (int r = 0; r < c->p; ++r)
+            if (r != root) a.ptrs.send[r] = nullptr;
+    a.p = c->p;
+    a.kind = kind;
+    a.root = root;
+    a.elem_bytes = int(dtype_bytes(dt));
+    a.blk_elems = blk_elems;
+    a.counts = counts;
+    a.recv_counts_out = recv_counts;
+    for (int r = 0; r < c->p; ++r) {
+        a.send_cap[r] = send_cap ? send_cap[r] : 0;
+        a.recv_cap[r] = recv_cap ? recv_cap[r] : 0;
+    }
+    a.timeout_ns = uint64_t(c->timeout_ns);
+    a.ctl = make_ctl(c);
+    cudaError_t e = launch_copy(a, c->num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
+struct RingPlan {
+    int kind;
+    size_t seg, chunk;
+    uint32_t nch, nsteps, rps;
+    bool needs_stage;
+};
+
+coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, size_t n, coll_dtype_t dt,
+                       coll_op_t op, int root, cudaStream_t s, const long long* counts = nullptr,
+                       const long long* send_cap = nullptr, const long long* recv_cap = nullptr,
+                       long long* recv_counts = nullptr) {
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt);
+    RingArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.p = p;
+    a.kind = pl.kind;
+    a.root = root;
+    a.n = n;
+    a.seg = pl.seg;
+    a.chunk = pl.chunk;
+    a.nch = pl.nch;
+    a.nsteps = pl.nsteps;
+    a.ranks_per_step = pl.rps;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.skip_rank = int(c->fault_skip_rank);
+    a.timeout_ns = uint64_t(c->timeout_ns);
+    a.counts = counts;
+    a.recv_counts_out = recv_counts;
+    for (int r = 0; r < p; ++r) {
+        a.send_cap[r] = send_cap ? send_cap[r] : 0;
+        a.recv_cap[r] = recv_cap ? recv_cap[r] : 0;
+    }
+    a.st = c->dstate;
+    a.ctl = make_ctl(c);
+
+    coll_status_t st;
+    if (pl.kind != RING_ALLTOALL && pl.kind != RING_ALLTOALLV) {
+        st = ensure_flags(c, size_t(pl.nsteps) * pl.rps * pl.nch);
+        if (st != COLL_OK) return st;
+    }
+    if (pl.needs_stage) {
+        a.stage_stride = round_up(n * 4, 256);
+        st = ensure_stage(c, a.stage_stride * size_t(p));
+        if (st != COLL_OK) return st;
+        a.stage = c->stage;
+    }
+    a.flags = c->flags;
+    a.epoch = next_epoch(c);
+
+    // 16-byte hops need every segment and chunk start 16-byte aligned in the element and partial
+    // buffers, and 16-byte aligned bases.
+    const bool chain = (pl.kind == RING_REDUCE || pl.kind == RING_BCAST);  // chunks of [0, n), no segments
+    bool vec = (chain || ((pl.seg * d) % 16 == 0 && (pl.seg * 4) % 16 == 0)) && (pl.chunk * d) % 16 == 0;
+    for (int r = 0; r < p; ++r)
+        vec = vec && (!a.ptrs.send[r] || aligned16(a.ptrs.send[r])) && (!a.ptrs.recv[r] || aligned16(a.ptrs.recv[r]));
+    a.vec = vec ? 1 : 0;
+
+    int ctas = int(c->ring_ctas > 0 ? c->ring_ctas : c->ring_ctas_max);
+    if (pl.kind != RING_ALLTOALLV) {
+        const size_t tasks = size_t(pl.nsteps) * pl.rps * pl.nch;
+        if (tasks < size_t(ctas)) ctas = int(std::max<size_t>(tasks, 1));
+    }
+    cudaError_t e = launch_ring(a, dt, op, ctas, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ring executor launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
+uint32_t chunks_of(size_t seg, size_t chunk) { return uint32_t(std::max<size_t>(1, (seg + chunk - 1) / chunk)); }
+
+long long env_ll(const char* name, long long dflt) {
+    const char* v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    char* end = nullptr;
+    long long x = std::strtoll(v, &end, 0);
+    return (end && *end == 0) ? x : dflt;
+}
+
+coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
+    std::string k(key);
+    if (k == "chunk_bytes") {
+        if (value < 256 || value % 256 != 0 || value > (1LL << 30))
+            return fail(COLL_ERR_INVALID_ARG, "chunk_bytes must be a multiple of 256 in [256, 2^30]");
+        c->chunk_bytes = value;
+    } else if (k == "ring_ctas") {
+        if (value < 0 || value > 65535) return fail(COLL_ERR_INVALID_ARG, "ring_ctas out of range");
+        c->ring_ctas = value;
+    } else if (k == "timeout_ns") {
+        if (value < 1000) return fail(COLL_ERR_INVALID_ARG, "timeout_ns must be at least 1000");
+        c->timeout_ns = value;
+    } else if (k == "fault_skip_rank") {
+        if (value < -1 || value >= c->p) return fail(COLL_ERR_INVALID_ARG, "fault_skip_rank out of range");
+        c->fault_skip_rank = value;
+    } else {
+        return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
+    }
+    return COLL_OK;
+}
+
+}  // namespace
+
+// =================================================================================================
+extern "C" {
+
+const char* sim_comm_last_error(void) { return g_last_error.c_str(); }
+
+const char* coll_status_string(coll_status_t s) {
+    switch (s) {
+        case COLL_OK: return "COLL_OK";
+        case COLL_ERR_INVALID_ARG: return "COLL_ERR_INVALID_ARG";
+        case COLL_ERR_UNSUPPORTED: return "COLL_ERR_UNSUPPORTED";
+        case COLL_ERR_CUDA: return "COLL_ERR_CUDA";
+        case COLL_ERR_TIMEOUT: return "COLL_ERR_TIMEOUT";
+        case COLL_ERR_ABORTED: return "COLL_ERR_ABORTED";
+        case COLL_ERR_OVERFLOW: return "COLL_ERR_OVERFLOW";
+        case COLL_ERR_INTERNAL: return "COLL_ERR_INTERNAL";
+        default: return "COLL_ERR_UNKNOWN";
+    }
+}
+
+sim_comm_t sim_comm_create(int p) {
+    if (p < 1 || p > SIM_COMM_MAX_RANKS) {
+        fail(COLL_ERR_INVALID_ARG, "p must be in [1, 64]");
+        return nullptr;
+    }
+    sim_comm* c = new sim_comm();
+    c->p = p;
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+    if (e == cudaSuccess) e = cudaMalloc(&c->dstate, sizeof(DevState));
+    if (e == cudaSuccess) e = cudaMemset(c->dstate, 0, sizeof(DevState));
+    if (e == cudaSuccess) e = cudaHostAlloc(&c->host_words, 64, cudaHostAllocMapped);
+    if (e == cudaSuccess) {
+        std::memset(c->host_words, 0, 64);
+        e = cudaHostGetDevicePointer(&c->dev_words, c->host_words, 0);
+    }
+    if (e != cudaSuccess) {
+        cuda_fail(e, "sim_comm_create");
+        if (c->dstate) cudaFree(c->dstate);
+        if (c->host_words) cudaFreeHost(c->host_words);
+        delete c;
+        return nullptr;
+    }
+    c->ring_ctas_max = ring_max_ctas(c->num_sms);
+    // Options from the environment; bad values are ignored (the defaults stay).
+    const long long cb = env_ll("SIMCOMM_CHUNK_BYTES", c->chunk_bytes);
+    if (set_option_impl(c, "chunk_bytes", cb) != COLL_OK) c->chunk_bytes = 1 << 20;
+    const long long rc = env_ll("SIMCOMM_RING_CTAS", 0);
+    if (set_option_impl(c, "ring_ctas", rc) != COLL_OK) c->ring_ctas = 0;
+    const long long to = env_ll("SIMCOMM_TIMEOUT_NS", c->timeout_ns);
+    if (set_option_impl(c, "timeout_ns", to) != COLL_OK) c->timeout_ns = 2000000000LL;
+    const long long fr = env_ll("SIMCOMM_FAULT_SKIP_RANK", -1);
+    if (set_option_impl(c, "fault_skip_rank", fr) != COLL_OK) c->fault_skip_rank = -1;
+    g_last_error.clear();
+    return c;
+}
+
+coll_status_t sim_comm_destroy(sim_comm_t c) {
+    if (!c) return COLL_OK;
+    cudaDeviceSynchronize();
+    if (c->flags) cudaFree(c->flags);
+    if (c->stage) cudaFree(c->stage);
+    if (c->dstate) cudaFree(c->dstate);
+    if (c->host_words) cudaFreeHost(c->host_words);
+    delete c;
+    return COLL_OK;
+}
+
+int sim_comm_size(sim_comm_t c) { return c ? c->p : -1; }
+
+coll_status_t sim_comm_set_option(sim_comm_t c, const char* key, long long value) {
+    if (!c || !key) return fail(COLL_ERR_INVALID_ARG, "null communicator or key");
+    return set_option_impl(c, key, value);
+}
+
+coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* value) {
+    if (!c || !key || !value) return fail(COLL_ERR_INVALID_ARG, "null argument");
+    std::string k(key);
+    if (k == "chunk_bytes") *value = c->chunk_bytes;
+    else if (k == "ring_ctas") *value = c->ring_ctas;
+    else if (k == "timeout_ns") *value = c->timeout_ns;
+    else if (k == "fault_skip_rank") *value = c->fault_skip_rank;
+    else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
+    return COLL_OK;
+}
+
+coll_status_t sim_comm_get_async_error(sim_comm_t c, coll_status_t* out) {
+    if (!c || !out) return fail(COLL_ERR_INVALID_ARG, "null argument");
+    *out = coll_status_t(static_cast<volatile uint32_t*>(c->host_words)[0]);
+    return COLL_OK;
+}
+
+coll_status_t sim_comm_abort(sim_comm_t c) {
+    if (!c) return fail(COLL_ERR_INVALID_ARG, "null communicator");
+    static_cast<volatile uint32_t*>(c->host_words)[1] = 1u;
+    return COLL_OK;
+}
+
+coll_status_t sim_comm_reset(sim_comm_t c) {
+    if (!c) return fail(COLL_ERR_INVALID_ARG, "null communicator");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset: device synchronisation");
+    e = cudaMemset(c->dstate, 0, sizeof(DevState));
+    if (e == cudaSuccess && c->flags) e = cudaMemset(c->flags, 0, c->flags_cap * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset");
+    c->epoch = 0;
+    volatile uint32_t* hw = c->host_words;
+    hw[0] = 0u;
+    hw[1] = 0u;
+    return COLL_OK;
+}
+
+coll_status_t sim_comm_launch_count(sim_comm_t c, unsigned long long* out) {
+    if (!c || !out) return fail(COLL_ERR_INVALID_ARG, "null argument");
+    *out = c->launches;
+    return COLL_OK;
+}
+
+// ---- collectives -------------------------------------------------------------------------------
+
+coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, coll_algo_t algo,
+                             coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt), bytes = n * d;
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], bytes, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], bytes, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + bytes, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + bytes, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_SAME, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, b, n, dt, op, MODE_ALLREDUCE, 0, s);
+    RingPlan pl;
+    pl.kind = RING_ALLREDUCE;
+    pl.seg = (n + size_t(p) - 1) / size_t(p);
+    pl.chunk = size_t(c->chunk_bytes) / 4;  // chunk counted in the fp32/int32 partial type
+    pl.nch = chunks_of(pl.seg, pl.chunk);
+    pl.nsteps = uint32_t(2 * (p - 1));
+    pl.rps = uint32_t(p);
+    pl.needs_stage = true;
+    return run_ring(c, b, pl, n, dt, op, 0, s);
+}
+
+coll_status_t coll_reduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, int root,
+                          coll_algo_t algo, coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
+    const int p = c->p;
+    if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), bytes = n * d;
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], bytes, d, "send")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + bytes, false, r});
+    }
+    if ((st = check_ptr(b.recv[root], bytes, d, "root recv")) != COLL_OK) return st;
+    rs.push_back({uintptr_t(b.recv[root]), uintptr_t(b.recv[root]) + bytes, true, root});
+    if ((st = check_ranges(rs, INPLACE_SAME, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Only recv[root] is touched; the kernels are handed a copy of the array with the others null.
+    std::vector<void*> recv(p, nullptr);
+    recv[root] = b.recv[root];
+    coll_bufs_t bb{b.send, recv.data()};
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, bb, n, dt, op, MODE_REDUCE, root, s);
+    RingPlan pl;
+    pl.kind = RING_REDUCE;
+    pl.seg = n;
+    pl.chunk = size_t(c->chunk_bytes) / 4;
+    pl.nch = chunks_of(n, pl.chunk);
+    pl.nsteps = uint32_t(p - 1);
+    pl.rps = 1;
+    pl.needs_stage = true;
+    return run_ring(c, bb, pl, n, dt, op, root, s);
+}
+
+coll_status_t coll_broadcast(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                             coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    const int p = c->p;
+    if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), bytes = n * d;
+    std::vector<Range> rs;
+    if ((st = check_ptr(b.send[root], bytes, d, "root send")) != COLL_OK) return st;
+    rs.push_back({uintptr_t(b.send[root]), uintptr_t(b.send[root]) + bytes, false, root});
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.recv[r], bytes, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + bytes, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_SAME, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    std::vector<const void*> send(p, nullptr);
+    send[root] = b.send[root];
+    coll_bufs_t bb{send.data(), b.recv};
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_copy(c, bb, COPY_BCAST, n, dt, root, false, s);
+    RingPlan pl;
+    pl.kind = RING_BCAST;
+    pl.seg = n;
+    pl.chunk = size_t(c->chunk_bytes) / d;
+    pl.nch = chunks_of(n, pl.chunk);
+    pl.nsteps = uint32_t(p);
+    pl.rps = 1;
+    pl.needs_stage = false;
+    return run_ring(c, bb, pl, n, dt, COLL_SUM, root, s);
+}
+
+coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                  coll_algo_t algo, coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
+    const int p = c->p;
+    if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "ReduceScatter needs n divisible by p");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], n * d, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], m * d, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + n * d, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + m * d, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_RS, m * d)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, b, n, dt, op, MODE_REDUCE_SCATTER, 0, s);
+    RingPlan pl;
+    pl.kind = RING_REDUCE_SCATTER;
+    pl.seg = m;
+    pl.chunk = size_t(c->chunk_bytes) / 4;
+    pl.nch = chunks_of(m, pl.chunk);
+    pl.nsteps = uint32_t(p - 1);
+    pl.rps = uint32_t(p);
+    pl.needs_stage = true;
+    return run_ring(c, b, pl, n, dt, op, 0, s);
+}
+
+coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                             coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    const int p = c->p;
+    if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "AllGather needs n divisible by p");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], m * d, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], n * d, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + m * d, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + n * d, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_AG, m * d)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_copy(c, b, COPY_ALLGATHER, m, dt, 0, true, s);
+    RingPlan pl;
+    pl.kind = RING_ALLGATHER;
+    pl.seg = m;
+    pl.chunk = size_t(c->chunk_bytes) / d;
+    pl.nch = chunks_of(m, pl.chunk);
+    pl.nsteps = uint32_t(p);
+    pl.rps = uint32_t(p);
+    pl.needs_stage = false;
+    return run_ring(c, b, pl, n, dt, COLL_SUM, 0, s);
+}
+
+coll_status_t coll_alltoall(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                            coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    const int p = c->p;
+    if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "All-to-All needs n divisible by p");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], n * d, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], n * d, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + n * d, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + n * d, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_NONE, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (algo == COLL_ALGO_DIRECT || p == 1) return run_copy(c, b, COPY_ALLTOALL, m, dt, 0, true, s);
+    RingPlan pl;
+    pl.kind = RING_ALLTOALL;
+    pl.seg = m;
+    pl.chunk = size_t(c->chunk_bytes) / d;
+    pl.nch = chunks_of(m, pl.chunk);
+    pl.nsteps = uint32_t(p);
+    pl.rps = uint32_t(p);
+    pl.needs_stage = false;
+    return run_ring(c, b, pl, n, dt, COLL_SUM, 0, s);
+}
+
+coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* counts_dev, const long long* send_cap,
+                             const long long* recv_cap, coll_dtype_t dt, coll_algo_t algo, coll_stream_t stream,
+                             long long* recv_counts_dev) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    if (!counts_dev || !send_cap || !recv_cap) return fail(COLL_ERR_INVALID_ARG, "null counts or capacities");
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    if (reinterpret_cast<uintptr_t>(counts_dev) % 8 != 0 ||
+        (recv_counts_dev && reinterpret_cast<uintptr_t>(recv_counts_dev) % 8 != 0))
+        return fail(COLL_ERR_INVALID_ARG, "count arrays must be 8-byte aligned");
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if (send_cap[r] < 0 || recv_cap[r] < 0) return fail(COLL_ERR_INVALID_ARG, "negative capacity");
+        const size_t sb = size_t(send_cap[r]) * d, rb = size_t(recv_cap[r]) * d;
+        if ((st = check_ptr(b.send[r], sb, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], rb, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + sb, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + rb, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_NONE, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (algo == COLL_ALGO_DIRECT || p == 1)
+        return run_copy(c, b, COPY_ALLTOALLV, 0, dt, 0, true, s, counts_dev, send_cap, recv_cap, recv_counts_dev);
+    RingPlan pl;
+    pl.kind = RING_ALLTOALLV;
+    pl.seg = 0;
+    pl.chunk = size_t(c->chunk_bytes) / d;
+    pl.nch = 0;  // from the largest count, on the device
+    pl.nsteps = uint32_t(p);
+    pl.rps = uint32_t(p);
+    pl.needs_stage = false;
+    return run_ring(c, b, pl, 0, dt, COLL_SUM, 0, s, counts_dev, send_cap, recv_cap, recv_counts_dev);
+}
+
+}  // extern "C"

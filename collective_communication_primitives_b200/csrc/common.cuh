@@ -1,0 +1,256 @@
+// Device-side building blocks shared by the simulated-communicator kernels (sm_100a).
+//
+// Memory access helpers are inline PTX: 16-byte streaming loads/stores, L2-coherent loads for
+// data other CTAs produced in the same kernel, gpu-scope acquire/release flags, and the
+// cp.async.bulk (TMA bulk copy) + mbarrier primitives of the copy engine. No multicast form of
+// any bulk copy is used anywhere.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace simcomm {
+
+// ---- element types -------------------------------------------------------------------------------
+
+template <int DT> struct Elem;
+template <> struct Elem<COLL_INT32> { using T = int32_t;  using A = int32_t; static constexpr int kBytes = 4; };
+template <> struct Elem<COLL_FP32>  { using T = float;    using A = float;   static constexpr int kBytes = 4; };
+template <> struct Elem<COLL_BF16>  { using T = uint16_t; using A = float;   static constexpr int kBytes = 2; };
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+// fp32 -> bf16 round-to-nearest-even, via the CUDA intrinsic.
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// The reduction operator: SUM (also used by AVG), MIN, MAX. MIN/MAX are written as a left fold
+// that keeps the earlier operand on ties; int32 SUM wraps around.
+template <int OP> __device__ __forceinline__ float op_f(float a, float b) {
+    if (OP == COLL_MIN) return (b < a) ? b : a;
+    if (OP == COLL_MAX) return (a < b) ? b : a;
+    return a + b;
+}
+template <int OP> __device__ __forceinline__ int32_t op_i(int32_t a, int32_t b) {
+    if (OP == COLL_MIN) return (b < a) ? b : a;
+    if (OP == COLL_MAX) return (a < b) ? b : a;
+    return int32_t(uint32_t(a) + uint32_t(b));
+}
+
+// ---- 16-byte packs: 4 fp32 / 4 int32 / 8 bf16 lanes, widened to the accumulator type ----------
+
+template <int DT> struct Pack16;
+
+template <> struct Pack16<COLL_FP32> {
+    static constexpr int L = 4;
+    using A = float;
+    __device__ static void unpack(const uint4& v, float (&a)[4]) {
+        a[0] = __uint_as_float(v.x); a[1] = __uint_as_float(v.y);
+        a[2] = __uint_as_float(v.z); a[3] = __uint_as_float(v.w);
+    }
+    __device__ static uint4 pack(const float (&a)[4]) {
+        return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]), __float_as_uint(a[3]));
+    }
+};
+
+template <> struct Pack16<COLL_INT32> {
+    static constexpr int L = 4;
+    using A = int32_t;
+    __device__ static void unpack(const uint4& v, int32_t (&a)[4]) {
+        a[0] = int32_t(v.x); a[1] = int32_t(v.y); a[2] = int32_t(v.z); a[3] = int32_t(v.w);
+    }
+    __device__ static uint4 pack(const int32_t (&a)[4]) {
+        return make_uint4(uint32_t(a[0]), uint32_t(a[1]), uint32_t(a[2]), uint32_t(a[3]));
+    }
+};
+
+template <> struct Pack16<COLL_BF16> {
+    static constexpr int L = 8;
+    using A = float;
+    __device__ static void unpack(const uint4& v, float (&a)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            a[2 * k] = bf16_bits_to_float(w[k] & 0xFFFFu);
+            a[2 * k + 1] = bf16_bits_to_float(w[k] >> 16);
+        }
+    }
+    __device__ static uint4 pack(const float (&a)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = uint32_t(float_to_bf16_bits(a[2 * k])) | (uint32_t(float_to_bf16_bits(a[2 * k + 1])) << 16);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <int DT, int OP, typename A, int L>
+__device__ __forceinline__ void fold_into(A (&acc)[L], const A (&x)[L]) {
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+        if constexpr (DT == COLL_INT32) acc[l] = op_i<OP>(acc[l], x[l]);
+        else acc[l] = op_f<OP>(acc[l], x[l]);
+    }
+}
+
+// Element-wise access (plain loads: inputs are not written by the kernel that reads them).
+template <int DT>
+__device__ __forceinline__ typename Elem<DT>::A load_elem(const void* base, size_t e) {
+    if constexpr (DT == COLL_BF16) return bf16_bits_to_float(static_cast<const uint16_t*>(base)[e]);
+    else return static_cast<const typename Elem<DT>::T*>(base)[e];
+}
+template <int DT>
+__device__ __forceinline__ void store_elem(void* base, size_t e, typename Elem<DT>::A v) {
+    if constexpr (DT == COLL_BF16) static_cast<uint16_t*>(base)[e] = float_to_bf16_bits(v);
+    else static_cast<typename Elem<DT>::T*>(base)[e] = v;
+}
+
+// ---- global memory access ------------------------------------------------------------------------
+
+// Streaming 16-byte load of an input (not allocated in L1).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// 16-byte load through L2 only: for data that other CTAs wrote earlier in the same kernel.
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_cg_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint16_t ld_cg_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint8_t ld_cg_u8(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.cg.u8 %0, [%1];" : "=r"(v) : "l"(p));
+    return uint8_t(v);
+}
+
+// ---- flags and status ------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Record the first asynchronous error of the communicator: the device word decides the winner, the
+// winner mirrors the code into the host-mapped word the host polls.
+__device__ __forceinline__ void raise_status(const Ctl& ctl, uint32_t code) {
+    if (atomicCAS(ctl.status, 0u, code) == 0u) {
+        *ctl.host_status = code;
+        __threadfence_system();
+    }
+}
+
+__device__ __forceinline__ bool status_failed(const Ctl& ctl) {
+    return *reinterpret_cast<volatile uint32_t*>(ctl.status) != 0u;
+}
+
+// Bounded wait until *flag == want. Gives up when another CTA failed, when the host asked to
+// abort, after timeout_ns of global time or after kMaxSpin polls; then records the reason and
+// returns false. Called by one thread.
+constexpr uint32_t kMaxSpin = 1u << 26;
+__device__ __forceinline__ bool wait_flag(const Ctl& ctl, const uint32_t* flag, uint32_t want, uint64_t timeout_ns) {
+    if (ld_acquire_gpu(flag) == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1; it < kMaxSpin; ++it) {
+        if (ld_acquire_gpu(flag) == want) return true;
+        if ((it & 15u) == 0u) {
+            if (status_failed(ctl)) return false;
+            if (*ctl.abort_flag != 0u) { raise_status(ctl, COLL_ERR_ABORTED); return false; }
+            if (globaltimer_ns() - t0 > timeout_ns) { raise_status(ctl, COLL_ERR_TIMEOUT); return false; }
+        }
+        if (it > 64u) __nanosleep(64);
+    }
+    raise_status(ctl, COLL_ERR_TIMEOUT);
+    return false;
+}
+
+// ---- TMA bulk copies and mbarriers (shared::cta addresses, no multicast) -------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0u;
+}
+// Global -> shared bulk copy completing on an mbarrier. dst/src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+// Shared -> global bulk copy tracked by bulk groups.
+__device__ __forceinline__ void bulk_s2g(void* gdst, const void* smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(gdst), "r"(smem_u32(smem_src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk group has finished READING shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk group has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Bounded mbarrier wait; false (and a recorded error) if the phase never completes.
+__device__ __forceinline__ bool mbar_wait_bounded(const Ctl& ctl, uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1; it < kMaxSpin; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u && globaltimer_ns() - t0 > timeout_ns) break;
+    }
+    raise_status(ctl, COLL_ERR_INTERNAL);
+    return false;
+}
+
+}  // namespace simcomm

@@ -1,0 +1,106 @@
+// Internal structures shared by the host API (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "simcomm.h"
+
+namespace simcomm {
+
+constexpr int kMaxRanks = SIM_COMM_MAX_RANKS;
+
+// Device scratch header of a communicator (device memory, zero-initialised).
+struct DevState {
+    uint32_t status;    // first asynchronous error (coll_status_t), 0 = OK
+    uint32_t task_ctr;  // ring executor: next task to claim
+    uint32_t done_ctr;  // ring executor: CTAs that left the task loop
+    uint32_t pad;
+};
+
+// What a kernel needs to report errors and notice an abort.
+struct Ctl {
+    uint32_t* status;                  // &DevState::status
+    volatile uint32_t* host_status;    // device alias of a host-mapped word the host polls
+    volatile const uint32_t* abort_flag;  // device alias of the host-mapped abort flag
+};
+
+struct RankPtrs {
+    const void* send[kMaxRanks];
+    void* recv[kMaxRanks];
+};
+
+// ---- direct fused reduction (AllReduce / Reduce / ReduceScatter) ---------------------------------
+enum DirectMode { MODE_ALLREDUCE = 0, MODE_REDUCE = 1, MODE_REDUCE_SCATTER = 2 };
+
+struct DirectReduceArgs {
+    RankPtrs ptrs;
+    int p;
+    int mode;
+    int root;
+    int vec;           // 1: 16-byte packs, 0: element-wise
+    size_t n;          // per-rank full element count
+    size_t seg;        // ReduceScatter: elements per owner (n / p); otherwise n
+    float scale;       // AVG: 1/p; otherwise 1
+    Ctl ctl;
+};
+
+// ---- copy engine (Broadcast / AllGather / All-to-All / All-to-Allv) ------------------------------
+enum CopyKind { COPY_BCAST = 0, COPY_ALLGATHER = 1, COPY_ALLTOALL = 2, COPY_ALLTOALLV = 3 };
+
+struct CopyArgs {
+    RankPtrs ptrs;
+    int p;
+    int kind;
+    int root;
+    int elem_bytes;
+    size_t blk_elems;                  // BCAST: n; ALLGATHER: shard n/p; ALLTOALL: block n/p
+    const long long* counts;           // ALLTOALLV: device [p][p]
+    long long* recv_counts_out;        // ALLTOALLV: device [p] or null
+    long long send_cap[kMaxRanks];     // ALLTOALLV: elements per send buffer
+    long long recv_cap[kMaxRanks];     // ALLTOALLV: elements per recv buffer
+    uint64_t timeout_ns;
+    Ctl ctl;
+};
+
+// ---- ring executor -----------------------------------------------------------------------------
+enum RingKind {
+    RING_ALLREDUCE = 0, RING_REDUCE_SCATTER = 1, RING_ALLGATHER = 2, RING_REDUCE = 3,
+    RING_BCAST = 4, RING_ALLTOALL = 5, RING_ALLTOALLV = 6
+};
+
+struct RingArgs {
+    RankPtrs ptrs;
+    int p;
+    int kind;
+    int root;
+    int vec;                 // 1: vectorised reduce hops (all offsets 16-byte aligned)
+    size_t n;                // per-rank full element count
+    size_t seg;              // elements of one segment (the unit a step moves)
+    size_t chunk;            // elements of one pipelined chunk
+    uint32_t nch;            // chunks per segment (ALLTOALLV: upper bound, refined on device)
+    uint32_t nsteps;         // steps of the schedule
+    uint32_t ranks_per_step; // p for ring steps, 1 for the Reduce/Broadcast chains
+    uint32_t epoch;          // flags equal to epoch mean "done in this call"
+    float scale;
+    int skip_rank;           // fault injection: this rank never signals (-1 = off)
+    uint64_t timeout_ns;
+    char* stage;             // partial buffers, one per rank
+    size_t stage_stride;     // bytes between ranks' partial buffers
+    uint32_t* flags;         // [nsteps][ranks_per_step][nch]
+    DevState* st;
+    const long long* counts; // ALLTOALLV
+    long long* recv_counts_out;
+    long long send_cap[kMaxRanks];
+    long long recv_cap[kMaxRanks];
+    Ctl ctl;
+};
+
+// Launchers (each returns the launch error; grid sizes are decided inside).
+cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, int num_sms, cudaStream_t s);
+cudaError_t launch_copy(const CopyArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStream_t s);
+int ring_max_ctas(int num_sms);
+
+}  // namespace simcomm

@@ -1,0 +1,224 @@
+"""Python binding of the simulated-communicator library ``libsimcomm.so`` (C ABI: include/simcomm.h).
+
+Argument marshalling only: tensors become device pointers and the current CUDA stream becomes the
+stream handle; every step of every collective runs in the library's CUDA kernels. There is no
+fallback: without the built library (``python -m collective_communication_primitives_b200.build``)
+creating a communicator raises.
+"""
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsimcomm.so")
+
+STATUS = {0: "COLL_OK", 1: "COLL_ERR_INVALID_ARG", 2: "COLL_ERR_UNSUPPORTED", 3: "COLL_ERR_CUDA",
+          4: "COLL_ERR_TIMEOUT", 5: "COLL_ERR_ABORTED", 6: "COLL_ERR_OVERFLOW", 7: "COLL_ERR_INTERNAL"}
+OK, INVALID_ARG, UNSUPPORTED, CUDA, TIMEOUT, ABORTED, OVERFLOW, INTERNAL = range(8)
+DTYPES = {"int32": 0, "fp32": 1, "bf16": 2}
+OPS = {"sum": 0, "min": 1, "max": 2, "avg": 3}
+ALGOS = {"direct": 0, "ring": 1}
+
+_lib = None
+
+
+class SimCommError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Bufs(ctypes.Structure):
+    _fields_ = [("send", ctypes.POINTER(ctypes.c_void_p)), ("recv", ctypes.POINTER(ctypes.c_void_p))]
+
+
+def load_library(path=LIB_PATH):
+    """Load libsimcomm.so and declare its signatures. Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m collective_communication_primitives_b200.build`"
+                           " (there is no fallback path)")
+    L = ctypes.CDLL(path)
+    vp, sz, i32, ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
+    llp = ctypes.POINTER(ctypes.c_longlong)
+    st = ctypes.c_int
+    L.sim_comm_create.argtypes = [i32]
+    L.sim_comm_create.restype = vp
+    L.sim_comm_destroy.argtypes = [vp]
+    L.sim_comm_destroy.restype = st
+    L.sim_comm_size.argtypes = [vp]
+    L.sim_comm_size.restype = i32
+    L.sim_comm_last_error.argtypes = []
+    L.sim_comm_last_error.restype = ctypes.c_char_p
+    L.coll_status_string.argtypes = [st]
+    L.coll_status_string.restype = ctypes.c_char_p
+    L.sim_comm_set_option.argtypes = [vp, ctypes.c_char_p, ll]
+    L.sim_comm_set_option.restype = st
+    L.sim_comm_get_option.argtypes = [vp, ctypes.c_char_p, llp]
+    L.sim_comm_get_option.restype = st
+    L.sim_comm_get_async_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    L.sim_comm_get_async_error.restype = st
+    L.sim_comm_abort.argtypes = [vp]
+    L.sim_comm_abort.restype = st
+    L.sim_comm_reset.argtypes = [vp]
+    L.sim_comm_reset.restype = st
+    L.sim_comm_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.sim_comm_launch_count.restype = st
+    L.coll_allreduce.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
+    L.coll_reduce.argtypes = [vp, _Bufs, sz, i32, i32, i32, i32, vp]
+    L.coll_broadcast.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
+    L.coll_reduce_scatter.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
+    L.coll_allgather.argtypes = [vp, _Bufs, sz, i32, i32, vp]
+    L.coll_alltoall.argtypes = [vp, _Bufs, sz, i32, i32, vp]
+    L.coll_alltoallv.argtypes = [vp, _Bufs, vp, llp, llp, i32, i32, vp, vp]
+    for name in ("coll_allreduce", "coll_reduce", "coll_broadcast", "coll_reduce_scatter", "coll_allgather",
+                 "coll_alltoall", "coll_alltoallv"):
+        getattr(L, name).restype = st
+    _lib = L
+    return L
+
+
+def _ptr(x):
+    """Device address of a tensor (or an int address, or None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _dtype_of(t):
+    import torch
+    m = {torch.int32: "int32", torch.float32: "fp32", torch.bfloat16: "bf16"}
+    if t.dtype not in m:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return m[t.dtype]
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class SimComm:
+    """A communicator of p logical ranks on the current CUDA device."""
+
+    def __init__(self, p):
+        self._L = load_library()
+        h = self._L.sim_comm_create(int(p))
+        if not h:
+            raise SimCommError(CUDA, self._L.sim_comm_last_error().decode())
+        self._h = ctypes.c_void_p(h)
+        self.p = int(p)
+
+    # -- lifecycle ---------------------------------------------------------------------------------
+    def close(self):
+        if getattr(self, "_h", None):
+            self._L.sim_comm_destroy(self._h)
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, status):
+        if status != OK:
+            raise SimCommError(status, self._L.sim_comm_last_error().decode())
+
+    def set_option(self, key, value):
+        self._check(self._L.sim_comm_set_option(self._h, key.encode(), int(value)))
+
+    def get_option(self, key):
+        v = ctypes.c_longlong()
+        self._check(self._L.sim_comm_get_option(self._h, key.encode(), ctypes.byref(v)))
+        return v.value
+
+    def async_error(self):
+        s = ctypes.c_int()
+        self._check(self._L.sim_comm_get_async_error(self._h, ctypes.byref(s)))
+        return s.value
+
+    def abort(self):
+        self._check(self._L.sim_comm_abort(self._h))
+
+    def reset(self):
+        self._check(self._L.sim_comm_reset(self._h))
+
+    def launch_count(self):
+        v = ctypes.c_ulonglong()
+        self._check(self._L.sim_comm_launch_count(self._h, ctypes.byref(v)))
+        return v.value
+
+    # -- marshalling -------------------------------------------------------------------------------
+    def _bufs(self, sends, recvs):
+        p = self.p
+        s = (ctypes.c_void_p * p)(*[_ptr(x) for x in sends])
+        r = (ctypes.c_void_p * p)(*[_ptr(x) for x in recvs])
+        self._keep = (s, r)
+        return _Bufs(ctypes.cast(s, ctypes.POINTER(ctypes.c_void_p)), ctypes.cast(r, ctypes.POINTER(ctypes.c_void_p)))
+
+    @staticmethod
+    def _resolve(dtype, tensors):
+        if dtype is not None:
+            return DTYPES[dtype]
+        for t in tensors:
+            if t is not None and not isinstance(t, int):
+                return DTYPES[_dtype_of(t)]
+        raise ValueError("dtype is needed when only raw pointers are given")
+
+    # -- collectives (n follows include/simcomm.h: the per-rank FULL buffer) -----------------------
+    def allreduce(self, sends, recvs, op="sum", algo="direct", n=None, dtype=None, stream=None):
+        n = sends[0].numel() if n is None else n
+        self._check(self._L.coll_allreduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+                                           OPS[op], ALGOS[algo], _stream(stream)))
+
+    def reduce(self, sends, recvs, root, op="sum", algo="direct", n=None, dtype=None, stream=None):
+        n = sends[0].numel() if n is None else n
+        self._check(self._L.coll_reduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends), OPS[op],
+                                        int(root), ALGOS[algo], _stream(stream)))
+
+    def broadcast(self, sends, recvs, root, algo="direct", n=None, dtype=None, stream=None):
+        n = recvs[0].numel() if n is None else n
+        self._check(self._L.coll_broadcast(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, recvs),
+                                           int(root), ALGOS[algo], _stream(stream)))
+
+    def reduce_scatter(self, sends, recvs, op="sum", algo="direct", n=None, dtype=None, stream=None):
+        n = sends[0].numel() if n is None else n
+        self._check(self._L.coll_reduce_scatter(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+                                                OPS[op], ALGOS[algo], _stream(stream)))
+
+    def allgather(self, sends, recvs, algo="direct", n=None, dtype=None, stream=None):
+        n = recvs[0].numel() if n is None else n
+        self._check(self._L.coll_allgather(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, recvs),
+                                           ALGOS[algo], _stream(stream)))
+
+    def alltoall(self, sends, recvs, algo="direct", n=None, dtype=None, stream=None):
+        n = sends[0].numel() if n is None else n
+        self._check(self._L.coll_alltoall(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+                                          ALGOS[algo], _stream(stream)))
+
+    def alltoallv(self, sends, recvs, counts, send_cap=None, recv_cap=None, algo="direct", recv_counts=None,
+                  dtype=None, stream=None):
+        """counts: device int64 [p][p] tensor (c[i][j] elements from i to j). Capacities default to the
+        buffers' sizes."""
+        p = self.p
+        send_cap = [sends[i].numel() for i in range(p)] if send_cap is None else send_cap
+        recv_cap = [recvs[j].numel() for j in range(p)] if recv_cap is None else recv_cap
+        sc = (ctypes.c_longlong * p)(*[int(x) for x in send_cap])
+        rc = (ctypes.c_longlong * p)(*[int(x) for x in recv_cap])
+        self._check(self._L.coll_alltoallv(self._h, self._bufs(sends, recvs), ctypes.c_void_p(_ptr(counts)), sc, rc,
+                                           self._resolve(dtype, sends), ALGOS[algo], _stream(stream),
+                                           ctypes.c_void_p(_ptr(recv_counts)) if recv_counts is not None else None))

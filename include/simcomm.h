@@ -1,0 +1,186 @@
+/*
+ * simcomm.h — C ABI of the simulated-communicator collectives on one B200.
+ *
+ * A communicator of p logical ranks lives inside one GPU: rank r owns its own device buffers,
+ * and a collective reads and writes all p ranks' buffers in HBM. Every call only enqueues work
+ * on the caller's CUDA stream and returns; completion is observed through that stream.
+ *
+ * Pages cited (title, then section):
+ *   [Atlas]  "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives)
+ *   [Primer] "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
+ *            (charlestar.github.io/2026/08/20/gpu-collective-communication)
+ *
+ * Common conventions
+ *   - n is the per-rank FULL buffer element count ([Primer] "先统一通信量的记号": B is the full
+ *     logical tensor): the AllReduce input/output, the ReduceScatter input, the AllGather output,
+ *     the All-to-All send buffer. ReduceScatter outputs, AllGather inputs and All-to-All blocks
+ *     hold n/p elements.
+ *   - A root is a rank index in [0, p), not a device number ([Atlas] §0, §1.1).
+ *   - bufs.send and bufs.recv are HOST arrays of p DEVICE pointers (rank order). The arrays are
+ *     read during the call only; the device buffers are owned by the caller and must stay alive,
+ *     and unchanged by other work, until the stream reaches the end of the collective
+ *     ([Primer] "CUDA Stream：API 返回不代表结果可被 Host 或其他 Stream 读取").
+ *   - Buffers are contiguous and element-aligned. 16-byte-aligned buffers whose block sizes are
+ *     multiples of 16 bytes take the vector/bulk-copy paths; anything else takes a slower
+ *     element-wise path with the same results.
+ *   - bf16 data is reduced in fp32 and rounded once (round to nearest, ties to even) to bf16.
+ *     AVG is SUM times 1/p in fp32, applied before that rounding. int32 SUM wraps around
+ *     (two's complement). MIN/MAX keep the earlier rank on ties. AVG is not defined for int32.
+ *   - In place is allowed only in the forms of [Primer] "In-place 不是“任意让输入输出指向同一地址”":
+ *     AllReduce send[r] == recv[r]; AllGather send[r] == recv[r] + r·(n/p); ReduceScatter
+ *     recv[r] == send[r] + r·(n/p); Reduce/Broadcast the root's send == recv. Any other overlap
+ *     between an output and any buffer is rejected with COLL_ERR_INVALID_ARG. All-to-All and
+ *     All-to-Allv are never in place.
+ *   - One communicator runs one collective at a time: calls on different streams must be ordered
+ *     by the caller (the communicator's scratch is shared between calls).
+ *
+ * Errors
+ *   - Synchronous (returned, nothing enqueued): COLL_ERR_INVALID_ARG (null handle or pointer, bad
+ *     root/dtype/op/algo, n not divisible by p where required, illegal aliasing), COLL_ERR_UNSUPPORTED,
+ *     COLL_ERR_CUDA (a CUDA call failed; sim_comm_last_error() has the message), and the sticky
+ *     asynchronous error of an earlier call, if the host has already seen it.
+ *   - Asynchronous (set on the device, read with sim_comm_get_async_error): COLL_ERR_TIMEOUT (a
+ *     ring step waited longer than the timeout for its predecessor), COLL_ERR_ABORTED
+ *     (sim_comm_abort was called while a ring step waited), COLL_ERR_OVERFLOW (an All-to-Allv
+ *     count exceeds a capacity; nothing is copied). Collectives are not transactions: after an
+ *     asynchronous error the outputs of the failed call are unspecified, and later calls do no
+ *     work until sim_comm_reset ([Primer] "Collective 的故障语义不是事务").
+ */
+#ifndef SIMCOMM_H
+#define SIMCOMM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SIM_COMM_MAX_RANKS 64
+
+typedef struct sim_comm* sim_comm_t;
+
+typedef enum {
+    COLL_OK = 0,
+    COLL_ERR_INVALID_ARG = 1,
+    COLL_ERR_UNSUPPORTED = 2,
+    COLL_ERR_CUDA = 3,
+    COLL_ERR_TIMEOUT = 4,
+    COLL_ERR_ABORTED = 5,
+    COLL_ERR_OVERFLOW = 6,
+    COLL_ERR_INTERNAL = 7
+} coll_status_t;
+
+typedef enum { COLL_INT32 = 0, COLL_FP32 = 1, COLL_BF16 = 2 } coll_dtype_t;
+
+typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_t;
+
+/* DIRECT: one fused pass reads all p inputs and writes every owner's output.
+ * RING:   the ring schedule of [Atlas] §2.2, chunk-pipelined as in [Atlas] §3.5. */
+typedef enum { COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1 } coll_algo_t;
+
+typedef struct {
+    const void* const* send; /* host array [p] of device pointers (inputs) */
+    void* const* recv;       /* host array [p] of device pointers (outputs) */
+} coll_bufs_t;
+
+/* A cudaStream_t passed as an opaque pointer; NULL means the legacy default stream. */
+typedef void* coll_stream_t;
+
+/* ---- communicator lifecycle ([Primer] "Communicator 定义了“谁必须一起出现”") ----------------- */
+
+/* Create a communicator of p ranks (1 <= p <= SIM_COMM_MAX_RANKS) on the current CUDA device.
+ * Allocates its scratch (status words, ring flags; ring partial buffers grow on first use).
+ * Returns NULL on failure; sim_comm_last_error() then says why. */
+sim_comm_t sim_comm_create(int p);
+
+/* Free the communicator and its scratch. Synchronises the device first. NULL is accepted. */
+coll_status_t sim_comm_destroy(sim_comm_t comm);
+
+/* Number of ranks, or -1 for a NULL handle. */
+int sim_comm_size(sim_comm_t comm);
+
+/* Message of the last failed call on this thread (a static string owned by the library). */
+const char* sim_comm_last_error(void);
+
+/* Name of a status code (a static string). */
+const char* coll_status_string(coll_status_t status);
+
+/* Options (also read from the environment at create time as SIMCOMM_<KEY upper-case>):
+ *   "chunk_bytes"  ring pipelining chunk in bytes of the reduce-scatter wire type (default 1 MiB,
+ *                  a multiple of 256, [Atlas] §3.5)
+ *   "ring_ctas"    CTAs of the ring executor (0 = as many as fit on the GPU; default 0)
+ *   "timeout_ns"   longest wait of one ring step for its predecessor (default 2e9)
+ *   "fault_skip_rank"  debugging: the ring executor never signals this rank's steps, so its
+ *                  successor times out (-1 = off, the default). Host-side fault injection only.
+ * Returns COLL_ERR_INVALID_ARG for an unknown key or a value out of range. */
+coll_status_t sim_comm_set_option(sim_comm_t comm, const char* key, long long value);
+coll_status_t sim_comm_get_option(sim_comm_t comm, const char* key, long long* value);
+
+/* Non-blocking: *out receives COLL_OK or the first asynchronous error any kernel of this
+ * communicator reported (polls a host-mapped word the kernels write; [Primer] section on failure
+ * semantics: query the asynchronous error, abort, rebuild). */
+coll_status_t sim_comm_get_async_error(sim_comm_t comm, coll_status_t* out);
+
+/* Ask running and future ring steps to stop: a waiting step gives up with COLL_ERR_ABORTED.
+ * Later calls return COLL_ERR_ABORTED until sim_comm_reset. Non-blocking. */
+coll_status_t sim_comm_abort(sim_comm_t comm);
+
+/* Wait for the device, clear the error state, the abort flag and the ring flags, so the
+ * communicator can be used again. */
+coll_status_t sim_comm_reset(sim_comm_t comm);
+
+/* Kernels this communicator has launched so far (for launch accounting). */
+coll_status_t sim_comm_launch_count(sim_comm_t comm, unsigned long long* out);
+
+/* ---- collectives ------------------------------------------------------------------------------ */
+
+/* AllReduce ([Atlas] §1.4; [Primer] "AllReduce：Partial 变成 Replicated"):
+ * recv[r][i] = ⊕_q send[q][i] for every rank r, i < n. Identical results on every rank. */
+coll_status_t coll_allreduce(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                             coll_op_t op, coll_algo_t algo, coll_stream_t stream);
+
+/* Reduce ([Atlas] §1.3, worked figure): recv[root][i] = ⊕_q send[q][i]. Only recv[root] is
+ * written; the other recv pointers are ignored and may be NULL. */
+coll_status_t coll_reduce(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                          coll_op_t op, int root, coll_algo_t algo, coll_stream_t stream);
+
+/* Broadcast ([Atlas] §1.1): recv[r][i] = send[root][i] for every rank r, the root included.
+ * Only send[root] is read; the other send pointers are ignored and may be NULL. */
+coll_status_t coll_broadcast(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                             int root, coll_algo_t algo, coll_stream_t stream);
+
+/* ReduceScatter ([Atlas] §1.5): with m = n/p, recv[r][k] = ⊕_q send[q][r·m + k], k < m.
+ * send buffers hold n elements, recv buffers m. n must be divisible by p. */
+coll_status_t coll_reduce_scatter(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                                  coll_op_t op, coll_algo_t algo, coll_stream_t stream);
+
+/* AllGather ([Atlas] §1.2): with m = n/p, recv[r][q·m + k] = send[q][k], k < m (shards
+ * concatenated in rank order). send buffers hold m elements, recv buffers n. n divisible by p. */
+coll_status_t coll_allgather(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                             coll_algo_t algo, coll_stream_t stream);
+
+/* All-to-All, equal split ([Atlas] §1.6): with m = n/p, recv[j][i·m + k] = send[i][j·m + k]
+ * (the [src][dst] block matrix transposed). Both buffers hold n elements. n divisible by p. */
+coll_status_t coll_alltoall(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
+                            coll_algo_t algo, coll_stream_t stream);
+
+/* All-to-Allv, uneven split ([Primer] "Ragged All-to-All：MoE 的真实输入通常不等长"):
+ *   counts_dev   DEVICE int64 [p][p] row-major, c[i][j] = elements source i sends to destination j
+ *                (the one matrix both sides read, so sends and receives always agree).
+ *   send_cap     HOST int64 [p]: elements send[i] holds.   recv_cap  HOST int64 [p]: recv[j] holds.
+ *   recv_counts_dev  DEVICE int64 [p] output Σ_i c[i][j], or NULL.
+ * Source i packs its blocks in destination order, destination j stores them in source order:
+ *   sdispl_i[j] = Σ_{j'<j} c[i][j'],  rdispl_j[i] = Σ_{i'<i} c[i'][j],
+ *   recv[j][rdispl_j[i] + k] = send[i][sdispl_i[j] + k],  k < c[i][j].
+ * The device checks every row sum against send_cap and every column sum against recv_cap; if any
+ * count is negative or a sum exceeds its capacity, nothing is copied and the call reports
+ * COLL_ERR_OVERFLOW asynchronously. counts_dev must stay unchanged until the call completes. */
+coll_status_t coll_alltoallv(sim_comm_t comm, coll_bufs_t bufs, const long long* counts_dev,
+                             const long long* send_cap, const long long* recv_cap, coll_dtype_t dtype,
+                             coll_algo_t algo, coll_stream_t stream, long long* recv_counts_dev);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIMCOMM_H */

@@ -1,0 +1,66 @@
+"""The C-ABI library builds, loads and exports every entry point include/simcomm.h declares; the
+host-side argument checks work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from collective_communication_primitives_b200 import build as B
+from collective_communication_primitives_b200 import simcomm as SC
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "simcomm.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)) - {"defined"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return ctypes.CDLL(B.LIB)
+
+
+def test_header_declares_the_collectives():
+    names = declared_functions()
+    for want in ("sim_comm_create", "sim_comm_destroy", "coll_allreduce", "coll_reduce", "coll_broadcast",
+                 "coll_reduce_scatter", "coll_allgather", "coll_alltoall", "coll_alltoallv",
+                 "sim_comm_get_async_error", "sim_comm_abort", "sim_comm_reset"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [f for f in declared_functions() if not hasattr(lib, f)]
+    assert not missing, missing
+
+
+def test_binding_declares_every_symbol(lib):
+    L = SC.load_library()
+    for f in declared_functions():
+        assert getattr(L, f).restype is not None or f in ("sim_comm_last_error",)
+
+
+def test_status_strings(lib):
+    L = SC.load_library()
+    for code, name in SC.STATUS.items():
+        assert L.coll_status_string(code).decode() == name
+
+
+def test_null_communicator_is_rejected_without_a_gpu(lib):
+    L = SC.load_library()
+    bufs = SC._Bufs()
+    assert L.coll_allreduce(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_alltoallv(None, bufs, None, None, None, 1, 0, None, None) == SC.INVALID_ARG
+    assert L.sim_comm_size(None) == -1
+    assert L.sim_comm_destroy(None) == SC.OK
+    assert L.sim_comm_abort(None) == SC.INVALID_ARG
+
+
+def test_create_rejects_bad_rank_counts(lib):
+    L = SC.load_library()
+    assert not L.sim_comm_create(0)
+    assert b"p must be" in L.sim_comm_last_error()
+    assert not L.sim_comm_create(65)
