@@ -25,7 +25,7 @@ struct sim_comm {
     DevState* dstate = nullptr;     // device scratch header
     uint32_t* host_words = nullptr; // host-mapped: [0] status mirror, [1] abort flag
     uint32_t* dev_words = nullptr;  // device alias of host_words
-    uint32_t* flags = nullptr;      // ring flags
+    unsigned long long* flags = nullptr;  // ring chunk flags
     size_t flags_cap = 0;           // elements
     char* stage = nullptr;          // ring partial buffers
     size_t stage_cap = 0;           // bytes
@@ -151,9 +151,9 @@ coll_status_t ensure_flags(sim_comm* c, size_t count) {
     if (c->flags) cudaFree(c->flags);  // synchronises the device: no kernel still uses the old flags
     c->flags = nullptr;
     c->flags_cap = 0;
-    cudaError_t e = cudaMalloc(&c->flags, count * sizeof(uint32_t));
+    cudaError_t e = cudaMalloc(&c->flags, count * sizeof(unsigned long long));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(ring flags)");
-    e = cudaMemset(c->flags, 0, count * sizeof(uint32_t));
+    e = cudaMemset(c->flags, 0, count * sizeof(unsigned long long));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(ring flags)");
     c->flags_cap = count;
     return COLL_OK;
@@ -173,7 +173,7 @@ coll_status_t ensure_stage(sim_comm* c, size_t bytes) {
 uint32_t next_epoch(sim_comm* c) {
     c->epoch += 1;
     if (c->epoch == 0) {  // wrapped: old flags could alias a future epoch, so clear them
-        if (c->flags) cudaMemset(c->flags, 0, c->flags_cap * sizeof(uint32_t));
+        if (c->flags) cudaMemset(c->flags, 0, c->flags_cap * sizeof(unsigned long long));
         c->epoch = 1;
     }
     return c->epoch;
@@ -248,6 +248,10 @@ struct RingPlan {
     bool needs_stage;
 };
 
+// One CTA task moves 128 KiB of the step's wire type (the partial type for reduce steps): a chunk
+// is split into that many tasks so that several SMs carry one chunk through each step.
+constexpr size_t kRingTaskBytes = 128 * 1024;
+
 coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, size_t n, coll_dtype_t dt,
                        coll_op_t op, int root, cudaStream_t s, const long long* counts = nullptr,
                        const long long* send_cap = nullptr, const long long* recv_cap = nullptr,
@@ -263,6 +267,13 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     a.n = n;
     a.seg = pl.seg;
     a.chunk = pl.chunk;
+    {
+        const bool reduce_kind = (pl.kind == RING_ALLREDUCE || pl.kind == RING_REDUCE_SCATTER || pl.kind == RING_REDUCE);
+        const size_t wire = reduce_kind ? 4 : d;
+        a.tile = std::min(pl.chunk, std::max<size_t>(16, kRingTaskBytes / wire));
+        a.ntile = uint32_t((pl.chunk + a.tile - 1) / a.tile);
+    }
+    a.elem_bytes = int(d);
     a.nch = pl.nch;
     a.nsteps = pl.nsteps;
     a.ranks_per_step = pl.rps;
@@ -302,7 +313,7 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
 
     int ctas = int(c->ring_ctas > 0 ? c->ring_ctas : c->ring_ctas_max);
     if (pl.kind != RING_ALLTOALLV) {
-        const size_t tasks = size_t(pl.nsteps) * pl.rps * pl.nch;
+        const size_t tasks = size_t(pl.nsteps) * pl.rps * pl.nch * a.ntile;
         if (tasks < size_t(ctas)) ctas = int(std::max<size_t>(tasks, 1));
     }
     cudaError_t e = launch_ring(a, dt, op, ctas, s);
@@ -446,7 +457,7 @@ coll_status_t sim_comm_reset(sim_comm_t c) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset: device synchronisation");
     e = cudaMemset(c->dstate, 0, sizeof(DevState));
-    if (e == cudaSuccess && c->flags) e = cudaMemset(c->flags, 0, c->flags_cap * sizeof(uint32_t));
+    if (e == cudaSuccess && c->flags) e = cudaMemset(c->flags, 0, c->flags_cap * sizeof(unsigned long long));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset");
     c->epoch = 0;

@@ -156,6 +156,11 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
@@ -182,11 +187,12 @@ __device__ __forceinline__ bool status_failed(const Ctl& ctl) {
 // abort, after timeout_ns of global time or after kMaxSpin polls; then records the reason and
 // returns false. Called by one thread.
 constexpr uint32_t kMaxSpin = 1u << 26;
-__device__ __forceinline__ bool wait_flag(const Ctl& ctl, const uint32_t* flag, uint32_t want, uint64_t timeout_ns) {
-    if (ld_acquire_gpu(flag) == want) return true;
+__device__ __forceinline__ bool wait_flag(const Ctl& ctl, const unsigned long long* flag, unsigned long long want,
+                                          uint64_t timeout_ns) {
+    if (ld_acquire_gpu_u64(flag) == want) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; it < kMaxSpin; ++it) {
-        if (ld_acquire_gpu(flag) == want) return true;
+        if (ld_acquire_gpu_u64(flag) == want) return true;
         if ((it & 15u) == 0u) {
             if (status_failed(ctl)) return false;
             if (*ctl.abort_flag != 0u) { raise_status(ctl, COLL_ERR_ABORTED); return false; }
@@ -196,6 +202,22 @@ __device__ __forceinline__ bool wait_flag(const Ctl& ctl, const uint32_t* flag, 
     }
     raise_status(ctl, COLL_ERR_TIMEOUT);
     return false;
+}
+
+// Count one finished task of a chunk: the flag holds (epoch << 32) | tasks finished in this call;
+// a flag left from an earlier call (older epoch) starts again at 1. The fence makes the CTA's
+// writes (ordered before this call by a __syncthreads) visible before the count.
+__device__ __forceinline__ void signal_chunk(const Ctl& ctl, unsigned long long* flag, uint32_t epoch) {
+    __threadfence();
+    const unsigned long long tag = (unsigned long long)epoch << 32;
+    unsigned long long v = *reinterpret_cast<volatile unsigned long long*>(flag);
+    for (uint32_t it = 0; it < kMaxSpin; ++it) {
+        const unsigned long long nv = ((v >> 32) == epoch) ? v + 1 : (tag | 1ull);
+        const unsigned long long old = atomicCAS(flag, v, nv);
+        if (old == v) return;
+        v = old;
+    }
+    raise_status(ctl, COLL_ERR_INTERNAL);
 }
 
 // ---- TMA bulk copies and mbarriers (shared::cta addresses, no multicast) -------------------------

@@ -18,11 +18,11 @@
 // section "Ragged All-to-All".
 #include "a2av.cuh"
 #include "common.cuh"
+#include "tile_geom.h"
 
 namespace simcomm {
 
 constexpr int kCopyThreads = 32;
-constexpr uint32_t kTile = 32768;
 constexpr int kStages = 4;
 
 static_assert(kStages <= 32, "stage phases live in one 32-bit mask");
@@ -78,39 +78,6 @@ __device__ __forceinline__ bool congruent(const CopyArgs& a, const SegDesc& d) {
     return true;
 }
 
-__device__ __forceinline__ uint32_t tile_count(const SegDesc& d, bool cong) {
-    if (d.len == 0) return 0;
-    const size_t delta = cong ? (reinterpret_cast<uintptr_t>(d.src) & 15u) : 0;
-    return uint32_t((d.len + delta + kTile - 1) / kTile);
-}
-
-struct TileGeom {
-    size_t lo, hi;       // byte range of the tile within the segment
-    size_t blo, bhi;     // bulk (16-byte aligned) part, blo == bhi when empty
-};
-
-__device__ __forceinline__ TileGeom tile_geom(const SegDesc& d, bool cong, uint32_t k) {
-    TileGeom g;
-    if (!cong) {
-        g.lo = size_t(k) * kTile;
-        g.hi = min(g.lo + kTile, d.len);
-        g.blo = g.bhi = g.lo;
-        return g;
-    }
-    const uintptr_t s = reinterpret_cast<uintptr_t>(d.src);
-    const size_t delta = s & 15u;
-    g.lo = (k == 0) ? 0 : size_t(k) * kTile - delta;
-    g.hi = min(size_t(k + 1) * kTile - delta, d.len);
-    size_t blo = (16 - ((s + g.lo) & 15u)) & 15u;
-    blo = g.lo + blo;
-    size_t bhi = g.hi - ((s + g.hi) & 15u);
-    if (blo > g.hi) blo = g.hi;
-    if (bhi < blo) bhi = blo;
-    g.blo = blo;
-    g.bhi = bhi;
-    return g;
-}
-
 // Warp copy of bytes [x, y) of a segment with 2-byte accesses (element sizes are 2 or 4 bytes,
 // so every address and length here is even).
 __device__ __forceinline__ void warp_copy_bytes(const CopyArgs& a, const SegDesc& d, size_t x, size_t y) {
@@ -159,7 +126,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     // tile counts per segment, then an inclusive scan into prefix[1..nseg]
     for (int s = lane; s < nseg; s += 32) {
         const SegDesc d = segment<KIND>(a, s, sd, rd);
-        prefix[s + 1] = tile_count(d, congruent(a, d));
+        prefix[s + 1] = tile_count(reinterpret_cast<uintptr_t>(d.src), d.len, congruent(a, d));
     }
     __syncwarp();
     if (lane == 0) prefix[0] = 0;
@@ -194,7 +161,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         const int s = find_segment(prefix, nseg, t);
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
-        const TileGeom g = tile_geom(d, cong, t - prefix[s]);
+        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, t - prefix[s]);
         if (lane == 0 && g.bhi > g.blo) {
             const int st = int(k % kStages);
             mbar_arrive_expect_tx(&bars[st], uint32_t(g.bhi - g.blo));
@@ -207,7 +174,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         const int s = find_segment(prefix, nseg, t);
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
-        const TileGeom g = tile_geom(d, cong, t - prefix[s]);
+        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, t - prefix[s]);
         if (g.bhi > g.blo) {
             const int st = int(k % kStages);
             bool ok = true;

@@ -76,10 +76,13 @@ struct RingArgs {
     int kind;
     int root;
     int vec;                 // 1: vectorised reduce hops (all offsets 16-byte aligned)
+    int elem_bytes;          // bytes per element
     size_t n;                // per-rank full element count
     size_t seg;              // elements of one segment (the unit a step moves)
     size_t chunk;            // elements of one pipelined chunk
-    uint32_t nch;            // chunks per segment (ALLTOALLV: upper bound, refined on device)
+    size_t tile;             // elements one CTA task moves (a chunk is split into ntile of them)
+    uint32_t ntile;          // CTA tasks per chunk
+    uint32_t nch;            // chunks per segment (ALLTOALLV: computed on the device)
     uint32_t nsteps;         // steps of the schedule
     uint32_t ranks_per_step; // p for ring steps, 1 for the Reduce/Broadcast chains
     uint32_t epoch;          // flags equal to epoch mean "done in this call"
@@ -88,7 +91,7 @@ struct RingArgs {
     uint64_t timeout_ns;
     char* stage;             // partial buffers, one per rank
     size_t stage_stride;     // bytes between ranks' partial buffers
-    uint32_t* flags;         // [nsteps][ranks_per_step][nch]
+    unsigned long long* flags;  // [nsteps][ranks_per_step][nch]: (epoch << 32) | finished tiles
     DevState* st;
     const long long* counts; // ALLTOALLV
     long long* recv_counts_out;

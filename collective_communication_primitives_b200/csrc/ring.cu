@@ -12,12 +12,13 @@
 //   Reduce: chain root+1 -> ... -> root;  Broadcast: chain root -> ... -> root-1;
 //   All-to-All(v): p shift steps, at step s rank r sends its block for rank (r+s) mod p there.
 //
-// Execution: every (step, chunk, rank) is a task. CTAs claim tasks from a counter in step-major
-// order, so a task's predecessor (step-1, chunk, rank-1) was claimed earlier by a CTA that is
-// running; waiting for it therefore always ends. A finished task release-stores the call's epoch
-// into its flag; its successor acquire-loads that flag with a bounded wait. One chunk is the
-// pipelining unit: chunk c of step s+1 starts as soon as chunk c of step s is done on the
-// predecessor, while other chunks are still in earlier steps.
+// Execution: a chunk (the pipelining unit) is split into `ntile` tiles; every (step, chunk, rank,
+// tile) is a CTA task. CTAs claim tasks from a counter in step-major order, so every task of a
+// step's predecessor chunk (step-1, chunk, rank-1) was claimed earlier by a CTA that is running;
+// waiting for it therefore always ends. A finished task adds one to its chunk's flag, tagged with
+// the call's epoch; a successor acquire-loads the flag with a bounded wait until all tiles of the
+// predecessor chunk are done. Chunk c of step s+1 starts as soon as chunk c of step s is done on
+// the predecessor, while other chunks are still in earlier steps.
 #include "a2av.cuh"
 #include "common.cuh"
 
@@ -25,6 +26,7 @@ namespace simcomm {
 
 constexpr int kRingThreads = 256;
 constexpr int kHopUnroll = 4;
+constexpr int kCopyUnroll = 8;
 
 // ---- hop bodies (run by the whole CTA) ------------------------------------------------------------
 
@@ -139,15 +141,15 @@ __device__ __forceinline__ void hop_copy(const void* src, void* dst, size_t byte
     const uint4* vs = reinterpret_cast<const uint4*>(s + head);
     uint4* vd = reinterpret_cast<uint4*>(d + head);
     const size_t nv = body / 16;
-    for (size_t v0 = threadIdx.x; v0 < nv; v0 += size_t(kRingThreads) * kHopUnroll) {
-        uint4 t[kHopUnroll];
+    for (size_t v0 = threadIdx.x; v0 < nv; v0 += size_t(kRingThreads) * kCopyUnroll) {
+        uint4 t[kCopyUnroll];
 #pragma unroll
-        for (int u = 0; u < kHopUnroll; ++u) {
+        for (int u = 0; u < kCopyUnroll; ++u) {
             const size_t v = v0 + size_t(u) * kRingThreads;
             if (v < nv) t[u] = ld_cg_v4(vs + v);
         }
 #pragma unroll
-        for (int u = 0; u < kHopUnroll; ++u) {
+        for (int u = 0; u < kCopyUnroll; ++u) {
             const size_t v = v0 + size_t(u) * kRingThreads;
             if (v < nv) st_v4(vd + v, t[u]);
         }
@@ -158,184 +160,62 @@ __device__ __forceinline__ void hop_copy(const void* src, void* dst, size_t byte
 
 // ---- the executor ------------------------------------------------------------------------------
 
-struct Task {
-    bool wait;         // wait for the predecessor's flag before working
-    uint32_t pred;     // its flag index
-};
-
 __device__ __forceinline__ int md(int a, int p) { return ((a % p) + p) % p; }
 
-template <int DT, int OP, bool SCALE>
-__global__ void __launch_bounds__(kRingThreads) k_ring(const __grid_constant__ RingArgs a) {
-    extern __shared__ __align__(16) unsigned char dyn_smem[];
+// Sub-tile t of chunk c of the element range [base, end): [lo, hi), empty when past the end.
+struct Range { size_t lo, hi; };
+__device__ __forceinline__ Range sub_range(const RingArgs& a, size_t base, size_t end, uint32_t c, uint32_t t) {
+    const size_t clo = base + size_t(c) * a.chunk;
+    const size_t chi = min(clo + a.chunk, end);
+    const size_t lo = min(clo + size_t(t) * a.tile, chi);
+    return Range{lo, min(lo + a.tile, chi)};
+}
+
+// Task loop shared by every schedule. A task is (step g, chunk c, rank r, tile t), claimed in that
+// order (step-major). waits(g, r, &pred) names the predecessor chunk flag, if any; work(g, c, r, t)
+// moves the data; signaller(g, r) is the rank whose progress the task reports (fault injection
+// silences one rank).
+template <int KIND, typename Pred, typename Work>
+__device__ __forceinline__ void run_tasks(const RingArgs& a, uint32_t nch, uint32_t total, Pred pred, Work work) {
     __shared__ uint32_t s_task;
     __shared__ int s_ok;
-    __shared__ uint32_t s_nch;
-
-    const int p = a.p;
-    const size_t d = size_t(Elem<DT>::kBytes);
-    constexpr size_t kAcc = sizeof(typename Elem<DT>::A);
-    long long* sd = reinterpret_cast<long long*>(dyn_smem);
-    long long* rd = sd + p * p;
-
-    // One thread decides whether this CTA runs, so the decision is uniform across the CTA.
-    if (threadIdx.x == 0) s_ok = !status_failed(a.ctl);
-    __syncthreads();
-    bool run = s_ok;
-    __syncthreads();
-    uint32_t nch = a.nch;
-    if (a.kind == RING_ALLTOALLV && run) {
-        if (threadIdx.x < 32) {
-            const A2avPlan plan = a2av_plan_warp(a.counts, p, a.send_cap, a.recv_cap, sd, rd, a.recv_counts_out, a.ctl);
-            if (threadIdx.x == 0) {
-                s_ok = plan.ok;
-                s_nch = plan.max_count > 0 ? uint32_t((size_t(plan.max_count) + a.chunk - 1) / a.chunk) : 0u;
-            }
-        }
-        __syncthreads();
-        run = s_ok;
-        nch = s_nch;
-    }
+    constexpr bool kFlags = (KIND != RING_ALLTOALL && KIND != RING_ALLTOALLV);
     const uint32_t rps = a.ranks_per_step;
-    const uint32_t per_step = rps * nch;
-    const uint32_t total = run ? a.nsteps * per_step : 0u;
-
-    while (total) {
+    const uint32_t per_rank = a.ntile;
+    const uint32_t per_chunk = rps * per_rank;
+    const uint32_t per_step = nch * per_chunk;
+    const unsigned long long want = ((unsigned long long)a.epoch << 32) | a.ntile;
+    while (true) {
         if (threadIdx.x == 0) s_task = status_failed(a.ctl) ? total : atomicAdd(&a.st->task_ctr, 1u);
         __syncthreads();
-        const uint32_t t = s_task;
-        if (t >= total) break;
-        const uint32_t g = t / per_step;
-        const uint32_t rem = t - g * per_step;
-        const uint32_t c = rem / rps;
-        const int r = int(rem - c * rps);
-        const uint32_t my_flag = (g * rps + uint32_t(r)) * nch + c;
-        Task tk{false, 0};
+        const uint32_t task = s_task;
+        if (task >= total) break;
+        const uint32_t g = task / per_step;
+        uint32_t rem = task - g * per_step;
+        const uint32_t c = rem / per_chunk;
+        rem -= c * per_chunk;
+        const int r = int(rem / per_rank);
+        const uint32_t t = rem - uint32_t(r) * per_rank;
+        int pred_rank = -1;
         int signal_rank = r;
-
-        switch (a.kind) {
-            case RING_ALLREDUCE:
-            case RING_REDUCE_SCATTER:
-                if (g >= 1) tk = Task{true, ((g - 1) * rps + uint32_t(md(r - 1, p))) * nch + c};
-                break;
-            case RING_ALLGATHER:
-                if (g >= 2) tk = Task{true, ((g - 1) * rps + uint32_t(md(r - 1, p))) * nch + c};
-                break;
-            case RING_REDUCE:
-                signal_rank = md(a.root + 2 + int(g), p);
-                if (g >= 1) tk = Task{true, (g - 1) * nch + c};
-                break;
-            case RING_BCAST:
-                signal_rank = md(a.root + int(g), p);
-                if (g >= 2) tk = Task{true, (g - 1) * nch + c};
-                break;
-            default:
-                break;
-        }
-        if (tk.wait) {
-            if (threadIdx.x == 0) s_ok = wait_flag(a.ctl, a.flags + tk.pred, a.epoch, a.timeout_ns);
+        const bool must_wait = pred(g, r, &pred_rank, &signal_rank);
+        if (kFlags && must_wait) {
+            if (threadIdx.x == 0) {
+                const unsigned long long* f = a.flags + (size_t(g - 1) * rps + uint32_t(pred_rank)) * nch + c;
+                s_ok = wait_flag(a.ctl, f, want, a.timeout_ns);
+            }
             __syncthreads();
             if (!s_ok) break;
         }
-
-        switch (a.kind) {
-            case RING_ALLREDUCE:
-            case RING_REDUCE_SCATTER: {
-                const int w = md(r - 1, p);
-                const bool rs_phase = (a.kind == RING_REDUCE_SCATTER) || g < uint32_t(p - 1);
-                const int s = rs_phase ? int(g) + 1 : int(g) - (p - 1) + 1;
-                const int k = rs_phase ? md(r - 1 - s, p) : md(r - s, p);
-                const size_t sb = min(size_t(k) * a.seg, a.n), se = min(sb + a.seg, a.n);
-                const size_t lo = min(sb + size_t(c) * a.chunk, se), hi = min(lo + a.chunk, se);
-                if (hi > lo) {
-                    if (rs_phase) {
-                        const bool first = (s == 1), last = (s == p - 1);
-                        const void* wire = first ? static_cast<const void*>(static_cast<const char*>(a.ptrs.send[w]) + lo * d)
-                                                 : static_cast<const void*>(a.stage + size_t(w) * a.stage_stride + lo * kAcc);
-                        const void* own = static_cast<const char*>(a.ptrs.send[r]) + lo * d;
-                        void* dst;
-                        if (!last) dst = a.stage + size_t(r) * a.stage_stride + lo * kAcc;
-                        else if (a.kind == RING_ALLREDUCE) dst = static_cast<char*>(a.ptrs.recv[r]) + lo * d;
-                        else dst = static_cast<char*>(a.ptrs.recv[r]) + (lo - sb) * d;
-                        hop_reduce<DT, OP, SCALE>(wire, !first, own, dst, last, hi - lo, a.scale, a.vec != 0);
-                    } else {
-                        hop_copy(static_cast<const char*>(a.ptrs.recv[w]) + lo * d,
-                                 static_cast<char*>(a.ptrs.recv[r]) + lo * d, (hi - lo) * d);
-                    }
-                }
-                break;
-            }
-            case RING_ALLGATHER: {
-                // g = 0: the own shard into the own output; g = s >= 1: segment (r-s) mod p from r-1
-                const int k = (g == 0) ? r : md(r - int(g), p);
-                const size_t lo = min(size_t(c) * a.chunk, a.seg), hi = min(lo + a.chunk, a.seg);
-                if (hi > lo) {
-                    char* dst = static_cast<char*>(a.ptrs.recv[r]) + (size_t(k) * a.seg + lo) * d;
-                    const char* src;
-                    if (g == 0) src = static_cast<const char*>(a.ptrs.send[r]) + lo * d;
-                    else if (g == 1) src = static_cast<const char*>(a.ptrs.send[md(r - 1, p)]) + lo * d;
-                    else src = static_cast<const char*>(a.ptrs.recv[md(r - 1, p)]) + (size_t(k) * a.seg + lo) * d;
-                    if (src != dst) hop_copy(src, dst, (hi - lo) * d);
-                }
-                break;
-            }
-            case RING_REDUCE: {
-                // hop h = g+1 at rank q = root+1+h, its predecessor w = q-1
-                const int h = int(g) + 1;
-                const int q = md(a.root + 1 + h, p), w = md(q - 1, p);
-                const size_t lo = min(size_t(c) * a.chunk, a.n), hi = min(lo + a.chunk, a.n);
-                if (hi > lo) {
-                    const bool first = (h == 1), last = (h == p - 1);
-                    const void* wire = first ? static_cast<const void*>(static_cast<const char*>(a.ptrs.send[w]) + lo * d)
-                                             : static_cast<const void*>(a.stage + size_t(w) * a.stage_stride + lo * kAcc);
-                    const void* own = static_cast<const char*>(a.ptrs.send[q]) + lo * d;
-                    void* dst = last ? static_cast<void*>(static_cast<char*>(a.ptrs.recv[a.root]) + lo * d)
-                                     : static_cast<void*>(a.stage + size_t(q) * a.stage_stride + lo * kAcc);
-                    hop_reduce<DT, OP, SCALE>(wire, !first, own, dst, last, hi - lo, a.scale, a.vec != 0);
-                }
-                break;
-            }
-            case RING_BCAST: {
-                // hop 0: the root's own output; hop h >= 1: rank root+h copies from its predecessor
-                const int q = md(a.root + int(g), p);
-                const size_t lo = min(size_t(c) * a.chunk, a.n), hi = min(lo + a.chunk, a.n);
-                if (hi > lo) {
-                    const char* src = (g <= 1) ? static_cast<const char*>(a.ptrs.send[a.root])
-                                               : static_cast<const char*>(a.ptrs.recv[md(q - 1, p)]);
-                    char* dst = static_cast<char*>(a.ptrs.recv[q]);
-                    if (src + lo * d != dst + lo * d) hop_copy(src + lo * d, dst + lo * d, (hi - lo) * d);
-                }
-                break;
-            }
-            case RING_ALLTOALL:
-            case RING_ALLTOALLV: {
-                const int j = md(r + int(g), p);
-                size_t len, soff, roff;
-                if (a.kind == RING_ALLTOALL) {
-                    len = a.seg; soff = size_t(j) * a.seg; roff = size_t(r) * a.seg;
-                } else {
-                    len = size_t(a.counts[r * p + j]); soff = size_t(sd[r * p + j]); roff = size_t(rd[r * p + j]);
-                }
-                const size_t lo = min(size_t(c) * a.chunk, len), hi = min(lo + a.chunk, len);
-                if (hi > lo)
-                    hop_copy(static_cast<const char*>(a.ptrs.send[r]) + (soff + lo) * d,
-                             static_cast<char*>(a.ptrs.recv[j]) + (roff + lo) * d, (hi - lo) * d);
-                break;
-            }
-            default:
-                break;
-        }
-
+        work(g, c, r, t);
         __syncthreads();
-        // The All-to-All schedules have no dependent steps and no flags.
-        const bool has_flags = (a.kind != RING_ALLTOALL && a.kind != RING_ALLTOALLV);
-        if (threadIdx.x == 0 && has_flags && signal_rank != a.skip_rank) {
-            __threadfence();
-            st_release_gpu(a.flags + my_flag, a.epoch);
-        }
+        if (kFlags && threadIdx.x == 0 && signal_rank != a.skip_rank)
+            signal_chunk(a.ctl, a.flags + (size_t(g) * rps + uint32_t(r)) * nch + c, a.epoch);
     }
+}
 
-    // Leave: the last CTA out resets the task counter for the next call on this communicator.
+// The last CTA to leave resets the task counter for the next call on this communicator.
+__device__ __forceinline__ void leave(const RingArgs& a) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -347,34 +227,203 @@ __global__ void __launch_bounds__(kRingThreads) k_ring(const __grid_constant__ R
     }
 }
 
-template <int DT, int OP, bool SCALE>
-static cudaError_t launch_ring_typed(const RingArgs& a, int ctas, cudaStream_t s) {
-    const size_t smem = (a.kind == RING_ALLTOALLV) ? 2 * size_t(a.p) * a.p * sizeof(long long) : 0;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_ring<DT, OP, SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(2 * size_t(kMaxRanks) * kMaxRanks * sizeof(long long)));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
+// One thread decides whether the CTA runs at all (uniform across the CTA).
+__device__ __forceinline__ bool cta_may_run(const RingArgs& a) {
+    __shared__ int s_run;
+    if (threadIdx.x == 0) s_run = !status_failed(a.ctl);
+    __syncthreads();
+    const bool run = s_run;
+    __syncthreads();
+    return run;
+}
+
+// Reduce schedules: ring AllReduce (reduce-scatter steps then all-gather steps), ring
+// ReduceScatter, and the Reduce chain.
+template <int DT, int OP, bool SCALE, int KIND>
+__global__ void __launch_bounds__(kRingThreads, 2) k_ring_reduce(const __grid_constant__ RingArgs a) {
+    const int p = a.p;
+    const size_t d = size_t(Elem<DT>::kBytes);
+    constexpr size_t kAcc = sizeof(typename Elem<DT>::A);
+    const bool run = cta_may_run(a);
+    const uint32_t total = run ? a.nsteps * a.nch * a.ranks_per_step * a.ntile : 0u;
+
+    auto pred = [&](uint32_t g, int r, int* pr, int* sr) -> bool {
+        if constexpr (KIND == RING_REDUCE) {
+            *sr = md(a.root + 2 + int(g), p);  // hop h = g+1 runs at rank root+1+h
+            *pr = 0;
+            return g >= 1;
+        } else {
+            *pr = md(r - 1, p);
+            return g >= 1;
+        }
+    };
+    auto work = [&](uint32_t g, uint32_t c, int r, uint32_t t) {
+        if constexpr (KIND == RING_REDUCE) {
+            const int h = int(g) + 1;
+            const int q = md(a.root + 1 + h, p), w = md(q - 1, p);
+            const Range rg = sub_range(a, 0, a.n, c, t);
+            if (rg.hi <= rg.lo) return;
+            const bool first = (h == 1), last = (h == p - 1);
+            const void* wire = first ? static_cast<const void*>(static_cast<const char*>(a.ptrs.send[w]) + rg.lo * d)
+                                     : static_cast<const void*>(a.stage + size_t(w) * a.stage_stride + rg.lo * kAcc);
+            const void* own = static_cast<const char*>(a.ptrs.send[q]) + rg.lo * d;
+            void* dst = last ? static_cast<void*>(static_cast<char*>(a.ptrs.recv[a.root]) + rg.lo * d)
+                             : static_cast<void*>(a.stage + size_t(q) * a.stage_stride + rg.lo * kAcc);
+            hop_reduce<DT, OP, SCALE>(wire, !first, own, dst, last, rg.hi - rg.lo, a.scale, a.vec != 0);
+        } else {
+            const int w = md(r - 1, p);
+            const bool rs_phase = (KIND == RING_REDUCE_SCATTER) || g < uint32_t(p - 1);
+            const int s = rs_phase ? int(g) + 1 : int(g) - (p - 1) + 1;
+            const int k = rs_phase ? md(r - 1 - s, p) : md(r - s, p);
+            const size_t sb = min(size_t(k) * a.seg, a.n), se = min(sb + a.seg, a.n);
+            const Range rg = sub_range(a, sb, se, c, t);
+            if (rg.hi <= rg.lo) return;
+            if (rs_phase) {
+                const bool first = (s == 1), last = (s == p - 1);
+                const void* wire = first
+                    ? static_cast<const void*>(static_cast<const char*>(a.ptrs.send[w]) + rg.lo * d)
+                    : static_cast<const void*>(a.stage + size_t(w) * a.stage_stride + rg.lo * kAcc);
+                const void* own = static_cast<const char*>(a.ptrs.send[r]) + rg.lo * d;
+                void* dst;
+                if (!last) dst = a.stage + size_t(r) * a.stage_stride + rg.lo * kAcc;
+                else if (KIND == RING_ALLREDUCE) dst = static_cast<char*>(a.ptrs.recv[r]) + rg.lo * d;
+                else dst = static_cast<char*>(a.ptrs.recv[r]) + (rg.lo - sb) * d;
+                hop_reduce<DT, OP, SCALE>(wire, !first, own, dst, last, rg.hi - rg.lo, a.scale, a.vec != 0);
+            } else {
+                hop_copy(static_cast<const char*>(a.ptrs.recv[w]) + rg.lo * d,
+                         static_cast<char*>(a.ptrs.recv[r]) + rg.lo * d, (rg.hi - rg.lo) * d);
+            }
+        }
+    };
+    if (total) run_tasks<KIND>(a, a.nch, total, pred, work);
+    leave(a);
+}
+
+// Copy schedules: ring AllGather, the Broadcast chain, and the All-to-All(v) shift exchange.
+template <int KIND>
+__global__ void __launch_bounds__(kRingThreads, 2) k_ring_copy(const __grid_constant__ RingArgs a) {
+    extern __shared__ __align__(16) unsigned char dyn_smem[];
+    __shared__ uint32_t s_nch;
+    __shared__ int s_plan_ok;
+    const int p = a.p;
+    const size_t d = size_t(a.elem_bytes);
+    long long* sd = reinterpret_cast<long long*>(dyn_smem);
+    long long* rd = sd + p * p;
+    bool run = cta_may_run(a);
+    uint32_t nch = a.nch;
+    if constexpr (KIND == RING_ALLTOALLV) {
+        if (run) {
+            if (threadIdx.x < 32) {
+                const A2avPlan plan =
+                    a2av_plan_warp(a.counts, p, a.send_cap, a.recv_cap, sd, rd, a.recv_counts_out, a.ctl);
+                if (threadIdx.x == 0) {
+                    s_plan_ok = plan.ok;
+                    s_nch = plan.max_count > 0 ? uint32_t((size_t(plan.max_count) + a.chunk - 1) / a.chunk) : 0u;
+                }
+            }
+            __syncthreads();
+            run = s_plan_ok;
+            nch = s_nch;
+        }
     }
-    k_ring<DT, OP, SCALE><<<ctas, kRingThreads, smem, s>>>(a);
+    const uint32_t total = run ? a.nsteps * nch * a.ranks_per_step * a.ntile : 0u;
+
+    auto pred = [&](uint32_t g, int r, int* pr, int* sr) -> bool {
+        if constexpr (KIND == RING_ALLGATHER) {
+            *pr = md(r - 1, p);
+            return g >= 2;  // step 1 reads the predecessor's own shard straight from its input
+        } else if constexpr (KIND == RING_BCAST) {
+            *sr = md(a.root + int(g), p);
+            *pr = 0;
+            return g >= 2;  // hop 1 reads the root's input
+        } else {
+            return false;
+        }
+    };
+    auto work = [&](uint32_t g, uint32_t c, int r, uint32_t t) {
+        if constexpr (KIND == RING_ALLGATHER) {
+            // g = 0: the own shard into the own output; g = s >= 1: segment (r-s) mod p from r-1
+            const int k = (g == 0) ? r : md(r - int(g), p);
+            const Range rg = sub_range(a, 0, a.seg, c, t);
+            if (rg.hi <= rg.lo) return;
+            char* dst = static_cast<char*>(a.ptrs.recv[r]) + (size_t(k) * a.seg + rg.lo) * d;
+            const char* src;
+            if (g == 0) src = static_cast<const char*>(a.ptrs.send[r]) + rg.lo * d;
+            else if (g == 1) src = static_cast<const char*>(a.ptrs.send[md(r - 1, p)]) + rg.lo * d;
+            else src = static_cast<const char*>(a.ptrs.recv[md(r - 1, p)]) + (size_t(k) * a.seg + rg.lo) * d;
+            if (src != dst) hop_copy(src, dst, (rg.hi - rg.lo) * d);
+        } else if constexpr (KIND == RING_BCAST) {
+            // hop 0: the root's own output; hop h >= 1: rank root+h copies from its predecessor
+            const int q = md(a.root + int(g), p);
+            const Range rg = sub_range(a, 0, a.n, c, t);
+            if (rg.hi <= rg.lo) return;
+            const char* src = (g <= 1) ? static_cast<const char*>(a.ptrs.send[a.root])
+                                       : static_cast<const char*>(a.ptrs.recv[md(q - 1, p)]);
+            char* dst = static_cast<char*>(a.ptrs.recv[q]);
+            if (src != dst) hop_copy(src + rg.lo * d, dst + rg.lo * d, (rg.hi - rg.lo) * d);
+        } else {
+            const int j = md(r + int(g), p);
+            size_t len, soff, roff;
+            if constexpr (KIND == RING_ALLTOALL) {
+                len = a.seg; soff = size_t(j) * a.seg; roff = size_t(r) * a.seg;
+            } else {
+                len = size_t(a.counts[r * p + j]); soff = size_t(sd[r * p + j]); roff = size_t(rd[r * p + j]);
+            }
+            const Range rg = sub_range(a, 0, len, c, t);
+            if (rg.hi <= rg.lo) return;
+            hop_copy(static_cast<const char*>(a.ptrs.send[r]) + (soff + rg.lo) * d,
+                     static_cast<char*>(a.ptrs.recv[j]) + (roff + rg.lo) * d, (rg.hi - rg.lo) * d);
+        }
+    };
+    if (total) run_tasks<KIND>(a, nch, total, pred, work);
+    leave(a);
+}
+
+// ---- launch ------------------------------------------------------------------------------------
+
+template <typename K>
+static cudaError_t launch_with_smem(K kernel, int ctas, size_t smem, const RingArgs& a, cudaStream_t s) {
+    if (smem > 0) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+    }
+    kernel<<<ctas, kRingThreads, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int DT, int OP, bool SCALE>
+static cudaError_t launch_reduce_kind(const RingArgs& a, int ctas, cudaStream_t s) {
+    switch (a.kind) {
+        case RING_ALLREDUCE: return launch_with_smem(k_ring_reduce<DT, OP, SCALE, RING_ALLREDUCE>, ctas, 0, a, s);
+        case RING_REDUCE_SCATTER:
+            return launch_with_smem(k_ring_reduce<DT, OP, SCALE, RING_REDUCE_SCATTER>, ctas, 0, a, s);
+        case RING_REDUCE: return launch_with_smem(k_ring_reduce<DT, OP, SCALE, RING_REDUCE>, ctas, 0, a, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 template <int DT>
 static cudaError_t launch_ring_dt(const RingArgs& a, int op, int ctas, cudaStream_t s) {
     switch (op) {
-        case COLL_SUM: return launch_ring_typed<DT, COLL_SUM, false>(a, ctas, s);
-        case COLL_MIN: return launch_ring_typed<DT, COLL_MIN, false>(a, ctas, s);
-        case COLL_MAX: return launch_ring_typed<DT, COLL_MAX, false>(a, ctas, s);
+        case COLL_SUM: return launch_reduce_kind<DT, COLL_SUM, false>(a, ctas, s);
+        case COLL_MIN: return launch_reduce_kind<DT, COLL_MIN, false>(a, ctas, s);
+        case COLL_MAX: return launch_reduce_kind<DT, COLL_MAX, false>(a, ctas, s);
         case COLL_AVG:
             if constexpr (DT == COLL_INT32) return cudaErrorInvalidValue;
-            else return launch_ring_typed<DT, COLL_SUM, true>(a, ctas, s);
+            else return launch_reduce_kind<DT, COLL_SUM, true>(a, ctas, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStream_t s) {
+    switch (a.kind) {
+        case RING_ALLGATHER: return launch_with_smem(k_ring_copy<RING_ALLGATHER>, ctas, 0, a, s);
+        case RING_BCAST: return launch_with_smem(k_ring_copy<RING_BCAST>, ctas, 0, a, s);
+        case RING_ALLTOALL: return launch_with_smem(k_ring_copy<RING_ALLTOALL>, ctas, 0, a, s);
+        case RING_ALLTOALLV:
+            return launch_with_smem(k_ring_copy<RING_ALLTOALLV>, ctas, 2 * size_t(a.p) * a.p * sizeof(long long), a, s);
+        default: break;
+    }
     switch (dtype) {
         case COLL_INT32: return launch_ring_dt<COLL_INT32>(a, op, ctas, s);
         case COLL_FP32: return launch_ring_dt<COLL_FP32>(a, op, ctas, s);
@@ -385,8 +434,8 @@ cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStre
 
 int ring_max_ctas(int num_sms) {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_ring<COLL_FP32, COLL_SUM, false>, kRingThreads,
-                                                      0) != cudaSuccess || per_sm < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_ring_reduce<COLL_FP32, COLL_SUM, false, RING_ALLREDUCE>,
+                                                      kRingThreads, 0) != cudaSuccess || per_sm < 1)
         per_sm = 1;
     return num_sms * per_sm;
 }

@@ -431,7 +431,7 @@ def test_synchronous_argument_errors():
         c.reduce_scatter(t, [t[r][:16] for r in range(p)])
     assert e.value.status == SC.INVALID_ARG
     with pytest.raises(SC.SimCommError) as e:
-        c.allreduce([None] * p, u)
+        c.allreduce([None] * p, u, n=64)
     assert e.value.status == SC.INVALID_ARG
     with pytest.raises(SC.SimCommError) as e:
         c.set_option("chunk_bytes", 100)
