@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--n", type=int, default=N_BUCKET, help="elements per rank (default: the 25 Mi bucket)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ops", default="", help="comma-separated substrings: run only the matching rows")
+    ap.add_argument("--option", action="append", default=[], help="communicator option key=value")
     return ap.parse_args()
 
 
@@ -144,59 +146,58 @@ def build_step(comm, wl):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clock and throttle reasons sampled through NVML every 20 ms while the timed region runs
+    (nvidia-smi's command-line loop as a fallback)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.stop = threading.Event()
+        self.thread = None
+
+    def _nvml_loop(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            self.stop.wait(0.02)
+        pynvml.nvmlShutdown()
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml  # noqa: F401
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
             self.thread.start()
+            time.sleep(0.05)
         except Exception:
-            self.proc = None
+            self.thread = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        if self.thread:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        reasons = set()
+        for _, _, rs in self.samples:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
                     reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 def time_device(ops, steps, warmup, stream):
@@ -362,7 +363,13 @@ def main():
     wl = Workload(args.n, device)
     comm = SC.SimComm(P)
     comm.set_option("chunk_bytes", 1 << 20)
+    for kv in args.option:
+        k, v = kv.split("=", 1)
+        comm.set_option(k, int(v))
     ops = build_step(comm, wl)
+    if args.ops:
+        keys = [k for k in args.ops.split(",") if k]
+        ops = [o for o in ops if any(k in o[0] for k in keys)]
     eff_per_step = sum(o[3] for o in ops)
 
     if world > 1:
@@ -421,6 +428,7 @@ def main():
         "config": {"workload": f"DP gradient bucket, p={P} ranks x {args.n} elements per rank, every hot-path row "
                                f"(direct and ring) per step", "p": P, "n_per_rank": args.n,
                    "chunk_bytes": 1 << 20, "l2": "inputs larger than L2 (100 MiB per rank fp32)",
+                   "ops": [o[0] for o in ops], "options": args.option,
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline,
         "per_op": per_op_json,

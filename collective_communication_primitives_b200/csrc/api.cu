@@ -34,6 +34,10 @@ struct sim_comm {
     long long ring_ctas = 0;
     long long timeout_ns = 2000000000LL;
     long long fault_skip_rank = -1;
+    long long copy_variant = -1;
+    long long copy_order = -1;
+    long long direct_pack = 0;
+    long long direct_ctas_per_sm = 16;
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
 };
@@ -195,17 +199,19 @@ coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, col
     a.scale = (op == COLL_AVG) ? 1.0f / float(c->p) : 1.0f;
     a.ctl = make_ctl(c);
     const size_t d = dtype_bytes(dt);
-    bool vec = true;
-    for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.send[r]);
-    if (mode == MODE_ALLREDUCE)
-        for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.recv[r]);
-    else if (mode == MODE_REDUCE)
-        vec = vec && aligned16(a.ptrs.recv[root]);
-    else {
-        for (int r = 0; r < c->p; ++r) vec = vec && aligned16(a.ptrs.recv[r]);
-        vec = vec && (a.seg * d) % 16 == 0;
-    }
-    a.vec = vec ? 1 : 0;
+    // The widest pack (32, then 16 bytes) every touched buffer is aligned to; ReduceScatter also
+    // needs its owner segments to start on that boundary.
+    auto all_aligned = [&](uintptr_t mask) {
+        bool ok = true;
+        for (int r = 0; r < c->p; ++r) ok = ok && (uintptr_t(a.ptrs.send[r]) & mask) == 0;
+        if (mode == MODE_REDUCE) return ok && (uintptr_t(a.ptrs.recv[root]) & mask) == 0;
+        for (int r = 0; r < c->p; ++r) ok = ok && (uintptr_t(a.ptrs.recv[r]) & mask) == 0;
+        if (mode == MODE_REDUCE_SCATTER) ok = ok && ((a.seg * d) & mask) == 0;
+        return ok;
+    };
+    a.vec = all_aligned(31) ? 2 : (all_aligned(15) ? 1 : 0);
+    if (c->direct_pack == 16 && a.vec == 2) a.vec = 1;
+    a.ctas_per_sm = int(c->direct_ctas_per_sm);
     cudaError_t e = launch_direct_reduce(a, dt, op, c->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "direct reduction launch");
     c->launches += 1;
@@ -234,8 +240,13 @@ coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_e
         a.recv_cap[r] = recv_cap ? recv_cap[r] : 0;
     }
     a.timeout_ns = uint64_t(c->timeout_ns);
+    int variant = 0, order = 0;
+    copy_defaults(kind, &variant, &order);
+    if (c->copy_variant >= 0) variant = int(c->copy_variant);
+    if (c->copy_order >= 0) order = int(c->copy_order);
+    a.order = order;
     a.ctl = make_ctl(c);
-    cudaError_t e = launch_copy(a, c->num_sms, s);
+    cudaError_t e = launch_copy(a, c->num_sms, variant, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
     c->launches += 1;
     return COLL_OK;
@@ -347,6 +358,18 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     } else if (k == "fault_skip_rank") {
         if (value < -1 || value >= c->p) return fail(COLL_ERR_INVALID_ARG, "fault_skip_rank out of range");
         c->fault_skip_rank = value;
+    } else if (k == "copy_variant") {
+        if (value < -1 || value >= copy_num_variants()) return fail(COLL_ERR_INVALID_ARG, "copy_variant out of range");
+        c->copy_variant = value;
+    } else if (k == "copy_order") {
+        if (value < -1 || value > 1) return fail(COLL_ERR_INVALID_ARG, "copy_order must be -1, 0 or 1");
+        c->copy_order = value;
+    } else if (k == "direct_pack") {
+        if (value != 0 && value != 16 && value != 32) return fail(COLL_ERR_INVALID_ARG, "direct_pack must be 0, 16 or 32");
+        c->direct_pack = value;
+    } else if (k == "direct_ctas_per_sm") {
+        if (value < 1 || value > 32) return fail(COLL_ERR_INVALID_ARG, "direct_ctas_per_sm must be in [1, 32]");
+        c->direct_ctas_per_sm = value;
     } else {
         return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     }
@@ -407,6 +430,8 @@ sim_comm_t sim_comm_create(int p) {
     if (set_option_impl(c, "timeout_ns", to) != COLL_OK) c->timeout_ns = 2000000000LL;
     const long long fr = env_ll("SIMCOMM_FAULT_SKIP_RANK", -1);
     if (set_option_impl(c, "fault_skip_rank", fr) != COLL_OK) c->fault_skip_rank = -1;
+    const long long cv = env_ll("SIMCOMM_COPY_VARIANT", c->copy_variant);
+    if (set_option_impl(c, "copy_variant", cv) != COLL_OK) c->copy_variant = -1;
     g_last_error.clear();
     return c;
 }
@@ -436,6 +461,10 @@ coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* valu
     else if (k == "ring_ctas") *value = c->ring_ctas;
     else if (k == "timeout_ns") *value = c->timeout_ns;
     else if (k == "fault_skip_rank") *value = c->fault_skip_rank;
+    else if (k == "copy_variant") *value = c->copy_variant;
+    else if (k == "copy_order") *value = c->copy_order;
+    else if (k == "direct_pack") *value = c->direct_pack;
+    else if (k == "direct_ctas_per_sm") *value = c->direct_ctas_per_sm;
     else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     return COLL_OK;
 }

@@ -42,50 +42,74 @@ template <int OP> __device__ __forceinline__ int32_t op_i(int32_t a, int32_t b) 
     return int32_t(uint32_t(a) + uint32_t(b));
 }
 
-// ---- 16-byte packs: 4 fp32 / 4 int32 / 8 bf16 lanes, widened to the accumulator type ----------
+// ---- packs of W 32-bit words (W = 4: 16 bytes, W = 8: 32 bytes) --------------------------------
+// A pack holds W fp32 / W int32 / 2W bf16 lanes, widened to the accumulator type.
 
-template <int DT> struct Pack16;
+template <int W> struct Words { uint32_t w[W]; };
 
-template <> struct Pack16<COLL_FP32> {
-    static constexpr int L = 4;
+template <int DT, int W> struct PackW;
+
+template <int W> struct PackW<COLL_FP32, W> {
+    static constexpr int L = W;
     using A = float;
-    __device__ static void unpack(const uint4& v, float (&a)[4]) {
-        a[0] = __uint_as_float(v.x); a[1] = __uint_as_float(v.y);
-        a[2] = __uint_as_float(v.z); a[3] = __uint_as_float(v.w);
-    }
-    __device__ static uint4 pack(const float (&a)[4]) {
-        return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]), __float_as_uint(a[3]));
-    }
-};
-
-template <> struct Pack16<COLL_INT32> {
-    static constexpr int L = 4;
-    using A = int32_t;
-    __device__ static void unpack(const uint4& v, int32_t (&a)[4]) {
-        a[0] = int32_t(v.x); a[1] = int32_t(v.y); a[2] = int32_t(v.z); a[3] = int32_t(v.w);
-    }
-    __device__ static uint4 pack(const int32_t (&a)[4]) {
-        return make_uint4(uint32_t(a[0]), uint32_t(a[1]), uint32_t(a[2]), uint32_t(a[3]));
-    }
-};
-
-template <> struct Pack16<COLL_BF16> {
-    static constexpr int L = 8;
-    using A = float;
-    __device__ static void unpack(const uint4& v, float (&a)[8]) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    __device__ static void unpack(const Words<W>& v, float (&a)[L]) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            a[2 * k] = bf16_bits_to_float(w[k] & 0xFFFFu);
-            a[2 * k + 1] = bf16_bits_to_float(w[k] >> 16);
+        for (int k = 0; k < W; ++k) a[k] = __uint_as_float(v.w[k]);
+    }
+    __device__ static Words<W> pack(const float (&a)[L]) {
+        Words<W> v;
+#pragma unroll
+        for (int k = 0; k < W; ++k) v.w[k] = __float_as_uint(a[k]);
+        return v;
+    }
+};
+
+template <int W> struct PackW<COLL_INT32, W> {
+    static constexpr int L = W;
+    using A = int32_t;
+    __device__ static void unpack(const Words<W>& v, int32_t (&a)[L]) {
+#pragma unroll
+        for (int k = 0; k < W; ++k) a[k] = int32_t(v.w[k]);
+    }
+    __device__ static Words<W> pack(const int32_t (&a)[L]) {
+        Words<W> v;
+#pragma unroll
+        for (int k = 0; k < W; ++k) v.w[k] = uint32_t(a[k]);
+        return v;
+    }
+};
+
+template <int W> struct PackW<COLL_BF16, W> {
+    static constexpr int L = 2 * W;
+    using A = float;
+    __device__ static void unpack(const Words<W>& v, float (&a)[L]) {
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            a[2 * k] = bf16_bits_to_float(v.w[k] & 0xFFFFu);
+            a[2 * k + 1] = bf16_bits_to_float(v.w[k] >> 16);
         }
     }
-    __device__ static uint4 pack(const float (&a)[8]) {
-        uint32_t w[4];
+    __device__ static Words<W> pack(const float (&a)[L]) {
+        Words<W> v;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[k] = uint32_t(float_to_bf16_bits(a[2 * k])) | (uint32_t(float_to_bf16_bits(a[2 * k + 1])) << 16);
-        return make_uint4(w[0], w[1], w[2], w[3]);
+        for (int k = 0; k < W; ++k)
+            v.w[k] = uint32_t(float_to_bf16_bits(a[2 * k])) | (uint32_t(float_to_bf16_bits(a[2 * k + 1])) << 16);
+        return v;
+    }
+};
+
+// 16-byte packs (the ring executor's unit).
+template <int DT> struct Pack16 {
+    using P = PackW<DT, 4>;
+    static constexpr int L = P::L;
+    using A = typename P::A;
+    __device__ static void unpack(const uint4& v, A (&a)[L]) {
+        Words<4> w{{v.x, v.y, v.z, v.w}};
+        P::unpack(w, a);
+    }
+    __device__ static uint4 pack(const A (&a)[L]) {
+        const Words<4> w = P::pack(a);
+        return make_uint4(w.w[0], w.w[1], w.w[2], w.w[3]);
     }
 };
 
@@ -130,6 +154,34 @@ __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
 
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Streaming load / plain store of a pack of W words (W = 8 uses the 256-bit forms of sm_100).
+template <int W> __device__ __forceinline__ Words<W> ld_stream_words(const void* p);
+template <> __device__ __forceinline__ Words<4> ld_stream_words<4>(const void* p) {
+    Words<4> v;
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]) : "l"(p));
+    return v;
+}
+template <> __device__ __forceinline__ Words<8> ld_stream_words<8>(const void* p) {
+    Words<8> v;
+    asm volatile("ld.global.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+                   "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+template <int W> __device__ __forceinline__ void st_words(void* p, const Words<W>& v);
+template <> __device__ __forceinline__ void st_words<4>(void* p, const Words<4>& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3])
+                 : "memory");
+}
+template <> __device__ __forceinline__ void st_words<8>(void* p, const Words<8>& v) {
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                    "r"(v.w[7])
                  : "memory");
 }
 

@@ -20,12 +20,19 @@
 #include "common.cuh"
 #include "tile_geom.h"
 
+#include <algorithm>
+
 namespace simcomm {
 
 constexpr int kCopyThreads = 32;
-constexpr int kStages = 4;
 
-static_assert(kStages <= 32, "stage phases live in one 32-bit mask");
+// Pipeline shapes (stages x tile bytes, CTAs per SM), selected with the "copy_variant" option.
+struct CopyShape { int stages; uint32_t tile; int ctas_per_sm; };
+constexpr CopyShape kCopyShapes[] = {
+    {4, 32768, 1}, {6, 32768, 1}, {3, 65536, 1}, {2, 65536, 1},
+    {4, 16384, 2}, {6, 16384, 2}, {2, 32768, 3}, {8, 16384, 1},
+};
+constexpr int kNumCopyShapes = int(sizeof(kCopyShapes) / sizeof(kCopyShapes[0]));
 
 struct SegDesc {
     const char* src;
@@ -104,8 +111,9 @@ __device__ __forceinline__ int find_segment(const uint32_t* prefix, int nseg, ui
     return lo;
 }
 
-template <int KIND>
+template <int KIND, int kStages, uint32_t kTile>
 __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ CopyArgs a) {
+    static_assert(kStages <= 32, "stage phases live in one 32-bit mask");
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x;
     if (status_failed(a.ctl)) return;
@@ -126,14 +134,15 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     // tile counts per segment, then an inclusive scan into prefix[1..nseg]
     for (int s = lane; s < nseg; s += 32) {
         const SegDesc d = segment<KIND>(a, s, sd, rd);
-        prefix[s + 1] = tile_count(reinterpret_cast<uintptr_t>(d.src), d.len, congruent(a, d));
+        prefix[s + 1] = tile_count(reinterpret_cast<uintptr_t>(d.src), d.len, congruent(a, d), kTile);
     }
     __syncwarp();
     if (lane == 0) prefix[0] = 0;
-    uint32_t carry = 0;
+    uint32_t carry = 0, tmax = 0;
     for (int b = 0; b < nseg; b += 32) {
         const int s = b + lane;
         uint32_t v = (s < nseg) ? prefix[s + 1] : 0u;
+        tmax = max(tmax, v);
 #pragma unroll
         for (int dd = 1; dd < 32; dd <<= 1) {
             const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, v, dd);
@@ -142,8 +151,22 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         if (s < nseg) prefix[s + 1] = carry + v;
         carry += __shfl_sync(0xFFFFFFFFu, v, 31);
     }
+#pragma unroll
+    for (int dd = 16; dd > 0; dd >>= 1) tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
     __syncwarp();
-    const uint32_t total = prefix[nseg];
+    // Task order: segment-major, or interleaved (tile k of every segment before tile k+1 of any,
+    // so all sources and destinations are streamed at once; empty slots are skipped).
+    const uint32_t total = a.order ? tmax * uint32_t(nseg) : prefix[nseg];
+    auto locate = [&](uint32_t t, int* sg, uint32_t* k) -> bool {
+        if (!a.order) {
+            *sg = find_segment(prefix, nseg, t);
+            *k = t - prefix[*sg];
+            return true;
+        }
+        *sg = int(t % uint32_t(nseg));
+        *k = t / uint32_t(nseg);
+        return *k < prefix[*sg + 1] - prefix[*sg];
+    };
 
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
@@ -158,10 +181,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
 
     auto issue = [&](uint32_t k) {
         const uint32_t t = blockIdx.x + k * gridDim.x;
-        const int s = find_segment(prefix, nseg, t);
+        int s;
+        uint32_t ti;
+        if (!locate(t, &s, &ti)) return;
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
-        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, t - prefix[s]);
+        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, ti, kTile);
         if (lane == 0 && g.bhi > g.blo) {
             const int st = int(k % kStages);
             mbar_arrive_expect_tx(&bars[st], uint32_t(g.bhi - g.blo));
@@ -171,10 +196,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
 
     auto consume = [&](uint32_t k) {
         const uint32_t t = blockIdx.x + k * gridDim.x;
-        const int s = find_segment(prefix, nseg, t);
+        int s;
+        uint32_t ti;
+        if (!locate(t, &s, &ti)) return;
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
-        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, t - prefix[s]);
+        const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, ti, kTile);
         if (g.bhi > g.blo) {
             const int st = int(k % kStages);
             bool ok = true;
@@ -218,36 +245,209 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     __syncwarp();
 }
 
-static size_t copy_smem_bytes(int kind, int p) {
+// ---- load/store path -----------------------------------------------------------------------------
+// Tasks of kLsuTask bytes of a segment, handed to 256-thread CTAs round-robin; a task is copied
+// with 16-byte loads and stores (8 in flight per thread) where source and destination agree
+// modulo 16, else with 2-byte accesses. Measured faster than the bulk-copy pipeline for 1:1
+// copies (All-to-All(v)); the fan-out (Broadcast, AllGather) stays on bulk copies.
+constexpr int kLsuThreads = 256;
+constexpr int kLsuUnroll = 8;
+constexpr uint32_t kLsuTask = 128 * 1024;
+
+__device__ __forceinline__ void cta_copy_bytes(const char* s, char* d, size_t bytes) {
+    size_t head = bytes, body = 0;
+    if (((reinterpret_cast<uintptr_t>(s) ^ reinterpret_cast<uintptr_t>(d)) & 15u) == 0) {
+        head = (16 - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u;
+        if (head > bytes) head = bytes;
+        body = (bytes - head) & ~size_t(15);
+    }
+    for (size_t b = 2 * size_t(threadIdx.x); b < head; b += 2 * kLsuThreads)
+        *reinterpret_cast<uint16_t*>(d + b) = *reinterpret_cast<const uint16_t*>(s + b);
+    const uint4* vs = reinterpret_cast<const uint4*>(s + head);
+    uint4* vd = reinterpret_cast<uint4*>(d + head);
+    const size_t nv = body / 16;
+    for (size_t v0 = threadIdx.x; v0 < nv; v0 += size_t(kLsuThreads) * kLsuUnroll) {
+        uint4 t[kLsuUnroll];
+#pragma unroll
+        for (int u = 0; u < kLsuUnroll; ++u) {
+            const size_t v = v0 + size_t(u) * kLsuThreads;
+            if (v < nv) t[u] = ld_stream_v4(vs + v);
+        }
+#pragma unroll
+        for (int u = 0; u < kLsuUnroll; ++u) {
+            const size_t v = v0 + size_t(u) * kLsuThreads;
+            if (v < nv) st_v4(vd + v, t[u]);
+        }
+    }
+    for (size_t b = head + body + 2 * size_t(threadIdx.x); b < bytes; b += 2 * kLsuThreads)
+        *reinterpret_cast<uint16_t*>(d + b) = *reinterpret_cast<const uint16_t*>(s + b);
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_constant__ CopyArgs a) {
+    static_assert(KIND == COPY_ALLTOALL || KIND == COPY_ALLTOALLV, "1:1 segments only");
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ int s_run;
+    const int p = a.p;
+    const int nseg = p * p;
+    long long* sd = reinterpret_cast<long long*>(smem);
+    long long* rd = sd + ((KIND == COPY_ALLTOALLV) ? p * p : 0);
+    uint32_t* prefix = reinterpret_cast<uint32_t*>(rd + ((KIND == COPY_ALLTOALLV) ? p * p : 0));
+    if (threadIdx.x == 0) s_run = !status_failed(a.ctl);
+    __syncthreads();
+    if (!s_run) return;
+    if constexpr (KIND == COPY_ALLTOALLV) {
+        if (threadIdx.x < 32) {
+            const A2avPlan plan = a2av_plan_warp(a.counts, p, a.send_cap, a.recv_cap, sd, rd, a.recv_counts_out, a.ctl);
+            if (threadIdx.x == 0) s_run = plan.ok;
+        }
+        __syncthreads();
+        if (!s_run) return;
+    }
+    // tasks per segment and their prefix sums (warp 0)
+    __shared__ uint32_t s_tmax;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        if (lane == 0) prefix[0] = 0;
+        uint32_t carry = 0, tmax = 0;
+        for (int b = 0; b < nseg; b += 32) {
+            const int sg = b + lane;
+            uint32_t v = 0;
+            if (sg < nseg) {
+                const SegDesc d = segment<KIND>(a, sg, sd, rd);
+                v = uint32_t((d.len + kLsuTask - 1) / kLsuTask);
+            }
+            tmax = max(tmax, v);
+#pragma unroll
+            for (int dd = 1; dd < 32; dd <<= 1) {
+                const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, v, dd);
+                if (lane >= dd) v += o;
+            }
+            if (sg < nseg) prefix[sg + 1] = carry + v;
+            carry += __shfl_sync(0xFFFFFFFFu, v, 31);
+        }
+#pragma unroll
+        for (int dd = 16; dd > 0; dd >>= 1) tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
+        if (lane == 0) s_tmax = tmax;
+    }
+    __syncthreads();
+    const uint32_t total = a.order ? s_tmax * uint32_t(nseg) : prefix[nseg];
+    for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
+        int sg;
+        uint32_t k;
+        if (a.order) {
+            sg = int(t % uint32_t(nseg));
+            k = t / uint32_t(nseg);
+            if (k >= prefix[sg + 1] - prefix[sg]) continue;
+        } else {
+            sg = find_segment(prefix, nseg, t);
+            k = t - prefix[sg];
+        }
+        const SegDesc d = segment<KIND>(a, sg, sd, rd);
+        const size_t lo = size_t(k) * kLsuTask;
+        const size_t hi = min(lo + kLsuTask, d.len);
+        cta_copy_bytes(d.src + lo, d.dst + lo, hi - lo);
+    }
+}
+
+static size_t lsu_smem_bytes(int kind, int p) {
+    size_t b = (kind == COPY_ALLTOALLV) ? 2 * size_t(p) * p * sizeof(long long) : 0;
+    return b + (size_t(p) * p + 1) * sizeof(uint32_t);
+}
+
+template <int KIND>
+static cudaError_t launch_lsu(const CopyArgs& a, int num_sms, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_copy_lsu<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(lsu_smem_bytes(KIND, kMaxRanks)));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    k_copy_lsu<KIND><<<num_sms * 2, kLsuThreads, lsu_smem_bytes(KIND, a.p), s>>>(a);
+    return cudaGetLastError();
+}
+
+static size_t copy_smem_bytes(int kind, int p, int stages, uint32_t tile) {
     const int nseg = (kind == COPY_BCAST) ? 1 : (kind == COPY_ALLGATHER) ? p : p * p;
-    size_t b = size_t(kStages) * kTile + size_t(kStages) * sizeof(uint64_t);
+    size_t b = size_t(stages) * tile + size_t(stages) * sizeof(uint64_t);
     if (kind == COPY_ALLTOALLV) b += 2 * size_t(p) * p * sizeof(long long);
     b += (size_t(nseg) + 1) * sizeof(uint32_t);
     return (b + 127) & ~size_t(127);
 }
 
-template <int KIND>
-static cudaError_t launch_kind(const CopyArgs& a, int num_sms, cudaStream_t s) {
-    const size_t smem = copy_smem_bytes(KIND, a.p);
+static int max_smem_optin() {
+    static int v = -1;
+    if (v < 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            v = 48 * 1024;
+    }
+    return v;
+}
+
+template <int KIND, int V>
+static cudaError_t launch_shape(const CopyArgs& a, int num_sms, cudaStream_t s) {
+    constexpr CopyShape sh = kCopyShapes[V];
+    auto kernel = k_copy<KIND, sh.stages, sh.tile>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_copy<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(copy_smem_bytes(KIND, kMaxRanks)));
+        const size_t want = std::min<size_t>(copy_smem_bytes(KIND, kMaxRanks, sh.stages, sh.tile), size_t(max_smem_optin()));
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(want));
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    k_copy<KIND><<<num_sms, kCopyThreads, smem, s>>>(a);
+    kernel<<<num_sms * sh.ctas_per_sm, kCopyThreads, copy_smem_bytes(KIND, a.p, sh.stages, sh.tile), s>>>(a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_copy(const CopyArgs& a, int num_sms, cudaStream_t s) {
+template <int KIND>
+static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
+    if (variant < 0 || variant >= kNumCopyShapes ||
+        copy_smem_bytes(KIND, a.p, kCopyShapes[variant].stages, kCopyShapes[variant].tile) > size_t(max_smem_optin()))
+        variant = 0;  // the baseline shape fits every p
+    switch (variant) {
+        case 1: return launch_shape<KIND, 1>(a, num_sms, s);
+        case 2: return launch_shape<KIND, 2>(a, num_sms, s);
+        case 3: return launch_shape<KIND, 3>(a, num_sms, s);
+        case 4: return launch_shape<KIND, 4>(a, num_sms, s);
+        case 5: return launch_shape<KIND, 5>(a, num_sms, s);
+        case 6: return launch_shape<KIND, 6>(a, num_sms, s);
+        case 7: return launch_shape<KIND, 7>(a, num_sms, s);
+        default: return launch_shape<KIND, 0>(a, num_sms, s);
+    }
+}
+
+// Per-collective defaults, the fastest measured on B200 at the DP-bucket size (p = 8, 100 MiB per
+// rank): Broadcast and AllGather on the bulk-copy pipeline with 6 stages of 16 KiB and 2 CTAs per
+// SM; All-to-All on 4 stages of 32 KiB with the interleaved tile order; All-to-Allv (whose skewed
+// blocks leave most interleaved slots empty) on the load/store path, block after block.
+constexpr int kVariantLsu = kNumCopyShapes;
+
+void copy_defaults(int kind, int* variant, int* order) {
+    switch (kind) {
+        case COPY_ALLTOALL: *variant = 0; *order = 1; break;
+        case COPY_ALLTOALLV: *variant = kVariantLsu; *order = 0; break;
+        default: *variant = 5; *order = 0; break;
+    }
+}
+
+cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
+    if (variant == kVariantLsu) {
+        if (a.kind == COPY_ALLTOALL) return launch_lsu<COPY_ALLTOALL>(a, num_sms, s);
+        if (a.kind == COPY_ALLTOALLV) return launch_lsu<COPY_ALLTOALLV>(a, num_sms, s);
+        variant = 5;  // fan-out collectives have no load/store variant
+    }
     switch (a.kind) {
-        case COPY_BCAST: return launch_kind<COPY_BCAST>(a, num_sms, s);
-        case COPY_ALLGATHER: return launch_kind<COPY_ALLGATHER>(a, num_sms, s);
-        case COPY_ALLTOALL: return launch_kind<COPY_ALLTOALL>(a, num_sms, s);
-        case COPY_ALLTOALLV: return launch_kind<COPY_ALLTOALLV>(a, num_sms, s);
+        case COPY_BCAST: return launch_kind<COPY_BCAST>(a, num_sms, variant, s);
+        case COPY_ALLGATHER: return launch_kind<COPY_ALLGATHER>(a, num_sms, variant, s);
+        case COPY_ALLTOALL: return launch_kind<COPY_ALLTOALL>(a, num_sms, variant, s);
+        case COPY_ALLTOALLV: return launch_kind<COPY_ALLTOALLV>(a, num_sms, variant, s);
         default: return cudaErrorInvalidValue;
     }
 }
+
+int copy_num_variants() { return kNumCopyShapes + 1; }
 
 }  // namespace simcomm

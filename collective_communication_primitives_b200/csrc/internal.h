@@ -39,10 +39,11 @@ struct DirectReduceArgs {
     int p;
     int mode;
     int root;
-    int vec;           // 1: 16-byte packs, 0: element-wise
+    int vec;           // 2: 32-byte packs, 1: 16-byte packs, 0: element-wise
     size_t n;          // per-rank full element count
     size_t seg;        // ReduceScatter: elements per owner (n / p); otherwise n
     float scale;       // AVG: 1/p; otherwise 1
+    int ctas_per_sm;   // grid = SMs x this (capped by the work)
     Ctl ctl;
 };
 
@@ -56,6 +57,7 @@ struct CopyArgs {
     int root;
     int elem_bytes;
     size_t blk_elems;                  // BCAST: n; ALLGATHER: shard n/p; ALLTOALL: block n/p
+    int order;                         // tile order: 0 segment-major, 1 interleaved over segments
     const long long* counts;           // ALLTOALLV: device [p][p]
     long long* recv_counts_out;        // ALLTOALLV: device [p] or null
     long long send_cap[kMaxRanks];     // ALLTOALLV: elements per send buffer
@@ -102,7 +104,9 @@ struct RingArgs {
 
 // Launchers (each returns the launch error; grid sizes are decided inside).
 cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, int num_sms, cudaStream_t s);
-cudaError_t launch_copy(const CopyArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s);
+int copy_num_variants();
+void copy_defaults(int kind, int* variant, int* order);
 cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 int ring_max_ctas(int num_sms);
 

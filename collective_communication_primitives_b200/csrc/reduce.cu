@@ -1,6 +1,6 @@
 // Direct fused reduction: AllReduce, Reduce and ReduceScatter in one pass.
 //
-// Each thread takes a 16-byte position i of the reduced range, loads that position from all p
+// Each thread takes a 32-byte (or 16-byte) position i of the reduced range, loads that position from all p
 // ranks' inputs (all loads issued before the first add), folds them in rank order in fp32 (bf16 is
 // widened; int32 wraps), scales by 1/p for AVG, rounds once, and stores the result to every owner:
 // all p outputs for AllReduce, the root's output for Reduce, the owner's shard for ReduceScatter.
@@ -57,9 +57,10 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_scalar(const __grid_cons
 
 // P > 0: p is a compile-time constant and all p loads of a position are in flight together.
 // P == 0: p is read at run time and ranks are loaded kDirGroup at a time.
-template <int DT, int OP, int P, bool SCALE>
+// W: 32-bit words per pack (4: 16-byte accesses, 8: 32-byte accesses).
+template <int DT, int OP, int P, bool SCALE, int W>
 __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constant__ DirectReduceArgs a) {
-    using PK = Pack16<DT>;
+    using PK = PackW<DT, W>;
     using A = typename PK::A;
     constexpr int L = PK::L;
     constexpr int G = (P > 0) ? P : kDirGroup;
@@ -83,14 +84,14 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
 
             A acc[kDirUnroll][L];
             for (int q0 = 0; q0 < p; q0 += G) {
-                uint4 v[kDirUnroll][G];
+                Words<W> v[kDirUnroll][G];
 #pragma unroll
                 for (int u = 0; u < kDirUnroll; ++u)
 #pragma unroll
                     for (int j = 0; j < G; ++j)
                         if (ok[u] && (P > 0 || q0 + j < p))
-                            v[u][j] = ld_stream_v4(static_cast<const uint4*>(a.ptrs.send[q0 + j]) + in_base + i0 +
-                                                   size_t(u) * kDirThreads);
+                            v[u][j] = ld_stream_words<W>(static_cast<const Words<W>*>(a.ptrs.send[q0 + j]) +
+                                                         in_base + i0 + size_t(u) * kDirThreads);
 #pragma unroll
                 for (int u = 0; u < kDirUnroll; ++u) {
 #pragma unroll
@@ -114,19 +115,21 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
 #pragma unroll
                     for (int l = 0; l < L; ++l) acc[u][l] = acc[u][l] * a.scale;
                 }
-                const uint4 out = PK::pack(acc[u]);
+                const Words<W> out = PK::pack(acc[u]);
                 const size_t idx = i0 + size_t(u) * kDirThreads;
                 if (a.mode == MODE_ALLREDUCE) {
                     if constexpr (P > 0) {
 #pragma unroll
-                        for (int r = 0; r < P; ++r) st_v4(static_cast<uint4*>(a.ptrs.recv[r]) + in_base + idx, out);
+                        for (int r = 0; r < P; ++r)
+                            st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out);
                     } else {
-                        for (int r = 0; r < p; ++r) st_v4(static_cast<uint4*>(a.ptrs.recv[r]) + in_base + idx, out);
+                        for (int r = 0; r < p; ++r)
+                            st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out);
                     }
                 } else if (a.mode == MODE_REDUCE) {
-                    st_v4(static_cast<uint4*>(a.ptrs.recv[a.root]) + in_base + idx, out);
+                    st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[a.root]) + in_base + idx, out);
                 } else {
-                    st_v4(static_cast<uint4*>(a.ptrs.recv[sg]) + idx, out);
+                    st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[sg]) + idx, out);
                 }
             }
         }
@@ -143,23 +146,37 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
 
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStream_t s) {
-    const int max_blocks = num_sms * 4;
+    const int max_blocks = num_sms * (a.ctas_per_sm > 0 ? a.ctas_per_sm : 4);
     if (!a.vec) {
         const size_t want = (a.n + kDirThreads - 1) / kDirThreads;
         const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
         k_direct_scalar<DT, OP, SCALE><<<grid, kDirThreads, 0, s>>>(a);
         return cudaGetLastError();
     }
-    constexpr int L = Pack16<DT>::L;
+    // 32-byte packs when every buffer allows them, else 16-byte packs
+    if (a.vec == 2) {
+        constexpr int L = PackW<DT, 8>::L;
+        const size_t packs = a.seg / L;
+        const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
+        const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
+        switch (a.p) {
+            case 2: k_direct_vec<DT, OP, 2, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
+            case 4: k_direct_vec<DT, OP, 4, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
+            case 8: k_direct_vec<DT, OP, 8, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
+            default: k_direct_vec<DT, OP, 0, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
+        }
+        return cudaGetLastError();
+    }
+    constexpr int L = PackW<DT, 4>::L;
     const size_t packs = a.seg / L;
     const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
     const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
     switch (a.p) {
-        case 2: k_direct_vec<DT, OP, 2, SCALE><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 3: k_direct_vec<DT, OP, 3, SCALE><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 4: k_direct_vec<DT, OP, 4, SCALE><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 8: k_direct_vec<DT, OP, 8, SCALE><<<grid, kDirThreads, 0, s>>>(a); break;
-        default: k_direct_vec<DT, OP, 0, SCALE><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 2: k_direct_vec<DT, OP, 2, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 3: k_direct_vec<DT, OP, 3, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 4: k_direct_vec<DT, OP, 4, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 8: k_direct_vec<DT, OP, 8, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
+        default: k_direct_vec<DT, OP, 0, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
     }
     return cudaGetLastError();
 }

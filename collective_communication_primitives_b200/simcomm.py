@@ -182,32 +182,32 @@ class SimComm:
     # -- collectives (n follows include/simcomm.h: the per-rank FULL buffer) -----------------------
     def allreduce(self, sends, recvs, op="sum", algo="direct", n=None, dtype=None, stream=None):
         n = sends[0].numel() if n is None else n
-        self._check(self._L.coll_allreduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+        self._check(self._L.coll_allreduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                            OPS[op], ALGOS[algo], _stream(stream)))
 
     def reduce(self, sends, recvs, root, op="sum", algo="direct", n=None, dtype=None, stream=None):
         n = sends[0].numel() if n is None else n
-        self._check(self._L.coll_reduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends), OPS[op],
+        self._check(self._L.coll_reduce(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)), OPS[op],
                                         int(root), ALGOS[algo], _stream(stream)))
 
     def broadcast(self, sends, recvs, root, algo="direct", n=None, dtype=None, stream=None):
         n = recvs[0].numel() if n is None else n
-        self._check(self._L.coll_broadcast(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, recvs),
+        self._check(self._L.coll_broadcast(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                            int(root), ALGOS[algo], _stream(stream)))
 
     def reduce_scatter(self, sends, recvs, op="sum", algo="direct", n=None, dtype=None, stream=None):
         n = sends[0].numel() if n is None else n
-        self._check(self._L.coll_reduce_scatter(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+        self._check(self._L.coll_reduce_scatter(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                                 OPS[op], ALGOS[algo], _stream(stream)))
 
     def allgather(self, sends, recvs, algo="direct", n=None, dtype=None, stream=None):
         n = recvs[0].numel() if n is None else n
-        self._check(self._L.coll_allgather(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, recvs),
+        self._check(self._L.coll_allgather(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                            ALGOS[algo], _stream(stream)))
 
     def alltoall(self, sends, recvs, algo="direct", n=None, dtype=None, stream=None):
         n = sends[0].numel() if n is None else n
-        self._check(self._L.coll_alltoall(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, sends),
+        self._check(self._L.coll_alltoall(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                           ALGOS[algo], _stream(stream)))
 
     def alltoallv(self, sends, recvs, counts, send_cap=None, recv_cap=None, algo="direct", recv_counts=None,
@@ -220,5 +220,5 @@ class SimComm:
         sc = (ctypes.c_longlong * p)(*[int(x) for x in send_cap])
         rc = (ctypes.c_longlong * p)(*[int(x) for x in recv_cap])
         self._check(self._L.coll_alltoallv(self._h, self._bufs(sends, recvs), ctypes.c_void_p(_ptr(counts)), sc, rc,
-                                           self._resolve(dtype, sends), ALGOS[algo], _stream(stream),
+                                           self._resolve(dtype, list(sends) + list(recvs)), ALGOS[algo], _stream(stream),
                                            ctypes.c_void_p(_ptr(recv_counts)) if recv_counts is not None else None))

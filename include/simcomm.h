@@ -112,6 +112,14 @@ const char* coll_status_string(coll_status_t status);
  *   "timeout_ns"   longest wait of one ring step for its predecessor (default 2e9)
  *   "fault_skip_rank"  debugging: the ring executor never signals this rank's steps, so its
  *                  successor times out (-1 = off, the default). Host-side fault injection only.
+ *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v): -1 = the default per
+ *                  collective; 0..7 = a bulk-copy pipeline shape (stages x tile bytes, CTAs per SM);
+ *                  8 = the 16-byte load/store path (All-to-All(v) only)
+ *   "copy_order"   tile order of the direct copy paths: -1 = the default per collective,
+ *                  1 = interleaved over all blocks, 0 = block after block
+ *   "direct_pack"  access width of the fused reduction: 0 = widest the alignment allows
+ *                  (32 bytes), 16 = at most 16 bytes
+ *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16)
  * Returns COLL_ERR_INVALID_ARG for an unknown key or a value out of range. */
 coll_status_t sim_comm_set_option(sim_comm_t comm, const char* key, long long value);
 coll_status_t sim_comm_get_option(sim_comm_t comm, const char* key, long long* value);

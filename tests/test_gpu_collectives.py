@@ -26,6 +26,8 @@ def comm(p):
     c.set_option("chunk_bytes", 1 << 20)
     c.set_option("fault_skip_rank", -1)
     c.set_option("timeout_ns", 2_000_000_000)
+    c.set_option("copy_variant", -1)
+    c.set_option("copy_order", -1)
     return c
 
 
@@ -531,3 +533,49 @@ def test_launch_count_counts_kernels():
     c.allgather([x[:128] for x in t], u)
     torch.cuda.synchronize()
     assert c.launch_count() - before == 3
+
+
+@pytest.mark.parametrize("order", [-1, 0, 1])
+@pytest.mark.parametrize("variant", list(range(-1, 9)))
+@pytest.mark.parametrize("p", [3, 8])
+def test_copy_engine_variants(variant, p, order):
+    """Every copy path (the per-collective default, each bulk-copy pipeline shape and the
+    load/store path) in both tile orders gives the oracle's results."""
+    c = comm(p)
+    c.set_option("copy_variant", variant)
+    c.set_option("copy_order", order)
+    try:
+        for n, off in ((p * 7, 0), (p * 40961, 1), (p * 300007, 0)):
+            m = n // p
+            ins = make_inputs("int24", p, n, "int32", f"cv.{p}.{n}")
+            src = [Guarded(n, "int32", offset=off, fill=x) for x in ins]
+            out = [Guarded(n, "int32") for _ in ins]
+            c.broadcast([b.t for b in src], [b.t for b in out], 1, algo="direct")
+            finish(c, src + out)
+            for r in range(p):
+                np.testing.assert_array_equal(out[r].numpy(), ins[1])
+            shards = [x[:m].copy() for x in ins]
+            sh = [Guarded(m, "int32", offset=off, fill=x) for x in shards]
+            ag = [Guarded(n, "int32", offset=off) for _ in ins]
+            c.allgather([b.t for b in sh], [b.t for b in ag], algo="direct")
+            finish(c, sh + ag)
+            for r, w in enumerate(O.allgather(shards, "int32")):
+                np.testing.assert_array_equal(ag[r].numpy(), w)
+            a2a = [Guarded(n, "int32") for _ in ins]
+            c.alltoall([b.t for b in src], [b.t for b in a2a], algo="direct")
+            finish(c, a2a)
+            for r, w in enumerate(O.alltoall(ins, "int32")):
+                np.testing.assert_array_equal(a2a[r].numpy(), w)
+            counts = np.random.default_rng(n).integers(0, m // p + 3, size=(p, p))
+            rows = counts.sum(axis=1)
+            vsrc = [Guarded(int(rows[i]), "int32", fill=ins[i][:rows[i]]) for i in range(p)]
+            cap = int(counts.sum(axis=0).max())
+            vdst = [Guarded(cap, "int32") for _ in range(p)]
+            c.alltoallv([b.t for b in vsrc], [b.t for b in vdst], torch.tensor(counts, device="cuda"), algo="direct")
+            finish(c, vsrc + vdst)
+            want, _ = O.alltoallv([ins[i][:rows[i]] for i in range(p)], counts, "int32")
+            for j in range(p):
+                np.testing.assert_array_equal(vdst[j].numpy()[:want[j].size], want[j])
+    finally:
+        c.set_option("copy_variant", -1)
+        c.set_option("copy_order", -1)

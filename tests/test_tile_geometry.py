@@ -14,12 +14,13 @@ PROGRAM = r'''
 #include <initializer_list>
 #include "tile_geom.h"
 using namespace simcomm;
+static uint32_t kTile = 32768;
 static int check(uint64_t src, size_t len, bool cong) {
-    uint32_t n = tile_count(src, len, cong);
+    uint32_t n = tile_count(src, len, cong, kTile);
     if (len == 0) return n == 0 ? 0 : 1;
     size_t covered = 0;
     for (uint32_t k = 0; k < n; ++k) {
-        TileGeom g = tile_geom(src, len, cong, k);
+        TileGeom g = tile_geom(src, len, cong, k, kTile);
         if (g.lo != covered) return 2;
         if (!(g.lo < g.hi && g.hi <= len)) return 3;
         if (!(g.lo <= g.blo && g.blo <= g.bhi && g.bhi <= g.hi)) return 4;
@@ -35,11 +36,13 @@ static int check(uint64_t src, size_t len, bool cong) {
     return covered == len ? 0 : 10;
 }
 int main() {
+  int bad = 0;
+  for (uint32_t tsz : {16384u, 32768u, 65536u}) {
+    kTile = tsz;
     const size_t lens[] = {1, 2, 3, 4, 6, 8, 12, 14, 15, 16, 17, 18, 30, 31, 32, 33, 46, 100,
                            kTile - 17, kTile - 16, kTile - 2, kTile - 1, kTile, kTile + 1, kTile + 2,
                            kTile + 14, kTile + 15, kTile + 16, 2 * kTile - 4, 2 * kTile, 3 * kTile + 6,
                            1000003, 4194304};
-    int bad = 0;
     for (uint64_t base : {0x7f0000000000ull, 0x7f0000000100ull})
         for (int off = 0; off < 16; off += 2)
             for (size_t len : lens)
@@ -50,6 +53,7 @@ int main() {
     for (size_t len = 0; len < 200; len += 2)
         for (int off = 0; off < 16; off += 2)
             if (int r = check(0x1000 + off, len, true)) { std::printf("FAIL small off=%d len=%zu code=%d\n", off, len, r); ++bad; }
+  }
     std::printf(bad ? "BAD\n" : "OK\n");
     return bad ? 1 : 0;
 }
