@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -738,3 +739,130 @@ coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* count
 }
 
 }  // extern "C"
+
+// =================================================================================================
+// Ring AllReduce without any allocation.
+//
+// Some callers cannot call cudaMalloc: code that runs while a CUDA graph is being captured with a
+// no-allocation policy, code inside a memory-pool or allocator implementation, or a process that
+// must not grow its device footprint after start-up. For them this entry point runs the same ring
+// AllReduce kernel as coll_allreduce(..., COLL_ALGO_RING, ...) on a fixed scratch area that is part
+// of the library image: a file-scope device array of kStaticScratchBytes. No communicator is
+// created and nothing is allocated or freed per call.
+//
+// The array lives in device memory of every GPU that loads this library until the process exits.
+// In host code its name is only a host-side handle, never a device address: a kernel given it
+// would fault, or silently use the wrong memory where the GPU can reach host memory. Its device
+// address is therefore looked up once per device, with that device current, by the first call on
+// that device (cudaGetSymbolAddress); that first call should come before any stream capture.
+// Every call shares the array and it keeps the last call's contents: each call clears the control
+// words and chunk flags it needs on its stream before the kernel, and calls whose work overlaps on
+// the GPU (other streams, other host threads) race on the array and must be ordered by the caller.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_mu;
+char* g_static_base[kMaxStaticDevices] = {};
+int g_static_sms[kMaxStaticDevices] = {};
+int g_static_ctas[kMaxStaticDevices] = {};
+
+}  // namespace
+
+extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                                     int* async_status_dev, coll_stream_t stream) {
+    coll_status_t st;
+    if (p < 2 || p > SIM_COMM_MAX_RANKS) return fail(COLL_ERR_INVALID_ARG, "p must be in [2, 64]");
+    if ((st = check_reduce_args(dt, op)) != COLL_OK) return st;
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), bytes = n * d;
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], bytes, d, "send")) != COLL_OK) return st;
+        if ((st = check_ptr(b.recv[r], bytes, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + bytes, false, r});
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + bytes, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_SAME, 0)) != COLL_OK) return st;
+
+    // Layout of the scratch: control words, chunk flags, then one partial buffer per rank.
+    const size_t seg = (n + size_t(p) - 1) / size_t(p);
+    const size_t chunk = (size_t(1) << 20) / 4;
+    const uint32_t nch = chunks_of(seg, chunk);
+    const uint32_t nsteps = uint32_t(2 * (p - 1));
+    const size_t ctl_bytes = 256;
+    const size_t flag_bytes = round_up(size_t(nsteps) * p * nch * sizeof(unsigned long long), 256);
+    const size_t stride = round_up(n * 4, 256);
+    const size_t need = ctl_bytes + flag_bytes + size_t(p) * stride;
+    if (need > kStaticScratchBytes)
+        return fail(COLL_ERR_INVALID_ARG, "coll_allreduce_ring_noalloc needs " + std::to_string(need) +
+                                              " bytes of scratch; its static scratch holds " +
+                                              std::to_string(kStaticScratchBytes) + " (p * n * 4 must stay below ~32 MiB)");
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxStaticDevices) return fail(COLL_ERR_UNSUPPORTED, "device ordinal above 63");
+    char* base;
+    int ctas;
+    {
+        std::lock_guard<std::mutex> lock(g_static_mu);
+        if (!g_static_base[dev]) {
+            void* ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+            e = cudaDeviceGetAttribute(&g_static_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+            g_static_ctas[dev] = ring_max_ctas(g_static_sms[dev]);
+            g_static_base[dev] = static_cast<char*>(ptr);
+        }
+        base = g_static_base[dev];
+        ctas = g_static_ctas[dev];
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the control words and flags must start at zero for this call
+    e = cudaMemsetAsync(base, 0, ctl_bytes + flag_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(static scratch)");
+
+    RingArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.p = p;
+    a.kind = RING_ALLREDUCE;
+    a.root = 0;
+    a.n = n;
+    a.seg = seg;
+    a.chunk = chunk;
+    a.tile = std::min(chunk, std::max<size_t>(16, kRingTaskBytes / 4));
+    a.ntile = uint32_t((chunk + a.tile - 1) / a.tile);
+    a.elem_bytes = int(d);
+    a.nch = nch;
+    a.nsteps = nsteps;
+    a.ranks_per_step = uint32_t(p);
+    a.epoch = 1;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.skip_rank = -1;
+    a.timeout_ns = 2000000000ULL;
+    a.st = reinterpret_cast<DevState*>(base);
+    a.ctl.status = &a.st->status;
+    a.ctl.host_status = reinterpret_cast<uint32_t*>(base + 64);
+    a.ctl.abort_flag = reinterpret_cast<uint32_t*>(base + 68);
+    a.flags = reinterpret_cast<unsigned long long*>(base + ctl_bytes);
+    a.stage = base + ctl_bytes + flag_bytes;
+    a.stage_stride = stride;
+    bool vec = (seg * d) % 16 == 0 && (seg * 4) % 16 == 0 && (chunk * d) % 16 == 0;
+    for (int r = 0; r < p; ++r) vec = vec && aligned16(a.ptrs.send[r]) && aligned16(a.ptrs.recv[r]);
+    a.vec = vec ? 1 : 0;
+    const size_t tasks = size_t(nsteps) * p * nch * a.ntile;
+    if (tasks < size_t(ctas)) ctas = int(std::max<size_t>(tasks, 1));
+    e = launch_ring(a, dt, op, ctas, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ring executor launch");
+    if (async_status_dev) {
+        e = cudaMemcpyAsync(async_status_dev, &a.st->status, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(status)");
+    }
+    return COLL_OK;
+}

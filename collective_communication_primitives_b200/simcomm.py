@@ -72,8 +72,9 @@ def load_library(path=LIB_PATH):
     L.coll_allgather.argtypes = [vp, _Bufs, sz, i32, i32, vp]
     L.coll_alltoall.argtypes = [vp, _Bufs, sz, i32, i32, vp]
     L.coll_alltoallv.argtypes = [vp, _Bufs, vp, llp, llp, i32, i32, vp, vp]
+    L.coll_allreduce_ring_noalloc.argtypes = [i32, _Bufs, sz, i32, i32, vp, vp]
     for name in ("coll_allreduce", "coll_reduce", "coll_broadcast", "coll_reduce_scatter", "coll_allgather",
-                 "coll_alltoall", "coll_alltoallv"):
+                 "coll_alltoall", "coll_alltoallv", "coll_allreduce_ring_noalloc"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -222,3 +223,21 @@ class SimComm:
         self._check(self._L.coll_alltoallv(self._h, self._bufs(sends, recvs), ctypes.c_void_p(_ptr(counts)), sc, rc,
                                            self._resolve(dtype, list(sends) + list(recvs)), ALGOS[algo], _stream(stream),
                                            ctypes.c_void_p(_ptr(recv_counts)) if recv_counts is not None else None))
+
+
+def allreduce_ring_noalloc(sends, recvs, op="sum", n=None, dtype=None, status=None, stream=None):
+    """Ring AllReduce on the library's static scratch: no communicator, no allocation (for callers
+    that cannot allocate device memory; see include/simcomm.h). `status` is an optional device int32
+    tensor that receives the call's asynchronous status."""
+    L = load_library()
+    p = len(sends)
+    n = sends[0].numel() if n is None else n
+    s = (ctypes.c_void_p * p)(*[_ptr(x) for x in sends])
+    r = (ctypes.c_void_p * p)(*[_ptr(x) for x in recvs])
+    bufs = _Bufs(ctypes.cast(s, ctypes.POINTER(ctypes.c_void_p)), ctypes.cast(r, ctypes.POINTER(ctypes.c_void_p)))
+    dt = SimComm._resolve(dtype, list(sends) + list(recvs))
+    rc = L.coll_allreduce_ring_noalloc(p, bufs, n, dt, OPS[op], ctypes.c_void_p(_ptr(status)) if status is not None
+                                       else None, _stream(stream))
+    if rc != OK:
+        raise SimCommError(rc, L.sim_comm_last_error().decode())
+

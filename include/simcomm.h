@@ -187,6 +187,32 @@ coll_status_t coll_alltoallv(sim_comm_t comm, coll_bufs_t bufs, const long long*
                              const long long* send_cap, const long long* recv_cap, coll_dtype_t dtype,
                              coll_algo_t algo, coll_stream_t stream, long long* recv_counts_dev);
 
+/* ---- no-allocation variant ------------------------------------------------------------------ */
+
+/* Ring AllReduce that allocates nothing. (The pages have no counterpart: this is a library
+ * facility, not part of the collective's definition.)
+ *
+ * For callers that cannot call cudaMalloc: code running while a CUDA graph is captured under a
+ * no-allocation policy, code inside an allocator or memory pool, or a process that must not grow
+ * its device footprint after start-up. It computes exactly what coll_allreduce(..., COLL_ALGO_RING,
+ * ...) computes on a communicator of p ranks (same kernel, same schedule, same rounding), but needs
+ * no communicator: its scratch (control words, chunk flags, one fp32/int32 partial buffer per
+ * rank) is a fixed 32 MiB device array inside the library, held on every GPU that loads the
+ * library until the process exits.
+ *   p, bufs, n, dtype, op  as for coll_allreduce (2 <= p <= 64).
+ *   async_status_dev  DEVICE int the caller owns, or NULL: receives COLL_OK or the asynchronous
+ *                     error of this call (COLL_ERR_TIMEOUT if a ring step waited 2 s), in stream
+ *                     order.
+ * Limits and errors: the scratch must hold p * round_up(4n, 256) bytes of partials plus the flags
+ * (about p * n * 4 < 32 MiB, e.g. n up to ~1M elements at p = 8); larger calls return
+ * COLL_ERR_INVALID_ARG with the sizes in sim_comm_last_error(). Other argument errors as for
+ * coll_allreduce. The first call on a device looks up the scratch's device address on that device
+ * (make that first call before any stream capture). Every call shares the scratch and clears what
+ * must start at zero on its own stream; calls that overlap on the GPU race on it and must be
+ * ordered by the caller. */
+coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t bufs, size_t n, coll_dtype_t dtype, coll_op_t op,
+                                          int* async_status_dev, coll_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
