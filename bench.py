@@ -31,6 +31,10 @@ N_BUCKET = 26_214_400
 HIDDEN = 4096
 ROOT_RANK = 2
 FALLBACK_HBM_GBS = 6650.0
+# dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of a row's kernel, with the
+# per-rank element count of that capture; scaled to the bench's size by elements moved. Empty
+# until a capture of the current build is taken.
+NCU_TRAFFIC = {}
 
 
 def parse():
@@ -44,6 +48,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ops", default="", help="comma-separated substrings: run only the matching rows")
     ap.add_argument("--option", action="append", default=[], help="communicator option key=value")
+    ap.add_argument("--sweep", action="store_true",
+                    help="size/rank sweep with alpha-beta fits instead of the step (one GPU)")
+    ap.add_argument("--sweep-ps", default="2,4,8,16,64")
+    ap.add_argument("--sweep-max-bytes", type=int, default=1 << 30, help="largest per-rank message")
+    ap.add_argument("--sweep-out", default="", help="write the sweep's markdown summary here")
     return ap.parse_args()
 
 
@@ -55,6 +64,26 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# multi-GPU: independent replicas (one simulated communicator per GPU); the only cross-rank
+# traffic is the timing plumbing below
+
+def reduce_max(x, device=None):
+    """Max of a host scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbps(world, bytes_per_step_per_rank, ms_per_step):
+    """Whole-job throughput: every rank moves its step's bytes; the slowest rank sets the time."""
+    return world * bytes_per_step_per_rank / (ms_per_step / 1e3) / 1e9
 
 
 # ---------------------------------------------------------------------------------------------
@@ -339,11 +368,131 @@ def reference_arm(args):
 
 
 # ---------------------------------------------------------------------------------------------
+# size / rank sweep: latency, algbw, busbw and alpha-beta fits per (op, path, p)
+
+SWEEP_OPS = ("allreduce", "reduce", "broadcast", "reduce_scatter", "allgather", "alltoall")
+SWEEP_CAP_BYTES = 64 << 30  # total device memory a point may hold
+
+
+def sweep(args):
+    import numpy as np
+    import torch
+
+    from collective_communication_primitives_b200 import bytemodel as BM
+    from collective_communication_primitives_b200 import simcomm as SC
+    torch.cuda.set_device(0)
+    dev = "cuda:0"
+    stream = torch.cuda.current_stream()
+    sizes = []
+    b = 1024
+    while b <= args.sweep_max_bytes:
+        sizes.append(b)
+        b *= 4
+    rows = []
+    for p in [int(x) for x in args.sweep_ps.split(",")]:
+        comm = SC.SimComm(p)
+        for algo in ("direct", "ring"):
+            for nbytes in sizes:
+                n = max(p, (nbytes // 4) // p * p)     # int32 elements, divisible by p
+                hold = 2 * p * n * 4 + (p * n * 4 if algo == "ring" else 0)
+                if hold > SWEEP_CAP_BYTES:
+                    continue
+                x = [torch.randint(-2**24, 2**24, (n,), dtype=torch.int32, device=dev) for _ in range(p)]
+                y = [torch.empty(n, dtype=torch.int32, device=dev) for _ in range(p)]
+                m = n // p
+                calls = {
+                    "allreduce": lambda: comm.allreduce(x, y, op="sum", algo=algo),
+                    "reduce": lambda: comm.reduce(x, y, 0, op="sum", algo=algo),
+                    "broadcast": lambda: comm.broadcast(x, y, 0, algo=algo),
+                    "reduce_scatter": lambda: comm.reduce_scatter(x, [t[:m] for t in y], op="sum", algo=algo),
+                    "allgather": lambda: comm.allgather([t[:m] for t in x], y, algo=algo),
+                    "alltoall": lambda: comm.alltoall(x, y, algo=algo),
+                }
+                for op in SWEEP_OPS:
+                    f = calls[op]
+                    for _ in range(3):
+                        f()
+                    torch.cuda.synchronize()
+                    ts = []
+                    for _ in range(10):
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record(stream)
+                        f()
+                        e1.record(stream)
+                        e1.synchronize()
+                        ts.append(e0.elapsed_time(e1))
+                    ms = float(np.median(ts))
+                    msg = n * 4  # per-rank message: the AllReduce in/out, ReduceScatter input, AllGather output
+                    hbm = BM.direct_hbm_bytes(op, p, n, 4)
+                    algbw = msg / (ms / 1e3) / 1e9
+                    rows.append({"p": p, "algo": algo, "op": op, "bytes_per_rank": msg, "ms": ms,
+                                 "algbw_GBps": algbw, "busbw_GBps": algbw * BM.busbw_factor(op, p),
+                                 "hbm_GBps": hbm / (ms / 1e3) / 1e9,
+                                 "l2_resident": p * msg * 2 < 2 * 126e6})
+                    assert comm.async_error() == SC.OK
+                del x, y
+                torch.cuda.empty_cache()
+        comm.close()
+    fits = []
+    for p in sorted({r["p"] for r in rows}):
+        for algo in ("direct", "ring"):
+            for op in SWEEP_OPS:
+                pts = [r for r in rows if r["p"] == p and r["algo"] == algo and r["op"] == op]
+                if len(pts) < 3:
+                    continue
+                mb = np.array([r["bytes_per_rank"] for r in pts], float)
+                t = np.array([r["ms"] * 1e-3 for r in pts])
+                A = np.stack([np.ones_like(mb), mb], axis=1)
+                (alpha, inv_beta), *_ = np.linalg.lstsq(A, t, rcond=None)
+                fit = {"p": p, "algo": algo, "op": op, "alpha_us": alpha * 1e6,
+                       "beta_GBps": (1.0 / inv_beta) / 1e9 if inv_beta > 0 else None}
+                if algo == "ring" and op == "allreduce" and p > 1:
+                    # the ring model: T = 2(p-1) alpha_hop + 2(p-1)/p * m / beta
+                    A2 = np.stack([np.full_like(mb, 2 * (p - 1)), 2 * (p - 1) / p * mb], axis=1)
+                    (ah, ib), *_ = np.linalg.lstsq(A2, t, rcond=None)
+                    fit["ring_alpha_hop_us"] = ah * 1e6
+                    fit["ring_beta_GBps"] = (1.0 / ib) / 1e9 if ib > 0 else None
+                fits.append(fit)
+    for r in rows:
+        print(json.dumps({"sweep_point": r}))
+    for f in fits:
+        print(json.dumps({"sweep_fit": f}))
+    if args.sweep_out:
+        write_sweep_md(args.sweep_out, rows, fits)
+
+
+def write_sweep_md(path, rows, fits):
+    lines = ["# Size / rank sweep: latency, bandwidth and alpha-beta fits", "",
+             "int32 SUM data, per-rank message m = n*4 bytes (the AllReduce buffer, the ReduceScatter input,",
+             "the AllGather output, the All-to-All send buffer); median of 10 CUDA-event-timed calls after 3",
+             "warm-ups. algbw = m / t; busbw = algbw x the bus-bandwidth factor; hbm = minimum HBM bytes of the",
+             "call / t. Points whose p*m*2 fits in ~2x the 126 MB L2 are marked L2.", "",
+             "## Fits: t = alpha + m / beta (least squares over the sizes of each line)", "",
+             "| p | path | op | alpha (us) | beta (GB/s of m) | ring model: alpha per hop (us) | ring model: beta (GB/s) |",
+             "|---:|---|---|---:|---:|---:|---:|"]
+    for f in fits:
+        rb = f.get("ring_beta_GBps")
+        lines.append(f"| {f['p']} | {f['algo']} | {f['op']} | {f['alpha_us']:.2f} | "
+                     f"{f['beta_GBps']:.1f} | " + (f"{f['ring_alpha_hop_us']:.2f} | {rb:.1f} |" if rb else "| |"))
+    lines += ["", "## Points", "", "| p | path | op | m (bytes) | t (us) | algbw GB/s | busbw GB/s | HBM GB/s | L2 |",
+              "|---:|---|---|---:|---:|---:|---:|---:|---|"]
+    for r in rows:
+        lines.append(f"| {r['p']} | {r['algo']} | {r['op']} | {r['bytes_per_rank']} | {r['ms']*1e3:.1f} | "
+                     f"{r['algbw_GBps']:.1f} | {r['busbw_GBps']:.1f} | {r['hbm_GBps']:.1f} | "
+                     f"{'L2' if r['l2_resident'] else ''} |")
+    with open(path, "w") as fh:
+        fh.write("\n".join(lines) + "\n")
+
+
+# ---------------------------------------------------------------------------------------------
 
 def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.sweep:
+        sweep(args)
         return
     import torch
     import torch.distributed as dist
@@ -382,9 +531,7 @@ def main():
     clocks = clk.summary()
     torch.cuda.synchronize()
     if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = reduce_max(total_ms, device)
         dist.barrier()
 
     e2e = None
@@ -392,34 +539,42 @@ def main():
         e_ms, h2d, d2h = time_e2e(comm, wl, ops, max(3, args.steps // 4), 1, stream)
         e_steps = max(3, args.steps // 4)
         if world > 1:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * eff_per_step * e_steps / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+            e_ms = reduce_max(e_ms, device)
+        e2e = {"value": job_gbps(world, eff_per_step, e_ms / e_steps), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     hbm, peak_kind = peaks()
     ms_per_step = total_ms / args.steps
-    value = world * eff_per_step / (ms_per_step / 1e3) / 1e9
+    value = job_gbps(world, eff_per_step, ms_per_step)
     per_op_json = {}
     for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
         per_op_json[name] = {"ms": round(ms, 4), "effective_GBps": round(eff / (ms / 1e3) / 1e9, 1),
                              "kernel_GBps": round(kb / (ms / 1e3) / 1e9, 1),
                              "frac_of_measured_peak": round(kb / (ms / 1e3) / 1e9 / hbm, 4)}
-    # the dominant kernel: the kernel family with the largest share of the step's device time
-    fam = {}
-    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
-        f = fam.setdefault(kernel, [0.0, 0, 0])
-        f[0] += ms
-        f[1] += kb
-        f[2] += 1
-    dom = max(fam, key=lambda k: fam[k][0])
-    d_ms, d_bytes, d_launches = fam[dom]
-    achieved = d_bytes / (d_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
-                "traffic": None, "share_of_step": round(d_ms / sum(per_op), 4),
-                "bytes_per_launch": d_bytes // d_launches}
+    # The dominant kernel: each row is one launch of one kernel, so the row with the largest share
+    # of the step's device time names it. achieved = that kernel's algorithmic bytes per launch
+    # (its byte model: the minimum for direct rows, the ring schedule's hop traffic for ring rows)
+    # over its average launch time measured above with CUDA events.
+    i_dom = max(range(len(ops)), key=lambda i: per_op[i])
+    name, kernel, _, eff, kb = ops[i_dom]
+    d_ms = per_op[i_dom]
+    achieved = kb / (d_ms / 1e3) / 1e9
+    traffic = None
+    if name in NCU_TRAFFIC and args.n in (NCU_TRAFFIC[name][1], N_BUCKET):
+        t_bytes, t_n = NCU_TRAFFIC[name]
+        traffic = int(t_bytes * args.n / t_n)
+    roofline = {"bound": "hbm", "kernel": f"{name} ({kernel})", "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
+                "traffic": traffic, "algorithmic_bytes_per_launch": int(kb),
+                "share_of_step": round(d_ms / sum(per_op), 4), "ms_per_launch": round(d_ms, 4)}
+    # The four direct kernels the throughput target names (>= 80% of the ~8 TB/s nominal peak).
+    star = {}
+    for (nm, kernel, _, eff, kb), ms in zip(ops, per_op):
+        if nm in ("allreduce_avg_fp32_direct", "allreduce_avg_bf16_direct", "reduce_scatter_sum_fp32_direct",
+                  "allgather_fp32_direct", "alltoall_fp32_direct"):
+            g = kb / (ms / 1e3) / 1e9
+            star[nm] = {"GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
+                        "frac_of_nominal_8TBps": round(g / 8000.0, 4)}
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -431,6 +586,7 @@ def main():
                    "ops": [o[0] for o in ops], "options": args.option,
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline,
+        "north_star_direct": star,
         "per_op": per_op_json,
         "gpu_launches": int(launches),
         "clocks": clocks,
