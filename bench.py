@@ -35,6 +35,7 @@ FALLBACK_HBM_GBS = 6650.0
 # per-rank element count of that capture; scaled to the bench's size by elements moved. Empty
 # until a capture of the current build is taken.
 NCU_TRAFFIC = {}
+SPACER_CYCLES = 4_000_000  # ~2 ms of a spinning kernel ahead of a timed region
 
 
 def parse():
@@ -240,6 +241,8 @@ def time_device(ops, steps, warmup, stream):
           for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    # keep the GPU busy while the host enqueues, so host-side call overhead never shows as idle time
+    torch.cuda._sleep(SPACER_CYCLES)
     start.record(stream)
     for s in range(steps):
         for i, op in enumerate(ops):
@@ -391,10 +394,11 @@ def sweep(args):
     rows = []
     for p in [int(x) for x in args.sweep_ps.split(",")]:
         comm = SC.SimComm(p)
-        for algo in ("direct", "ring"):
+        algos = ("direct", "ring", "rd", "hd") if p & (p - 1) == 0 else ("direct", "ring")
+        for algo in algos:
             for nbytes in sizes:
                 n = max(p, (nbytes // 4) // p * p)     # int32 elements, divisible by p
-                hold = 2 * p * n * 4 + (p * n * 4 if algo == "ring" else 0)
+                hold = 2 * p * n * 4 + {"direct": 0, "ring": 1, "rd": 2, "hd": 1}[algo] * p * n * 4
                 if hold > SWEEP_CAP_BYTES:
                     continue
                 x = [torch.randint(-2**24, 2**24, (n,), dtype=torch.int32, device=dev) for _ in range(p)]
@@ -408,20 +412,22 @@ def sweep(args):
                     "allgather": lambda: comm.allgather([t[:m] for t in x], y, algo=algo),
                     "alltoall": lambda: comm.alltoall(x, y, algo=algo),
                 }
-                for op in SWEEP_OPS:
+                for op in (SWEEP_OPS if algo in ("direct", "ring") else ("allreduce",)):
                     f = calls[op]
                     for _ in range(3):
                         f()
                     torch.cuda.synchronize()
-                    ts = []
-                    for _ in range(10):
-                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                        e0.record(stream)
+                    # 10 back-to-back calls enqueued behind a spinning kernel: device time per call,
+                    # without host-side call overhead (which would otherwise leave the GPU idle)
+                    reps = 10
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    torch.cuda._sleep(SPACER_CYCLES)
+                    e0.record(stream)
+                    for _ in range(reps):
                         f()
-                        e1.record(stream)
-                        e1.synchronize()
-                        ts.append(e0.elapsed_time(e1))
-                    ms = float(np.median(ts))
+                    e1.record(stream)
+                    e1.synchronize()
+                    ms = e0.elapsed_time(e1) / reps
                     msg = n * 4  # per-rank message: the AllReduce in/out, ReduceScatter input, AllGather output
                     hbm = BM.direct_hbm_bytes(op, p, n, 4)
                     algbw = msg / (ms / 1e3) / 1e9
@@ -435,7 +441,7 @@ def sweep(args):
         comm.close()
     fits = []
     for p in sorted({r["p"] for r in rows}):
-        for algo in ("direct", "ring"):
+        for algo in ("direct", "ring", "rd", "hd"):
             for op in SWEEP_OPS:
                 pts = [r for r in rows if r["p"] == p and r["algo"] == algo and r["op"] == op]
                 if len(pts) < 3:
@@ -464,16 +470,18 @@ def sweep(args):
 def write_sweep_md(path, rows, fits):
     lines = ["# Size / rank sweep: latency, bandwidth and alpha-beta fits", "",
              "int32 SUM data, per-rank message m = n*4 bytes (the AllReduce buffer, the ReduceScatter input,",
-             "the AllGather output, the All-to-All send buffer); median of 10 CUDA-event-timed calls after 3",
-             "warm-ups. algbw = m / t; busbw = algbw x the bus-bandwidth factor; hbm = minimum HBM bytes of the",
+             "the AllGather output, the All-to-All send buffer); 10 back-to-back calls after 3 warm-ups, enqueued",
+             "behind a spinning kernel and timed with CUDA events (device time per call, launch gaps included). algbw = m / t; busbw = algbw x the bus-bandwidth factor; hbm = minimum HBM bytes of the",
              "call / t. Points whose p*m*2 fits in ~2x the 126 MB L2 are marked L2.", "",
              "## Fits: t = alpha + m / beta (least squares over the sizes of each line)", "",
              "| p | path | op | alpha (us) | beta (GB/s of m) | ring model: alpha per hop (us) | ring model: beta (GB/s) |",
              "|---:|---|---|---:|---:|---:|---:|"]
+    def num(x, fmt):
+        return format(x, fmt) if x is not None else "n/a"
     for f in fits:
-        rb = f.get("ring_beta_GBps")
-        lines.append(f"| {f['p']} | {f['algo']} | {f['op']} | {f['alpha_us']:.2f} | "
-                     f"{f['beta_GBps']:.1f} | " + (f"{f['ring_alpha_hop_us']:.2f} | {rb:.1f} |" if rb else "| |"))
+        lines.append(f"| {f['p']} | {f['algo']} | {f['op']} | {num(f['alpha_us'], '.2f')} | "
+                     f"{num(f['beta_GBps'], '.1f')} | {num(f.get('ring_alpha_hop_us'), '.2f')} | "
+                     f"{num(f.get('ring_beta_GBps'), '.1f')} |")
     lines += ["", "## Points", "", "| p | path | op | m (bytes) | t (us) | algbw GB/s | busbw GB/s | HBM GB/s | L2 |",
               "|---:|---|---|---:|---:|---:|---:|---:|---|"]
     for r in rows:

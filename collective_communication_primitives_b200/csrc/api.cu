@@ -39,6 +39,7 @@ struct sim_comm {
     long long copy_order = -1;
     long long direct_pack = 0;
     long long direct_ctas_per_sm = 16;
+    long long l2_hint = 0;
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
 };
@@ -67,9 +68,14 @@ coll_status_t check_reduce_args(coll_dtype_t dt, coll_op_t op) {
     return COLL_OK;
 }
 
-coll_status_t check_algo(coll_algo_t algo) {
-    if (algo != COLL_ALGO_DIRECT && algo != COLL_ALGO_RING) return fail(COLL_ERR_INVALID_ARG, "unknown algorithm");
-    return COLL_OK;
+// Direct and ring exist for every collective; the butterfly algorithms for AllReduce only.
+coll_status_t check_algo(coll_algo_t algo, bool allreduce = false) {
+    if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
+    if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD) {
+        if (allreduce) return COLL_OK;
+        return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling exist for AllReduce only");
+    }
+    return fail(COLL_ERR_INVALID_ARG, "unknown algorithm");
 }
 
 // The sticky state: an abort requested on the host, or an asynchronous error already reported.
@@ -213,6 +219,7 @@ coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, col
     a.vec = all_aligned(31) ? 2 : (all_aligned(15) ? 1 : 0);
     if (c->direct_pack == 16 && a.vec == 2) a.vec = 1;
     a.ctas_per_sm = int(c->direct_ctas_per_sm);
+    a.l2_hint = int(c->l2_hint);
     cudaError_t e = launch_direct_reduce(a, dt, op, c->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "direct reduction launch");
     c->launches += 1;
@@ -246,6 +253,7 @@ coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_e
     if (c->copy_variant >= 0) variant = int(c->copy_variant);
     if (c->copy_order >= 0) order = int(c->copy_order);
     a.order = order;
+    a.l2_hint = int(c->l2_hint);
     a.ctl = make_ctl(c);
     cudaError_t e = launch_copy(a, c->num_sms, variant, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
@@ -282,8 +290,10 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     {
         const bool reduce_kind = (pl.kind == RING_ALLREDUCE || pl.kind == RING_REDUCE_SCATTER || pl.kind == RING_REDUCE);
         const size_t wire = reduce_kind ? 4 : d;
-        a.tile = std::min(pl.chunk, std::max<size_t>(16, kRingTaskBytes / wire));
-        a.ntile = uint32_t((pl.chunk + a.tile - 1) / a.tile);
+        // a chunk is at most a segment long (the All-to-Allv's block sizes are known on the device only)
+        const size_t span = (pl.kind == RING_ALLTOALLV || pl.seg == 0) ? pl.chunk : std::min(pl.chunk, pl.seg);
+        a.tile = std::min(span, std::max<size_t>(16, kRingTaskBytes / wire));
+        a.ntile = uint32_t((span + a.tile - 1) / a.tile);
     }
     a.elem_bytes = int(d);
     a.nch = pl.nch;
@@ -334,6 +344,56 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     return COLL_OK;
 }
 
+// Recursive doubling / halving-doubling AllReduce on the butterfly executor.
+coll_status_t run_butterfly(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, int kind,
+                            cudaStream_t s) {
+    const int p = c->p;
+    if (p & (p - 1)) return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling need p a power of two");
+    int L = 0;
+    while ((1 << L) < p) ++L;
+    const size_t d = dtype_bytes(dt);
+    ButterflyArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.p = p;
+    a.kind = kind;
+    a.log2p = L;
+    a.n = n;
+    a.seg = (n + size_t(p) - 1) / size_t(p);
+    a.tile = 32768;  // 128 KiB of fp32/int32 partials per CTA task
+    a.nsteps = uint32_t(kind == BFLY_RD ? L : 2 * L);
+    a.start[0] = 0;
+    for (uint32_t g = 0; g < a.nsteps; ++g) {
+        size_t elems;  // the most elements one rank handles at step g
+        if (kind == BFLY_RD) elems = n;
+        else if (int(g) < L) elems = size_t(p >> (g + 1)) * a.seg;    // the kept half of a block group
+        else elems = (size_t(1) << (int(g) - L)) * a.seg;             // the partner's group of blocks
+        elems = std::min(elems, n);
+        a.ntile[g] = uint32_t(std::max<size_t>(1, (elems + a.tile - 1) / a.tile));
+        a.start[g + 1] = a.start[g] + uint32_t(p) * a.ntile[g];
+    }
+    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.timeout_ns = uint64_t(c->timeout_ns);
+    a.st = c->dstate;
+    a.ctl = make_ctl(c);
+    a.stage_stride = round_up(n * 4, 256);
+    const size_t nbuf = (kind == BFLY_RD) ? 2 * size_t(p) : size_t(p);
+    if (L > 1 || kind == BFLY_HD) {
+        coll_status_t st = ensure_stage(c, a.stage_stride * nbuf);
+        if (st != COLL_OK) return st;
+        a.stage = c->stage;
+    }
+    bool vec = (kind == BFLY_RD) || ((a.seg * d) % 16 == 0 && (a.seg * 4) % 16 == 0);
+    for (int r = 0; r < p; ++r) vec = vec && aligned16(a.ptrs.send[r]) && aligned16(a.ptrs.recv[r]);
+    a.vec = vec ? 1 : 0;
+    int ctas = c->ring_ctas > 0 ? int(c->ring_ctas) : c->ring_ctas_max;
+    if (a.start[a.nsteps] < uint32_t(ctas)) ctas = int(std::max<uint32_t>(a.start[a.nsteps], 1));
+    cudaError_t e = launch_butterfly(a, dt, op, ctas, s);
+    if (e != cudaSuccess) return cuda_fail(e, "butterfly executor launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
 uint32_t chunks_of(size_t seg, size_t chunk) { return uint32_t(std::max<size_t>(1, (seg + chunk - 1) / chunk)); }
 
 long long env_ll(const char* name, long long dflt) {
@@ -365,6 +425,9 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     } else if (k == "copy_order") {
         if (value < -1 || value > 1) return fail(COLL_ERR_INVALID_ARG, "copy_order must be -1, 0 or 1");
         c->copy_order = value;
+    } else if (k == "l2_hint") {
+        if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "l2_hint must be 0 or 1");
+        c->l2_hint = value;
     } else if (k == "direct_pack") {
         if (value != 0 && value != 16 && value != 32) return fail(COLL_ERR_INVALID_ARG, "direct_pack must be 0, 16 or 32");
         c->direct_pack = value;
@@ -465,6 +528,7 @@ coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* valu
     else if (k == "copy_variant") *value = c->copy_variant;
     else if (k == "copy_order") *value = c->copy_order;
     else if (k == "direct_pack") *value = c->direct_pack;
+    else if (k == "l2_hint") *value = c->l2_hint;
     else if (k == "direct_ctas_per_sm") *value = c->direct_ctas_per_sm;
     else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     return COLL_OK;
@@ -509,7 +573,9 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
                              coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
-    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
+    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo, true)) != COLL_OK) return st;
+    if ((algo == COLL_ALGO_RD || algo == COLL_ALGO_HD) && (c->p & (c->p - 1)))
+        return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling need p a power of two");
     if (n == 0) return COLL_OK;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const int p = c->p;
@@ -524,6 +590,8 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     if ((st = check_ranges(rs, INPLACE_SAME, 0)) != COLL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, b, n, dt, op, MODE_ALLREDUCE, 0, s);
+    if (algo == COLL_ALGO_RD) return run_butterfly(c, b, n, dt, op, BFLY_RD, s);
+    if (algo == COLL_ALGO_HD) return run_butterfly(c, b, n, dt, op, BFLY_HD, s);
     RingPlan pl;
     pl.kind = RING_ALLREDUCE;
     pl.seg = (n + size_t(p) - 1) / size_t(p);
@@ -700,6 +768,60 @@ coll_status_t coll_alltoall(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t 
     return run_ring(c, b, pl, n, dt, COLL_SUM, 0, s);
 }
 
+coll_status_t coll_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                           coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    if (algo != COLL_ALGO_DIRECT) return fail(COLL_ERR_UNSUPPORTED, "Scatter has the direct path only");
+    const int p = c->p;
+    if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
+    if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Scatter needs n divisible by p");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<Range> rs;
+    if ((st = check_ptr(b.send[root], n * d, d, "root send")) != COLL_OK) return st;
+    rs.push_back({uintptr_t(b.send[root]), uintptr_t(b.send[root]) + n * d, false, root});
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.recv[r], m * d, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + m * d, true, r});
+    }
+    if ((st = check_ranges(rs, INPLACE_RS, m * d)) != COLL_OK) return st;  // recv[root] = send[root] + root·m
+    std::vector<const void*> send(p, nullptr);
+    send[root] = b.send[root];
+    coll_bufs_t bb{send.data(), b.recv};
+    return run_copy(c, bb, COPY_SCATTER, m, dt, root, false, static_cast<cudaStream_t>(stream));
+}
+
+coll_status_t coll_gather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                          coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_algo(algo)) != COLL_OK) return st;
+    if (algo != COLL_ALGO_DIRECT) return fail(COLL_ERR_UNSUPPORTED, "Gather has the direct path only");
+    const int p = c->p;
+    if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
+    if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Gather needs n divisible by p");
+    if (n == 0) return COLL_OK;
+    if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(b.send[r], m * d, d, "send")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + m * d, false, r});
+    }
+    if ((st = check_ptr(b.recv[root], n * d, d, "root recv")) != COLL_OK) return st;
+    rs.push_back({uintptr_t(b.recv[root]), uintptr_t(b.recv[root]) + n * d, true, root});
+    if ((st = check_ranges(rs, INPLACE_AG, m * d)) != COLL_OK) return st;  // send[root] = recv[root] + root·m
+    std::vector<void*> recv(p, nullptr);
+    recv[root] = b.recv[root];
+    coll_bufs_t bb{b.send, recv.data()};
+    return run_copy(c, bb, COPY_GATHER, m, dt, root, true, static_cast<cudaStream_t>(stream));
+}
+
 coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* counts_dev, const long long* send_cap,
                              const long long* recv_cap, coll_dtype_t dt, coll_algo_t algo, coll_stream_t stream,
                              long long* recv_counts_dev) {
@@ -848,8 +970,9 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     a.timeout_ns = 2000000000ULL;
     a.st = reinterpret_cast<DevState*>(base);
     a.ctl.status = &a.st->status;
-    a.ctl.host_status = reinterpret_cast<uint32_t*>(base + 64);
-    a.ctl.abort_flag = reinterpret_cast<uint32_t*>(base + 68);
+    static_assert(sizeof(DevState) + 8 <= 256, "control words must fit the 256-byte control region");
+    a.ctl.host_status = reinterpret_cast<uint32_t*>(base + sizeof(DevState));
+    a.ctl.abort_flag = reinterpret_cast<uint32_t*>(base + sizeof(DevState) + 4);
     a.flags = reinterpret_cast<unsigned long long*>(base + ctl_bytes);
     a.stage = base + ctl_bytes + flag_bytes;
     a.stage_stride = stride;

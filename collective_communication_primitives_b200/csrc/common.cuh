@@ -208,6 +208,17 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -235,25 +246,69 @@ __device__ __forceinline__ bool status_failed(const Ctl& ctl) {
     return *reinterpret_cast<volatile uint32_t*>(ctl.status) != 0u;
 }
 
-// Bounded wait until *flag == want. Gives up when another CTA failed, when the host asked to
-// abort, after timeout_ns of global time or after kMaxSpin polls; then records the reason and
-// returns false. Called by one thread.
-constexpr uint32_t kMaxSpin = 1u << 26;
-__device__ __forceinline__ bool wait_flag(const Ctl& ctl, const unsigned long long* flag, unsigned long long want,
-                                          uint64_t timeout_ns) {
-    if (ld_acquire_gpu_u64(flag) == want) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1; it < kMaxSpin; ++it) {
-        if (ld_acquire_gpu_u64(flag) == want) return true;
-        if ((it & 15u) == 0u) {
-            if (status_failed(ctl)) return false;
-            if (*ctl.abort_flag != 0u) { raise_status(ctl, COLL_ERR_ABORTED); return false; }
-            if (globaltimer_ns() - t0 > timeout_ns) { raise_status(ctl, COLL_ERR_TIMEOUT); return false; }
+constexpr uint32_t kMaxSpin = 1u << 30;  // poll cap of every bounded wait (the timeout comes first)
+
+// How a waiting thread polls (a build-time choice). Measured on B200: any __nanosleep in a wait
+// loop (even 100 ns, or 1 us after a long wait) made a woken waiter notice its predecessor
+// hundreds of microseconds late, turning every dependent ring step into a ~250 us stall; tight
+// acquire polling (mode 0) was the fastest everywhere. Modes 2 and 3 remain for experiments.
+//   0: acquire loads back to back (default);   1: relaxed loads, one acquire fence on success;
+//   2: relaxed loads with a short sleep between polls;   3: acquire loads with a short sleep.
+#ifndef SIMCOMM_WAIT_MODE
+#define SIMCOMM_WAIT_MODE 0
+#endif
+#ifndef SIMCOMM_WAIT_SLEEP_NS
+#define SIMCOMM_WAIT_SLEEP_NS 100
+#endif
+
+template <typename T> __device__ __forceinline__ T poll_load(const T* p);
+template <> __device__ __forceinline__ unsigned long long poll_load(const unsigned long long* p) {
+    return (SIMCOMM_WAIT_MODE == 0 || SIMCOMM_WAIT_MODE == 3) ? ld_acquire_gpu_u64(p) : ld_relaxed_gpu_u64(p);
+}
+template <> __device__ __forceinline__ uint32_t poll_load(const uint32_t* p) {
+    return (SIMCOMM_WAIT_MODE == 0 || SIMCOMM_WAIT_MODE == 3) ? ld_acquire_gpu(p) : ld_relaxed_gpu(p);
+}
+
+// Bounded wait until done(*p), called by one thread. Every 256 polls (policy above) the thread
+// checks whether another CTA already failed and the global timer (timeout), and reads the
+// host-mapped abort word at most every 50 us (a round trip to host memory). Gives up (recording
+// the reason) on failure, abort, timeout_ns of global time, or kMaxSpin polls. On success the
+// caller's later loads see the producer's writes (acquire).
+template <typename T, typename Done>
+__device__ __forceinline__ bool bounded_wait(const Ctl& ctl, const T* p, Done done, uint64_t timeout_ns) {
+    uint64_t t0 = 0, last_abort_check = 0;
+    for (uint32_t it = 0; it < kMaxSpin; ++it) {
+        if (done(poll_load(p))) {
+            if (SIMCOMM_WAIT_MODE == 1 || SIMCOMM_WAIT_MODE == 2) fence_acq_rel_gpu();
+            return true;
         }
-        if (it > 64u) __nanosleep(64);
+        if (it == 0) {
+            t0 = last_abort_check = globaltimer_ns();
+            continue;
+        }
+        if (SIMCOMM_WAIT_MODE >= 2) __nanosleep(SIMCOMM_WAIT_SLEEP_NS);
+        if ((it & 255u) == 0u) {
+            if (status_failed(ctl)) return false;
+            const uint64_t now = globaltimer_ns();
+            if (now - t0 > timeout_ns) { raise_status(ctl, COLL_ERR_TIMEOUT); return false; }
+            if (now - last_abort_check > 50000u) {
+                last_abort_check = now;
+                if (*ctl.abort_flag != 0u) { raise_status(ctl, COLL_ERR_ABORTED); return false; }
+            }
+        }
     }
     raise_status(ctl, COLL_ERR_TIMEOUT);
     return false;
+}
+
+__device__ __forceinline__ bool wait_flag(const Ctl& ctl, const unsigned long long* flag, unsigned long long want,
+                                          uint64_t timeout_ns) {
+    return bounded_wait(ctl, flag, [want](unsigned long long v) { return v == want; }, timeout_ns);
+}
+
+// Bounded wait until a 32-bit counter reaches `want`.
+__device__ __forceinline__ bool wait_counter(const Ctl& ctl, const uint32_t* ctr, uint32_t want, uint64_t timeout_ns) {
+    return bounded_wait(ctl, ctr, [want](uint32_t v) { return v >= want; }, timeout_ns);
 }
 
 // Count one finished task of a chunk: the flag holds (epoch << 32) | tasks finished in this call;
@@ -314,6 +369,59 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 }
 // Wait until every committed bulk group has completed (writes performed).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// L2 policy that evicts the touched lines first (streaming data read or written once).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void bulk_g2s_hint(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
+                                              uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        :: "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void bulk_s2g_hint(void* gdst, const void* smem_src, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
+                 :: "l"(gdst), "r"(smem_u32(smem_src)), "r"(bytes), "l"(pol) : "memory");
+}
+// 16/32-byte streaming access with an L2 policy.
+template <int W> __device__ __forceinline__ Words<W> ld_stream_words_hint(const void* p, uint64_t pol);
+template <> __device__ __forceinline__ Words<4> ld_stream_words_hint<4>(const void* p, uint64_t pol) {
+    Words<4> v;
+    asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]) : "l"(p), "l"(pol));
+    return v;
+}
+template <> __device__ __forceinline__ Words<8> ld_stream_words_hint<8>(const void* p, uint64_t pol) {
+    Words<8> v;
+    asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+                   "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p), "l"(pol));
+    return v;
+}
+template <int W> __device__ __forceinline__ void st_words_hint(void* p, const Words<W>& v, uint64_t pol);
+template <> __device__ __forceinline__ void st_words_hint<4>(void* p, const Words<4>& v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;"
+                 :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "l"(pol) : "memory");
+}
+template <> __device__ __forceinline__ void st_words_hint<8>(void* p, const Words<8>& v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8}, %9;"
+                 :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+                    "r"(v.w[6]), "r"(v.w[7]), "l"(pol)
+                 : "memory");
+}
+// Streaming load/store of a pack, with (HINT) or without an evict-first L2 policy.
+template <int W, bool HINT> __device__ __forceinline__ Words<W> ld_pack(const void* p, uint64_t pol) {
+    if constexpr (HINT) return ld_stream_words_hint<W>(p, pol);
+    else return ld_stream_words<W>(p);
+}
+template <int W, bool HINT> __device__ __forceinline__ void st_pack(void* p, const Words<W>& v, uint64_t pol) {
+    if constexpr (HINT) st_words_hint<W>(p, v, pol);
+    else st_words<W>(p, v);
+}
 
 // Bounded mbarrier wait; false (and a recorded error) if the phase never completes.
 __device__ __forceinline__ bool mbar_wait_bounded(const Ctl& ctl, uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {

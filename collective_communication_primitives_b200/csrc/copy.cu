@@ -1,10 +1,12 @@
-// Copy engine: Broadcast, AllGather, All-to-All and All-to-Allv over TMA bulk copies.
+// Copy engine: Broadcast, AllGather, All-to-All, All-to-Allv, Scatter and Gather over TMA bulk copies.
 //
 // A collective is a list of segments (source range -> one or all ranks' destination ranges):
 //   Broadcast  1 segment:   send[root]               -> recv[r]            for every r
 //   AllGather  p segments:  send[q]                  -> recv[r] + q·m      for every r
 //   All-to-All p² segments: send[i] + j·m            -> recv[j] + i·m
 //   All-to-Allv p² segments: send[i] + sdispl[i][j]   -> recv[j] + rdispl[i][j], c[i][j] elements
+//   Scatter    p segments:  send[root] + r·m         -> recv[r]
+//   Gather     p segments:  send[r]                  -> recv[root] + r·m
 // Segments are cut into tiles of at most kTile bytes whose interior lies on 16-byte boundaries.
 // One warp per CTA runs a kStages-deep pipeline: one lane issues a cp.async.bulk load of a tile into
 // shared memory (completing on an mbarrier), then one cp.async.bulk store per destination. A
@@ -62,6 +64,16 @@ __device__ __forceinline__ SegDesc segment(const CopyArgs& a, int s, const long 
         d.dst = static_cast<char*>(a.ptrs.recv[j]) + size_t(i) * a.blk_elems * e;
         d.fanout = false;
         d.len = a.blk_elems * e;
+    } else if constexpr (KIND == COPY_SCATTER) {
+        d.src = static_cast<const char*>(a.ptrs.send[a.root]) + size_t(s) * a.blk_elems * e;
+        d.dst = static_cast<char*>(a.ptrs.recv[s]);
+        d.fanout = false;
+        d.len = (d.src == d.dst) ? 0 : a.blk_elems * e;  // in place: the root's block stays
+    } else if constexpr (KIND == COPY_GATHER) {
+        d.src = static_cast<const char*>(a.ptrs.send[s]);
+        d.dst = static_cast<char*>(a.ptrs.recv[a.root]) + size_t(s) * a.blk_elems * e;
+        d.fanout = false;
+        d.len = (d.src == d.dst) ? 0 : a.blk_elems * e;
     } else {
         const int i = s / a.p, j = s % a.p;
         d.src = static_cast<const char*>(a.ptrs.send[i]) + size_t(sd[s]) * e;
@@ -119,7 +131,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     if (status_failed(a.ctl)) return;
 
     const int p = a.p;
-    const int nseg = (KIND == COPY_BCAST) ? 1 : (KIND == COPY_ALLGATHER) ? p : p * p;
+    const int nseg = (KIND == COPY_BCAST) ? 1 : (KIND == COPY_ALLTOALL || KIND == COPY_ALLTOALLV) ? p * p : p;
     unsigned char* stages = smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kStages) * kTile);
     long long* sd = reinterpret_cast<long long*>(bars + kStages);
@@ -177,6 +189,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
 
     const uint32_t my_n = (total > blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     uint32_t phase = 0;  // bit s: parity of the next completion of stage s
+    const uint64_t pol = a.l2_hint ? l2_evict_first_policy() : 0;
     bool failed = false;
 
     auto issue = [&](uint32_t k) {
@@ -190,7 +203,10 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         if (lane == 0 && g.bhi > g.blo) {
             const int st = int(k % kStages);
             mbar_arrive_expect_tx(&bars[st], uint32_t(g.bhi - g.blo));
-            bulk_g2s(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st]);
+            if (a.l2_hint)
+                bulk_g2s_hint(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st], pol);
+            else
+                bulk_g2s(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st]);
         }
     };
 
@@ -216,8 +232,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
                 if (d.fanout) {
                     for (int r = 0; r < p; ++r) {
                         char* dst = fan_dst(a, d, r);
-                        if (dst != d.src) bulk_s2g(dst + g.blo, src, bytes);
+                        if (dst == d.src) continue;
+                        if (a.l2_hint) bulk_s2g_hint(dst + g.blo, src, bytes, pol);
+                        else bulk_s2g(dst + g.blo, src, bytes);
                     }
+                } else if (a.l2_hint) {
+                    bulk_s2g_hint(d.dst + g.blo, src, bytes, pol);
                 } else {
                     bulk_s2g(d.dst + g.blo, src, bytes);
                 }
@@ -254,7 +274,8 @@ constexpr int kLsuThreads = 256;
 constexpr int kLsuUnroll = 8;
 constexpr uint32_t kLsuTask = 128 * 1024;
 
-__device__ __forceinline__ void cta_copy_bytes(const char* s, char* d, size_t bytes) {
+template <bool HINT>
+__device__ __forceinline__ void cta_copy_bytes(const char* s, char* d, size_t bytes, uint64_t pol) {
     size_t head = bytes, body = 0;
     if (((reinterpret_cast<uintptr_t>(s) ^ reinterpret_cast<uintptr_t>(d)) & 15u) == 0) {
         head = (16 - (reinterpret_cast<uintptr_t>(s) & 15u)) & 15u;
@@ -263,27 +284,27 @@ __device__ __forceinline__ void cta_copy_bytes(const char* s, char* d, size_t by
     }
     for (size_t b = 2 * size_t(threadIdx.x); b < head; b += 2 * kLsuThreads)
         *reinterpret_cast<uint16_t*>(d + b) = *reinterpret_cast<const uint16_t*>(s + b);
-    const uint4* vs = reinterpret_cast<const uint4*>(s + head);
-    uint4* vd = reinterpret_cast<uint4*>(d + head);
+    const Words<4>* vs = reinterpret_cast<const Words<4>*>(s + head);
+    Words<4>* vd = reinterpret_cast<Words<4>*>(d + head);
     const size_t nv = body / 16;
     for (size_t v0 = threadIdx.x; v0 < nv; v0 += size_t(kLsuThreads) * kLsuUnroll) {
-        uint4 t[kLsuUnroll];
+        Words<4> t[kLsuUnroll];
 #pragma unroll
         for (int u = 0; u < kLsuUnroll; ++u) {
             const size_t v = v0 + size_t(u) * kLsuThreads;
-            if (v < nv) t[u] = ld_stream_v4(vs + v);
+            if (v < nv) t[u] = ld_pack<4, HINT>(vs + v, pol);
         }
 #pragma unroll
         for (int u = 0; u < kLsuUnroll; ++u) {
             const size_t v = v0 + size_t(u) * kLsuThreads;
-            if (v < nv) st_v4(vd + v, t[u]);
+            if (v < nv) st_pack<4, HINT>(vd + v, t[u], pol);
         }
     }
     for (size_t b = head + body + 2 * size_t(threadIdx.x); b < bytes; b += 2 * kLsuThreads)
         *reinterpret_cast<uint16_t*>(d + b) = *reinterpret_cast<const uint16_t*>(s + b);
 }
 
-template <int KIND>
+template <int KIND, bool HINT>
 __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_constant__ CopyArgs a) {
     static_assert(KIND == COPY_ALLTOALL || KIND == COPY_ALLTOALLV, "1:1 segments only");
     extern __shared__ __align__(128) unsigned char smem[];
@@ -332,6 +353,8 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     }
     __syncthreads();
     const uint32_t total = a.order ? s_tmax * uint32_t(nseg) : prefix[nseg];
+    uint64_t pol = 0;
+    if constexpr (HINT) pol = l2_evict_first_policy();
     for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
         int sg;
         uint32_t k;
@@ -346,7 +369,7 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
         const SegDesc d = segment<KIND>(a, sg, sd, rd);
         const size_t lo = size_t(k) * kLsuTask;
         const size_t hi = min(lo + kLsuTask, d.len);
-        cta_copy_bytes(d.src + lo, d.dst + lo, hi - lo);
+        cta_copy_bytes<HINT>(d.src + lo, d.dst + lo, hi - lo, pol);
     }
 }
 
@@ -355,21 +378,26 @@ static size_t lsu_smem_bytes(int kind, int p) {
     return b + (size_t(p) * p + 1) * sizeof(uint32_t);
 }
 
-template <int KIND>
-static cudaError_t launch_lsu(const CopyArgs& a, int num_sms, cudaStream_t s) {
+template <int KIND, bool HINT>
+static cudaError_t launch_lsu_hint(const CopyArgs& a, int num_sms, cudaStream_t s) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_copy_lsu<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_copy_lsu<KIND, HINT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(lsu_smem_bytes(KIND, kMaxRanks)));
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    k_copy_lsu<KIND><<<num_sms * 2, kLsuThreads, lsu_smem_bytes(KIND, a.p), s>>>(a);
+    k_copy_lsu<KIND, HINT><<<num_sms * 2, kLsuThreads, lsu_smem_bytes(KIND, a.p), s>>>(a);
     return cudaGetLastError();
 }
 
+template <int KIND>
+static cudaError_t launch_lsu(const CopyArgs& a, int num_sms, cudaStream_t s) {
+    return a.l2_hint ? launch_lsu_hint<KIND, true>(a, num_sms, s) : launch_lsu_hint<KIND, false>(a, num_sms, s);
+}
+
 static size_t copy_smem_bytes(int kind, int p, int stages, uint32_t tile) {
-    const int nseg = (kind == COPY_BCAST) ? 1 : (kind == COPY_ALLGATHER) ? p : p * p;
+    const int nseg = (kind == COPY_BCAST) ? 1 : (kind == COPY_ALLTOALL || kind == COPY_ALLTOALLV) ? p * p : p;
     size_t b = size_t(stages) * tile + size_t(stages) * sizeof(uint64_t);
     if (kind == COPY_ALLTOALLV) b += 2 * size_t(p) * p * sizeof(long long);
     b += (size_t(nseg) + 1) * sizeof(uint32_t);
@@ -427,7 +455,9 @@ constexpr int kVariantLsu = kNumCopyShapes;
 
 void copy_defaults(int kind, int* variant, int* order) {
     switch (kind) {
-        case COPY_ALLTOALL: *variant = 0; *order = 1; break;
+        case COPY_ALLTOALL:
+        case COPY_SCATTER:
+        case COPY_GATHER: *variant = 0; *order = 1; break;
         case COPY_ALLTOALLV: *variant = kVariantLsu; *order = 0; break;
         default: *variant = 5; *order = 0; break;
     }
@@ -437,13 +467,15 @@ cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_
     if (variant == kVariantLsu) {
         if (a.kind == COPY_ALLTOALL) return launch_lsu<COPY_ALLTOALL>(a, num_sms, s);
         if (a.kind == COPY_ALLTOALLV) return launch_lsu<COPY_ALLTOALLV>(a, num_sms, s);
-        variant = 5;  // fan-out collectives have no load/store variant
+        variant = 5;  // the other collectives have no load/store variant
     }
     switch (a.kind) {
         case COPY_BCAST: return launch_kind<COPY_BCAST>(a, num_sms, variant, s);
         case COPY_ALLGATHER: return launch_kind<COPY_ALLGATHER>(a, num_sms, variant, s);
         case COPY_ALLTOALL: return launch_kind<COPY_ALLTOALL>(a, num_sms, variant, s);
         case COPY_ALLTOALLV: return launch_kind<COPY_ALLTOALLV>(a, num_sms, variant, s);
+        case COPY_SCATTER: return launch_kind<COPY_SCATTER>(a, num_sms, variant, s);
+        case COPY_GATHER: return launch_kind<COPY_GATHER>(a, num_sms, variant, s);
         default: return cudaErrorInvalidValue;
     }
 }

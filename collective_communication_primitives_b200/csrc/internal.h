@@ -14,9 +14,10 @@ constexpr int kMaxRanks = SIM_COMM_MAX_RANKS;
 // Device scratch header of a communicator (device memory, zero-initialised).
 struct DevState {
     uint32_t status;    // first asynchronous error (coll_status_t), 0 = OK
-    uint32_t task_ctr;  // ring executor: next task to claim
-    uint32_t done_ctr;  // ring executor: CTAs that left the task loop
+    uint32_t task_ctr;  // ring / butterfly executor: next task to claim
+    uint32_t done_ctr;  // ring / butterfly executor: CTAs that left the task loop
     uint32_t pad;
+    uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
 };
 
 // What a kernel needs to report errors and notice an abort.
@@ -44,11 +45,13 @@ struct DirectReduceArgs {
     size_t seg;        // ReduceScatter: elements per owner (n / p); otherwise n
     float scale;       // AVG: 1/p; otherwise 1
     int ctas_per_sm;   // grid = SMs x this (capped by the work)
+    int l2_hint;       // 1: evict-first L2 policy on the streaming loads and stores
     Ctl ctl;
 };
 
 // ---- copy engine (Broadcast / AllGather / All-to-All / All-to-Allv) ------------------------------
-enum CopyKind { COPY_BCAST = 0, COPY_ALLGATHER = 1, COPY_ALLTOALL = 2, COPY_ALLTOALLV = 3 };
+enum CopyKind { COPY_BCAST = 0, COPY_ALLGATHER = 1, COPY_ALLTOALL = 2, COPY_ALLTOALLV = 3, COPY_SCATTER = 4,
+                COPY_GATHER = 5 };
 
 struct CopyArgs {
     RankPtrs ptrs;
@@ -56,8 +59,9 @@ struct CopyArgs {
     int kind;
     int root;
     int elem_bytes;
-    size_t blk_elems;                  // BCAST: n; ALLGATHER: shard n/p; ALLTOALL: block n/p
+    size_t blk_elems;                  // BCAST: n; ALLGATHER, ALLTOALL, SCATTER, GATHER: block n/p
     int order;                         // tile order: 0 segment-major, 1 interleaved over segments
+    int l2_hint;                       // 1: evict-first L2 policy on the bulk/streaming copies
     const long long* counts;           // ALLTOALLV: device [p][p]
     long long* recv_counts_out;        // ALLTOALLV: device [p] or null
     long long send_cap[kMaxRanks];     // ALLTOALLV: elements per send buffer
@@ -102,7 +106,32 @@ struct RingArgs {
     Ctl ctl;
 };
 
+// ---- butterfly executor: recursive doubling and halving-doubling AllReduce ---------------------
+enum ButterflyKind { BFLY_RD = 0, BFLY_HD = 1 };
+constexpr int kMaxBflySteps = 16;
+
+struct ButterflyArgs {
+    RankPtrs ptrs;
+    int p;
+    int kind;
+    int log2p;
+    int vec;                 // 1: 16-byte hops (every range start 16-byte aligned)
+    size_t n;
+    size_t seg;              // block size (ceil(n/p)), HD only
+    size_t tile;             // elements per CTA task
+    uint32_t nsteps;
+    uint32_t ntile[kMaxBflySteps];   // tasks per rank at each step
+    uint32_t start[kMaxBflySteps + 1];  // first task of each step
+    float scale;
+    uint64_t timeout_ns;
+    char* stage;             // RD: two partial buffers per rank; HD: one
+    size_t stage_stride;
+    DevState* st;
+    Ctl ctl;
+};
+
 // Launchers (each returns the launch error; grid sizes are decided inside).
+cudaError_t launch_butterfly(const ButterflyArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, int num_sms, cudaStream_t s);
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s);
 int copy_num_variants();

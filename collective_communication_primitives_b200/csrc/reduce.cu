@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_scalar(const __grid_cons
 // P > 0: p is a compile-time constant and all p loads of a position are in flight together.
 // P == 0: p is read at run time and ranks are loaded kDirGroup at a time.
 // W: 32-bit words per pack (4: 16-byte accesses, 8: 32-byte accesses).
-template <int DT, int OP, int P, bool SCALE, int W>
+template <int DT, int OP, int P, bool SCALE, int W, bool HINT>
 __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constant__ DirectReduceArgs a) {
     using PK = PackW<DT, W>;
     using A = typename PK::A;
@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
     const int p = (P > 0) ? P : a.p;
     const int nseg = (a.mode == MODE_REDUCE_SCATTER) ? p : 1;
     const size_t seg_packs = a.seg / L;
+    uint64_t pol = 0;
+    if constexpr (HINT) pol = l2_evict_first_policy();
     const size_t step = size_t(gridDim.x) * kDirThreads * kDirUnroll;
 
     for (int sg = 0; sg < nseg; ++sg) {
@@ -90,8 +92,8 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
 #pragma unroll
                     for (int j = 0; j < G; ++j)
                         if (ok[u] && (P > 0 || q0 + j < p))
-                            v[u][j] = ld_stream_words<W>(static_cast<const Words<W>*>(a.ptrs.send[q0 + j]) +
-                                                         in_base + i0 + size_t(u) * kDirThreads);
+                            v[u][j] = ld_pack<W, HINT>(static_cast<const Words<W>*>(a.ptrs.send[q0 + j]) +
+                                                           in_base + i0 + size_t(u) * kDirThreads, pol);
 #pragma unroll
                 for (int u = 0; u < kDirUnroll; ++u) {
 #pragma unroll
@@ -121,15 +123,15 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
                     if constexpr (P > 0) {
 #pragma unroll
                         for (int r = 0; r < P; ++r)
-                            st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out);
+                            st_pack<W, HINT>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out, pol);
                     } else {
                         for (int r = 0; r < p; ++r)
-                            st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out);
+                            st_pack<W, HINT>(static_cast<Words<W>*>(a.ptrs.recv[r]) + in_base + idx, out, pol);
                     }
                 } else if (a.mode == MODE_REDUCE) {
-                    st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[a.root]) + in_base + idx, out);
+                    st_pack<W, HINT>(static_cast<Words<W>*>(a.ptrs.recv[a.root]) + in_base + idx, out, pol);
                 } else {
-                    st_words<W>(static_cast<Words<W>*>(a.ptrs.recv[sg]) + idx, out);
+                    st_pack<W, HINT>(static_cast<Words<W>*>(a.ptrs.recv[sg]) + idx, out, pol);
                 }
             }
         }
@@ -159,11 +161,20 @@ static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStre
         const size_t packs = a.seg / L;
         const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
         const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
+        if (a.l2_hint) {
+            switch (a.p) {
+                case 2: k_direct_vec<DT, OP, 2, SCALE, 8, true><<<grid, kDirThreads, 0, s>>>(a); break;
+                case 4: k_direct_vec<DT, OP, 4, SCALE, 8, true><<<grid, kDirThreads, 0, s>>>(a); break;
+                case 8: k_direct_vec<DT, OP, 8, SCALE, 8, true><<<grid, kDirThreads, 0, s>>>(a); break;
+                default: k_direct_vec<DT, OP, 0, SCALE, 8, true><<<grid, kDirThreads, 0, s>>>(a); break;
+            }
+            return cudaGetLastError();
+        }
         switch (a.p) {
-            case 2: k_direct_vec<DT, OP, 2, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
-            case 4: k_direct_vec<DT, OP, 4, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
-            case 8: k_direct_vec<DT, OP, 8, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
-            default: k_direct_vec<DT, OP, 0, SCALE, 8><<<grid, kDirThreads, 0, s>>>(a); break;
+            case 2: k_direct_vec<DT, OP, 2, SCALE, 8, false><<<grid, kDirThreads, 0, s>>>(a); break;
+            case 4: k_direct_vec<DT, OP, 4, SCALE, 8, false><<<grid, kDirThreads, 0, s>>>(a); break;
+            case 8: k_direct_vec<DT, OP, 8, SCALE, 8, false><<<grid, kDirThreads, 0, s>>>(a); break;
+            default: k_direct_vec<DT, OP, 0, SCALE, 8, false><<<grid, kDirThreads, 0, s>>>(a); break;
         }
         return cudaGetLastError();
     }
@@ -172,11 +183,11 @@ static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStre
     const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
     const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
     switch (a.p) {
-        case 2: k_direct_vec<DT, OP, 2, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 3: k_direct_vec<DT, OP, 3, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 4: k_direct_vec<DT, OP, 4, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
-        case 8: k_direct_vec<DT, OP, 8, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
-        default: k_direct_vec<DT, OP, 0, SCALE, 4><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 2: k_direct_vec<DT, OP, 2, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 3: k_direct_vec<DT, OP, 3, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 4: k_direct_vec<DT, OP, 4, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
+        case 8: k_direct_vec<DT, OP, 8, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
+        default: k_direct_vec<DT, OP, 0, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
     }
     return cudaGetLastError();
 }

@@ -16,7 +16,7 @@ STATUS = {0: "COLL_OK", 1: "COLL_ERR_INVALID_ARG", 2: "COLL_ERR_UNSUPPORTED", 3:
 OK, INVALID_ARG, UNSUPPORTED, CUDA, TIMEOUT, ABORTED, OVERFLOW, INTERNAL = range(8)
 DTYPES = {"int32": 0, "fp32": 1, "bf16": 2}
 OPS = {"sum": 0, "min": 1, "max": 2, "avg": 3}
-ALGOS = {"direct": 0, "ring": 1}
+ALGOS = {"direct": 0, "ring": 1, "rd": 2, "hd": 3}
 
 _lib = None
 
@@ -72,9 +72,11 @@ def load_library(path=LIB_PATH):
     L.coll_allgather.argtypes = [vp, _Bufs, sz, i32, i32, vp]
     L.coll_alltoall.argtypes = [vp, _Bufs, sz, i32, i32, vp]
     L.coll_alltoallv.argtypes = [vp, _Bufs, vp, llp, llp, i32, i32, vp, vp]
+    L.coll_scatter.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
+    L.coll_gather.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_allreduce_ring_noalloc.argtypes = [i32, _Bufs, sz, i32, i32, vp, vp]
     for name in ("coll_allreduce", "coll_reduce", "coll_broadcast", "coll_reduce_scatter", "coll_allgather",
-                 "coll_alltoall", "coll_alltoallv", "coll_allreduce_ring_noalloc"):
+                 "coll_alltoall", "coll_alltoallv", "coll_scatter", "coll_gather", "coll_allreduce_ring_noalloc"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -210,6 +212,20 @@ class SimComm:
         n = sends[0].numel() if n is None else n
         self._check(self._L.coll_alltoall(self._h, self._bufs(sends, recvs), n, self._resolve(dtype, list(sends) + list(recvs)),
                                           ALGOS[algo], _stream(stream)))
+
+    def scatter(self, sends, recvs, root, algo="direct", n=None, dtype=None, stream=None):
+        """n: the root's full buffer (p blocks); only sends[root] is read."""
+        n = sends[root].numel() if n is None else n
+        self._check(self._L.coll_scatter(self._h, self._bufs(sends, recvs), n,
+                                         self._resolve(dtype, list(sends) + list(recvs)), int(root), ALGOS[algo],
+                                         _stream(stream)))
+
+    def gather(self, sends, recvs, root, algo="direct", n=None, dtype=None, stream=None):
+        """n: the root's full buffer (p blocks); only recvs[root] is written."""
+        n = recvs[root].numel() if n is None else n
+        self._check(self._L.coll_gather(self._h, self._bufs(sends, recvs), n,
+                                        self._resolve(dtype, list(sends) + list(recvs)), int(root), ALGOS[algo],
+                                        _stream(stream)))
 
     def alltoallv(self, sends, recvs, counts, send_cap=None, recv_cap=None, algo="direct", recv_counts=None,
                   dtype=None, stream=None):

@@ -9,6 +9,7 @@
  *   [Atlas]  "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives)
  *   [Primer] "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
  *            (charlestar.github.io/2026/08/20/gpu-collective-communication)
+ *   [Eight]  "详解分布式训练8大集合通信原语：从Send/Recv到All2All" (bjdmk.com.cn/news/4699717)
  *
  * Common conventions
  *   - n is the per-rank FULL buffer element count ([Primer] "先统一通信量的记号": B is the full
@@ -75,8 +76,12 @@ typedef enum { COLL_INT32 = 0, COLL_FP32 = 1, COLL_BF16 = 2 } coll_dtype_t;
 typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_t;
 
 /* DIRECT: one fused pass reads all p inputs and writes every owner's output.
- * RING:   the ring schedule of [Atlas] §2.2, chunk-pipelined as in [Atlas] §3.5. */
-typedef enum { COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1 } coll_algo_t;
+ * RING:   the ring schedule of [Atlas] §2.2, chunk-pipelined as in [Atlas] §3.5.
+ * RD:     recursive doubling ([Atlas] §2.3): log2 p exchange-and-reduce steps. AllReduce only,
+ *         p a power of two (else COLL_ERR_UNSUPPORTED).
+ * HD:     recursive halving-doubling ([Atlas] §2.3): a halving reduce-scatter then a doubling
+ *         all-gather, 2 log2 p steps. AllReduce only, p a power of two. */
+typedef enum { COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3 } coll_algo_t;
 
 typedef struct {
     const void* const* send; /* host array [p] of device pointers (inputs) */
@@ -120,6 +125,8 @@ const char* coll_status_string(coll_status_t status);
  *   "direct_pack"  access width of the fused reduction: 0 = widest the alignment allows
  *                  (32 bytes), 16 = at most 16 bytes
  *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16)
+ *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
+ *                  paths (data read or written once), 0 = none (default)
  * Returns COLL_ERR_INVALID_ARG for an unknown key or a value out of range. */
 coll_status_t sim_comm_set_option(sim_comm_t comm, const char* key, long long value);
 coll_status_t sim_comm_get_option(sim_comm_t comm, const char* key, long long* value);
@@ -171,6 +178,19 @@ coll_status_t coll_allgather(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_d
  * (the [src][dst] block matrix transposed). Both buffers hold n elements. n divisible by p. */
 coll_status_t coll_alltoall(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype,
                             coll_algo_t algo, coll_stream_t stream);
+
+/* Scatter ([Eight] "3.3 Scatter"; [Atlas] §0: the single-root form): with m = n/p,
+ * recv[r][k] = send[root][r·m + k]. Only send[root] (n elements) is read; recv buffers hold m.
+ * In place: recv[root] == send[root] + root·m. Direct path only (COLL_ALGO_RING:
+ * COLL_ERR_UNSUPPORTED). */
+coll_status_t coll_scatter(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype, int root,
+                           coll_algo_t algo, coll_stream_t stream);
+
+/* Gather ([Eight] "4.3 Gather"; [Atlas] §0): with m = n/p, recv[root][r·m + k] = send[r][k]. Only
+ * recv[root] (n elements) is written; send buffers hold m. In place: send[root] == recv[root] +
+ * root·m. Direct path only. */
+coll_status_t coll_gather(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtype_t dtype, int root,
+                          coll_algo_t algo, coll_stream_t stream);
 
 /* All-to-Allv, uneven split ([Primer] "Ragged All-to-All：MoE 的真实输入通常不等长"):
  *   counts_dev   DEVICE int64 [p][p] row-major, c[i][j] = elements source i sends to destination j

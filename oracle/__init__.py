@@ -45,6 +45,10 @@ def lib():
             "oracle_ring_reduce": [i32, pp, vp, sz, i32, i32, i32],
             "oracle_ring_broadcast": [i32, vp, pp, sz, i32, i32],
             "oracle_ring_alltoall": [i32, pp, pp, sz, i32],
+            "oracle_scatter": [i32, vp, pp, sz, i32, i32],
+            "oracle_gather": [i32, pp, vp, sz, i32, i32],
+            "oracle_rd_allreduce": [i32, pp, pp, sz, i32, i32],
+            "oracle_hd_allreduce": [i32, pp, pp, sz, i32, i32],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -148,6 +152,24 @@ def alltoallv(inputs, counts, dtype):
     return outs, rc
 
 
+def scatter(root_input, p, dtype, root):
+    """Scatter: block r of the root's [p·m] buffer goes to rank r."""
+    x = _arr(root_input, dtype)
+    outs = _outs(p, x.size // p, dtype)
+    _check(lib().oracle_scatter(p, x.ctypes.data, _ptrs(outs), x.size, DTYPE_CODES[dtype], root), "scatter")
+    return outs
+
+
+def gather(inputs, dtype, root):
+    """Gather: rank r's [m] block lands at block r of the root's [p·m] buffer."""
+    ins = [_arr(x, dtype) for x in inputs]
+    p = len(ins)
+    n = p * ins[0].size
+    res = np.zeros(n, dtype=NP_DTYPES[dtype])
+    _check(lib().oracle_gather(p, _ptrs(ins), res.ctypes.data, n, DTYPE_CODES[dtype], root), "gather")
+    return res
+
+
 def ring_allreduce(inputs, dtype, op):
     ins = [_arr(x, dtype) for x in inputs]
     n = ins[0].size
@@ -197,6 +219,26 @@ def ring_alltoall(inputs, dtype):
     p, n = len(ins), ins[0].size
     outs = _outs(p, n, dtype)
     _check(lib().oracle_ring_alltoall(p, _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype]), "ring_alltoall")
+    return outs
+
+
+def rd_allreduce(inputs, dtype, op):
+    """Recursive-doubling AllReduce (p a power of two)."""
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    outs = _outs(len(ins), n, dtype)
+    _check(lib().oracle_rd_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
+           "rd_allreduce")
+    return outs
+
+
+def hd_allreduce(inputs, dtype, op):
+    """Recursive halving-doubling AllReduce (p a power of two)."""
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    outs = _outs(len(ins), n, dtype)
+    _check(lib().oracle_hd_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
+           "hd_allreduce")
     return outs
 
 

@@ -10,6 +10,7 @@
  *   [Atlas]  "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives)
  *   [Primer] "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
  *            (charlestar.github.io/2026/08/20/gpu-collective-communication)
+ *   [Eight]  "详解分布式训练8大集合通信原语：从Send/Recv到All2All" (bjdmk.com.cn/news/4699717)
  *
  * Conventions (our own; the pages write the data layouts only as figures):
  *   - p ranks; rank r's buffer is in[r] / out[r], a host pointer.
@@ -28,6 +29,7 @@
  * its result) is "parity unpinned": the page's p = 4 trace is garbled, so the schedule follows the
  * reading that makes rank r own block r.
  */
+#include <algorithm>
 #include <cfenv>
 #include <cmath>
 #include <cstdint>
@@ -343,6 +345,27 @@ int oracle_alltoallv(int p, const void* const* in, void* const* out, const int64
     return 0;
 }
 
+/* [Eight] "3.3 Scatter": the root's data is cut into p blocks in rank order and block r goes to
+ * rank r ([Atlas] §0 lists Gather/Scatter as the single-root forms): out_r[k] = in_root[r·m + k],
+ * m = n/p. Only the root's input is read. */
+int oracle_scatter(int p, const void* in_root, void* const* out, size_t n, int dtype, int root) {
+    if (!valid_common(p, dtype) || root < 0 || root >= p || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p);
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < m; ++k) copy_element(in_root, size_t(r) * m + k, out[r], k, dtype);
+    return 0;
+}
+
+/* [Eight] "4.3 Gather": every rank's block is collected at the root only, in rank order:
+ * out_root[r·m + k] = in_r[k], m = n/p. Only the root's output is written. */
+int oracle_gather(int p, const void* const* in, void* out_root, size_t n, int dtype, int root) {
+    if (!valid_common(p, dtype) || root < 0 || root >= p || n % size_t(p) != 0) return -1;
+    size_t m = n / size_t(p);
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < m; ++k) copy_element(in[r], k, out_root, size_t(r) * m + k, dtype);
+    return 0;
+}
+
 /* ===================== ring schedule emulation ================================================== */
 /* [Atlas] §2.2: ranks form the ring r0 -> r1 -> ... -> r_{p-1} -> r0, every buffer is cut into p
  * chunks, a ring reduce-scatter of p-1 steps is followed by a ring all-gather of p-1 steps.
@@ -499,6 +522,105 @@ int oracle_ring_alltoall(int p, const void* const* in, void* const* out, size_t 
                 std::memcpy(static_cast<char*>(out[j]) + size_t(r) * m * d,
                             static_cast<const char*>(in[r]) + size_t(j) * m * d, m * d);
         }
+    return 0;
+}
+
+/* ===================== recursive doubling / halving-doubling ====================================== */
+/* [Atlas] §2.3 (p a power of two). Reading (the page gives the exchange pattern, not the operand
+ * order): when partners r and r^d combine, the lower rank's data comes first, so both compute the
+ * same value; partials travel in fp32 for fp32 and bf16 data and are rounded once at the end. */
+
+static bool power_of_two(int p) { return p >= 1 && (p & (p - 1)) == 0; }
+
+/* Recursive doubling: at step k (distance d = 2^k) every rank replaces its vector by
+ * vec[min(r, r^d)] ⊕ vec[max(r, r^d)]; after log2(p) steps every rank holds the reduction. */
+int oracle_rd_allreduce(int p, const void* const* in, void* const* out, size_t n, int dtype, int op) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD) || !power_of_two(p)) return -1;
+    std::vector<RingAcc> cur(p, RingAcc{dtype, op, {}, {}});
+    for (int r = 0; r < p; ++r) {
+        cur[r].resize(n);
+        for (size_t k = 0; k < n; ++k) cur[r].load(in[r], k);
+    }
+    for (int d = 1; d < p; d <<= 1) {
+        std::vector<RingAcc> next = cur;  // every rank reads the values of the previous step
+        for (int r = 0; r < p; ++r) {
+            const int lo = std::min(r, r ^ d), hi = std::max(r, r ^ d);
+            for (size_t k = 0; k < n; ++k) {
+                if (dtype == DT_INT32) {
+                    int32_t a = cur[lo].i[k], b = cur[hi].i[k];
+                    next[r].i[k] = (op == OP_SUM) ? int32_t(uint32_t(a) + uint32_t(b)) : apply_minmax(op, a, b);
+                } else {
+                    volatile float a = cur[lo].f[k], b = cur[hi].f[k];
+                    if (op == OP_MIN || op == OP_MAX) next[r].f[k] = apply_minmax(op, float(a), float(b));
+                    else { volatile float sum = a + b; next[r].f[k] = sum; }
+                }
+            }
+        }
+        cur.swap(next);
+    }
+    for (int r = 0; r < p; ++r)
+        for (size_t k = 0; k < n; ++k) cur[r].store_final(p, out[r], k, k);
+    return 0;
+}
+
+/* Recursive halving-doubling (reduce-scatter by halving, then all-gather by doubling). The buffer
+ * is cut into p blocks as in the ring (ring_segment). Halving step with distance d = p/2, p/4, ..., 1:
+ * rank r's blocks are the aligned group of 2d blocks containing block r; it keeps the half that
+ * contains block r and computes kept = mine ⊕ partner's (lower rank first) while the partner keeps
+ * the other half. After the last step rank r holds the complete block r. Doubling steps with
+ * d = 1, 2, ..., p/2: partners exchange the groups of d blocks they hold. */
+int oracle_hd_allreduce(int p, const void* const* in, void* const* out, size_t n, int dtype, int op) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD) || !power_of_two(p)) return -1;
+    std::vector<RingAcc> cur(p, RingAcc{dtype, op, {}, {}});
+    for (int r = 0; r < p; ++r) {
+        cur[r].resize(n);
+        for (size_t k = 0; k < n; ++k) cur[r].load(in[r], k);
+    }
+    for (int d = p / 2; d >= 1; d >>= 1) {
+        std::vector<RingAcc> next = cur;
+        for (int r = 0; r < p; ++r) {
+            const int partner = r ^ d, lo = std::min(r, partner), hi = std::max(r, partner);
+            const int group = (r / (2 * d)) * (2 * d);
+            const int kb = (r & d) ? group + d : group;  // first block of the kept half
+            size_t b0, e0, b1, e1;
+            ring_segment(n, p, kb, &b0, &e0);
+            ring_segment(n, p, kb + d - 1, &b1, &e1);
+            for (size_t k = b0; k < e1; ++k) {
+                if (dtype == DT_INT32) {
+                    int32_t a = cur[lo].i[k], b = cur[hi].i[k];
+                    next[r].i[k] = (op == OP_SUM) ? int32_t(uint32_t(a) + uint32_t(b)) : apply_minmax(op, a, b);
+                } else {
+                    volatile float a = cur[lo].f[k], b = cur[hi].f[k];
+                    if (op == OP_MIN || op == OP_MAX) next[r].f[k] = apply_minmax(op, float(a), float(b));
+                    else { volatile float sum = a + b; next[r].f[k] = sum; }
+                }
+            }
+        }
+        cur.swap(next);
+    }
+    /* rank r rounds its complete block r; then the doubling exchanges spread the blocks */
+    for (int r = 0; r < p; ++r) {
+        size_t b, e;
+        ring_segment(n, p, r, &b, &e);
+        for (size_t k = b; k < e; ++k) cur[r].store_final(p, out[r], k, k);
+    }
+    size_t dsz = elem_size(dtype);
+    for (int d = 1; d < p; d <<= 1) {
+        std::vector<std::vector<char>> snapshot(p);
+        for (int r = 0; r < p; ++r) {
+            const char* o = static_cast<const char*>(out[r]);
+            snapshot[r].assign(o, o + n * dsz);
+        }
+        for (int r = 0; r < p; ++r) {
+            const int partner = r ^ d;
+            const int pg = (partner / d) * d;  // the partner's group of d blocks
+            size_t b0, e0, b1, e1;
+            ring_segment(n, p, pg, &b0, &e0);
+            ring_segment(n, p, pg + d - 1, &b1, &e1);
+            if (e1 > b0)
+                std::memcpy(static_cast<char*>(out[r]) + b0 * dsz, snapshot[partner].data() + b0 * dsz, (e1 - b0) * dsz);
+        }
+    }
     return 0;
 }
 

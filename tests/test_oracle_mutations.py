@@ -25,6 +25,11 @@ MUTANTS = {
     "ring_broadcast_wrong_hop": ("int src = mod(root + h - 1, p), dst = mod(root + h, p);", "int src = mod(root + h - 1, p), dst = mod(root + h + 1, p);"),
     "double_bf16_wrong_quantum": ("int q = e - 8;", "int q = e - 9;"),
     "ring_avg_scale_missing": ("if (op == OP_AVG) { volatile float scale = 1.0f / float(p); v = v * scale; }\n        store_float(out, dtype, oi, v);\n    }\n};", "store_float(out, dtype, oi, v);\n    }\n};"),
+    "rd_wrong_partner": ("const int lo = std::min(r, r ^ d), hi = std::max(r, r ^ d);", "const int lo = std::min(r, (r + d) % p), hi = std::max(r, (r + d) % p);"),
+    "hd_ascending_halving": ("for (int d = p / 2; d >= 1; d >>= 1) {", "for (int d = 1; d < p; d <<= 1) {"),
+    "hd_keeps_wrong_half": ("const int kb = (r & d) ? group + d : group;", "const int kb = (r & d) ? group : group + d;"),
+    "scatter_wrong_block": ("copy_element(in_root, size_t(r) * m + k, out[r], k, dtype);", "copy_element(in_root, size_t((r + 1) % p) * m + k, out[r], k, dtype);"),
+    "gather_wrong_block": ("copy_element(in[r], k, out_root, size_t(r) * m + k, dtype);", "copy_element(in[r], k, out_root, size_t(p - 1 - r) * m + k, dtype);"),
     "int_sum_saturates": ("if (op == OP_SUM) i[k] = int32_t(uint32_t(received_i) + uint32_t(o));", "if (op == OP_SUM) i[k] = int32_t(std::max<int64_t>(INT32_MIN, std::min<int64_t>(INT32_MAX, int64_t(received_i) + o)));"),
 }
 
@@ -44,6 +49,8 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                    check=True)
     env = dict(os.environ, ORACLE_LIB=str(lib))
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_rd_hd.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_rooted.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"mutant {name} survived the pins:\n{res.stdout[-2000:]}"
