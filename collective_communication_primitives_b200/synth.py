@@ -116,19 +116,17 @@ def uniform01(label, n, seed=0):
     return (_z(key, 0, n) >> np.uint64(11)).astype(np.float64) * 2.0**-53
 
 
-def moe_counts(p=8, tokens=8192, experts=64, topk=2, zipf_s=1.1, hidden=4096, seed=0):
-    """Send-count matrix c[i][j] (elements) of a top-2 MoE dispatch.
+def moe_routes(p=8, tokens=8192, experts=64, topk=2, zipf_s=1.1, seed=0):
+    """Router output of a top-k MoE layer: expert ids, int32 array [p][tokens][topk].
 
     Every source rank routes ``tokens`` tokens; each picks ``topk`` distinct experts, the first with
     probability w_e ∝ (e+1)^-s, each next one from w renormalised without the experts already
     picked. Expert e lives on rank e // (experts / p), so rank 0 holds the most popular experts.
-    Each assignment is one row of ``hidden`` elements.
     """
     if experts % p:
         raise ValueError("experts must split evenly over ranks")
-    per_rank = experts // p
     w = (np.arange(experts, dtype=np.float64) + 1.0) ** (-zipf_s)
-    counts = np.zeros((p, p), dtype=np.int64)
+    routes = np.zeros((p, tokens, topk), dtype=np.int32)
     for i in range(p):
         u = uniform01(f"moe.route.rank{i}", tokens * topk, seed).reshape(tokens, topk)
         avail = np.ones((tokens, experts), dtype=bool)
@@ -145,8 +143,29 @@ def moe_counts(p=8, tokens=8192, experts=64, topk=2, zipf_s=1.1, hidden=4096, se
                     cand = np.nonzero(avail[t])[0]
                     e[t] = cand[np.searchsorted(cdf[t, cand], target[t], side="right").clip(max=len(cand) - 1)]
             avail[np.arange(tokens), e] = False
-            np.add.at(counts[i], e // per_rank, 1)
+            routes[i, :, k] = e
+    return routes
+
+
+def moe_counts(p=8, tokens=8192, experts=64, topk=2, zipf_s=1.1, hidden=4096, seed=0):
+    """Send-count matrix c[i][j] (elements) of a top-k MoE dispatch: the assignments of
+    :func:`moe_routes` counted per destination rank, ``hidden`` elements per assignment."""
+    routes = moe_routes(p, tokens, experts, topk, zipf_s, seed)
+    per_rank = experts // p
+    counts = np.zeros((p, p), dtype=np.int64)
+    for i in range(p):
+        counts[i] = np.bincount(routes[i].ravel() // per_rank, minlength=p)
     return counts * hidden
+
+
+def moe_gate_weights(p=8, tokens=8192, topk=2, seed=0):
+    """Gate weights of the router output, fp32 [p][tokens][topk]: positive, each token's summing to 1
+    (up to fp32 rounding)."""
+    out = np.zeros((p, tokens, topk), dtype=np.float32)
+    for i in range(p):
+        u = 0.05 + uniform01(f"moe.gate.rank{i}", tokens * topk, seed).reshape(tokens, topk)
+        out[i] = (u / u.sum(axis=1, keepdims=True)).astype(np.float32)
+    return out
 
 
 def count_matrix_stats(counts):

@@ -17,7 +17,7 @@ _LIB = None
 
 DTYPE_CODES = {"int32": 0, "fp32": 1, "bf16": 2}
 OP_CODES = {"sum": 0, "min": 1, "max": 2, "avg": 3}
-ACC_CODES = {"exact": 0, "rankfold": 1}
+ACC_CODES = {"exact": 0, "rankfold": 1, "slotfold": 1}
 NP_DTYPES = {"int32": np.int32, "fp32": np.float32, "bf16": np.uint16}
 
 
@@ -49,6 +49,8 @@ def lib():
             "oracle_gather": [i32, pp, vp, sz, i32, i32],
             "oracle_rd_allreduce": [i32, pp, pp, sz, i32, i32],
             "oracle_hd_allreduce": [i32, pp, pp, sz, i32, i32],
+            "oracle_moe_dispatch": [i32, pp, pp, sz, i32, sz, i32, i32, sz, pp, i64p, pp, i64p],
+            "oracle_moe_combine": [i32, pp, pp, pp, pp, sz, i32, sz, i32, i32, pp, i32],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -239,6 +241,50 @@ def hd_allreduce(inputs, dtype, op):
     outs = _outs(len(ins), n, dtype)
     _check(lib().oracle_hd_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
            "hd_allreduce")
+    return outs
+
+
+def moe_dispatch(x, idx, experts, cap_rows, dtype):
+    """MoE dispatch: count -> exchange counts -> prefix sums -> pack/permute -> Alltoallv.
+
+    x: p arrays [T][H] (token rows of each source rank); idx: p int32 arrays [T][k] of expert ids.
+    Returns dict(recv=[p arrays [cap_rows][H]], expert_counts=[p][E], pos=[p arrays [T][k]] (row of
+    each assignment in its owner's receive buffer), recv_counts=[p]); raises OverflowError when a
+    destination would receive more than cap_rows rows."""
+    xs = [_arr(a, dtype) for a in x]
+    ids = [np.ascontiguousarray(a, dtype=np.int32) for a in idx]
+    p = len(xs)
+    T, k = ids[0].shape
+    H = xs[0].shape[1] if xs[0].ndim == 2 else (xs[0].size // T if T else 0)
+    recv = [np.zeros((cap_rows, H), dtype=NP_DTYPES[dtype]) for _ in range(p)]
+    pos = [np.full((T, k), -1, dtype=np.int32) for _ in range(p)]
+    ec = np.zeros((p, experts), dtype=np.int64)
+    rc = np.zeros(p, dtype=np.int64)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    status = lib().oracle_moe_dispatch(p, _ptrs(xs), _ptrs(ids), T, k, H, experts, DTYPE_CODES[dtype], cap_rows,
+                                       _ptrs(recv), ec.ctypes.data_as(i64p), _ptrs(pos), rc.ctypes.data_as(i64p))
+    if status == 1:
+        raise OverflowError("a destination would receive more rows than its capacity")
+    _check(status, "moe_dispatch")
+    return {"recv": recv, "expert_counts": ec, "pos": pos, "recv_counts": rc}
+
+
+def moe_combine(y, idx, weights, dtype, experts, residual=None, acc="exact"):
+    """MoE combine: reverse Alltoallv -> unpermute -> weighted sum (+ residual).
+
+    y: p arrays [rows][H] of expert outputs in the dispatch receive layout; idx: the router's expert
+    ids [T][k]; weights: fp32 [T][k]; residual: None or p arrays [T][H]. acc "exact" (double,
+    rounded once) or "slotfold" (fp32 left fold in slot order). Returns p arrays [T][H]."""
+    ys = [_arr(a, dtype) for a in y]
+    ids = [np.ascontiguousarray(a, dtype=np.int32) for a in idx]
+    ws = [np.ascontiguousarray(a, dtype=np.float32) for a in weights]
+    p = len(ys)
+    T, k = ids[0].shape
+    H = ys[0].shape[1]
+    res = None if residual is None else [_arr(a, dtype) for a in residual]
+    outs = [np.zeros((T, H), dtype=NP_DTYPES[dtype]) for _ in range(p)]
+    _check(lib().oracle_moe_combine(p, _ptrs(ys), _ptrs(ids), _ptrs(ws), None if res is None else _ptrs(res), T, k, H,
+                                    experts, DTYPE_CODES[dtype], _ptrs(outs), ACC_CODES[acc]), "moe_combine")
     return outs
 
 

@@ -624,6 +624,163 @@ int oracle_hd_allreduce(int p, const void* const* in, void* const* out, size_t n
     return 0;
 }
 
+/* ===================== MoE dispatch and combine ================================================= */
+/* [Primer] "Ragged All-to-All：MoE 的真实输入通常不等长" lists the steps around the variable-split
+ * exchange, in this order: router output, counting assignments per destination, exchanging the
+ * counts, prefix-summing them into offsets, packing/permuting the payload, the variable-split
+ * All-to-All, the experts' compute, the reverse variable-split All-to-All, and unpermute/combine.
+ * [Primer] "Expert Parallel：All-to-All 搬运的是 Assignment": the unit that moves is an expert
+ * assignment (a token routed to k experts travels k times), and the combine step weights the
+ * returning expert outputs with the gate weights and adds the residual, back in source-token layout.
+ *
+ * Readings (ours; the pages name the steps but not these rules):
+ *   - E experts, E a multiple of p; expert e lives on rank e / (E/p);
+ *   - the router output of rank i is idx_i[t][s] (token t < T, slot s < k) and, for the combine,
+ *     the gate weights w_i[t][s] (fp32);
+ *   - pack/permute lists rank i's assignments (t, s) by expert id, ties in token order and then
+ *     slot order (a stable sort of the flattened list t*k + s by expert), so every block a
+ *     destination receives is grouped by expert;
+ *   - the exchange is the Alltoallv above with c_ij = rows from i to j (H elements a row); the
+ *     destination layout is [from rank 0 | from rank 1 | ...];
+ *   - combine: out_i[t] = residual_i[t] (when given) + Σ_s w_i[t][s] * y_i(t, s), where y_i(t, s)
+ *     is the row the expert owner returns for assignment (t, s). acc EXACT sums in double and
+ *     rounds once; acc SLOTFOLD (= 1) is the fp32 left fold in slot order (residual first; without
+ *     a residual the fold starts at the slot-0 product), every product and sum rounded to fp32.
+ * A capacity shortfall (some destination would receive more than cap_rows rows) writes nothing and
+ * returns 1; an expert id outside [0, E) is outside the definitions (-1). */
+
+struct MoeRoute {
+    int E_loc = 0;
+    std::vector<std::vector<int64_t>> cnt;    // [p][E] assignments from rank i to expert e
+    std::vector<int64_t> c;                   // [p][p] rows from rank i to rank j
+    std::vector<std::vector<int64_t>> order;  // [p][T*k] flattened assignment ids in packed order
+};
+
+static int moe_route(int p, const int32_t* const* idx, size_t T, int k, int E, MoeRoute* R) {
+    if (p < 1 || k < 1 || E < p || E % p != 0) return -1;
+    const size_t A = T * size_t(k);
+    R->E_loc = E / p;
+    R->cnt.assign(p, std::vector<int64_t>(E, 0));
+    R->c.assign(size_t(p) * p, 0);
+    R->order.assign(p, std::vector<int64_t>());
+    for (int i = 0; i < p; ++i) {
+        for (size_t a = 0; a < A; ++a) {  // count assignments per expert, hence per destination
+            const int32_t e = idx[i][a];
+            if (e < 0 || e >= E) return -1;
+            R->cnt[i][e] += 1;
+            R->c[size_t(i) * p + e / R->E_loc] += 1;
+        }
+        std::vector<int64_t>& ord = R->order[i];  // pack/permute: stable by expert id
+        ord.resize(A);
+        for (size_t a = 0; a < A; ++a) ord[a] = int64_t(a);
+        const int32_t* ids = idx[i];
+        std::stable_sort(ord.begin(), ord.end(), [ids](int64_t x, int64_t y) { return ids[x] < ids[y]; });
+    }
+    return 0;
+}
+
+int oracle_moe_dispatch(int p, const void* const* x, const int32_t* const* idx, size_t T, int k, size_t H, int E,
+                        int dtype, size_t cap_rows, void* const* recv, int64_t* expert_counts,
+                        int32_t* const* pos, int64_t* recv_counts) {
+    if (!valid_common(p, dtype)) return -1;
+    MoeRoute R;
+    if (moe_route(p, idx, T, k, E, &R) != 0) return -1;
+    const size_t A = T * size_t(k), d = elem_size(dtype);
+    // exchange counts + capacity: rows arriving at each destination
+    std::vector<int64_t> rows_in(p, 0);
+    for (int i = 0; i < p; ++i)
+        for (int j = 0; j < p; ++j) rows_in[j] += R.c[size_t(i) * p + j];
+    for (int j = 0; j < p; ++j)
+        if (size_t(rows_in[j]) > cap_rows) return 1;
+    // pack: send_i holds rank i's rows in packed order
+    std::vector<std::vector<unsigned char>> send(p);
+    std::vector<const void*> send_ptrs(p);
+    for (int i = 0; i < p; ++i) {
+        send[i].resize(std::max<size_t>(A * H * d, 1));
+        for (size_t q = 0; q < A; ++q) {
+            const size_t t = size_t(R.order[i][q]) / size_t(k);
+            std::memcpy(send[i].data() + q * H * d, static_cast<const char*>(x[i]) + t * H * d, H * d);
+        }
+        send_ptrs[i] = send[i].data();
+    }
+    // variable-split exchange: element counts are rows times H
+    std::vector<int64_t> ce(size_t(p) * p);
+    for (size_t a = 0; a < ce.size(); ++a) ce[a] = R.c[a] * int64_t(H);
+    if (oracle_alltoallv(p, send_ptrs.data(), recv, ce.data(), dtype, nullptr) != 0) return -1;
+    // where every assignment landed: its row in the owner's receive buffer
+    if (pos) {
+        for (int i = 0; i < p; ++i) {
+            for (size_t q = 0; q < A; ++q) {
+                const int64_t a = R.order[i][q];
+                const int j = idx[i][a] / R.E_loc;
+                int64_t sdispl = 0, rdispl = 0;
+                for (int jj = 0; jj < j; ++jj) sdispl += R.c[size_t(i) * p + jj];
+                for (int ii = 0; ii < i; ++ii) rdispl += R.c[size_t(ii) * p + j];
+                pos[i][a] = int32_t(rdispl + (int64_t(q) - sdispl));
+            }
+        }
+    }
+    if (expert_counts)
+        for (int i = 0; i < p; ++i)
+            for (int e = 0; e < E; ++e) expert_counts[size_t(i) * E + e] = R.cnt[i][e];
+    if (recv_counts)
+        for (int j = 0; j < p; ++j) recv_counts[j] = rows_in[j];
+    return 0;
+}
+
+int oracle_moe_combine(int p, const void* const* y, const int32_t* const* idx, const float* const* w,
+                       const void* const* residual, size_t T, int k, size_t H, int E, int dtype, void* const* out,
+                       int acc) {
+    if (p < 1 || (dtype != DT_FP32 && dtype != DT_BF16) || (acc != ACC_EXACT && acc != ACC_RANKFOLD)) return -1;
+    MoeRoute R;
+    if (moe_route(p, idx, T, k, E, &R) != 0) return -1;
+    const size_t A = T * size_t(k), d = elem_size(dtype);
+    // reverse variable-split exchange (counts transposed): back_i holds, in packed order, the rows
+    // the experts returned for rank i's assignments
+    std::vector<std::vector<unsigned char>> back(p);
+    std::vector<void*> back_ptrs(p);
+    for (int i = 0; i < p; ++i) {
+        back[i].assign(std::max<size_t>(A * H * d, 1), 0);
+        back_ptrs[i] = back[i].data();
+    }
+    std::vector<int64_t> ct(size_t(p) * p);
+    for (int i = 0; i < p; ++i)
+        for (int j = 0; j < p; ++j) ct[size_t(j) * p + i] = R.c[size_t(i) * p + j] * int64_t(H);
+    if (oracle_alltoallv(p, y, back_ptrs.data(), ct.data(), dtype, nullptr) != 0) return -1;
+    // unpermute + weighted combine
+    for (int i = 0; i < p; ++i) {
+        std::vector<int64_t> qpos(A);
+        for (size_t q = 0; q < A; ++q) qpos[size_t(R.order[i][q])] = int64_t(q);
+        for (size_t t = 0; t < T; ++t) {
+            for (size_t h = 0; h < H; ++h) {
+                if (acc == ACC_EXACT) {
+                    double sum = residual ? load_as_double(residual[i], dtype, t * H + h) : 0.0;
+                    for (int s = 0; s < k; ++s) {
+                        const size_t q = size_t(qpos[t * k + s]);
+                        sum += double(w[i][t * k + s]) * load_as_double(back[i].data(), dtype, q * H + h);
+                    }
+                    store_double_rounded_once(out[i], dtype, t * H + h, sum);
+                } else {
+                    float f;
+                    int s0 = 0;
+                    if (residual) {
+                        f = load_as_float(residual[i], dtype, t * H + h);
+                    } else {
+                        f = w[i][t * k] * load_as_float(back[i].data(), dtype, size_t(qpos[t * k]) * H + h);
+                        s0 = 1;
+                    }
+                    for (int s = s0; s < k; ++s) {
+                        const size_t q = size_t(qpos[t * k + s]);
+                        f = f + w[i][t * k + s] * load_as_float(back[i].data(), dtype, q * H + h);
+                    }
+                    store_float(out[i], dtype, t * H + h, f);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
 /* ===================== helpers the tests pin directly ============================================ */
 
 uint16_t oracle_float_to_bf16(float f) { return float_to_bf16_rne(f); }

@@ -30,6 +30,13 @@ MUTANTS = {
     "hd_keeps_wrong_half": ("const int kb = (r & d) ? group + d : group;", "const int kb = (r & d) ? group : group + d;"),
     "scatter_wrong_block": ("copy_element(in_root, size_t(r) * m + k, out[r], k, dtype);", "copy_element(in_root, size_t((r + 1) % p) * m + k, out[r], k, dtype);"),
     "gather_wrong_block": ("copy_element(in[r], k, out_root, size_t(r) * m + k, dtype);", "copy_element(in[r], k, out_root, size_t(p - 1 - r) * m + k, dtype);"),
+    "moe_ties_reversed": ("std::stable_sort(ord.begin(), ord.end(), [ids](int64_t x, int64_t y) { return ids[x] < ids[y]; });", "std::sort(ord.begin(), ord.end(), [ids](int64_t x, int64_t y) { return ids[x] < ids[y] || (ids[x] == ids[y] && x > y); });"),
+    "moe_owner_modulo": ("R->c[size_t(i) * p + e / R->E_loc] += 1;", "R->c[size_t(i) * p + e % p] += 1;"),
+    "moe_pos_no_source_offset": ("for (int ii = 0; ii < i; ++ii) rdispl += R.c[size_t(ii) * p + j];", ""),
+    "moe_pack_wrong_token": ("const size_t t = size_t(R.order[i][q]) / size_t(k);", "const size_t t = size_t(R.order[i][q]) % T;"),
+    "moe_combine_weight_slot_swapped": ("sum += double(w[i][t * k + s]) *", "sum += double(w[i][t * k + (k - 1 - s)]) *"),
+    "moe_combine_drops_residual": ("double sum = residual ? load_as_double(residual[i], dtype, t * H + h) : 0.0;", "double sum = 0.0;"),
+    "moe_reverse_untransposed": ("ct[size_t(j) * p + i] = R.c[size_t(i) * p + j] * int64_t(H);", "ct[size_t(i) * p + j] = R.c[size_t(i) * p + j] * int64_t(H);"),
     "int_sum_saturates": ("if (op == OP_SUM) i[k] = int32_t(uint32_t(received_i) + uint32_t(o));", "if (op == OP_SUM) i[k] = int32_t(std::max<int64_t>(INT32_MIN, std::min<int64_t>(INT32_MAX, int64_t(received_i) + o)));"),
 }
 
@@ -51,6 +58,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                           os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                           os.path.join(ROOT, "tests", "test_oracle_rd_hd.py"),
-                          os.path.join(ROOT, "tests", "test_oracle_rooted.py")],
+                          os.path.join(ROOT, "tests", "test_oracle_rooted.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_moe.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"mutant {name} survived the pins:\n{res.stdout[-2000:]}"
