@@ -11,6 +11,8 @@
 //   §1.3 Reduce:        out_root[i] = ⊕_r in_r[i]
 //   §1.4 AllReduce:     out_r[i]    = ⊕_r' in_r'[i] for every r
 //   §1.5 ReduceScatter: out_r[k]    = ⊕_q in_q[r·m + k], m = n/p
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace simcomm {
@@ -77,7 +79,9 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
     if constexpr (HINT) pol = l2_evict_first_policy();
     const size_t step = size_t(gridDim.x) * kDirThreads * kDirUnroll;
 
-    for (int sg = 0; sg < nseg; ++sg) {
+    // ReduceScatter segments are spread over blockIdx.y (all of them in parallel when a segment is
+    // too short to fill the grid); AllReduce and Reduce have one segment and gridDim.y == 1.
+    for (int sg = blockIdx.y; sg < nseg; sg += gridDim.y) {
         const size_t in_base = size_t(sg) * seg_packs;
         for (size_t i0 = size_t(blockIdx.x) * kDirThreads * kDirUnroll + threadIdx.x; i0 < seg_packs; i0 += step) {
             bool ok[kDirUnroll];
@@ -138,13 +142,23 @@ __global__ void __launch_bounds__(kDirThreads) k_direct_vec(const __grid_constan
     }
 
     // Ragged tail of AllReduce/Reduce (n not a multiple of the pack): the last block, element-wise.
-    if (a.mode != MODE_REDUCE_SCATTER && blockIdx.x == gridDim.x - 1) {
+    if (a.mode != MODE_REDUCE_SCATTER && blockIdx.x == gridDim.x - 1 && blockIdx.y == 0) {
         for (size_t e = seg_packs * L + threadIdx.x; e < a.n; e += kDirThreads)
             reduce_one_element<DT, OP, SCALE>(a, p, e);
     }
 }
 
 // ---- launch ------------------------------------------------------------------------------------
+
+// Grid of the 16/32-byte path: x covers the packs of one segment (at most max_blocks), y the
+// ReduceScatter segments that fit beside it in max_blocks.
+static dim3 vec_grid(const DirectReduceArgs& a, size_t packs, int max_blocks) {
+    const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
+    const int gx = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
+    int gy = 1;
+    if (a.mode == MODE_REDUCE_SCATTER) gy = std::max(1, std::min(a.p, max_blocks / gx));
+    return dim3(unsigned(gx), unsigned(gy), 1u);
+}
 
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStream_t s) {
@@ -157,10 +171,7 @@ static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStre
     }
     // 32-byte packs when every buffer allows them, else 16-byte packs
     if (a.vec == 2) {
-        constexpr int L = PackW<DT, 8>::L;
-        const size_t packs = a.seg / L;
-        const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
-        const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
+        const dim3 grid = vec_grid(a, a.seg / PackW<DT, 8>::L, max_blocks);
         if (a.l2_hint) {
             switch (a.p) {
                 case 2: k_direct_vec<DT, OP, 2, SCALE, 8, true><<<grid, kDirThreads, 0, s>>>(a); break;
@@ -178,10 +189,7 @@ static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStre
         }
         return cudaGetLastError();
     }
-    constexpr int L = PackW<DT, 4>::L;
-    const size_t packs = a.seg / L;
-    const size_t want = (packs + size_t(kDirThreads) * kDirUnroll - 1) / (size_t(kDirThreads) * kDirUnroll);
-    const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));
+    const dim3 grid = vec_grid(a, a.seg / PackW<DT, 4>::L, max_blocks);
     switch (a.p) {
         case 2: k_direct_vec<DT, OP, 2, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
         case 3: k_direct_vec<DT, OP, 3, SCALE, 4, false><<<grid, kDirThreads, 0, s>>>(a); break;
