@@ -49,6 +49,7 @@ def lib():
             "oracle_gather": [i32, pp, vp, sz, i32, i32],
             "oracle_rd_allreduce": [i32, pp, pp, sz, i32, i32],
             "oracle_hd_allreduce": [i32, pp, pp, sz, i32, i32],
+            "oracle_tree_allreduce": [i32, pp, pp, sz, i32, i32, i32],
             "oracle_moe_dispatch": [i32, pp, pp, sz, i32, sz, i32, i32, sz, pp, i64p, pp, i64p],
             "oracle_moe_combine": [i32, pp, pp, pp, pp, sz, i32, sz, i32, i32, pp, i32],
         }
@@ -241,6 +242,17 @@ def hd_allreduce(inputs, dtype, op):
     outs = _outs(len(ins), n, dtype)
     _check(lib().oracle_hd_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op]),
            "hd_allreduce")
+    return outs
+
+
+def tree_allreduce(inputs, dtype, op, double_tree=False):
+    """Tree AllReduce: reduce up a heap-numbered binary tree, broadcast down; the double tree runs
+    the second half of the elements on the mirrored tree."""
+    ins = [_arr(x, dtype) for x in inputs]
+    n = ins[0].size
+    outs = _outs(len(ins), n, dtype)
+    _check(lib().oracle_tree_allreduce(len(ins), _ptrs(ins), _ptrs(outs), n, DTYPE_CODES[dtype], OP_CODES[op],
+                                       1 if double_tree else 0), "tree_allreduce")
     return outs
 
 

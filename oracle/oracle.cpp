@@ -624,6 +624,58 @@ int oracle_hd_allreduce(int p, const void* const* in, void* const* out, size_t n
     return 0;
 }
 
+/* ===================== tree AllReduce ============================================================ */
+/* [Primer] "Tree AllReduce 为什么更适合延迟敏感区间": reduce up a tree to its root, then broadcast
+ * the result down the same tree, in a number of rounds logarithmic in p. [Atlas] §2.4 "double
+ * binary tree": two complementary binary trees over the same ranks, drawn as tree A = 0 -> {1, 2},
+ * 1 -> {3, 4}, 2 -> {5, 6} and tree B = the same shape with rank p-1-m where tree A has rank m.
+ * Readings (ours): a tree is the heap numbering of positions m = 0..p-1 (children 2m+1 and 2m+2
+ * when < p, the root at position 0); tree A puts rank m at position m, tree B rank p-1-m. A
+ * position's partial is its rank's input ⊕ its left child's partial ⊕ its right child's partial,
+ * folded in that order, in fp32 for fp32/bf16 data (wrapping int32 for int32 sums); the root's
+ * value is scaled for AVG, rounded once and passed down unchanged. The single tree (double_tree =
+ * 0) reduces all n elements on tree A; the double tree (double_tree = 1) reduces elements
+ * [0, ceil(n/2)) on tree A and the rest on tree B. */
+int oracle_tree_allreduce(int p, const void* const* in, void* const* out, size_t n, int dtype, int op,
+                          int double_tree) {
+    if (!valid_reduce_args(p, dtype, op, ACC_RANKFOLD) || (double_tree != 0 && double_tree != 1)) return -1;
+    const size_t half = double_tree ? (n + 1) / 2 : n;
+    std::vector<float> f(p);
+    std::vector<int32_t> iv(p);
+    for (size_t k = 0; k < n; ++k) {
+        const bool mirror = k >= half;
+        for (int m = p - 1; m >= 0; --m) {  // children sit at larger positions: they are done first
+            const int r = mirror ? p - 1 - m : m;
+            float af = 0.0f;
+            int32_t ai = 0;
+            if (dtype == DT_INT32) ai = static_cast<const int32_t*>(in[r])[k];
+            else af = load_as_float(in[r], dtype, k);
+            for (int c = 2 * m + 1; c <= 2 * m + 2 && c < p; ++c) {
+                if (dtype == DT_INT32) {
+                    ai = (op == OP_SUM) ? int32_t(uint32_t(ai) + uint32_t(iv[c])) : apply_minmax(op, ai, iv[c]);
+                } else if (op == OP_MIN || op == OP_MAX) {
+                    af = apply_minmax(op, af, f[c]);
+                } else {
+                    volatile float s = af + f[c];
+                    af = s;
+                }
+            }
+            f[m] = af;
+            iv[m] = ai;
+        }
+        for (int r = 0; r < p; ++r) {
+            if (dtype == DT_INT32) {
+                static_cast<int32_t*>(out[r])[k] = iv[0];
+            } else {
+                float v = f[0];
+                if (op == OP_AVG) { volatile float scale = 1.0f / float(p); v = v * scale; }
+                store_float(out[r], dtype, k, v);
+            }
+        }
+    }
+    return 0;
+}
+
 /* ===================== MoE dispatch and combine ================================================= */
 /* [Primer] "Ragged All-to-All：MoE 的真实输入通常不等长" lists the steps around the variable-split
  * exchange, in this order: router output, counting assignments per destination, exchanging the

@@ -37,6 +37,9 @@ MUTANTS = {
     "moe_combine_weight_slot_swapped": ("sum += double(w[i][t * k + s]) *", "sum += double(w[i][t * k + (k - 1 - s)]) *"),
     "moe_combine_drops_residual": ("double sum = residual ? load_as_double(residual[i], dtype, t * H + h) : 0.0;", "double sum = 0.0;"),
     "moe_reverse_untransposed": ("ct[size_t(j) * p + i] = R.c[size_t(i) * p + j] * int64_t(H);", "ct[size_t(i) * p + j] = R.c[size_t(i) * p + j] * int64_t(H);"),
+    "tree_children_swapped": ("for (int c = 2 * m + 1; c <= 2 * m + 2 && c < p; ++c) {", "for (int c = std::min(2 * m + 2, p - 1); c >= 2 * m + 1; --c) {"),
+    "tree_b_not_mirrored": ("const int r = mirror ? p - 1 - m : m;", "const int r = m;"),
+    "tree_split_floor": ("const size_t half = double_tree ? (n + 1) / 2 : n;", "const size_t half = double_tree ? n / 2 : n;"),
     "int_sum_saturates": ("if (op == OP_SUM) i[k] = int32_t(uint32_t(received_i) + uint32_t(o));", "if (op == OP_SUM) i[k] = int32_t(std::max<int64_t>(INT32_MIN, std::min<int64_t>(INT32_MAX, int64_t(received_i) + o)));"),
 }
 
@@ -59,6 +62,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                           os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                           os.path.join(ROOT, "tests", "test_oracle_rd_hd.py"),
                           os.path.join(ROOT, "tests", "test_oracle_rooted.py"),
-                          os.path.join(ROOT, "tests", "test_oracle_moe.py")],
+                          os.path.join(ROOT, "tests", "test_oracle_moe.py"),
+                          os.path.join(ROOT, "tests", "test_oracle_tree.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"mutant {name} survived the pins:\n{res.stdout[-2000:]}"
