@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--sweep-ps", default="2,4,8,16,64")
     ap.add_argument("--sweep-max-bytes", type=int, default=1 << 30, help="largest per-rank message")
     ap.add_argument("--sweep-out", default="", help="write the sweep's markdown summary here")
+    ap.add_argument("--moe", action="store_true",
+                    help="time only the MoE dispatch and combine on the MoE workload (one GPU)")
+    ap.add_argument("--no-moe", action="store_true", help="leave the MoE block out of the step's line")
     return ap.parse_args()
 
 
@@ -288,6 +291,107 @@ def time_e2e(comm, wl, ops, steps, warmup, stream):
 
 
 # ---------------------------------------------------------------------------------------------
+# MoE dispatch and combine on the MoE workload
+
+MOE = {"p": P, "tokens": 8192, "topk": 2, "experts": 64, "hidden": HIDDEN, "zipf_s": 1.1}
+
+
+class MoeWorkload:
+    """p ranks x 8192 tokens, top-2 of 64 experts with Zipf(1.1) popularity, 4096-wide bf16 rows;
+    every receive buffer holds p*T*k rows (the worst case: all assignments to one rank)."""
+
+    def __init__(self, device):
+        import numpy as np
+        import torch
+
+        from collective_communication_primitives_b200 import synth as S
+        p, T, k, E, H = P, MOE["tokens"], MOE["topk"], MOE["experts"], MOE["hidden"]
+        self.p, self.T, self.k, self.E, self.H = p, T, k, E, H
+        ids = S.moe_routes(p, T, E, k, MOE["zipf_s"], 0)
+        ws = S.moe_gate_weights(p, T, k, 0)
+
+        def bf16_rows(label, rows):
+            return torch.from_numpy(S.normal(label, rows * H, 1.0, "bf16").view(np.int16)).view(torch.bfloat16) \
+                .view(rows, H)
+
+        self.host_x = [bf16_rows(f"moe.x.rank{i}", T).pin_memory() for i in range(p)]
+        self.x = [h.to(device) for h in self.host_x]
+        self.res = [bf16_rows(f"moe.res.rank{i}", T).to(device) for i in range(p)]
+        self.idx = [torch.from_numpy(ids[i]).to(device) for i in range(p)]
+        self.w = [torch.from_numpy(ws[i]).to(device) for i in range(p)]
+        self.cap = p * T * k
+        self.recv = [torch.empty(self.cap, H, dtype=torch.bfloat16, device=device) for _ in range(p)]
+        self.pos = [torch.empty(T, k, dtype=torch.int32, device=device) for _ in range(p)]
+        self.out = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(p)]
+        self.recv_counts = torch.empty(p, dtype=torch.int64, device=device)
+        self.expert_counts = torch.empty(p, E, dtype=torch.int64, device=device)
+        self.col_rows = np.bincount((ids // (E // p)).reshape(-1), minlength=p)
+
+
+def moe_ops(comm, mw):
+    from collective_communication_primitives_b200 import bytemodel as BM
+    p, T, k, H = mw.p, mw.T, mw.k, mw.H
+    bd = BM.moe_dispatch_bytes(p, T, k, H, 2)
+    bc = BM.moe_combine_bytes(p, T, k, H, 2, residual=True)
+    return [
+        ("moe_dispatch_bf16", "moe_dispatch (count+scan+copy)",
+         lambda: comm.moe_dispatch(mw.x, mw.idx, mw.E, mw.recv, route_pos=mw.pos, expert_counts=mw.expert_counts,
+                                   recv_counts=mw.recv_counts), bd, bd),
+        ("moe_combine_bf16", "moe_combine",
+         lambda: comm.moe_combine(mw.recv, mw.idx, mw.pos, mw.w, mw.E, mw.out, residual=mw.res), bc, bc),
+    ]
+
+
+def moe_block(comm, mw, steps, warmup, stream, hbm):
+    """Device time of the MoE dispatch and combine (behind a spacer, CUDA events) and their HBM
+    roofline fractions."""
+    ops = moe_ops(comm, mw)
+    _, per_op = time_device(ops, steps, warmup, stream)
+    blk = {"workload": f"MoE layer, p={mw.p} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} experts (Zipf 1.1), "
+                       f"{mw.H}-wide bf16 rows", "max_recv_rows": int(mw.col_rows.max())}
+    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
+        g = kb / (ms / 1e3) / 1e9
+        blk[name] = {"ms": round(ms, 4), "GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
+                     "algorithmic_bytes": int(kb), "launches_per_call": 3 if "dispatch" in name else 1}
+    return blk
+
+
+def moe_main(args):
+    import torch
+
+    from collective_communication_primitives_b200 import simcomm as SC
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    mw = MoeWorkload("cuda:0")
+    comm = SC.SimComm(P)
+    hbm, peak_kind = peaks()
+    ops = moe_ops(comm, mw)
+    launches0 = comm.launch_count()
+    with ClockSampler(0) as clk:
+        total_ms, per_op = time_device(ops, args.steps, args.warmup, stream)
+    launches = (comm.launch_count() - launches0) * args.steps // (args.steps + args.warmup)
+    assert comm.async_error() == SC.OK
+    eff = sum(o[3] for o in ops)
+    ms = total_ms / args.steps
+    i_dom = max(range(len(ops)), key=lambda i: per_op[i])
+    name, kernel, _, _, kb = ops[i_dom]
+    achieved = kb / (per_op[i_dom] / 1e3) / 1e9
+    out = {"metric": METRIC, "value": round(eff / (ms / 1e3) / 1e9, 1), "unit": "GB/s", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 rows, fp32 combine", "data": "synthetic",
+           "config": {"workload": f"MoE dispatch + combine, p={P} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} "
+                                  f"experts (Zipf 1.1), {mw.H}-wide bf16 rows", "l2": "inputs larger than L2"},
+           "roofline": {"bound": "hbm", "kernel": f"{name} ({kernel})", "achieved": round(achieved, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": peak_kind, "traffic": None,
+                        "algorithmic_bytes_per_launch": int(kb), "ms_per_launch": round(per_op[i_dom], 4)},
+           "per_op": {o[0]: {"ms": round(t, 4), "GBps": round(o[4] / (t / 1e3) / 1e9, 1),
+                             "frac_of_measured": round(o[4] / (t / 1e3) / 1e9 / hbm, 4)} for o, t in zip(ops, per_op)},
+           "gpu_launches": int(launches), "clocks": clk.summary()}
+    print(json.dumps(out))
+    comm.close()
+
+
+# ---------------------------------------------------------------------------------------------
 # the oracle as a CPU baseline (and as the reference arm)
 
 def oracle_inputs(n):
@@ -394,13 +498,16 @@ def sweep(args):
     rows = []
     for p in [int(x) for x in args.sweep_ps.split(",")]:
         comm = SC.SimComm(p)
-        algos = ("direct", "ring", "rd", "hd") if p & (p - 1) == 0 else ("direct", "ring")
+        algos = ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll") if p & (p - 1) == 0 else \
+            ("direct", "ring", "tree", "dbtree", "ll")
         for algo in algos:
             for nbytes in sizes:
                 n = max(p, (nbytes // 4) // p * p)     # int32 elements, divisible by p
-                hold = 2 * p * n * 4 + {"direct": 0, "ring": 1, "rd": 2, "hd": 1}[algo] * p * n * 4
+                hold = 2 * p * n * 4 + {"direct": 0, "ring": 1, "rd": 2, "hd": 1, "tree": 1, "dbtree": 1, "ll": 0}[algo] * p * n * 4
                 if hold > SWEEP_CAP_BYTES:
                     continue
+                if algo == "ll" and p * (2 * p - 3) * -(-n // p) * 8 > (256 << 20):
+                    continue  # the LL protocol's receive slots are capped (small messages only)
                 x = [torch.randint(-2**24, 2**24, (n,), dtype=torch.int32, device=dev) for _ in range(p)]
                 y = [torch.empty(n, dtype=torch.int32, device=dev) for _ in range(p)]
                 m = n // p
@@ -441,7 +548,7 @@ def sweep(args):
         comm.close()
     fits = []
     for p in sorted({r["p"] for r in rows}):
-        for algo in ("direct", "ring", "rd", "hd"):
+        for algo in ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll"):
             for op in SWEEP_OPS:
                 pts = [r for r in rows if r["p"] == p and r["algo"] == algo and r["op"] == op]
                 if len(pts) < 3:
@@ -501,6 +608,9 @@ def main():
         return
     if args.sweep:
         sweep(args)
+        return
+    if args.moe:
+        moe_main(args)
         return
     import torch
     import torch.distributed as dist
@@ -601,6 +711,10 @@ def main():
     }
     if e2e:
         out["e2e"] = e2e
+    if not args.no_moe and not args.ops:
+        mw = MoeWorkload(device)
+        out["moe"] = moe_block(comm, mw, max(3, args.steps // 2), args.warmup, stream, hbm)
+        del mw
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -94,3 +94,19 @@ def busbw_factor(op, p):
     if op in ("broadcast", "reduce"):
         return 1.0
     raise ValueError(op)
+
+
+def moe_dispatch_bytes(p, tokens, k, hidden, d):
+    """Minimum HBM bytes of one MoE dispatch over p ranks: every token row read once, every
+    assignment row (k per token) written once, the expert ids read and the routing map written
+    (4 bytes per assignment each); the per-tile counting scratch is not counted."""
+    a = tokens * k
+    return p * (tokens * hidden * d + a * hidden * d + 2 * 4 * a)
+
+
+def moe_combine_bytes(p, tokens, k, hidden, d, residual=True):
+    """Minimum HBM bytes of one MoE combine over p ranks: every assignment's expert-output row read
+    once, the residual read (when given) and the output written once per token, and the expert id,
+    routing-map entry and gate weight read per assignment (4 bytes each)."""
+    a = tokens * k
+    return p * (a * hidden * d + (2 if residual else 1) * tokens * hidden * d + 3 * 4 * a)

@@ -30,6 +30,12 @@ struct sim_comm {
     size_t flags_cap = 0;           // elements
     char* stage = nullptr;          // ring partial buffers
     size_t stage_cap = 0;           // bytes
+    unsigned long long* ll = nullptr;  // LL receive slots
+    size_t ll_cap = 0;              // bytes
+    uint32_t ll_epoch = 0;          // LL tags: slot q of call e carries e * 128 + 1 + q
+    int ll_ctas_max = 0;
+    char* moe = nullptr;            // MoE dispatch counting and prefix scratch
+    size_t moe_cap = 0;             // bytes
     uint32_t epoch = 0;
     long long chunk_bytes = 1 << 20;
     long long ring_ctas = 0;
@@ -71,9 +77,11 @@ coll_status_t check_reduce_args(coll_dtype_t dt, coll_op_t op) {
 // Direct and ring exist for every collective; the butterfly algorithms for AllReduce only.
 coll_status_t check_algo(coll_algo_t algo, bool allreduce = false) {
     if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
-    if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD) {
+    if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE ||
+        algo == COLL_ALGO_RING_LL) {
         if (allreduce) return COLL_OK;
-        return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling exist for AllReduce only");
+        return fail(COLL_ERR_UNSUPPORTED,
+                    "recursive doubling, halving-doubling, the trees and the LL ring exist for AllReduce only");
     }
     return fail(COLL_ERR_INVALID_ARG, "unknown algorithm");
 }
@@ -93,6 +101,7 @@ Ctl make_ctl(sim_comm* c) {
     ctl.status = &c->dstate->status;
     ctl.host_status = c->dev_words;
     ctl.abort_flag = c->dev_words + 1;
+    ctl.abort_clock = &c->dstate->abort_clock;
     return ctl;
 }
 
@@ -167,6 +176,17 @@ coll_status_t ensure_flags(sim_comm* c, size_t count) {
     e = cudaMemset(c->flags, 0, count * sizeof(unsigned long long));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(ring flags)");
     c->flags_cap = count;
+    return COLL_OK;
+}
+
+coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
+    if (bytes <= c->moe_cap) return COLL_OK;
+    if (c->moe) cudaFree(c->moe);  // synchronises the device: no kernel still uses the old scratch
+    c->moe = nullptr;
+    c->moe_cap = 0;
+    cudaError_t e = cudaMalloc(&c->moe, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(MoE scratch)");
+    c->moe_cap = bytes;
     return COLL_OK;
 }
 
@@ -344,6 +364,127 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     return COLL_OK;
 }
 
+// Ring AllReduce on the low-latency protocol (flags inside the data), for small messages.
+constexpr size_t kLLMaxBytes = size_t(256) << 20;
+
+coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+    const int p = c->p;
+    LLArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.p = p;
+    a.n = n;
+    a.seg = (n + size_t(p) - 1) / size_t(p);
+    a.nslots = uint32_t(2 * p - 3);
+    const size_t bytes = size_t(p) * a.nslots * a.seg * sizeof(unsigned long long);
+    if (bytes > kLLMaxBytes)
+        return fail(COLL_ERR_UNSUPPORTED, "the LL protocol is for small messages: p * (2p-3) * ceil(n/p) * 8 bytes of "
+                                          "receive slots must stay within 256 MiB (use COLL_ALGO_RING)");
+    if (bytes > c->ll_cap) {
+        if (c->ll) cudaFree(c->ll);  // synchronises the device: no kernel still uses the old slots
+        c->ll = nullptr;
+        c->ll_cap = 0;
+        cudaError_t e = cudaMalloc(&c->ll, bytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(LL slots)");
+        e = cudaMemset(c->ll, 0, bytes);  // tag 0 is never a live tag
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(LL slots)");
+        c->ll_cap = bytes;
+    }
+    // tags must never repeat while old words may still sit in the slots: start again (and clear
+    // the slots, in stream order) before e * 128 + 127 would leave 32 bits
+    c->ll_epoch += 1;
+    if (c->ll_epoch >= (1u << 25)) {
+        cudaError_t e = cudaMemsetAsync(c->ll, 0, c->ll_cap, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(LL slots)");
+        c->ll_epoch = 1;
+    }
+    a.tag = c->ll_epoch * 128u + 1u;
+    a.ll = c->ll;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.timeout_ns = uint64_t(c->timeout_ns);
+    a.ctl = make_ctl(c);
+    // CTAs per rank: about 4 elements per thread, all CTAs resident at once (cooperative launch)
+    if (c->ll_ctas_max == 0) c->ll_ctas_max = ring_ll_max_ctas(c->num_sms);
+    const int g_cap = c->ll_ctas_max / p;
+    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
+    const size_t want = (a.seg + 1023) / 1024;
+    a.G = int(std::max<size_t>(1, std::min<size_t>(want, size_t(g_cap))));
+    cudaError_t e = launch_ring_ll(a, dt, op, s);
+    if (e != cudaSuccess) return cuda_fail(e, "LL ring launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
+// Single / double binary tree AllReduce on the tree executor.
+coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, bool dbl,
+                       cudaStream_t s) {
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt);
+    TreeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.p = p;
+    a.ntrees = dbl ? 2 : 1;
+    a.n = n;
+    a.half = dbl ? (n + 1) / 2 : n;
+    a.chunk = size_t(c->chunk_bytes) / 4;  // chunk bytes count the fp32/int32 partials, as on the ring
+    a.tile = std::min(a.chunk, kRingTaskBytes / 4);
+    a.ntile = uint32_t((a.chunk + a.tile - 1) / a.tile);
+    const size_t len[2] = {a.half, n - a.half};
+    for (int t = 0; t < a.ntrees; ++t) a.nch[t] = uint32_t((len[t] + a.chunk - 1) / a.chunk);
+    a.nchmax = std::max(a.nch[0], a.nch[1]);
+    // a chunk of at most one tile when the range is short: no empty tasks
+    if (a.nchmax == 1) {
+        const size_t longest = std::max(len[0], len[1]);
+        a.tile = std::min(a.tile, std::max<size_t>(16, longest));
+        a.ntile = uint32_t((std::min(a.chunk, longest) + a.tile - 1) / a.tile);
+        a.chunk = size_t(a.ntile) * a.tile;
+    }
+    // levels: internal positions (2m+1 < p) reduce, deepest level first; then every non-root
+    // position copies its parent's result, root side first
+    auto level_of = [](int m) { int L = 0; while ((2 << L) <= m + 1) ++L; return L; };
+    const int internal_last = p / 2 - 1, depth = level_of(p - 1);
+    const int reduce_levels = level_of(internal_last) + 1;
+    uint32_t g = 0;
+    for (int L = reduce_levels - 1; L >= 0; --L, ++g) {
+        a.step_kind[g] = 0;
+        a.step_first[g] = uint32_t((1 << L) - 1);
+        a.step_count[g] = uint32_t(std::min((2 << L) - 1, internal_last + 1) - ((1 << L) - 1));
+    }
+    for (int L = 1; L <= depth; ++L, ++g) {
+        a.step_kind[g] = 1;
+        a.step_first[g] = uint32_t((1 << L) - 1);
+        a.step_count[g] = uint32_t(std::min((2 << L) - 1, p) - ((1 << L) - 1));
+    }
+    a.nsteps = g;
+    a.start[0] = 0;
+    for (uint32_t k = 0; k < a.nsteps; ++k)
+        a.start[k + 1] = a.start[k] + (a.nch[0] + (a.ntrees == 2 ? a.nch[1] : 0)) * a.step_count[k] * a.ntile;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.timeout_ns = uint64_t(c->timeout_ns);
+    a.st = c->dstate;
+    a.ctl = make_ctl(c);
+    coll_status_t st = ensure_flags(c, size_t(4) * p * a.nchmax);
+    if (st != COLL_OK) return st;
+    a.flags = c->flags;
+    a.epoch = next_epoch(c);
+    a.stage_stride = round_up(n * 4, 256);
+    if ((st = ensure_stage(c, a.stage_stride * size_t(p))) != COLL_OK) return st;
+    a.stage = c->stage;
+    // 16-byte packs need every range start (half, chunk and tile starts) on a 16-byte boundary of
+    // the element and of the partial buffers
+    bool vec = (a.half * d) % 16 == 0 && (a.half * 4) % 16 == 0 && (a.tile * d) % 16 == 0 &&
+               (a.tile * 4) % 16 == 0 && (a.chunk * 4) % 16 == 0;
+    for (int r = 0; r < p; ++r) vec = vec && aligned16(a.ptrs.send[r]) && aligned16(a.ptrs.recv[r]);
+    a.vec = vec ? 1 : 0;
+    int ctas = c->ring_ctas > 0 ? int(c->ring_ctas) : c->ring_ctas_max;
+    if (a.start[a.nsteps] < uint32_t(ctas)) ctas = int(std::max<uint32_t>(a.start[a.nsteps], 1));
+    cudaError_t e = launch_tree(a, dt, op, ctas, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tree executor launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
 // Recursive doubling / halving-doubling AllReduce on the butterfly executor.
 coll_status_t run_butterfly(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, int kind,
                             cudaStream_t s) {
@@ -505,6 +646,8 @@ coll_status_t sim_comm_destroy(sim_comm_t c) {
     cudaDeviceSynchronize();
     if (c->flags) cudaFree(c->flags);
     if (c->stage) cudaFree(c->stage);
+    if (c->moe) cudaFree(c->moe);
+    if (c->ll) cudaFree(c->ll);
     if (c->dstate) cudaFree(c->dstate);
     if (c->host_words) cudaFreeHost(c->host_words);
     delete c;
@@ -592,6 +735,8 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, b, n, dt, op, MODE_ALLREDUCE, 0, s);
     if (algo == COLL_ALGO_RD) return run_butterfly(c, b, n, dt, op, BFLY_RD, s);
     if (algo == COLL_ALGO_HD) return run_butterfly(c, b, n, dt, op, BFLY_HD, s);
+    if (algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE) return run_tree(c, b, n, dt, op, algo == COLL_ALGO_DBTREE, s);
+    if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, op, s);
     RingPlan pl;
     pl.kind = RING_ALLREDUCE;
     pl.seg = (n + size_t(p) - 1) / size_t(p);
@@ -862,6 +1007,168 @@ coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* count
 
 }  // extern "C"
 
+// ---- MoE dispatch and combine -------------------------------------------------------------------
+
+namespace {
+
+// Shape checks shared by dispatch and combine.
+coll_status_t check_moe_shape(sim_comm* c, size_t tokens, int k, size_t hidden, int experts) {
+    const int p = c->p;
+    if (k < 1 || k > kMoeMaxTopk) return fail(COLL_ERR_INVALID_ARG, "k must be in [1, 32]");
+    if (experts < p || experts % p != 0 || experts > kMoeMaxExperts)
+        return fail(COLL_ERR_INVALID_ARG, "experts must be a multiple of p in [p, 4096]");
+    if (hidden == 0) return fail(COLL_ERR_INVALID_ARG, "hidden must be positive");
+    if (tokens > size_t(INT32_MAX) / size_t(k)) return fail(COLL_ERR_INVALID_ARG, "tokens * k must fit in int32");
+    return COLL_OK;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+coll_status_t coll_moe_dispatch(sim_comm_t c, const void* const* x, const int32_t* const* topk_idx, size_t tokens,
+                                int k, size_t hidden, int experts, coll_dtype_t dt, void* const* recv,
+                                size_t recv_cap_rows, int32_t* const* route_pos, long long* expert_counts_dev,
+                                long long* recv_counts_dev, coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
+    if (recv_cap_rows > size_t(INT32_MAX)) return fail(COLL_ERR_INVALID_ARG, "recv_cap_rows must fit in int32");
+    if (!x || !topk_idx || !recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    if ((expert_counts_dev && reinterpret_cast<uintptr_t>(expert_counts_dev) % 8 != 0) ||
+        (recv_counts_dev && reinterpret_cast<uintptr_t>(recv_counts_dev) % 8 != 0))
+        return fail(COLL_ERR_INVALID_ARG, "count arrays must be 8-byte aligned");
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt), row = hidden * d, A = tokens * size_t(k);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(x[r], tokens * row, d, "token")) != COLL_OK) return st;
+        if ((st = check_ptr(topk_idx[r], A * 4, 4, "expert id")) != COLL_OK) return st;
+        if ((st = check_ptr(recv[r], recv_cap_rows * row, d, "recv")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(x[r]), uintptr_t(x[r]) + tokens * row, false, r});
+        rs.push_back({uintptr_t(topk_idx[r]), uintptr_t(topk_idx[r]) + A * 4, false, r});
+        rs.push_back({uintptr_t(recv[r]), uintptr_t(recv[r]) + recv_cap_rows * row, true, r});
+        if (route_pos) {
+            if ((st = check_ptr(route_pos[r], A * 4, 4, "route_pos")) != COLL_OK) return st;
+            rs.push_back({uintptr_t(route_pos[r]), uintptr_t(route_pos[r]) + A * 4, true, r});
+        }
+    }
+    if ((st = check_ranges(rs, INPLACE_NONE, 0)) != COLL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) {  // nothing routed: only the count outputs change
+        cudaError_t e = cudaSuccess;
+        if (expert_counts_dev) e = cudaMemsetAsync(expert_counts_dev, 0, size_t(p) * experts * sizeof(long long), s);
+        if (e == cudaSuccess && recv_counts_dev) e = cudaMemsetAsync(recv_counts_dev, 0, size_t(p) * sizeof(long long), s);
+        return e == cudaSuccess ? COLL_OK : cuda_fail(e, "cudaMemsetAsync(MoE counts)");
+    }
+    MoeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.p = p;
+    a.k = k;
+    a.E = experts;
+    a.E_loc = experts / p;
+    a.elem_bytes = int(d);
+    a.T = tokens;
+    a.H = hidden;
+    a.A = A;
+    a.cap_rows = recv_cap_rows;
+    a.ntiles = uint32_t((A + kMoeTile - 1) / kMoeTile);
+    for (int r = 0; r < p; ++r) {
+        a.src[r] = x[r];
+        a.idx[r] = topk_idx[r];
+        a.dst[r] = recv[r];
+        a.pos[r] = route_pos ? route_pos[r] : nullptr;
+    }
+    // scratch: tile counts [p][ntiles][E], in-tile ranks [p][A], totals and first rows [p][E] each
+    const size_t b_hist = align_up(size_t(p) * a.ntiles * experts * 4, 256);
+    const size_t b_rank = align_up(size_t(p) * A * 4, 256);
+    const size_t b_pe = align_up(size_t(p) * experts * 4, 256);
+    if ((st = ensure_moe(c, b_hist + b_rank + 2 * b_pe)) != COLL_OK) return st;
+    a.tile_hist = reinterpret_cast<int32_t*>(c->moe);
+    a.rank_in_tile = reinterpret_cast<int32_t*>(c->moe + b_hist);
+    a.cnt = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank);
+    a.base = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + b_pe);
+    a.expert_counts_out = expert_counts_dev;
+    a.recv_counts_out = recv_counts_dev;
+    a.st = c->dstate;
+    a.ctl = make_ctl(c);
+    cudaError_t e = launch_moe_dispatch(a, c->num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "MoE dispatch launch");
+    c->launches += 3;
+    return COLL_OK;
+}
+
+coll_status_t coll_moe_combine(sim_comm_t c, const void* const* y, size_t y_rows, const int32_t* const* topk_idx,
+                               const int32_t* const* route_pos, const float* const* topk_weight,
+                               const void* const* residual, size_t tokens, int k, size_t hidden, int experts,
+                               coll_dtype_t dt, void* const* out, coll_stream_t stream) {
+    coll_status_t st = check_usable(c);
+    if (st != COLL_OK) return st;
+    if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if (dt == COLL_INT32) return fail(COLL_ERR_UNSUPPORTED, "the weighted combine needs fp32 or bf16 rows");
+    if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
+    if (!y || !topk_idx || !route_pos || !topk_weight || !out) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+    if (tokens == 0) return COLL_OK;
+    const int p = c->p;
+    const size_t d = dtype_bytes(dt), row = hidden * d, A = tokens * size_t(k);
+    std::vector<Range> rs;
+    for (int r = 0; r < p; ++r) {
+        if ((st = check_ptr(y[r], y_rows * row, d, "expert output")) != COLL_OK) return st;
+        if ((st = check_ptr(topk_idx[r], A * 4, 4, "expert id")) != COLL_OK) return st;
+        if ((st = check_ptr(route_pos[r], A * 4, 4, "route_pos")) != COLL_OK) return st;
+        if ((st = check_ptr(topk_weight[r], A * 4, 4, "gate weight")) != COLL_OK) return st;
+        if ((st = check_ptr(out[r], tokens * row, d, "out")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(y[r]), uintptr_t(y[r]) + y_rows * row, false, r});
+        rs.push_back({uintptr_t(topk_idx[r]), uintptr_t(topk_idx[r]) + A * 4, false, r});
+        rs.push_back({uintptr_t(route_pos[r]), uintptr_t(route_pos[r]) + A * 4, false, r});
+        rs.push_back({uintptr_t(topk_weight[r]), uintptr_t(topk_weight[r]) + A * 4, false, r});
+        rs.push_back({uintptr_t(out[r]), uintptr_t(out[r]) + tokens * row, true, r});
+        if (residual && (st = check_ptr(residual[r], tokens * row, d, "residual")) != COLL_OK) return st;
+    }
+    if ((st = check_ranges(rs, INPLACE_NONE, 0)) != COLL_OK) return st;
+    // a residual may be its own rank's output (out = residual + Σ w y, element by element), and
+    // must not overlap any other output
+    for (int r = 0; residual && r < p; ++r) {
+        const Range res{uintptr_t(residual[r]), uintptr_t(residual[r]) + tokens * row, false, r};
+        for (int q = 0; q < p; ++q) {
+            const Range o{uintptr_t(out[q]), uintptr_t(out[q]) + tokens * row, true, q};
+            if (overlap(res, o) && !(q == r && res.lo == o.lo))
+                return fail(COLL_ERR_INVALID_ARG, "a residual overlaps an output other than its own rank's");
+        }
+    }
+    MoeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.p = p;
+    a.k = k;
+    a.E = experts;
+    a.E_loc = experts / p;
+    a.elem_bytes = int(d);
+    a.has_res = residual ? 1 : 0;
+    a.T = tokens;
+    a.H = hidden;
+    a.A = A;
+    a.cap_rows = y_rows;
+    for (int r = 0; r < p; ++r) {
+        a.src[r] = y[r];
+        a.idx[r] = topk_idx[r];
+        a.pos[r] = const_cast<int32_t*>(route_pos[r]);
+        a.w[r] = topk_weight[r];
+        a.dst[r] = out[r];
+        a.res[r] = residual ? residual[r] : nullptr;
+    }
+    a.st = c->dstate;
+    a.ctl = make_ctl(c);
+    cudaError_t e = launch_moe_combine(a, int(dt), c->num_sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "MoE combine launch");
+    c->launches += 1;
+    return COLL_OK;
+}
+
+}  // extern "C"
+
 // =================================================================================================
 // Ring AllReduce without any allocation.
 //
@@ -973,6 +1280,7 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     static_assert(sizeof(DevState) + 8 <= 256, "control words must fit the 256-byte control region");
     a.ctl.host_status = reinterpret_cast<uint32_t*>(base + sizeof(DevState));
     a.ctl.abort_flag = reinterpret_cast<uint32_t*>(base + sizeof(DevState) + 4);
+    a.ctl.abort_clock = &a.st->abort_clock;
     a.flags = reinterpret_cast<unsigned long long*>(base + ctl_bytes);
     a.stage = base + ctl_bytes + flag_bytes;
     a.stage_stride = stride;

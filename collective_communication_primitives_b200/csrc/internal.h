@@ -16,8 +16,9 @@ struct DevState {
     uint32_t status;    // first asynchronous error (coll_status_t), 0 = OK
     uint32_t task_ctr;  // ring / butterfly executor: next task to claim
     uint32_t done_ctr;  // ring / butterfly executor: CTAs that left the task loop
-    uint32_t pad;
+    uint32_t moe_ctr;   // MoE dispatch scan: blocks finished (the last one resets it)
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
+    unsigned long long abort_clock;  // global time of the last read of the host abort word
 };
 
 // What a kernel needs to report errors and notice an abort.
@@ -25,6 +26,7 @@ struct Ctl {
     uint32_t* status;                  // &DevState::status
     volatile uint32_t* host_status;    // device alias of a host-mapped word the host polls
     volatile const uint32_t* abort_flag;  // device alias of the host-mapped abort flag
+    unsigned long long* abort_clock;      // &DevState::abort_clock: rations the reads of abort_flag
 };
 
 struct RankPtrs {
@@ -130,6 +132,81 @@ struct ButterflyArgs {
     Ctl ctl;
 };
 
+// ---- tree executor: single and double binary tree AllReduce -------------------------------------
+
+constexpr int kMaxTreeSteps = 16;
+struct TreeArgs {
+    RankPtrs ptrs;
+    int p;
+    int ntrees;              // 1: tree A over [0, n); 2: tree A over [0, half), tree B over [half, n)
+    int vec;                 // 1: 16-byte packs (every range start 16-byte aligned)
+    size_t n, half;
+    size_t chunk;            // elements of one pipelined chunk
+    size_t tile;             // elements one CTA task moves
+    uint32_t ntile;          // tasks per chunk
+    uint32_t nch[2];         // chunks of each tree's range
+    uint32_t nchmax;
+    uint32_t nsteps;         // reduce levels (deepest first), then broadcast levels (root side first)
+    uint32_t step_kind[kMaxTreeSteps];   // 0 reduce, 1 broadcast
+    uint32_t step_first[kMaxTreeSteps];  // first heap position of the step
+    uint32_t step_count[kMaxTreeSteps];  // positions in the step
+    uint32_t start[kMaxTreeSteps + 1];   // first task of each step
+    uint32_t epoch;
+    float scale;
+    uint64_t timeout_ns;
+    char* stage;             // partials, one buffer per rank
+    size_t stage_stride;
+    unsigned long long* flags;  // [phase][tree][position][nchmax]: (epoch << 32) | finished tiles
+    DevState* st;
+    Ctl ctl;
+};
+
+// ---- low-latency (LL) ring AllReduce --------------------------------------------------------------
+
+struct LLArgs {
+    RankPtrs ptrs;
+    int p;
+    int G;                   // CTAs per rank
+    size_t n;                // elements per rank
+    size_t seg;              // ring segment, ceil(n / p)
+    uint32_t nslots;         // receive slots per rank: one per step that crosses a hop, 2p - 3
+    uint32_t tag;            // this call's tag of slot 0 (slot q carries tag + q)
+    float scale;
+    uint64_t timeout_ns;
+    unsigned long long* ll;  // [p][nslots][seg] 64-bit words: (tag << 32) | 32 data bits
+    Ctl ctl;
+};
+
+// ---- MoE dispatch and combine ------------------------------------------------------------------
+
+constexpr int kMoeTile = 256;         // assignments per counting tile (one per thread)
+constexpr int kMoeMaxExperts = 4096;  // the counting tile keeps one int per expert in shared memory
+constexpr int kMoeMaxTopk = 32;       // one lane per slot of a token
+
+struct MoeArgs {
+    const void* src[kMaxRanks];      // dispatch: token rows x_i [T][H]; combine: expert outputs y_j [rows][H]
+    const int32_t* idx[kMaxRanks];   // router output [T][k] expert ids
+    int32_t* pos[kMaxRanks];         // [T][k] row of each assignment at its owner (dispatch writes it, or null)
+    void* dst[kMaxRanks];            // dispatch: receive buffers [cap_rows][H]; combine: outputs [T][H]
+    const float* w[kMaxRanks];       // combine: gate weights [T][k]
+    const void* res[kMaxRanks];      // combine: residual [T][H] (has_res)
+    int p, k, E, E_loc;
+    int elem_bytes;
+    int has_res;
+    size_t T, H;                     // tokens per rank, elements per row
+    size_t A;                        // assignments per rank, T*k
+    size_t cap_rows;                 // rows of every receive buffer (dispatch) / expert-output buffer (combine)
+    uint32_t ntiles;                 // counting tiles per rank, ceil(A / kMoeTile)
+    int32_t* tile_hist;              // [p][ntiles][E] per-tile expert counts, then exclusive prefix over tiles
+    int32_t* rank_in_tile;           // [p][A] rank of an assignment among its tile's same-expert ones
+    int32_t* cnt;                    // [p][E] assignments from rank i to expert e
+    int32_t* base;                   // [p][E] first receive row of (rank i, expert e) at the expert's owner
+    long long* expert_counts_out;    // [p][E] or null
+    long long* recv_counts_out;      // [p] or null
+    DevState* st;
+    Ctl ctl;
+};
+
 // Launchers (each returns the launch error; grid sizes are decided inside).
 cudaError_t launch_butterfly(const ButterflyArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, int num_sms, cudaStream_t s);
@@ -138,5 +215,10 @@ int copy_num_variants();
 void copy_defaults(int kind, int* variant, int* order);
 cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 int ring_max_ctas(int num_sms);
+cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s);
+int ring_ll_max_ctas(int num_sms);
+cudaError_t launch_tree(const TreeArgs& a, int dtype, int op, int ctas, cudaStream_t s);
+cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStream_t s);
 
 }  // namespace simcomm

@@ -1,0 +1,177 @@
+// Low-latency (LL) ring AllReduce: the flag travels inside the data.
+//
+// "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives), §3.4
+// protocols: the Simple protocol moves data and then raises a separate flag behind a memory fence;
+// LL puts a flag beside every 4 bytes of data in one 8-byte store, so the receiver polls the data
+// itself and the sender needs no fence, at half the bandwidth; it serves small messages. (LL128 puts
+// 8 bytes of flag in every 128-byte line; it is not built here.)
+// Schedule and arithmetic are those of the ring AllReduce (§2.2, our reading of the garbled trace):
+// reduce-scatter step s = 1..p-1, rank r computes segment (r-1-s) mod p as received ⊕ own, partials
+// in fp32 for fp32/bf16 data, the owner scales for AVG and rounds once; all-gather step s = 1..p-1,
+// rank r receives segment (r-s) mod p from rank r-1. Its result therefore equals the ring path's bit
+// for bit.
+//
+// Execution: one cooperative launch (every CTA resident at once, so waiting on another CTA always
+// ends). CTAs [r*G, (r+1)*G) play rank r; thread t of rank r owns the same element positions of
+// every segment, and at every step needs only what thread t of rank r-1 produced the step before,
+// so threads never synchronise with each other. A value crosses a hop as one 64-bit store
+// (tag << 32 | value bits) into the receiver's slot for that step; the receiver polls those 64 bits
+// until the tag is this call's tag for that step (bounded, like every wait). The first hop reads the
+// predecessor's input in place.
+#include "common.cuh"
+
+namespace simcomm {
+
+constexpr int kLLThreads = 256;
+
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+
+// Wait until the slot holds this step's tag; returns its 32 data bits through *val.
+__device__ __forceinline__ bool ll_wait(const Ctl& ctl, const unsigned long long* w, uint32_t tag, uint64_t timeout_ns,
+                                        uint32_t* val) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0; it < kMaxSpin; ++it) {
+        const unsigned long long v = ld_relaxed_gpu_u64(w);
+        if (uint32_t(v >> 32) == tag) {
+            *val = uint32_t(v);
+            return true;
+        }
+        if (it == 0) {
+            t0 = globaltimer_ns();
+            continue;
+        }
+        if ((it & 255u) == 0u) {
+            if (status_failed(ctl)) return false;
+            const uint64_t now = globaltimer_ns();
+            if (now - t0 > timeout_ns) { raise_status(ctl, COLL_ERR_TIMEOUT); return false; }
+            if (abort_requested(ctl, now)) { raise_status(ctl, COLL_ERR_ABORTED); return false; }
+        }
+    }
+    raise_status(ctl, COLL_ERR_TIMEOUT);
+    return false;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t acc_bits(typename Elem<DT>::A v) {
+    if constexpr (DT == COLL_INT32) return uint32_t(v);
+    else return __float_as_uint(v);
+}
+template <int DT>
+__device__ __forceinline__ typename Elem<DT>::A acc_of(uint32_t b) {
+    if constexpr (DT == COLL_INT32) return int32_t(b);
+    else return __uint_as_float(b);
+}
+// The element's output bits (the rounded value) and back.
+template <int DT>
+__device__ __forceinline__ uint32_t out_bits(typename Elem<DT>::A v) {
+    if constexpr (DT == COLL_BF16) return uint32_t(float_to_bf16_bits(v));
+    else if constexpr (DT == COLL_FP32) return __float_as_uint(v);
+    else return uint32_t(v);
+}
+template <int DT>
+__device__ __forceinline__ void store_bits(void* base, size_t e, uint32_t b) {
+    if constexpr (DT == COLL_BF16) static_cast<uint16_t*>(base)[e] = uint16_t(b);
+    else static_cast<uint32_t*>(base)[e] = b;
+}
+
+template <int DT, int OP, bool SCALE>
+__global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ LLArgs a) {
+    using A = typename Elem<DT>::A;
+    const int p = a.p;
+    const int r = int(blockIdx.x) / a.G;
+    const int pred = (r + p - 1) % p;
+    const size_t i0 = size_t(int(blockIdx.x) % a.G) * kLLThreads + threadIdx.x;
+    const size_t stride = size_t(a.G) * kLLThreads;
+    unsigned long long* mine = a.ll + size_t(r) * a.nslots * a.seg;
+    unsigned long long* next = a.ll + size_t((r + 1) % p) * a.nslots * a.seg;
+    if (status_failed(a.ctl)) return;
+    auto seg_of = [&](int s) { return ((r - s) % p + p) % p; };  // rank r's segment at all-gather step s
+    // reduce-scatter
+    for (int s = 1; s <= p - 1; ++s) {
+        const int k = ((r - 1 - s) % p + p) % p;
+        for (size_t i = i0; i < a.seg; i += stride) {
+            const size_t e = size_t(k) * a.seg + i;
+            if (e >= a.n) break;
+            A w;
+            if (s == 1) {
+                w = load_elem<DT>(a.ptrs.send[pred], e);
+            } else {
+                uint32_t b;
+                if (!ll_wait(a.ctl, mine + size_t(s - 2) * a.seg + i, a.tag + uint32_t(s - 2), a.timeout_ns, &b)) return;
+                w = acc_of<DT>(b);
+            }
+            const A o = load_elem<DT>(a.ptrs.send[r], e);
+            if constexpr (DT == COLL_INT32) w = op_i<OP>(w, o);
+            else w = op_f<OP>(w, o);
+            if (s < p - 1) {
+                const uint32_t q = uint32_t(s - 1);  // the successor's slot for step s+1
+                st_relaxed_gpu_u64(next + size_t(q) * a.seg + i,
+                                   ((unsigned long long)(a.tag + q) << 32) | acc_bits<DT>(w));
+            } else {
+                if constexpr (SCALE) w = w * a.scale;
+                const uint32_t ob = out_bits<DT>(w);
+                store_bits<DT>(a.ptrs.recv[r], e, ob);
+                if (p > 1) {
+                    const uint32_t q = uint32_t(p - 2);  // the successor's slot for all-gather step 1
+                    st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, ((unsigned long long)(a.tag + q) << 32) | ob);
+                }
+            }
+        }
+    }
+    // all-gather
+    for (int s = 1; s <= p - 1; ++s) {
+        const int k = seg_of(s);
+        const uint32_t q = uint32_t(p - 2 + s - 1);
+        for (size_t i = i0; i < a.seg; i += stride) {
+            const size_t e = size_t(k) * a.seg + i;
+            if (e >= a.n) break;
+            uint32_t b;
+            if (!ll_wait(a.ctl, mine + size_t(q) * a.seg + i, a.tag + q, a.timeout_ns, &b)) return;
+            store_bits<DT>(a.ptrs.recv[r], e, b);
+            if (s < p - 1)
+                st_relaxed_gpu_u64(next + size_t(q + 1) * a.seg + i, ((unsigned long long)(a.tag + q + 1) << 32) | b);
+        }
+    }
+}
+
+template <int DT, int OP, bool SCALE>
+static cudaError_t launch_ll_typed(const LLArgs& a, cudaStream_t s) {
+    void* args[] = {const_cast<LLArgs*>(&a)};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE>),
+                                       dim3(unsigned(a.p * a.G)), dim3(kLLThreads), args, 0, s);
+}
+
+template <int DT>
+static cudaError_t launch_ll_dt(const LLArgs& a, int op, cudaStream_t s) {
+    switch (op) {
+        case COLL_SUM: return launch_ll_typed<DT, COLL_SUM, false>(a, s);
+        case COLL_MIN: return launch_ll_typed<DT, COLL_MIN, false>(a, s);
+        case COLL_MAX: return launch_ll_typed<DT, COLL_MAX, false>(a, s);
+        case COLL_AVG:
+            if constexpr (DT == COLL_INT32) return cudaErrorInvalidValue;
+            else return launch_ll_typed<DT, COLL_SUM, true>(a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s) {
+    switch (dtype) {
+        case COLL_INT32: return launch_ll_dt<COLL_INT32>(a, op, s);
+        case COLL_FP32: return launch_ll_dt<COLL_FP32>(a, op, s);
+        case COLL_BF16: return launch_ll_dt<COLL_BF16>(a, op, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// CTAs of the LL kernel that fit on the device at once (the cooperative-launch limit).
+int ring_ll_max_ctas(int num_sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_ring_ll<COLL_BF16, COLL_SUM, true>, kLLThreads, 0) !=
+            cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return num_sms * per_sm;
+}
+
+}  // namespace simcomm

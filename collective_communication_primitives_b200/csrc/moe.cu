@@ -1,0 +1,387 @@
+// MoE dispatch and combine: the steps on either side of the variable-split exchange, fused with it.
+//
+// Steps ("Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All",
+// charlestar.github.io/2026/08/20/gpu-collective-communication, sections "Ragged All-to-All" and
+// "Expert Parallel"): router output -> count assignments per destination -> exchange counts ->
+// prefix-sum offsets -> pack/permute -> variable-split All-to-All -> expert compute -> reverse
+// variable-split All-to-All -> unpermute and weighted combine (+ residual). One expert assignment
+// (token t of rank i picked by slot s) is one row of H elements.
+//
+// Layout rules (our reading): expert e lives on rank e / (E/p); rank i's rows for rank j arrive in
+// j's receive buffer after those of ranks 0..i-1, ordered by expert id, then token, then slot.
+//
+// Because all ranks share one memory, the pack and the exchange are one copy: every token row is
+// read once and written straight into the k receive rows its assignments own; the reverse
+// exchange, the unpermute and the weighted sum are likewise one pass that reads each token's k
+// expert-output rows where the experts left them. Kernels:
+//   k_moe_count   one CTA per (rank, tile of 256 assignments): validates expert ids, counts them per
+//                 expert, and ranks every assignment among the tile's assignments of the same expert
+//                 (warps in order; __match_any_sync groups equal experts inside a warp);
+//   k_moe_scan    one CTA per rank: exclusive prefix of the tile counts over tiles, per expert; the
+//                 last CTA to finish turns the per-rank totals into the count matrix c_ij, checks
+//                 every destination's capacity and computes each (rank, expert)'s first receive row;
+//   k_moe_dispatch_copy  one warp per token: the k destination rows (written to the routing map and
+//                 kept in shared memory for the warp), then 16/32-byte streaming loads of the token
+//                 row and k stores;
+//   k_moe_combine one warp per token: fp32 left fold in slot order (residual first), rounded once.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace simcomm {
+
+constexpr int kMoeThreads = kMoeTile;  // counting: one assignment per thread
+constexpr int kScanThreads = 1024;
+constexpr int kCopyThreads = 256;      // dispatch / combine: 8 warps, one token per warp at a time
+constexpr int kCopyUnroll = 4;         // packs in flight per lane
+
+__device__ __forceinline__ bool cta_failed(const Ctl& ctl) {
+    __shared__ int s_fail;
+    if (threadIdx.x == 0) s_fail = status_failed(ctl);
+    __syncthreads();
+    const bool f = s_fail != 0;
+    __syncthreads();
+    return f;
+}
+
+// ---- counting -----------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kMoeThreads) k_moe_count(const __grid_constant__ MoeArgs a) {
+    extern __shared__ int s_cnt[];  // [E]
+    if (cta_failed(a.ctl)) return;
+    const int i = blockIdx.y;
+    const uint32_t tile = blockIdx.x;
+    for (int e = threadIdx.x; e < a.E; e += kMoeThreads) s_cnt[e] = 0;
+    __syncthreads();
+
+    const size_t asg = size_t(tile) * kMoeTile + threadIdx.x;
+    const bool valid = asg < a.A;
+    int e = valid ? a.idx[i][asg] : -1;
+    if (valid && (e < 0 || e >= a.E)) {
+        raise_status(a.ctl, COLL_ERR_INVALID_ARG);
+        e = -1;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int rank = 0;
+    // warps take their turn in order so that ranks follow the assignment order
+    for (int w = 0; w < kMoeThreads / 32; ++w) {
+        if (warp == w) {
+            const unsigned same = __match_any_sync(0xffffffffu, e);
+            const int leader = __ffs(same) - 1;
+            int first = 0;
+            if (lane == leader && e >= 0) {
+                first = s_cnt[e];
+                s_cnt[e] = first + __popc(same);
+            }
+            first = __shfl_sync(0xffffffffu, first, leader);
+            rank = first + __popc(same & ((1u << lane) - 1u));
+        }
+        __syncthreads();
+    }
+    if (valid) a.rank_in_tile[size_t(i) * a.A + asg] = rank;
+    int32_t* hist = a.tile_hist + (size_t(i) * a.ntiles + tile) * a.E;
+    for (int x = threadIdx.x; x < a.E; x += kMoeThreads) hist[x] = s_cnt[x];
+}
+
+// ---- prefix sums and the count matrix ------------------------------------------------------------
+
+__global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant__ MoeArgs a) {
+    extern __shared__ int s_c[];  // [p][p] in the last CTA
+    __shared__ int s_last;
+    if (cta_failed(a.ctl)) return;
+    const int i = blockIdx.x;
+    constexpr int kBatch = 16;
+    // per expert: exclusive prefix of the tile counts over the tiles of rank i, and the total
+    for (int e = threadIdx.x; e < a.E; e += kScanThreads) {
+        int32_t* col = a.tile_hist + size_t(i) * a.ntiles * a.E + e;
+        int run = 0;
+        for (uint32_t t0 = 0; t0 < a.ntiles; t0 += kBatch) {
+            int v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) v[u] = (t0 + u < a.ntiles) ? col[size_t(t0 + u) * a.E] : 0;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                if (t0 + u < a.ntiles) {
+                    col[size_t(t0 + u) * a.E] = run;
+                    run += v[u];
+                }
+            }
+        }
+        a.cnt[size_t(i) * a.E + e] = run;
+    }
+    // the last CTA to finish sees every rank's totals
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&a.st->moe_ctr, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int p = a.p;
+    for (int ij = threadIdx.x; ij < p * p; ij += kScanThreads) {  // c_ij: rows from rank i to rank j
+        const int r = ij / p, j = ij % p;
+        int s = 0;
+        for (int x = j * a.E_loc; x < (j + 1) * a.E_loc; ++x) s += __ldcg(a.cnt + size_t(r) * a.E + x);
+        s_c[ij] = s;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < p; j += kScanThreads) {  // rows arriving at rank j, against its capacity
+        long long tot = 0;
+        for (int r = 0; r < p; ++r) tot += s_c[r * p + j];
+        if (size_t(tot) > a.cap_rows) raise_status(a.ctl, COLL_ERR_OVERFLOW);
+        if (a.recv_counts_out) a.recv_counts_out[j] = tot;
+    }
+    for (int ie = threadIdx.x; ie < p * a.E; ie += kScanThreads) {  // first row of (rank i, expert e)
+        const int r = ie / a.E, e = ie % a.E, j = e / a.E_loc;
+        int b = 0;
+        for (int q = 0; q < r; ++q) b += s_c[q * p + j];
+        for (int x = j * a.E_loc; x < e; ++x) b += __ldcg(a.cnt + size_t(r) * a.E + x);
+        a.base[ie] = b;
+        if (a.expert_counts_out) a.expert_counts_out[ie] = __ldcg(a.cnt + ie);
+    }
+    if (threadIdx.x == 0) a.st->moe_ctr = 0;
+}
+
+// ---- dispatch: permute/pack fused with the exchange ---------------------------------------------
+
+template <int W>
+__global__ void __launch_bounds__(kCopyThreads) k_moe_dispatch_copy(const __grid_constant__ MoeArgs a) {
+    __shared__ char* s_dst[kCopyThreads / 32][kMoeMaxTopk];  // per warp: the k destination rows of its token
+    if (cta_failed(a.ctl)) return;
+    const int i = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t row_bytes = a.H * size_t(a.elem_bytes);
+    const char* src = static_cast<const char*>(a.src[i]);
+    char* const* dsts = s_dst[warp];
+    for (size_t t = size_t(blockIdx.x) * (kCopyThreads / 32) + warp; t < a.T; t += size_t(gridDim.x) * (kCopyThreads / 32)) {
+        // lane s < k: the receive row of slot s
+        bool bad = false;
+        if (lane < a.k) {
+            const size_t asg = t * a.k + lane;
+            const int e = a.idx[i][asg];
+            const long long row = (long long)a.base[size_t(i) * a.E + e] +
+                                  a.tile_hist[(size_t(i) * a.ntiles + asg / kMoeTile) * a.E + e] +
+                                  a.rank_in_tile[size_t(i) * a.A + asg];
+            bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
+            if (bad) raise_status(a.ctl, COLL_ERR_INTERNAL);
+            if (a.pos[i]) a.pos[i][asg] = bad ? -1 : int32_t(row);
+            s_dst[warp][lane] = bad ? nullptr : static_cast<char*>(a.dst[e / a.E_loc]) + size_t(row) * row_bytes;
+        }
+        __syncwarp();
+        if (!__any_sync(0xffffffffu, bad)) {
+            const char* s_row = src + t * row_bytes;
+            if constexpr (W > 0) {
+                constexpr size_t kPack = size_t(W) * 4;
+                const size_t npk = row_bytes / kPack;
+                for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
+                    Words<W> v[kCopyUnroll];
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u)
+                        if (c0 + u * 32 < npk) v[u] = ld_stream_words<W>(s_row + (c0 + u * 32) * kPack);
+                    for (int s = 0; s < a.k; ++s) {
+                        char* d_row = dsts[s];
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u)
+                            if (c0 + u * 32 < npk) st_words<W>(d_row + (c0 + u * 32) * kPack, v[u]);
+                    }
+                }
+            } else {
+                // element-size-agnostic path: 2-byte units (every row is a whole number of them)
+                const size_t nu = row_bytes / 2;
+                for (size_t c0 = lane; c0 < nu; c0 += 32) {
+                    const uint16_t v = *reinterpret_cast<const uint16_t*>(s_row + c0 * 2);
+                    for (int s = 0; s < a.k; ++s) *reinterpret_cast<uint16_t*>(dsts[s] + c0 * 2) = v;
+                }
+            }
+        }
+        __syncwarp();  // the next token rewrites this warp's destination rows
+    }
+}
+
+// ---- combine: reverse exchange + unpermute + weighted sum ---------------------------------------
+
+template <int DT>
+__device__ __forceinline__ void unpack4(const uint4& v, float (&x)[16 / Elem<DT>::kBytes]) {
+    if constexpr (DT == COLL_BF16) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            x[2 * q] = bf16_bits_to_float(w[q] & 0xffffu);
+            x[2 * q + 1] = bf16_bits_to_float(w[q] >> 16);
+        }
+    } else {
+        x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+        x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ uint4 pack4(const float (&x)[16 / Elem<DT>::kBytes]) {
+    if constexpr (DT == COLL_BF16) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            w[q] = uint32_t(float_to_bf16_bits(x[2 * q])) | (uint32_t(float_to_bf16_bits(x[2 * q + 1])) << 16);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+    }
+}
+
+template <int DT>
+__device__ __forceinline__ float load_f(const void* base, size_t e) {
+    if constexpr (DT == COLL_BF16) return bf16_bits_to_float(static_cast<const uint16_t*>(base)[e]);
+    else return static_cast<const float*>(base)[e];
+}
+
+template <int DT>
+__device__ __forceinline__ void store_f(void* base, size_t e, float v) {
+    if constexpr (DT == COLL_BF16) static_cast<uint16_t*>(base)[e] = float_to_bf16_bits(v);
+    else static_cast<float*>(base)[e] = v;
+}
+
+// VEC: 16-byte packs (every row start 16-byte aligned); otherwise one element per lane.
+template <int DT, bool VEC>
+__global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_constant__ MoeArgs a) {
+    constexpr int L = 16 / Elem<DT>::kBytes;
+    __shared__ const char* s_y[kCopyThreads / 32][kMoeMaxTopk];  // per warp: the token's k expert-output rows
+    __shared__ float s_w[kCopyThreads / 32][kMoeMaxTopk];        // and their gate weights
+    if (cta_failed(a.ctl)) return;
+    const int i = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t d = size_t(Elem<DT>::kBytes);
+    const char* const* ys = s_y[warp];
+    const float* ws = s_w[warp];
+    for (size_t t = size_t(blockIdx.x) * (kCopyThreads / 32) + warp; t < a.T; t += size_t(gridDim.x) * (kCopyThreads / 32)) {
+        bool bad = false;
+        if (lane < a.k) {
+            const size_t asg = t * a.k + lane;
+            const int e = a.idx[i][asg];
+            const int r = a.pos[i][asg];
+            bad = e < 0 || e >= a.E || r < 0 || size_t(r) >= a.cap_rows;
+            s_y[warp][lane] = bad ? nullptr : static_cast<const char*>(a.src[e / a.E_loc]) + size_t(r) * a.H * d;
+            s_w[warp][lane] = a.w[i][asg];
+        }
+        __syncwarp();
+        if (__any_sync(0xffffffffu, bad)) {
+            if (lane == 0) raise_status(a.ctl, COLL_ERR_INVALID_ARG);
+            __syncwarp();
+            continue;
+        }
+        char* o_row = static_cast<char*>(a.dst[i]) + t * a.H * d;
+        const char* r_row = a.has_res ? static_cast<const char*>(a.res[i]) + t * a.H * d : nullptr;
+        if constexpr (VEC) {
+            const size_t npk = a.H / L;
+            for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
+                float acc[kCopyUnroll][L];
+                int s0 = 0;
+                if (r_row) {
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u)
+                        if (c0 + u * 32 < npk) unpack4<DT>(ld_stream_v4(r_row + (c0 + u * 32) * 16), acc[u]);
+                } else {
+                    const float w0 = ws[0];
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u) {
+                        if (c0 + u * 32 < npk) {
+                            unpack4<DT>(ld_stream_v4(ys[0] + (c0 + u * 32) * 16), acc[u]);
+#pragma unroll
+                            for (int l = 0; l < L; ++l) acc[u][l] = w0 * acc[u][l];
+                        }
+                    }
+                    s0 = 1;
+                }
+                for (int s = s0; s < a.k; ++s) {
+                    const char* y_row = ys[s];
+                    const float w = ws[s];
+                    uint4 v[kCopyUnroll];
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u)
+                        if (c0 + u * 32 < npk) v[u] = ld_stream_v4(y_row + (c0 + u * 32) * 16);
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u) {
+                        if (c0 + u * 32 < npk) {
+                            float y[L];
+                            unpack4<DT>(v[u], y);
+#pragma unroll
+                            for (int l = 0; l < L; ++l) acc[u][l] = acc[u][l] + w * y[l];
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kCopyUnroll; ++u)
+                    if (c0 + u * 32 < npk) st_v4(o_row + (c0 + u * 32) * 16, pack4<DT>(acc[u]));
+            }
+        } else {
+            for (size_t h = lane; h < a.H; h += 32) {
+                float acc;
+                int s0 = 0;
+                if (r_row) {
+                    acc = load_f<DT>(r_row, h);
+                } else {
+                    acc = ws[0] * load_f<DT>(ys[0], h);
+                    s0 = 1;
+                }
+                for (int s = s0; s < a.k; ++s) acc = acc + ws[s] * load_f<DT>(ys[s], h);
+                store_f<DT>(o_row, h, acc);
+            }
+        }
+        __syncwarp();  // the next token rewrites this warp's rows and weights
+    }
+}
+
+// ---- launch --------------------------------------------------------------------------------------
+
+static dim3 token_grid(const MoeArgs& a, int num_sms) {
+    const size_t warps_per_cta = kCopyThreads / 32;
+    const size_t want = (a.T + warps_per_cta - 1) / warps_per_cta;
+    const size_t per_rank = std::max<size_t>(1, size_t(num_sms) * 8 / size_t(a.p));
+    return dim3(unsigned(std::max<size_t>(1, std::min(want, per_rank))), unsigned(a.p), 1u);
+}
+
+cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
+    const size_t smem_count = size_t(a.E) * sizeof(int);
+    if (smem_count > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_moe_count, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_count));
+        if (e != cudaSuccess) return e;
+    }
+    k_moe_count<<<dim3(a.ntiles, unsigned(a.p), 1u), kMoeThreads, smem_count, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_moe_scan<<<unsigned(a.p), kScanThreads, size_t(a.p) * a.p * sizeof(int), s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 32-byte packs when every row start is 32-byte aligned, else 16-byte, else 2-byte units
+    const size_t row_bytes = a.H * size_t(a.elem_bytes);
+    bool al32 = row_bytes % 32 == 0, al16 = row_bytes % 16 == 0;
+    for (int r = 0; r < a.p; ++r) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a.src[r]), y = reinterpret_cast<uintptr_t>(a.dst[r]);
+        al32 = al32 && x % 32 == 0 && y % 32 == 0;
+        al16 = al16 && x % 16 == 0 && y % 16 == 0;
+    }
+    const dim3 grid = token_grid(a, num_sms);
+    if (al32) k_moe_dispatch_copy<8><<<grid, kCopyThreads, 0, s>>>(a);
+    else if (al16) k_moe_dispatch_copy<4><<<grid, kCopyThreads, 0, s>>>(a);
+    else k_moe_dispatch_copy<0><<<grid, kCopyThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStream_t s) {
+    const size_t row_bytes = a.H * size_t(a.elem_bytes);
+    bool vec = row_bytes % 16 == 0;
+    for (int r = 0; r < a.p; ++r) {
+        vec = vec && reinterpret_cast<uintptr_t>(a.src[r]) % 16 == 0 && reinterpret_cast<uintptr_t>(a.dst[r]) % 16 == 0;
+        if (a.has_res) vec = vec && reinterpret_cast<uintptr_t>(a.res[r]) % 16 == 0;
+    }
+    const dim3 grid = token_grid(a, num_sms);
+    if (dtype == COLL_BF16) {
+        if (vec) k_moe_combine<COLL_BF16, true><<<grid, kCopyThreads, 0, s>>>(a);
+        else k_moe_combine<COLL_BF16, false><<<grid, kCopyThreads, 0, s>>>(a);
+    } else if (dtype == COLL_FP32) {
+        if (vec) k_moe_combine<COLL_FP32, true><<<grid, kCopyThreads, 0, s>>>(a);
+        else k_moe_combine<COLL_FP32, false><<<grid, kCopyThreads, 0, s>>>(a);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace simcomm

@@ -16,7 +16,7 @@ STATUS = {0: "COLL_OK", 1: "COLL_ERR_INVALID_ARG", 2: "COLL_ERR_UNSUPPORTED", 3:
 OK, INVALID_ARG, UNSUPPORTED, CUDA, TIMEOUT, ABORTED, OVERFLOW, INTERNAL = range(8)
 DTYPES = {"int32": 0, "fp32": 1, "bf16": 2}
 OPS = {"sum": 0, "min": 1, "max": 2, "avg": 3}
-ALGOS = {"direct": 0, "ring": 1, "rd": 2, "hd": 3}
+ALGOS = {"direct": 0, "ring": 1, "rd": 2, "hd": 3, "tree": 4, "dbtree": 5, "ll": 6}
 
 _lib = None
 
@@ -75,8 +75,12 @@ def load_library(path=LIB_PATH):
     L.coll_scatter.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_gather.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_allreduce_ring_noalloc.argtypes = [i32, _Bufs, sz, i32, i32, vp, vp]
+    pp = ctypes.POINTER(ctypes.c_void_p)
+    L.coll_moe_dispatch.argtypes = [vp, pp, pp, sz, i32, sz, i32, i32, pp, sz, pp, vp, vp, vp]
+    L.coll_moe_combine.argtypes = [vp, pp, sz, pp, pp, pp, pp, sz, i32, sz, i32, i32, pp, vp]
     for name in ("coll_allreduce", "coll_reduce", "coll_broadcast", "coll_reduce_scatter", "coll_allgather",
-                 "coll_alltoall", "coll_alltoallv", "coll_scatter", "coll_gather", "coll_allreduce_ring_noalloc"):
+                 "coll_alltoall", "coll_alltoallv", "coll_scatter", "coll_gather", "coll_allreduce_ring_noalloc",
+                 "coll_moe_dispatch", "coll_moe_combine"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -239,6 +243,38 @@ class SimComm:
         self._check(self._L.coll_alltoallv(self._h, self._bufs(sends, recvs), ctypes.c_void_p(_ptr(counts)), sc, rc,
                                            self._resolve(dtype, list(sends) + list(recvs)), ALGOS[algo], _stream(stream),
                                            ctypes.c_void_p(_ptr(recv_counts)) if recv_counts is not None else None))
+
+    # -- MoE dispatch / combine ----------------------------------------------------------------------
+    def _parr(self, tensors):
+        """HOST array of p device pointers (None when tensors is None)."""
+        if tensors is None:
+            return None
+        a = (ctypes.c_void_p * self.p)(*[_ptr(t) for t in tensors])
+        self._keep_moe = getattr(self, "_keep_moe", [])[-16:] + [a]
+        return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+
+    def moe_dispatch(self, x, topk_idx, experts, recv, route_pos=None, expert_counts=None, recv_counts=None,
+                     dtype=None, stream=None):
+        """x[i]: [T][H] token rows; topk_idx[i]: [T][k] int32 expert ids; recv[j]: [cap][H]. Optional
+        outputs: route_pos[i] [T][k] int32, expert_counts [p][E] int64, recv_counts [p] int64."""
+        T, k = topk_idx[0].shape
+        H = x[0].shape[1] if x[0].dim() == 2 else x[0].numel() // max(T, 1)
+        cap = recv[0].shape[0]
+        self._check(self._L.coll_moe_dispatch(
+            self._h, self._parr(x), self._parr(topk_idx), T, k, H, int(experts),
+            self._resolve(dtype, list(x) + list(recv)), self._parr(recv), cap, self._parr(route_pos),
+            ctypes.c_void_p(_ptr(expert_counts)) if expert_counts is not None else None,
+            ctypes.c_void_p(_ptr(recv_counts)) if recv_counts is not None else None, _stream(stream)))
+
+    def moe_combine(self, y, topk_idx, route_pos, topk_weight, experts, out, residual=None, dtype=None,
+                    stream=None):
+        """out[i][t] = residual[i][t] + Σ_s w[i][t][s] * y[owner][route_pos[i][t][s]] (fp32, slot order)."""
+        T, k = topk_idx[0].shape
+        H = out[0].shape[1]
+        self._check(self._L.coll_moe_combine(
+            self._h, self._parr(y), y[0].shape[0], self._parr(topk_idx), self._parr(route_pos),
+            self._parr(topk_weight), self._parr(residual), T, k, H, int(experts),
+            self._resolve(dtype, list(y) + list(out)), self._parr(out), _stream(stream)))
 
 
 def allreduce_ring_noalloc(sends, recvs, op="sum", n=None, dtype=None, status=None, stream=None):

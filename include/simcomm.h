@@ -51,6 +51,7 @@
 #define SIMCOMM_H
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -80,8 +81,21 @@ typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_
  * RD:     recursive doubling ([Atlas] §2.3): log2 p exchange-and-reduce steps. AllReduce only,
  *         p a power of two (else COLL_ERR_UNSUPPORTED).
  * HD:     recursive halving-doubling ([Atlas] §2.3): a halving reduce-scatter then a doubling
- *         all-gather, 2 log2 p steps. AllReduce only, p a power of two. */
-typedef enum { COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3 } coll_algo_t;
+ *         all-gather, 2 log2 p steps. AllReduce only, p a power of two.
+ * TREE:   reduce up a binary tree to its root, then broadcast down ([Primer] "Tree AllReduce 为什么
+ *         更适合延迟敏感区间"): heap numbering, position m has children 2m+1 and 2m+2, rank m at
+ *         position m; a position folds (own ⊕ left) ⊕ right in fp32; chunk-pipelined. AllReduce only.
+ * DBTREE: double binary tree ([Atlas] §2.4): elements [0, ceil(n/2)) on the tree above, the rest on
+ *         its mirror (rank p-1-m at position m). AllReduce only.
+ * RING_LL: the ring AllReduce on the low-latency protocol of [Atlas] §3.4 (every 4 data bytes travel
+ *         with a 4-byte flag in one 8-byte store; no separate flags or fences): same schedule and
+ *         rounding as RING, so the same result bit for bit. AllReduce only, small messages: the
+ *         communicator keeps p * (2p-3) * ceil(n/p) * 8 bytes of receive slots, at most 256 MiB
+ *         (else COLL_ERR_UNSUPPORTED). */
+typedef enum {
+    COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3, COLL_ALGO_TREE = 4, COLL_ALGO_DBTREE = 5,
+    COLL_ALGO_RING_LL = 6
+} coll_algo_t;
 
 typedef struct {
     const void* const* send; /* host array [p] of device pointers (inputs) */
@@ -206,6 +220,58 @@ coll_status_t coll_gather(sim_comm_t comm, coll_bufs_t bufs, size_t n, coll_dtyp
 coll_status_t coll_alltoallv(sim_comm_t comm, coll_bufs_t bufs, const long long* counts_dev,
                              const long long* send_cap, const long long* recv_cap, coll_dtype_t dtype,
                              coll_algo_t algo, coll_stream_t stream, long long* recv_counts_dev);
+
+/* ---- MoE dispatch and combine ---------------------------------------------------------------- */
+
+/* The steps on either side of the All-to-Allv in an expert-parallel MoE layer ([Primer] "Ragged
+ * All-to-All：MoE 的真实输入通常不等长": router output -> count per destination -> exchange
+ * counts -> prefix-sum offsets -> pack/permute -> variable-split exchange -> experts -> reverse
+ * exchange -> unpermute/combine; [Primer] "Expert Parallel": one row travels per expert
+ * assignment, and the combine weights the returned rows and adds the residual). Rules (our
+ * reading): E experts, E a multiple of p, expert e lives on rank e / (E/p); every rank routes the
+ * same number of tokens T, each to k experts (router output idx[t][s], t < T, s < k); rows hold H
+ * elements, row-major, contiguous.
+ *
+ * Dispatch: counting, prefix sums, packing and the exchange in one call. Rank i's assignments are
+ * packed by expert id, ties in token order then slot order; rank j receives [rows from rank 0 |
+ * rows from rank 1 | ...], i.e. the All-to-Allv layout, every source block grouped by expert:
+ *   x            HOST array of p DEVICE pointers, x[i] = [T][H] token rows of rank i.
+ *   topk_idx     HOST array of p DEVICE pointers, [T][k] int32 expert ids in [0, E).
+ *   recv         HOST array of p DEVICE pointers, [recv_cap_rows][H]; rows past the received
+ *                count are left untouched.
+ *   route_pos    HOST array of p DEVICE pointers [T][k] int32, or NULL: the row of recv[e/(E/p)]
+ *                that received assignment (t, s), the routing map the combine needs.
+ *   expert_counts_dev  DEVICE int64 [p][E] or NULL: assignments from rank i to expert e (expert e's
+ *                rows from rank i follow those of the owner's lower experts inside rank i's block).
+ *   recv_counts_dev    DEVICE int64 [p] or NULL: rows rank j received.
+ * Any dtype (rows are copied bit for bit). Synchronous errors: k not in [1, 32], E not a multiple
+ * of p in [p, 4096], H = 0, T*k or recv_cap_rows beyond int32, null or misaligned pointers,
+ * overlapping outputs or an output overlapping an input. Asynchronous errors: an expert id outside
+ * [0, E) -> COLL_ERR_INVALID_ARG, a rank that would receive more than recv_cap_rows rows ->
+ * COLL_ERR_OVERFLOW; in both cases no row is copied. The scratch for counting is owned by the
+ * communicator. T = 0 only zeroes the count outputs. */
+coll_status_t coll_moe_dispatch(sim_comm_t comm, const void* const* x, const int32_t* const* topk_idx, size_t tokens,
+                                int k, size_t hidden, int experts, coll_dtype_t dtype, void* const* recv,
+                                size_t recv_cap_rows, int32_t* const* route_pos, long long* expert_counts_dev,
+                                long long* recv_counts_dev, coll_stream_t stream);
+
+/* Combine: reverse exchange, unpermute and weighted sum in one call:
+ *   out[i][t] = residual[i][t] + Σ_{s<k} w[i][t][s] * y[e/(E/p)][route_pos[i][t][s]],  e = idx[i][t][s]
+ * accumulated in fp32 in slot order (the residual first; without a residual the sum starts at the
+ * slot-0 product), every product and sum rounded to fp32, then rounded once to the row type.
+ *   y            HOST array of p DEVICE pointers, [y_rows][H]: expert outputs in the dispatch's
+ *                receive layout (e.g. recv after the experts ran in place).
+ *   topk_idx, route_pos  as given to and returned by coll_moe_dispatch.
+ *   topk_weight  HOST array of p DEVICE pointers, [T][k] fp32 gate weights.
+ *   residual     HOST array of p DEVICE pointers [T][H], or NULL (no residual term); residual[i]
+ *                may equal out[i] (in place).
+ *   out          HOST array of p DEVICE pointers [T][H].
+ * dtype fp32 or bf16 (int32 -> COLL_ERR_UNSUPPORTED). An expert id outside [0, E) or a route_pos
+ * outside [0, y_rows) is reported asynchronously as COLL_ERR_INVALID_ARG (that token is skipped). */
+coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_rows, const int32_t* const* topk_idx,
+                               const int32_t* const* route_pos, const float* const* topk_weight,
+                               const void* const* residual, size_t tokens, int k, size_t hidden, int experts,
+                               coll_dtype_t dtype, void* const* out, coll_stream_t stream);
 
 /* ---- no-allocation variant ------------------------------------------------------------------ */
 
