@@ -34,7 +34,9 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of a row's kernel, with the
 # per-rank element count of that capture; scaled to the bench's size by elements moved. Empty
 # until a capture of the current build is taken.
-NCU_TRAFFIC = {}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a row's kernel, from an
+# ncu capture of the current build, and the per-rank element count it was captured at.
+NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_195_191_040 + 1_420_263_424, 26_214_400)}
 SPACER_CYCLES = 4_000_000  # ~2 ms of a spinning kernel ahead of a timed region
 
 
@@ -57,6 +59,7 @@ def parse():
     ap.add_argument("--moe", action="store_true",
                     help="time only the MoE dispatch and combine on the MoE workload (one GPU)")
     ap.add_argument("--no-moe", action="store_true", help="leave the MoE block out of the step's line")
+    ap.add_argument("--moe-tokens", type=int, default=8192, help="tokens per rank of the MoE layer (--moe)")
     return ap.parse_args()
 
 
@@ -130,6 +133,21 @@ class Workload:
         self.v_recv = [torch.empty(int(self.counts_host[:, j].sum()), dtype=torch.float32, device=device)
                        for j in range(P)]
         self.rows = rows
+
+    def twin(self, device):
+        """A second set of the buffers a host copy touches (the inputs and the AllReduce outputs), the
+        rest shared, so that one step's copies can overlap another step's kernels."""
+        import copy
+
+        import torch
+        t = copy.copy(self)
+        t.x32 = [torch.empty_like(x) for x in self.x32]
+        t.x16 = [torch.empty_like(x) for x in self.x16]
+        t.ar32 = [torch.empty_like(x) for x in self.ar32]
+        t.ar16 = [torch.empty_like(x) for x in self.ar16]
+        t.shards = [x[:self.m] for x in t.x32]
+        t.v_send = [x[:int(self.counts_host[i].sum())] for i, x in enumerate(t.x32)]
+        return t
 
 
 def build_step(comm, wl):
@@ -259,30 +277,57 @@ def time_device(ops, steps, warmup, stream):
     return total_ms, per_op
 
 
-def time_e2e(comm, wl, ops, steps, warmup, stream):
-    """Same step through the public API with host buffers: pinned inputs copied in, the step run,
-    both AllReduce results copied out, all inside the timed region."""
+def time_e2e(comm, wl, make_ops, steps, warmup, stream, device):
+    """The step through the public API with host buffers: every step copies all its inputs in from
+    pinned host memory and both AllReduce results out, inside the timed region. Two buffer sets make
+    a 2-deep pipeline: step k+1's host-to-device copies (one stream) and step k-1's device-to-host
+    reads (another stream) overlap step k's kernels, ordered by events."""
     import torch
+    sets = [wl, wl.twin(device)]
+    ops = [make_ops(w) for w in sets]
     out_host32 = [torch.empty(wl.n, dtype=torch.float32).pin_memory() for _ in range(P)]
     out_host16 = [torch.empty(wl.n, dtype=torch.bfloat16).pin_memory() for _ in range(P)]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_h2d = [torch.cuda.Event() for _ in sets]
+    ev_comp = [torch.cuda.Event() for _ in sets]
+    ev_d2h = [torch.cuda.Event() for _ in sets]
+    used = [False, False]
 
-    def one():
-        for r in range(P):
-            wl.x32[r].copy_(wl.host_f32[r], non_blocking=True)
-            wl.x16[r].copy_(wl.host_b16[r], non_blocking=True)
-        for op in ops:
+    def step(k):
+        b = k % 2
+        w = sets[b]
+        with torch.cuda.stream(h2d_s):
+            if used[b]:
+                h2d_s.wait_event(ev_comp[b])  # the kernels that read these inputs are done
+            for r in range(P):
+                w.x32[r].copy_(wl.host_f32[r], non_blocking=True)
+                w.x16[r].copy_(wl.host_b16[r], non_blocking=True)
+            ev_h2d[b].record(h2d_s)
+        stream.wait_event(ev_h2d[b])
+        if used[b]:
+            stream.wait_event(ev_d2h[b])  # the previous results in these buffers were read back
+        for op in ops[b]:
             op[2]()
-        for r in range(P):
-            out_host32[r].copy_(wl.ar32[r], non_blocking=True)
-            out_host16[r].copy_(wl.ar16[r], non_blocking=True)
+        ev_comp[b].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_comp[b])
+            for r in range(P):
+                out_host32[r].copy_(w.ar32[r], non_blocking=True)
+                out_host16[r].copy_(w.ar16[r], non_blocking=True)
+            ev_d2h[b].record(d2h_s)
+        used[b] = True
 
-    for _ in range(warmup):
-        one()
+    for k in range(warmup):
+        step(k)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for _ in range(steps):
-        one()
+    h2d_s.wait_event(start)
+    for k in range(warmup, warmup + steps):
+        step(k)
+    for b in range(2):
+        if used[b]:
+            stream.wait_event(ev_d2h[b])
     end.record(stream)
     torch.cuda.synchronize()
     h2d = P * wl.n * (4 + 2)
@@ -300,12 +345,12 @@ class MoeWorkload:
     """p ranks x 8192 tokens, top-2 of 64 experts with Zipf(1.1) popularity, 4096-wide bf16 rows;
     every receive buffer holds p*T*k rows (the worst case: all assignments to one rank)."""
 
-    def __init__(self, device):
+    def __init__(self, device, tokens=None):
         import numpy as np
         import torch
 
         from collective_communication_primitives_b200 import synth as S
-        p, T, k, E, H = P, MOE["tokens"], MOE["topk"], MOE["experts"], MOE["hidden"]
+        p, T, k, E, H = P, tokens or MOE["tokens"], MOE["topk"], MOE["experts"], MOE["hidden"]
         self.p, self.T, self.k, self.E, self.H = p, T, k, E, H
         ids = S.moe_routes(p, T, E, k, MOE["zipf_s"], 0)
         ws = S.moe_gate_weights(p, T, k, 0)
@@ -362,8 +407,11 @@ def moe_main(args):
     from collective_communication_primitives_b200 import simcomm as SC
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
-    mw = MoeWorkload("cuda:0")
+    mw = MoeWorkload("cuda:0", args.moe_tokens)
     comm = SC.SimComm(P)
+    for kv in args.option:
+        k, v = kv.split("=", 1)
+        comm.set_option(k, int(v))
     hbm, peak_kind = peaks()
     ops = moe_ops(comm, mw)
     launches0 = comm.launch_count()
@@ -380,7 +428,8 @@ def moe_main(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 rows, fp32 combine", "data": "synthetic",
            "config": {"workload": f"MoE dispatch + combine, p={P} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} "
-                                  f"experts (Zipf 1.1), {mw.H}-wide bf16 rows", "l2": "inputs larger than L2"},
+                                  f"experts (Zipf 1.1), {mw.H}-wide bf16 rows", "l2": "inputs larger than L2",
+                      "options": args.option},
            "roofline": {"bound": "hbm", "kernel": f"{name} ({kernel})", "achieved": round(achieved, 1), "peak": hbm,
                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": peak_kind, "traffic": None,
                         "algorithmic_bytes_per_launch": int(kb), "ms_per_launch": round(per_op[i_dom], 4)},
@@ -633,10 +682,12 @@ def main():
     for kv in args.option:
         k, v = kv.split("=", 1)
         comm.set_option(k, int(v))
-    ops = build_step(comm, wl)
-    if args.ops:
-        keys = [k for k in args.ops.split(",") if k]
-        ops = [o for o in ops if any(k in o[0] for k in keys)]
+    keys = [k for k in args.ops.split(",") if k]
+
+    def make_ops(w):
+        return [o for o in build_step(comm, w) if not keys or any(k in o[0] for k in keys)]
+
+    ops = make_ops(wl)
     eff_per_step = sum(o[3] for o in ops)
 
     if world > 1:
@@ -654,12 +705,14 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = time_e2e(comm, wl, ops, max(3, args.steps // 4), 1, stream)
+        e_ms, h2d, d2h = time_e2e(comm, wl, make_ops, max(3, args.steps // 4), 1, stream, device)
         e_steps = max(3, args.steps // 4)
         if world > 1:
             e_ms = reduce_max(e_ms, device)
         e2e = {"value": job_gbps(world, eff_per_step, e_ms / e_steps), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / e_steps, 3),
+               "pipeline": "2 buffer sets: step k+1's host-to-device copies and step k-1's device-to-host "
+                           "reads overlap step k's kernels"}
 
     hbm, peak_kind = peaks()
     ms_per_step = total_ms / args.steps
@@ -670,9 +723,11 @@ def main():
                              "kernel_GBps": round(kb / (ms / 1e3) / 1e9, 1),
                              "frac_of_measured_peak": round(kb / (ms / 1e3) / 1e9 / hbm, 4)}
     # The dominant kernel: each row is one launch of one kernel, so the row with the largest share
-    # of the step's device time names it. achieved = that kernel's algorithmic bytes per launch
-    # (its byte model: the minimum for direct rows, the ring schedule's hop traffic for ring rows)
-    # over its average launch time measured above with CUDA events.
+    # of the step's device time names it. achieved = that kernel's algorithmic bytes per launch (its
+    # byte model: the minimum for direct rows; for ring rows the schedule's hop traffic, every hop
+    # reading a partial and an input and writing a partial or an output, which ncu's DRAM counters
+    # confirm at this size) over its average launch time measured above with CUDA events. The
+    # collective's minimum bytes (any schedule) are reported beside it.
     i_dom = max(range(len(ops)), key=lambda i: per_op[i])
     name, kernel, _, eff, kb = ops[i_dom]
     d_ms = per_op[i_dom]
@@ -684,6 +739,7 @@ def main():
     roofline = {"bound": "hbm", "kernel": f"{name} ({kernel})", "achieved": round(achieved, 1), "peak": hbm,
                 "unit": "GB/s", "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
                 "traffic": traffic, "algorithmic_bytes_per_launch": int(kb),
+                "minimum_bytes_per_launch": int(eff),
                 "share_of_step": round(d_ms / sum(per_op), 4), "ms_per_launch": round(d_ms, 4)}
     # The four direct kernels the throughput target names (>= 80% of the ~8 TB/s nominal peak).
     star = {}

@@ -46,6 +46,7 @@ struct sim_comm {
     long long direct_pack = 0;
     long long direct_ctas_per_sm = 16;
     long long l2_hint = 0;
+    long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
 };
@@ -575,6 +576,9 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     } else if (k == "direct_ctas_per_sm") {
         if (value < 1 || value > 32) return fail(COLL_ERR_INVALID_ARG, "direct_ctas_per_sm must be in [1, 32]");
         c->direct_ctas_per_sm = value;
+    } else if (k == "moe_tma") {
+        if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "moe_tma must be 0 or 1");
+        c->moe_tma = value;
     } else {
         return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     }
@@ -673,6 +677,7 @@ coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* valu
     else if (k == "direct_pack") *value = c->direct_pack;
     else if (k == "l2_hint") *value = c->l2_hint;
     else if (k == "direct_ctas_per_sm") *value = c->direct_ctas_per_sm;
+    else if (k == "moe_tma") *value = c->moe_tma;
     else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     return COLL_OK;
 }
@@ -1093,6 +1098,8 @@ coll_status_t coll_moe_dispatch(sim_comm_t c, const void* const* x, const int32_
     a.base = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + b_pe);
     a.expert_counts_out = expert_counts_dev;
     a.recv_counts_out = recv_counts_dev;
+    a.tma = int(c->moe_tma);
+    a.timeout_ns = uint64_t(c->timeout_ns);
     a.st = c->dstate;
     a.ctl = make_ctl(c);
     cudaError_t e = launch_moe_dispatch(a, c->num_sms, s);

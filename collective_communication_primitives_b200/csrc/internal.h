@@ -203,6 +203,8 @@ struct MoeArgs {
     int32_t* base;                   // [p][E] first receive row of (rank i, expert e) at the expert's owner
     long long* expert_counts_out;    // [p][E] or null
     long long* recv_counts_out;      // [p] or null
+    int tma;                         // dispatch copy: 1 bulk copies through shared memory, 0 loads/stores
+    uint64_t timeout_ns;
     DevState* st;
     Ctl ctl;
 };

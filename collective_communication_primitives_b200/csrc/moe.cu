@@ -34,6 +34,7 @@ constexpr int kMoeThreads = kMoeTile;  // counting: one assignment per thread
 constexpr int kScanThreads = 1024;
 constexpr int kCopyThreads = 256;      // dispatch / combine: 8 warps, one token per warp at a time
 constexpr int kCopyUnroll = 4;         // packs in flight per lane
+constexpr int kCombineRegSlots = 2;    // combine: slots whose rows are loaded together with the residual
 
 __device__ __forceinline__ bool cta_failed(const Ctl& ctl) {
     __shared__ int s_fail;
@@ -143,20 +144,34 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
 
 // ---- dispatch: permute/pack fused with the exchange ---------------------------------------------
 
+// Token batches: lane b*kslot + s holds slot s of the batch's b-th token (kslot = k rounded up to a
+// power of two, so a batch holds 32/kslot tokens); the routes of a whole batch are looked up with one
+// round of loads, then its tokens are copied one after another.
+__device__ __forceinline__ int slot_width(int k) {
+    int w = 1;
+    while (w < k) w <<= 1;
+    return w;
+}
+
 template <int W>
 __global__ void __launch_bounds__(kCopyThreads) k_moe_dispatch_copy(const __grid_constant__ MoeArgs a) {
-    __shared__ char* s_dst[kCopyThreads / 32][kMoeMaxTopk];  // per warp: the k destination rows of its token
+    __shared__ char* s_dst[kCopyThreads / 32][32];  // per warp: destination row of (batch token, slot)
     if (cta_failed(a.ctl)) return;
     const int i = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t row_bytes = a.H * size_t(a.elem_bytes);
     const char* src = static_cast<const char*>(a.src[i]);
     char* const* dsts = s_dst[warp];
-    for (size_t t = size_t(blockIdx.x) * (kCopyThreads / 32) + warp; t < a.T; t += size_t(gridDim.x) * (kCopyThreads / 32)) {
-        // lane s < k: the receive row of slot s
+    const int kslot = slot_width(a.k), per_batch = 32 / kslot;
+    const int my_b = lane / kslot, my_s = lane % kslot;
+    // this warp's tokens: first, first + stride, first + 2 * stride, ...; a batch takes per_batch of them
+    const size_t first = size_t(blockIdx.x) * (kCopyThreads / 32) + warp;
+    const size_t stride = size_t(gridDim.x) * (kCopyThreads / 32);
+    for (size_t t0 = first; t0 < a.T; t0 += stride * per_batch) {
+        const size_t my_t = t0 + size_t(my_b) * stride;
         bool bad = false;
-        if (lane < a.k) {
-            const size_t asg = t * a.k + lane;
+        if (my_s < a.k && my_t < a.T) {
+            const size_t asg = my_t * a.k + my_s;
             const int e = a.idx[i][asg];
             const long long row = (long long)a.base[size_t(i) * a.E + e] +
                                   a.tile_hist[(size_t(i) * a.ntiles + asg / kMoeTile) * a.E + e] +
@@ -168,33 +183,143 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_dispatch_copy(const __grid
         }
         __syncwarp();
         if (!__any_sync(0xffffffffu, bad)) {
-            const char* s_row = src + t * row_bytes;
-            if constexpr (W > 0) {
-                constexpr size_t kPack = size_t(W) * 4;
-                const size_t npk = row_bytes / kPack;
-                for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
-                    Words<W> v[kCopyUnroll];
-#pragma unroll
-                    for (int u = 0; u < kCopyUnroll; ++u)
-                        if (c0 + u * 32 < npk) v[u] = ld_stream_words<W>(s_row + (c0 + u * 32) * kPack);
-                    for (int s = 0; s < a.k; ++s) {
-                        char* d_row = dsts[s];
+            for (int b = 0; b < per_batch; ++b) {
+                const size_t t = t0 + size_t(b) * stride;
+                if (t >= a.T) break;
+                const char* s_row = src + t * row_bytes;
+                char* const* d = dsts + b * kslot;
+                if constexpr (W > 0) {
+                    constexpr size_t kPack = size_t(W) * 4;
+                    const size_t npk = row_bytes / kPack;
+                    for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
+                        Words<W> v[kCopyUnroll];
 #pragma unroll
                         for (int u = 0; u < kCopyUnroll; ++u)
-                            if (c0 + u * 32 < npk) st_words<W>(d_row + (c0 + u * 32) * kPack, v[u]);
+                            if (c0 + u * 32 < npk) v[u] = ld_stream_words<W>(s_row + (c0 + u * 32) * kPack);
+                        for (int s = 0; s < a.k; ++s) {
+                            char* d_row = d[s];
+#pragma unroll
+                            for (int u = 0; u < kCopyUnroll; ++u)
+                                if (c0 + u * 32 < npk) st_words<W>(d_row + (c0 + u * 32) * kPack, v[u]);
+                        }
                     }
-                }
-            } else {
-                // element-size-agnostic path: 2-byte units (every row is a whole number of them)
-                const size_t nu = row_bytes / 2;
-                for (size_t c0 = lane; c0 < nu; c0 += 32) {
-                    const uint16_t v = *reinterpret_cast<const uint16_t*>(s_row + c0 * 2);
-                    for (int s = 0; s < a.k; ++s) *reinterpret_cast<uint16_t*>(dsts[s] + c0 * 2) = v;
+                } else {
+                    // element-size-agnostic path: 2-byte units (every row is a whole number of them)
+                    const size_t nu = row_bytes / 2;
+                    for (size_t c0 = lane; c0 < nu; c0 += 32) {
+                        const uint16_t v = *reinterpret_cast<const uint16_t*>(s_row + c0 * 2);
+                        for (int s = 0; s < a.k; ++s) *reinterpret_cast<uint16_t*>(d[s] + c0 * 2) = v;
+                    }
                 }
             }
         }
-        __syncwarp();  // the next token rewrites this warp's destination rows
+        __syncwarp();  // the next batch rewrites this warp's destination rows
     }
+}
+
+// Bulk-copy variant: one warp per CTA; a task is one tile (at most kMoeTmaTile bytes) of one token
+// row, loaded into shared memory by one bulk copy completing on an mbarrier and stored by one bulk
+// copy per slot, with kMoeTmaStages tiles in flight. Needs rows of whole 16-byte units at 16-byte
+// aligned bases (then every row start is aligned). No multicast form of any bulk copy is used.
+constexpr int kMoeTmaStages = 8;
+constexpr uint32_t kMoeTmaTile = 8192;
+constexpr int kMoeTmaCtasPerSm = 3;
+
+__global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__ MoeArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ char* s_dst[kMoeMaxTopk];
+    const int lane = threadIdx.x;
+    if (status_failed(a.ctl)) return;  // one word read by every lane: the whole warp leaves together
+    unsigned char* stages = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kMoeTmaStages) * kMoeTmaTile);
+    const size_t row_bytes = a.H * size_t(a.elem_bytes);
+    const size_t nq = (row_bytes + kMoeTmaTile - 1) / kMoeTmaTile;
+    const size_t total = size_t(a.p) * a.T * nq;
+    if (lane == 0) {
+        for (int s = 0; s < kMoeTmaStages; ++s) mbar_init(&bars[s], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    __syncwarp();
+    const size_t my_n = (total > blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    uint32_t phase = 0;  // bit s: parity of the next completion of stage s
+    size_t issued = 0;   // tasks whose load has been issued
+    struct Task { int i; size_t t, off; uint32_t bytes; };
+    auto task_of = [&](size_t k) {
+        const size_t u = blockIdx.x + k * gridDim.x;
+        const size_t tok = u / nq;
+        Task x;
+        x.i = int(tok / a.T);
+        x.t = tok % a.T;
+        x.off = (u % nq) * kMoeTmaTile;
+        x.bytes = uint32_t(min(size_t(kMoeTmaTile), row_bytes - x.off));
+        return x;
+    };
+    auto issue = [&](size_t k) {
+        issued = k + 1;
+        if (lane != 0) return;
+        const Task x = task_of(k);
+        const int st = int(k % kMoeTmaStages);
+        mbar_arrive_expect_tx(&bars[st], x.bytes);
+        bulk_g2s(stages + size_t(st) * kMoeTmaTile, static_cast<const char*>(a.src[x.i]) + x.t * row_bytes + x.off,
+                 x.bytes, &bars[st]);
+    };
+    auto wait_stage = [&](size_t k) -> bool {  // the load of task k has landed
+        const int st = int(k % kMoeTmaStages);
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(a.ctl, &bars[st], (phase >> st) & 1u, a.timeout_ns);
+        phase ^= (1u << st);
+        return __shfl_sync(0xffffffffu, ok, 0);
+    };
+    // 0: done; 1: stop (a row out of range: nothing stored); 2: stop at once (a load never landed)
+    auto consume = [&](size_t k) -> int {
+        const Task x = task_of(k);
+        bool bad = false;
+        if (lane < a.k) {  // lane s: the receive row of slot s (written to the routing map once per row)
+            const size_t asg = x.t * a.k + lane;
+            const int e = a.idx[x.i][asg];
+            const long long row = (long long)a.base[size_t(x.i) * a.E + e] +
+                                  a.tile_hist[(size_t(x.i) * a.ntiles + asg / kMoeTile) * a.E + e] +
+                                  a.rank_in_tile[size_t(x.i) * a.A + asg];
+            bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
+            if (x.off == 0 && a.pos[x.i]) a.pos[x.i][asg] = bad ? -1 : int32_t(row);
+            s_dst[lane] = bad ? nullptr : static_cast<char*>(a.dst[e / a.E_loc]) + size_t(row) * row_bytes;
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        __syncwarp();
+        if (!wait_stage(k)) return 2;
+        if (bad) {
+            if (lane == 0) raise_status(a.ctl, COLL_ERR_INTERNAL);
+            return 1;
+        }
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            const unsigned char* tile = stages + size_t(k % kMoeTmaStages) * kMoeTmaTile;
+            for (int s = 0; s < a.k; ++s) bulk_s2g(s_dst[s] + x.off, tile, x.bytes);
+            bulk_commit();
+        }
+        __syncwarp();  // s_dst is rewritten by the next task
+        return 0;
+    };
+    const size_t pre = my_n < size_t(kMoeTmaStages - 1) ? my_n : size_t(kMoeTmaStages - 1);
+    for (size_t k = 0; k < pre; ++k) issue(k);
+    for (size_t k = 0; k < my_n; ++k) {
+        const size_t kk = k + kMoeTmaStages - 1;
+        if (kk < my_n) {
+            // stage kk % kMoeTmaStages last held task k-1, whose stores are the newest group
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            issue(kk);
+        }
+        const int r = consume(k);
+        if (r != 0) {
+            if (r == 1)  // let the loads already issued land before the shared memory goes away
+                for (size_t j = k + 1; j < issued; ++j) wait_stage(j);
+            break;
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
 }
 
 // ---- combine: reverse exchange + unpermute + weighted sum ---------------------------------------
@@ -271,45 +396,83 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
         const char* r_row = a.has_res ? static_cast<const char*>(a.res[i]) + t * a.H * d : nullptr;
         if constexpr (VEC) {
             const size_t npk = a.H / L;
-            for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
-                float acc[kCopyUnroll][L];
-                int s0 = 0;
-                if (r_row) {
-#pragma unroll
-                    for (int u = 0; u < kCopyUnroll; ++u)
-                        if (c0 + u * 32 < npk) unpack4<DT>(ld_stream_v4(r_row + (c0 + u * 32) * 16), acc[u]);
-                } else {
-                    const float w0 = ws[0];
+            if (a.k <= kCombineRegSlots) {
+                // every load of a chunk (the residual and up to kCombineRegSlots rows) in flight at once
+                for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
+                    uint4 rv[kCopyUnroll], yv[kCombineRegSlots][kCopyUnroll];
 #pragma unroll
                     for (int u = 0; u < kCopyUnroll; ++u) {
-                        if (c0 + u * 32 < npk) {
-                            unpack4<DT>(ld_stream_v4(ys[0] + (c0 + u * 32) * 16), acc[u]);
+                        if (c0 + u * 32 >= npk) continue;
+                        if (r_row) rv[u] = ld_stream_v4(r_row + (c0 + u * 32) * 16);
 #pragma unroll
-                            for (int l = 0; l < L; ++l) acc[u][l] = w0 * acc[u][l];
-                        }
+                        for (int s = 0; s < kCombineRegSlots; ++s)
+                            if (s < a.k) yv[s][u] = ld_stream_v4(ys[s] + (c0 + u * 32) * 16);
                     }
-                    s0 = 1;
-                }
-                for (int s = s0; s < a.k; ++s) {
-                    const char* y_row = ys[s];
-                    const float w = ws[s];
-                    uint4 v[kCopyUnroll];
-#pragma unroll
-                    for (int u = 0; u < kCopyUnroll; ++u)
-                        if (c0 + u * 32 < npk) v[u] = ld_stream_v4(y_row + (c0 + u * 32) * 16);
 #pragma unroll
                     for (int u = 0; u < kCopyUnroll; ++u) {
-                        if (c0 + u * 32 < npk) {
-                            float y[L];
-                            unpack4<DT>(v[u], y);
+                        if (c0 + u * 32 >= npk) continue;
+                        float acc[L], y[L];
+                        int s0 = 0;
+                        if (r_row) {
+                            unpack4<DT>(rv[u], acc);
+                        } else {
+                            unpack4<DT>(yv[0][u], acc);
 #pragma unroll
-                            for (int l = 0; l < L; ++l) acc[u][l] = acc[u][l] + w * y[l];
+                            for (int l = 0; l < L; ++l) acc[l] = ws[0] * acc[l];
+                            s0 = 1;
                         }
+#pragma unroll
+                        for (int s = 0; s < kCombineRegSlots; ++s) {
+                            if (s < s0 || s >= a.k) continue;
+                            unpack4<DT>(yv[s][u], y);
+                            const float w = ws[s];
+#pragma unroll
+                            for (int l = 0; l < L; ++l) acc[l] = acc[l] + w * y[l];
+                        }
+                        st_v4(o_row + (c0 + u * 32) * 16, pack4<DT>(acc));
                     }
                 }
+            } else {
+                for (size_t c0 = lane; c0 < npk; c0 += 32 * kCopyUnroll) {
+                    float acc[kCopyUnroll][L];
+                    int s0 = 0;
+                    if (r_row) {
 #pragma unroll
-                for (int u = 0; u < kCopyUnroll; ++u)
-                    if (c0 + u * 32 < npk) st_v4(o_row + (c0 + u * 32) * 16, pack4<DT>(acc[u]));
+                        for (int u = 0; u < kCopyUnroll; ++u)
+                            if (c0 + u * 32 < npk) unpack4<DT>(ld_stream_v4(r_row + (c0 + u * 32) * 16), acc[u]);
+                    } else {
+                        const float w0 = ws[0];
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u) {
+                            if (c0 + u * 32 < npk) {
+                                unpack4<DT>(ld_stream_v4(ys[0] + (c0 + u * 32) * 16), acc[u]);
+#pragma unroll
+                                for (int l = 0; l < L; ++l) acc[u][l] = w0 * acc[u][l];
+                            }
+                        }
+                        s0 = 1;
+                    }
+                    for (int s = s0; s < a.k; ++s) {
+                        const char* y_row = ys[s];
+                        const float w = ws[s];
+                        uint4 v[kCopyUnroll];
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u)
+                            if (c0 + u * 32 < npk) v[u] = ld_stream_v4(y_row + (c0 + u * 32) * 16);
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u) {
+                            if (c0 + u * 32 < npk) {
+                                float y[L];
+                                unpack4<DT>(v[u], y);
+#pragma unroll
+                                for (int l = 0; l < L; ++l) acc[u][l] = acc[u][l] + w * y[l];
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kCopyUnroll; ++u)
+                        if (c0 + u * 32 < npk) st_v4(o_row + (c0 + u * 32) * 16, pack4<DT>(acc[u]));
+                }
             }
         } else {
             for (size_t h = lane; h < a.H; h += 32) {
@@ -331,11 +494,20 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
 
 // ---- launch --------------------------------------------------------------------------------------
 
-static dim3 token_grid(const MoeArgs& a, int num_sms) {
+// One wave: the CTAs that fit on the device at once (resident_per_sm from the kernel's occupancy),
+// split evenly over the ranks, each striding over its rank's tokens.
+static dim3 token_grid(const MoeArgs& a, int num_sms, int resident_per_sm) {
     const size_t warps_per_cta = kCopyThreads / 32;
     const size_t want = (a.T + warps_per_cta - 1) / warps_per_cta;
-    const size_t per_rank = std::max<size_t>(1, size_t(num_sms) * 8 / size_t(a.p));
+    const size_t per_rank = std::max<size_t>(1, size_t(num_sms) * size_t(std::max(resident_per_sm, 1)) / size_t(a.p));
     return dim3(unsigned(std::max<size_t>(1, std::min(want, per_rank))), unsigned(a.p), 1u);
+}
+
+template <typename K>
+static int resident_per_sm(K kernel) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kCopyThreads, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
 }
 
 cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
@@ -349,7 +521,8 @@ cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     k_moe_scan<<<unsigned(a.p), kScanThreads, size_t(a.p) * a.p * sizeof(int), s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 32-byte packs when every row start is 32-byte aligned, else 16-byte, else 2-byte units
+    // bulk copies when chosen and every row start is 16-byte aligned; else 32-byte packs when every
+    // row start is 32-byte aligned, else 16-byte, else 2-byte units
     const size_t row_bytes = a.H * size_t(a.elem_bytes);
     bool al32 = row_bytes % 32 == 0, al16 = row_bytes % 16 == 0;
     for (int r = 0; r < a.p; ++r) {
@@ -357,10 +530,20 @@ cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
         al32 = al32 && x % 32 == 0 && y % 32 == 0;
         al16 = al16 && x % 16 == 0 && y % 16 == 0;
     }
-    const dim3 grid = token_grid(a, num_sms);
-    if (al32) k_moe_dispatch_copy<8><<<grid, kCopyThreads, 0, s>>>(a);
-    else if (al16) k_moe_dispatch_copy<4><<<grid, kCopyThreads, 0, s>>>(a);
-    else k_moe_dispatch_copy<0><<<grid, kCopyThreads, 0, s>>>(a);
+    if (a.tma && al16) {
+        const size_t smem = size_t(kMoeTmaStages) * kMoeTmaTile + kMoeTmaStages * sizeof(uint64_t);
+        e = cudaFuncSetAttribute(k_moe_dispatch_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        const size_t tasks = size_t(a.p) * a.T * ((row_bytes + kMoeTmaTile - 1) / kMoeTmaTile);
+        const size_t ctas = std::min(tasks, size_t(num_sms) * kMoeTmaCtasPerSm);
+        k_moe_dispatch_tma<<<unsigned(std::max<size_t>(ctas, 1)), 32, smem, s>>>(a);
+    } else if (al32) {
+        k_moe_dispatch_copy<8><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<8>)), kCopyThreads, 0, s>>>(a);
+    } else if (al16) {
+        k_moe_dispatch_copy<4><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<4>)), kCopyThreads, 0, s>>>(a);
+    } else {
+        k_moe_dispatch_copy<0><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<0>)), kCopyThreads, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
@@ -371,13 +554,15 @@ cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStr
         vec = vec && reinterpret_cast<uintptr_t>(a.src[r]) % 16 == 0 && reinterpret_cast<uintptr_t>(a.dst[r]) % 16 == 0;
         if (a.has_res) vec = vec && reinterpret_cast<uintptr_t>(a.res[r]) % 16 == 0;
     }
-    const dim3 grid = token_grid(a, num_sms);
+    auto go = [&](auto kernel) {
+        kernel<<<token_grid(a, num_sms, resident_per_sm(kernel)), kCopyThreads, 0, s>>>(a);
+    };
     if (dtype == COLL_BF16) {
-        if (vec) k_moe_combine<COLL_BF16, true><<<grid, kCopyThreads, 0, s>>>(a);
-        else k_moe_combine<COLL_BF16, false><<<grid, kCopyThreads, 0, s>>>(a);
+        if (vec) go(k_moe_combine<COLL_BF16, true>);
+        else go(k_moe_combine<COLL_BF16, false>);
     } else if (dtype == COLL_FP32) {
-        if (vec) k_moe_combine<COLL_FP32, true><<<grid, kCopyThreads, 0, s>>>(a);
-        else k_moe_combine<COLL_FP32, false><<<grid, kCopyThreads, 0, s>>>(a);
+        if (vec) go(k_moe_combine<COLL_FP32, true>);
+        else go(k_moe_combine<COLL_FP32, false>);
     } else {
         return cudaErrorInvalidValue;
     }

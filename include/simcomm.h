@@ -128,7 +128,8 @@ const char* coll_status_string(coll_status_t status);
  *   "chunk_bytes"  ring pipelining chunk in bytes of the reduce-scatter wire type (default 1 MiB,
  *                  a multiple of 256, [Atlas] §3.5)
  *   "ring_ctas"    CTAs of the ring executor (0 = as many as fit on the GPU; default 0)
- *   "timeout_ns"   longest wait of one ring step for its predecessor (default 2e9)
+ *   "timeout_ns"   longest device-side wait (a ring, tree or butterfly step for its predecessor, an
+ *                  LL word, a bulk copy) before the call gives up with COLL_ERR_TIMEOUT (default 2e9)
  *   "fault_skip_rank"  debugging: the ring executor never signals this rank's steps, so its
  *                  successor times out (-1 = off, the default). Host-side fault injection only.
  *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v): -1 = the default per
@@ -141,6 +142,9 @@ const char* coll_status_string(coll_status_t status);
  *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16)
  *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
  *                  paths (data read or written once), 0 = none (default)
+ *   "moe_tma"      copy kernel of coll_moe_dispatch: 0 = 32/16-byte loads and stores (default,
+ *                  measured faster), 1 = bulk copies through shared memory (rows of whole 16-byte
+ *                  units at 16-byte aligned bases; otherwise the load/store kernel runs)
  * Returns COLL_ERR_INVALID_ARG for an unknown key or a value out of range. */
 coll_status_t sim_comm_set_option(sim_comm_t comm, const char* key, long long value);
 coll_status_t sim_comm_get_option(sim_comm_t comm, const char* key, long long* value);

@@ -78,16 +78,22 @@ DISPATCH_CASES = [
     (16, 64, 2, 32, 8, "fp32", "uniform", 0),
     (64, 8, 2, 64, 4, "int32", "uniform", 0),
     (2, 4000, 8, 256, 12, "fp32", "uniform", 0),
+    (3, 50, 2, 6, 5000, "bf16", "skew", 0),     # 10,000-byte rows: two bulk tiles per row
+    (2, 40, 3, 4, 4100, "fp32", "uniform", 0),  # 16,400-byte rows: three bulk tiles, a short last one
 ]
 
 
 @pytest.mark.parametrize("p,T,k,E,H,dtype,kind,offset", DISPATCH_CASES)
-def test_dispatch_parity(p, T, k, E, H, dtype, kind, offset):
+@pytest.mark.parametrize("tma", [1, 0])
+def test_dispatch_parity(p, T, k, E, H, dtype, kind, offset, tma):
+    """Both copy kernels: bulk copies through shared memory (rows of whole 16-byte units at aligned
+    bases, else the load/store kernel runs) and 32/16/2-byte loads and stores."""
     ids = make_routes(p, T, k, E, kind, seed=p * 31 + T)
     xs = make_rows(p, T, H, dtype, f"moe.dispatch.{p}.{T}.{H}")
     ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, dtype)
     cap = int(ref["recv_counts"].max()) + 3
     with SC.SimComm(p) as comm:
+        comm.set_option("moe_tma", tma)
         x_g, r_g, _, pos_t, ec, rc = dispatch_case(comm, xs, ids, E, cap, dtype, offset)
         assert comm.async_error() == SC.OK
     np.testing.assert_array_equal(rc.cpu().numpy(), ref["recv_counts"])
