@@ -235,6 +235,33 @@ def test_full_size_moe_workload():
         np.testing.assert_array_equal(got, want[i])
 
 
+@pytest.mark.parametrize("p,T,k,E,H", [(64, 40, 32, 4096, 8), (64, 3, 1, 64, 2), (8, 1, 32, 4096, 16)])
+def test_dispatch_and_combine_at_the_limits(p, T, k, E, H):
+    """The largest shapes the interface accepts: 64 ranks, 32 slots per token, 4,096 experts."""
+    ids = make_routes(p, T, k, E, "uniform", seed=E + k)
+    xs = make_rows(p, T, H, "fp32", f"moe.limits.{p}.{k}.{E}")
+    ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, "fp32")
+    cap = int(ref["recv_counts"].max())
+    with SC.SimComm(p) as comm:
+        x_g, r_g, idx_t, pos_t, ec, rc = dispatch_case(comm, xs, ids, E, cap, "fp32")
+        assert comm.async_error() == SC.OK
+        np.testing.assert_array_equal(ec.cpu().numpy(), ref["expert_counts"])
+        for i in range(p):
+            np.testing.assert_array_equal(pos_t[i].cpu().numpy(), ref["pos"][i])
+        for j in range(p):
+            n = int(ref["recv_counts"][j])
+            np.testing.assert_array_equal(r_g[j].numpy().reshape(cap, H)[:n], ref["recv"][j][:n])
+        ws = S.moe_gate_weights(p, T, k, 1)
+        w_t = [to_torch(w.ravel(), "fp32").view(T, k) for w in ws]
+        out = [torch.empty(T, H, device="cuda") for _ in range(p)]
+        comm.moe_combine([rows2d(g, H) for g in r_g], idx_t, pos_t, w_t, E, out)
+        torch.cuda.synchronize()
+        assert comm.async_error() == SC.OK
+    want = oracle.moe_combine([r[:cap] for r in ref["recv"]], list(ids), list(ws), "fp32", E, acc="slotfold")
+    for i in range(p):
+        np.testing.assert_array_equal(out[i].cpu().numpy(), want[i])
+
+
 def test_dispatch_overflow_and_invalid_ids_copy_nothing():
     p, T, k, E, H, dtype = 4, 200, 2, 8, 16, "fp32"
     ids = make_routes(p, T, k, E, "one", seed=1)
