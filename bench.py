@@ -373,6 +373,34 @@ class MoeWorkload:
         self.col_rows = np.bincount((ids // (E // p)).reshape(-1), minlength=p)
 
 
+MOE_CPU_TOKENS = 2048  # the MoE CPU baseline: the first 2,048 tokens of every rank (a quarter of the layer)
+
+
+def moe_cpu_baseline():
+    """The oracle's dispatch + combine, as it stands and single-threaded, on the first MOE_CPU_TOKENS
+    tokens of every rank of the same seeded layer (the generators are counter-based, so these are
+    the GPU workload's own first tokens, routes and gate weights)."""
+    import numpy as np
+
+    import oracle as O
+    from collective_communication_primitives_b200 import bytemodel as BM
+    from collective_communication_primitives_b200 import synth as S
+    p, T, k, E, H = P, MOE_CPU_TOKENS, MOE["topk"], MOE["experts"], MOE["hidden"]
+    ids = S.moe_routes(p, T, E, k, MOE["zipf_s"], 0)
+    ws = S.moe_gate_weights(p, T, k, 0)
+    x = [S.normal(f"moe.x.rank{i}", T * H, 1.0, "bf16").reshape(T, H) for i in range(p)]
+    res = [S.normal(f"moe.res.rank{i}", T * H, 1.0, "bf16").reshape(T, H) for i in range(p)]
+    cap = int(np.bincount((ids // (E // p)).reshape(-1), minlength=p).max())
+    t0 = time.perf_counter()
+    d = O.moe_dispatch(x, list(ids), E, cap, "bf16")
+    O.moe_combine(d["recv"], list(ids), list(ws), "bf16", E, residual=res, acc="slotfold")
+    secs = time.perf_counter() - t0
+    nbytes = BM.moe_dispatch_bytes(p, T, k, H, 2) + BM.moe_combine_bytes(p, T, k, H, 2, residual=True)
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"dispatch + combine of the first {T} tokens of each of the {p} ranks, single-threaded "
+                      f"C++ oracle, {secs:.1f} s"}
+
+
 def moe_ops(comm, mw):
     from collective_communication_primitives_b200 import bytemodel as BM
     p, T, k, H = mw.p, mw.T, mw.k, mw.H
@@ -387,13 +415,15 @@ def moe_ops(comm, mw):
     ]
 
 
-def moe_block(comm, mw, steps, warmup, stream, hbm):
+def moe_block(comm, mw, steps, warmup, stream, hbm, cpu=False):
     """Device time of the MoE dispatch and combine (behind a spacer, CUDA events) and their HBM
     roofline fractions."""
     ops = moe_ops(comm, mw)
     _, per_op = time_device(ops, steps, warmup, stream)
     blk = {"workload": f"MoE layer, p={mw.p} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} experts (Zipf 1.1), "
                        f"{mw.H}-wide bf16 rows", "max_recv_rows": int(mw.col_rows.max())}
+    if cpu:
+        blk["cpu_baseline"] = moe_cpu_baseline()
     for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
         g = kb / (ms / 1e3) / 1e9
         blk[name] = {"ms": round(ms, 4), "GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
@@ -436,6 +466,8 @@ def moe_main(args):
            "per_op": {o[0]: {"ms": round(t, 4), "GBps": round(o[4] / (t / 1e3) / 1e9, 1),
                              "frac_of_measured": round(o[4] / (t / 1e3) / 1e9 / hbm, 4)} for o, t in zip(ops, per_op)},
            "gpu_launches": int(launches), "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = moe_cpu_baseline()
     print(json.dumps(out))
     comm.close()
 
@@ -769,7 +801,8 @@ def main():
         out["e2e"] = e2e
     if not args.no_moe and not args.ops:
         mw = MoeWorkload(device)
-        out["moe"] = moe_block(comm, mw, max(3, args.steps // 2), args.warmup, stream, hbm)
+        out["moe"] = moe_block(comm, mw, max(3, args.steps // 2), args.warmup, stream, hbm,
+                               cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
         del mw
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline()
