@@ -79,7 +79,7 @@ coll_status_t check_reduce_args(coll_dtype_t dt, coll_op_t op) {
 coll_status_t check_algo(coll_algo_t algo, bool allreduce = false) {
     if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
     if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE ||
-        algo == COLL_ALGO_RING_LL) {
+        algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL) {
         if (allreduce) return COLL_OK;
         return fail(COLL_ERR_UNSUPPORTED,
                     "recursive doubling, halving-doubling, the trees and the LL ring exist for AllReduce only");
@@ -365,55 +365,104 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     return COLL_OK;
 }
 
-// Ring AllReduce on the low-latency protocol (flags inside the data), for small messages.
+// The LL protocol's receive slots (flags inside the data): grown on demand, never cleared between
+// calls because tags never repeat while old words may sit in them.
 constexpr size_t kLLMaxBytes = size_t(256) << 20;
 
-coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
-    const int p = c->p;
-    LLArgs a;
-    std::memset(&a, 0, sizeof(a));
-    fill_ptrs(a.ptrs, b, p, true, true);
-    a.p = p;
-    a.n = n;
-    a.seg = (n + size_t(p) - 1) / size_t(p);
-    a.nslots = uint32_t(2 * p - 3);
-    const size_t bytes = size_t(p) * a.nslots * a.seg * sizeof(unsigned long long);
+coll_status_t ensure_ll_slots(sim_comm* c, size_t bytes) {
     if (bytes > kLLMaxBytes)
-        return fail(COLL_ERR_UNSUPPORTED, "the LL protocol is for small messages: p * (2p-3) * ceil(n/p) * 8 bytes of "
-                                          "receive slots must stay within 256 MiB (use COLL_ALGO_RING)");
-    if (bytes > c->ll_cap) {
-        if (c->ll) cudaFree(c->ll);  // synchronises the device: no kernel still uses the old slots
-        c->ll = nullptr;
-        c->ll_cap = 0;
-        cudaError_t e = cudaMalloc(&c->ll, bytes);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(LL slots)");
-        e = cudaMemset(c->ll, 0, bytes);  // tag 0 is never a live tag
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(LL slots)");
-        c->ll_cap = bytes;
-    }
-    // tags must never repeat while old words may still sit in the slots: start again (and clear
-    // the slots, in stream order) before e * 128 + 127 would leave 32 bits
+        return fail(COLL_ERR_UNSUPPORTED, "the LL protocol is for small messages: its receive slots must stay "
+                                          "within 256 MiB (use COLL_ALGO_RING or COLL_ALGO_RD)");
+    if (bytes <= c->ll_cap) return COLL_OK;
+    if (c->ll) cudaFree(c->ll);  // synchronises the device: no kernel still uses the old slots
+    c->ll = nullptr;
+    c->ll_cap = 0;
+    cudaError_t e = cudaMalloc(&c->ll, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(LL slots)");
+    e = cudaMemset(c->ll, 0, bytes);  // tag 0 is never a live tag
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(LL slots)");
+    c->ll_cap = bytes;
+    return COLL_OK;
+}
+
+// This call's tag of slot 0 (slot q carries tag + q, q < 128). Before e * 128 + 127 would leave 32
+// bits the counter starts again and the slots are cleared, in stream order.
+coll_status_t next_ll_tag(sim_comm* c, cudaStream_t s, uint32_t* tag) {
     c->ll_epoch += 1;
     if (c->ll_epoch >= (1u << 25)) {
         cudaError_t e = cudaMemsetAsync(c->ll, 0, c->ll_cap, s);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(LL slots)");
         c->ll_epoch = 1;
     }
-    a.tag = c->ll_epoch * 128u + 1u;
+    *tag = c->ll_epoch * 128u + 1u;
+    return COLL_OK;
+}
+
+coll_status_t launch_ll(sim_comm* c, LLArgs& a, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
     a.ll = c->ll;
-    a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.scale = (op == COLL_AVG) ? 1.0f / float(a.p) : 1.0f;
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.ctl = make_ctl(c);
-    // CTAs per rank: about 4 elements per thread, all CTAs resident at once (cooperative launch)
-    if (c->ll_ctas_max == 0) c->ll_ctas_max = ring_ll_max_ctas(c->num_sms);
-    const int g_cap = c->ll_ctas_max / p;
-    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
-    const size_t want = (a.seg + 1023) / 1024;
-    a.G = int(std::max<size_t>(1, std::min<size_t>(want, size_t(g_cap))));
     cudaError_t e = launch_ring_ll(a, dt, op, s);
-    if (e != cudaSuccess) return cuda_fail(e, "LL ring launch");
+    if (e != cudaSuccess) return cuda_fail(e, "LL launch");
     c->launches += 1;
     return COLL_OK;
+}
+
+int ll_ctas_cap(sim_comm* c) {
+    if (c->ll_ctas_max == 0) c->ll_ctas_max = ring_ll_max_ctas(c->num_sms);
+    return c->ll_ctas_max;
+}
+
+// Ring AllReduce on the low-latency protocol, for small messages.
+coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+    const int p = c->p;
+    LLArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.kind = LL_RING;
+    a.p = p;
+    a.n = n;
+    a.seg = (n + size_t(p) - 1) / size_t(p);
+    a.nslots = uint32_t(2 * p - 3);
+    coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * a.seg * sizeof(unsigned long long));
+    if (st != COLL_OK) return st;
+    if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    // CTAs per rank: about 4 elements per thread, all CTAs resident at once (cooperative launch)
+    const int g_cap = ll_ctas_cap(c) / p;
+    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
+    a.G = int(std::max<size_t>(1, std::min<size_t>((a.seg + 1023) / 1024, size_t(g_cap))));
+    return launch_ll(c, a, dt, op, s);
+}
+
+// Recursive-doubling AllReduce on the low-latency protocol: every rank's whole vector in registers
+// of one resident grid, at most 8 elements per thread.
+coll_status_t run_rd_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+    const int p = c->p;
+    if (p & (p - 1)) return fail(COLL_ERR_UNSUPPORTED, "recursive doubling needs p a power of two");
+    int L = 0;
+    while ((1 << L) < p) ++L;
+    LLArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.kind = LL_RD;
+    a.p = p;
+    a.n = n;
+    a.seg = n;
+    a.nslots = uint32_t(L);
+    const int g_cap = ll_ctas_cap(c) / p;
+    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
+    const size_t per_thread = (n + size_t(g_cap) * 256 - 1) / (size_t(g_cap) * 256);
+    if (per_thread > 8)
+        return fail(COLL_ERR_UNSUPPORTED, "the LL recursive doubling holds at most 8 elements per thread of one "
+                                          "resident grid (use COLL_ALGO_RD for larger messages)");
+    a.ept = per_thread <= 1 ? 1 : per_thread <= 2 ? 2 : per_thread <= 4 ? 4 : 8;
+    // CTAs per rank: the fewest that keep ept elements per thread
+    a.G = int(std::max<size_t>(1, (n + size_t(a.ept) * 256 - 1) / (size_t(a.ept) * 256)));
+    coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * n * sizeof(unsigned long long));
+    if (st != COLL_OK) return st;
+    if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    return launch_ll(c, a, dt, op, s);
 }
 
 // Single / double binary tree AllReduce on the tree executor.
@@ -722,7 +771,7 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo, true)) != COLL_OK) return st;
-    if ((algo == COLL_ALGO_RD || algo == COLL_ALGO_HD) && (c->p & (c->p - 1)))
+    if ((algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_RD_LL) && (c->p & (c->p - 1)))
         return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling need p a power of two");
     if (n == 0) return COLL_OK;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
@@ -742,6 +791,7 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     if (algo == COLL_ALGO_HD) return run_butterfly(c, b, n, dt, op, BFLY_HD, s);
     if (algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE) return run_tree(c, b, n, dt, op, algo == COLL_ALGO_DBTREE, s);
     if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, op, s);
+    if (algo == COLL_ALGO_RD_LL) return run_rd_ll(c, b, n, dt, op, s);
     RingPlan pl;
     pl.kind = RING_ALLREDUCE;
     pl.seg = (n + size_t(p) - 1) / size_t(p);

@@ -163,17 +163,20 @@ struct TreeArgs {
 
 // ---- low-latency (LL) ring AllReduce --------------------------------------------------------------
 
+enum LLKind { LL_RING = 0, LL_RD = 1 };
 struct LLArgs {
     RankPtrs ptrs;
+    int kind;                // LL_RING or LL_RD
+    int ept;                 // LL_RD: elements per thread, held in registers (1, 2, 4 or 8)
     int p;
     int G;                   // CTAs per rank
     size_t n;                // elements per rank
     size_t seg;              // ring segment, ceil(n / p)
-    uint32_t nslots;         // receive slots per rank: one per step that crosses a hop, 2p - 3
+    uint32_t nslots;         // receive slots per rank: one per step that crosses a hop (ring 2p - 3, RD log2 p)
     uint32_t tag;            // this call's tag of slot 0 (slot q carries tag + q)
     float scale;
     uint64_t timeout_ns;
-    unsigned long long* ll;  // [p][nslots][seg] 64-bit words: (tag << 32) | 32 data bits
+    unsigned long long* ll;  // ring [p][nslots][seg], RD [p][nslots][n] 64-bit words: (tag << 32) | 32 data bits
     Ctl ctl;
 };
 

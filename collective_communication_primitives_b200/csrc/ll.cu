@@ -1,4 +1,4 @@
-// Low-latency (LL) ring AllReduce: the flag travels inside the data.
+// Low-latency (LL) ring and recursive-doubling AllReduce: the flag travels inside the data.
 //
 // "集合通信：原语、算法、NCCL 实现与拓扑映射" (llm-infra-atlas.github.io/hpc/04_collectives), §3.4
 // protocols: the Simple protocol moves data and then raises a separate flag behind a memory fence;
@@ -136,11 +136,73 @@ __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ 
     }
 }
 
+// Recursive doubling on the LL protocol ("集合通信：原语、算法、NCCL 实现与拓扑映射" §2.3 schedule,
+// §3.4 protocol): log2 p steps; at step k every rank sends its whole partial vector to the rank at
+// distance 2^k and combines the two, the lower rank's value first (the same arithmetic as the
+// butterfly executor's recursive doubling, so the same bits). Thread t of rank r keeps EPT of its
+// rank's elements (t, t + S, ..., S = threads per rank) in registers across the steps; at each step
+// it first stores all of them into the partner's slot for that step, then polls its own slot for the
+// partner's values, so two partners never wait on each other in a cycle.
+template <int DT, int OP, bool SCALE, int EPT>
+__global__ void __launch_bounds__(kLLThreads) k_rd_ll(const __grid_constant__ LLArgs a) {
+    using A = typename Elem<DT>::A;
+    const int p = a.p;
+    const int r = int(blockIdx.x) / a.G;
+    const size_t S = size_t(a.G) * kLLThreads;
+    const size_t t0 = size_t(int(blockIdx.x) % a.G) * kLLThreads + threadIdx.x;
+    if (status_failed(a.ctl)) return;
+    A v[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const size_t e = t0 + size_t(j) * S;
+        v[j] = (e < a.n) ? load_elem<DT>(a.ptrs.send[r], e) : A(0);
+    }
+    for (int k = 0; (1 << k) < p; ++k) {
+        const int q = r ^ (1 << k);
+        const uint32_t tag = a.tag + uint32_t(k);
+        unsigned long long* theirs = a.ll + (size_t(q) * a.nslots + k) * a.n;
+        const unsigned long long* mine = a.ll + (size_t(r) * a.nslots + k) * a.n;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const size_t e = t0 + size_t(j) * S;
+            if (e < a.n) st_relaxed_gpu_u64(theirs + e, ((unsigned long long)tag << 32) | acc_bits<DT>(v[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const size_t e = t0 + size_t(j) * S;
+            if (e >= a.n) continue;
+            uint32_t b;
+            if (!ll_wait(a.ctl, mine + e, tag, a.timeout_ns, &b)) return;
+            const A w = acc_of<DT>(b);
+            const A lo = (r < q) ? v[j] : w, hi = (r < q) ? w : v[j];
+            if constexpr (DT == COLL_INT32) v[j] = op_i<OP>(lo, hi);
+            else v[j] = op_f<OP>(lo, hi);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+        const size_t e = t0 + size_t(j) * S;
+        if (e >= a.n) continue;
+        A x = v[j];
+        if constexpr (SCALE) x = x * a.scale;
+        store_bits<DT>(a.ptrs.recv[r], e, out_bits<DT>(x));
+    }
+}
+
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_ll_typed(const LLArgs& a, cudaStream_t s) {
     void* args[] = {const_cast<LLArgs*>(&a)};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE>),
-                                       dim3(unsigned(a.p * a.G)), dim3(kLLThreads), args, 0, s);
+    const void* f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE>);
+    if (a.kind == LL_RD) {
+        switch (a.ept) {
+            case 1: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 1>); break;
+            case 2: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 2>); break;
+            case 4: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 4>); break;
+            case 8: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 8>); break;
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    return cudaLaunchCooperativeKernel(f, dim3(unsigned(a.p * a.G)), dim3(kLLThreads), args, 0, s);
 }
 
 template <int DT>
@@ -165,13 +227,17 @@ cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s) {
     }
 }
 
-// CTAs of the LL kernel that fit on the device at once (the cooperative-launch limit).
+// CTAs of the LL kernels that fit on the device at once (the cooperative-launch limit; the kernel
+// with the most registers sets it).
 int ring_ll_max_ctas(int num_sms) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_ring_ll<COLL_BF16, COLL_SUM, true>, kLLThreads, 0) !=
-            cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    return num_sms * per_sm;
+    int a = 0, b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, k_ring_ll<COLL_BF16, COLL_SUM, true>, kLLThreads, 0) !=
+            cudaSuccess || a < 1)
+        a = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_rd_ll<COLL_FP32, COLL_SUM, true, 8>, kLLThreads, 0) !=
+            cudaSuccess || b < 1)
+        b = 1;
+    return num_sms * (a < b ? a : b);
 }
 
 }  // namespace simcomm

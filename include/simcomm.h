@@ -91,10 +91,15 @@ typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_
  *         with a 4-byte flag in one 8-byte store; no separate flags or fences): same schedule and
  *         rounding as RING, so the same result bit for bit. AllReduce only, small messages: the
  *         communicator keeps p * (2p-3) * ceil(n/p) * 8 bytes of receive slots, at most 256 MiB
- *         (else COLL_ERR_UNSUPPORTED). */
+ *         (else COLL_ERR_UNSUPPORTED).
+ * RD_LL:  recursive doubling (as RD) on the LL protocol: same arithmetic as RD, so the same bits.
+ *         AllReduce only, p a power of two, small messages: each rank's vector is held in registers
+ *         of one resident grid (at most 8 elements per thread, about 1.2M / p elements on a B200)
+ *         and p * log2(p) * n * 8 bytes of receive slots stay within 256 MiB (else
+ *         COLL_ERR_UNSUPPORTED). */
 typedef enum {
     COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3, COLL_ALGO_TREE = 4, COLL_ALGO_DBTREE = 5,
-    COLL_ALGO_RING_LL = 6
+    COLL_ALGO_RING_LL = 6, COLL_ALGO_RD_LL = 7
 } coll_algo_t;
 
 typedef struct {

@@ -72,3 +72,49 @@ def test_ll_limits():
     with pytest.raises(SC.SimCommError) as e:
         c.allgather([x[:8] for x in t], u, algo="ll")
     assert e.value.status == SC.UNSUPPORTED
+
+
+@pytest.mark.parametrize("p", [2, 4, 8, 16, 64])
+@pytest.mark.parametrize("dtype", ["int32", "fp32", "bf16"])
+@pytest.mark.parametrize("op", ["sum", "min", "max", "avg"])
+def test_rd_ll_allreduce_parity(p, dtype, op):
+    """Recursive doubling on the LL protocol: the same arithmetic as the butterfly executor's
+    recursive doubling, so it must equal the oracle's recursive-doubling emulation bit for bit."""
+    if dtype == "int32" and op == "avg":
+        pytest.skip("AVG is not defined for int32")
+    c = comm(p)
+    for n in (1, 7, 100, 4099, 18001) if p <= 16 else (1, 7, 100, 4099):
+        ins = make_inputs("int24" if dtype == "int32" else "normal", p, n, dtype, f"rdll.{p}.{n}", sigma=1e-3)
+        src = [Guarded(n, dtype, fill=x) for x in ins]
+        out = [Guarded(n, dtype) for _ in ins]
+        for _ in range(2):
+            c.allreduce([b.t for b in src], [b.t for b in out], op=op, algo="rd_ll")
+        torch.cuda.synchronize()
+        assert c.async_error() == SC.OK
+        want = O.rd_allreduce(ins, dtype, op)
+        for r in range(p):
+            assert out[r].guards_intact() and src[r].guards_intact()
+            np.testing.assert_array_equal(out[r].numpy(), want[r], err_msg=f"n={n} r={r}")
+
+
+def test_rd_ll_in_place_and_limits():
+    c = comm(8)
+    n = 8 * 1001
+    xs = make_inputs("normal", 8, n, "bf16", "rdll.ip", sigma=1.0)
+    want = O.rd_allreduce(xs, "bf16", "avg")
+    buf = [Guarded(n, "bf16", offset=1, fill=x) for x in xs]
+    c.allreduce([b.t for b in buf], [b.t for b in buf], op="avg", algo="rd_ll")
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    for r in range(8):
+        np.testing.assert_array_equal(buf[r].numpy(), want[r])
+    big = [torch.zeros(4 << 20, device="cuda") for _ in range(8)]  # more than 8 elements per thread
+    with pytest.raises(SC.SimCommError) as e:
+        c.allreduce(big, big, algo="rd_ll")
+    assert e.value.status == SC.UNSUPPORTED
+    c3 = SC.SimComm(3)
+    t = [torch.ones(16, device="cuda") for _ in range(3)]
+    with pytest.raises(SC.SimCommError) as e:
+        c3.allreduce(t, t, algo="rd_ll")
+    assert e.value.status == SC.UNSUPPORTED
+    c3.close()
