@@ -530,6 +530,20 @@ def cpu_baseline():
                       f"single-threaded C++ oracle, {secs:.1f} s"}
 
 
+# The rows of one step, in the order build_step() issues them (the oracle step runs the same rows).
+STEP_ROWS = tuple(f"{op}_{algo}" for algo in ("direct", "ring") for op in (
+    "allreduce_avg_fp32", "allreduce_avg_bf16", "reduce_sum_fp32", "broadcast_fp32", "reduce_scatter_sum_fp32",
+    "allgather_fp32", "alltoall_fp32", "alltoallv_fp32"))
+
+
+def step_config(n, world, rows, options):
+    """The `config` of the step's JSON line, shared by this arm and the reference arm."""
+    return {"workload": f"DP gradient bucket, p={P} ranks x {n} elements per rank, every hot-path row "
+                        f"(direct and ring) per step", "p": P, "n_per_rank": n,
+            "chunk_bytes": 1 << 20, "l2": "inputs larger than L2 (100 MiB per rank fp32)",
+            "ops": rows, "options": options, "parallelism": f"replicas x{world}"}
+
+
 def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -543,13 +557,13 @@ def reference_arm(args):
         tot_s += s
         tot_b += b
     v = tot_b / tot_s / 1e9
-    sample = f"each step: every row on a 1/8-size bucket (p={P}, n={REF_SAMPLE_N} per rank), single-threaded C++ oracle"
+    sample = (f"each step: every row of the step on the first {REF_SAMPLE_N} elements of each rank's bucket (1/8 of "
+              f"the workload; the counter-based inputs are the GPU run's own), single-threaded C++ oracle")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"DP gradient bucket, p={P} ranks x {REF_SAMPLE_N} elements (1/8 sample)",
-                   "p": P, "n_per_rank": REF_SAMPLE_N},
+        "config": step_config(N_BUCKET, args.gpus, list(STEP_ROWS), args.option),
         "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
@@ -789,11 +803,7 @@ def main():
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": f"DP gradient bucket, p={P} ranks x {args.n} elements per rank, every hot-path row "
-                               f"(direct and ring) per step", "p": P, "n_per_rank": args.n,
-                   "chunk_bytes": 1 << 20, "l2": "inputs larger than L2 (100 MiB per rank fp32)",
-                   "ops": [o[0] for o in ops], "options": args.option,
-                   "parallelism": f"replicas x{world}"},
+        "config": step_config(args.n, world, [o[0] for o in ops], args.option),
         "roofline": roofline,
         "north_star_direct": star,
         "per_op": per_op_json,
