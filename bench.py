@@ -36,7 +36,7 @@ FALLBACK_HBM_GBS = 6650.0
 # until a capture of the current build is taken.
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a row's kernel, from an
 # ncu capture of the current build, and the per-rank element count it was captured at.
-NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_195_191_040 + 1_420_263_424, 26_214_400)}
+NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_187_871_232 + 1_420_613_120, 26_214_400)}
 SPACER_CYCLES = 4_000_000  # ~2 ms of a spinning kernel ahead of a timed region
 
 
