@@ -77,8 +77,9 @@ coll_status_t check_reduce_args(coll_dtype_t dt, coll_op_t op) {
 }
 
 // Direct and ring exist for every collective; the butterfly algorithms for AllReduce only.
-coll_status_t check_algo(coll_algo_t algo, bool allreduce = false) {
+coll_status_t check_algo(coll_algo_t algo, bool allreduce = false, bool ll_ring = false) {
     if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
+    if (algo == COLL_ALGO_RING_LL && ll_ring) return COLL_OK;
     if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE ||
         algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL) {
         if (allreduce) return COLL_OK;
@@ -415,17 +416,19 @@ int ll_ctas_cap(sim_comm* c) {
     return c->ll_ctas_max;
 }
 
-// Ring AllReduce on the low-latency protocol, for small messages.
-coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+// Ring AllReduce / ReduceScatter / AllGather on the low-latency protocol, for small messages. n is
+// the per-rank full buffer (the AllReduce buffer, the ReduceScatter input, the AllGather output).
+coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s,
+                          int kind = LL_RING) {
     const int p = c->p;
     LLArgs a;
     std::memset(&a, 0, sizeof(a));
     fill_ptrs(a.ptrs, b, p, true, true);
-    a.kind = LL_RING;
+    a.kind = kind;
     a.p = p;
     a.n = n;
     a.seg = (n + size_t(p) - 1) / size_t(p);
-    a.nslots = uint32_t(2 * p - 3);
+    a.nslots = uint32_t(kind == LL_RING ? 2 * p - 3 : p - 2);  // one per step that crosses a hop
     coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * a.seg * sizeof(unsigned long long));
     if (st != COLL_OK) return st;
     if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
@@ -883,7 +886,7 @@ coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dt
                                   coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
-    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
+    if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo, false, true)) != COLL_OK) return st;
     const int p = c->p;
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "ReduceScatter needs n divisible by p");
     if (n == 0) return COLL_OK;
@@ -899,6 +902,7 @@ coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dt
     if ((st = check_ranges(rs, INPLACE_RS, m * d)) != COLL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (algo == COLL_ALGO_DIRECT || p == 1) return run_direct_reduce(c, b, n, dt, op, MODE_REDUCE_SCATTER, 0, s);
+    if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, op, s, LL_RING_RS);
     RingPlan pl;
     pl.kind = RING_REDUCE_SCATTER;
     pl.seg = m;
@@ -915,7 +919,7 @@ coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
-    if ((st = check_algo(algo)) != COLL_OK) return st;
+    if ((st = check_algo(algo, false, true)) != COLL_OK) return st;
     const int p = c->p;
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "AllGather needs n divisible by p");
     if (n == 0) return COLL_OK;
@@ -931,6 +935,7 @@ coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     if ((st = check_ranges(rs, INPLACE_AG, m * d)) != COLL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (algo == COLL_ALGO_DIRECT || p == 1) return run_copy(c, b, COPY_ALLGATHER, m, dt, 0, true, s);
+    if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, COLL_SUM, s, LL_RING_AG);
     RingPlan pl;
     pl.kind = RING_ALLGATHER;
     pl.seg = m;

@@ -163,10 +163,10 @@ struct TreeArgs {
 
 // ---- low-latency (LL) ring AllReduce --------------------------------------------------------------
 
-enum LLKind { LL_RING = 0, LL_RD = 1 };
+enum LLKind { LL_RING = 0, LL_RD = 1, LL_RING_RS = 2, LL_RING_AG = 3 };
 struct LLArgs {
     RankPtrs ptrs;
-    int kind;                // LL_RING or LL_RD
+    int kind;                // LL_RING (AllReduce), LL_RING_RS, LL_RING_AG or LL_RD
     int ept;                 // LL_RD: elements per thread, held in registers (1, 2, 4 or 8)
     int p;
     int G;                   // CTAs per rank

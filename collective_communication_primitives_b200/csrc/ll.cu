@@ -76,7 +76,19 @@ __device__ __forceinline__ void store_bits(void* base, size_t e, uint32_t b) {
     else static_cast<uint32_t*>(base)[e] = b;
 }
 
-template <int DT, int OP, bool SCALE>
+// The element's bits as stored (bf16: 16 bits, fp32/int32: 32 bits).
+template <int DT>
+__device__ __forceinline__ uint32_t raw_bits(const void* base, size_t e) {
+    if constexpr (DT == COLL_BF16) return static_cast<const uint16_t*>(base)[e];
+    else return static_cast<const uint32_t*>(base)[e];
+}
+
+// MODE LL_RING (AllReduce): the reduce-scatter steps then the all-gather steps; slots: reduce-scatter
+// step s (2..p-1) in slot s-2, all-gather step s (1..p-1) in slot p-2+s-1. MODE LL_RING_RS
+// (ReduceScatter): the reduce-scatter steps only, the owner's segment written to its output at
+// offset 0. MODE LL_RING_AG (AllGather): the all-gather steps only, the input being the rank's own
+// segment: step 1 reads the predecessor's input in place, steps s >= 2 go through slot s-2.
+template <int DT, int OP, bool SCALE, int MODE>
 __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ LLArgs a) {
     using A = typename Elem<DT>::A;
     const int p = a.p;
@@ -88,50 +100,67 @@ __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ 
     unsigned long long* next = a.ll + size_t((r + 1) % p) * a.nslots * a.seg;
     if (status_failed(a.ctl)) return;
     auto seg_of = [&](int s) { return ((r - s) % p + p) % p; };  // rank r's segment at all-gather step s
-    // reduce-scatter
-    for (int s = 1; s <= p - 1; ++s) {
-        const int k = ((r - 1 - s) % p + p) % p;
-        for (size_t i = i0; i < a.seg; i += stride) {
-            const size_t e = size_t(k) * a.seg + i;
-            if (e >= a.n) break;
-            A w;
-            if (s == 1) {
-                w = load_elem<DT>(a.ptrs.send[pred], e);
-            } else {
-                uint32_t b;
-                if (!ll_wait(a.ctl, mine + size_t(s - 2) * a.seg + i, a.tag + uint32_t(s - 2), a.timeout_ns, &b)) return;
-                w = acc_of<DT>(b);
-            }
-            const A o = load_elem<DT>(a.ptrs.send[r], e);
-            if constexpr (DT == COLL_INT32) w = op_i<OP>(w, o);
-            else w = op_f<OP>(w, o);
-            if (s < p - 1) {
-                const uint32_t q = uint32_t(s - 1);  // the successor's slot for step s+1
-                st_relaxed_gpu_u64(next + size_t(q) * a.seg + i,
-                                   ((unsigned long long)(a.tag + q) << 32) | acc_bits<DT>(w));
-            } else {
-                if constexpr (SCALE) w = w * a.scale;
-                const uint32_t ob = out_bits<DT>(w);
-                store_bits<DT>(a.ptrs.recv[r], e, ob);
-                if (p > 1) {
-                    const uint32_t q = uint32_t(p - 2);  // the successor's slot for all-gather step 1
-                    st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, ((unsigned long long)(a.tag + q) << 32) | ob);
+    auto word = [&](uint32_t q, uint32_t bits) { return ((unsigned long long)(a.tag + q) << 32) | bits; };
+    if constexpr (MODE != LL_RING_AG) {
+        for (int s = 1; s <= p - 1; ++s) {  // reduce-scatter: segment (r-1-s) mod p = received ⊕ own
+            const int k = ((r - 1 - s) % p + p) % p;
+            for (size_t i = i0; i < a.seg; i += stride) {
+                const size_t e = size_t(k) * a.seg + i;
+                if (e >= a.n) break;
+                A w;
+                if (s == 1) {
+                    w = load_elem<DT>(a.ptrs.send[pred], e);
+                } else {
+                    uint32_t b;
+                    if (!ll_wait(a.ctl, mine + size_t(s - 2) * a.seg + i, a.tag + uint32_t(s - 2), a.timeout_ns, &b))
+                        return;
+                    w = acc_of<DT>(b);
+                }
+                const A o = load_elem<DT>(a.ptrs.send[r], e);
+                if constexpr (DT == COLL_INT32) w = op_i<OP>(w, o);
+                else w = op_f<OP>(w, o);
+                if (s < p - 1) {
+                    const uint32_t q = uint32_t(s - 1);  // the successor's slot for step s+1
+                    st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, acc_bits<DT>(w)));
+                } else {
+                    if constexpr (SCALE) w = w * a.scale;
+                    const uint32_t ob = out_bits<DT>(w);
+                    if constexpr (MODE == LL_RING_RS) {
+                        store_bits<DT>(a.ptrs.recv[r], i, ob);  // k == r: the owner's segment
+                    } else {
+                        store_bits<DT>(a.ptrs.recv[r], e, ob);
+                        const uint32_t q = uint32_t(p - 2);  // the successor's slot for all-gather step 1
+                        st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, ob));
+                    }
                 }
             }
         }
     }
-    // all-gather
-    for (int s = 1; s <= p - 1; ++s) {
-        const int k = seg_of(s);
-        const uint32_t q = uint32_t(p - 2 + s - 1);
-        for (size_t i = i0; i < a.seg; i += stride) {
-            const size_t e = size_t(k) * a.seg + i;
-            if (e >= a.n) break;
-            uint32_t b;
-            if (!ll_wait(a.ctl, mine + size_t(q) * a.seg + i, a.tag + q, a.timeout_ns, &b)) return;
-            store_bits<DT>(a.ptrs.recv[r], e, b);
-            if (s < p - 1)
-                st_relaxed_gpu_u64(next + size_t(q + 1) * a.seg + i, ((unsigned long long)(a.tag + q + 1) << 32) | b);
+    if constexpr (MODE != LL_RING_RS) {
+        if constexpr (MODE == LL_RING_AG) {  // the own segment into the own output
+            for (size_t i = i0; i < a.seg; i += stride) {
+                const size_t e = size_t(r) * a.seg + i;
+                if (e >= a.n) break;
+                store_bits<DT>(a.ptrs.recv[r], e, raw_bits<DT>(a.ptrs.send[r], i));
+            }
+        }
+        for (int s = 1; s <= p - 1; ++s) {  // all-gather: segment (r-s) mod p from rank r-1
+            const int k = seg_of(s);
+            // this step's slot (unused when AllGather's first step reads in place) and the next one's
+            const int q_in = (MODE == LL_RING_AG) ? s - 2 : p - 2 + s - 1;
+            const uint32_t q_out = uint32_t(q_in + 1);
+            for (size_t i = i0; i < a.seg; i += stride) {
+                const size_t e = size_t(k) * a.seg + i;
+                if (e >= a.n) break;
+                uint32_t b;
+                if (MODE == LL_RING_AG && s == 1) {
+                    b = raw_bits<DT>(a.ptrs.send[pred], i);  // the predecessor's own segment, in place
+                } else if (!ll_wait(a.ctl, mine + size_t(q_in) * a.seg + i, a.tag + uint32_t(q_in), a.timeout_ns, &b)) {
+                    return;
+                }
+                store_bits<DT>(a.ptrs.recv[r], e, b);
+                if (s < p - 1) st_relaxed_gpu_u64(next + size_t(q_out) * a.seg + i, word(q_out, b));
+            }
         }
     }
 }
@@ -192,7 +221,9 @@ __global__ void __launch_bounds__(kLLThreads) k_rd_ll(const __grid_constant__ LL
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_ll_typed(const LLArgs& a, cudaStream_t s) {
     void* args[] = {const_cast<LLArgs*>(&a)};
-    const void* f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE>);
+    const void* f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING>);
+    if (a.kind == LL_RING_RS) f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING_RS>);
+    if (a.kind == LL_RING_AG) f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING_AG>);
     if (a.kind == LL_RD) {
         switch (a.ept) {
             case 1: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 1>); break;
@@ -231,7 +262,7 @@ cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s) {
 // with the most registers sets it).
 int ring_ll_max_ctas(int num_sms) {
     int a = 0, b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, k_ring_ll<COLL_BF16, COLL_SUM, true>, kLLThreads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, k_ring_ll<COLL_BF16, COLL_SUM, true, LL_RING>, kLLThreads, 0) !=
             cudaSuccess || a < 1)
         a = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k_rd_ll<COLL_FP32, COLL_SUM, true, 8>, kLLThreads, 0) !=

@@ -87,11 +87,11 @@ typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_
  *         position m; a position folds (own ⊕ left) ⊕ right in fp32; chunk-pipelined. AllReduce only.
  * DBTREE: double binary tree ([Atlas] §2.4): elements [0, ceil(n/2)) on the tree above, the rest on
  *         its mirror (rank p-1-m at position m). AllReduce only.
- * RING_LL: the ring AllReduce on the low-latency protocol of [Atlas] §3.4 (every 4 data bytes travel
+ * RING_LL: the ring schedule on the low-latency protocol of [Atlas] §3.4 (every 4 data bytes travel
  *         with a 4-byte flag in one 8-byte store; no separate flags or fences): same schedule and
- *         rounding as RING, so the same result bit for bit. AllReduce only, small messages: the
- *         communicator keeps p * (2p-3) * ceil(n/p) * 8 bytes of receive slots, at most 256 MiB
- *         (else COLL_ERR_UNSUPPORTED).
+ *         rounding as RING, so the same result bit for bit. AllReduce, ReduceScatter and AllGather;
+ *         small messages: the communicator keeps p * (2p-3) (AllReduce) or p * (p-2) (the others)
+ *         * ceil(n/p) * 8 bytes of receive slots, at most 256 MiB (else COLL_ERR_UNSUPPORTED).
  * RD_LL:  recursive doubling (as RD) on the LL protocol: same arithmetic as RD, so the same bits.
  *         AllReduce only, p a power of two, small messages: each rank's vector is held in registers
  *         of one resident grid (at most 8 elements per thread, about 1.2M / p elements on a B200)

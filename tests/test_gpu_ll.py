@@ -69,8 +69,8 @@ def test_ll_limits():
     assert e.value.status == SC.UNSUPPORTED
     t = [torch.ones(64, device="cuda") for _ in range(8)]
     u = [torch.zeros(64, device="cuda") for _ in range(8)]
-    with pytest.raises(SC.SimCommError) as e:
-        c.allgather([x[:8] for x in t], u, algo="ll")
+    with pytest.raises(SC.SimCommError) as e:  # the LL ring serves AllReduce, ReduceScatter, AllGather
+        c.alltoall(t, u, algo="ll")
     assert e.value.status == SC.UNSUPPORTED
 
 
@@ -118,3 +118,68 @@ def test_rd_ll_in_place_and_limits():
         c3.allreduce(t, t, algo="rd_ll")
     assert e.value.status == SC.UNSUPPORTED
     c3.close()
+
+
+@pytest.mark.parametrize("p", [2, 3, 5, 8, 16, 64])
+@pytest.mark.parametrize("dtype", ["int32", "fp32", "bf16"])
+@pytest.mark.parametrize("op", ["sum", "min", "avg"])
+def test_ll_reduce_scatter_parity(p, dtype, op):
+    """The ring ReduceScatter on the LL protocol equals the oracle's ring reduce-scatter emulation."""
+    if dtype == "int32" and op == "avg":
+        pytest.skip("AVG is not defined for int32")
+    c = comm(p)
+    for m in (1, 3, 257, 4099):
+        n = m * p
+        ins = make_inputs("int24" if dtype == "int32" else "normal", p, n, dtype, f"llrs.{p}.{m}", sigma=1e-3)
+        src = [Guarded(n, dtype, fill=x) for x in ins]
+        out = [Guarded(m, dtype) for _ in ins]
+        c.reduce_scatter([b.t for b in src], [b.t for b in out], op=op, algo="ll")
+        torch.cuda.synchronize()
+        assert c.async_error() == SC.OK
+        want = O.ring_reduce_scatter(ins, dtype, op)
+        for r in range(p):
+            assert out[r].guards_intact()
+            np.testing.assert_array_equal(out[r].numpy(), want[r], err_msg=f"m={m} r={r}")
+
+
+@pytest.mark.parametrize("p", [2, 3, 5, 8, 16, 64])
+@pytest.mark.parametrize("dtype", ["int32", "fp32", "bf16"])
+def test_ll_allgather_parity(p, dtype):
+    """The ring AllGather on the LL protocol equals the oracle's ring all-gather (and AllGather's layout)."""
+    c = comm(p)
+    for m in (1, 3, 257, 4099):
+        n = m * p
+        shards = make_inputs("int24" if dtype == "int32" else "normal", p, m, dtype, f"llag.{p}.{m}")
+        src = [Guarded(m, dtype, fill=x) for x in shards]
+        out = [Guarded(n, dtype) for _ in shards]
+        c.allgather([b.t for b in src], [b.t for b in out], algo="ll")
+        torch.cuda.synchronize()
+        assert c.async_error() == SC.OK
+        want = O.ring_allgather(shards, dtype)
+        for r in range(p):
+            assert out[r].guards_intact()
+            np.testing.assert_array_equal(out[r].numpy(), want[r], err_msg=f"m={m} r={r}")
+
+
+def test_ll_reduce_scatter_and_allgather_in_place():
+    p, m = 4, 1001
+    n = p * m
+    c = comm(p)
+    xs = make_inputs("normal", p, n, "fp32", "llip.rs", sigma=1.0)
+    want = O.ring_reduce_scatter(xs, "fp32", "sum")
+    full = [Guarded(n, "fp32", fill=x) for x in xs]
+    c.reduce_scatter([b.t for b in full], [b.t[r * m:(r + 1) * m] for r, b in enumerate(full)], op="sum", algo="ll")
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    for r in range(p):
+        np.testing.assert_array_equal(full[r].numpy()[r * m:(r + 1) * m], want[r])
+    shards = make_inputs("normal", p, m, "bf16", "llip.ag", sigma=1.0)
+    want = O.ring_allgather(shards, "bf16")
+    bufs = [Guarded(n, "bf16") for _ in range(p)]
+    for r in range(p):
+        bufs[r].t[r * m:(r + 1) * m].copy_(torch.from_numpy(shards[r].view(np.int16)).view(torch.bfloat16).cuda())
+    c.allgather([b.t[r * m:(r + 1) * m] for r, b in enumerate(bufs)], [b.t for b in bufs], algo="ll")
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    for r in range(p):
+        np.testing.assert_array_equal(bufs[r].numpy(), want[r])
