@@ -403,6 +403,7 @@ coll_status_t next_ll_tag(sim_comm* c, cudaStream_t s, uint32_t* tag) {
 coll_status_t launch_ll(sim_comm* c, LLArgs& a, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
     a.ll = c->ll;
     a.scale = (op == COLL_AVG) ? 1.0f / float(a.p) : 1.0f;
+    a.skip_rank = int(c->fault_skip_rank);
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.ctl = make_ctl(c);
     cudaError_t e = launch_ring_ll(a, dt, op, s);
@@ -515,6 +516,7 @@ coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t
     for (uint32_t k = 0; k < a.nsteps; ++k)
         a.start[k + 1] = a.start[k] + (a.nch[0] + (a.ntrees == 2 ? a.nch[1] : 0)) * a.step_count[k] * a.ntile;
     a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.skip_rank = int(c->fault_skip_rank);
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.st = c->dstate;
     a.ctl = make_ctl(c);
@@ -568,6 +570,7 @@ coll_status_t run_butterfly(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dt
         a.start[g + 1] = a.start[g] + uint32_t(p) * a.ntile[g];
     }
     a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
+    a.skip_rank = int(c->fault_skip_rank);
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.st = c->dstate;
     a.ctl = make_ctl(c);

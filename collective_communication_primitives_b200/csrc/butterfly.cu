@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kBflyThreads, 2) k_butterfly(const __grid_cons
                           static_cast<char*>(a.ptrs.recv[r]) + lo * d, (hi - lo) * d);
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && r != a.skip_rank) {  // fault injection: one rank's tasks never count
             __threadfence();
             atomicAdd(&a.st->step_ctr[g], 1u);
         }

@@ -125,6 +125,7 @@ struct ButterflyArgs {
     uint32_t ntile[kMaxBflySteps];   // tasks per rank at each step
     uint32_t start[kMaxBflySteps + 1];  // first task of each step
     float scale;
+    int skip_rank;           // fault injection: this rank's tasks are never counted (-1 = off)
     uint64_t timeout_ns;
     char* stage;             // RD: two partial buffers per rank; HD: one
     size_t stage_stride;
@@ -153,6 +154,7 @@ struct TreeArgs {
     uint32_t start[kMaxTreeSteps + 1];   // first task of each step
     uint32_t epoch;
     float scale;
+    int skip_rank;           // fault injection: this rank never signals (-1 = off)
     uint64_t timeout_ns;
     char* stage;             // partials, one buffer per rank
     size_t stage_stride;
@@ -175,6 +177,7 @@ struct LLArgs {
     uint32_t nslots;         // receive slots per rank: one per step that crosses a hop (ring 2p - 3, RD log2 p)
     uint32_t tag;            // this call's tag of slot 0 (slot q carries tag + q)
     float scale;
+    int skip_rank;           // fault injection: this rank never sends (-1 = off)
     uint64_t timeout_ns;
     unsigned long long* ll;  // ring [p][nslots][seg], RD [p][nslots][n] 64-bit words: (tag << 32) | 32 data bits
     Ctl ctl;

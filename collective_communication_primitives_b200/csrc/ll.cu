@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ 
                 else w = op_f<OP>(w, o);
                 if (s < p - 1) {
                     const uint32_t q = uint32_t(s - 1);  // the successor's slot for step s+1
-                    st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, acc_bits<DT>(w)));
+                    if (r != a.skip_rank) st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, acc_bits<DT>(w)));
                 } else {
                     if constexpr (SCALE) w = w * a.scale;
                     const uint32_t ob = out_bits<DT>(w);
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ 
                     } else {
                         store_bits<DT>(a.ptrs.recv[r], e, ob);
                         const uint32_t q = uint32_t(p - 2);  // the successor's slot for all-gather step 1
-                        st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, ob));
+                        if (r != a.skip_rank) st_relaxed_gpu_u64(next + size_t(q) * a.seg + i, word(q, ob));
                     }
                 }
             }
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kLLThreads) k_ring_ll(const __grid_constant__ 
                     return;
                 }
                 store_bits<DT>(a.ptrs.recv[r], e, b);
-                if (s < p - 1) st_relaxed_gpu_u64(next + size_t(q_out) * a.seg + i, word(q_out, b));
+                if (s < p - 1 && r != a.skip_rank) st_relaxed_gpu_u64(next + size_t(q_out) * a.seg + i, word(q_out, b));
             }
         }
     }
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kLLThreads) k_rd_ll(const __grid_constant__ LL
 #pragma unroll
         for (int j = 0; j < EPT; ++j) {
             const size_t e = t0 + size_t(j) * S;
-            if (e < a.n) st_relaxed_gpu_u64(theirs + e, ((unsigned long long)tag << 32) | acc_bits<DT>(v[j]));
+            if (e < a.n && r != a.skip_rank) st_relaxed_gpu_u64(theirs + e, ((unsigned long long)tag << 32) | acc_bits<DT>(v[j]));
         }
 #pragma unroll
         for (int j = 0; j < EPT; ++j) {

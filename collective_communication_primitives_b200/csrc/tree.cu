@@ -215,7 +215,8 @@ __global__ void __launch_bounds__(kTreeThreads, 2) k_tree(const __grid_constant_
             }
         }
         __syncthreads();
-        if (threadIdx.x == 0) signal_chunk(a.ctl, tree_flag(a, reduce ? 0 : 1, b, m, c), a.epoch);
+        if (threadIdx.x == 0 && rank_at(m) != a.skip_rank)  // fault injection silences one rank
+            signal_chunk(a.ctl, tree_flag(a, reduce ? 0 : 1, b, m, c), a.epoch);
     }
     // Leave: the last CTA out resets the task counter for the next call.
     __syncthreads();

@@ -1,0 +1,82 @@
+"""Failure detection of the latency schedules, tested without a GPU fault: host-side fault injection
+(option fault_skip_rank: one rank never signals or sends) makes a successor's bounded wait run out,
+so the call reports COLL_ERR_TIMEOUT (or COLL_ERR_ABORTED after sim_comm_abort) and the kernel
+returns; sim_comm_reset makes the communicator usable again."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from collective_communication_primitives_b200 import simcomm as SC
+
+pytestmark = pytest.mark.gpu
+
+
+def run(c, kind, algo, t, u, p, n):
+    if kind == "allreduce":
+        c.allreduce(t, u, algo=algo)
+    elif kind == "reduce_scatter":
+        c.reduce_scatter(t, [x[:n // p] for x in u], algo=algo)
+    else:
+        c.allgather([x[:n // p] for x in t], u, algo=algo)
+
+
+CASES = [("allreduce", a) for a in ("tree", "dbtree", "rd", "hd", "ll", "rd_ll")] + \
+        [("reduce_scatter", "ll"), ("allgather", "ll")]
+
+
+@pytest.mark.parametrize("kind,algo", CASES)
+def test_timeout_when_a_rank_is_silent(kind, algo):
+    p, n = 4, 4 * 4096
+    c = SC.SimComm(p)
+    c.set_option("chunk_bytes", 4096)
+    c.set_option("timeout_ns", 100_000_000)
+    c.set_option("fault_skip_rank", 1)
+    t = [torch.ones(n, device="cuda") for _ in range(p)]
+    u = [torch.zeros(n, device="cuda") for _ in range(p)]
+    t0 = time.time()
+    run(c, kind, algo, t, u, p, n)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 5.0
+    assert c.async_error() == SC.TIMEOUT
+    with pytest.raises(SC.SimCommError) as e:  # refused until reset
+        run(c, kind, algo, t, u, p, n)
+    assert e.value.status == SC.TIMEOUT
+    c.set_option("fault_skip_rank", -1)
+    c.reset()
+    run(c, kind, algo, t, u, p, n)
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    if kind == "allgather":
+        assert torch.equal(u[2], torch.ones_like(u[2]))
+    elif kind == "reduce_scatter":
+        assert torch.equal(u[2][:n // p], torch.full_like(u[2][:n // p], float(p)))
+    else:
+        assert torch.equal(u[2], torch.full_like(u[2], float(p)))
+    c.close()
+
+
+@pytest.mark.parametrize("algo", ["tree", "ll", "rd_ll", "hd"])
+def test_abort_stops_a_waiting_schedule(algo):
+    p, n = 4, 4 * 4096
+    c = SC.SimComm(p)
+    c.set_option("chunk_bytes", 4096)
+    c.set_option("timeout_ns", 5_000_000_000)
+    c.set_option("fault_skip_rank", 1)  # an inner tree position (a silent leaf would hold nobody up)
+    t = [torch.ones(n, device="cuda") for _ in range(p)]
+    u = [torch.zeros(n, device="cuda") for _ in range(p)]
+    t0 = time.time()
+    c.allreduce(t, u, algo=algo)
+    time.sleep(0.05)
+    c.abort()
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 4.0
+    assert c.async_error() == SC.ABORTED
+    c.set_option("fault_skip_rank", -1)
+    c.reset()
+    c.allreduce(t, u, algo=algo)
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    assert np.array_equal(u[3].cpu().numpy(), np.full(n, float(p), np.float32))
+    c.close()
