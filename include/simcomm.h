@@ -137,8 +137,10 @@ const char* coll_status_string(coll_status_t status);
  *                  of this size; default 256 KiB, a multiple of 256 in [4 KiB, 64 MiB])
  *   "timeout_ns"   longest device-side wait (a ring, tree or butterfly step for its predecessor, an
  *                  LL word, a bulk copy) before the call gives up with COLL_ERR_TIMEOUT (default 2e9)
- *   "fault_skip_rank"  debugging: the ring executor never signals this rank's steps, so its
- *                  successor times out (-1 = off, the default). Host-side fault injection only.
+ *   "fault_skip_rank"  debugging: this rank is silenced (the ring and tree executors never signal
+ *                  its chunks, the butterfly executor never counts its tasks, the LL kernels never
+ *                  send its words), so a successor times out (-1 = off, the default). Host-side
+ *                  fault injection only.
  *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v): -1 = the default per
  *                  collective; 0..7 = a bulk-copy pipeline shape (stages x tile bytes, CTAs per SM);
  *                  8 = the 16-byte load/store path (All-to-All(v) only)
