@@ -791,12 +791,12 @@ def main():
                 "minimum_bytes_per_launch": int(eff),
                 "share_of_step": round(d_ms / sum(per_op), 4), "ms_per_launch": round(d_ms, 4)}
     # The four direct kernels the throughput target names (>= 80% of the ~8 TB/s nominal peak).
-    star = {}
+    target = {}
     for (nm, kernel, _, eff, kb), ms in zip(ops, per_op):
         if nm in ("allreduce_avg_fp32_direct", "allreduce_avg_bf16_direct", "reduce_scatter_sum_fp32_direct",
                   "allgather_fp32_direct", "alltoall_fp32_direct"):
             g = kb / (ms / 1e3) / 1e9
-            star[nm] = {"GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
+            target[nm] = {"GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
                         "frac_of_nominal_8TBps": round(g / 8000.0, 4)}
 
     out = {
@@ -805,7 +805,7 @@ def main():
         "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
         "config": step_config(args.n, world, [o[0] for o in ops], args.option),
         "roofline": roofline,
-        "north_star_direct": star,
+        "target_direct": target,
         "per_op": per_op_json,
         "gpu_launches": int(launches),
         "clocks": clocks,
