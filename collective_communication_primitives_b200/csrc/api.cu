@@ -81,7 +81,7 @@ coll_status_t check_algo(coll_algo_t algo, bool allreduce = false, bool ll_ring 
     if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
     if (algo == COLL_ALGO_RING_LL && ll_ring) return COLL_OK;
     if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE ||
-        algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL) {
+        algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL || algo == COLL_ALGO_TREE_LL) {
         if (allreduce) return COLL_OK;
         return fail(COLL_ERR_UNSUPPORTED,
                     "recursive doubling, halving-doubling, the trees and the LL ring exist for AllReduce only");
@@ -440,6 +440,27 @@ coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtyp
     return launch_ll(c, a, dt, op, s);
 }
 
+// Single binary tree AllReduce on the low-latency protocol: three slots per rank (left child, right
+// child, parent), any p.
+coll_status_t run_tree_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+    const int p = c->p;
+    LLArgs a;
+    std::memset(&a, 0, sizeof(a));
+    fill_ptrs(a.ptrs, b, p, true, true);
+    a.kind = LL_TREE;
+    a.p = p;
+    a.n = n;
+    a.seg = n;
+    a.nslots = 3;
+    coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * n * sizeof(unsigned long long));
+    if (st != COLL_OK) return st;
+    if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    const int g_cap = ll_ctas_cap(c) / p;
+    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
+    a.G = int(std::max<size_t>(1, std::min<size_t>((n + 1023) / 1024, size_t(g_cap))));
+    return launch_ll(c, a, dt, op, s);
+}
+
 // Recursive-doubling AllReduce on the low-latency protocol: every rank's whole vector in registers
 // of one resident grid, at most 8 elements per thread.
 coll_status_t run_rd_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
@@ -488,11 +509,13 @@ coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t
     const size_t len[2] = {a.half, n - a.half};
     for (int t = 0; t < a.ntrees; ++t) a.nch[t] = uint32_t((len[t] + a.chunk - 1) / a.chunk);
     a.nchmax = std::max(a.nch[0], a.nch[1]);
-    // a chunk of at most one tile when the range is short: no empty tasks
+    // a short range is one chunk cut into about 4 tasks (parallelism within each level) of whole
+    // 64-element packs, at least 1024 elements each, so no task is empty
     if (a.nchmax == 1) {
         const size_t longest = std::max(len[0], len[1]);
-        a.tile = std::min(a.tile, std::max<size_t>(16, longest));
-        a.ntile = uint32_t((std::min(a.chunk, longest) + a.tile - 1) / a.tile);
+        const size_t quarter = round_up(std::max<size_t>((longest + 3) / 4, 1024), 64);
+        a.tile = std::min(a.tile, quarter);
+        a.ntile = uint32_t((longest + a.tile - 1) / a.tile);
         a.chunk = size_t(a.ntile) * a.tile;
     }
     // levels: internal positions (2m+1 < p) reduce, deepest level first; then every non-root
@@ -527,10 +550,10 @@ coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t
     a.stage_stride = round_up(n * 4, 256);
     if ((st = ensure_stage(c, a.stage_stride * size_t(p))) != COLL_OK) return st;
     a.stage = c->stage;
-    // 16-byte packs need every range start (half, chunk and tile starts) on a 16-byte boundary of
-    // the element and of the partial buffers
-    bool vec = (a.half * d) % 16 == 0 && (a.half * 4) % 16 == 0 && (a.tile * d) % 16 == 0 &&
-               (a.tile * 4) % 16 == 0 && (a.chunk * 4) % 16 == 0;
+    // 16-byte packs need every range start (chunk and tile starts, and the second tree's start) on a
+    // 16-byte boundary of the element and of the partial buffers
+    bool vec = (a.tile * d) % 16 == 0 && (a.tile * 4) % 16 == 0 && (a.chunk * d) % 16 == 0 && (a.chunk * 4) % 16 == 0;
+    if (a.ntrees == 2) vec = vec && (a.half * d) % 16 == 0 && (a.half * 4) % 16 == 0;
     for (int r = 0; r < p; ++r) vec = vec && aligned16(a.ptrs.send[r]) && aligned16(a.ptrs.recv[r]);
     a.vec = vec ? 1 : 0;
     int ctas = c->ring_ctas > 0 ? int(c->ring_ctas) : c->ring_ctas_max;
@@ -804,6 +827,7 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     if (algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE) return run_tree(c, b, n, dt, op, algo == COLL_ALGO_DBTREE, s);
     if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, op, s);
     if (algo == COLL_ALGO_RD_LL) return run_rd_ll(c, b, n, dt, op, s);
+    if (algo == COLL_ALGO_TREE_LL) return run_tree_ll(c, b, n, dt, op, s);
     RingPlan pl;
     pl.kind = RING_ALLREDUCE;
     pl.seg = (n + size_t(p) - 1) / size_t(p);

@@ -165,10 +165,10 @@ struct TreeArgs {
 
 // ---- low-latency (LL) ring AllReduce --------------------------------------------------------------
 
-enum LLKind { LL_RING = 0, LL_RD = 1, LL_RING_RS = 2, LL_RING_AG = 3 };
+enum LLKind { LL_RING = 0, LL_RD = 1, LL_RING_RS = 2, LL_RING_AG = 3, LL_TREE = 4 };
 struct LLArgs {
     RankPtrs ptrs;
-    int kind;                // LL_RING (AllReduce), LL_RING_RS, LL_RING_AG or LL_RD
+    int kind;                // LL_RING (AllReduce), LL_RING_RS, LL_RING_AG, LL_RD or LL_TREE
     int ept;                 // LL_RD: elements per thread, held in registers (1, 2, 4 or 8)
     int p;
     int G;                   // CTAs per rank
@@ -179,7 +179,7 @@ struct LLArgs {
     float scale;
     int skip_rank;           // fault injection: this rank never sends (-1 = off)
     uint64_t timeout_ns;
-    unsigned long long* ll;  // ring [p][nslots][seg], RD [p][nslots][n] 64-bit words: (tag << 32) | 32 data bits
+    unsigned long long* ll;  // ring [p][nslots][seg], RD and tree [p][nslots][n] words: (tag << 32) | 32 data bits
     Ctl ctl;
 };
 

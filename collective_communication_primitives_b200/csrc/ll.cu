@@ -218,12 +218,72 @@ __global__ void __launch_bounds__(kLLThreads) k_rd_ll(const __grid_constant__ LL
     }
 }
 
+// The binary tree on the LL protocol ("Collective Communication：…" "Tree AllReduce 为什么更适合延迟
+// 敏感区间": reduce up a tree, broadcast down; the same heap tree and fold as the tree executor's
+// single tree, so the same bits): position m holds rank m, children 2m+1 and 2m+2. Rank r's slots:
+// 0 and 1 receive its left and right child's partial, 2 receives its parent's result. Thread t of
+// every rank owns the same elements; per element a position waits for its children's words (a leaf
+// for none), folds (own ⊕ left) ⊕ right, and sends the partial to its parent (the root instead
+// scales, rounds and writes its output); then it waits for its parent's result (the root for none),
+// writes it and forwards it to its children. Every wait is on a deeper position (reduce) or a
+// shallower one (broadcast), so no two threads wait on each other in a cycle.
+template <int DT, int OP, bool SCALE>
+__global__ void __launch_bounds__(kLLThreads) k_tree_ll(const __grid_constant__ LLArgs a) {
+    using A = typename Elem<DT>::A;
+    const int p = a.p;
+    const int r = int(blockIdx.x) / a.G;
+    const size_t i0 = size_t(int(blockIdx.x) % a.G) * kLLThreads + threadIdx.x;
+    const size_t stride = size_t(a.G) * kLLThreads;
+    if (status_failed(a.ctl)) return;
+    const int kid0 = 2 * r + 1, kid1 = 2 * r + 2, parent = (r - 1) / 2;
+    const unsigned long long* mine = a.ll + size_t(r) * a.nslots * a.n;
+    auto slot_of = [&](int rank, int q) { return a.ll + (size_t(rank) * a.nslots + q) * a.n; };
+    const bool silent = (r == a.skip_rank);
+    // reduce up
+    for (size_t e = i0; e < a.n; e += stride) {
+        A x = load_elem<DT>(a.ptrs.send[r], e);
+        for (int c = 0; c < 2; ++c) {
+            if ((c == 0 ? kid0 : kid1) >= p) break;
+            uint32_t b;
+            if (!ll_wait(a.ctl, mine + size_t(c) * a.n + e, a.tag + uint32_t(c), a.timeout_ns, &b)) return;
+            if constexpr (DT == COLL_INT32) x = op_i<OP>(x, acc_of<DT>(b));
+            else x = op_f<OP>(x, acc_of<DT>(b));
+        }
+        if (r == 0) {
+            if constexpr (SCALE) x = x * a.scale;
+            const uint32_t ob = out_bits<DT>(x);
+            store_bits<DT>(a.ptrs.recv[0], e, ob);
+            for (int c = 0; c < 2; ++c) {  // the result starts down the tree
+                const int kid = (c == 0) ? kid0 : kid1;
+                if (kid < p && !silent)
+                    st_relaxed_gpu_u64(slot_of(kid, 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | ob);
+            }
+        } else if (!silent) {
+            const int side = (r == 2 * parent + 1) ? 0 : 1;  // which child of the parent this rank is
+            st_relaxed_gpu_u64(slot_of(parent, side) + e,
+                               ((unsigned long long)(a.tag + uint32_t(side)) << 32) | acc_bits<DT>(x));
+        }
+    }
+    if (r == 0) return;
+    // broadcast down
+    for (size_t e = i0; e < a.n; e += stride) {
+        uint32_t b;
+        if (!ll_wait(a.ctl, mine + size_t(2) * a.n + e, a.tag + 2u, a.timeout_ns, &b)) return;
+        store_bits<DT>(a.ptrs.recv[r], e, b);
+        for (int c = 0; c < 2; ++c) {
+            const int kid = (c == 0) ? kid0 : kid1;
+            if (kid < p && !silent) st_relaxed_gpu_u64(slot_of(kid, 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | b);
+        }
+    }
+}
+
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_ll_typed(const LLArgs& a, cudaStream_t s) {
     void* args[] = {const_cast<LLArgs*>(&a)};
     const void* f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING>);
     if (a.kind == LL_RING_RS) f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING_RS>);
     if (a.kind == LL_RING_AG) f = reinterpret_cast<const void*>(&k_ring_ll<DT, OP, SCALE, LL_RING_AG>);
+    if (a.kind == LL_TREE) f = reinterpret_cast<const void*>(&k_tree_ll<DT, OP, SCALE>);
     if (a.kind == LL_RD) {
         switch (a.ept) {
             case 1: f = reinterpret_cast<const void*>(&k_rd_ll<DT, OP, SCALE, 1>); break;

@@ -96,10 +96,12 @@ typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_
  *         AllReduce only, p a power of two, small messages: each rank's vector is held in registers
  *         of one resident grid (at most 8 elements per thread, about 1.2M / p elements on a B200)
  *         and p * log2(p) * n * 8 bytes of receive slots stay within 256 MiB (else
- *         COLL_ERR_UNSUPPORTED). */
+ *         COLL_ERR_UNSUPPORTED).
+ * TREE_LL: the single binary tree (as TREE: same fold, so the same bits) on the LL protocol, any p;
+ *         AllReduce only, small messages: p * 3 * n * 8 bytes of receive slots within 256 MiB. */
 typedef enum {
     COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3, COLL_ALGO_TREE = 4, COLL_ALGO_DBTREE = 5,
-    COLL_ALGO_RING_LL = 6, COLL_ALGO_RD_LL = 7
+    COLL_ALGO_RING_LL = 6, COLL_ALGO_RD_LL = 7, COLL_ALGO_TREE_LL = 8
 } coll_algo_t;
 
 typedef struct {

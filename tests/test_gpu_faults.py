@@ -22,7 +22,7 @@ def run(c, kind, algo, t, u, p, n):
         c.allgather([x[:n // p] for x in t], u, algo=algo)
 
 
-CASES = [("allreduce", a) for a in ("tree", "dbtree", "rd", "hd", "ll", "rd_ll")] + \
+CASES = [("allreduce", a) for a in ("tree", "dbtree", "rd", "hd", "ll", "rd_ll", "tree_ll")] + \
         [("reduce_scatter", "ll"), ("allgather", "ll")]
 
 
@@ -57,7 +57,7 @@ def test_timeout_when_a_rank_is_silent(kind, algo):
     c.close()
 
 
-@pytest.mark.parametrize("algo", ["tree", "ll", "rd_ll", "hd"])
+@pytest.mark.parametrize("algo", ["tree", "ll", "rd_ll", "hd", "tree_ll"])
 def test_abort_stops_a_waiting_schedule(algo):
     p, n = 4, 4 * 4096
     c = SC.SimComm(p)
