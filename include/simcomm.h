@@ -41,9 +41,11 @@
  *     COLL_ERR_CUDA (a CUDA call failed; sim_comm_last_error() has the message), and the sticky
  *     asynchronous error of an earlier call, if the host has already seen it.
  *   - Asynchronous (set on the device, read with sim_comm_get_async_error): COLL_ERR_TIMEOUT (a
- *     ring step waited longer than the timeout for its predecessor), COLL_ERR_ABORTED
- *     (sim_comm_abort was called while a ring step waited), COLL_ERR_OVERFLOW (an All-to-Allv
- *     count exceeds a capacity; nothing is copied). Collectives are not transactions: after an
+ *     bounded device wait ran out: a ring, tree or butterfly step for its predecessor, an LL word,
+ *     a bulk copy), COLL_ERR_ABORTED (sim_comm_abort was called while such a wait was running),
+ *     COLL_ERR_OVERFLOW (an All-to-Allv count or an MoE dispatch exceeds a capacity; nothing is
+ *     copied), COLL_ERR_INVALID_ARG (an MoE expert id or routing-map entry out of range),
+ *     COLL_ERR_INTERNAL (an invariant check failed). Collectives are not transactions: after an
  *     asynchronous error the outputs of the failed call are unspecified, and later calls do no
  *     work until sim_comm_reset ([Primer] "Collective 的故障语义不是事务").
  */

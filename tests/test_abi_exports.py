@@ -64,3 +64,23 @@ def test_create_rejects_bad_rank_counts(lib):
     assert not L.sim_comm_create(0)
     assert b"p must be" in L.sim_comm_last_error()
     assert not L.sim_comm_create(65)
+
+
+def header_enum(prefix):
+    text = open(os.path.join(ROOT, "include", "simcomm.h")).read()
+    return {m.group(1): int(m.group(2)) for m in re.finditer(rf"\b{prefix}(\w+)\s*=\s*(\d+)", text)}
+
+
+def test_binding_codes_match_the_header():
+    algos = header_enum("COLL_ALGO_")
+    names = {"direct": "DIRECT", "ring": "RING", "rd": "RD", "hd": "HD", "tree": "TREE", "dbtree": "DBTREE",
+             "ll": "RING_LL", "rd_ll": "RD_LL", "tree_ll": "TREE_LL"}
+    assert set(names.values()) == set(algos)
+    for key, hname in names.items():
+        assert SC.ALGOS[key] == algos[hname], key
+    dtypes = header_enum("COLL_")
+    assert SC.DTYPES == {"int32": dtypes["INT32"], "fp32": dtypes["FP32"], "bf16": dtypes["BF16"]}
+    assert SC.OPS == {"sum": dtypes["SUM"], "min": dtypes["MIN"], "max": dtypes["MAX"], "avg": dtypes["AVG"]}
+    status = header_enum("COLL_ERR_")
+    status["OK"] = header_enum("COLL_")["OK"]
+    assert {v: "COLL_ERR_" + k if k != "OK" else "COLL_OK" for k, v in status.items()} == SC.STATUS
