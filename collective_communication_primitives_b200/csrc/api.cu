@@ -46,7 +46,7 @@ struct sim_comm {
     long long direct_pack = 0;
     long long direct_ctas_per_sm = 16;
     long long l2_hint = 0;
-    long long ring_task_bytes = 256 * 1024;  // bytes of the wire type one ring / tree task moves
+    long long ring_task_bytes = 0;  // bytes of the wire type one ring / tree task moves; 0 = by message size
     long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
@@ -293,7 +293,15 @@ struct RingPlan {
 
 // One CTA task moves 128 KiB of the step's wire type (the partial type for reduce steps): a chunk
 // is split into that many tasks so that several SMs carry one chunk through each step.
-constexpr size_t kRingTaskBytes = 256 * 1024;  // bytes of the wire type one ring or tree task moves (measured best)
+constexpr size_t kRingTaskBytes = 256 * 1024;  // bytes of the wire type one ring or tree task moves
+
+// Task size of the ring and tree executors. Measured on B200 (p = 2..64): 256 KiB tasks are 2-6%
+// faster than 128 KiB ones from 64 MiB of wire bytes per rank up, and 10-50% slower at 1-16 MiB,
+// where the schedule needs more, shorter tasks per step to keep its pipeline full.
+size_t task_bytes(const sim_comm* c, size_t wire_bytes_per_rank) {
+    if (c->ring_task_bytes > 0) return size_t(c->ring_task_bytes);
+    return wire_bytes_per_rank >= (size_t(64) << 20) ? kRingTaskBytes : kRingTaskBytes / 2;
+}
 
 coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, size_t n, coll_dtype_t dt,
                        coll_op_t op, int root, cudaStream_t s, const long long* counts = nullptr,
@@ -315,7 +323,10 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
         const size_t wire = reduce_kind ? 4 : d;
         // a chunk is at most a segment long (the All-to-Allv's block sizes are known on the device only)
         const size_t span = (pl.kind == RING_ALLTOALLV || pl.seg == 0) ? pl.chunk : std::min(pl.chunk, pl.seg);
-        a.tile = std::min(span, std::max<size_t>(16, size_t(c->ring_task_bytes) / wire));
+        size_t per_rank = n * wire;  // the All-to-Allv's largest send buffer stands in for its message
+        if (pl.kind == RING_ALLTOALLV && send_cap)
+            for (int r = 0; r < p; ++r) per_rank = std::max(per_rank, size_t(std::max<long long>(send_cap[r], 0)) * d);
+        a.tile = std::min(span, std::max<size_t>(16, task_bytes(c, per_rank) / wire));
         a.ntile = uint32_t((span + a.tile - 1) / a.tile);
     }
     a.elem_bytes = int(d);
@@ -504,7 +515,7 @@ coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t
     a.n = n;
     a.half = dbl ? (n + 1) / 2 : n;
     a.chunk = size_t(c->chunk_bytes) / 4;  // chunk bytes count the fp32/int32 partials, as on the ring
-    a.tile = std::min(a.chunk, size_t(c->ring_task_bytes) / 4);
+    a.tile = std::min(a.chunk, task_bytes(c, n * 4) / 4);
     a.ntile = uint32_t((a.chunk + a.tile - 1) / a.tile);
     const size_t len[2] = {a.half, n - a.half};
     for (int t = 0; t < a.ntrees; ++t) a.nch[t] = uint32_t((len[t] + a.chunk - 1) / a.chunk);
@@ -656,8 +667,8 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
         if (value < 1 || value > 32) return fail(COLL_ERR_INVALID_ARG, "direct_ctas_per_sm must be in [1, 32]");
         c->direct_ctas_per_sm = value;
     } else if (k == "ring_task_bytes") {
-        if (value < 4096 || value > (64 << 20) || value % 256 != 0)
-            return fail(COLL_ERR_INVALID_ARG, "ring_task_bytes must be a multiple of 256 in [4 KiB, 64 MiB]");
+        if (value != 0 && (value < 4096 || value > (64 << 20) || value % 256 != 0))
+            return fail(COLL_ERR_INVALID_ARG, "ring_task_bytes must be 0 or a multiple of 256 in [4 KiB, 64 MiB]");
         c->ring_task_bytes = value;
     } else if (k == "moe_tma") {
         if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "moe_tma must be 0 or 1");

@@ -138,7 +138,8 @@ const char* coll_status_string(coll_status_t status);
  *                  a multiple of 256, [Atlas] §3.5)
  *   "ring_ctas"    CTAs of the ring executor (0 = as many as fit on the GPU; default 0)
  *   "ring_task_bytes"  bytes of the wire type one ring or tree task moves (a chunk is cut into tasks
- *                  of this size; default 256 KiB, a multiple of 256 in [4 KiB, 64 MiB])
+ *                  of this size): 0 = by message size, 256 KiB from 64 MiB of wire bytes per rank
+ *                  up, else 128 KiB (default); or a multiple of 256 in [4 KiB, 64 MiB]
  *   "timeout_ns"   longest device-side wait (a ring, tree or butterfly step for its predecessor, an
  *                  LL word, a bulk copy) before the call gives up with COLL_ERR_TIMEOUT (default 2e9)
  *   "fault_skip_rank"  debugging: this rank is silenced (the ring and tree executors never signal
