@@ -20,12 +20,15 @@
  *   - dtype 0 = int32, 1 = fp32, 2 = bf16 (stored as the upper 16 bits of an IEEE fp32).
  *   - op 0 = sum, 1 = min, 2 = max, 3 = avg (sum times 1/p).
  *   - acc 0 = EXACT: sums in double in rank order, rounded once to the output type.
- *     acc 1 = RANKFOLD: the fp32 left fold acc = x0; acc = acc + x1; ... in rank order.
+ *     acc 1 = RANKFOLD: the fp32 left fold acc = x0; acc = acc + x1; ... in rank order (for the
+ *     MoE combine, the same fold over a token's slots; see that section).
  *
- * Return value: 0 on success, -1 on an argument the definitions do not cover.
+ * Return value: 0 on success, -1 on an argument the definitions do not cover; the MoE dispatch
+ * also returns 1 when a destination's capacity is too small.
  *
  * Parity pins: every function here is pinned by a CPU test against the pages' worked example,
- * figure layouts, identities, closed forms or brute force. The ring schedule itself (as opposed to
+ * figure layouts, hand-derived small examples, identities, closed forms or brute force, and a
+ * mutation test plants plausible mistakes in a copy of this file and checks that a pin fails. The ring schedule itself (as opposed to
  * its result) is "parity unpinned": the page's p = 4 trace is garbled, so the schedule follows the
  * reading that makes rank r own block r.
  */
