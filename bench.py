@@ -371,6 +371,7 @@ class MoeWorkload:
         self.recv_counts = torch.empty(p, dtype=torch.int64, device=device)
         self.expert_counts = torch.empty(p, E, dtype=torch.int64, device=device)
         self.col_rows = np.bincount((ids // (E // p)).reshape(-1), minlength=p)
+        self.rank_rows = np.stack([np.bincount(ids[i].reshape(-1) // (E // p), minlength=p) for i in range(p)])
 
 
 MOE_CPU_TOKENS = 2048  # the MoE CPU baseline: the first 2,048 tokens of every rank (a quarter of the layer)
@@ -418,10 +419,12 @@ def moe_ops(comm, mw):
 def moe_block(comm, mw, steps, warmup, stream, hbm, cpu=False):
     """Device time of the MoE dispatch and combine (behind a spacer, CUDA events) and their HBM
     roofline fractions."""
+    from collective_communication_primitives_b200 import synth as S
     ops = moe_ops(comm, mw)
     _, per_op = time_device(ops, steps, warmup, stream)
     blk = {"workload": f"MoE layer, p={mw.p} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} experts (Zipf 1.1), "
-                       f"{mw.H}-wide bf16 rows", "max_recv_rows": int(mw.col_rows.max())}
+                       f"{mw.H}-wide bf16 rows", "max_recv_rows": int(mw.col_rows.max()),
+           "rank_counts": S.count_matrix_stats(mw.rank_rows)}
     if cpu:
         blk["cpu_baseline"] = moe_cpu_baseline()
     for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
@@ -523,11 +526,64 @@ CPU_SAMPLE_N = N_BUCKET             # the CPU baseline: one full step (about 10-
 REF_SAMPLE_N = N_BUCKET // 8        # one reference-arm step: 1/8 of the bucket
 
 
+def oracle_slices(inp, parts):
+    """Cut the step's inputs into `parts` independent steps on contiguous element ranges of every
+    rank's bucket (each a multiple of p * 64 elements), the All-to-Allv counts redrawn per range."""
+    n, unit = inp["n"], P * 64
+    per = max(unit, (n // parts) // unit * unit)
+    cuts = [min(n, i * per) for i in range(parts)] + [n]
+    out = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        if hi <= lo:
+            continue
+        x32 = [x[lo:hi] for x in inp["x32"]]
+        counts = moe_rows_counts(hi - lo, P) * HIDDEN
+        out.append({"n": hi - lo, "x32": x32, "x16": [x[lo:hi] for x in inp["x16"]], "counts": counts,
+                    "vsend": [x32[i][:int(counts[i].sum())] for i in range(P)]})
+    return out
+
+
+def oracle_step_threads(inp, threads):
+    """The oracle step run by `threads` host threads at once, each on its own slice of the bucket
+    (the oracle's C calls release the interpreter lock); returns (wall seconds, effective bytes,
+    threads used)."""
+    parts = oracle_slices(inp, threads)
+    res = [None] * len(parts)
+    go = threading.Barrier(len(parts) + 1)
+
+    def work(i):
+        go.wait()
+        res[i] = oracle_step(parts[i])
+
+    ts = [threading.Thread(target=work, args=(i,)) for i in range(len(parts))]
+    for t in ts:
+        t.start()
+    go.wait()
+    t0 = time.perf_counter()
+    for t in ts:
+        t.join()
+    return time.perf_counter() - t0, sum(r[1] for r in res), len(parts)
+
+
+def host_threads():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
 def cpu_baseline():
-    secs, eff = oracle_step(oracle_inputs(CPU_SAMPLE_N))
+    """The oracle as it stands, timed twice on the same full-bucket step: single-threaded, and on
+    every host core with one contiguous element range of each rank's bucket per thread."""
+    inp = oracle_inputs(CPU_SAMPLE_N)
+    secs, eff = oracle_step(inp)
+    mt_secs, mt_eff, used = oracle_step_threads(inp, host_threads())
     return {"value": eff / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"one step of every row on the full bucket (p={P}, n={CPU_SAMPLE_N} per rank), "
-                      f"single-threaded C++ oracle, {secs:.1f} s"}
+                      f"single-threaded C++ oracle, {secs:.1f} s",
+            "all_cores": {"value": mt_eff / mt_secs / 1e9, "unit": "GB/s", "cores": used,
+                          "sample": f"the same step cut into {used} contiguous element ranges of every rank's "
+                                    f"bucket, one oracle step per host thread, all at once, {mt_secs:.1f} s wall"}}
 
 
 # The rows of one step, in the order build_step() issues them (the oracle step runs the same rows).
@@ -538,10 +594,12 @@ STEP_ROWS = tuple(f"{op}_{algo}" for algo in ("direct", "ring") for op in (
 
 def step_config(n, world, rows, options):
     """The `config` of the step's JSON line, shared by this arm and the reference arm."""
+    from collective_communication_primitives_b200 import synth as S
+    v_stats = dict(S.count_matrix_stats(moe_rows_counts(n, P)), unit=f"rows of {HIDDEN} elements")
     return {"workload": f"DP gradient bucket, p={P} ranks x {n} elements per rank, every hot-path row "
                         f"(direct and ring) per step", "p": P, "n_per_rank": n,
             "chunk_bytes": 1 << 20, "l2": "inputs larger than L2 (100 MiB per rank fp32)",
-            "ops": rows, "options": options, "parallelism": f"replicas x{world}"}
+            "ops": rows, "alltoallv_counts": v_stats, "options": options, "parallelism": f"replicas x{world}"}
 
 
 def reference_arm(args):

@@ -37,3 +37,26 @@ def test_moe_byte_models():
     assert BM.moe_dispatch_bytes(8, 8192, 2, 4096, 2) == 8 * (8192 * 4096 * 2 + 16384 * 4096 * 2 + 8 * 16384)
     assert BM.moe_combine_bytes(8, 8192, 2, 4096, 2) == 8 * (16384 * 4096 * 2 + 2 * 8192 * 4096 * 2 + 12 * 16384)
     assert BM.moe_combine_bytes(1, 1, 1, 1, 4, residual=False) == 4 + 4 + 12
+
+
+def test_oracle_slices_cover_the_bucket_and_threads_agree():
+    """The all-cores CPU baseline cuts the step into contiguous ranges that tile every rank's bucket;
+    each range is an independent step whose elementwise rows equal the full step's on that range."""
+    import numpy as np
+
+    import oracle as O
+    n = bench.P * 64 * 10 + bench.P * 64 * 3  # 13 units: ragged against 4 threads
+    inp = bench.oracle_inputs(n)
+    parts = bench.oracle_slices(inp, 4)
+    assert sum(q["n"] for q in parts) == n and all(q["n"] % (bench.P * 64) == 0 for q in parts)
+    lo = 0
+    full = O.allreduce(inp["x32"], "fp32", "avg", acc="rankfold")
+    for q in parts:
+        assert q["x32"][0].base is not None or q["x32"][0] is inp["x32"][0]  # views, no copies
+        np.testing.assert_array_equal(q["x32"][3], inp["x32"][3][lo:lo + q["n"]])
+        got = O.allreduce(q["x32"], "fp32", "avg", acc="rankfold")
+        np.testing.assert_array_equal(got[0], full[0][lo:lo + q["n"]])
+        assert int(q["counts"].sum(axis=1).max()) <= q["n"]
+        lo += q["n"]
+    secs, eff, used = bench.oracle_step_threads(inp, 4)
+    assert used == len(parts) and secs > 0 and eff > 0
