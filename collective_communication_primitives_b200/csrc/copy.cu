@@ -123,6 +123,73 @@ __device__ __forceinline__ int find_segment(const uint32_t* prefix, int nseg, ui
     return lo;
 }
 
+// ---- interleaved task order over blocks of unequal size --------------------------------------------
+// Level k holds tile k of every block that has more than k tiles; the interleaved order runs the
+// levels one after another, blocks in index order within a level. With blocks of equal size that is
+// t -> (block t % nseg, tile t / nseg); with unequal ones (skewed All-to-Allv counts) a table of the
+// first task of every level maps a task to its level, and a ballot over the blocks finds its block,
+// so no slot is empty and every CTA gets an equal share of real tasks.
+constexpr int kMaxLevels = 8192;
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, v, d);
+        if (lane >= d) v += o;
+    }
+    return v;
+}
+
+// lvl[k], k = 0..tmax: tasks on the levels below k. prefix[s+1] - prefix[s] = tiles of block s, at most
+// tmax. One full warp.
+__device__ void build_levels(const uint32_t* prefix, int nseg, uint32_t tmax, uint32_t* lvl, int lane) {
+    for (uint32_t v = lane; v <= tmax; v += 32) lvl[v] = 0;
+    __syncwarp();
+    for (int s = lane; s < nseg; s += 32) atomicAdd(&lvl[prefix[s + 1] - prefix[s]], 1u);  // blocks per tile count
+    __syncwarp();
+    uint32_t carry_c = 0, carry_l = 0;
+    for (uint32_t b = 0; b <= tmax; b += 32) {
+        const uint32_t v = b + uint32_t(lane);
+        const uint32_t h = v <= tmax ? lvl[v] : 0u;
+        const uint32_t hs = warp_incl_scan(h, lane);
+        const uint32_t act = v <= tmax ? uint32_t(nseg) - (carry_c + hs) : 0u;  // blocks with more than v tiles
+        const uint32_t ls = warp_incl_scan(act, lane);
+        __syncwarp();
+        if (v <= tmax) lvl[v] = carry_l + ls - act;
+        carry_c += __shfl_sync(0xFFFFFFFFu, hs, 31);
+        carry_l += __shfl_sync(0xFFFFFFFFu, ls, 31);
+    }
+    __syncwarp();
+}
+
+// The j-th block (in index order) of those with more than lv tiles. One full warp.
+__device__ __forceinline__ int level_pick(const uint32_t* prefix, int nseg, uint32_t lv, uint32_t j, int lane) {
+    for (int b = 0; b < nseg; b += 32) {
+        const int s = b + lane;
+        const bool act = s < nseg && prefix[s + 1] - prefix[s] > lv;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, act);
+        const uint32_t c = uint32_t(__popc(m));
+        if (j < c) {
+            const bool me = act && uint32_t(__popc(m & ((1u << lane) - 1u))) == j;
+            return b + __ffs(__ballot_sync(0xFFFFFFFFu, me)) - 1;
+        }
+        j -= c;
+    }
+    return 0;  // not reached for j below the level's task count
+}
+
+// Task t (< lvl[tmax]) of the interleaved order: its block and its tile within the block. One full warp.
+__device__ __forceinline__ void level_locate(const uint32_t* prefix, int nseg, const uint32_t* lvl, uint32_t tmax,
+                                             uint32_t t, int lane, int* sg, uint32_t* k) {
+    uint32_t lo = 0, hi = tmax;  // lvl[lo] <= t < lvl[hi]
+    while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (lvl[mid] <= t) lo = mid; else hi = mid;
+    }
+    *k = lo;
+    *sg = level_pick(prefix, nseg, lo, t - lvl[lo], lane);
+}
+
 template <int KIND, int kStages, uint32_t kTile>
 __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ CopyArgs a) {
     static_assert(kStages <= 32, "stage phases live in one 32-bit mask");
@@ -137,6 +204,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     long long* sd = reinterpret_cast<long long*>(bars + kStages);
     long long* rd = sd + ((KIND == COPY_ALLTOALLV) ? p * p : 0);
     uint32_t* prefix = reinterpret_cast<uint32_t*>(rd + ((KIND == COPY_ALLTOALLV) ? p * p : 0));
+    uint32_t* lvl = prefix + nseg + 1;  // a.level_cap + 1 entries
 
     if constexpr (KIND == COPY_ALLTOALLV) {
         const A2avPlan plan = a2av_plan_warp(a.counts, p, a.send_cap, a.recv_cap, sd, rd, a.recv_counts_out, a.ctl);
@@ -150,11 +218,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     }
     __syncwarp();
     if (lane == 0) prefix[0] = 0;
-    uint32_t carry = 0, tmax = 0;
+    uint32_t carry = 0, tmax = 0, tmin = 0xFFFFFFFFu;
     for (int b = 0; b < nseg; b += 32) {
         const int s = b + lane;
         uint32_t v = (s < nseg) ? prefix[s + 1] : 0u;
         tmax = max(tmax, v);
+        if (s < nseg) tmin = min(tmin, v);
 #pragma unroll
         for (int dd = 1; dd < 32; dd <<= 1) {
             const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, v, dd);
@@ -164,15 +233,25 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         carry += __shfl_sync(0xFFFFFFFFu, v, 31);
     }
 #pragma unroll
-    for (int dd = 16; dd > 0; dd >>= 1) tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
+    for (int dd = 16; dd > 0; dd >>= 1) {
+        tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
+        tmin = min(tmin, __shfl_xor_sync(0xFFFFFFFFu, tmin, dd));
+    }
     __syncwarp();
     // Task order: segment-major, or interleaved (tile k of every segment before tile k+1 of any,
-    // so all sources and destinations are streamed at once; empty slots are skipped).
-    const uint32_t total = a.order ? tmax * uint32_t(nseg) : prefix[nseg];
+    // so all sources and destinations are streamed at once): through the level table when the
+    // segments differ in size and it fits, else with empty slots skipped.
+    const bool levels = a.order && tmin != tmax && tmax <= uint32_t(a.level_cap);
+    if (levels) build_levels(prefix, nseg, tmax, lvl, lane);
+    const uint32_t total = (a.order && !levels) ? tmax * uint32_t(nseg) : prefix[nseg];
     auto locate = [&](uint32_t t, int* sg, uint32_t* k) -> bool {
         if (!a.order) {
             *sg = find_segment(prefix, nseg, t);
             *k = t - prefix[*sg];
+            return true;
+        }
+        if (levels) {
+            level_locate(prefix, nseg, lvl, tmax, t, lane, sg, k);
             return true;
         }
         *sg = int(t % uint32_t(nseg));
@@ -192,16 +271,36 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     const uint64_t pol = a.l2_hint ? l2_evict_first_policy() : 0;
     bool failed = false;
 
+    // A task is located once, when its load is issued, and handed to its consume through the stage's
+    // slot. Tasks are issued in increasing order, so the level pointer only moves forward.
+    __shared__ int s_task_sg[kStages];
+    __shared__ uint32_t s_task_ti[kStages];  // kNoTask: an empty slot of the interleaved order
+    constexpr uint32_t kNoTask = 0xFFFFFFFFu;
+    uint32_t lv = 0;
     auto issue = [&](uint32_t k) {
         const uint32_t t = blockIdx.x + k * gridDim.x;
-        int s;
-        uint32_t ti;
-        if (!locate(t, &s, &ti)) return;
+        int s = 0;
+        uint32_t ti = 0;
+        bool ok = true;
+        if (levels) {
+            while (lvl[lv + 1] <= t) ++lv;  // lv < tmax: t < lvl[tmax]
+            s = level_pick(prefix, nseg, lv, t - lvl[lv], lane);
+            ti = lv;
+        } else {
+            ok = locate(t, &s, &ti);
+        }
+        const int st = int(k % kStages);
+        __syncwarp();
+        if (lane == 0) {
+            s_task_sg[st] = s;
+            s_task_ti[st] = ok ? ti : kNoTask;
+        }
+        __syncwarp();
+        if (!ok) return;
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
         const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, ti, kTile);
         if (lane == 0 && g.bhi > g.blo) {
-            const int st = int(k % kStages);
             mbar_arrive_expect_tx(&bars[st], uint32_t(g.bhi - g.blo));
             if (a.l2_hint)
                 bulk_g2s_hint(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st], pol);
@@ -211,10 +310,9 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     };
 
     auto consume = [&](uint32_t k) {
-        const uint32_t t = blockIdx.x + k * gridDim.x;
-        int s;
-        uint32_t ti;
-        if (!locate(t, &s, &ti)) return;
+        const int s = s_task_sg[k % kStages];
+        const uint32_t ti = s_task_ti[k % kStages];
+        if (ti == kNoTask) return;
         const SegDesc d = segment<KIND>(a, s, sd, rd);
         const bool cong = congruent(a, d);
         const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, ti, kTile);
@@ -314,6 +412,7 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     long long* sd = reinterpret_cast<long long*>(smem);
     long long* rd = sd + ((KIND == COPY_ALLTOALLV) ? p * p : 0);
     uint32_t* prefix = reinterpret_cast<uint32_t*>(rd + ((KIND == COPY_ALLTOALLV) ? p * p : 0));
+    uint32_t* lvl = prefix + nseg + 1;  // a.level_cap + 1 entries
     if (threadIdx.x == 0) s_run = !status_failed(a.ctl);
     __syncthreads();
     if (!s_run) return;
@@ -325,18 +424,19 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
         __syncthreads();
         if (!s_run) return;
     }
-    // tasks per segment and their prefix sums (warp 0)
-    __shared__ uint32_t s_tmax;
+    // tasks per segment and their prefix sums (warp 0), and the level table of the interleaved order
+    __shared__ uint32_t s_tmax, s_levels;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         if (lane == 0) prefix[0] = 0;
-        uint32_t carry = 0, tmax = 0;
+        uint32_t carry = 0, tmax = 0, tmin = 0xFFFFFFFFu;
         for (int b = 0; b < nseg; b += 32) {
             const int sg = b + lane;
             uint32_t v = 0;
             if (sg < nseg) {
                 const SegDesc d = segment<KIND>(a, sg, sd, rd);
                 v = uint32_t((d.len + kLsuTask - 1) / kLsuTask);
+                tmin = min(tmin, v);
             }
             tmax = max(tmax, v);
 #pragma unroll
@@ -348,17 +448,30 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
             carry += __shfl_sync(0xFFFFFFFFu, v, 31);
         }
 #pragma unroll
-        for (int dd = 16; dd > 0; dd >>= 1) tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
-        if (lane == 0) s_tmax = tmax;
+        for (int dd = 16; dd > 0; dd >>= 1) {
+            tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, dd));
+            tmin = min(tmin, __shfl_xor_sync(0xFFFFFFFFu, tmin, dd));
+        }
+        __syncwarp();
+        const bool levels = a.order && tmin != tmax && tmax <= uint32_t(a.level_cap);
+        if (levels) build_levels(prefix, nseg, tmax, lvl, lane);
+        if (lane == 0) {
+            s_tmax = tmax;
+            s_levels = levels;
+        }
     }
     __syncthreads();
-    const uint32_t total = a.order ? s_tmax * uint32_t(nseg) : prefix[nseg];
+    const uint32_t tmax = s_tmax;
+    const bool levels = s_levels != 0;
+    const uint32_t total = (a.order && !levels) ? tmax * uint32_t(nseg) : prefix[nseg];
     uint64_t pol = 0;
     if constexpr (HINT) pol = l2_evict_first_policy();
     for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
         int sg;
         uint32_t k;
-        if (a.order) {
+        if (a.order && levels) {
+            level_locate(prefix, nseg, lvl, tmax, t, threadIdx.x & 31, &sg, &k);  // every warp alike
+        } else if (a.order) {
             sg = int(t % uint32_t(nseg));
             k = t / uint32_t(nseg);
             if (k >= prefix[sg + 1] - prefix[sg]) continue;
@@ -373,9 +486,12 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     }
 }
 
-static size_t lsu_smem_bytes(int kind, int p) {
+// Level-table entries for the interleaved order (0 when the order is block after block).
+static int level_cap(const CopyArgs& a) { return a.order ? kMaxLevels : 0; }
+
+static size_t lsu_smem_bytes(int kind, int p, int levels) {
     size_t b = (kind == COPY_ALLTOALLV) ? 2 * size_t(p) * p * sizeof(long long) : 0;
-    return b + (size_t(p) * p + 1) * sizeof(uint32_t);
+    return b + (size_t(p) * p + 1) * sizeof(uint32_t) + (levels ? size_t(levels) + 1 : 0) * sizeof(uint32_t);
 }
 
 template <int KIND, bool HINT>
@@ -383,11 +499,13 @@ static cudaError_t launch_lsu_hint(const CopyArgs& a, int num_sms, cudaStream_t 
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_copy_lsu<KIND, HINT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(lsu_smem_bytes(KIND, kMaxRanks)));
+                                             int(lsu_smem_bytes(KIND, kMaxRanks, kMaxLevels)));
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    k_copy_lsu<KIND, HINT><<<num_sms * 2, kLsuThreads, lsu_smem_bytes(KIND, a.p), s>>>(a);
+    CopyArgs b = a;
+    b.level_cap = level_cap(a);
+    k_copy_lsu<KIND, HINT><<<num_sms * 2, kLsuThreads, lsu_smem_bytes(KIND, a.p, b.level_cap), s>>>(b);
     return cudaGetLastError();
 }
 
@@ -396,11 +514,12 @@ static cudaError_t launch_lsu(const CopyArgs& a, int num_sms, cudaStream_t s) {
     return a.l2_hint ? launch_lsu_hint<KIND, true>(a, num_sms, s) : launch_lsu_hint<KIND, false>(a, num_sms, s);
 }
 
-static size_t copy_smem_bytes(int kind, int p, int stages, uint32_t tile) {
+static size_t copy_smem_bytes(int kind, int p, int stages, uint32_t tile, int levels = 0) {
     const int nseg = (kind == COPY_BCAST) ? 1 : (kind == COPY_ALLTOALL || kind == COPY_ALLTOALLV) ? p * p : p;
     size_t b = size_t(stages) * tile + size_t(stages) * sizeof(uint64_t);
     if (kind == COPY_ALLTOALLV) b += 2 * size_t(p) * p * sizeof(long long);
     b += (size_t(nseg) + 1) * sizeof(uint32_t);
+    if (levels) b += (size_t(levels) + 1) * sizeof(uint32_t);
     return (b + 127) & ~size_t(127);
 }
 
@@ -415,25 +534,45 @@ static int max_smem_optin() {
     return v;
 }
 
+static int max_smem_per_sm() {
+    static int v = -1;
+    if (v < 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
+            v = 100 * 1024;
+    }
+    return v;
+}
+
 template <int KIND, int V>
 static cudaError_t launch_shape(const CopyArgs& a, int num_sms, cudaStream_t s) {
     constexpr CopyShape sh = kCopyShapes[V];
     auto kernel = k_copy<KIND, sh.stages, sh.tile>;
     static bool attr_set = false;
     if (!attr_set) {
-        const size_t want = std::min<size_t>(copy_smem_bytes(KIND, kMaxRanks, sh.stages, sh.tile), size_t(max_smem_optin()));
+        // the kernel's static shared memory (its stage slots) comes on top of the dynamic part
+        const size_t want = std::min<size_t>(copy_smem_bytes(KIND, kMaxRanks, sh.stages, sh.tile, kMaxLevels),
+                                             size_t(max_smem_optin()) - 1024);
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(want));
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    kernel<<<num_sms * sh.ctas_per_sm, kCopyThreads, copy_smem_bytes(KIND, a.p, sh.stages, sh.tile), s>>>(a);
+    // the level table takes what the shape leaves of its share of the SM's shared memory (so the
+    // shape's CTAs per SM still fit), up to kMaxLevels entries
+    CopyArgs b = a;
+    const size_t base = copy_smem_bytes(KIND, a.p, sh.stages, sh.tile);
+    const long long budget = std::min<long long>(max_smem_optin() - 1024, max_smem_per_sm() / sh.ctas_per_sm - 2048);
+    const long long room = (budget - static_cast<long long>(base) - 128) / 4 - 1;
+    b.level_cap = int(std::max(0LL, std::min<long long>(level_cap(a), room)));
+    kernel<<<num_sms * sh.ctas_per_sm, kCopyThreads, copy_smem_bytes(KIND, a.p, sh.stages, sh.tile, b.level_cap), s>>>(b);
     return cudaGetLastError();
 }
 
 template <int KIND>
 static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
     if (variant < 0 || variant >= kNumCopyShapes ||
-        copy_smem_bytes(KIND, a.p, kCopyShapes[variant].stages, kCopyShapes[variant].tile) > size_t(max_smem_optin()))
+        copy_smem_bytes(KIND, a.p, kCopyShapes[variant].stages, kCopyShapes[variant].tile) > size_t(max_smem_optin()) - 1024)
         variant = 0;  // the baseline shape fits every p
     switch (variant) {
         case 1: return launch_shape<KIND, 1>(a, num_sms, s);

@@ -63,6 +63,7 @@ struct CopyArgs {
     int elem_bytes;
     size_t blk_elems;                  // BCAST: n; ALLGATHER, ALLTOALL, SCATTER, GATHER: block n/p
     int order;                         // tile order: 0 segment-major, 1 interleaved over segments
+    int level_cap;                     // order 1: entries of the shared-memory level table (0 = none)
     int l2_hint;                       // 1: evict-first L2 policy on the bulk/streaming copies
     const long long* counts;           // ALLTOALLV: device [p][p]
     long long* recv_counts_out;        // ALLTOALLV: device [p] or null

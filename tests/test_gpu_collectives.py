@@ -579,3 +579,63 @@ def test_copy_engine_variants(variant, p, order):
     finally:
         c.set_option("copy_variant", -1)
         c.set_option("copy_order", -1)
+
+
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("variant", [-1, 0, 4, 8])
+def test_alltoallv_skewed_blocks_every_order(variant, order):
+    """Hot-destination counts (one column far larger than the rest, some blocks empty): the
+    interleaved order's level table gives every task exactly once."""
+    p, m = 8, 300007
+    c = comm(p)
+    c.set_option("copy_variant", variant)
+    c.set_option("copy_order", order)
+    try:
+        ins = make_inputs("int24", p, m, "int32", f"skew.{p}")
+        counts = np.zeros((p, p), dtype=np.int64)
+        for i in range(p):
+            counts[i, 0] = m // 2 + 977 * i
+            for j in range(1, p):
+                counts[i, j] = 0 if (i + j) % 4 == 0 else 1031 * ((i * 3 + j) % 5) + 13
+        rows = counts.sum(axis=1)
+        assert rows.max() <= m
+        vsrc = [Guarded(int(rows[i]), "int32", fill=ins[i][:rows[i]]) for i in range(p)]
+        cap = int(counts.sum(axis=0).max())
+        vdst = [Guarded(cap, "int32") for _ in range(p)]
+        rc = torch.zeros(p, dtype=torch.int64, device="cuda")
+        c.alltoallv([b.t for b in vsrc], [b.t for b in vdst], torch.tensor(counts, device="cuda"), algo="direct",
+                    recv_counts=rc)
+        finish(c, vsrc + vdst)
+        want, _ = O.alltoallv([ins[i][:rows[i]] for i in range(p)], counts, "int32")
+        for j in range(p):
+            np.testing.assert_array_equal(vdst[j].numpy()[:want[j].size], want[j])
+        assert rc.cpu().tolist() == counts.sum(axis=0).tolist()
+    finally:
+        c.set_option("copy_variant", -1)
+        c.set_option("copy_order", -1)
+
+
+def test_alltoallv_interleaved_beyond_the_level_table():
+    """A block of more tiles than the level table holds (over 8,192 tiles of 16 KiB): the interleaved
+    order falls back to skipping empty slots and still gives the oracle's result."""
+    p = 2
+    c = comm(p)
+    c.set_option("copy_variant", 4)  # 16 KiB tiles
+    c.set_option("copy_order", 1)
+    try:
+        big = 8300 * 4096 + 5  # int32 elements: 8,301 tiles
+        counts = np.array([[3, big], [7, 11]], dtype=np.int64)
+        rows = counts.sum(axis=1)
+        ins = [make_inputs("int24", 1, int(rows[i]), "int32", f"lvl.big.{i}")[0] for i in range(p)]
+        vsrc = [torch.from_numpy(x).cuda() for x in ins]
+        cols = counts.sum(axis=0)
+        vdst = [torch.zeros(int(cols[j]), dtype=torch.int32, device="cuda") for j in range(p)]
+        c.alltoallv(vsrc, vdst, torch.tensor(counts, device="cuda"), algo="direct")
+        torch.cuda.synchronize()
+        assert c.async_error() == SC.OK
+        want, _ = O.alltoallv(ins, counts, "int32")
+        for j in range(p):
+            np.testing.assert_array_equal(vdst[j].cpu().numpy(), want[j])
+    finally:
+        c.set_option("copy_variant", -1)
+        c.set_option("copy_order", -1)
