@@ -45,10 +45,17 @@ __device__ __forceinline__ bool cta_failed(const Ctl& ctl) {
     return f;
 }
 
+// Programmatic dependent launch: the scan and the copy are launched while their predecessor in the
+// stream still runs, and wait here (before touching anything it writes) until it has finished and
+// its memory is visible; the predecessor lets them launch from its first instruction.
+__device__ __forceinline__ void wait_for_predecessor() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- counting -----------------------------------------------------------------------------------
 
 __global__ void __launch_bounds__(kMoeThreads) k_moe_count(const __grid_constant__ MoeArgs a) {
     extern __shared__ int s_cnt[];  // [E]
+    allow_dependents();
     if (cta_failed(a.ctl)) return;
     const int i = blockIdx.y;
     const uint32_t tile = blockIdx.x;
@@ -86,29 +93,47 @@ __global__ void __launch_bounds__(kMoeThreads) k_moe_count(const __grid_constant
 
 // ---- prefix sums and the count matrix ------------------------------------------------------------
 
+__device__ __forceinline__ int warp_incl_scan_i(int v, int lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += o;
+    }
+    return v;
+}
+
+constexpr int kScanChunks = 4;        // tile counts of one expert a lane holds at once (128 tiles per pass)
+constexpr int kScanSmemCnt = 4096;    // the last CTA stages the [p][E] totals in shared memory up to this many
+
 __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant__ MoeArgs a) {
-    extern __shared__ int s_c[];  // [p][p] in the last CTA
+    extern __shared__ int s_dyn[];  // [p][p] count matrix, then [p][E] totals (when they fit)
     __shared__ int s_last;
+    wait_for_predecessor();
+    allow_dependents();
     if (cta_failed(a.ctl)) return;
     const int i = blockIdx.x;
-    constexpr int kBatch = 16;
-    // per expert: exclusive prefix of the tile counts over the tiles of rank i, and the total
-    for (int e = threadIdx.x; e < a.E; e += kScanThreads) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kWarps = kScanThreads / 32;
+    // per expert (a warp each, lanes over tiles): exclusive prefix of the tile counts of rank i, and the total
+    for (int e = warp; e < a.E; e += kWarps) {
         int32_t* col = a.tile_hist + size_t(i) * a.ntiles * a.E + e;
         int run = 0;
-        for (uint32_t t0 = 0; t0 < a.ntiles; t0 += kBatch) {
-            int v[kBatch];
+        for (uint32_t t0 = 0; t0 < a.ntiles; t0 += 32 * kScanChunks) {
+            int v[kScanChunks];
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) v[u] = (t0 + u < a.ntiles) ? col[size_t(t0 + u) * a.E] : 0;
+            for (int c = 0; c < kScanChunks; ++c) {
+                const uint32_t t = t0 + uint32_t(c * 32 + lane);
+                v[c] = t < a.ntiles ? col[size_t(t) * a.E] : 0;
+            }
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                if (t0 + u < a.ntiles) {
-                    col[size_t(t0 + u) * a.E] = run;
-                    run += v[u];
-                }
+            for (int c = 0; c < kScanChunks; ++c) {
+                const uint32_t t = t0 + uint32_t(c * 32 + lane);
+                const int incl = warp_incl_scan_i(v[c], lane);
+                if (t < a.ntiles) col[size_t(t) * a.E] = run + incl - v[c];
+                run += __shfl_sync(0xffffffffu, incl, 31);
             }
         }
-        a.cnt[size_t(i) * a.E + e] = run;
+        if (lane == 0) a.cnt[size_t(i) * a.E + e] = run;
     }
     // the last CTA to finish sees every rank's totals
     __threadfence();
@@ -118,11 +143,18 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
     if (!s_last) return;
     __threadfence();
     const int p = a.p;
+    int* s_c = s_dyn;
+    const bool staged = p * a.E <= kScanSmemCnt;
+    int* s_cnt = s_dyn + p * p;
+    if (staged)
+        for (int x = threadIdx.x; x < p * a.E; x += kScanThreads) s_cnt[x] = __ldcg(a.cnt + x);
+    __syncthreads();
+    auto cnt_at = [&](int r, int x) -> int { return staged ? s_cnt[r * a.E + x] : __ldcg(a.cnt + size_t(r) * a.E + x); };
     for (int ij = threadIdx.x; ij < p * p; ij += kScanThreads) {  // c_ij: rows from rank i to rank j
         const int r = ij / p, j = ij % p;
-        int s = 0;
-        for (int x = j * a.E_loc; x < (j + 1) * a.E_loc; ++x) s += __ldcg(a.cnt + size_t(r) * a.E + x);
-        s_c[ij] = s;
+        int sum = 0;
+        for (int x = j * a.E_loc; x < (j + 1) * a.E_loc; ++x) sum += cnt_at(r, x);
+        s_c[ij] = sum;
     }
     __syncthreads();
     for (int j = threadIdx.x; j < p; j += kScanThreads) {  // rows arriving at rank j, against its capacity
@@ -135,9 +167,9 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
         const int r = ie / a.E, e = ie % a.E, j = e / a.E_loc;
         int b = 0;
         for (int q = 0; q < r; ++q) b += s_c[q * p + j];
-        for (int x = j * a.E_loc; x < e; ++x) b += __ldcg(a.cnt + size_t(r) * a.E + x);
+        for (int x = j * a.E_loc; x < e; ++x) b += cnt_at(r, x);
         a.base[ie] = b;
-        if (a.expert_counts_out) a.expert_counts_out[ie] = __ldcg(a.cnt + ie);
+        if (a.expert_counts_out) a.expert_counts_out[ie] = cnt_at(r, e);
     }
     if (threadIdx.x == 0) a.st->moe_ctr = 0;
 }
@@ -156,6 +188,7 @@ __device__ __forceinline__ int slot_width(int k) {
 template <int W>
 __global__ void __launch_bounds__(kCopyThreads) k_moe_dispatch_copy(const __grid_constant__ MoeArgs a) {
     __shared__ char* s_dst[kCopyThreads / 32][32];  // per warp: destination row of (batch token, slot)
+    wait_for_predecessor();
     if (cta_failed(a.ctl)) return;
     const int i = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -229,6 +262,7 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ char* s_dst[kMoeMaxTopk];
     const int lane = threadIdx.x;
+    wait_for_predecessor();
     if (status_failed(a.ctl)) return;  // one word read by every lane: the whole warp leaves together
     unsigned char* stages = smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kMoeTmaStages) * kMoeTmaTile);
@@ -510,6 +544,24 @@ static int resident_per_sm(K kernel) {
     return n;
 }
 
+// A launch that may begin while the stream's previous kernel still runs (the kernel waits for it
+// with griddepcontrol.wait before reading what it wrote).
+static cudaError_t launch_after(void (*kernel)(MoeArgs), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                const MoeArgs& a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
     const size_t smem_count = size_t(a.E) * sizeof(int);
     if (smem_count > 48 * 1024) {
@@ -519,8 +571,10 @@ cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
     k_moe_count<<<dim3(a.ntiles, unsigned(a.p), 1u), kMoeThreads, smem_count, s>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_moe_scan<<<unsigned(a.p), kScanThreads, size_t(a.p) * a.p * sizeof(int), s>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t smem_scan = (size_t(a.p) * a.p + (size_t(a.p) * a.E <= size_t(kScanSmemCnt) ? size_t(a.p) * a.E : 0)) *
+                             sizeof(int);
+    if ((e = launch_after(k_moe_scan, dim3(unsigned(a.p)), dim3(kScanThreads), smem_scan, s, a)) != cudaSuccess)
+        return e;
     // bulk copies when chosen and every row start is 16-byte aligned; else 32-byte packs when every
     // row start is 32-byte aligned, else 16-byte, else 2-byte units
     const size_t row_bytes = a.H * size_t(a.elem_bytes);
@@ -536,15 +590,14 @@ cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         const size_t tasks = size_t(a.p) * a.T * ((row_bytes + kMoeTmaTile - 1) / kMoeTmaTile);
         const size_t ctas = std::min(tasks, size_t(num_sms) * kMoeTmaCtasPerSm);
-        k_moe_dispatch_tma<<<unsigned(std::max<size_t>(ctas, 1)), 32, smem, s>>>(a);
-    } else if (al32) {
-        k_moe_dispatch_copy<8><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<8>)), kCopyThreads, 0, s>>>(a);
-    } else if (al16) {
-        k_moe_dispatch_copy<4><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<4>)), kCopyThreads, 0, s>>>(a);
-    } else {
-        k_moe_dispatch_copy<0><<<token_grid(a, num_sms, resident_per_sm(k_moe_dispatch_copy<0>)), kCopyThreads, 0, s>>>(a);
+        return launch_after(k_moe_dispatch_tma, dim3(unsigned(std::max<size_t>(ctas, 1))), dim3(32), smem, s, a);
     }
-    return cudaGetLastError();
+    auto copy = [&](auto kernel) {
+        return launch_after(kernel, token_grid(a, num_sms, resident_per_sm(kernel)), dim3(kCopyThreads), 0, s, a);
+    };
+    if (al32) return copy(k_moe_dispatch_copy<8>);
+    if (al16) return copy(k_moe_dispatch_copy<4>);
+    return copy(k_moe_dispatch_copy<0>);
 }
 
 cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStream_t s) {
