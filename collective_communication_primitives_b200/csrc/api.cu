@@ -5,8 +5,10 @@
 // as [Atlas] and "Collective Communication：AllReduce、AllGather、ReduceScatter 与 All-to-All"
 // (charlestar.github.io/2026/08/20/gpu-collective-communication) as [Primer].
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
+#include <cctype>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -18,6 +20,14 @@
 #include "simcomm.h"
 
 using namespace simcomm;
+
+// One traced call: its record and the two events that bracket its kernels on the caller's stream.
+struct TraceSlot {
+    sim_comm_trace_record_t rec{};
+    cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+    bool timed = false;
+};
+constexpr size_t kTraceCap = 4096;
 
 struct sim_comm {
     int p = 0;
@@ -50,6 +60,10 @@ struct sim_comm {
     long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
+    long long trace = 0;                  // 1: keep a record of every call (sim_comm_trace_read)
+    std::vector<TraceSlot> trace_ring;    // the last kTraceCap calls
+    unsigned long long trace_seq = 0;     // calls recorded so far
+    unsigned long long trace_next = 0;    // seq of the oldest record not yet read
 };
 
 namespace {
@@ -628,13 +642,9 @@ coll_status_t run_butterfly(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dt
 
 uint32_t chunks_of(size_t seg, size_t chunk) { return uint32_t(std::max<size_t>(1, (seg + chunk - 1) / chunk)); }
 
-long long env_ll(const char* name, long long dflt) {
-    const char* v = std::getenv(name);
-    if (!v || !*v) return dflt;
-    char* end = nullptr;
-    long long x = std::strtoll(v, &end, 0);
-    return (end && *end == 0) ? x : dflt;
-}
+constexpr const char* kOptionKeys[] = {"chunk_bytes", "ring_ctas", "ring_task_bytes", "timeout_ns",
+                                       "fault_skip_rank", "copy_variant", "copy_order", "direct_pack",
+                                       "direct_ctas_per_sm", "l2_hint", "moe_tma", "trace"};
 
 coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     std::string k(key);
@@ -673,11 +683,62 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     } else if (k == "moe_tma") {
         if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "moe_tma must be 0 or 1");
         c->moe_tma = value;
+    } else if (k == "trace") {
+        if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "trace must be 0 or 1");
+        c->trace = value;
     } else {
         return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     }
     return COLL_OK;
 }
+
+// Brackets one entry-point call: an NVTX range (seen by a profiler that collects NVTX; a no-op
+// otherwise) and, while the communicator's "trace" option is on, a record of the call with CUDA
+// events around its kernels. Event timing is skipped on a stream that is being captured.
+struct TraceScope {
+    sim_comm* c = nullptr;
+    TraceSlot* slot = nullptr;
+    cudaStream_t s = nullptr;
+    unsigned long long launches0 = 0;
+
+    TraceScope(sim_comm* comm, const char* coll, size_t n, int dtype, int op, int root, int algo,
+               coll_stream_t stream) {
+        nvtxRangePushA(coll);
+        if (!comm || !comm->trace) return;
+        c = comm;
+        s = static_cast<cudaStream_t>(stream);
+        if (c->trace_ring.size() < kTraceCap) c->trace_ring.resize(kTraceCap);
+        slot = &c->trace_ring[c->trace_seq % kTraceCap];
+        slot->rec = sim_comm_trace_record_t{};
+        slot->rec.seq = c->trace_seq;
+        slot->rec.coll = coll;
+        slot->rec.p = c->p;
+        slot->rec.n = n;
+        slot->rec.dtype = dtype;
+        slot->rec.op = op;
+        slot->rec.root = root;
+        slot->rec.algo = algo;
+        slot->rec.device_ms = -1.0f;
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        slot->timed = cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone;
+        if (slot->timed && !slot->ev0)
+            slot->timed = cudaEventCreate(&slot->ev0) == cudaSuccess && cudaEventCreate(&slot->ev1) == cudaSuccess;
+        if (slot->timed) slot->timed = cudaEventRecord(slot->ev0, s) == cudaSuccess;
+        launches0 = c->launches;
+    }
+
+    coll_status_t done(coll_status_t st) {
+        if (slot) {
+            slot->rec.status = int(st);
+            slot->rec.launches = unsigned(c->launches - launches0);
+            if (slot->timed) slot->timed = cudaEventRecord(slot->ev1, s) == cudaSuccess;
+            c->trace_seq += 1;
+            if (c->trace_seq - c->trace_next > kTraceCap) c->trace_next = c->trace_seq - kTraceCap;
+        }
+        nvtxRangePop();
+        return st;
+    }
+};
 
 }  // namespace
 
@@ -724,17 +785,16 @@ sim_comm_t sim_comm_create(int p) {
         return nullptr;
     }
     c->ring_ctas_max = ring_max_ctas(c->num_sms);
-    // Options from the environment; bad values are ignored (the defaults stay).
-    const long long cb = env_ll("SIMCOMM_CHUNK_BYTES", c->chunk_bytes);
-    if (set_option_impl(c, "chunk_bytes", cb) != COLL_OK) c->chunk_bytes = 1 << 20;
-    const long long rc = env_ll("SIMCOMM_RING_CTAS", 0);
-    if (set_option_impl(c, "ring_ctas", rc) != COLL_OK) c->ring_ctas = 0;
-    const long long to = env_ll("SIMCOMM_TIMEOUT_NS", c->timeout_ns);
-    if (set_option_impl(c, "timeout_ns", to) != COLL_OK) c->timeout_ns = 2000000000LL;
-    const long long fr = env_ll("SIMCOMM_FAULT_SKIP_RANK", -1);
-    if (set_option_impl(c, "fault_skip_rank", fr) != COLL_OK) c->fault_skip_rank = -1;
-    const long long cv = env_ll("SIMCOMM_COPY_VARIANT", c->copy_variant);
-    if (set_option_impl(c, "copy_variant", cv) != COLL_OK) c->copy_variant = -1;
+    // Options from the environment (SIMCOMM_<KEY>); a value the option rejects leaves the default.
+    for (const char* key : kOptionKeys) {
+        std::string env = "SIMCOMM_";
+        for (const char* q = key; *q; ++q) env += char(std::toupper(static_cast<unsigned char>(*q)));
+        const char* v = std::getenv(env.c_str());
+        if (!v || !*v) continue;
+        char* end = nullptr;
+        const long long x = std::strtoll(v, &end, 0);
+        if (end && *end == 0) set_option_impl(c, key, x);
+    }
     g_last_error.clear();
     return c;
 }
@@ -748,7 +808,29 @@ coll_status_t sim_comm_destroy(sim_comm_t c) {
     if (c->ll) cudaFree(c->ll);
     if (c->dstate) cudaFree(c->dstate);
     if (c->host_words) cudaFreeHost(c->host_words);
+    for (TraceSlot& t : c->trace_ring) {
+        if (t.ev0) cudaEventDestroy(t.ev0);
+        if (t.ev1) cudaEventDestroy(t.ev1);
+    }
     delete c;
+    return COLL_OK;
+}
+
+coll_status_t sim_comm_trace_read(sim_comm_t c, sim_comm_trace_record_t* out, int cap, int* count) {
+    if (!c || !count || cap < 0 || (cap > 0 && !out)) return fail(COLL_ERR_INVALID_ARG, "null argument or negative cap");
+    int got = 0;
+    while (got < cap && c->trace_next < c->trace_seq) {
+        TraceSlot& t = c->trace_ring[c->trace_next % kTraceCap];
+        out[got] = t.rec;
+        if (t.timed && t.rec.launches > 0) {
+            float ms = -1.0f;
+            if (cudaEventSynchronize(t.ev1) == cudaSuccess && cudaEventElapsedTime(&ms, t.ev0, t.ev1) == cudaSuccess)
+                out[got].device_ms = ms;
+        }
+        ++got;
+        ++c->trace_next;
+    }
+    *count = got;
     return COLL_OK;
 }
 
@@ -773,6 +855,7 @@ coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* valu
     else if (k == "direct_ctas_per_sm") *value = c->direct_ctas_per_sm;
     else if (k == "moe_tma") *value = c->moe_tma;
     else if (k == "ring_task_bytes") *value = c->ring_task_bytes;
+    else if (k == "trace") *value = c->trace;
     else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
     return COLL_OK;
 }
@@ -812,8 +895,8 @@ coll_status_t sim_comm_launch_count(sim_comm_t c, unsigned long long* out) {
 
 // ---- collectives -------------------------------------------------------------------------------
 
-coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, coll_algo_t algo,
-                             coll_stream_t stream) {
+static coll_status_t coll_allreduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                         coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo, true)) != COLL_OK) return st;
@@ -850,8 +933,8 @@ coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     return run_ring(c, b, pl, n, dt, op, 0, s);
 }
 
-coll_status_t coll_reduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, int root,
-                          coll_algo_t algo, coll_stream_t stream) {
+static coll_status_t coll_reduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, int root,
+                                      coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo)) != COLL_OK) return st;
@@ -885,8 +968,8 @@ coll_status_t coll_reduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt
     return run_ring(c, bb, pl, n, dt, op, root, s);
 }
 
-coll_status_t coll_broadcast(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
-                             coll_stream_t stream) {
+static coll_status_t coll_broadcast_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root,
+                                         coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -920,8 +1003,8 @@ coll_status_t coll_broadcast(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     return run_ring(c, bb, pl, n, dt, COLL_SUM, root, s);
 }
 
-coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
-                                  coll_algo_t algo, coll_stream_t stream) {
+static coll_status_t coll_reduce_scatter_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                              coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if ((st = check_reduce_args(dt, op)) != COLL_OK || (st = check_algo(algo, false, true)) != COLL_OK) return st;
@@ -952,8 +1035,8 @@ coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dt
     return run_ring(c, b, pl, n, dt, op, 0, s);
 }
 
-coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
-                             coll_stream_t stream) {
+static coll_status_t coll_allgather_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                                         coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -985,8 +1068,8 @@ coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t
     return run_ring(c, b, pl, n, dt, COLL_SUM, 0, s);
 }
 
-coll_status_t coll_alltoall(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
-                            coll_stream_t stream) {
+static coll_status_t coll_alltoall_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                                        coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1017,8 +1100,8 @@ coll_status_t coll_alltoall(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t 
     return run_ring(c, b, pl, n, dt, COLL_SUM, 0, s);
 }
 
-coll_status_t coll_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
-                           coll_stream_t stream) {
+static coll_status_t coll_scatter_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root,
+                                       coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1044,8 +1127,8 @@ coll_status_t coll_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t d
     return run_copy(c, bb, COPY_SCATTER, m, dt, root, false, static_cast<cudaStream_t>(stream));
 }
 
-coll_status_t coll_gather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
-                          coll_stream_t stream) {
+static coll_status_t coll_gather_impl(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root,
+                                      coll_algo_t algo, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1071,9 +1154,9 @@ coll_status_t coll_gather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt
     return run_copy(c, bb, COPY_GATHER, m, dt, root, true, static_cast<cudaStream_t>(stream));
 }
 
-coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* counts_dev, const long long* send_cap,
-                             const long long* recv_cap, coll_dtype_t dt, coll_algo_t algo, coll_stream_t stream,
-                             long long* recv_counts_dev) {
+static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long long* counts_dev,
+                                         const long long* send_cap, const long long* recv_cap, coll_dtype_t dt,
+                                         coll_algo_t algo, coll_stream_t stream, long long* recv_counts_dev) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1132,10 +1215,11 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 extern "C" {
 
-coll_status_t coll_moe_dispatch(sim_comm_t c, const void* const* x, const int32_t* const* topk_idx, size_t tokens,
-                                int k, size_t hidden, int experts, coll_dtype_t dt, void* const* recv,
-                                size_t recv_cap_rows, int32_t* const* route_pos, long long* expert_counts_dev,
-                                long long* recv_counts_dev, coll_stream_t stream) {
+static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, const int32_t* const* topk_idx,
+                                            size_t tokens, int k, size_t hidden, int experts, coll_dtype_t dt,
+                                            void* const* recv, size_t recv_cap_rows, int32_t* const* route_pos,
+                                            long long* expert_counts_dev, long long* recv_counts_dev,
+                                            coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1207,10 +1291,11 @@ coll_status_t coll_moe_dispatch(sim_comm_t c, const void* const* x, const int32_
     return COLL_OK;
 }
 
-coll_status_t coll_moe_combine(sim_comm_t c, const void* const* y, size_t y_rows, const int32_t* const* topk_idx,
-                               const int32_t* const* route_pos, const float* const* topk_weight,
-                               const void* const* residual, size_t tokens, int k, size_t hidden, int experts,
-                               coll_dtype_t dt, void* const* out, coll_stream_t stream) {
+static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, size_t y_rows,
+                                           const int32_t* const* topk_idx, const int32_t* const* route_pos,
+                                           const float* const* topk_weight, const void* const* residual,
+                                           size_t tokens, int k, size_t hidden, int experts, coll_dtype_t dt,
+                                           void* const* out, coll_stream_t stream) {
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
@@ -1403,3 +1488,82 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     }
     return COLL_OK;
 }
+
+// ---- traced entry points --------------------------------------------------------------------------
+
+extern "C" {
+
+coll_status_t coll_allreduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, coll_algo_t algo,
+                             coll_stream_t stream) {
+    TraceScope ts(c, "allreduce", n, int(dt), int(op), -1, int(algo), stream);
+    return ts.done(coll_allreduce_impl(c, b, n, dt, op, algo, stream));
+}
+
+coll_status_t coll_reduce(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op, int root,
+                          coll_algo_t algo, coll_stream_t stream) {
+    TraceScope ts(c, "reduce", n, int(dt), int(op), root, int(algo), stream);
+    return ts.done(coll_reduce_impl(c, b, n, dt, op, root, algo, stream));
+}
+
+coll_status_t coll_broadcast(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                             coll_stream_t stream) {
+    TraceScope ts(c, "broadcast", n, int(dt), -1, root, int(algo), stream);
+    return ts.done(coll_broadcast_impl(c, b, n, dt, root, algo, stream));
+}
+
+coll_status_t coll_reduce_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_op_t op,
+                                  coll_algo_t algo, coll_stream_t stream) {
+    TraceScope ts(c, "reduce_scatter", n, int(dt), int(op), -1, int(algo), stream);
+    return ts.done(coll_reduce_scatter_impl(c, b, n, dt, op, algo, stream));
+}
+
+coll_status_t coll_allgather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                             coll_stream_t stream) {
+    TraceScope ts(c, "allgather", n, int(dt), -1, -1, int(algo), stream);
+    return ts.done(coll_allgather_impl(c, b, n, dt, algo, stream));
+}
+
+coll_status_t coll_alltoall(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, coll_algo_t algo,
+                            coll_stream_t stream) {
+    TraceScope ts(c, "alltoall", n, int(dt), -1, -1, int(algo), stream);
+    return ts.done(coll_alltoall_impl(c, b, n, dt, algo, stream));
+}
+
+coll_status_t coll_scatter(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                           coll_stream_t stream) {
+    TraceScope ts(c, "scatter", n, int(dt), -1, root, int(algo), stream);
+    return ts.done(coll_scatter_impl(c, b, n, dt, root, algo, stream));
+}
+
+coll_status_t coll_gather(sim_comm_t c, coll_bufs_t b, size_t n, coll_dtype_t dt, int root, coll_algo_t algo,
+                          coll_stream_t stream) {
+    TraceScope ts(c, "gather", n, int(dt), -1, root, int(algo), stream);
+    return ts.done(coll_gather_impl(c, b, n, dt, root, algo, stream));
+}
+
+coll_status_t coll_alltoallv(sim_comm_t c, coll_bufs_t b, const long long* counts_dev, const long long* send_cap,
+                             const long long* recv_cap, coll_dtype_t dt, coll_algo_t algo, coll_stream_t stream,
+                             long long* recv_counts_dev) {
+    TraceScope ts(c, "alltoallv", 0, int(dt), -1, -1, int(algo), stream);
+    return ts.done(coll_alltoallv_impl(c, b, counts_dev, send_cap, recv_cap, dt, algo, stream, recv_counts_dev));
+}
+
+coll_status_t coll_moe_dispatch(sim_comm_t c, const void* const* x, const int32_t* const* topk_idx, size_t tokens,
+                                int k, size_t hidden, int experts, coll_dtype_t dt, void* const* recv,
+                                size_t recv_cap_rows, int32_t* const* route_pos, long long* expert_counts_dev,
+                                long long* recv_counts_dev, coll_stream_t stream) {
+    TraceScope ts(c, "moe_dispatch", tokens, int(dt), -1, -1, -1, stream);
+    return ts.done(coll_moe_dispatch_impl(c, x, topk_idx, tokens, k, hidden, experts, dt, recv, recv_cap_rows,
+                                          route_pos, expert_counts_dev, recv_counts_dev, stream));
+}
+
+coll_status_t coll_moe_combine(sim_comm_t c, const void* const* y, size_t y_rows, const int32_t* const* topk_idx,
+                               const int32_t* const* route_pos, const float* const* topk_weight,
+                               const void* const* residual, size_t tokens, int k, size_t hidden, int experts,
+                               coll_dtype_t dt, void* const* out, coll_stream_t stream) {
+    TraceScope ts(c, "moe_combine", tokens, int(dt), -1, -1, -1, stream);
+    return ts.done(coll_moe_combine_impl(c, y, y_rows, topk_idx, route_pos, topk_weight, residual, tokens, k, hidden,
+                                         experts, dt, out, stream));
+}
+
+}  // extern "C"

@@ -31,6 +31,13 @@ class _Bufs(ctypes.Structure):
     _fields_ = [("send", ctypes.POINTER(ctypes.c_void_p)), ("recv", ctypes.POINTER(ctypes.c_void_p))]
 
 
+class TraceRecord(ctypes.Structure):
+    """sim_comm_trace_record_t: one traced call."""
+    _fields_ = [("seq", ctypes.c_ulonglong), ("coll", ctypes.c_char_p), ("p", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("op", ctypes.c_int), ("root", ctypes.c_int), ("algo", ctypes.c_int), ("status", ctypes.c_int),
+                ("n", ctypes.c_ulonglong), ("launches", ctypes.c_uint), ("device_ms", ctypes.c_float)]
+
+
 def load_library(path=LIB_PATH):
     """Load libsimcomm.so and declare its signatures. Raises if it has not been built."""
     global _lib
@@ -65,6 +72,8 @@ def load_library(path=LIB_PATH):
     L.sim_comm_reset.restype = st
     L.sim_comm_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_ulonglong)]
     L.sim_comm_launch_count.restype = st
+    L.sim_comm_trace_read.argtypes = [vp, ctypes.POINTER(TraceRecord), i32, ctypes.POINTER(ctypes.c_int)]
+    L.sim_comm_trace_read.restype = st
     L.coll_allreduce.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_reduce.argtypes = [vp, _Bufs, sz, i32, i32, i32, i32, vp]
     L.coll_broadcast.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
@@ -168,6 +177,19 @@ class SimComm:
         v = ctypes.c_ulonglong()
         self._check(self._L.sim_comm_launch_count(self._h, ctypes.byref(v)))
         return v.value
+
+    def trace_read(self, cap=4096):
+        """The traced calls not read yet (option "trace" = 1), oldest first, as dicts with the fields of
+        sim_comm_trace_record_t (coll decoded to str). Waits for their events."""
+        buf = (TraceRecord * cap)()
+        got = ctypes.c_int()
+        self._check(self._L.sim_comm_trace_read(self._h, buf, cap, ctypes.byref(got)))
+        out = []
+        for r in buf[:got.value]:
+            d = {name: getattr(r, name) for name, _ in TraceRecord._fields_}
+            d["coll"] = d["coll"].decode()
+            out.append(d)
+        return out
 
     # -- marshalling -------------------------------------------------------------------------------
     def _bufs(self, sends, recvs):

@@ -133,7 +133,8 @@ const char* sim_comm_last_error(void);
 /* Name of a status code (a static string). */
 const char* coll_status_string(coll_status_t status);
 
-/* Options (also read from the environment at create time as SIMCOMM_<KEY upper-case>):
+/* Options (each also read from the environment at create time as SIMCOMM_<KEY upper-case>, e.g.
+ * SIMCOMM_CHUNK_BYTES; a value the option rejects leaves the default):
  *   "chunk_bytes"  ring pipelining chunk in bytes of the reduce-scatter wire type (default 1 MiB,
  *                  a multiple of 256, [Atlas] §3.5)
  *   "ring_ctas"    CTAs of the ring executor (0 = as many as fit on the GPU; default 0)
@@ -159,6 +160,9 @@ const char* coll_status_string(coll_status_t status);
  *   "moe_tma"      copy kernel of coll_moe_dispatch: 0 = 32/16-byte loads and stores (default,
  *                  measured faster), 1 = bulk copies through shared memory (rows of whole 16-byte
  *                  units at 16-byte aligned bases; otherwise the load/store kernel runs)
+ *   "trace"        1 = keep a record of every call (sim_comm_trace_read), 0 = off (default).
+ *                  Every entry point also opens an NVTX range named after its collective, whatever
+ *                  this option says (a no-op unless a profiler collects NVTX).
  * Returns COLL_ERR_INVALID_ARG for an unknown key or a value out of range. */
 coll_status_t sim_comm_set_option(sim_comm_t comm, const char* key, long long value);
 coll_status_t sim_comm_get_option(sim_comm_t comm, const char* key, long long* value);
@@ -178,6 +182,33 @@ coll_status_t sim_comm_reset(sim_comm_t comm);
 
 /* Kernels this communicator has launched so far (for launch accounting). */
 coll_status_t sim_comm_launch_count(sim_comm_t comm, unsigned long long* out);
+
+/* Per-call trace: the per-communicator record the [Primer] section "性能诊断第一步" asks for
+ * (collective, count, dtype, group size, duration, algorithm), so that duration percentiles per
+ * message size can be drawn from it. While option "trace" is 1 every entry-point call of this
+ * communicator is recorded, with a CUDA event recorded on the caller's stream just before the
+ * call's first kernel and one just after its last. */
+typedef struct {
+    unsigned long long seq;   /* number of the call among the traced calls of this communicator */
+    const char* coll;         /* "allreduce", "reduce", ..., "moe_combine" (a static string) */
+    int p;                    /* ranks */
+    int dtype;                /* coll_dtype_t */
+    int op;                   /* coll_op_t, or -1 where the call takes none */
+    int root;                 /* root rank, or -1 where the call takes none */
+    int algo;                 /* coll_algo_t, or -1 for the MoE calls */
+    int status;               /* coll_status_t the call returned (asynchronous errors are not here) */
+    unsigned long long n;     /* element count as passed; tokens for the MoE calls; 0 for All-to-Allv,
+                                 whose counts stay on the device */
+    unsigned int launches;    /* kernels the call enqueued */
+    float device_ms;          /* time between the two events; -1 when the call launched nothing or its
+                                 stream was being captured into a graph */
+} sim_comm_trace_record_t;
+
+/* Copies up to cap of the oldest records not read yet into out, in call order, and their number
+ * into *count. Blocks until those calls' events have completed, so read off the hot path. The
+ * communicator keeps the last 4096 traced calls; older unread records are lost (a gap in seq).
+ * COLL_ERR_INVALID_ARG for a NULL comm or count, a negative cap, or a NULL out with cap > 0. */
+coll_status_t sim_comm_trace_read(sim_comm_t comm, sim_comm_trace_record_t* out, int cap, int* count);
 
 /* ---- collectives ------------------------------------------------------------------------------ */
 

@@ -84,3 +84,26 @@ def test_binding_codes_match_the_header():
     status = header_enum("COLL_ERR_")
     status["OK"] = header_enum("COLL_")["OK"]
     assert {v: "COLL_ERR_" + k if k != "OK" else "COLL_OK" for k, v in status.items()} == SC.STATUS
+
+
+def test_trace_record_layout_matches_the_header(tmp_path):
+    """The binding's TraceRecord has the offsets and size that a C compiler gives the header's
+    sim_comm_trace_record_t."""
+    import subprocess
+    fields = [name for name, _ in SC.TraceRecord._fields_]
+    src = tmp_path / "layout.c"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    body = "".join(f'    printf("%zu ", offsetof(sim_comm_trace_record_t, {f}));\n' for f in fields)
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"simcomm.h\"\nint main(void) {\n" + body +
+                   '    printf("%zu\\n", sizeof(sim_comm_trace_record_t));\n    return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [getattr(SC.TraceRecord, f).offset for f in fields] + [ctypes.sizeof(SC.TraceRecord)]
+    assert got == want
+
+
+def test_trace_read_rejects_bad_arguments(lib):
+    L = SC.load_library()
+    count = ctypes.c_int(-1)
+    assert L.sim_comm_trace_read(None, None, 0, ctypes.byref(count)) == SC.INVALID_ARG
