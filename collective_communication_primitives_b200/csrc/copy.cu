@@ -486,6 +486,13 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     }
 }
 
+// The current device as one bit of a mask (0 for devices 63 and up, which set the attribute every launch).
+static unsigned long long device_bit() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 63) return 0;
+    return 1ull << dev;
+}
+
 // Level-table entries for the interleaved order (0 when the order is block after block).
 static int level_cap(const CopyArgs& a) { return a.order ? kMaxLevels : 0; }
 
@@ -496,12 +503,13 @@ static size_t lsu_smem_bytes(int kind, int p, int levels) {
 
 template <int KIND, bool HINT>
 static cudaError_t launch_lsu_hint(const CopyArgs& a, int num_sms, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static unsigned long long attr_set = 0;  // bit d: set on device d (a function attribute is per device)
+    const unsigned long long bit = device_bit();
+    if (!(attr_set & bit)) {
         cudaError_t e = cudaFuncSetAttribute(k_copy_lsu<KIND, HINT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(lsu_smem_bytes(KIND, kMaxRanks, kMaxLevels)));
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set |= bit;
     }
     CopyArgs b = a;
     b.level_cap = level_cap(a);
@@ -549,14 +557,15 @@ template <int KIND, int V>
 static cudaError_t launch_shape(const CopyArgs& a, int num_sms, cudaStream_t s) {
     constexpr CopyShape sh = kCopyShapes[V];
     auto kernel = k_copy<KIND, sh.stages, sh.tile>;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static unsigned long long attr_set = 0;  // bit d: set on device d
+    const unsigned long long bit = device_bit();
+    if (!(attr_set & bit)) {
         // the kernel's static shared memory (its stage slots) comes on top of the dynamic part
         const size_t want = std::min<size_t>(copy_smem_bytes(KIND, kMaxRanks, sh.stages, sh.tile, kMaxLevels),
                                              size_t(max_smem_optin()) - 1024);
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(want));
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set |= bit;
     }
     // the level table takes what the shape leaves of its share of the SM's shared memory (so the
     // shape's CTAs per SM still fit), up to kMaxLevels entries
