@@ -60,6 +60,7 @@ struct sim_comm {
     long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
+    bool capturing = false;               // the current call's stream is being captured into a graph
     long long trace = 0;                  // 1: keep a record of every call (sim_comm_trace_read)
     std::vector<TraceSlot> trace_ring;    // the last kTraceCap calls
     unsigned long long trace_seq = 0;     // calls recorded so far
@@ -182,9 +183,31 @@ void fill_ptrs(RankPtrs& rp, const coll_bufs_t& b, int p, bool use_send, bool us
 }
 
 // ---- scratch -----------------------------------------------------------------------------------
+// Scratch grows with cudaMalloc/cudaFree, which a stream capture does not allow: under capture a
+// call whose scratch is too small is refused (the same call made once before capturing sizes it).
+coll_status_t grow_in_capture(const char* what) {
+    return fail(COLL_ERR_UNSUPPORTED, std::string("the ") + what + " must grow, which a stream capture does not allow: "
+                                      "make the same call once before capturing");
+}
+
+bool stream_capturing(cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    return cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone;
+}
+
+// Flags and LL slots tell this call's signals from older ones by the epoch or tag the host gives
+// each call. A captured graph replays its call with the same epoch and tags, so under capture the
+// region the call uses is cleared first, in stream order (a memset node of the graph).
+coll_status_t clear_for_replay(sim_comm* c, void* p, size_t bytes, cudaStream_t s) {
+    if (!c->capturing || bytes == 0) return COLL_OK;
+    cudaError_t e = cudaMemsetAsync(p, 0, bytes, s);
+    return e == cudaSuccess ? COLL_OK : cuda_fail(e, "cudaMemsetAsync(scratch cleared for graph replay)");
+}
+
 
 coll_status_t ensure_flags(sim_comm* c, size_t count) {
     if (count <= c->flags_cap) return COLL_OK;
+    if (c->capturing) return grow_in_capture("ring flags");
     if (c->flags) cudaFree(c->flags);  // synchronises the device: no kernel still uses the old flags
     c->flags = nullptr;
     c->flags_cap = 0;
@@ -198,6 +221,7 @@ coll_status_t ensure_flags(sim_comm* c, size_t count) {
 
 coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
     if (bytes <= c->moe_cap) return COLL_OK;
+    if (c->capturing) return grow_in_capture("MoE scratch");
     if (c->moe) cudaFree(c->moe);  // synchronises the device: no kernel still uses the old scratch
     c->moe = nullptr;
     c->moe_cap = 0;
@@ -209,6 +233,7 @@ coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
 
 coll_status_t ensure_stage(sim_comm* c, size_t bytes) {
     if (bytes <= c->stage_cap) return COLL_OK;
+    if (c->capturing) return grow_in_capture("partial buffers");
     if (c->stage) cudaFree(c->stage);
     c->stage = nullptr;
     c->stage_cap = 0;
@@ -372,6 +397,10 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
     }
     a.flags = c->flags;
     a.epoch = next_epoch(c);
+    if (pl.kind != RING_ALLTOALL && pl.kind != RING_ALLTOALLV) {
+        st = clear_for_replay(c, c->flags, size_t(pl.nsteps) * pl.rps * pl.nch * sizeof(unsigned long long), s);
+        if (st != COLL_OK) return st;
+    }
 
     // 16-byte hops need every segment and chunk start 16-byte aligned in the element and partial
     // buffers, and 16-byte aligned bases.
@@ -401,6 +430,7 @@ coll_status_t ensure_ll_slots(sim_comm* c, size_t bytes) {
         return fail(COLL_ERR_UNSUPPORTED, "the LL protocol is for small messages: its receive slots must stay "
                                           "within 256 MiB (use COLL_ALGO_RING or COLL_ALGO_RD)");
     if (bytes <= c->ll_cap) return COLL_OK;
+    if (c->capturing) return grow_in_capture("LL slots");
     if (c->ll) cudaFree(c->ll);  // synchronises the device: no kernel still uses the old slots
     c->ll = nullptr;
     c->ll_cap = 0;
@@ -458,6 +488,8 @@ coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtyp
     coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * a.seg * sizeof(unsigned long long));
     if (st != COLL_OK) return st;
     if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    if ((st = clear_for_replay(c, c->ll, size_t(p) * a.nslots * a.seg * sizeof(unsigned long long), s)) != COLL_OK)
+        return st;
     // CTAs per rank: about 4 elements per thread, all CTAs resident at once (cooperative launch)
     const int g_cap = ll_ctas_cap(c) / p;
     if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
@@ -480,6 +512,8 @@ coll_status_t run_tree_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtyp
     coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * n * sizeof(unsigned long long));
     if (st != COLL_OK) return st;
     if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    if ((st = clear_for_replay(c, c->ll, size_t(p) * a.nslots * n * sizeof(unsigned long long), s)) != COLL_OK)
+        return st;
     const int g_cap = ll_ctas_cap(c) / p;
     if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
     a.G = int(std::max<size_t>(1, std::min<size_t>((n + 1023) / 1024, size_t(g_cap))));
@@ -513,6 +547,8 @@ coll_status_t run_rd_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_
     coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * n * sizeof(unsigned long long));
     if (st != COLL_OK) return st;
     if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
+    if ((st = clear_for_replay(c, c->ll, size_t(p) * a.nslots * n * sizeof(unsigned long long), s)) != COLL_OK)
+        return st;
     return launch_ll(c, a, dt, op, s);
 }
 
@@ -572,6 +608,8 @@ coll_status_t run_tree(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t
     if (st != COLL_OK) return st;
     a.flags = c->flags;
     a.epoch = next_epoch(c);
+    if ((st = clear_for_replay(c, c->flags, size_t(4) * p * a.nchmax * sizeof(unsigned long long), s)) != COLL_OK)
+        return st;
     a.stage_stride = round_up(n * 4, 256);
     if ((st = ensure_stage(c, a.stage_stride * size_t(p))) != COLL_OK) return st;
     a.stage = c->stage;
@@ -693,8 +731,9 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
 }
 
 // Brackets one entry-point call: an NVTX range (seen by a profiler that collects NVTX; a no-op
-// otherwise) and, while the communicator's "trace" option is on, a record of the call with CUDA
-// events around its kernels. Event timing is skipped on a stream that is being captured.
+// otherwise), notes whether the call's stream is being captured into a graph, and, while the
+// communicator's "trace" option is on, records the call with CUDA events around its kernels (not on
+// a stream that is being captured).
 struct TraceScope {
     sim_comm* c = nullptr;
     TraceSlot* slot = nullptr;
@@ -704,7 +743,9 @@ struct TraceScope {
     TraceScope(sim_comm* comm, const char* coll, size_t n, int dtype, int op, int root, int algo,
                coll_stream_t stream) {
         nvtxRangePushA(coll);
-        if (!comm || !comm->trace) return;
+        if (!comm) return;
+        comm->capturing = stream_capturing(static_cast<cudaStream_t>(stream));
+        if (!comm->trace) return;
         c = comm;
         s = static_cast<cudaStream_t>(stream);
         if (c->trace_ring.size() < kTraceCap) c->trace_ring.resize(kTraceCap);
@@ -719,8 +760,7 @@ struct TraceScope {
         slot->rec.root = root;
         slot->rec.algo = algo;
         slot->rec.device_ms = -1.0f;
-        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-        slot->timed = cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone;
+        slot->timed = !c->capturing;
         if (slot->timed && !slot->ev0)
             slot->timed = cudaEventCreate(&slot->ev0) == cudaSuccess && cudaEventCreate(&slot->ev1) == cudaSuccess;
         if (slot->timed) slot->timed = cudaEventRecord(slot->ev0, s) == cudaSuccess;

@@ -34,6 +34,12 @@
  *     All-to-Allv are never in place.
  *   - One communicator runs one collective at a time: calls on different streams must be ordered
  *     by the caller (the communicator's scratch is shared between calls).
+ *   - Calls may be captured into a CUDA graph (stream capture) and the graph replayed any number
+ *     of times, with eager calls of the same communicator in between. A captured call's scratch
+ *     must already exist: make the same call once before capturing; a call that would have to grow
+ *     the scratch under capture returns COLL_ERR_UNSUPPORTED and enqueues nothing. The schedules
+ *     whose signals carry a per-call epoch or tag (ring, tree, LL) add a memset node that clears
+ *     the flags or slots they use, so each replay starts clean.
  *
  * Errors
  *   - Synchronous (returned, nothing enqueued): COLL_ERR_INVALID_ARG (null handle or pointer, bad
