@@ -651,20 +651,20 @@ def sweep(args):
     rows = []
     for p in [int(x) for x in args.sweep_ps.split(",")]:
         comm = SC.SimComm(p)
-        algos = ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll") if p & (p - 1) == 0 else \
-            ("direct", "ring", "tree", "dbtree", "ll", "tree_ll")
+        algos = ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll", "dbtree_ll") \
+            if p & (p - 1) == 0 else ("direct", "ring", "tree", "dbtree", "ll", "tree_ll", "dbtree_ll")
         for algo in algos:
             for nbytes in sizes:
                 n = max(p, (nbytes // 4) // p * p)     # int32 elements, divisible by p
                 hold = 2 * p * n * 4 + {"direct": 0, "ring": 1, "rd": 2, "hd": 1, "tree": 1, "dbtree": 1, "ll": 0,
-                                        "rd_ll": 0, "tree_ll": 0}[algo] * p * n * 4
+                                        "rd_ll": 0, "tree_ll": 0, "dbtree_ll": 0}[algo] * p * n * 4
                 if hold > SWEEP_CAP_BYTES:
                     continue
                 if algo == "ll" and p * (2 * p - 3) * -(-n // p) * 8 > (256 << 20):
                     continue  # the LL protocol's receive slots are capped (small messages only)
                 if algo == "rd_ll" and (n > (1 << 20) // p or p * p.bit_length() * n * 8 > (256 << 20)):
                     continue  # registers of one resident grid hold the vector (small messages only)
-                if algo == "tree_ll" and p * 3 * n * 8 > (256 << 20):
+                if algo in ("tree_ll", "dbtree_ll") and p * 3 * n * 8 > (256 << 20):
                     continue  # the LL protocol's receive slots are capped (small messages only)
                 x = [torch.randint(-2**24, 2**24, (n,), dtype=torch.int32, device=dev) for _ in range(p)]
                 y = [torch.empty(n, dtype=torch.int32, device=dev) for _ in range(p)]
@@ -706,7 +706,7 @@ def sweep(args):
         comm.close()
     fits = []
     for p in sorted({r["p"] for r in rows}):
-        for algo in ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll"):
+        for algo in ("direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll", "dbtree_ll"):
             for op in SWEEP_OPS:
                 pts = [r for r in rows if r["p"] == p and r["algo"] == algo and r["op"] == op]
                 if len(pts) < 3:

@@ -96,7 +96,8 @@ coll_status_t check_algo(coll_algo_t algo, bool allreduce = false, bool ll_ring 
     if (algo == COLL_ALGO_DIRECT || algo == COLL_ALGO_RING) return COLL_OK;
     if (algo == COLL_ALGO_RING_LL && ll_ring) return COLL_OK;
     if (algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE ||
-        algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL || algo == COLL_ALGO_TREE_LL) {
+        algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RD_LL || algo == COLL_ALGO_TREE_LL ||
+        algo == COLL_ALGO_DBTREE_LL) {
         if (allreduce) return COLL_OK;
         return fail(COLL_ERR_UNSUPPORTED,
                     "recursive doubling, halving-doubling, the trees and the LL ring exist for AllReduce only");
@@ -497,9 +498,11 @@ coll_status_t run_ring_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtyp
     return launch_ll(c, a, dt, op, s);
 }
 
-// Single binary tree AllReduce on the low-latency protocol: three slots per rank (left child, right
-// child, parent), any p.
-coll_status_t run_tree_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, cudaStream_t s) {
+// Single or double binary tree AllReduce on the low-latency protocol: three slots per rank (left
+// child, right child, parent), any p. The double tree sends elements [ceil(n/2), n) over the mirror
+// tree, in CTAs of their own.
+coll_status_t run_tree_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtype_t dt, coll_op_t op, bool dbl,
+                          cudaStream_t s) {
     const int p = c->p;
     LLArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -507,16 +510,21 @@ coll_status_t run_tree_ll(sim_comm* c, const coll_bufs_t& b, size_t n, coll_dtyp
     a.kind = LL_TREE;
     a.p = p;
     a.n = n;
-    a.seg = n;
+    a.seg = dbl ? (n + 1) / 2 : n;  // elements of tree A
     a.nslots = 3;
     coll_status_t st = ensure_ll_slots(c, size_t(p) * a.nslots * n * sizeof(unsigned long long));
     if (st != COLL_OK) return st;
     if ((st = next_ll_tag(c, s, &a.tag)) != COLL_OK) return st;
     if ((st = clear_for_replay(c, c->ll, size_t(p) * a.nslots * n * sizeof(unsigned long long), s)) != COLL_OK)
         return st;
+    // CTAs per rank and tree: about 4 elements per thread, all CTAs resident at once
     const int g_cap = ll_ctas_cap(c) / p;
-    if (g_cap < 1) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
-    a.G = int(std::max<size_t>(1, std::min<size_t>((n + 1023) / 1024, size_t(g_cap))));
+    if (g_cap < (dbl ? 2 : 1)) return fail(COLL_ERR_UNSUPPORTED, "too many ranks for one resident LL grid");
+    const size_t nb = n - a.seg;
+    const int g_tree = dbl ? g_cap / 2 : g_cap;
+    a.GA = int(std::max<size_t>(1, std::min<size_t>((a.seg + 1023) / 1024, size_t(g_tree))));
+    const int gb = nb ? int(std::max<size_t>(1, std::min<size_t>((nb + 1023) / 1024, size_t(g_tree)))) : 0;
+    a.G = a.GA + gb;
     return launch_ll(c, a, dt, op, s);
 }
 
@@ -961,7 +969,8 @@ static coll_status_t coll_allreduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     if (algo == COLL_ALGO_TREE || algo == COLL_ALGO_DBTREE) return run_tree(c, b, n, dt, op, algo == COLL_ALGO_DBTREE, s);
     if (algo == COLL_ALGO_RING_LL) return run_ring_ll(c, b, n, dt, op, s);
     if (algo == COLL_ALGO_RD_LL) return run_rd_ll(c, b, n, dt, op, s);
-    if (algo == COLL_ALGO_TREE_LL) return run_tree_ll(c, b, n, dt, op, s);
+    if (algo == COLL_ALGO_TREE_LL || algo == COLL_ALGO_DBTREE_LL)
+        return run_tree_ll(c, b, n, dt, op, algo == COLL_ALGO_DBTREE_LL, s);
     RingPlan pl;
     pl.kind = RING_ALLREDUCE;
     pl.seg = (n + size_t(p) - 1) / size_t(p);

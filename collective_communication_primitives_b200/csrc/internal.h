@@ -173,8 +173,9 @@ struct LLArgs {
     int ept;                 // LL_RD: elements per thread, held in registers (1, 2, 4 or 8)
     int p;
     int G;                   // CTAs per rank
+    int GA;                  // LL_TREE: CTAs per rank on tree A's elements (the other G - GA carry tree B's)
     size_t n;                // elements per rank
-    size_t seg;              // ring segment, ceil(n / p)
+    size_t seg;              // ring segment, ceil(n / p); LL_TREE: elements of tree A (n for the single tree)
     uint32_t nslots;         // receive slots per rank: one per step that crosses a hop (ring 2p - 3, RD log2 p)
     uint32_t tag;            // this call's tag of slot 0 (slot q carries tag + q)
     float scale;

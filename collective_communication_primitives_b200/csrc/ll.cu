@@ -226,53 +226,63 @@ __global__ void __launch_bounds__(kLLThreads) k_rd_ll(const __grid_constant__ LL
 // for none), folds (own ⊕ left) ⊕ right, and sends the partial to its parent (the root instead
 // scales, rounds and writes its output); then it waits for its parent's result (the root for none),
 // writes it and forwards it to its children. Every wait is on a deeper position (reduce) or a
-// shallower one (broadcast), so no two threads wait on each other in a cycle.
+// shallower one (broadcast), so no two threads wait on each other in a cycle. The double tree
+// ([Atlas] §2.4) runs the second half of the elements over the mirror tree in CTAs of their own.
 template <int DT, int OP, bool SCALE>
 __global__ void __launch_bounds__(kLLThreads) k_tree_ll(const __grid_constant__ LLArgs a) {
     using A = typename Elem<DT>::A;
     const int p = a.p;
     const int r = int(blockIdx.x) / a.G;
-    const size_t i0 = size_t(int(blockIdx.x) % a.G) * kLLThreads + threadIdx.x;
-    const size_t stride = size_t(a.G) * kLLThreads;
+    const int g = int(blockIdx.x) % a.G;
+    // The double tree: CTAs [0, GA) of a rank carry tree A's elements [0, seg) (rank m at heap
+    // position m), the others tree B's [seg, n) (the mirror: rank m at position p - 1 - m). The single
+    // tree has GA = G and seg = n. A CTA serves one tree, so every lane of a warp holds the same
+    // position: lanes never wait on each other's sends through a warp's reconvergence.
+    const bool tb = g >= a.GA;
+    const size_t lo = tb ? a.seg : 0, hi = tb ? a.n : a.seg;
+    const size_t i0 = lo + size_t(tb ? g - a.GA : g) * kLLThreads + threadIdx.x;
+    const size_t stride = size_t(tb ? a.G - a.GA : a.GA) * kLLThreads;
     if (status_failed(a.ctl)) return;
-    const int kid0 = 2 * r + 1, kid1 = 2 * r + 2, parent = (r - 1) / 2;
+    const int pos = tb ? p - 1 - r : r;
+    auto rank_at = [&](int q) { return tb ? p - 1 - q : q; };
     const unsigned long long* mine = a.ll + size_t(r) * a.nslots * a.n;
     auto slot_of = [&](int rank, int q) { return a.ll + (size_t(rank) * a.nslots + q) * a.n; };
     const bool silent = (r == a.skip_rank);
+    const int ppos = (pos - 1) / 2;
+    const int side = (pos == 2 * ppos + 1) ? 0 : 1;  // which child of its parent this position is
     // reduce up
-    for (size_t e = i0; e < a.n; e += stride) {
+    for (size_t e = i0; e < hi; e += stride) {
         A x = load_elem<DT>(a.ptrs.send[r], e);
         for (int c = 0; c < 2; ++c) {
-            if ((c == 0 ? kid0 : kid1) >= p) break;
+            if (2 * pos + 1 + c >= p) break;
             uint32_t b;
             if (!ll_wait(a.ctl, mine + size_t(c) * a.n + e, a.tag + uint32_t(c), a.timeout_ns, &b)) return;
             if constexpr (DT == COLL_INT32) x = op_i<OP>(x, acc_of<DT>(b));
             else x = op_f<OP>(x, acc_of<DT>(b));
         }
-        if (r == 0) {
+        if (pos == 0) {
             if constexpr (SCALE) x = x * a.scale;
             const uint32_t ob = out_bits<DT>(x);
-            store_bits<DT>(a.ptrs.recv[0], e, ob);
+            store_bits<DT>(a.ptrs.recv[r], e, ob);
             for (int c = 0; c < 2; ++c) {  // the result starts down the tree
-                const int kid = (c == 0) ? kid0 : kid1;
-                if (kid < p && !silent)
-                    st_relaxed_gpu_u64(slot_of(kid, 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | ob);
+                if (1 + c < p && !silent)
+                    st_relaxed_gpu_u64(slot_of(rank_at(1 + c), 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | ob);
             }
         } else if (!silent) {
-            const int side = (r == 2 * parent + 1) ? 0 : 1;  // which child of the parent this rank is
-            st_relaxed_gpu_u64(slot_of(parent, side) + e,
+            st_relaxed_gpu_u64(slot_of(rank_at(ppos), side) + e,
                                ((unsigned long long)(a.tag + uint32_t(side)) << 32) | acc_bits<DT>(x));
         }
     }
-    if (r == 0) return;
+    if (pos == 0) return;
     // broadcast down
-    for (size_t e = i0; e < a.n; e += stride) {
+    for (size_t e = i0; e < hi; e += stride) {
         uint32_t b;
         if (!ll_wait(a.ctl, mine + size_t(2) * a.n + e, a.tag + 2u, a.timeout_ns, &b)) return;
         store_bits<DT>(a.ptrs.recv[r], e, b);
         for (int c = 0; c < 2; ++c) {
-            const int kid = (c == 0) ? kid0 : kid1;
-            if (kid < p && !silent) st_relaxed_gpu_u64(slot_of(kid, 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | b);
+            const int kp = 2 * pos + 1 + c;
+            if (kp < p && !silent)
+                st_relaxed_gpu_u64(slot_of(rank_at(kp), 2) + e, ((unsigned long long)(a.tag + 2u) << 32) | b);
         }
     }
 }

@@ -16,7 +16,8 @@ STATUS = {0: "COLL_OK", 1: "COLL_ERR_INVALID_ARG", 2: "COLL_ERR_UNSUPPORTED", 3:
 OK, INVALID_ARG, UNSUPPORTED, CUDA, TIMEOUT, ABORTED, OVERFLOW, INTERNAL = range(8)
 DTYPES = {"int32": 0, "fp32": 1, "bf16": 2}
 OPS = {"sum": 0, "min": 1, "max": 2, "avg": 3}
-ALGOS = {"direct": 0, "ring": 1, "rd": 2, "hd": 3, "tree": 4, "dbtree": 5, "ll": 6, "rd_ll": 7, "tree_ll": 8}
+ALGOS = {"direct": 0, "ring": 1, "rd": 2, "hd": 3, "tree": 4, "dbtree": 5, "ll": 6, "rd_ll": 7, "tree_ll": 8,
+         "dbtree_ll": 9}
 
 _lib = None
 

@@ -106,10 +106,12 @@ typedef enum { COLL_SUM = 0, COLL_MIN = 1, COLL_MAX = 2, COLL_AVG = 3 } coll_op_
  *         and p * log2(p) * n * 8 bytes of receive slots stay within 256 MiB (else
  *         COLL_ERR_UNSUPPORTED).
  * TREE_LL: the single binary tree (as TREE: same fold, so the same bits) on the LL protocol, any p;
- *         AllReduce only, small messages: p * 3 * n * 8 bytes of receive slots within 256 MiB. */
+ *         AllReduce only, small messages: p * 3 * n * 8 bytes of receive slots within 256 MiB.
+ * DBTREE_LL: the double binary tree (as DBTREE: same split and fold, so the same bits) on the LL
+ *         protocol, any p; AllReduce only, the same slot limit as TREE_LL. */
 typedef enum {
     COLL_ALGO_DIRECT = 0, COLL_ALGO_RING = 1, COLL_ALGO_RD = 2, COLL_ALGO_HD = 3, COLL_ALGO_TREE = 4, COLL_ALGO_DBTREE = 5,
-    COLL_ALGO_RING_LL = 6, COLL_ALGO_RD_LL = 7, COLL_ALGO_TREE_LL = 8
+    COLL_ALGO_RING_LL = 6, COLL_ALGO_RD_LL = 7, COLL_ALGO_TREE_LL = 8, COLL_ALGO_DBTREE_LL = 9
 } coll_algo_t;
 
 typedef struct {

@@ -74,7 +74,8 @@ def header_enum(prefix):
 def test_binding_codes_match_the_header():
     algos = header_enum("COLL_ALGO_")
     names = {"direct": "DIRECT", "ring": "RING", "rd": "RD", "hd": "HD", "tree": "TREE", "dbtree": "DBTREE",
-             "ll": "RING_LL", "rd_ll": "RD_LL", "tree_ll": "TREE_LL"}
+             "ll": "RING_LL", "rd_ll": "RD_LL", "tree_ll": "TREE_LL",
+             "dbtree_ll": "DBTREE_LL"}
     assert set(names.values()) == set(algos)
     for key, hname in names.items():
         assert SC.ALGOS[key] == algos[hname], key

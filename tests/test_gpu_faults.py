@@ -22,7 +22,7 @@ def run(c, kind, algo, t, u, p, n):
         c.allgather([x[:n // p] for x in t], u, algo=algo)
 
 
-CASES = [("allreduce", a) for a in ("tree", "dbtree", "rd", "hd", "ll", "rd_ll", "tree_ll")] + \
+CASES = [("allreduce", a) for a in ("tree", "dbtree", "rd", "hd", "ll", "rd_ll", "tree_ll", "dbtree_ll")] + \
         [("reduce_scatter", "ll"), ("allgather", "ll")]
 
 

@@ -13,7 +13,8 @@ from gpu_helpers import make_inputs, to_torch
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("algo", ["direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll"])
+@pytest.mark.parametrize("algo", ["direct", "ring", "rd", "hd", "tree", "dbtree", "ll", "rd_ll", "tree_ll",
+                                  "dbtree_ll"])
 def test_allreduce_graph_replays(algo):
     p, n = 8, 3 * 4096 + 40  # int32: exact, so every schedule matches the plain sum bit for bit
     c = SC.SimComm(p)

@@ -188,32 +188,35 @@ def test_ll_reduce_scatter_and_allgather_in_place():
 @pytest.mark.parametrize("p", [2, 3, 5, 8, 13, 16, 63, 64])
 @pytest.mark.parametrize("dtype", ["int32", "fp32", "bf16"])
 @pytest.mark.parametrize("op", ["sum", "max", "avg"])
-def test_tree_ll_allreduce_parity(p, dtype, op):
-    """The single binary tree on the LL protocol equals the oracle's tree fold bit for bit."""
+@pytest.mark.parametrize("algo", ["tree_ll", "dbtree_ll"])
+def test_tree_ll_allreduce_parity(p, dtype, op, algo):
+    """The single and double binary trees on the LL protocol equal the oracle's tree folds bit for
+    bit."""
     if dtype == "int32" and op == "avg":
         pytest.skip("AVG is not defined for int32")
     c = comm(p)
-    for n in (1, 7, 100, 4099) + ((70001,) if p <= 16 else ()):
+    for n in (1, 2, 3, 7, 100, 4099) + ((70001,) if p <= 16 else ()):
         ins = make_inputs("int24" if dtype == "int32" else "normal", p, n, dtype, f"trll.{p}.{n}", sigma=1e-3)
         src = [Guarded(n, dtype, fill=x) for x in ins]
         out = [Guarded(n, dtype) for _ in ins]
         for _ in range(2):
-            c.allreduce([b.t for b in src], [b.t for b in out], op=op, algo="tree_ll")
+            c.allreduce([b.t for b in src], [b.t for b in out], op=op, algo=algo)
         torch.cuda.synchronize()
         assert c.async_error() == SC.OK
-        want = O.tree_allreduce(ins, dtype, op)
+        want = O.tree_allreduce(ins, dtype, op, double_tree=(algo == "dbtree_ll"))
         for r in range(p):
             assert out[r].guards_intact() and src[r].guards_intact()
             np.testing.assert_array_equal(out[r].numpy(), want[r], err_msg=f"n={n} r={r}")
 
 
-def test_tree_ll_in_place():
+@pytest.mark.parametrize("algo", ["tree_ll", "dbtree_ll"])
+def test_tree_ll_in_place(algo):
     c = comm(5)
     n = 5 * 1001 + 2
     xs = make_inputs("normal", 5, n, "bf16", "trll.ip", sigma=1.0)
-    want = O.tree_allreduce(xs, "bf16", "avg")
+    want = O.tree_allreduce(xs, "bf16", "avg", double_tree=(algo == "dbtree_ll"))
     buf = [Guarded(n, "bf16", offset=1, fill=x) for x in xs]
-    c.allreduce([b.t for b in buf], [b.t for b in buf], op="avg", algo="tree_ll")
+    c.allreduce([b.t for b in buf], [b.t for b in buf], op="avg", algo=algo)
     torch.cuda.synchronize()
     assert c.async_error() == SC.OK
     for r in range(5):
