@@ -61,6 +61,8 @@ struct sim_comm {
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
     bool capturing = false;               // the current call's stream is being captured into a graph
+    bool captured_any = false;            // some call was captured: graphs may hold scratch pointers
+    std::vector<void*> retired;           // scratch replaced after a capture, freed at destroy
     long long trace = 0;                  // 1: keep a record of every call (sim_comm_trace_read)
     std::vector<TraceSlot> trace_ring;    // the last kTraceCap calls
     unsigned long long trace_seq = 0;     // calls recorded so far
@@ -186,6 +188,16 @@ void fill_ptrs(RankPtrs& rp, const coll_bufs_t& b, int p, bool use_send, bool us
 // ---- scratch -----------------------------------------------------------------------------------
 // Scratch grows with cudaMalloc/cudaFree, which a stream capture does not allow: under capture a
 // call whose scratch is too small is refused (the same call made once before capturing sizes it).
+// Scratch that a grown buffer replaces. A graph captured earlier keeps the old pointers in its
+// kernel arguments and memset nodes, so once any call has been captured the old buffer stays
+// allocated until the communicator is destroyed; before that it is freed at once (cudaFree
+// synchronises the device, so no kernel still uses it).
+void release_scratch(sim_comm* c, void* p) {
+    if (!p) return;
+    if (c->captured_any) c->retired.push_back(p);
+    else cudaFree(p);
+}
+
 coll_status_t grow_in_capture(const char* what) {
     return fail(COLL_ERR_UNSUPPORTED, std::string("the ") + what + " must grow, which a stream capture does not allow: "
                                       "make the same call once before capturing");
@@ -209,12 +221,13 @@ coll_status_t clear_for_replay(sim_comm* c, void* p, size_t bytes, cudaStream_t 
 coll_status_t ensure_flags(sim_comm* c, size_t count) {
     if (count <= c->flags_cap) return COLL_OK;
     if (c->capturing) return grow_in_capture("ring flags");
-    if (c->flags) cudaFree(c->flags);  // synchronises the device: no kernel still uses the old flags
+    release_scratch(c, c->flags);
     c->flags = nullptr;
     c->flags_cap = 0;
     cudaError_t e = cudaMalloc(&c->flags, count * sizeof(unsigned long long));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(ring flags)");
     e = cudaMemset(c->flags, 0, count * sizeof(unsigned long long));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();  // zeroed before any stream's next kernel
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(ring flags)");
     c->flags_cap = count;
     return COLL_OK;
@@ -223,7 +236,7 @@ coll_status_t ensure_flags(sim_comm* c, size_t count) {
 coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
     if (bytes <= c->moe_cap) return COLL_OK;
     if (c->capturing) return grow_in_capture("MoE scratch");
-    if (c->moe) cudaFree(c->moe);  // synchronises the device: no kernel still uses the old scratch
+    release_scratch(c, c->moe);
     c->moe = nullptr;
     c->moe_cap = 0;
     cudaError_t e = cudaMalloc(&c->moe, bytes);
@@ -235,7 +248,7 @@ coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
 coll_status_t ensure_stage(sim_comm* c, size_t bytes) {
     if (bytes <= c->stage_cap) return COLL_OK;
     if (c->capturing) return grow_in_capture("partial buffers");
-    if (c->stage) cudaFree(c->stage);
+    release_scratch(c, c->stage);
     c->stage = nullptr;
     c->stage_cap = 0;
     cudaError_t e = cudaMalloc(&c->stage, bytes);
@@ -432,12 +445,13 @@ coll_status_t ensure_ll_slots(sim_comm* c, size_t bytes) {
                                           "within 256 MiB (use COLL_ALGO_RING or COLL_ALGO_RD)");
     if (bytes <= c->ll_cap) return COLL_OK;
     if (c->capturing) return grow_in_capture("LL slots");
-    if (c->ll) cudaFree(c->ll);  // synchronises the device: no kernel still uses the old slots
+    release_scratch(c, c->ll);
     c->ll = nullptr;
     c->ll_cap = 0;
     cudaError_t e = cudaMalloc(&c->ll, bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(LL slots)");
     e = cudaMemset(c->ll, 0, bytes);  // tag 0 is never a live tag
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();  // zeroed before any stream's next kernel
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(LL slots)");
     c->ll_cap = bytes;
     return COLL_OK;
@@ -753,6 +767,7 @@ struct TraceScope {
         nvtxRangePushA(coll);
         if (!comm) return;
         comm->capturing = stream_capturing(static_cast<cudaStream_t>(stream));
+        if (comm->capturing) comm->captured_any = true;
         if (!comm->trace) return;
         c = comm;
         s = static_cast<cudaStream_t>(stream);
@@ -856,6 +871,7 @@ coll_status_t sim_comm_destroy(sim_comm_t c) {
     if (c->ll) cudaFree(c->ll);
     if (c->dstate) cudaFree(c->dstate);
     if (c->host_words) cudaFreeHost(c->host_words);
+    for (void* q : c->retired) cudaFree(q);
     for (TraceSlot& t : c->trace_ring) {
         if (t.ev0) cudaEventDestroy(t.ev0);
         if (t.ev1) cudaEventDestroy(t.ev1);

@@ -39,7 +39,9 @@
  *     must already exist: make the same call once before capturing; a call that would have to grow
  *     the scratch under capture returns COLL_ERR_UNSUPPORTED and enqueues nothing. The schedules
  *     whose signals carry a per-call epoch or tag (ring, tree, LL) add a memset node that clears
- *     the flags or slots they use, so each replay starts clean.
+ *     the flags or slots they use, so each replay starts clean. Once a call has been captured,
+ *     scratch that a later (larger) call replaces stays allocated until sim_comm_destroy, since a
+ *     graph may still use it; destroy the communicator only after its graphs.
  *
  * Errors
  *   - Synchronous (returned, nothing enqueued): COLL_ERR_INVALID_ARG (null handle or pointer, bad

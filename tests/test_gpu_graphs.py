@@ -120,3 +120,39 @@ def test_scratch_growth_is_refused_under_capture():
         assert torch.equal(y[0], torch.full_like(y[0], float(p)))
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("algo", ["ring", "tree", "ll"])
+def test_graph_replays_after_the_scratch_grew(algo):
+    """An eager call larger than the captured one grows the communicator's scratch; the graph still
+    holds the old buffers, which stay allocated, so its replays stay correct."""
+    p, n_small, n_big = 4, 4 * 3001, 4 * 60001
+    c = SC.SimComm(p)
+    try:
+        x = [torch.zeros(n_small, dtype=torch.int32, device="cuda") for _ in range(p)]
+        y = [torch.zeros(n_small, dtype=torch.int32, device="cuda") for _ in range(p)]
+        c.allreduce(x, y, algo=algo)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            c.allreduce(x, y, algo=algo)
+        big_in = make_inputs("int24", p, n_big, "int32", f"graph.grow.{algo}")
+        bx = [to_torch(a, "int32") for a in big_in]
+        by = [torch.empty_like(t) for t in bx]
+        c.allreduce(bx, by, algo=algo)  # grows the flags / partials / slots
+        torch.cuda.synchronize()
+        assert c.async_error() == SC.OK
+        np.testing.assert_array_equal(by[1].cpu().numpy(), O.allreduce(big_in, "int32", "sum")[1])
+        for it in range(2):
+            ins = make_inputs("int24", p, n_small, "int32", f"graph.grow.{algo}.{it}")
+            for r in range(p):
+                x[r].copy_(to_torch(ins[r], "int32"))
+            g.replay()
+            torch.cuda.synchronize()
+            assert c.async_error() == SC.OK
+            want = O.allreduce(ins, "int32", "sum")
+            for r in range(p):
+                np.testing.assert_array_equal(y[r].cpu().numpy(), want[r])
+        del g
+    finally:
+        c.close()
