@@ -186,8 +186,6 @@ void fill_ptrs(RankPtrs& rp, const coll_bufs_t& b, int p, bool use_send, bool us
 }
 
 // ---- scratch -----------------------------------------------------------------------------------
-// Scratch grows with cudaMalloc/cudaFree, which a stream capture does not allow: under capture a
-// call whose scratch is too small is refused (the same call made once before capturing sizes it).
 // Scratch that a grown buffer replaces. A graph captured earlier keeps the old pointers in its
 // kernel arguments and memset nodes, so once any call has been captured the old buffer stays
 // allocated until the communicator is destroyed; before that it is freed at once (cudaFree
@@ -198,6 +196,8 @@ void release_scratch(sim_comm* c, void* p) {
     else cudaFree(p);
 }
 
+// Scratch grows with cudaMalloc/cudaFree, which a stream capture does not allow: under capture a
+// call whose scratch is too small is refused (the same call made once before capturing sizes it).
 coll_status_t grow_in_capture(const char* what) {
     return fail(COLL_ERR_UNSUPPORTED, std::string("the ") + what + " must grow, which a stream capture does not allow: "
                                       "make the same call once before capturing");
