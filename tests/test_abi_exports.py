@@ -50,10 +50,28 @@ def test_status_strings(lib):
 
 
 def test_null_communicator_is_rejected_without_a_gpu(lib):
+    """Every entry point that takes a communicator refuses a NULL one before touching the device."""
     L = SC.load_library()
     bufs = SC._Bufs()
     assert L.coll_allreduce(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_reduce(None, bufs, 16, 1, 0, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_broadcast(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_reduce_scatter(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_allgather(None, bufs, 16, 1, 0, None) == SC.INVALID_ARG
+    assert L.coll_alltoall(None, bufs, 16, 1, 0, None) == SC.INVALID_ARG
+    assert L.coll_scatter(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
+    assert L.coll_gather(None, bufs, 16, 1, 0, 0, None) == SC.INVALID_ARG
     assert L.coll_alltoallv(None, bufs, None, None, None, 1, 0, None, None) == SC.INVALID_ARG
+    assert L.coll_moe_dispatch(None, None, None, 4, 2, 8, 4, 2, None, 16, None, None, None, None) == SC.INVALID_ARG
+    assert L.coll_moe_combine(None, None, 16, None, None, None, None, 4, 2, 8, 4, 2, None, None) == SC.INVALID_ARG
+    v = ctypes.c_longlong()
+    assert L.sim_comm_set_option(None, b"trace", 1) == SC.INVALID_ARG
+    assert L.sim_comm_get_option(None, b"trace", ctypes.byref(v)) == SC.INVALID_ARG
+    st = ctypes.c_int()
+    assert L.sim_comm_get_async_error(None, ctypes.byref(st)) == SC.INVALID_ARG
+    assert L.sim_comm_reset(None) == SC.INVALID_ARG
+    n = ctypes.c_ulonglong()
+    assert L.sim_comm_launch_count(None, ctypes.byref(n)) == SC.INVALID_ARG
     assert L.sim_comm_size(None) == -1
     assert L.sim_comm_destroy(None) == SC.OK
     assert L.sim_comm_abort(None) == SC.INVALID_ARG
