@@ -126,3 +126,13 @@ def test_trace_read_rejects_bad_arguments(lib):
     L = SC.load_library()
     count = ctypes.c_int(-1)
     assert L.sim_comm_trace_read(None, None, 0, ctypes.byref(count)) == SC.INVALID_ARG
+
+
+def test_noalloc_entry_checks_its_arguments_without_a_gpu(lib):
+    L = SC.load_library()
+    bufs = SC._Bufs()
+    assert L.coll_allreduce_ring_noalloc(1, bufs, 16, 1, 0, None, None) == SC.INVALID_ARG
+    assert b"p must be" in L.sim_comm_last_error()
+    assert L.coll_allreduce_ring_noalloc(65, bufs, 16, 1, 0, None, None) == SC.INVALID_ARG
+    assert L.coll_allreduce_ring_noalloc(4, bufs, 16, 7, 0, None, None) == SC.INVALID_ARG
+    assert L.coll_allreduce_ring_noalloc(4, bufs, 16, SC.DTYPES["int32"], SC.OPS["avg"], None, None) == SC.UNSUPPORTED
