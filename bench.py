@@ -8,7 +8,12 @@ values. One step runs every row of the hot path once on it:
   bucket's shards, equal All-to-All, and All-to-Allv of the bucket as 6,400 rows of 4,096 elements
   routed by a seeded top-2 / Zipf(1.1) router over 64 experts.
 value = Σ (minimum HBM bytes of each call: every input read once, every output written once) /
-device time of the step, summed over ranks (replicas) for N GPUs.
+device time of the step, summed over ranks (replicas) for N GPUs. The rows run back to back, so a
+row's dirty L2 lines drain during the next row; each row is therefore also timed alone on a clean
+L2 with its own write-back charged to it (per_op ms_attributed), and the direct rows are summed
+on their own (direct_only). The ZeRO-shard (ReduceScatter of 256 Mi bf16 per rank, AllGather of
+32 Mi-element bf16 shards) and MoE All-to-All (8,192 x 4,096 bf16 per rank, equal and top-2 /
+Zipf counts) workloads are timed the same way in the `configs` block.
 
 Prints one JSON line. ``--impl reference`` times the CPU oracle on a bounded sample instead.
 """
@@ -60,6 +65,15 @@ def parse():
                     help="time only the MoE dispatch and combine on the MoE workload (one GPU)")
     ap.add_argument("--no-moe", action="store_true", help="leave the MoE block out of the step's line")
     ap.add_argument("--moe-tokens", type=int, default=8192, help="tokens per rank of the MoE layer (--moe)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave the ZeRO-shard and MoE All-to-All blocks out of the step's line")
+    ap.add_argument("--ceilings", action="store_true",
+                    help="measure the HBM ceilings of the kernels' access patterns (load, store, copy, bulk "
+                         "store) instead of the step (one GPU)")
+    ap.add_argument("--ceilings-bytes", type=int, default=2 << 30, help="bytes each ceiling probe streams")
+    ap.add_argument("--ceilings-out", default="", help="write the ceilings' markdown summary here")
+    ap.add_argument("--no-attr", action="store_true",
+                    help="skip the per-row timing with each row's write-back charged to it")
     return ap.parse_args()
 
 
@@ -277,6 +291,58 @@ def time_device(ops, steps, warmup, stream):
     return total_ms, per_op
 
 
+FLUSH_BYTES = 256 << 20  # twice the 126 MB L2: reading it evicts every line an earlier kernel left
+
+
+class L2Flush:
+    """A read-only pass over FLUSH_BYTES (a torch reduction): every line an earlier kernel left in
+    L2, its dirty output lines included, is evicted, and a dirty line's write-back is paid inside
+    this pass. It writes nothing large itself, so it leaves only clean lines behind."""
+
+    def __init__(self, device):
+        import torch
+        self.buf = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.out = torch.empty((), dtype=torch.float32, device=device)
+
+    def __call__(self):
+        import torch
+        torch.sum(self.buf, 0, out=self.out)
+
+
+def time_attributed(ops, steps, warmup, stream, flush):
+    """Per-row device time with the row's own HBM write-back charged to it: each row runs on a clean
+    L2 (after a flush) and is followed, inside its own event pair, by a flush that writes back the
+    dirty lines the row left. The flush's own time on a clean L2 (median of as many runs) is
+    subtracted. Returns (per-row ms, flush ms)."""
+    import torch
+    for _ in range(warmup):
+        for op in ops:
+            op[2]()
+            flush()
+    reps = max(steps, 5)
+    fl = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
+          for _ in range(steps)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(SPACER_CYCLES)
+    flush()
+    for e0, e1 in fl:
+        e0.record(stream)
+        flush()
+        e1.record(stream)
+    for s in range(steps):
+        for i, op in enumerate(ops):
+            ev[s][i][0].record(stream)
+            op[2]()
+            flush()
+            ev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    flush_ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in fl)
+    per_op = [sum(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)) / steps - flush_ms
+              for i in range(len(ops))]
+    return per_op, flush_ms
+
+
 def time_e2e(comm, wl, make_ops, steps, warmup, stream, device):
     """The step through the public API with host buffers: every step copies all its inputs in from
     pinned host memory and both AllReduce results out, inside the timed region. Two buffer sets make
@@ -473,6 +539,107 @@ def moe_main(args):
         out["cpu_baseline"] = moe_cpu_baseline()
     print(json.dumps(out))
     comm.close()
+
+
+# ---------------------------------------------------------------------------------------------
+# The ZeRO-shard and MoE All-to-All workloads: every row timed with its own write-back charged
+
+ZERO_N = 256 << 20            # bf16 elements per rank of the ZeRO partial-gradient tensor (512 MiB)
+A2A_TOKENS = 8192             # tokens per rank of the MoE equal All-to-All
+
+
+def device_normal(shape, sigma, gen, device):
+    """Seeded N(0, sigma) bf16 drawn on the device (the values do not change a copy's or a
+    reduction's time; the parity tests draw the same shapes from the counter-based host generator)."""
+    import torch
+    x = torch.empty(shape, dtype=torch.float32, device=device)
+    x.normal_(0.0, sigma, generator=gen)
+    return x.to(torch.bfloat16)
+
+
+def zero_block(comm, steps, warmup, stream, flush, hbm, device):
+    """ZeRO/FSDP shards: ReduceScatter of a 256 Mi-element bf16 partial gradient per rank (N(0,1e-2))
+    to 32 Mi-element owner shards, then AllGather of 32 Mi-element bf16 parameter shards (N(0,0.02))
+    back to 256 Mi per rank; direct and ring."""
+    import torch
+
+    from collective_communication_primitives_b200 import bytemodel as BM
+    p, n = P, ZERO_N
+    m = n // p
+    gen = torch.Generator(device=device)
+    gen.manual_seed(3)
+    grads = [device_normal(n, 1e-2, gen, device) for _ in range(p)]
+    params = [device_normal(m, 0.02, gen, device) for _ in range(p)]
+    shards = [torch.empty(m, dtype=torch.bfloat16, device=device) for _ in range(p)]
+    full = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(p)]
+    ops = []
+    for algo in ("direct", "ring"):
+        ops.append((f"reduce_scatter_sum_bf16_{algo}", algo,
+                    lambda a=algo: comm.reduce_scatter(grads, shards, op="sum", algo=a),
+                    BM.direct_hbm_bytes("reduce_scatter", p, n, 2),
+                    BM.ring_hbm_bytes("reduce_scatter", p, n, 2, 4) if algo == "ring"
+                    else BM.direct_hbm_bytes("reduce_scatter", p, n, 2)))
+        ops.append((f"allgather_bf16_{algo}", algo, lambda a=algo: comm.allgather(params, full, algo=a),
+                    BM.direct_hbm_bytes("allgather", p, n, 2),
+                    BM.ring_hbm_bytes("allgather", p, n, 2) if algo == "ring"
+                    else BM.direct_hbm_bytes("allgather", p, n, 2)))
+    blk = {"workload": f"ZeRO shards, p={p} ranks: ReduceScatter of {n} bf16 per rank to {m}-element shards; "
+                       f"AllGather of {m}-element bf16 shards to {n} per rank",
+           "l2": "each row on a clean L2 and followed, inside its own timing, by a read of 256 MiB that writes "
+                 "back its dirty lines; that read's clean-L2 time subtracted"}
+    blk.update(attributed_rows(ops, steps, warmup, stream, flush, hbm))
+    del grads, params, shards, full
+    torch.cuda.empty_cache()
+    return blk
+
+
+def moe_a2a_block(comm, steps, warmup, stream, flush, hbm, device):
+    """MoE dispatch All-to-All: 8,192 tokens x 4,096 bf16 (N(0,1)) per rank, equal split (1,024
+    tokens per destination), and the uneven All-to-Allv whose per-destination counts come from the
+    seeded top-2 / Zipf(1.1) router over 64 experts (16,384 rows per rank); direct and ring."""
+    import torch
+
+    from collective_communication_primitives_b200 import bytemodel as BM
+    from collective_communication_primitives_b200 import synth as S
+    p, H = P, HIDDEN
+    n = A2A_TOKENS * H
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4)
+    x = [device_normal(n, 1.0, gen, device) for _ in range(p)]
+    y = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(p)]
+    rows = S.moe_counts(p=p, tokens=A2A_TOKENS, experts=64, topk=2, zipf_s=1.1, hidden=1)
+    counts_host = rows * H
+    counts = torch.from_numpy(counts_host).to(device)
+    v_send = [device_normal(int(counts_host[i].sum()), 1.0, gen, device) for i in range(p)]
+    v_recv = [torch.empty(int(counts_host[:, j].sum()), dtype=torch.bfloat16, device=device) for j in range(p)]
+    moved = int(counts_host.sum())
+    ops = []
+    for algo in ("direct", "ring"):
+        ops.append((f"alltoall_bf16_{algo}", algo, lambda a=algo: comm.alltoall(x, y, algo=a),
+                    BM.direct_hbm_bytes("alltoall", p, n, 2), BM.direct_hbm_bytes("alltoall", p, n, 2)))
+        ops.append((f"alltoallv_bf16_{algo}", algo, lambda a=algo: comm.alltoallv(v_send, v_recv, counts, algo=a),
+                    BM.direct_hbm_bytes("alltoallv", p, 0, 2, moved_elems=moved),
+                    BM.direct_hbm_bytes("alltoallv", p, 0, 2, moved_elems=moved)))
+    blk = {"workload": f"MoE dispatch All-to-All, p={p} ranks x {A2A_TOKENS} tokens x {H} bf16: equal split "
+                       f"({A2A_TOKENS // p} tokens per destination) and All-to-Allv on top-2 / Zipf(1.1) counts over "
+                       f"64 experts", "alltoallv_rows": dict(S.count_matrix_stats(rows), total=int(rows.sum())),
+           "l2": "as zero_shards"}
+    blk.update(attributed_rows(ops, steps, warmup, stream, flush, hbm))
+    del x, y, v_send, v_recv
+    torch.cuda.empty_cache()
+    return blk
+
+
+def attributed_rows(ops, steps, warmup, stream, flush, hbm):
+    per_op, flush_ms = time_attributed(ops, steps, warmup, stream, flush)
+    rows = {}
+    for (name, algo, _, eff, kb), ms in zip(ops, per_op):
+        rows[name] = {"ms": round(ms, 4), "effective_GBps": round(eff / (ms / 1e3) / 1e9, 1),
+                      "kernel_GBps": round(kb / (ms / 1e3) / 1e9, 1),
+                      "frac_of_measured_peak": round(kb / (ms / 1e3) / 1e9 / hbm, 4),
+                      "frac_of_nominal_8TBps": round(kb / (ms / 1e3) / 1e9 / 8000.0, 4),
+                      "minimum_bytes": int(eff), "model_bytes": int(kb)}
+    return {"rows": rows, "flush_ms": round(flush_ms, 4)}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -758,6 +925,70 @@ def write_sweep_md(path, rows, fits):
 
 
 # ---------------------------------------------------------------------------------------------
+# HBM ceilings of the access patterns the kernels use
+
+def ceilings(args):
+    """Each access pattern of the library's kernels alone (sim_hbm_probe) over a buffer 16x the L2,
+    at several CTAs per SM; plus torch's copy_ (the measured peak's own method) for reference.
+    GB/s counts every byte read plus every byte written, best of 5 launches after 2 warm-ups."""
+    import torch
+
+    from collective_communication_primitives_b200 import simcomm as SC
+    torch.cuda.set_device(0)
+    dev = "cuda:0"
+    nb = args.ceilings_bytes // (16 << 10) * (16 << 10)
+    src = torch.ones(nb // 4, dtype=torch.float32, device=dev)
+    dst = torch.empty(nb // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    hbm, peak_kind = peaks()
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    rows = []
+    with ClockSampler(0) as clk:
+        for kind in ("load", "store", "copy", "bulk_store"):
+            moved = nb * (2 if kind == "copy" else 1)
+            for cps in ((1, 2, 4, 8) if kind != "bulk_store" else (1, 2, 4, 8, 12)):
+                ms = timed(lambda: SC.hbm_probe(kind, dst if kind != "load" else None,
+                                                src if kind in ("load", "copy") else None, nb, cps))
+                rows.append({"pattern": kind, "ctas_per_sm": cps, "bytes_moved": moved, "ms": round(ms, 4),
+                             "GBps": round(moved / (ms / 1e3) / 1e9, 1)})
+        ms = timed(lambda: dst.copy_(src))
+        rows.append({"pattern": "torch copy_", "ctas_per_sm": None, "bytes_moved": 2 * nb, "ms": round(ms, 4),
+                     "GBps": round(2 * nb / (ms / 1e3) / 1e9, 1)})
+        ms = timed(lambda: dst.fill_(2.0))
+        rows.append({"pattern": "torch fill_", "ctas_per_sm": None, "bytes_moved": nb, "ms": round(ms, 4),
+                     "GBps": round(nb / (ms / 1e3) / 1e9, 1)})
+    best = {}
+    for r in rows:
+        if r["pattern"] not in best or r["GBps"] > best[r["pattern"]]["GBps"]:
+            best[r["pattern"]] = r
+    out = {"ceilings": {k: {"GBps": v["GBps"], "ctas_per_sm": v["ctas_per_sm"], "frac_of_measured": round(v["GBps"] / hbm, 4)}
+                        for k, v in best.items()},
+           "peak": hbm, "peak_source": peak_kind, "bytes": nb, "rows": rows, "clocks": clk.summary()}
+    print(json.dumps(out))
+    if args.ceilings_out:
+        lines = [f"| pattern | CTAs per SM | GB/s (read + written) | of measured {hbm:.1f} GB/s |",
+                 "|---|---:|---:|---:|"]
+        for r in rows:
+            lines.append(f"| {r['pattern']} | {r['ctas_per_sm'] if r['ctas_per_sm'] else '-'} | {r['GBps']:.1f} | "
+                         f"{r['GBps'] / hbm:.3f} |")
+        with open(args.ceilings_out, "w") as fh:
+            fh.write("\n".join(lines) + "\n")
+
 
 def main():
     args = parse()
@@ -769,6 +1000,9 @@ def main():
         return
     if args.moe:
         moe_main(args)
+        return
+    if args.ceilings:
+        ceilings(args)
         return
     import torch
     import torch.distributed as dist
@@ -830,11 +1064,34 @@ def main():
     hbm, peak_kind = peaks()
     ms_per_step = total_ms / args.steps
     value = job_gbps(world, eff_per_step, ms_per_step)
+    # Each row again, on a clean L2 and charged with its own write-back (the back-to-back times above
+    # let a row's dirty lines drain during the next row).
+    flush = L2Flush(device)
+    attr = None
+    if not args.no_attr:
+        attr, flush_ms = time_attributed(ops, args.steps, args.warmup, stream, flush)
     per_op_json = {}
-    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
+    for i, ((name, kernel, _, eff, kb), ms) in enumerate(zip(ops, per_op)):
         per_op_json[name] = {"ms": round(ms, 4), "effective_GBps": round(eff / (ms / 1e3) / 1e9, 1),
                              "kernel_GBps": round(kb / (ms / 1e3) / 1e9, 1),
                              "frac_of_measured_peak": round(kb / (ms / 1e3) / 1e9 / hbm, 4)}
+        if attr:
+            a = attr[i]
+            per_op_json[name].update({"ms_attributed": round(a, 4), "kernel_GBps_attributed": round(kb / (a / 1e3) / 1e9, 1),
+                                      "frac_attributed": round(kb / (a / 1e3) / 1e9 / hbm, 4)})
+    # The direct rows alone (the collective's minimum bytes over the direct kernels' time).
+    d_idx = [i for i, o in enumerate(ops) if o[0].endswith("_direct")]
+    direct_only = None
+    if d_idx:
+        d_bytes = sum(ops[i][3] for i in d_idx)
+        d_ms = sum(per_op[i] for i in d_idx)
+        direct_only = {"value": round(job_gbps(world, d_bytes, d_ms), 1), "unit": "GB/s",
+                       "ms_per_step": round(d_ms, 4), "rows": len(d_idx),
+                       "timing": "back to back, as the step"}
+        if attr:
+            a_ms = sum(attr[i] for i in d_idx)
+            direct_only.update({"value_attributed": round(job_gbps(world, d_bytes, a_ms), 1),
+                                "ms_per_step_attributed": round(a_ms, 4)})
     # The dominant kernel: each row is one launch of one kernel, so the row with the largest share
     # of the step's device time names it. achieved = that kernel's algorithmic bytes per launch (its
     # byte model: the minimum for direct rows; for ring rows the schedule's hop traffic, every hop
@@ -854,14 +1111,28 @@ def main():
                 "traffic": traffic, "algorithmic_bytes_per_launch": int(kb),
                 "minimum_bytes_per_launch": int(eff),
                 "share_of_step": round(d_ms / sum(per_op), 4), "ms_per_launch": round(d_ms, 4)}
-    # The four direct kernels the throughput target names (>= 80% of the ~8 TB/s nominal peak).
+    # The four direct kernels the throughput target names (>= 80% of the ~8 TB/s nominal peak at
+    # >= 64 MB per rank), on every workload that runs them: each row charged with its own write-back
+    # where that timing ran (else back to back).
     target = {}
-    for (nm, kernel, _, eff, kb), ms in zip(ops, per_op):
+    for i, ((nm, kernel, _, eff, kb), ms) in enumerate(zip(ops, per_op)):
         if nm in ("allreduce_avg_fp32_direct", "allreduce_avg_bf16_direct", "reduce_scatter_sum_fp32_direct",
                   "allgather_fp32_direct", "alltoall_fp32_direct"):
-            g = kb / (ms / 1e3) / 1e9
-            target[nm] = {"GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
-                        "frac_of_nominal_8TBps": round(g / 8000.0, 4)}
+            t = attr[i] if attr else ms
+            g = kb / (t / 1e3) / 1e9
+            target["dp_bucket." + nm] = {"GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
+                                         "frac_of_nominal_8TBps": round(g / 8000.0, 4),
+                                         "back_to_back_GBps": round(kb / (ms / 1e3) / 1e9, 1)}
+    configs = {}
+    if not args.no_configs and not args.ops and args.n == N_BUCKET:
+        configs["zero_shards"] = zero_block(comm, args.steps, args.warmup, stream, flush, hbm, device)
+        configs["moe_alltoall"] = moe_a2a_block(comm, args.steps, args.warmup, stream, flush, hbm, device)
+        for cname, blk in configs.items():
+            for nm, row in blk["rows"].items():
+                if nm.endswith("_direct") and nm.split("_")[0] in ("reduce", "allgather", "alltoall"):
+                    target[f"{cname}.{nm}"] = {"GBps": row["kernel_GBps"], "frac_of_measured": row["frac_of_measured_peak"],
+                                               "frac_of_nominal_8TBps": row["frac_of_nominal_8TBps"]}
+    del flush
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -869,6 +1140,7 @@ def main():
         "vs_baseline": None, "dtype": "fp32+bf16 (fp32 accumulate)", "data": "synthetic",
         "config": step_config(args.n, world, [o[0] for o in ops], args.option),
         "roofline": roofline,
+        "direct_only": direct_only,
         "target_direct": target,
         "per_op": per_op_json,
         "gpu_launches": int(launches),
@@ -876,6 +1148,13 @@ def main():
     }
     if e2e:
         out["e2e"] = e2e
+    if attr:
+        out["attribution"] = {"flush_bytes": FLUSH_BYTES, "flush_ms_clean": round(flush_ms, 4),
+                              "how": "per row: clean L2, the row, a read of flush_bytes that writes back the "
+                                     "row's dirty lines, all inside the row's events; the read's clean-L2 time "
+                                     "subtracted"}
+    if configs:
+        out["configs"] = configs
     if not args.no_moe and not args.ops:
         mw = MoeWorkload(device)
         out["moe"] = moe_block(comm, mw, max(3, args.steps // 2), args.warmup, stream, hbm,

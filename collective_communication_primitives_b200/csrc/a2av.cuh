@@ -49,7 +49,9 @@ __device__ inline A2avPlan a2av_plan_warp(const long long* counts, int p, const 
         for (int j0 = 0; j0 < p; j0 += 32) {
             const int j = j0 + lane;
             const long long v = (j < p) ? counts[i * p + j] : 0;
-            if (v < 0) bad = true;
+            // a count above its row's capacity fails on its own, so with capacities at most 2^48
+            // (checked on the host) no row or column sum below can wrap around
+            if (v < 0 || v > send_cap[i]) bad = true;
             mx = max(mx, v);
             const long long incl = warp_inclusive_scan(v, lane);
             if (j < p) sd[i * p + j] = carry + incl - v;
@@ -63,6 +65,7 @@ __device__ inline A2avPlan a2av_plan_warp(const long long* counts, int p, const 
         for (int i0 = 0; i0 < p; i0 += 32) {
             const int i = i0 + lane;
             const long long v = (i < p) ? counts[i * p + j] : 0;
+            if (v > recv_cap[j]) bad = true;
             const long long incl = warp_inclusive_scan(v, lane);
             if (i < p) rd[i * p + j] = carry + incl - v;
             carry += __shfl_sync(0xFFFFFFFFu, incl, 31);

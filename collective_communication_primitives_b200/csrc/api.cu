@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <cctype>
+#include <climits>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -176,6 +177,33 @@ coll_status_t check_ptr(const void* p, size_t bytes, size_t elem, const char* wh
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Largest element count, capacity or row count x row length any entry point accepts. At 2^48
+// elements every byte count and offset the host or a kernel forms (a count x an element of at most
+// 8 bytes x 64 ranks, or a partial buffer of 4 bytes per element per rank) stays below 2^63, so no
+// size computation can wrap around; a wrapped size would pass the pointer and scratch checks with a
+// false small value. Checked before any multiplication.
+constexpr size_t kMaxCount = size_t(1) << 48;
+
+coll_status_t check_count(size_t n, const char* what) {
+    if (n > kMaxCount)
+        return fail(COLL_ERR_INVALID_ARG, std::string(what) + " exceeds 2^48 elements (" + std::to_string(n) + ")");
+    return COLL_OK;
+}
+
+// A probe moves whole 16 KiB tiles, at most 2^48 bytes.
+coll_status_t check_probe_bytes(size_t bytes) {
+    if (bytes % (16 * 1024) != 0 || bytes > kMaxCount)
+        return fail(COLL_ERR_INVALID_ARG, "probe bytes must be a multiple of 16 KiB, at most 2^48");
+    return COLL_OK;
+}
+
+// rows x row length within kMaxCount, without forming the product first
+coll_status_t check_rows(size_t rows, size_t row_elems, const char* what) {
+    if (row_elems != 0 && rows > kMaxCount / row_elems)
+        return fail(COLL_ERR_INVALID_ARG, std::string(what) + ": rows x hidden exceeds 2^48 elements");
+    return COLL_OK;
+}
 
 void fill_ptrs(RankPtrs& rp, const coll_bufs_t& b, int p, bool use_send, bool use_recv) {
     std::memset(&rp, 0, sizeof(rp));
@@ -351,9 +379,20 @@ constexpr size_t kRingTaskBytes = 256 * 1024;  // bytes of the wire type one rin
 // Task size of the ring and tree executors. Measured on B200 (p = 2..64): 256 KiB tasks are 2-6%
 // faster than 128 KiB ones from 64 MiB of wire bytes per rank up, and 10-50% slower at 1-16 MiB,
 // where the schedule needs more, shorter tasks per step to keep its pipeline full.
+size_t default_task_bytes(size_t wire_bytes_per_rank) {
+    return wire_bytes_per_rank >= (size_t(64) << 20) ? kRingTaskBytes : kRingTaskBytes / 2;
+}
+
 size_t task_bytes(const sim_comm* c, size_t wire_bytes_per_rank) {
     if (c->ring_task_bytes > 0) return size_t(c->ring_task_bytes);
-    return wire_bytes_per_rank >= (size_t(64) << 20) ? kRingTaskBytes : kRingTaskBytes / 2;
+    return default_task_bytes(wire_bytes_per_rank);
+}
+
+// CTA tasks of one ring chunk: a chunk spans at most `span` elements (a segment), and one task moves
+// `task` bytes of the wire type (at least 16 elements).
+void ring_tiles(size_t span, size_t wire, size_t task, size_t* tile, uint32_t* ntile) {
+    *tile = std::min(span, std::max<size_t>(16, task / wire));
+    *ntile = uint32_t((span + *tile - 1) / *tile);
 }
 
 coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, size_t n, coll_dtype_t dt,
@@ -379,8 +418,7 @@ coll_status_t run_ring(sim_comm* c, const coll_bufs_t& b, const RingPlan& pl, si
         size_t per_rank = n * wire;  // the All-to-Allv's largest send buffer stands in for its message
         if (pl.kind == RING_ALLTOALLV && send_cap)
             for (int r = 0; r < p; ++r) per_rank = std::max(per_rank, size_t(std::max<long long>(send_cap[r], 0)) * d);
-        a.tile = std::min(span, std::max<size_t>(16, task_bytes(c, per_rank) / wire));
-        a.ntile = uint32_t((span + a.tile - 1) / a.tile);
+        ring_tiles(span, wire, task_bytes(c, per_rank), &a.tile, &a.ntile);
     }
     a.elem_bytes = int(d);
     a.nch = pl.nch;
@@ -967,6 +1005,7 @@ static coll_status_t coll_allreduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     if ((algo == COLL_ALGO_RD || algo == COLL_ALGO_HD || algo == COLL_ALGO_RD_LL) && (c->p & (c->p - 1)))
         return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling need p a power of two");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const int p = c->p;
     const size_t d = dtype_bytes(dt), bytes = n * d;
@@ -1006,6 +1045,7 @@ static coll_status_t coll_reduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, col
     const int p = c->p;
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), bytes = n * d;
     std::vector<Range> rs;
@@ -1042,6 +1082,7 @@ static coll_status_t coll_broadcast_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     const int p = c->p;
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), bytes = n * d;
     std::vector<Range> rs;
@@ -1076,6 +1117,7 @@ static coll_status_t coll_reduce_scatter_impl(sim_comm_t c, coll_bufs_t b, size_
     const int p = c->p;
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "ReduceScatter needs n divisible by p");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1109,6 +1151,7 @@ static coll_status_t coll_allgather_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     const int p = c->p;
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "AllGather needs n divisible by p");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1142,6 +1185,7 @@ static coll_status_t coll_alltoall_impl(sim_comm_t c, coll_bufs_t b, size_t n, c
     const int p = c->p;
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "All-to-All needs n divisible by p");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1176,6 +1220,7 @@ static coll_status_t coll_scatter_impl(sim_comm_t c, coll_bufs_t b, size_t n, co
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Scatter needs n divisible by p");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1203,6 +1248,7 @@ static coll_status_t coll_gather_impl(sim_comm_t c, coll_bufs_t b, size_t n, col
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Gather needs n divisible by p");
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1236,6 +1282,9 @@ static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long
     std::vector<Range> rs;
     for (int r = 0; r < p; ++r) {
         if (send_cap[r] < 0 || recv_cap[r] < 0) return fail(COLL_ERR_INVALID_ARG, "negative capacity");
+        if ((st = check_count(size_t(send_cap[r]), "send_cap")) != COLL_OK ||
+            (st = check_count(size_t(recv_cap[r]), "recv_cap")) != COLL_OK)
+            return st;
         const size_t sb = size_t(send_cap[r]) * d, rb = size_t(recv_cap[r]) * d;
         if ((st = check_ptr(b.send[r], sb, d, "send")) != COLL_OK) return st;
         if ((st = check_ptr(b.recv[r], rb, d, "recv")) != COLL_OK) return st;
@@ -1270,8 +1319,9 @@ coll_status_t check_moe_shape(sim_comm* c, size_t tokens, int k, size_t hidden, 
     if (experts < p || experts % p != 0 || experts > kMoeMaxExperts)
         return fail(COLL_ERR_INVALID_ARG, "experts must be a multiple of p in [p, 4096]");
     if (hidden == 0) return fail(COLL_ERR_INVALID_ARG, "hidden must be positive");
+    if (check_count(hidden, "hidden") != COLL_OK) return COLL_ERR_INVALID_ARG;
     if (tokens > size_t(INT32_MAX) / size_t(k)) return fail(COLL_ERR_INVALID_ARG, "tokens * k must fit in int32");
-    return COLL_OK;
+    return check_rows(tokens, hidden, "tokens");
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -1290,6 +1340,7 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
     if (recv_cap_rows > size_t(INT32_MAX)) return fail(COLL_ERR_INVALID_ARG, "recv_cap_rows must fit in int32");
+    if ((st = check_rows(recv_cap_rows, hidden, "recv_cap_rows")) != COLL_OK) return st;
     if (!x || !topk_idx || !recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     if ((expert_counts_dev && reinterpret_cast<uintptr_t>(expert_counts_dev) % 8 != 0) ||
         (recv_counts_dev && reinterpret_cast<uintptr_t>(recv_counts_dev) % 8 != 0))
@@ -1366,6 +1417,7 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if (dt == COLL_INT32) return fail(COLL_ERR_UNSUPPORTED, "the weighted combine needs fp32 or bf16 rows");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
+    if ((st = check_rows(y_rows, hidden, "y_rows")) != COLL_OK) return st;
     if (!y || !topk_idx || !route_pos || !topk_weight || !out) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     if (tokens == 0) return COLL_OK;
     const int p = c->p;
@@ -1428,12 +1480,13 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
 // =================================================================================================
 // Ring AllReduce without any allocation.
 //
-// Some callers cannot call cudaMalloc: code that runs while a CUDA graph is being captured with a
-// no-allocation policy, code inside a memory-pool or allocator implementation, or a process that
-// must not grow its device footprint after start-up. For them this entry point runs the same ring
-// AllReduce kernel as coll_allreduce(..., COLL_ALGO_RING, ...) on a fixed scratch area that is part
-// of the library image: a file-scope device array of kStaticScratchBytes. No communicator is
-// created and nothing is allocated or freed per call.
+// Some callers cannot call cudaMalloc: code inside a memory-pool or allocator implementation (it
+// must not re-enter the allocator it implements), a process that must not grow its device footprint
+// after start-up, or code where a framework forbids allocation. For them this entry point runs the
+// same ring AllReduce kernel, with the same schedule and tiling, as coll_allreduce(...,
+// COLL_ALGO_RING, ...) with default options, on a fixed scratch area that is part of the library
+// image: a file-scope device array of kStaticScratchBytes. No communicator is created and nothing is
+// allocated or freed per call.
 //
 // The array lives in device memory of every GPU that loads this library until the process exits.
 // In host code its name is only a host-side handle, never a device address: a kernel given it
@@ -1449,6 +1502,16 @@ constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxStaticDevices = 64;
+
+// An integer option from the environment, or `dflt` when the variable is unset, not a whole
+// number, or outside [lo, hi].
+long long env_option(const char* name, long long dflt, long long lo, long long hi) {
+    const char* v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    char* end = nullptr;
+    const long long x = std::strtoll(v, &end, 0);
+    return (end && *end == 0 && x >= lo && x <= hi) ? x : dflt;
+}
 std::mutex g_static_mu;
 char* g_static_base[kMaxStaticDevices] = {};
 int g_static_sms[kMaxStaticDevices] = {};
@@ -1462,6 +1525,7 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     if (p < 2 || p > SIM_COMM_MAX_RANKS) return fail(COLL_ERR_INVALID_ARG, "p must be in [2, 64]");
     if ((st = check_reduce_args(dt, op)) != COLL_OK) return st;
     if (n == 0) return COLL_OK;
+    if ((st = check_count(n, "n")) != COLL_OK) return st;
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), bytes = n * d;
     std::vector<Range> rs;
@@ -1521,16 +1585,16 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     a.n = n;
     a.seg = seg;
     a.chunk = chunk;
-    a.tile = std::min(chunk, std::max<size_t>(16, kRingTaskBytes / 4));
-    a.ntile = uint32_t((chunk + a.tile - 1) / a.tile);
+    // the same tiling as coll_allreduce(..., COLL_ALGO_RING) with default options
+    ring_tiles(std::min(chunk, seg), 4, default_task_bytes(n * 4), &a.tile, &a.ntile);
     a.elem_bytes = int(d);
     a.nch = nch;
     a.nsteps = nsteps;
     a.ranks_per_step = uint32_t(p);
     a.epoch = 1;
     a.scale = (op == COLL_AVG) ? 1.0f / float(p) : 1.0f;
-    a.skip_rank = -1;
-    a.timeout_ns = 2000000000ULL;
+    a.skip_rank = int(env_option("SIMCOMM_FAULT_SKIP_RANK", -1, -1, p - 1));
+    a.timeout_ns = uint64_t(env_option("SIMCOMM_TIMEOUT_NS", 2000000000LL, 1000, LLONG_MAX));
     a.st = reinterpret_cast<DevState*>(base);
     a.ctl.status = &a.st->status;
     static_assert(sizeof(DevState) + 8 <= 256, "control words must fit the 256-byte control region");
@@ -1552,6 +1616,29 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(status)");
     }
     return COLL_OK;
+}
+
+// ---- HBM access-pattern probe ----------------------------------------------------------------------
+
+extern "C" coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
+                                       coll_stream_t stream) {
+    if (kind < PROBE_LOAD || kind > PROBE_BULK_STORE) return fail(COLL_ERR_INVALID_ARG, "unknown probe kind");
+    if (ctas_per_sm < 1 || ctas_per_sm > 32) return fail(COLL_ERR_INVALID_ARG, "ctas_per_sm must be in [1, 32]");
+    if (bytes == 0) return COLL_OK;
+    if (check_probe_bytes(bytes) != COLL_OK) return COLL_ERR_INVALID_ARG;
+    const bool reads = kind == PROBE_LOAD || kind == PROBE_COPY;
+    const bool writes = kind != PROBE_LOAD;
+    if ((reads && (!src || uintptr_t(src) % 256 != 0)) || (writes && (!dst || uintptr_t(dst) % 256 != 0)))
+        return fail(COLL_ERR_INVALID_ARG, "probe buffers must be non-null and 256-byte aligned");
+    if (reads && writes && overlap(Range{uintptr_t(src), uintptr_t(src) + bytes, false, 0},
+                                   Range{uintptr_t(dst), uintptr_t(dst) + bytes, true, 0}))
+        return fail(COLL_ERR_INVALID_ARG, "probe buffers overlap");
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "probe: device query");
+    e = launch_probe(kind, dst, src, bytes, ctas_per_sm, sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? COLL_OK : cuda_fail(e, "probe launch");
 }
 
 // ---- traced entry points --------------------------------------------------------------------------

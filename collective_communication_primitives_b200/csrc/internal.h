@@ -217,6 +217,9 @@ struct MoeArgs {
     Ctl ctl;
 };
 
+// ---- HBM access-pattern probes (not collectives) --------------------------------------------------
+enum ProbeKind { PROBE_LOAD = 0, PROBE_STORE = 1, PROBE_COPY = 2, PROBE_BULK_STORE = 3 };
+
 // Launchers (each returns the launch error; grid sizes are decided inside).
 cudaError_t launch_butterfly(const ButterflyArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, int num_sms, cudaStream_t s);
@@ -230,5 +233,7 @@ int ring_ll_max_ctas(int num_sms);
 cudaError_t launch_tree(const TreeArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStream_t s);
+cudaError_t launch_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm, int num_sms,
+                         cudaStream_t s);
 
 }  // namespace simcomm

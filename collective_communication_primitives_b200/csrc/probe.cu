@@ -1,0 +1,100 @@
+// HBM access-pattern probes: the bandwidth ceilings that the collectives' kernels are read against.
+//
+// Not a collective. Each probe streams one buffer (or two) through HBM with one access pattern of
+// the library's kernels, so that a kernel's throughput can be compared with what that pattern can
+// reach on the device: 32-byte loads alone (the fused reduction's input side), 32-byte stores alone,
+// 32-byte load + store (a 1:1 copy), and bulk stores (cp.async.bulk shared -> global) of one
+// shared-memory tile (the fan-out side of Broadcast and AllGather).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace simcomm {
+
+namespace {
+
+constexpr int kProbeThreads = 256;
+constexpr int kProbeUnroll = 4;
+constexpr uint32_t kProbeTile = 16 * 1024;  // bytes of one bulk store
+constexpr int kProbeBulkInFlight = 6;       // bulk store groups a CTA keeps in flight
+
+template <int KIND>
+__global__ void __launch_bounds__(kProbeThreads) k_probe_lsu(char* dst, const char* src, size_t nvec) {
+    const size_t stride = size_t(gridDim.x) * kProbeThreads * kProbeUnroll;
+    Words<8> pattern;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pattern.w[k] = 0x3C003C00u + uint32_t(k);
+    uint32_t acc = 0;
+    for (size_t v0 = size_t(blockIdx.x) * kProbeThreads * kProbeUnroll + threadIdx.x; v0 < nvec; v0 += stride) {
+        Words<8> t[kProbeUnroll];
+        if constexpr (KIND != PROBE_STORE) {
+#pragma unroll
+            for (int u = 0; u < kProbeUnroll; ++u) {
+                const size_t v = v0 + size_t(u) * kProbeThreads;
+                if (v < nvec) t[u] = ld_stream_words<8>(src + v * 32);
+            }
+        }
+        if constexpr (KIND == PROBE_LOAD) {
+#pragma unroll
+            for (int u = 0; u < kProbeUnroll; ++u)
+                if (v0 + size_t(u) * kProbeThreads < nvec) acc ^= t[u].w[0] ^ t[u].w[7];
+        } else {
+#pragma unroll
+            for (int u = 0; u < kProbeUnroll; ++u) {
+                const size_t v = v0 + size_t(u) * kProbeThreads;
+                if (v < nvec) st_words<8>(dst + v * 32, KIND == PROBE_STORE ? pattern : t[u]);
+            }
+        }
+    }
+    // the loads are volatile asm and cannot be dropped; dst[0..3] receives a word only in the
+    // impossible case below, so the load-only probe writes nothing
+    if constexpr (KIND == PROBE_LOAD)
+        if (acc == 0x9E3779B9u && threadIdx.x == kProbeThreads) *reinterpret_cast<uint32_t*>(dst) = acc;
+}
+
+// One warp per CTA: a shared-memory tile stored over and over to consecutive 16 KiB pieces of dst.
+__global__ void __launch_bounds__(32) k_probe_bulk_store(char* dst, size_t ntiles) {
+    __shared__ __align__(128) unsigned char tile[kProbeTile];
+    for (uint32_t b = threadIdx.x * 16; b < kProbeTile; b += 32 * 16)
+        *reinterpret_cast<uint4*>(tile + b) = make_uint4(b, b + 1, b + 2, b + 3);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (threadIdx.x != 0) return;
+    uint32_t issued = 0;
+    for (size_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        bulk_s2g(dst + t * kProbeTile, tile, kProbeTile);
+        bulk_commit();
+        if (++issued >= kProbeBulkInFlight)
+            asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(kProbeBulkInFlight - 1) : "memory");
+    }
+    bulk_wait_all();
+}
+
+}  // namespace
+
+cudaError_t launch_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm, int num_sms,
+                         cudaStream_t s) {
+    if (kind == PROBE_BULK_STORE) {
+        const size_t ntiles = bytes / kProbeTile;
+        const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<size_t>(ntiles, 1));
+        k_probe_bulk_store<<<unsigned(grid), 32, 0, s>>>(static_cast<char*>(dst), ntiles);
+        return cudaGetLastError();
+    }
+    const size_t nvec = bytes / 32;
+    const size_t per_cta = size_t(kProbeThreads) * kProbeUnroll;
+    const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<size_t>((nvec + per_cta - 1) / per_cta, 1));
+    char* d = static_cast<char*>(dst);
+    const char* x = static_cast<const char*>(src);
+    switch (kind) {
+        case PROBE_LOAD: k_probe_lsu<PROBE_LOAD><<<unsigned(grid), kProbeThreads, 0, s>>>(d, x, nvec); break;
+        case PROBE_STORE: k_probe_lsu<PROBE_STORE><<<unsigned(grid), kProbeThreads, 0, s>>>(d, x, nvec); break;
+        case PROBE_COPY: k_probe_lsu<PROBE_COPY><<<unsigned(grid), kProbeThreads, 0, s>>>(d, x, nvec); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace simcomm

@@ -85,12 +85,13 @@ def load_library(path=LIB_PATH):
     L.coll_scatter.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_gather.argtypes = [vp, _Bufs, sz, i32, i32, i32, vp]
     L.coll_allreduce_ring_noalloc.argtypes = [i32, _Bufs, sz, i32, i32, vp, vp]
+    L.sim_hbm_probe.argtypes = [i32, vp, vp, sz, i32, vp]
     pp = ctypes.POINTER(ctypes.c_void_p)
     L.coll_moe_dispatch.argtypes = [vp, pp, pp, sz, i32, sz, i32, i32, pp, sz, pp, vp, vp, vp]
     L.coll_moe_combine.argtypes = [vp, pp, sz, pp, pp, pp, pp, sz, i32, sz, i32, i32, pp, vp]
     for name in ("coll_allreduce", "coll_reduce", "coll_broadcast", "coll_reduce_scatter", "coll_allgather",
                  "coll_alltoall", "coll_alltoallv", "coll_scatter", "coll_gather", "coll_allreduce_ring_noalloc",
-                 "coll_moe_dispatch", "coll_moe_combine"):
+                 "coll_moe_dispatch", "coll_moe_combine", "sim_hbm_probe"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -316,3 +317,16 @@ def allreduce_ring_noalloc(sends, recvs, op="sum", n=None, dtype=None, status=No
     if rc != OK:
         raise SimCommError(rc, L.sim_comm_last_error().decode())
 
+
+PROBES = {"load": 0, "store": 1, "copy": 2, "bulk_store": 3}
+
+
+def hbm_probe(kind, dst, src, nbytes, ctas_per_sm, stream=None):
+    """One HBM access-pattern probe (sim_hbm_probe): `kind` in PROBES; dst/src device tensors (or None
+    where the kind does not use them), nbytes a multiple of 16 KiB."""
+    L = load_library()
+    rc = L.sim_hbm_probe(PROBES[kind], ctypes.c_void_p(_ptr(dst)) if dst is not None else None,
+                         ctypes.c_void_p(_ptr(src)) if src is not None else None, nbytes, ctas_per_sm,
+                         _stream(stream))
+    if rc != OK:
+        raise SimCommError(rc, L.sim_comm_last_error().decode())

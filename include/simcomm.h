@@ -34,14 +34,15 @@
  *     All-to-Allv are never in place.
  *   - One communicator runs one collective at a time: calls on different streams must be ordered
  *     by the caller (the communicator's scratch is shared between calls).
- *   - Calls may be captured into a CUDA graph (stream capture) and the graph replayed any number
- *     of times, with eager calls of the same communicator in between. A captured call's scratch
- *     must already exist: make the same call once before capturing; a call that would have to grow
- *     the scratch under capture returns COLL_ERR_UNSUPPORTED and enqueues nothing. The schedules
- *     whose signals carry a per-call epoch or tag (ring, tree, LL) add a memset node that clears
- *     the flags or slots they use, so each replay starts clean. Once a call has been captured,
- *     scratch that a later (larger) call replaces stays allocated until sim_comm_destroy, since a
- *     graph may still use it; destroy the communicator only after its graphs.
+ *   - Calls on a communicator may be captured into a CUDA graph (stream capture) and the graph
+ *     replayed any number of times, with eager calls of the same communicator in between. A
+ *     captured call's scratch must already exist: make the same call once before capturing; a call
+ *     that would have to grow the scratch under capture returns COLL_ERR_UNSUPPORTED and enqueues
+ *     nothing. The schedules whose signals carry a per-call epoch or tag (ring, tree, LL) add a
+ *     memset node that clears the flags or slots they use, so each replay starts clean. Once a call
+ *     has been captured, scratch that a later (larger) call replaces stays allocated until
+ *     sim_comm_destroy, since a graph may still use it; destroy the communicator only after its
+ *     graphs.
  *
  * Errors
  *   - Synchronous (returned, nothing enqueued): COLL_ERR_INVALID_ARG (null handle or pointer, bad
@@ -332,27 +333,52 @@ coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_r
                                const void* const* residual, size_t tokens, int k, size_t hidden, int experts,
                                coll_dtype_t dtype, void* const* out, coll_stream_t stream);
 
+/* ---- diagnostics ------------------------------------------------------------------------------ */
+
+/* HBM access-pattern probe (not a collective; the pages have no counterpart): streams `bytes` through
+ * HBM with one access pattern of the library's kernels, so that a kernel's throughput can be read
+ * against the ceiling of its own pattern on this device.
+ *   kind  0 = load only (32-byte loads of src; nothing is written),
+ *         1 = store only (32-byte stores of a fixed pattern to dst),
+ *         2 = copy (32-byte loads of src, stored to dst),
+ *         3 = bulk store only (cp.async.bulk stores of one 16 KiB shared-memory tile to dst, one warp
+ *             per CTA: the fan-out side of Broadcast and AllGather).
+ *   dst, src  DEVICE pointers, 256-byte aligned, non-overlapping; src is unused by kinds 1 and 3, dst
+ *             by kind 0 (either may then be NULL).
+ *   bytes     a multiple of 16 KiB (0: nothing is enqueued).
+ *   ctas_per_sm  CTAs per SM of the grid, in [1, 32].
+ * Enqueues one kernel on the stream. COLL_ERR_INVALID_ARG for a bad kind, size, pointer or overlap. */
+coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
+                            coll_stream_t stream);
+
 /* ---- no-allocation variant ------------------------------------------------------------------ */
 
 /* Ring AllReduce that allocates nothing. (The pages have no counterpart: this is a library
  * facility, not part of the collective's definition.)
  *
- * For callers that cannot call cudaMalloc: code running while a CUDA graph is captured under a
- * no-allocation policy, code inside an allocator or memory pool, or a process that must not grow
- * its device footprint after start-up. It computes exactly what coll_allreduce(..., COLL_ALGO_RING,
- * ...) computes on a communicator of p ranks (same kernel, same schedule, same rounding), but needs
- * no communicator: its scratch (control words, chunk flags, one fp32/int32 partial buffer per
- * rank) is a fixed 32 MiB device array inside the library, held on every GPU that loads the
- * library until the process exits.
+ * For callers that cannot call cudaMalloc: code inside a memory pool or allocator (which must not
+ * re-enter the allocator it implements), a process that must not grow its device footprint after
+ * start-up (its memory is budgeted up front, and cudaMalloc may also synchronise the device), or code
+ * that runs where a framework forbids allocation. It computes exactly what
+ * coll_allreduce(..., COLL_ALGO_RING, ...) computes on a communicator of p ranks with default options
+ * (same kernel, same schedule and tiling, same rounding), but needs no communicator: its scratch
+ * (control words, chunk flags, one fp32/int32 partial buffer per rank) is a fixed 32 MiB device array
+ * inside the library, held on every GPU that loads the library until the process exits.
  *   p, bufs, n, dtype, op  as for coll_allreduce (2 <= p <= 64).
  *   async_status_dev  DEVICE int the caller owns, or NULL: receives COLL_OK or the asynchronous
- *                     error of this call (COLL_ERR_TIMEOUT if a ring step waited 2 s), in stream
- *                     order.
+ *                     error of this call (COLL_ERR_TIMEOUT if a ring step waited longer than the
+ *                     timeout), in stream order.
+ * Two settings are read from the environment at every call, as a communicator reads its options at
+ * create time: SIMCOMM_TIMEOUT_NS, the longest wait of a ring step (default 2e9, at least 1000), and
+ * SIMCOMM_FAULT_SKIP_RANK, host-side fault injection (that rank never signals, so its successor
+ * times out; -1 = off, the default). A value out of range leaves the default.
  * Limits and errors: the scratch must hold p * round_up(4n, 256) bytes of partials plus the flags
  * (about p * n * 4 < 32 MiB, e.g. n up to ~1M elements at p = 8); larger calls return
  * COLL_ERR_INVALID_ARG with the sizes in sim_comm_last_error(). Other argument errors as for
  * coll_allreduce. The first call on a device looks up the scratch's device address on that device
- * (make that first call before any stream capture). Every call shares the scratch and clears what
+ * and keeps it for the life of the process (make that first call before any stream capture); after
+ * cudaDeviceReset or any other teardown of the device's primary context that address is stale, so
+ * do not call this entry point again in that process. Every call shares the scratch and clears what
  * must start at zero on its own stream; calls that overlap on the GPU race on it and must be
  * ordered by the caller. */
 coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t bufs, size_t n, coll_dtype_t dtype, coll_op_t op,

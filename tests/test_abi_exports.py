@@ -136,3 +136,22 @@ def test_noalloc_entry_checks_its_arguments_without_a_gpu(lib):
     assert L.coll_allreduce_ring_noalloc(65, bufs, 16, 1, 0, None, None) == SC.INVALID_ARG
     assert L.coll_allreduce_ring_noalloc(4, bufs, 16, 7, 0, None, None) == SC.INVALID_ARG
     assert L.coll_allreduce_ring_noalloc(4, bufs, 16, SC.DTYPES["int32"], SC.OPS["avg"], None, None) == SC.UNSUPPORTED
+
+
+def test_noalloc_rejects_counts_whose_byte_sizes_would_wrap(lib):
+    """n beyond 2^48 elements is refused before any size is formed: 2^62 fp32 elements would make
+    n * 4 wrap to 0 bytes, which the pointer and scratch checks would then accept."""
+    L = SC.load_library()
+    p = 4
+    fake = (ctypes.c_void_p * p)(*[0x7f0000000000 + 0x1000000 * r for r in range(p)])
+    out = (ctypes.c_void_p * p)(*[0x7f8000000000 + 0x1000000 * r for r in range(p)])
+    bufs = SC._Bufs(ctypes.cast(fake, ctypes.POINTER(ctypes.c_void_p)),
+                    ctypes.cast(out, ctypes.POINTER(ctypes.c_void_p)))
+    for n in (1 << 62, (1 << 48) + 1, (1 << 64) - 1):
+        assert L.coll_allreduce_ring_noalloc(p, bufs, n, SC.DTYPES["fp32"], SC.OPS["sum"], None, None) == \
+            SC.INVALID_ARG
+        assert b"2^48" in L.sim_comm_last_error()
+    nullbufs = SC._Bufs()  # refused on the size, before the NULL pointers are looked at
+    assert L.coll_allreduce_ring_noalloc(p, nullbufs, 1 << 62, SC.DTYPES["fp32"], SC.OPS["sum"], None, None) == \
+        SC.INVALID_ARG
+    assert b"2^48" in L.sim_comm_last_error()
