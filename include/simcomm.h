@@ -338,7 +338,9 @@ coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_r
 /* HBM access-pattern probe (not a collective; the pages have no counterpart): streams `bytes` through
  * HBM with one access pattern of the library's kernels, so that a kernel's throughput can be read
  * against the ceiling of its own pattern on this device.
- *   kind  0 = load only (32-byte loads of src; nothing is written),
+ *   kind  0 = load only (32-byte loads of src; their XOR is compared with a constant, and only in
+ *             the practically never taken equal case is one word written to dst[0..3], if dst is
+ *             not NULL),
  *         1 = store only (32-byte stores of a fixed pattern to dst),
  *         2 = copy (32-byte loads of src, stored to dst),
  *         3 = bulk store only (cp.async.bulk stores of one 16 KiB shared-memory tile to dst, one warp
