@@ -929,7 +929,8 @@ def write_sweep_md(path, rows, fits):
 
 def ceilings(args):
     """Each access pattern of the library's kernels alone (sim_hbm_probe) over a buffer 16x the L2,
-    at several CTAs per SM; plus torch's copy_ (the measured peak's own method) for reference.
+    at several CTAs per SM (the 1:8 bulk fan-out reads an eighth of it and writes it 8 times); plus
+    torch's copy_ (the measured peak's own method) and fill_ for reference.
     GB/s counts every byte read plus every byte written, best of 5 launches after 2 warm-ups."""
     import torch
 
@@ -966,6 +967,11 @@ def ceilings(args):
                                                 src if kind in ("load", "copy") else None, nb, cps))
                 rows.append({"pattern": kind, "ctas_per_sm": cps, "bytes_moved": moved, "ms": round(ms, 4),
                              "GBps": round(moved / (ms / 1e3) / 1e9, 1)})
+        fan_nb = nb // 8 // (32 << 10) * (32 << 10)
+        for cps in (1, 2, 3):
+            ms = timed(lambda: SC.hbm_probe("bulk_fanout", dst, src, fan_nb, cps))
+            rows.append({"pattern": "bulk_fanout", "ctas_per_sm": cps, "bytes_moved": 9 * fan_nb, "ms": round(ms, 4),
+                         "GBps": round(9 * fan_nb / (ms / 1e3) / 1e9, 1)})
         ms = timed(lambda: dst.copy_(src))
         rows.append({"pattern": "torch copy_", "ctas_per_sm": None, "bytes_moved": 2 * nb, "ms": round(ms, 4),
                      "GBps": round(2 * nb / (ms / 1e3) / 1e9, 1)})

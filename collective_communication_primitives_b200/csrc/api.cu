@@ -358,6 +358,7 @@ coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_e
     if (c->copy_order >= 0) order = int(c->copy_order);
     a.order = order;
     a.l2_hint = int(c->l2_hint);
+    a.st = c->dstate;
     a.ctl = make_ctl(c);
     cudaError_t e = launch_copy(a, c->num_sms, variant, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
@@ -772,7 +773,7 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
         if (value != 0 && value != 16 && value != 32) return fail(COLL_ERR_INVALID_ARG, "direct_pack must be 0, 16 or 32");
         c->direct_pack = value;
     } else if (k == "direct_ctas_per_sm") {
-        if (value < 1 || value > 32) return fail(COLL_ERR_INVALID_ARG, "direct_ctas_per_sm must be in [1, 32]");
+        if (value < 0 || value > 32) return fail(COLL_ERR_INVALID_ARG, "direct_ctas_per_sm must be in [0, 32]");
         c->direct_ctas_per_sm = value;
     } else if (k == "ring_task_bytes") {
         if (value != 0 && (value < 4096 || value > (64 << 20) || value % 256 != 0))
@@ -1622,16 +1623,19 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
 
 extern "C" coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
                                        coll_stream_t stream) {
-    if (kind < PROBE_LOAD || kind > PROBE_BULK_STORE) return fail(COLL_ERR_INVALID_ARG, "unknown probe kind");
+    if (kind < PROBE_LOAD || kind > PROBE_BULK_FANOUT) return fail(COLL_ERR_INVALID_ARG, "unknown probe kind");
     if (ctas_per_sm < 1 || ctas_per_sm > 32) return fail(COLL_ERR_INVALID_ARG, "ctas_per_sm must be in [1, 32]");
     if (bytes == 0) return COLL_OK;
     if (check_probe_bytes(bytes) != COLL_OK) return COLL_ERR_INVALID_ARG;
-    const bool reads = kind == PROBE_LOAD || kind == PROBE_COPY;
+    if (kind == PROBE_BULK_FANOUT && (bytes % (32 * 1024) != 0 || bytes > (size_t(1) << 40)))
+        return fail(COLL_ERR_INVALID_ARG, "fan-out probe bytes must be a multiple of 32 KiB, at most 2^40");
+    const bool reads = kind == PROBE_LOAD || kind == PROBE_COPY || kind == PROBE_BULK_FANOUT;
     const bool writes = kind != PROBE_LOAD;
+    const size_t dst_bytes = kind == PROBE_BULK_FANOUT ? bytes * kProbeFanCopies : bytes;
     if ((reads && (!src || uintptr_t(src) % 256 != 0)) || (writes && (!dst || uintptr_t(dst) % 256 != 0)))
         return fail(COLL_ERR_INVALID_ARG, "probe buffers must be non-null and 256-byte aligned");
     if (reads && writes && overlap(Range{uintptr_t(src), uintptr_t(src) + bytes, false, 0},
-                                   Range{uintptr_t(dst), uintptr_t(dst) + bytes, true, 0}))
+                                   Range{uintptr_t(dst), uintptr_t(dst) + dst_bytes, true, 0}))
         return fail(COLL_ERR_INVALID_ARG, "probe buffers overlap");
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);

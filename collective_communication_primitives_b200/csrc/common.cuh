@@ -336,6 +336,28 @@ __device__ __forceinline__ void signal_chunk(const Ctl& ctl, unsigned long long*
     raise_status(ctl, COLL_ERR_INTERNAL);
 }
 
+// ---- dynamic task distribution ---------------------------------------------------------------------
+// CTAs claim task numbers in increasing order from a counter in the communicator's scratch, so the
+// tasks in flight at any moment are neighbours in the task order: for tasks laid out in address
+// order, a narrow window of memory. (Measured on B200: a static grid-stride split of a stream over
+// persistent CTAs reached 6.3 TB/s of stores where in-order distribution reached 7.4, and copies
+// 6.4 against 6.9: with a static split the slowest CTA's share sets the end.) A CTA that finds the
+// communicator failed claims nothing; every CTA that ran its task loop leaves through leave_tasks,
+// and the last one to leave resets the counter for the next call.
+__device__ __forceinline__ uint32_t claim_task(const Ctl& ctl, uint32_t* next, uint32_t total) {
+    return status_failed(ctl) ? total : atomicAdd(next, 1u);
+}
+
+// Called by one thread per CTA after the CTA's last access to the counter.
+__device__ __forceinline__ void leave_tasks(uint32_t* next, uint32_t* done) {
+    __threadfence();
+    if (atomicAdd(done, 1u) == gridDim.x * gridDim.y * gridDim.z - 1) {
+        *next = 0;
+        *done = 0;
+        __threadfence();
+    }
+}
+
 // ---- TMA bulk copies and mbarriers (shared::cta addresses, no multicast) -------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

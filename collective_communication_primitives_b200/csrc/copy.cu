@@ -266,19 +266,17 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
     }
     __syncwarp();
 
-    const uint32_t my_n = (total > blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     uint32_t phase = 0;  // bit s: parity of the next completion of stage s
     const uint64_t pol = a.l2_hint ? l2_evict_first_policy() : 0;
     bool failed = false;
 
     // A task is located once, when its load is issued, and handed to its consume through the stage's
-    // slot. Tasks are issued in increasing order, so the level pointer only moves forward.
+    // slot. Tasks are claimed in increasing order, so the level pointer only moves forward.
     __shared__ int s_task_sg[kStages];
     __shared__ uint32_t s_task_ti[kStages];  // kNoTask: an empty slot of the interleaved order
     constexpr uint32_t kNoTask = 0xFFFFFFFFu;
     uint32_t lv = 0;
-    auto issue = [&](uint32_t k) {
-        const uint32_t t = blockIdx.x + k * gridDim.x;
+    auto issue = [&](uint32_t k, uint32_t t) {  // the k-th task of this CTA is task t
         int s = 0;
         uint32_t ti = 0;
         bool ok = true;
@@ -347,19 +345,34 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         if (g.hi > g.bhi) warp_copy_bytes(a, d, g.bhi, g.hi);
     };
 
-    const uint32_t pre = my_n < uint32_t(kStages - 1) ? my_n : uint32_t(kStages - 1);
-    for (uint32_t k = 0; k < pre; ++k) issue(k);
-    for (uint32_t k = 0; k < my_n && !failed; ++k) {
-        const uint32_t kk = k + kStages - 1;
-        if (kk < my_n) {
-            // stage kk % kStages was last used by tile k-1, whose stores are the newest group
+    // Tasks are claimed one at a time, kStages - 1 ahead of the one being stored.
+    uint32_t n_issued = 0;
+    bool more = true;
+    auto issue_next = [&]() {
+        uint32_t t = 0;
+        if (lane == 0) t = claim_task(a.ctl, &a.st->task_ctr, total);
+        t = __shfl_sync(0xFFFFFFFFu, t, 0);
+        if (t >= total) {
+            more = false;
+            return;
+        }
+        issue(n_issued, t);
+        ++n_issued;
+    };
+    for (int k = 0; k < kStages - 1 && more; ++k) issue_next();
+    for (uint32_t k = 0; k < n_issued && !failed; ++k) {
+        if (more) {
+            // the next task's stage was last used by task k-1, whose stores are the newest group
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
-            issue(kk);
+            issue_next();
         }
         consume(k);
     }
-    if (lane == 0) bulk_wait_all();
+    if (lane == 0) {
+        bulk_wait_all();
+        leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
+    }
     __syncwarp();
 }
 
@@ -466,7 +479,13 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     const uint32_t total = (a.order && !levels) ? tmax * uint32_t(nseg) : prefix[nseg];
     uint64_t pol = 0;
     if constexpr (HINT) pol = l2_evict_first_policy();
-    for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
+    __shared__ uint32_t s_t;
+    while (true) {
+        __syncthreads();  // every thread has read the previous task number
+        if (threadIdx.x == 0) s_t = claim_task(a.ctl, &a.st->task_ctr, total);
+        __syncthreads();
+        const uint32_t t = s_t;
+        if (t >= total) break;
         int sg;
         uint32_t k;
         if (a.order && levels) {
@@ -484,6 +503,7 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
         const size_t hi = min(lo + kLsuTask, d.len);
         cta_copy_bytes<HINT>(d.src + lo, d.dst + lo, hi - lo, pol);
     }
+    if (threadIdx.x == 0) leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
 }
 
 // The current device as one bit of a mask (0 for devices 63 and up, which set the attribute every launch).
@@ -596,18 +616,16 @@ static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cuda
 }
 
 // Per-collective defaults, the fastest measured on B200 at the DP-bucket size (p = 8, 100 MiB per
-// rank): Broadcast and AllGather on the bulk-copy pipeline with 6 stages of 16 KiB and 2 CTAs per
-// SM; All-to-All on 4 stages of 32 KiB with the interleaved tile order; All-to-Allv (whose skewed
-// blocks leave most interleaved slots empty) on the load/store path, block after block.
+// rank) with tasks claimed in order, each row charged with its own write-back: every bulk-copy
+// collective on 2 stages of 32 KiB with 3 CTAs per SM, block after block (All-to-All 0.259 ms
+// against 0.345-0.405 ms for the deeper 1-2 CTA shapes; Broadcast and AllGather 0.168 ms against
+// 0.170-0.176); All-to-Allv on the load/store path, block after block.
 constexpr int kVariantLsu = kNumCopyShapes;
 
 void copy_defaults(int kind, int* variant, int* order) {
     switch (kind) {
-        case COPY_ALLTOALL:
-        case COPY_SCATTER:
-        case COPY_GATHER: *variant = 0; *order = 1; break;
         case COPY_ALLTOALLV: *variant = kVariantLsu; *order = 0; break;
-        default: *variant = 5; *order = 0; break;
+        default: *variant = 6; *order = 0; break;
     }
 }
 

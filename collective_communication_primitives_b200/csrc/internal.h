@@ -14,8 +14,8 @@ constexpr int kMaxRanks = SIM_COMM_MAX_RANKS;
 // Device scratch header of a communicator (device memory, zero-initialised).
 struct DevState {
     uint32_t status;    // first asynchronous error (coll_status_t), 0 = OK
-    uint32_t task_ctr;  // ring / butterfly executor: next task to claim
-    uint32_t done_ctr;  // ring / butterfly executor: CTAs that left the task loop
+    uint32_t task_ctr;  // ring, tree, butterfly executors and the copy kernels: next task to claim
+    uint32_t done_ctr;  // the same kernels: CTAs that left the task loop (the last one resets both)
     uint32_t moe_ctr;   // MoE dispatch scan: blocks finished (the last one resets it)
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
     unsigned long long abort_clock;  // global time of the last read of the host abort word
@@ -70,6 +70,7 @@ struct CopyArgs {
     long long send_cap[kMaxRanks];     // ALLTOALLV: elements per send buffer
     long long recv_cap[kMaxRanks];     // ALLTOALLV: elements per recv buffer
     uint64_t timeout_ns;
+    DevState* st;                      // task counters (dynamic distribution)
     Ctl ctl;
 };
 
@@ -218,7 +219,8 @@ struct MoeArgs {
 };
 
 // ---- HBM access-pattern probes (not collectives) --------------------------------------------------
-enum ProbeKind { PROBE_LOAD = 0, PROBE_STORE = 1, PROBE_COPY = 2, PROBE_BULK_STORE = 3 };
+enum ProbeKind { PROBE_LOAD = 0, PROBE_STORE = 1, PROBE_COPY = 2, PROBE_BULK_STORE = 3, PROBE_BULK_FANOUT = 4 };
+constexpr int kProbeFanCopies = 8;  // PROBE_BULK_FANOUT writes this many copies of src
 
 // Launchers (each returns the launch error; grid sizes are decided inside).
 cudaError_t launch_butterfly(const ButterflyArgs& a, int dtype, int op, int ctas, cudaStream_t s);

@@ -4,7 +4,8 @@
 // the library's kernels, so that a kernel's throughput can be compared with what that pattern can
 // reach on the device: 32-byte loads alone (the fused reduction's input side), 32-byte stores alone,
 // 32-byte load + store (a 1:1 copy), and bulk stores (cp.async.bulk shared -> global) of one
-// shared-memory tile (the fan-out side of Broadcast and AllGather).
+// shared-memory tile (the fan-out side of Broadcast and AllGather), and a bulk fan-out of every tile
+// of one buffer to 8 copies (the whole Broadcast / AllGather pattern of 8 ranks).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -74,10 +75,75 @@ __global__ void __launch_bounds__(32) k_probe_bulk_store(char* dst, size_t ntile
     bulk_wait_all();
 }
 
+// Bulk fan-out 1:kProbeFan, the access pattern of a Broadcast or AllGather of kProbeFan ranks: every
+// 32 KiB tile of src is loaded once into shared memory and stored to dst + f * bytes for each f (dst
+// holds kProbeFan copies). One warp per CTA, kProbeFanStages tiles in flight, tiles claimed in order
+// from a counter that the host clears before the launch.
+constexpr int kProbeFan = 8;
+constexpr int kProbeFanStages = 4;
+constexpr uint32_t kProbeFanTile = 32 * 1024;
+__device__ uint32_t g_probe_ctr;
+
+__global__ void __launch_bounds__(32) k_probe_fanout(char* dst, const char* src, size_t bytes, uint32_t ntiles) {
+    extern __shared__ __align__(128) unsigned char stages[];
+    __shared__ uint64_t bars[kProbeFanStages];
+    __shared__ uint32_t tiles[kProbeFanStages];
+    if (threadIdx.x != 0) return;
+    for (int st = 0; st < kProbeFanStages; ++st) mbar_init(&bars[st], 1);
+    fence_barrier_init();
+    uint32_t phase = 0, head = 0, tail = 0;
+    bool more = true;
+    auto issue = [&]() {
+        const uint32_t t = atomicAdd(&g_probe_ctr, 1u);
+        if (t >= ntiles) {
+            more = false;
+            return;
+        }
+        const int st = int(head % kProbeFanStages);
+        tiles[st] = t;
+        mbar_arrive_expect_tx(&bars[st], kProbeFanTile);
+        bulk_g2s(stages + size_t(st) * kProbeFanTile, src + size_t(t) * kProbeFanTile, kProbeFanTile, &bars[st]);
+        ++head;
+    };
+    while (more && head < kProbeFanStages - 1) issue();
+    while (tail < head) {
+        const int st = int(tail % kProbeFanStages);
+        // a load that never lands ends the probe (bounded: the probe has no error channel)
+        bool ok = false;
+        for (uint32_t it = 0; it < kMaxSpin && !ok; ++it) ok = mbar_try_wait(&bars[st], (phase >> st) & 1u);
+        if (!ok) break;
+        phase ^= 1u << st;
+        for (int f = 0; f < kProbeFan; ++f)
+            bulk_s2g(dst + size_t(f) * bytes + size_t(tiles[st]) * kProbeFanTile, stages + size_t(st) * kProbeFanTile,
+                     kProbeFanTile);
+        bulk_commit();
+        ++tail;
+        if (more) {
+            bulk_wait_read_all();
+            issue();
+        }
+    }
+    bulk_wait_all();
+}
+
 }  // namespace
 
 cudaError_t launch_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm, int num_sms,
                          cudaStream_t s) {
+    if (kind == PROBE_BULK_FANOUT) {
+        const uint32_t ntiles = uint32_t(bytes / kProbeFanTile);
+        void* ctr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ctr, g_probe_ctr);
+        if (e == cudaSuccess) e = cudaMemsetAsync(ctr, 0, sizeof(uint32_t), s);
+        const size_t smem = size_t(kProbeFanStages) * kProbeFanTile;
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_probe_fanout, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<uint32_t>(ntiles, 1u));
+        k_probe_fanout<<<unsigned(grid), 32, smem, s>>>(static_cast<char*>(dst), static_cast<const char*>(src), bytes,
+                                                      ntiles);
+        return cudaGetLastError();
+    }
     if (kind == PROBE_BULK_STORE) {
         const size_t ntiles = bytes / kProbeTile;
         const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<size_t>(ntiles, 1));

@@ -162,7 +162,9 @@ static dim3 vec_grid(const DirectReduceArgs& a, size_t packs, int max_blocks) {
 
 template <int DT, int OP, bool SCALE>
 static cudaError_t launch_typed(const DirectReduceArgs& a, int num_sms, cudaStream_t s) {
-    const int max_blocks = num_sms * (a.ctas_per_sm > 0 ? a.ctas_per_sm : 4);
+    // ctas_per_sm == 0: one pass, every CTA takes one iteration's worth of positions (the blocks are
+    // dispatched in address order as SMs free up)
+    const int max_blocks = a.ctas_per_sm > 0 ? num_sms * a.ctas_per_sm : (1 << 30);
     if (!a.vec) {
         const size_t want = (a.n + kDirThreads - 1) / kDirThreads;
         const int grid = int(want < size_t(max_blocks) ? (want ? want : 1) : size_t(max_blocks));

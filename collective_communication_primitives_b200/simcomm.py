@@ -318,12 +318,13 @@ def allreduce_ring_noalloc(sends, recvs, op="sum", n=None, dtype=None, status=No
         raise SimCommError(rc, L.sim_comm_last_error().decode())
 
 
-PROBES = {"load": 0, "store": 1, "copy": 2, "bulk_store": 3}
+PROBES = {"load": 0, "store": 1, "copy": 2, "bulk_store": 3, "bulk_fanout": 4}
 
 
 def hbm_probe(kind, dst, src, nbytes, ctas_per_sm, stream=None):
     """One HBM access-pattern probe (sim_hbm_probe): `kind` in PROBES; dst/src device tensors (or None
-    where the kind does not use them), nbytes a multiple of 16 KiB."""
+    where the kind does not use them), nbytes a multiple of 16 KiB (bulk_fanout: of 32 KiB, and dst
+    holds 8 * nbytes)."""
     L = load_library()
     rc = L.sim_hbm_probe(PROBES[kind], ctypes.c_void_p(_ptr(dst)) if dst is not None else None,
                          ctypes.c_void_p(_ptr(src)) if src is not None else None, nbytes, ctas_per_sm,

@@ -165,7 +165,8 @@ const char* coll_status_string(coll_status_t status);
  *                  1 = interleaved over all blocks, 0 = block after block
  *   "direct_pack"  access width of the fused reduction: 0 = widest the alignment allows
  *                  (32 bytes), 16 = at most 16 bytes
- *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16)
+ *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16); 0 = one pass, a CTA per
+ *                  iteration's worth of positions
  *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
  *                  paths (data read or written once), 0 = none (default)
  *   "moe_tma"      copy kernel of coll_moe_dispatch: 0 = 32/16-byte loads and stores (default,
@@ -344,10 +345,14 @@ coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_r
  *         1 = store only (32-byte stores of a fixed pattern to dst),
  *         2 = copy (32-byte loads of src, stored to dst),
  *         3 = bulk store only (cp.async.bulk stores of one 16 KiB shared-memory tile to dst, one warp
- *             per CTA: the fan-out side of Broadcast and AllGather).
+ *             per CTA: the fan-out side of Broadcast and AllGather),
+ *         4 = bulk fan-out 1:8 (every 32 KiB tile of src loaded once into shared memory and stored
+ *             to dst + f·bytes for f = 0..7, tiles claimed in order: the whole Broadcast / AllGather
+ *             pattern of 8 ranks; dst holds 8·bytes). Not re-entrant: its tile counter is a device
+ *             variable of the library, so two kind-4 probes must not overlap on the GPU.
  *   dst, src  DEVICE pointers, 256-byte aligned, non-overlapping; src is unused by kinds 1 and 3, dst
  *             by kind 0 (either may then be NULL).
- *   bytes     a multiple of 16 KiB (0: nothing is enqueued).
+ *   bytes     a multiple of 16 KiB (kind 4: of 32 KiB, at most 2^40; 0: nothing is enqueued).
  *   ctas_per_sm  CTAs per SM of the grid, in [1, 32].
  * Enqueues one kernel on the stream. COLL_ERR_INVALID_ARG for a bad kind, size, pointer or overlap. */
 coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
