@@ -474,7 +474,7 @@ def moe_ops(comm, mw):
     bd = BM.moe_dispatch_bytes(p, T, k, H, 2)
     bc = BM.moe_combine_bytes(p, T, k, H, 2, residual=True)
     return [
-        ("moe_dispatch_bf16", "moe_dispatch (count+scan+copy)",
+        ("moe_dispatch_bf16", "moe_dispatch (count, prefix sums, copy)",
          lambda: comm.moe_dispatch(mw.x, mw.idx, mw.E, mw.recv, route_pos=mw.pos, expert_counts=mw.expert_counts,
                                    recv_counts=mw.recv_counts), bd, bd),
         ("moe_combine_bf16", "moe_combine",
@@ -485,18 +485,26 @@ def moe_ops(comm, mw):
 def moe_block(comm, mw, steps, warmup, stream, hbm, cpu=False):
     """Device time of the MoE dispatch and combine (behind a spacer, CUDA events) and their HBM
     roofline fractions."""
+    import torch
+
     from collective_communication_primitives_b200 import synth as S
     ops = moe_ops(comm, mw)
+    launches = []
+    for op in ops:  # kernels one call launches (the comm's own count)
+        l0 = comm.launch_count()
+        op[2]()
+        launches.append(comm.launch_count() - l0)
+    torch.cuda.synchronize()
     _, per_op = time_device(ops, steps, warmup, stream)
     blk = {"workload": f"MoE layer, p={mw.p} ranks x {mw.T} tokens, top-{mw.k} of {mw.E} experts (Zipf 1.1), "
                        f"{mw.H}-wide bf16 rows", "max_recv_rows": int(mw.col_rows.max()),
            "rank_counts": S.count_matrix_stats(mw.rank_rows)}
     if cpu:
         blk["cpu_baseline"] = moe_cpu_baseline()
-    for (name, kernel, _, eff, kb), ms in zip(ops, per_op):
+    for (name, kernel, _, eff, kb), ms, nl in zip(ops, per_op, launches):
         g = kb / (ms / 1e3) / 1e9
         blk[name] = {"ms": round(ms, 4), "GBps": round(g, 1), "frac_of_measured": round(g / hbm, 4),
-                     "algorithmic_bytes": int(kb), "launches_per_call": 3 if "dispatch" in name else 1}
+                     "algorithmic_bytes": int(kb), "launches_per_call": int(nl)}
     return blk
 
 

@@ -32,6 +32,7 @@ constexpr size_t kTraceCap = 4096;
 
 struct sim_comm {
     int p = 0;
+    int rank = -1;                  // a rank view: the one rank of p processes this handle computes for
     int device = 0;
     int num_sms = 0;
     DevState* dstate = nullptr;     // device scratch header
@@ -59,6 +60,7 @@ struct sim_comm {
     long long l2_hint = 0;
     long long ring_task_bytes = 0;  // bytes of the wire type one ring / tree task moves; 0 = by message size
     long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
+    long long moe_fused = 1;        // MoE dispatch: 1 one cooperative kernel, 0 three kernels
     unsigned long long launches = 0;
     int ring_ctas_max = 0;
     bool capturing = false;               // the current call's stream is being captured into a graph
@@ -330,24 +332,27 @@ coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, col
     return COLL_OK;
 }
 
+// p_override > 0: run the copy over that many segments' ranks instead of the communicator's p (a
+// rank view's single-source copies).
 coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_elems, coll_dtype_t dt, int root,
                        bool use_send_all, cudaStream_t s, const long long* counts = nullptr,
                        const long long* send_cap = nullptr, const long long* recv_cap = nullptr,
-                       long long* recv_counts = nullptr) {
+                       long long* recv_counts = nullptr, int p_override = 0) {
+    const int p = p_override > 0 ? p_override : c->p;
     CopyArgs a;
     std::memset(&a, 0, sizeof(a));
-    fill_ptrs(a.ptrs, b, c->p, true, true);
+    fill_ptrs(a.ptrs, b, p, true, true);
     if (!use_send_all)
-        for (int r = 0; r < c->p; ++r)
+        for (int r = 0; r < p; ++r)
             if (r != root) a.ptrs.send[r] = nullptr;
-    a.p = c->p;
+    a.p = p;
     a.kind = kind;
     a.root = root;
     a.elem_bytes = int(dtype_bytes(dt));
     a.blk_elems = blk_elems;
     a.counts = counts;
     a.recv_counts_out = recv_counts;
-    for (int r = 0; r < c->p; ++r) {
+    for (int r = 0; r < p; ++r) {
         a.send_cap[r] = send_cap ? send_cap[r] : 0;
         a.recv_cap[r] = recv_cap ? recv_cap[r] : 0;
     }
@@ -743,7 +748,7 @@ uint32_t chunks_of(size_t seg, size_t chunk) { return uint32_t(std::max<size_t>(
 
 constexpr const char* kOptionKeys[] = {"chunk_bytes", "ring_ctas", "ring_task_bytes", "timeout_ns",
                                        "fault_skip_rank", "copy_variant", "copy_order", "direct_pack",
-                                       "direct_ctas_per_sm", "l2_hint", "moe_tma", "trace"};
+                                       "direct_ctas_per_sm", "l2_hint", "moe_tma", "moe_fused", "trace"};
 
 coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     std::string k(key);
@@ -782,6 +787,9 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
     } else if (k == "moe_tma") {
         if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "moe_tma must be 0 or 1");
         c->moe_tma = value;
+    } else if (k == "moe_fused") {
+        if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "moe_fused must be 0 or 1");
+        c->moe_fused = value;
     } else if (k == "trace") {
         if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "trace must be 0 or 1");
         c->trace = value;
@@ -842,6 +850,78 @@ struct TraceScope {
     }
 };
 
+// ---- rank views: one rank of a communicator whose ranks are separate processes -------------------
+// The process of rank r holds a rank view (sim_comm_create_rank). bufs.send[q] is rank q's input as
+// this process maps it (its own buffer for q = r, a mapping from sim_ipc_open of rank q's buffer
+// otherwise) and bufs.recv[r] this rank's output; the other recv entries are ignored. A call
+// computes rank r's output only, reading every rank's input where it lies (a pull), with the same
+// kernels, fold order and rounding as the whole communicator's direct path, so rank r's output
+// equals that path's output for rank r bit for bit ([Atlas] §3.3: the P2P transport reads a peer's
+// buffer directly).
+
+enum RankColl { RK_ALLREDUCE, RK_REDUCE, RK_BCAST, RK_REDUCE_SCATTER, RK_ALLGATHER, RK_ALLTOALL, RK_SCATTER, RK_GATHER };
+
+// Checks the inputs this rank reads (every rank's, or only src_rank's) and its own output.
+coll_status_t rank_check(sim_comm* c, const coll_bufs_t& b, size_t in_bytes, size_t out_bytes, size_t d,
+                         int src_rank, InPlaceRule rule, size_t shard_bytes) {
+    coll_status_t st;
+    std::vector<Range> rs;
+    for (int q = 0; q < c->p; ++q) {
+        if (src_rank >= 0 && q != src_rank) continue;
+        if ((st = check_ptr(b.send[q], in_bytes, d, "send")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(b.send[q]), uintptr_t(b.send[q]) + in_bytes, false, q});
+    }
+    if ((st = check_ptr(b.recv[c->rank], out_bytes, d, "recv")) != COLL_OK) return st;
+    rs.push_back({uintptr_t(b.recv[c->rank]), uintptr_t(b.recv[c->rank]) + out_bytes, true, c->rank});
+    return check_ranges(rs, rule, shard_bytes);
+}
+
+coll_status_t rank_collective(sim_comm* c, RankColl coll, const coll_bufs_t& b, size_t n, coll_dtype_t dt,
+                              coll_op_t op, int root, coll_algo_t algo, cudaStream_t s) {
+    if (algo != COLL_ALGO_DIRECT)
+        return fail(COLL_ERR_UNSUPPORTED, "a rank view runs the direct path only (the ring, tree and LL schedules "
+                                          "wait on other ranks inside their kernels)");
+    const int p = c->p, r = c->rank;
+    if ((coll == RK_REDUCE || coll == RK_GATHER) && r != root) return COLL_OK;  // only the root has an output
+    const size_t d = dtype_bytes(dt), m = n / size_t(p);
+    std::vector<const void*> send(p, nullptr);
+    std::vector<void*> recv(p, nullptr);
+    recv[r] = b.recv[r];
+    coll_status_t st;
+    switch (coll) {
+        case RK_ALLREDUCE:
+        case RK_REDUCE:
+            if ((st = rank_check(c, b, n * d, n * d, d, -1, INPLACE_NONE, 0)) != COLL_OK) return st;
+            for (int q = 0; q < p; ++q) send[q] = b.send[q];
+            return run_direct_reduce(c, coll_bufs_t{send.data(), recv.data()}, n, dt, op, MODE_REDUCE, r, s);
+        case RK_REDUCE_SCATTER:  // this rank's block of every input, reduced
+            if ((st = rank_check(c, b, n * d, m * d, d, -1, INPLACE_NONE, 0)) != COLL_OK) return st;
+            for (int q = 0; q < p; ++q) send[q] = static_cast<const char*>(b.send[q]) + size_t(r) * m * d;
+            return run_direct_reduce(c, coll_bufs_t{send.data(), recv.data()}, m, dt, op, MODE_REDUCE, r, s);
+        case RK_ALLGATHER:  // every rank's shard, gathered into this rank's output
+        case RK_GATHER:
+            if ((st = rank_check(c, b, m * d, n * d, d, -1, INPLACE_NONE, 0)) != COLL_OK) return st;
+            for (int q = 0; q < p; ++q) send[q] = b.send[q];
+            return run_copy(c, coll_bufs_t{send.data(), recv.data()}, COPY_GATHER, m, dt, r, true, s);
+        case RK_ALLTOALL:  // block r of every rank's input
+            if ((st = rank_check(c, b, n * d, n * d, d, -1, INPLACE_NONE, 0)) != COLL_OK) return st;
+            for (int q = 0; q < p; ++q) send[q] = static_cast<const char*>(b.send[q]) + size_t(r) * m * d;
+            return run_copy(c, coll_bufs_t{send.data(), recv.data()}, COPY_GATHER, m, dt, r, true, s);
+        case RK_BCAST:  // the root's input copied to this rank's output (the root's own in place: nothing)
+        case RK_SCATTER: {  // block r of the root's input
+            const bool bc = coll == RK_BCAST;
+            if ((st = rank_check(c, b, n * d, (bc ? n : m) * d, d, root, bc ? INPLACE_SAME : INPLACE_RS, m * d)) !=
+                COLL_OK)
+                return st;
+            const void* src[1] = {static_cast<const char*>(b.send[root]) + (bc ? 0 : size_t(r) * m * d)};
+            void* dst[1] = {b.recv[r]};
+            return run_copy(c, coll_bufs_t{src, dst}, COPY_GATHER, bc ? n : m, dt, 0, true, s, nullptr, nullptr,
+                            nullptr, nullptr, 1);
+        }
+    }
+    return fail(COLL_ERR_INTERNAL, "unknown rank-view collective");
+}
+
 }  // namespace
 
 // =================================================================================================
@@ -901,6 +981,56 @@ sim_comm_t sim_comm_create(int p) {
     return c;
 }
 
+sim_comm_t sim_comm_create_rank(int p, int rank) {
+    if (p < 1 || p > SIM_COMM_MAX_RANKS || rank < 0 || rank >= p) {
+        fail(COLL_ERR_INVALID_ARG, "p must be in [1, 64] and rank in [0, p)");
+        return nullptr;
+    }
+    sim_comm_t c = sim_comm_create(p);
+    if (c) c->rank = rank;
+    return c;
+}
+
+int sim_comm_rank(sim_comm_t c) { return c ? c->rank : -2; }
+
+coll_status_t sim_ipc_alloc(size_t bytes, void** dev_ptr, sim_ipc_handle_t* handle) {
+    static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(sim_ipc_handle_t), "handle sizes differ");
+    if (!dev_ptr || !handle || bytes == 0) return fail(COLL_ERR_INVALID_ARG, "null argument or zero bytes");
+    if (bytes > kMaxCount) return fail(COLL_ERR_INVALID_ARG, "bytes exceed 2^48");
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(shared buffer)");
+    cudaIpcMemHandle_t h;
+    e = cudaIpcGetMemHandle(&h, p);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "cudaIpcGetMemHandle");
+    }
+    std::memcpy(handle, &h, sizeof(h));
+    *dev_ptr = p;
+    return COLL_OK;
+}
+
+coll_status_t sim_ipc_free(void* dev_ptr) {
+    if (!dev_ptr) return COLL_OK;
+    cudaError_t e = cudaFree(dev_ptr);
+    return e == cudaSuccess ? COLL_OK : cuda_fail(e, "cudaFree(shared buffer)");
+}
+
+coll_status_t sim_ipc_open(const sim_ipc_handle_t* handle, void** peer_ptr) {
+    if (!handle || !peer_ptr) return fail(COLL_ERR_INVALID_ARG, "null argument");
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    cudaError_t e = cudaIpcOpenMemHandle(peer_ptr, h, cudaIpcMemLazyEnablePeerAccess);
+    return e == cudaSuccess ? COLL_OK : cuda_fail(e, "cudaIpcOpenMemHandle");
+}
+
+coll_status_t sim_ipc_close(void* peer_ptr) {
+    if (!peer_ptr) return COLL_OK;
+    cudaError_t e = cudaIpcCloseMemHandle(peer_ptr);
+    return e == cudaSuccess ? COLL_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
+}
+
 coll_status_t sim_comm_destroy(sim_comm_t c) {
     if (!c) return COLL_OK;
     cudaDeviceSynchronize();
@@ -957,6 +1087,7 @@ coll_status_t sim_comm_get_option(sim_comm_t c, const char* key, long long* valu
     else if (k == "l2_hint") *value = c->l2_hint;
     else if (k == "direct_ctas_per_sm") *value = c->direct_ctas_per_sm;
     else if (k == "moe_tma") *value = c->moe_tma;
+    else if (k == "moe_fused") *value = c->moe_fused;
     else if (k == "ring_task_bytes") *value = c->ring_task_bytes;
     else if (k == "trace") *value = c->trace;
     else return fail(COLL_ERR_INVALID_ARG, "unknown option " + k);
@@ -1007,6 +1138,10 @@ static coll_status_t coll_allreduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
         return fail(COLL_ERR_UNSUPPORTED, "recursive doubling / halving-doubling need p a power of two");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_ALLREDUCE, b, n, dt, op, 0, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const int p = c->p;
     const size_t d = dtype_bytes(dt), bytes = n * d;
@@ -1047,6 +1182,10 @@ static coll_status_t coll_reduce_impl(sim_comm_t c, coll_bufs_t b, size_t n, col
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_REDUCE, b, n, dt, op, root, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), bytes = n * d;
     std::vector<Range> rs;
@@ -1084,6 +1223,10 @@ static coll_status_t coll_broadcast_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     if (root < 0 || root >= p) return fail(COLL_ERR_INVALID_ARG, "root must be a rank index in [0, p)");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_BCAST, b, n, dt, COLL_SUM, root, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), bytes = n * d;
     std::vector<Range> rs;
@@ -1119,6 +1262,10 @@ static coll_status_t coll_reduce_scatter_impl(sim_comm_t c, coll_bufs_t b, size_
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "ReduceScatter needs n divisible by p");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_REDUCE_SCATTER, b, n, dt, op, 0, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1153,6 +1300,10 @@ static coll_status_t coll_allgather_impl(sim_comm_t c, coll_bufs_t b, size_t n, 
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "AllGather needs n divisible by p");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_ALLGATHER, b, n, dt, COLL_SUM, 0, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1187,6 +1338,10 @@ static coll_status_t coll_alltoall_impl(sim_comm_t c, coll_bufs_t b, size_t n, c
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "All-to-All needs n divisible by p");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_ALLTOALL, b, n, dt, COLL_SUM, 0, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1222,6 +1377,10 @@ static coll_status_t coll_scatter_impl(sim_comm_t c, coll_bufs_t b, size_t n, co
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Scatter needs n divisible by p");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_SCATTER, b, n, dt, COLL_SUM, root, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1250,6 +1409,10 @@ static coll_status_t coll_gather_impl(sim_comm_t c, coll_bufs_t b, size_t n, col
     if (n % size_t(p) != 0) return fail(COLL_ERR_INVALID_ARG, "Gather needs n divisible by p");
     if (n == 0) return COLL_OK;
     if ((st = check_count(n, "n")) != COLL_OK) return st;
+    if (c->rank >= 0) {
+        if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
+        return rank_collective(c, RK_GATHER, b, n, dt, COLL_SUM, root, algo, static_cast<cudaStream_t>(stream));
+    }
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     const size_t d = dtype_bytes(dt), m = n / size_t(p);
     std::vector<Range> rs;
@@ -1273,6 +1436,7 @@ static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if ((st = check_algo(algo)) != COLL_OK) return st;
+    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "All-to-Allv is not built for rank views");
     if (!counts_dev || !send_cap || !recv_cap) return fail(COLL_ERR_INVALID_ARG, "null counts or capacities");
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     if (reinterpret_cast<uintptr_t>(counts_dev) % 8 != 0 ||
@@ -1339,6 +1503,7 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
+    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "the MoE dispatch is not built for rank views");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
     if (recv_cap_rows > size_t(INT32_MAX)) return fail(COLL_ERR_INVALID_ARG, "recv_cap_rows must fit in int32");
     if ((st = check_rows(recv_cap_rows, hidden, "recv_cap_rows")) != COLL_OK) return st;
@@ -1387,24 +1552,29 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
         a.dst[r] = recv[r];
         a.pos[r] = route_pos ? route_pos[r] : nullptr;
     }
-    // scratch: tile counts [p][ntiles][E], in-tile ranks [p][A], totals and first rows [p][E] each
+    // scratch: tile counts [p][ntiles][E], in-tile ranks [p][A], totals and first rows [p][E] each,
+    // the count matrix [p][p]
     const size_t b_hist = align_up(size_t(p) * a.ntiles * experts * 4, 256);
     const size_t b_rank = align_up(size_t(p) * A * 4, 256);
     const size_t b_pe = align_up(size_t(p) * experts * 4, 256);
-    if ((st = ensure_moe(c, b_hist + b_rank + 2 * b_pe)) != COLL_OK) return st;
+    const size_t b_pp = align_up(size_t(p) * p * 4, 256);
+    if ((st = ensure_moe(c, b_hist + b_rank + 2 * b_pe + b_pp)) != COLL_OK) return st;
     a.tile_hist = reinterpret_cast<int32_t*>(c->moe);
     a.rank_in_tile = reinterpret_cast<int32_t*>(c->moe + b_hist);
     a.cnt = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank);
     a.base = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + b_pe);
+    a.cmat = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + 2 * b_pe);
     a.expert_counts_out = expert_counts_dev;
     a.recv_counts_out = recv_counts_dev;
     a.tma = int(c->moe_tma);
+    a.fused = int(c->moe_fused);
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.st = c->dstate;
     a.ctl = make_ctl(c);
-    cudaError_t e = launch_moe_dispatch(a, c->num_sms, s);
+    int launched = 0;
+    cudaError_t e = launch_moe_dispatch(a, c->num_sms, s, &launched);
     if (e != cudaSuccess) return cuda_fail(e, "MoE dispatch launch");
-    c->launches += 3;
+    c->launches += unsigned(launched);
     return COLL_OK;
 }
 
@@ -1417,6 +1587,7 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if (dt == COLL_INT32) return fail(COLL_ERR_UNSUPPORTED, "the weighted combine needs fp32 or bf16 rows");
+    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "the MoE combine is not built for rank views");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
     if ((st = check_rows(y_rows, hidden, "y_rows")) != COLL_OK) return st;
     if (!y || !topk_idx || !route_pos || !topk_weight || !out) return fail(COLL_ERR_INVALID_ARG, "null buffer array");

@@ -16,9 +16,11 @@ struct DevState {
     uint32_t status;    // first asynchronous error (coll_status_t), 0 = OK
     uint32_t task_ctr;  // ring, tree, butterfly executors and the copy kernels: next task to claim
     uint32_t done_ctr;  // the same kernels: CTAs that left the task loop (the last one resets both)
-    uint32_t moe_ctr;   // MoE dispatch scan: blocks finished (the last one resets it)
+    uint32_t moe_ctr;   // MoE dispatch: scan blocks finished, or the fused kernel's grid-barrier arrivals
+                        // (zero between calls)
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
     unsigned long long abort_clock;  // global time of the last read of the host abort word
+    unsigned long long moe_task;     // fused MoE dispatch: next token row to claim (zero between calls)
 };
 
 // What a kernel needs to report errors and notice an abort.
@@ -210,9 +212,12 @@ struct MoeArgs {
     int32_t* rank_in_tile;           // [p][A] rank of an assignment among its tile's same-expert ones
     int32_t* cnt;                    // [p][E] assignments from rank i to expert e
     int32_t* base;                   // [p][E] first receive row of (rank i, expert e) at the expert's owner
+    int32_t* cmat;                   // fused dispatch: [p][p] rows from rank i to rank j
     long long* expert_counts_out;    // [p][E] or null
     long long* recv_counts_out;      // [p] or null
     int tma;                         // dispatch copy: 1 bulk copies through shared memory, 0 loads/stores
+    int fused;                       // dispatch: 1 one cooperative kernel (counting, sums and copy), 0 three
+                                     // kernels (the copy chosen by tma)
     uint64_t timeout_ns;
     DevState* st;
     Ctl ctl;
@@ -233,7 +238,7 @@ int ring_max_ctas(int num_sms);
 cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s);
 int ring_ll_max_ctas(int num_sms);
 cudaError_t launch_tree(const TreeArgs& a, int dtype, int op, int ctas, cudaStream_t s);
-cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s, int* kernels_launched);
 cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStream_t s);
 cudaError_t launch_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm, int num_sms,
                          cudaStream_t s);

@@ -356,6 +356,219 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
     __syncwarp();
 }
 
+// ---- fused dispatch: counting, prefix sums and the copy in one cooperative kernel -----------------
+//
+// Three kernels cost the dispatch ~23 us of launches and tiny serial phases before the copy starts
+// (8 + 16 us under ncu on 8 x 8192 tokens). Here one cooperative launch (every CTA resident) runs
+//   phase 1  counting: the k_moe_count work, a (rank, tile) per CTA pass, grid-strided;
+//   phase 2  a warp per (rank, expert) column: exclusive prefix of the tile counts over tiles, the
+//            total cnt[i][e] and c[i][j] += cnt[i][e] (integer atomics: exact in any order);
+//   phase 3  every CTA turns c into R[i][j] = Σ_{q<i} c[q][j] in shared memory and checks every
+//            destination's capacity (the same decision everywhere); a warp per (rank, destination)
+//            block writes base[i][e] = R[i][j] + Σ of cnt[i][·] over the block's lower experts;
+//   phase 4  the copy: warps claim batches of consecutive token rows in order and copy each row with
+//            32/16-byte loads and one store per slot;
+// with a bounded grid barrier between phases. Data other CTAs wrote in this kernel is read through
+// L2 (ld.global.cg): L1 is not coherent between SMs.
+constexpr int kFusedThreads = kMoeTile;  // a counting tile per CTA pass
+constexpr int kFusedUnroll = 8;          // packs in flight per lane in the copy
+
+__device__ __forceinline__ bool moe_grid_barrier(const MoeArgs& a, uint32_t k) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(&a.st->moe_ctr, 1u);
+        s_ok = wait_counter(a.ctl, &a.st->moe_ctr, k * gridDim.x, a.timeout_ns) && !status_failed(a.ctl);
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+template <int W>
+__global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __grid_constant__ MoeArgs a) {
+    extern __shared__ int s_dyn[];  // [E] counting histogram, then [p][p] c -> R, then [p] column totals
+    __shared__ char* s_dst[kFusedThreads / 32][32];
+    __shared__ int s_flag;
+    if (cta_failed(a.ctl)) return;
+    const int p = a.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int* s_cnt = s_dyn;
+    int* s_c = s_dyn + a.E;
+    int* s_tot = s_c + p * p;
+
+    // ---- phase 1: counting ----
+    if (blockIdx.x == 0)
+        for (int x = threadIdx.x; x < p * p; x += kFusedThreads) a.cmat[x] = 0;
+    const uint32_t ntask = uint32_t(p) * a.ntiles;
+    for (uint32_t g = blockIdx.x; g < ntask; g += gridDim.x) {
+        const int i = int(g / a.ntiles);
+        const uint32_t tile = g % a.ntiles;
+        __syncthreads();  // the previous tile's histogram has been written out
+        for (int e = threadIdx.x; e < a.E; e += kFusedThreads) s_cnt[e] = 0;
+        __syncthreads();
+        const size_t asg = size_t(tile) * kMoeTile + threadIdx.x;
+        const bool valid = asg < a.A;
+        int e = valid ? a.idx[i][asg] : -1;
+        if (valid && (e < 0 || e >= a.E)) {
+            raise_status(a.ctl, COLL_ERR_INVALID_ARG);
+            e = -1;
+        }
+        int rank = 0;
+        for (int w = 0; w < kFusedThreads / 32; ++w) {  // warps in order: ranks follow assignment order
+            if (warp == w) {
+                const unsigned same = __match_any_sync(0xffffffffu, e);
+                const int leader = __ffs(same) - 1;
+                int first = 0;
+                if (lane == leader && e >= 0) {
+                    first = s_cnt[e];
+                    s_cnt[e] = first + __popc(same);
+                }
+                first = __shfl_sync(0xffffffffu, first, leader);
+                rank = first + __popc(same & ((1u << lane) - 1u));
+            }
+            __syncthreads();
+        }
+        if (valid) a.rank_in_tile[size_t(i) * a.A + asg] = rank;
+        int32_t* hist = a.tile_hist + (size_t(i) * a.ntiles + tile) * a.E;
+        for (int x = threadIdx.x; x < a.E; x += kFusedThreads) hist[x] = s_cnt[x];
+    }
+    if (!moe_grid_barrier(a, 1)) return;
+
+    // ---- phase 2: per (rank, expert) column, prefix over tiles, totals ----
+    const uint32_t nwarps = gridDim.x * (kFusedThreads / 32);
+    const uint32_t gw = blockIdx.x * (kFusedThreads / 32) + uint32_t(warp);
+    for (uint32_t col = gw; col < uint32_t(p) * uint32_t(a.E); col += nwarps) {
+        const int i = int(col / uint32_t(a.E)), e = int(col % uint32_t(a.E));
+        int32_t* colp = a.tile_hist + size_t(i) * a.ntiles * a.E + e;
+        int run = 0;
+        for (uint32_t t0 = 0; t0 < a.ntiles; t0 += 32 * kScanChunks) {
+            int v[kScanChunks];
+#pragma unroll
+            for (int c = 0; c < kScanChunks; ++c) {
+                const uint32_t t = t0 + uint32_t(c * 32 + lane);
+                v[c] = t < a.ntiles ? __ldcg(colp + size_t(t) * a.E) : 0;
+            }
+#pragma unroll
+            for (int c = 0; c < kScanChunks; ++c) {
+                const uint32_t t = t0 + uint32_t(c * 32 + lane);
+                const int incl = warp_incl_scan_i(v[c], lane);
+                if (t < a.ntiles) colp[size_t(t) * a.E] = run + incl - v[c];
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+        if (lane == 0) {
+            a.cnt[size_t(i) * a.E + e] = run;
+            atomicAdd(&a.cmat[i * p + e / a.E_loc], run);
+            if (a.expert_counts_out) a.expert_counts_out[size_t(i) * a.E + e] = run;
+        }
+    }
+    if (!moe_grid_barrier(a, 2)) return;
+
+    // ---- phase 3: R = exclusive column prefix of c, capacity check, first rows ----
+    for (int x = threadIdx.x; x < p * p; x += kFusedThreads) s_c[x] = __ldcg(a.cmat + x);
+    if (threadIdx.x == 0) s_flag = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < p; j += kFusedThreads) {
+        int run = 0;
+        for (int q = 0; q < p; ++q) {
+            const int v = s_c[q * p + j];
+            s_c[q * p + j] = run;
+            run += v;
+        }
+        s_tot[j] = run;
+        if (size_t(run) > a.cap_rows) atomicOr(&s_flag, 1);
+        if (blockIdx.x == 0 && a.recv_counts_out) a.recv_counts_out[j] = run;
+    }
+    __syncthreads();
+    if (s_flag) {  // every CTA computed the same totals: nobody copies anything
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(a.ctl, COLL_ERR_OVERFLOW);
+        return;
+    }
+    for (uint32_t blk = gw; blk < uint32_t(p) * uint32_t(p); blk += nwarps) {
+        const int i = int(blk / uint32_t(p)), j = int(blk % uint32_t(p));
+        int run = s_c[i * p + j];
+        for (int e0 = j * a.E_loc; e0 < (j + 1) * a.E_loc; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < (j + 1) * a.E_loc ? __ldcg(a.cnt + size_t(i) * a.E + e) : 0;
+            const int incl = warp_incl_scan_i(v, lane);
+            if (e < (j + 1) * a.E_loc) a.base[size_t(i) * a.E + e] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    if (!moe_grid_barrier(a, 3)) return;
+
+    // ---- phase 4: the copy, batches of consecutive token rows claimed in order ----
+    const size_t row_bytes = a.H * size_t(a.elem_bytes);
+    const int kslot = slot_width(a.k), per_batch = 32 / kslot;
+    const int my_b = lane / kslot, my_s = lane % kslot;
+    const unsigned long long rows = (unsigned long long)p * a.T;
+    while (true) {
+        unsigned long long u0 = 0;
+        if (lane == 0) u0 = status_failed(a.ctl) ? rows : atomicAdd(&a.st->moe_task, (unsigned long long)per_batch);
+        u0 = __shfl_sync(0xffffffffu, u0, 0);
+        if (u0 >= rows) break;
+        const unsigned long long my_u = u0 + unsigned(my_b);
+        bool bad = false;
+        if (my_s < a.k && my_u < rows) {
+            const int i = int(my_u / a.T);
+            const size_t t = size_t(my_u % a.T);
+            const size_t asg = t * a.k + my_s;
+            const int e = a.idx[i][asg];
+            const long long row = (long long)__ldcg(a.base + size_t(i) * a.E + e) +
+                                  __ldcg(a.tile_hist + (size_t(i) * a.ntiles + asg / kMoeTile) * a.E + e) +
+                                  __ldcg(a.rank_in_tile + size_t(i) * a.A + asg);
+            bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
+            if (bad) raise_status(a.ctl, COLL_ERR_INTERNAL);
+            if (a.pos[i]) a.pos[i][asg] = bad ? -1 : int32_t(row);
+            s_dst[warp][lane] = bad ? nullptr : static_cast<char*>(a.dst[e / a.E_loc]) + size_t(row) * row_bytes;
+        }
+        __syncwarp();
+        if (!__any_sync(0xffffffffu, bad)) {
+            for (int b = 0; b < per_batch; ++b) {
+                const unsigned long long u = u0 + unsigned(b);
+                if (u >= rows) break;
+                const char* s_row = static_cast<const char*>(a.src[int(u / a.T)]) + size_t(u % a.T) * row_bytes;
+                char* const* d = s_dst[warp] + b * kslot;
+                if constexpr (W > 0) {
+                    constexpr size_t kPack = size_t(W) * 4;
+                    const size_t npk = row_bytes / kPack;
+                    for (size_t c0 = lane; c0 < npk; c0 += 32 * kFusedUnroll) {
+                        Words<W> v[kFusedUnroll];
+#pragma unroll
+                        for (int q = 0; q < kFusedUnroll; ++q)
+                            if (c0 + q * 32 < npk) v[q] = ld_stream_words<W>(s_row + (c0 + q * 32) * kPack);
+                        for (int sl = 0; sl < a.k; ++sl) {
+                            char* d_row = d[sl];
+#pragma unroll
+                            for (int q = 0; q < kFusedUnroll; ++q)
+                                if (c0 + q * 32 < npk) st_words<W>(d_row + (c0 + q * 32) * kPack, v[q]);
+                        }
+                    }
+                } else {
+                    const size_t nu = row_bytes / 2;  // 2-byte units (every row is a whole number of them)
+                    for (size_t c0 = lane; c0 < nu; c0 += 32) {
+                        const uint16_t v = *reinterpret_cast<const uint16_t*>(s_row + c0 * 2);
+                        for (int sl = 0; sl < a.k; ++sl) *reinterpret_cast<uint16_t*>(d[sl] + c0 * 2) = v;
+                    }
+                }
+            }
+        }
+        __syncwarp();  // the next batch rewrites this warp's destination rows
+    }
+    // the last CTA out clears the call's counters
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&a.st->done_ctr, 1u) == gridDim.x - 1) {
+            a.st->moe_task = 0;
+            a.st->moe_ctr = 0;
+            a.st->done_ctr = 0;
+            __threadfence();
+        }
+    }
+}
+
 // ---- combine: reverse exchange + unpermute + weighted sum ---------------------------------------
 
 template <int DT>
@@ -562,7 +775,52 @@ static cudaError_t launch_after(void (*kernel)(MoeArgs), dim3 grid, dim3 block, 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s) {
+// The fused dispatch on a cooperative launch: as many CTAs as are resident at once (needed by its
+// grid barriers). Returns cudaErrorNotSupported when the device cannot launch cooperatively.
+template <int W>
+static cudaError_t launch_fused(const MoeArgs& a, int num_sms, cudaStream_t s) {
+    auto kernel = k_moe_dispatch_fused<W>;
+    const size_t smem = (size_t(a.E) + size_t(a.p) * a.p + size_t(a.p)) * sizeof(int);
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorNotSupported;
+    dim3 grid(unsigned(num_sms * per_sm)), block(kFusedThreads);
+    MoeArgs b = a;
+    void* args[] = {&b};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kernel), grid, block, args, smem, s);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+static bool cooperative_ok() {
+    static int v = -1;
+    if (v < 0) {
+        int dev = 0, ok = 0;
+        v = (cudaGetDevice(&dev) == cudaSuccess &&
+             cudaDeviceGetAttribute(&ok, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && ok) ? 1 : 0;
+    }
+    return v == 1;
+}
+
+cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s, int* kernels_launched) {
+    *kernels_launched = 0;
+    if (a.fused && cooperative_ok()) {
+        *kernels_launched = 1;
+        const size_t row_bytes = a.H * size_t(a.elem_bytes);
+        bool al32 = row_bytes % 32 == 0, al16 = row_bytes % 16 == 0;
+        for (int r = 0; r < a.p; ++r) {
+            const uintptr_t x = reinterpret_cast<uintptr_t>(a.src[r]), y = reinterpret_cast<uintptr_t>(a.dst[r]);
+            al32 = al32 && x % 32 == 0 && y % 32 == 0;
+            al16 = al16 && x % 16 == 0 && y % 16 == 0;
+        }
+        if (al32) return launch_fused<8>(a, num_sms, s);
+        if (al16) return launch_fused<4>(a, num_sms, s);
+        return launch_fused<0>(a, num_sms, s);
+    }
+    *kernels_launched = 3;
     const size_t smem_count = size_t(a.E) * sizeof(int);
     if (smem_count > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_moe_count, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_count));

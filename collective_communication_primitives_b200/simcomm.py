@@ -32,6 +32,11 @@ class _Bufs(ctypes.Structure):
     _fields_ = [("send", ctypes.POINTER(ctypes.c_void_p)), ("recv", ctypes.POINTER(ctypes.c_void_p))]
 
 
+class IpcHandle(ctypes.Structure):
+    """sim_ipc_handle_t: 64 opaque bytes naming a shareable device buffer."""
+    _fields_ = [("reserved", ctypes.c_ubyte * 64)]
+
+
 class TraceRecord(ctypes.Structure):
     """sim_comm_trace_record_t: one traced call."""
     _fields_ = [("seq", ctypes.c_ulonglong), ("coll", ctypes.c_char_p), ("p", ctypes.c_int), ("dtype", ctypes.c_int),
@@ -53,6 +58,16 @@ def load_library(path=LIB_PATH):
     st = ctypes.c_int
     L.sim_comm_create.argtypes = [i32]
     L.sim_comm_create.restype = vp
+    L.sim_comm_create_rank.argtypes = [i32, i32]
+    L.sim_comm_create_rank.restype = vp
+    L.sim_comm_rank.argtypes = [vp]
+    L.sim_comm_rank.restype = i32
+    L.sim_ipc_alloc.argtypes = [sz, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(IpcHandle)]
+    L.sim_ipc_free.argtypes = [vp]
+    L.sim_ipc_open.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p)]
+    L.sim_ipc_close.argtypes = [vp]
+    for name in ("sim_ipc_alloc", "sim_ipc_free", "sim_ipc_open", "sim_ipc_close"):
+        getattr(L, name).restype = ctypes.c_int
     L.sim_comm_destroy.argtypes = [vp]
     L.sim_comm_destroy.restype = st
     L.sim_comm_size.argtypes = [vp]
@@ -124,15 +139,17 @@ def _stream(stream):
 
 
 class SimComm:
-    """A communicator of p logical ranks on the current CUDA device."""
+    """A communicator of p logical ranks on the current CUDA device (or, with `rank`, the rank view
+    that the process of that rank holds when every rank is its own process)."""
 
-    def __init__(self, p):
+    def __init__(self, p, rank=None):
         self._L = load_library()
-        h = self._L.sim_comm_create(int(p))
+        h = self._L.sim_comm_create(int(p)) if rank is None else self._L.sim_comm_create_rank(int(p), int(rank))
         if not h:
-            raise SimCommError(CUDA, self._L.sim_comm_last_error().decode())
+            raise SimCommError(CUDA if rank is None else INVALID_ARG, self._L.sim_comm_last_error().decode())
         self._h = ctypes.c_void_p(h)
         self.p = int(p)
+        self.rank = None if rank is None else int(rank)
 
     # -- lifecycle ---------------------------------------------------------------------------------
     def close(self):

@@ -132,6 +132,43 @@ typedef void* coll_stream_t;
  * Returns NULL on failure; sim_comm_last_error() then says why. */
 sim_comm_t sim_comm_create(int p);
 
+/* A rank view: the handle that the process running rank `rank` of a p-rank communicator holds when
+ * every rank is its own process (one per GPU, or several on one GPU), after [Atlas] §3.1-§3.3 (a
+ * communicator's ranks exchange buffer handles once, then the P2P transport reads peers' buffers
+ * directly). bufs.send[q] is then rank q's input as this process maps it (its own buffer for q =
+ * rank, a mapping from sim_ipc_open of rank q's buffer otherwise) and bufs.recv[rank] this rank's
+ * output; the other recv entries are ignored (may be NULL). A call computes this rank's output only,
+ * reading the inputs it needs where they lie, with the direct path's kernels, fold order and
+ * rounding, so the output equals the whole communicator's direct-path output for this rank bit for
+ * bit. Supported: AllReduce, Reduce, Broadcast, ReduceScatter, AllGather, All-to-All, Scatter,
+ * Gather, COLL_ALGO_DIRECT only (the other schedules wait on other ranks inside their kernels:
+ * COLL_ERR_UNSUPPORTED, as for All-to-Allv and the MoE calls). Reduce and Gather enqueue nothing
+ * on a non-root rank. No output may overlap any rank's input (a peer may still be reading it), except
+ * the root's own in-place Broadcast and Scatter forms. The ranks' calls are not synchronised by the
+ * library: before a call every rank's inputs must be complete, and no rank may modify its input until
+ * every rank's call that reads it has completed (e.g. every rank synchronises its stream and meets a
+ * host barrier before and after each call). NULL on failure (p in [1, 64], rank in [0, p)). */
+sim_comm_t sim_comm_create_rank(int p, int rank);
+
+/* The rank of a rank view, -1 for a whole communicator, -2 for NULL. */
+int sim_comm_rank(sim_comm_t comm);
+
+/* Device memory another process can map (cudaIpcGetMemHandle / cudaIpcOpenMemHandle): the buffers
+ * of a rank view's collectives. The handle is an opaque 64-byte value to send to the other ranks'
+ * processes (by any host channel). */
+typedef struct { unsigned char reserved[64]; } sim_ipc_handle_t;
+
+/* Allocates `bytes` (> 0, at most 2^48) of device memory on the current device and its handle.
+ * Free with sim_ipc_free in the same process, after every other process has closed its mapping. */
+coll_status_t sim_ipc_alloc(size_t bytes, void** dev_ptr, sim_ipc_handle_t* handle);
+coll_status_t sim_ipc_free(void* dev_ptr);
+
+/* Maps another process's buffer into this one (*peer_ptr: its base as seen here; peer access between
+ * GPUs is enabled on first use). A handle cannot be opened in the process that allocated it. Close
+ * with sim_ipc_close before the owner frees the buffer. */
+coll_status_t sim_ipc_open(const sim_ipc_handle_t* handle, void** peer_ptr);
+coll_status_t sim_ipc_close(void* peer_ptr);
+
 /* Free the communicator and its scratch. Synchronises the device first. NULL is accepted. */
 coll_status_t sim_comm_destroy(sim_comm_t comm);
 
@@ -169,9 +206,12 @@ const char* coll_status_string(coll_status_t status);
  *                  iteration's worth of positions
  *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
  *                  paths (data read or written once), 0 = none (default)
- *   "moe_tma"      copy kernel of coll_moe_dispatch: 0 = 32/16-byte loads and stores (default,
- *                  measured faster), 1 = bulk copies through shared memory (rows of whole 16-byte
- *                  units at 16-byte aligned bases; otherwise the load/store kernel runs)
+ *   "moe_fused"    coll_moe_dispatch as one cooperative kernel (counting, prefix sums and the copy
+ *                  with grid barriers between them; 1, the default, where the device supports
+ *                  cooperative launches) or as three kernels (0)
+ *   "moe_tma"      copy kernel of the three-kernel coll_moe_dispatch: 0 = 32/16-byte loads and stores
+ *                  (default, measured faster), 1 = bulk copies through shared memory (rows of whole
+ *                  16-byte units at 16-byte aligned bases; otherwise the load/store kernel runs)
  *   "trace"        1 = keep a record of every call (sim_comm_trace_read), 0 = off (default).
  *                  Every entry point also opens an NVTX range named after its collective, whatever
  *                  this option says (a no-op unless a profiler collects NVTX).

@@ -155,3 +155,21 @@ def test_noalloc_rejects_counts_whose_byte_sizes_would_wrap(lib):
     assert L.coll_allreduce_ring_noalloc(p, nullbufs, 1 << 62, SC.DTYPES["fp32"], SC.OPS["sum"], None, None) == \
         SC.INVALID_ARG
     assert b"2^48" in L.sim_comm_last_error()
+
+
+def test_rank_view_and_ipc_entries_check_their_arguments_without_a_gpu(lib):
+    L = SC.load_library()
+    assert not L.sim_comm_create_rank(4, 4)
+    assert b"rank in [0, p)" in L.sim_comm_last_error()
+    assert not L.sim_comm_create_rank(0, 0)
+    assert not L.sim_comm_create_rank(4, -1)
+    assert L.sim_comm_rank(None) == -2
+    ptr = ctypes.c_void_p()
+    h = SC.IpcHandle()
+    assert L.sim_ipc_alloc(0, ctypes.byref(ptr), ctypes.byref(h)) == SC.INVALID_ARG
+    assert L.sim_ipc_alloc(16, None, ctypes.byref(h)) == SC.INVALID_ARG
+    assert L.sim_ipc_alloc((1 << 48) + 1, ctypes.byref(ptr), ctypes.byref(h)) == SC.INVALID_ARG
+    assert L.sim_ipc_open(None, ctypes.byref(ptr)) == SC.INVALID_ARG
+    assert L.sim_ipc_open(ctypes.byref(h), None) == SC.INVALID_ARG
+    assert L.sim_ipc_free(None) == SC.OK and L.sim_ipc_close(None) == SC.OK
+    assert ctypes.sizeof(SC.IpcHandle) == 64

@@ -84,15 +84,17 @@ DISPATCH_CASES = [
 
 
 @pytest.mark.parametrize("p,T,k,E,H,dtype,kind,offset", DISPATCH_CASES)
-@pytest.mark.parametrize("tma", [1, 0])
-def test_dispatch_parity(p, T, k, E, H, dtype, kind, offset, tma):
-    """Both copy kernels: bulk copies through shared memory (rows of whole 16-byte units at aligned
-    bases, else the load/store kernel runs) and 32/16/2-byte loads and stores."""
+@pytest.mark.parametrize("fused,tma", [(1, 0), (0, 1), (0, 0)])
+def test_dispatch_parity(p, T, k, E, H, dtype, kind, offset, fused, tma):
+    """Every dispatch path: the fused cooperative kernel (32/16/2-byte copies), and the three-kernel
+    path with either copy kernel: bulk copies through shared memory (rows of whole 16-byte units at
+    aligned bases, else the load/store kernel runs) and 32/16/2-byte loads and stores."""
     ids = make_routes(p, T, k, E, kind, seed=p * 31 + T)
     xs = make_rows(p, T, H, dtype, f"moe.dispatch.{p}.{T}.{H}")
     ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, dtype)
     cap = int(ref["recv_counts"].max()) + 3
     with SC.SimComm(p) as comm:
+        comm.set_option("moe_fused", fused)
         comm.set_option("moe_tma", tma)
         x_g, r_g, _, pos_t, ec, rc = dispatch_case(comm, xs, ids, E, cap, dtype, offset)
         assert comm.async_error() == SC.OK
@@ -262,12 +264,14 @@ def test_dispatch_and_combine_at_the_limits(p, T, k, E, H):
         np.testing.assert_array_equal(out[i].cpu().numpy(), want[i])
 
 
-def test_dispatch_overflow_and_invalid_ids_copy_nothing():
+@pytest.mark.parametrize("fused", [1, 0])
+def test_dispatch_overflow_and_invalid_ids_copy_nothing(fused):
     p, T, k, E, H, dtype = 4, 200, 2, 8, 16, "fp32"
     ids = make_routes(p, T, k, E, "one", seed=1)
     xs = make_rows(p, T, H, dtype, "moe.err")
     need = p * T * k
     with SC.SimComm(p) as comm:
+        comm.set_option("moe_fused", fused)
         _, r_g, _, _, _, _ = dispatch_case(comm, xs, ids, E, need - 1, dtype)
         assert comm.async_error() == SC.OVERFLOW
         for g in r_g:

@@ -1,0 +1,157 @@
+"""Rank views on one GPU: every rank is its own process with its own CUDA context; buffers are
+allocated by the library (sim_ipc_alloc), their handles exchanged over gloo and mapped into the
+other processes (sim_ipc_open), and each rank's collective reads its peers' buffers directly. Each
+rank's output is compared bit for bit with the oracle (every rank regenerates every rank's seeded
+inputs). No kernel waits on another process: the ranks meet only at host barriers between calls.
+A rank that leaves between calls makes the others' next call fail on the host with
+COLL_ERR_TIMEOUT."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+pytestmark = pytest.mark.gpu
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _setup(rank, world, port, timeout_s):
+    import sys
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=timeout_s))
+    torch.cuda.set_device(0)
+
+
+def _bits(a):
+    import numpy as np
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def _collectives(rank, world, port, dtype, op, q):
+    try:
+        _setup(rank, world, port, 60)
+        import numpy as np
+        import torch.distributed as dist
+
+        import oracle as O
+        from collective_communication_primitives_b200 import ranks
+        from gpu_helpers import make_inputs, to_numpy, to_torch
+        p, m = world, 4099
+        n = p * m
+        d = ranks.BYTES[dtype]
+        kind = "int24" if dtype == "int32" else "normal"
+        ins = make_inputs(kind, p, n, dtype, f"ranks.{p}.{dtype}")
+        comm = ranks.RankComm()
+        sbuf, rbuf = ranks.SharedBuffer(n * d), ranks.SharedBuffer(n * d)
+        sbuf.view(dtype, n).copy_(to_torch(ins[rank], dtype))
+        sends = comm.register(sbuf)
+        out = rbuf.view(dtype, n)
+        sentinel = to_torch(np.full(n, 7, {"int32": np.int32, "fp32": np.float32, "bf16": np.uint16}[dtype]), dtype)
+
+        def got(count):
+            return to_numpy(out[:count], dtype)
+
+        def check(name, want):
+            w = np.asarray(want)
+            g = got(w.size)
+            assert np.array_equal(_bits(g), _bits(w)), f"{name}: rank {rank} differs"
+
+        acc = "exact" if (dtype == "int32" or op in ("min", "max")) else "rankfold"
+        comm.allreduce(sends, rbuf.ptr, n, dtype, op=op)
+        check("allreduce", O.allreduce(ins, dtype, op, acc=acc)[rank])
+        comm.reduce_scatter(sends, rbuf.ptr, n, dtype, op=op)
+        check("reduce_scatter", O.reduce_scatter(ins, dtype, op, acc=acc)[rank])
+        comm.alltoall(sends, rbuf.ptr, n, dtype)
+        check("alltoall", O.alltoall(ins, dtype)[rank])
+        root = p - 1
+        comm.broadcast(sends, rbuf.ptr, root, n, dtype)
+        check("broadcast", O.broadcast(ins[root], p, dtype, root)[rank])
+        comm.scatter(sends, rbuf.ptr, root, n, dtype)
+        check("scatter", O.scatter(ins[root], p, dtype, root)[rank])
+        out.copy_(sentinel)
+        comm.reduce(sends, rbuf.ptr, root, n, dtype, op=op)
+        if rank == root:
+            check("reduce", O.reduce(ins, dtype, op, root, acc=acc))
+        else:
+            check("reduce leaves non-roots untouched", to_numpy(sentinel, dtype))
+        # AllGather / Gather of the first m elements of every rank's input
+        shards = [x[:m] for x in ins]
+        comm.allgather(sends, rbuf.ptr, n, dtype)
+        check("allgather", O.allgather(shards, dtype)[rank])
+        out.copy_(sentinel)
+        comm.gather(sends, rbuf.ptr, 0, n, dtype)
+        check("gather", O.gather(shards, dtype, 0) if rank == 0 else to_numpy(sentinel, dtype))
+        assert comm.async_error() == 0
+        comm.sync()
+        comm.close()  # every mapping closed before any owner frees its buffers
+        dist.barrier()
+        sbuf.close()
+        rbuf.close()
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except Exception as e:  # reported to the parent
+        import traceback
+        q.put((rank, f"{type(e).__name__}: {e}\n{traceback.format_exc()}"))
+
+
+def _spawn(target, world, *args, timeout=300):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=target, args=(r, world, port, *args, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=timeout) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=120)
+    return res, [pr.exitcode for pr in procs]
+
+
+@pytest.mark.parametrize("world,dtype,op", [(2, "fp32", "sum"), (3, "bf16", "avg"), (4, "int32", "sum"),
+                                            (4, "fp32", "max")])
+def test_rank_views_match_the_oracle(world, dtype, op):
+    res, codes = _spawn(_collectives, world, dtype, op)
+    assert all(v == "ok" for v in res.values()), res
+    assert codes == [0] * world
+
+
+def _leaver(rank, world, port, q):
+    try:
+        _setup(rank, world, port, 5)
+        from collective_communication_primitives_b200 import ranks
+        from collective_communication_primitives_b200 import simcomm as SC
+        n = 2 * 1024
+        comm = ranks.RankComm()
+        sbuf, rbuf = ranks.SharedBuffer(n * 4), ranks.SharedBuffer(n * 4)
+        sbuf.view("fp32", n).fill_(1.0)
+        sends = comm.register(sbuf)
+        comm.allreduce(sends, rbuf.ptr, n, "fp32")  # both ranks take part once
+        if rank == 1:  # leaves between calls, with nothing of its own in flight
+            comm.close()
+            q.put((rank, "left"))
+            os._exit(0)
+        try:
+            comm.allreduce(sends, rbuf.ptr, n, "fp32")
+            q.put((rank, "no error"))
+        except SC.SimCommError as e:
+            q.put((rank, "timeout" if e.status == SC.TIMEOUT else f"status {e.status}"))
+        os._exit(0)  # the group is broken: no orderly shutdown
+    except Exception as e:
+        q.put((rank, f"{type(e).__name__}: {e}"))
+
+
+def test_a_rank_that_leaves_makes_the_next_call_time_out():
+    res, _ = _spawn(_leaver, 2, timeout=180)
+    assert res == {0: "timeout", 1: "left"}, res
