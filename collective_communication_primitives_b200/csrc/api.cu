@@ -1795,7 +1795,7 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
 extern "C" coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
                                        coll_stream_t stream) {
     if (kind < PROBE_LOAD || kind > PROBE_BULK_FANOUT) return fail(COLL_ERR_INVALID_ARG, "unknown probe kind");
-    if (ctas_per_sm < 1 || ctas_per_sm > 32) return fail(COLL_ERR_INVALID_ARG, "ctas_per_sm must be in [1, 32]");
+    if (ctas_per_sm < 0 || ctas_per_sm > 32) return fail(COLL_ERR_INVALID_ARG, "ctas_per_sm must be in [0, 32]");
     if (bytes == 0) return COLL_OK;
     if (check_probe_bytes(bytes) != COLL_OK) return COLL_ERR_INVALID_ARG;
     if (kind == PROBE_BULK_FANOUT && (bytes % (32 * 1024) != 0 || bytes > (size_t(1) << 40)))

@@ -616,17 +616,16 @@ static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cuda
 }
 
 // Per-collective defaults, the fastest measured on B200 at the DP-bucket size (p = 8, 100 MiB per
-// rank) with tasks claimed in order, each row charged with its own write-back: every bulk-copy
-// collective on 2 stages of 32 KiB with 3 CTAs per SM, block after block (All-to-All 0.259 ms
-// against 0.345-0.405 ms for the deeper 1-2 CTA shapes; Broadcast and AllGather 0.168 ms against
-// 0.170-0.176); All-to-Allv on the load/store path, block after block.
+// rank) with tasks claimed in order, each row charged with its own write-back: every collective on
+// 2 stages of 32 KiB with 3 CTAs per SM, block after block (All-to-All 0.257 ms against 0.345-0.405
+// ms for the deeper 1-2 CTA shapes; Broadcast and AllGather 0.166-0.167 ms against 0.170-0.176;
+// All-to-Allv on the Zipf counts 0.266 ms against 0.276 on the load/store path and 0.282 in the
+// interleaved order).
 constexpr int kVariantLsu = kNumCopyShapes;
 
-void copy_defaults(int kind, int* variant, int* order) {
-    switch (kind) {
-        case COPY_ALLTOALLV: *variant = kVariantLsu; *order = 0; break;
-        default: *variant = 6; *order = 0; break;
-    }
+void copy_defaults(int, int* variant, int* order) {
+    *variant = 6;
+    *order = 0;
 }
 
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {

@@ -139,20 +139,22 @@ cudaError_t launch_probe(int kind, void* dst, const void* src, size_t bytes, int
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_probe_fanout, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<uint32_t>(ntiles, 1u));
+        const size_t grid = std::min<size_t>(size_t(num_sms) * std::max(ctas_per_sm, 1), std::max<uint32_t>(ntiles, 1u));
         k_probe_fanout<<<unsigned(grid), 32, smem, s>>>(static_cast<char*>(dst), static_cast<const char*>(src), bytes,
                                                       ntiles);
         return cudaGetLastError();
     }
     if (kind == PROBE_BULK_STORE) {
         const size_t ntiles = bytes / kProbeTile;
-        const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<size_t>(ntiles, 1));
+        const size_t want = std::max<size_t>(ntiles, 1);  // one pass: a CTA per tile
+        const size_t grid = ctas_per_sm > 0 ? std::min<size_t>(size_t(num_sms) * ctas_per_sm, want) : want;
         k_probe_bulk_store<<<unsigned(grid), 32, 0, s>>>(static_cast<char*>(dst), ntiles);
         return cudaGetLastError();
     }
     const size_t nvec = bytes / 32;
     const size_t per_cta = size_t(kProbeThreads) * kProbeUnroll;
-    const size_t grid = std::min<size_t>(size_t(num_sms) * ctas_per_sm, std::max<size_t>((nvec + per_cta - 1) / per_cta, 1));
+    const size_t want = std::max<size_t>((nvec + per_cta - 1) / per_cta, 1);  // one pass: a CTA per iteration
+    const size_t grid = ctas_per_sm > 0 ? std::min<size_t>(size_t(num_sms) * ctas_per_sm, want) : want;
     char* d = static_cast<char*>(dst);
     const char* x = static_cast<const char*>(src);
     switch (kind) {

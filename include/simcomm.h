@@ -195,9 +195,10 @@ const char* coll_status_string(coll_status_t status);
  *                  its chunks, the butterfly executor never counts its tasks, the LL kernels never
  *                  send its words), so a successor times out (-1 = off, the default). Host-side
  *                  fault injection only.
- *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v): -1 = the default per
- *                  collective; 0..7 = a bulk-copy pipeline shape (stages x tile bytes, CTAs per SM);
- *                  8 = the 16-byte load/store path (All-to-All(v) only)
+ *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v)/Scatter/Gather: -1 = the
+ *                  default (2 stages x 32 KiB, 3 CTAs per SM); 0..7 = a bulk-copy pipeline shape
+ *                  (stages x tile bytes, CTAs per SM); 8 = the 16-byte load/store path (All-to-All(v)
+ *                  only). Every copy path takes its tiles in order from a shared counter.
  *   "copy_order"   tile order of the direct copy paths: -1 = the default per collective,
  *                  1 = interleaved over all blocks, 0 = block after block
  *   "direct_pack"  access width of the fused reduction: 0 = widest the alignment allows
@@ -393,7 +394,9 @@ coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_r
  *   dst, src  DEVICE pointers, 256-byte aligned, non-overlapping; src is unused by kinds 1 and 3, dst
  *             by kind 0 (either may then be NULL).
  *   bytes     a multiple of 16 KiB (kind 4: of 32 KiB, at most 2^40; 0: nothing is enqueued).
- *   ctas_per_sm  CTAs per SM of the grid, in [1, 32].
+ *   ctas_per_sm  CTAs per SM of a persistent grid-stride grid, in [1, 32]; 0 = one pass (kinds 0-3:
+ *             a CTA per 32 KiB of the loop or per 16 KiB tile, dispatched in address order as SMs free
+ *             up; kind 4: one CTA per SM).
  * Enqueues one kernel on the stream. COLL_ERR_INVALID_ARG for a bad kind, size, pointer or overlap. */
 coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, int ctas_per_sm,
                             coll_stream_t stream);
