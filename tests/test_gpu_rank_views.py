@@ -127,6 +127,15 @@ def test_rank_views_match_the_oracle(world, dtype, op):
     assert codes == [0] * world
 
 
+def _report_and_exit(q, item):
+    """Puts the result and flushes the queue's feeder thread before leaving without cleanup (the
+    process group is broken, so no orderly shutdown)."""
+    q.put(item)
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
 def _leaver(rank, world, port, q):
     try:
         _setup(rank, world, port, 5)
@@ -140,16 +149,14 @@ def _leaver(rank, world, port, q):
         comm.allreduce(sends, rbuf.ptr, n, "fp32")  # both ranks take part once
         if rank == 1:  # leaves between calls, with nothing of its own in flight
             comm.close()
-            q.put((rank, "left"))
-            os._exit(0)
+            _report_and_exit(q, (rank, "left"))
         try:
             comm.allreduce(sends, rbuf.ptr, n, "fp32")
-            q.put((rank, "no error"))
+            _report_and_exit(q, (rank, "no error"))
         except SC.SimCommError as e:
-            q.put((rank, "timeout" if e.status == SC.TIMEOUT else f"status {e.status}"))
-        os._exit(0)  # the group is broken: no orderly shutdown
+            _report_and_exit(q, (rank, "timeout" if e.status == SC.TIMEOUT else f"status {e.status}"))
     except Exception as e:
-        q.put((rank, f"{type(e).__name__}: {e}"))
+        _report_and_exit(q, (rank, f"{type(e).__name__}: {e}"))
 
 
 def test_a_rank_that_leaves_makes_the_next_call_time_out():
