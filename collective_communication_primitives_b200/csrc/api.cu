@@ -1714,7 +1714,7 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     const size_t chunk = (size_t(1) << 20) / 4;
     const uint32_t nch = chunks_of(seg, chunk);
     const uint32_t nsteps = uint32_t(2 * (p - 1));
-    const size_t ctl_bytes = 256;
+    const size_t ctl_bytes = round_up(sizeof(DevState) + 8, 256);
     const size_t flag_bytes = round_up(size_t(nsteps) * p * nch * sizeof(unsigned long long), 256);
     const size_t stride = round_up(n * 4, 256);
     const size_t need = ctl_bytes + flag_bytes + size_t(p) * stride;
@@ -1769,7 +1769,7 @@ extern "C" coll_status_t coll_allreduce_ring_noalloc(int p, coll_bufs_t b, size_
     a.timeout_ns = uint64_t(env_option("SIMCOMM_TIMEOUT_NS", 2000000000LL, 1000, LLONG_MAX));
     a.st = reinterpret_cast<DevState*>(base);
     a.ctl.status = &a.st->status;
-    static_assert(sizeof(DevState) + 8 <= 256, "control words must fit the 256-byte control region");
+
     a.ctl.host_status = reinterpret_cast<uint32_t*>(base + sizeof(DevState));
     a.ctl.abort_flag = reinterpret_cast<uint32_t*>(base + sizeof(DevState) + 4);
     a.ctl.abort_clock = &a.st->abort_clock;

@@ -21,6 +21,9 @@ struct DevState {
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
     unsigned long long abort_clock;  // global time of the last read of the host abort word
     unsigned long long moe_task;     // fused MoE dispatch: next token row to claim (zero between calls)
+    // fused MoE dispatch: grid barriers done so far, set by the last CTA to arrive; a 128-byte line
+    // of its own, so that the CTAs polling it do not queue behind the arrivals' atomics on moe_ctr
+    alignas(128) uint32_t moe_gen;
 };
 
 // What a kernel needs to report errors and notice an abort.

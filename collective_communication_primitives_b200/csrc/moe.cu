@@ -364,22 +364,43 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
 //   phase 2  a warp per (rank, expert) column: exclusive prefix of the tile counts over tiles, the
 //            total cnt[i][e] and c[i][j] += cnt[i][e] (integer atomics: exact in any order);
 //   phase 3  every CTA turns c into R[i][j] = Σ_{q<i} c[q][j] in shared memory and checks every
-//            destination's capacity (the same decision everywhere); a warp per (rank, destination)
-//            block writes base[i][e] = R[i][j] + Σ of cnt[i][·] over the block's lower experts;
+//            destination's capacity (the same decision everywhere); base[i][e] = R[i][j] + Σ of
+//            cnt[i][·] over the block's lower experts, built by every CTA in its shared memory when
+//            the table is small, else by a warp per (rank, destination) block in global memory
+//            (with a third barrier);
 //   phase 4  the copy: warps claim batches of consecutive token rows in order and copy each row with
 //            32/16-byte loads and one store per slot;
 // with a bounded grid barrier between phases. Data other CTAs wrote in this kernel is read through
 // L2 (ld.global.cg): L1 is not coherent between SMs.
+// Build-time knobs of the copy phase (measured on B200; the defaults are the fastest found).
+#ifndef SIMCOMM_MOE_FUSED_UNROLL
+#define SIMCOMM_MOE_FUSED_UNROLL 8   // packs in flight per lane
+#endif
+#ifndef SIMCOMM_MOE_FUSED_BATCH
+#define SIMCOMM_MOE_FUSED_BATCH 2    // most token rows a warp claims at once (at most 32 / k rounded up)
+#endif
 constexpr int kFusedThreads = kMoeTile;  // a counting tile per CTA pass
-constexpr int kFusedUnroll = 8;          // packs in flight per lane in the copy
+constexpr int kFusedUnroll = SIMCOMM_MOE_FUSED_UNROLL;
+constexpr int kWarpHistMaxE = 1024;      // per-warp counting histograms up to this many experts (32 KiB)
+constexpr int kSmemBaseMax = 8192;       // every CTA keeps base[p][E] in shared memory up to this many entries
 
+static size_t fused_smem_ints(int p, int E) {
+    const size_t hist = E <= kWarpHistMaxE ? size_t(kFusedThreads / 32) * E : size_t(E);
+    const size_t base = size_t(p) * E <= size_t(kSmemBaseMax) ? size_t(p) * E : 0;
+    return size_t(p) * p + p + std::max(hist, base);
+}
+
+// The k-th grid barrier of a call (k = 1, 2, ...): a CTA arrives on moe_ctr; the last of the k-th
+// round of arrivals publishes k in moe_gen, which the others poll (a line the arrivals do not touch:
+// with every CTA polling the arrival counter itself, the arrivals queued behind the polls and one
+// barrier took tens of microseconds).
 __device__ __forceinline__ bool moe_grid_barrier(const MoeArgs& a, uint32_t k) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        atomicAdd(&a.st->moe_ctr, 1u);
-        s_ok = wait_counter(a.ctl, &a.st->moe_ctr, k * gridDim.x, a.timeout_ns) && !status_failed(a.ctl);
+        if (atomicAdd(&a.st->moe_ctr, 1u) == k * gridDim.x - 1) st_release_gpu(&a.st->moe_gen, k);
+        s_ok = wait_counter(a.ctl, &a.st->moe_gen, k, a.timeout_ns) && !status_failed(a.ctl);
     }
     __syncthreads();
     return s_ok != 0;
@@ -387,15 +408,22 @@ __device__ __forceinline__ bool moe_grid_barrier(const MoeArgs& a, uint32_t k) {
 
 template <int W>
 __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __grid_constant__ MoeArgs a) {
-    extern __shared__ int s_dyn[];  // [E] counting histogram, then [p][p] c -> R, then [p] column totals
+    // dynamic shared memory: [p][p] c -> R, [p] column totals, then a region used first for the
+    // counting histograms ([8][E] per-warp counts when E <= kWarpHistMaxE, else [E]) and then, when
+    // p * E <= kSmemBaseMax, for the first rows base[p][E]
+    extern __shared__ int s_dyn[];
     __shared__ char* s_dst[kFusedThreads / 32][32];
     __shared__ int s_flag;
     if (cta_failed(a.ctl)) return;
     const int p = a.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int* s_cnt = s_dyn;
-    int* s_c = s_dyn + a.E;
+    int* s_c = s_dyn;
     int* s_tot = s_c + p * p;
+    int* s_cnt = s_tot + p;
+    const bool warp_hist = a.E <= kWarpHistMaxE;
+    const int hist_ints = warp_hist ? (kFusedThreads / 32) * a.E : a.E;
+    const bool smem_base = p * a.E <= kSmemBaseMax;
+    int* s_base = s_cnt;
 
     // ---- phase 1: counting ----
     if (blockIdx.x == 0)
@@ -405,7 +433,7 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         const int i = int(g / a.ntiles);
         const uint32_t tile = g % a.ntiles;
         __syncthreads();  // the previous tile's histogram has been written out
-        for (int e = threadIdx.x; e < a.E; e += kFusedThreads) s_cnt[e] = 0;
+        for (int e = threadIdx.x; e < hist_ints; e += kFusedThreads) s_cnt[e] = 0;
         __syncthreads();
         const size_t asg = size_t(tile) * kMoeTile + threadIdx.x;
         const bool valid = asg < a.A;
@@ -414,24 +442,41 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
             raise_status(a.ctl, COLL_ERR_INVALID_ARG);
             e = -1;
         }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int leader = __ffs(same) - 1;
+        const int below = __popc(same & ((1u << lane) - 1u));  // same-expert assignments before it in the warp
         int rank = 0;
-        for (int w = 0; w < kFusedThreads / 32; ++w) {  // warps in order: ranks follow assignment order
-            if (warp == w) {
-                const unsigned same = __match_any_sync(0xffffffffu, e);
-                const int leader = __ffs(same) - 1;
-                int first = 0;
-                if (lane == leader && e >= 0) {
-                    first = s_cnt[e];
-                    s_cnt[e] = first + __popc(same);
-                }
-                first = __shfl_sync(0xffffffffu, first, leader);
-                rank = first + __popc(same & ((1u << lane) - 1u));
-            }
+        int32_t* hist = a.tile_hist + (size_t(i) * a.ntiles + tile) * a.E;
+        if (warp_hist) {
+            // every warp counts its own experts, then an assignment's rank adds the counts of the
+            // warps before it: no turn-taking
+            if (lane == leader && e >= 0) s_cnt[warp * a.E + e] = __popc(same);
             __syncthreads();
+            if (e >= 0) {
+                for (int w = 0; w < warp; ++w) rank += s_cnt[w * a.E + e];
+                rank += below;
+            }
+            for (int x = threadIdx.x; x < a.E; x += kFusedThreads) {
+                int t = 0;
+#pragma unroll
+                for (int w = 0; w < kFusedThreads / 32; ++w) t += s_cnt[w * a.E + x];
+                hist[x] = t;
+            }
+        } else {
+            for (int w = 0; w < kFusedThreads / 32; ++w) {  // warps in order: ranks follow assignment order
+                if (warp == w) {
+                    int first = 0;
+                    if (lane == leader && e >= 0) {
+                        first = s_cnt[e];
+                        s_cnt[e] = first + __popc(same);
+                    }
+                    rank = __shfl_sync(0xffffffffu, first, leader) + below;
+                }
+                __syncthreads();
+            }
+            for (int x = threadIdx.x; x < a.E; x += kFusedThreads) hist[x] = s_cnt[x];
         }
         if (valid) a.rank_in_tile[size_t(i) * a.A + asg] = rank;
-        int32_t* hist = a.tile_hist + (size_t(i) * a.ntiles + tile) * a.E;
-        for (int x = threadIdx.x; x < a.E; x += kFusedThreads) hist[x] = s_cnt[x];
     }
     if (!moe_grid_barrier(a, 1)) return;
 
@@ -485,22 +530,38 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(a.ctl, COLL_ERR_OVERFLOW);
         return;
     }
-    for (uint32_t blk = gw; blk < uint32_t(p) * uint32_t(p); blk += nwarps) {
-        const int i = int(blk / uint32_t(p)), j = int(blk % uint32_t(p));
-        int run = s_c[i * p + j];
-        for (int e0 = j * a.E_loc; e0 < (j + 1) * a.E_loc; e0 += 32) {
-            const int e = e0 + lane;
-            const int v = e < (j + 1) * a.E_loc ? __ldcg(a.cnt + size_t(i) * a.E + e) : 0;
-            const int incl = warp_incl_scan_i(v, lane);
-            if (e < (j + 1) * a.E_loc) a.base[size_t(i) * a.E + e] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+    if (smem_base) {
+        // every CTA builds the whole table in its shared memory: no third barrier
+        for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) s_base[x] = __ldcg(a.cnt + x);
+        __syncthreads();
+        for (int blk = threadIdx.x; blk < p * p; blk += kFusedThreads) {  // (rank, destination) blocks
+            const int i = blk / p, j = blk % p;
+            int run = s_c[i * p + j];
+            for (int e = j * a.E_loc; e < (j + 1) * a.E_loc; ++e) {
+                const int v = s_base[i * a.E + e];
+                s_base[i * a.E + e] = run;
+                run += v;
+            }
         }
+        __syncthreads();
+    } else {
+        for (uint32_t blk = gw; blk < uint32_t(p) * uint32_t(p); blk += nwarps) {
+            const int i = int(blk / uint32_t(p)), j = int(blk % uint32_t(p));
+            int run = s_c[i * p + j];
+            for (int e0 = j * a.E_loc; e0 < (j + 1) * a.E_loc; e0 += 32) {
+                const int e = e0 + lane;
+                const int v = e < (j + 1) * a.E_loc ? __ldcg(a.cnt + size_t(i) * a.E + e) : 0;
+                const int incl = warp_incl_scan_i(v, lane);
+                if (e < (j + 1) * a.E_loc) a.base[size_t(i) * a.E + e] = run + incl - v;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+        if (!moe_grid_barrier(a, 3)) return;
     }
-    if (!moe_grid_barrier(a, 3)) return;
 
     // ---- phase 4: the copy, batches of consecutive token rows claimed in order ----
     const size_t row_bytes = a.H * size_t(a.elem_bytes);
-    const int kslot = slot_width(a.k), per_batch = 32 / kslot;
+    const int kslot = slot_width(a.k), per_batch = min(32 / kslot, SIMCOMM_MOE_FUSED_BATCH);
     const int my_b = lane / kslot, my_s = lane % kslot;
     const unsigned long long rows = (unsigned long long)p * a.T;
     while (true) {
@@ -510,12 +571,13 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         if (u0 >= rows) break;
         const unsigned long long my_u = u0 + unsigned(my_b);
         bool bad = false;
-        if (my_s < a.k && my_u < rows) {
+        if (my_s < a.k && my_b < per_batch && my_u < rows) {
             const int i = int(my_u / a.T);
             const size_t t = size_t(my_u % a.T);
             const size_t asg = t * a.k + my_s;
             const int e = a.idx[i][asg];
-            const long long row = (long long)__ldcg(a.base + size_t(i) * a.E + e) +
+            const int first = smem_base ? s_base[i * a.E + e] : __ldcg(a.base + size_t(i) * a.E + e);
+            const long long row = (long long)first +
                                   __ldcg(a.tile_hist + (size_t(i) * a.ntiles + asg / kMoeTile) * a.E + e) +
                                   __ldcg(a.rank_in_tile + size_t(i) * a.A + asg);
             bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
@@ -563,6 +625,7 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         if (atomicAdd(&a.st->done_ctr, 1u) == gridDim.x - 1) {
             a.st->moe_task = 0;
             a.st->moe_ctr = 0;
+            a.st->moe_gen = 0;
             a.st->done_ctr = 0;
             __threadfence();
         }
@@ -780,7 +843,7 @@ static cudaError_t launch_after(void (*kernel)(MoeArgs), dim3 grid, dim3 block, 
 template <int W>
 static cudaError_t launch_fused(const MoeArgs& a, int num_sms, cudaStream_t s) {
     auto kernel = k_moe_dispatch_fused<W>;
-    const size_t smem = (size_t(a.E) + size_t(a.p) * a.p + size_t(a.p)) * sizeof(int);
+    const size_t smem = fused_smem_ints(a.p, a.E) * sizeof(int);
     cudaError_t e = cudaSuccess;
     if (smem > 48 * 1024) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
