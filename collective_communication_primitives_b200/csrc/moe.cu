@@ -429,15 +429,24 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
     if (blockIdx.x == 0)
         for (int x = threadIdx.x; x < p * p; x += kFusedThreads) a.cmat[x] = 0;
     const uint32_t ntask = uint32_t(p) * a.ntiles;
+    // this thread's expert id in the CTA's g-th tile (-1 past the end); the next tile's id is loaded
+    // before the current tile is counted, so its latency overlaps the counting
+    auto load_id = [&](uint32_t g) -> int {
+        if (g >= ntask) return -1;
+        const size_t asg = size_t(g % a.ntiles) * kMoeTile + threadIdx.x;
+        return asg < a.A ? a.idx[g / a.ntiles][asg] : -1;
+    };
+    int e_next = load_id(blockIdx.x);
     for (uint32_t g = blockIdx.x; g < ntask; g += gridDim.x) {
         const int i = int(g / a.ntiles);
         const uint32_t tile = g % a.ntiles;
+        int e = e_next;
+        e_next = load_id(g + gridDim.x);
         __syncthreads();  // the previous tile's histogram has been written out
-        for (int e = threadIdx.x; e < hist_ints; e += kFusedThreads) s_cnt[e] = 0;
+        for (int x = threadIdx.x; x < hist_ints; x += kFusedThreads) s_cnt[x] = 0;
         __syncthreads();
         const size_t asg = size_t(tile) * kMoeTile + threadIdx.x;
         const bool valid = asg < a.A;
-        int e = valid ? a.idx[i][asg] : -1;
         if (valid && (e < 0 || e >= a.E)) {
             raise_status(a.ctl, COLL_ERR_INVALID_ARG);
             e = -1;
