@@ -36,12 +36,9 @@ N_BUCKET = 26_214_400
 HIDDEN = 4096
 ROOT_RANK = 2
 FALLBACK_HBM_GBS = 6650.0
-# dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of a row's kernel, with the
-# per-rank element count of that capture; scaled to the bench's size by elements moved. Empty
-# until a capture of the current build is taken.
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a row's kernel, from an
 # ncu capture of the current build, and the per-rank element count it was captured at.
-NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_187_871_232 + 1_420_613_120, 26_214_400)}
+NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_187_028_736 + 1_416_167_424, 26_214_400)}
 SPACER_CYCLES = 4_000_000  # ~2 ms of a spinning kernel ahead of a timed region
 
 
