@@ -506,6 +506,81 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     if (threadIdx.x == 0) leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
 }
 
+// ---- lean fan-out: Broadcast and AllGather on 16-byte aligned buffers -------------------------------
+// The fan-out pattern with nothing else on the critical path (the loop of the bulk fan-out probe):
+// one lane issues everything; each segment (the root's buffer, or a rank's shard) is cut into whole
+// 32 KiB tiles, the last one shorter (a multiple of 16 bytes when the segment is); task t is tile
+// t % per_seg of segment t / per_seg, claimed in order; a tile is loaded once and stored to every
+// destination except the source itself (the in-place forms). Used when every buffer is 16-byte
+// aligned and the segment a whole number of 16-byte units, so no tile needs a byte head or tail.
+constexpr int kFanStages = 4;
+constexpr uint32_t kFanTile = 32 * 1024;
+
+template <int KIND>
+__global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs a) {
+    static_assert(KIND == COPY_BCAST || KIND == COPY_ALLGATHER, "fan-out collectives only");
+    extern __shared__ __align__(128) unsigned char stages[];
+    __shared__ uint64_t bars[kFanStages];
+    __shared__ uint32_t s_task[kFanStages];
+    if (threadIdx.x != 0) return;
+    if (status_failed(a.ctl)) return;
+    const int p = a.p;
+    const size_t seg_bytes = a.blk_elems * size_t(a.elem_bytes);
+    const uint32_t per_seg = uint32_t((seg_bytes + kFanTile - 1) / kFanTile);
+    const uint32_t total = per_seg * uint32_t(KIND == COPY_BCAST ? 1 : p);
+    for (int st = 0; st < kFanStages; ++st) mbar_init(&bars[st], 1);
+    fence_barrier_init();
+    auto source = [&](uint32_t t) -> const char* {
+        const uint32_t q = t / per_seg;
+        return static_cast<const char*>(a.ptrs.send[KIND == COPY_BCAST ? a.root : int(q)]) +
+               size_t(t % per_seg) * kFanTile;
+    };
+    auto tile_bytes = [&](uint32_t t) -> uint32_t {
+        const size_t off = size_t(t % per_seg) * kFanTile;
+        return uint32_t(min(size_t(kFanTile), seg_bytes - off));
+    };
+    uint32_t phase = 0, head = 0, tail = 0;
+    bool more = true, failed = false;
+    auto issue = [&]() {
+        const uint32_t t = claim_task(a.ctl, &a.st->task_ctr, total);
+        if (t >= total) {
+            more = false;
+            return;
+        }
+        const int st = int(head % kFanStages);
+        s_task[st] = t;
+        mbar_arrive_expect_tx(&bars[st], tile_bytes(t));
+        bulk_g2s(stages + size_t(st) * kFanTile, source(t), tile_bytes(t), &bars[st]);
+        ++head;
+    };
+    while (more && head < kFanStages - 1) issue();
+    while (tail < head) {
+        const int st = int(tail % kFanStages);
+        if (!mbar_wait_bounded(a.ctl, &bars[st], (phase >> st) & 1u, a.timeout_ns)) {
+            failed = true;  // a load that never lands: stop issuing (the error is recorded)
+            break;
+        }
+        phase ^= 1u << st;
+        const uint32_t t = s_task[st];
+        const char* src = source(t);
+        const size_t dst_off = (KIND == COPY_ALLGATHER ? size_t(t / per_seg) * seg_bytes : 0) +
+                               size_t(t % per_seg) * kFanTile;
+        const uint32_t bytes = tile_bytes(t);
+        for (int r = 0; r < p; ++r) {
+            char* dst = static_cast<char*>(a.ptrs.recv[r]) + dst_off;
+            if (dst != src) bulk_s2g(dst, stages + size_t(st) * kFanTile, bytes);
+        }
+        bulk_commit();
+        ++tail;
+        if (more) {
+            bulk_wait_read_all();  // the next load reuses the stage task tail-1 was stored from
+            issue();
+        }
+    }
+    bulk_wait_all();
+    if (!failed) leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
+}
+
 // The current device as one bit of a mask (0 for devices 63 and up, which set the attribute every launch).
 static unsigned long long device_bit() {
     int dev = 0;
@@ -622,13 +697,46 @@ static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cuda
 // All-to-Allv on the Zipf counts 0.266 ms against 0.276 on the load/store path and 0.282 in the
 // interleaved order).
 constexpr int kVariantLsu = kNumCopyShapes;
+constexpr int kVariantFan1 = kNumCopyShapes + 1;  // lean fan-out, 1 CTA per SM
+constexpr int kVariantFan2 = kNumCopyShapes + 2;  // lean fan-out, 2 CTAs per SM
 
-void copy_defaults(int, int* variant, int* order) {
-    *variant = 6;
+void copy_defaults(int kind, int* variant, int* order) {
+    *variant = (kind == COPY_BCAST || kind == COPY_ALLGATHER) ? kVariantFan1 : 6;
     *order = 0;
 }
 
+// The lean fan-out path needs every touched buffer 16-byte aligned and whole 16-byte segments.
+static bool fanout_ok(const CopyArgs& a) {
+    if ((a.blk_elems * size_t(a.elem_bytes)) % 16 != 0) return false;
+    for (int r = 0; r < a.p; ++r) {
+        if (reinterpret_cast<uintptr_t>(a.ptrs.recv[r]) % 16 != 0) return false;
+        if ((a.kind == COPY_ALLGATHER || r == a.root) && reinterpret_cast<uintptr_t>(a.ptrs.send[r]) % 16 != 0)
+            return false;
+    }
+    return true;
+}
+
+template <int KIND>
+static cudaError_t launch_fanout(const CopyArgs& a, int num_sms, int ctas_per_sm, cudaStream_t s) {
+    static unsigned long long attr_set = 0;  // bit d: set on device d
+    const unsigned long long bit = device_bit();
+    const size_t smem = size_t(kFanStages) * kFanTile;
+    if (!(attr_set & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(k_fanout<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        attr_set |= bit;
+    }
+    k_fanout<KIND><<<num_sms * ctas_per_sm, 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
+    if (variant == kVariantFan1 || variant == kVariantFan2) {
+        const int cps = variant == kVariantFan1 ? 1 : 2;
+        if (a.kind == COPY_BCAST && fanout_ok(a)) return launch_fanout<COPY_BCAST>(a, num_sms, cps, s);
+        if (a.kind == COPY_ALLGATHER && fanout_ok(a)) return launch_fanout<COPY_ALLGATHER>(a, num_sms, cps, s);
+        variant = 6;  // other collectives, or unaligned buffers: the general engine
+    }
     if (variant == kVariantLsu) {
         if (a.kind == COPY_ALLTOALL) return launch_lsu<COPY_ALLTOALL>(a, num_sms, s);
         if (a.kind == COPY_ALLTOALLV) return launch_lsu<COPY_ALLTOALLV>(a, num_sms, s);
@@ -645,6 +753,6 @@ cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_
     }
 }
 
-int copy_num_variants() { return kNumCopyShapes + 1; }
+int copy_num_variants() { return kNumCopyShapes + 3; }
 
 }  // namespace simcomm
