@@ -337,7 +337,7 @@ coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, col
 coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_elems, coll_dtype_t dt, int root,
                        bool use_send_all, cudaStream_t s, const long long* counts = nullptr,
                        const long long* send_cap = nullptr, const long long* recv_cap = nullptr,
-                       long long* recv_counts = nullptr, int p_override = 0) {
+                       long long* recv_counts = nullptr, int p_override = 0, int only_dst = -1) {
     const int p = p_override > 0 ? p_override : c->p;
     CopyArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -364,6 +364,7 @@ coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_e
     a.order = order;
     a.l2_hint = int(c->l2_hint);
     a.st = c->dstate;
+    a.only_dst_plus1 = only_dst + 1;
     a.ctl = make_ctl(c);
     cudaError_t e = launch_copy(a, c->num_sms, variant, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
@@ -1436,7 +1437,6 @@ static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if ((st = check_algo(algo)) != COLL_OK) return st;
-    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "All-to-Allv is not built for rank views");
     if (!counts_dev || !send_cap || !recv_cap) return fail(COLL_ERR_INVALID_ARG, "null counts or capacities");
     if (!b.send || !b.recv) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
     if (reinterpret_cast<uintptr_t>(counts_dev) % 8 != 0 ||
@@ -1445,6 +1445,7 @@ static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long
     const int p = c->p;
     const size_t d = dtype_bytes(dt);
     std::vector<Range> rs;
+    const bool view = c->rank >= 0;  // a rank view writes only its own output
     for (int r = 0; r < p; ++r) {
         if (send_cap[r] < 0 || recv_cap[r] < 0) return fail(COLL_ERR_INVALID_ARG, "negative capacity");
         if ((st = check_count(size_t(send_cap[r]), "send_cap")) != COLL_OK ||
@@ -1452,12 +1453,23 @@ static coll_status_t coll_alltoallv_impl(sim_comm_t c, coll_bufs_t b, const long
             return st;
         const size_t sb = size_t(send_cap[r]) * d, rb = size_t(recv_cap[r]) * d;
         if ((st = check_ptr(b.send[r], sb, d, "send")) != COLL_OK) return st;
-        if ((st = check_ptr(b.recv[r], rb, d, "recv")) != COLL_OK) return st;
         rs.push_back({uintptr_t(b.send[r]), uintptr_t(b.send[r]) + sb, false, r});
+        if (view && r != c->rank) continue;
+        if ((st = check_ptr(b.recv[r], rb, d, "recv")) != COLL_OK) return st;
         rs.push_back({uintptr_t(b.recv[r]), uintptr_t(b.recv[r]) + rb, true, r});
     }
     if ((st = check_ranges(rs, INPLACE_NONE, 0)) != COLL_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (view) {
+        if (algo != COLL_ALGO_DIRECT)
+            return fail(COLL_ERR_UNSUPPORTED, "a rank view runs the direct path only");
+        // the blocks bound for this rank, pulled from every source (each rank holds the whole count
+        // matrix, so every rank computes the same displacements and capacity decision)
+        std::vector<void*> recv(p, nullptr);
+        recv[c->rank] = b.recv[c->rank];
+        return run_copy(c, coll_bufs_t{b.send, recv.data()}, COPY_ALLTOALLV, 0, dt, 0, true, s, counts_dev, send_cap,
+                        recv_cap, recv_counts_dev, 0, c->rank);
+    }
     if (algo == COLL_ALGO_DIRECT || p == 1)
         return run_copy(c, b, COPY_ALLTOALLV, 0, dt, 0, true, s, counts_dev, send_cap, recv_cap, recv_counts_dev);
     RingPlan pl;

@@ -75,11 +75,14 @@ __device__ __forceinline__ SegDesc segment(const CopyArgs& a, int s, const long 
         d.fanout = false;
         d.len = (d.src == d.dst) ? 0 : a.blk_elems * e;
     } else {
-        const int i = s / a.p, j = s % a.p;
-        d.src = static_cast<const char*>(a.ptrs.send[i]) + size_t(sd[s]) * e;
-        d.dst = static_cast<char*>(a.ptrs.recv[j]) + size_t(rd[s]) * e;
+        // a rank view's All-to-Allv has the p blocks bound for its own rank only: segment s is the
+        // block from source s
+        const int ij = a.only_dst_plus1 ? s * a.p + (a.only_dst_plus1 - 1) : s;
+        const int i = ij / a.p, j = ij % a.p;
+        d.src = static_cast<const char*>(a.ptrs.send[i]) + size_t(sd[ij]) * e;
+        d.dst = static_cast<char*>(a.ptrs.recv[j]) + size_t(rd[ij]) * e;
         d.fanout = false;
-        d.len = size_t(a.counts[s]) * e;
+        d.len = size_t(a.counts[ij]) * e;
     }
     return d;
 }
@@ -199,6 +202,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
 
     const int p = a.p;
     const int nseg = (KIND == COPY_BCAST) ? 1 : (KIND == COPY_ALLTOALL || KIND == COPY_ALLTOALLV) ? p * p : p;
+    const int nseg_run = (KIND == COPY_ALLTOALLV && a.only_dst_plus1) ? p : nseg;  // segments this call copies
     unsigned char* stages = smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kStages) * kTile);
     long long* sd = reinterpret_cast<long long*>(bars + kStages);
@@ -210,6 +214,8 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         const A2avPlan plan = a2av_plan_warp(a.counts, p, a.send_cap, a.recv_cap, sd, rd, a.recv_counts_out, a.ctl);
         if (!plan.ok) return;
     }
+    {
+    const int nseg = nseg_run;
 
     // tile counts per segment, then an inclusive scan into prefix[1..nseg]
     for (int s = lane; s < nseg; s += 32) {
@@ -374,6 +380,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
     }
     __syncwarp();
+    }
 }
 
 // ---- load/store path -----------------------------------------------------------------------------
@@ -421,7 +428,8 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int s_run;
     const int p = a.p;
-    const int nseg = p * p;
+    const int nseg_all = p * p;
+    const int nseg = (KIND == COPY_ALLTOALLV && a.only_dst_plus1) ? p : nseg_all;  // segments this call copies
     long long* sd = reinterpret_cast<long long*>(smem);
     long long* rd = sd + ((KIND == COPY_ALLTOALLV) ? p * p : 0);
     uint32_t* prefix = reinterpret_cast<uint32_t*>(rd + ((KIND == COPY_ALLTOALLV) ? p * p : 0));

@@ -76,6 +76,7 @@ struct CopyArgs {
     long long recv_cap[kMaxRanks];     // ALLTOALLV: elements per recv buffer
     uint64_t timeout_ns;
     DevState* st;                      // task counters (dynamic distribution)
+    int only_dst_plus1;                // ALLTOALLV of a rank view: 1 + the one destination it copies, 0 = all
     Ctl ctl;
 };
 

@@ -150,6 +150,12 @@ class RankComm(SC.SimComm):
     def gather(self, sends, recv, root, n, dtype, algo="direct"):
         self._call(super().gather, sends, self._outs(recv), root, algo=algo, n=n, dtype=dtype)
 
+    def alltoallv(self, sends, recv, counts, send_cap, recv_cap, dtype, algo="direct", recv_counts=None):
+        """counts: this process's device copy of the whole int64 [p][p] count matrix (the same on every
+        rank); send_cap / recv_cap: every rank's capacities, in elements."""
+        self._call(super().alltoallv, sends, self._outs(recv), counts, send_cap=send_cap, recv_cap=recv_cap,
+                   algo=algo, recv_counts=recv_counts, dtype=dtype)
+
     def close(self):
         for ptr in getattr(self, "_opened", []):
             self._L.sim_ipc_close(ctypes.c_void_p(ptr))

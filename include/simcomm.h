@@ -140,9 +140,11 @@ sim_comm_t sim_comm_create(int p);
  * output; the other recv entries are ignored (may be NULL). A call computes this rank's output only,
  * reading the inputs it needs where they lie, with the direct path's kernels, fold order and
  * rounding, so the output equals the whole communicator's direct-path output for this rank bit for
- * bit. Supported: AllReduce, Reduce, Broadcast, ReduceScatter, AllGather, All-to-All, Scatter,
+ * bit. Supported: AllReduce, Reduce, Broadcast, ReduceScatter, AllGather, All-to-All, All-to-Allv
+ * (counts_dev: this process's device copy of the whole count matrix, identical on every rank;
+ * send_cap and recv_cap: every rank's capacities; only this rank's blocks are copied), Scatter,
  * Gather, COLL_ALGO_DIRECT only (the other schedules wait on other ranks inside their kernels:
- * COLL_ERR_UNSUPPORTED, as for All-to-Allv and the MoE calls). Reduce and Gather enqueue nothing
+ * COLL_ERR_UNSUPPORTED, as for the MoE calls). Reduce and Gather enqueue nothing
  * on a non-root rank. No output may overlap any rank's input (a peer may still be reading it), except
  * the root's own in-place Broadcast and Scatter forms. The ranks' calls are not synchronised by the
  * library: before a call every rank's inputs must be complete, and no rank may modify its input until

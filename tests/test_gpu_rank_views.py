@@ -93,6 +93,18 @@ def _collectives(rank, world, port, dtype, op, q):
         out.copy_(sentinel)
         comm.gather(sends, rbuf.ptr, 0, n, dtype)
         check("gather", O.gather(shards, dtype, 0) if rank == 0 else to_numpy(sentinel, dtype))
+        # All-to-Allv on a seeded count matrix, the same on every rank; rank i sends the first
+        # Σ_j c[i][j] elements of its input
+        import torch
+
+        from collective_communication_primitives_b200 import synth as S
+        cmat = S.ints(f"ranks.counts.{p}", p * p, 0, m // p).astype(np.int64).reshape(p, p)
+        counts_dev = torch.from_numpy(cmat).cuda()
+        send_cap = [n] * p
+        recv_cap = [int(cmat[:, j].sum()) for j in range(p)]
+        comm.alltoallv(sends, rbuf.ptr, counts_dev, send_cap, recv_cap, dtype)
+        want_v, _ = O.alltoallv([ins[i][:int(cmat[i].sum())] for i in range(p)], cmat, dtype)
+        check("alltoallv", want_v[rank])
         assert comm.async_error() == 0
         comm.sync()
         comm.close()  # every mapping closed before any owner frees its buffers
