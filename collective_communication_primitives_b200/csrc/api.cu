@@ -325,7 +325,7 @@ coll_status_t run_direct_reduce(sim_comm* c, const coll_bufs_t& b, size_t n, col
     a.vec = all_aligned(31) ? 2 : (all_aligned(15) ? 1 : 0);
     if (c->direct_pack == 16 && a.vec == 2) a.vec = 1;
     a.ctas_per_sm = int(c->direct_ctas_per_sm);
-    a.l2_hint = int(c->l2_hint);
+    a.l2_hint = c->l2_hint == 1 ? 1 : 0;  // the fused reduction hints its loads and stores together
     cudaError_t e = launch_direct_reduce(a, dt, op, c->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "direct reduction launch");
     c->launches += 1;
@@ -773,7 +773,7 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
         if (value < -1 || value > 1) return fail(COLL_ERR_INVALID_ARG, "copy_order must be -1, 0 or 1");
         c->copy_order = value;
     } else if (k == "l2_hint") {
-        if (value != 0 && value != 1) return fail(COLL_ERR_INVALID_ARG, "l2_hint must be 0 or 1");
+        if (value < 0 || value > 2) return fail(COLL_ERR_INVALID_ARG, "l2_hint must be 0, 1 or 2");
         c->l2_hint = value;
     } else if (k == "direct_pack") {
         if (value != 0 && value != 16 && value != 32) return fail(COLL_ERR_INVALID_ARG, "direct_pack must be 0, 16 or 32");

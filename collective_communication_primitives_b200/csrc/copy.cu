@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_copy(const __grid_constant__ C
         const TileGeom g = tile_geom(reinterpret_cast<uintptr_t>(d.src), d.len, cong, ti, kTile);
         if (lane == 0 && g.bhi > g.blo) {
             mbar_arrive_expect_tx(&bars[st], uint32_t(g.bhi - g.blo));
-            if (a.l2_hint)
+            if (a.l2_hint == 1)
                 bulk_g2s_hint(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st], pol);
             else
                 bulk_g2s(stages + size_t(st) * kTile, d.src + g.blo, uint32_t(g.bhi - g.blo), &bars[st]);
@@ -538,6 +538,7 @@ __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs 
     const uint32_t total = per_seg * uint32_t(KIND == COPY_BCAST ? 1 : p);
     for (int st = 0; st < kFanStages; ++st) mbar_init(&bars[st], 1);
     fence_barrier_init();
+    const uint64_t pol = a.l2_hint ? l2_evict_first_policy() : 0;  // on the stores only
     auto source = [&](uint32_t t) -> const char* {
         const uint32_t q = t / per_seg;
         return static_cast<const char*>(a.ptrs.send[KIND == COPY_BCAST ? a.root : int(q)]) +
@@ -576,7 +577,9 @@ __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs 
         const uint32_t bytes = tile_bytes(t);
         for (int r = 0; r < p; ++r) {
             char* dst = static_cast<char*>(a.ptrs.recv[r]) + dst_off;
-            if (dst != src) bulk_s2g(dst, stages + size_t(st) * kFanTile, bytes);
+            if (dst == src) continue;
+            if (a.l2_hint) bulk_s2g_hint(dst, stages + size_t(st) * kFanTile, bytes, pol);
+            else bulk_s2g(dst, stages + size_t(st) * kFanTile, bytes);
         }
         bulk_commit();
         ++tail;

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(32) k_probe_bulk_store(char* dst, size_t ntile
 constexpr int kProbeFan = 8;
 constexpr int kProbeFanStages = 4;
 constexpr uint32_t kProbeFanTile = 32 * 1024;
+constexpr uint64_t kProbeWaitNs = 1000000000ull;  // 1 s
 __device__ uint32_t g_probe_ctr;
 
 __global__ void __launch_bounds__(32) k_probe_fanout(char* dst, const char* src, size_t bytes, uint32_t ntiles) {
@@ -108,9 +109,14 @@ __global__ void __launch_bounds__(32) k_probe_fanout(char* dst, const char* src,
     while (more && head < kProbeFanStages - 1) issue();
     while (tail < head) {
         const int st = int(tail % kProbeFanStages);
-        // a load that never lands ends the probe (bounded: the probe has no error channel)
-        bool ok = false;
-        for (uint32_t it = 0; it < kMaxSpin && !ok; ++it) ok = mbar_try_wait(&bars[st], (phase >> st) & 1u);
+        // a load that has not landed after kProbeWaitNs of global time ends the probe (the probe has
+        // no error channel; its caller sees the time, not the data)
+        bool ok = mbar_try_wait(&bars[st], (phase >> st) & 1u);
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 1; !ok && it < kMaxSpin; ++it) {
+            ok = mbar_try_wait(&bars[st], (phase >> st) & 1u);
+            if (!ok && (it & 255u) == 0u && globaltimer_ns() - t0 > kProbeWaitNs) break;
+        }
         if (!ok) break;
         phase ^= 1u << st;
         for (int f = 0; f < kProbeFan; ++f)

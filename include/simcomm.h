@@ -211,7 +211,8 @@ const char* coll_status_string(coll_status_t status);
  *   "direct_ctas_per_sm"  CTAs per SM of the fused reduction (default 16); 0 = one pass, a CTA per
  *                  iteration's worth of positions
  *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
- *                  paths (data read or written once), 0 = none (default)
+ *                  paths (data read or written once), 2 = on the stores of the bulk-copy paths
+ *                  only, 0 = none (default; measured fastest)
  *   "moe_fused"    coll_moe_dispatch as one cooperative kernel (counting, prefix sums and the copy
  *                  with grid barriers between them; 1, the default, where the device supports
  *                  cooperative launches) or as three kernels (0)
