@@ -121,9 +121,13 @@ class RankComm(SC.SimComm):
         return r
 
     def _call(self, fn, *args, **kw):
+        """Every rank meets both barriers even when the library refuses the call (then the refusal is
+        raised after the second one), so the ranks stay in step."""
         self.sync()
-        fn(*args, **kw)
-        self.sync()
+        try:
+            fn(*args, **kw)
+        finally:
+            self.sync()
 
     # every rank passes the registered input pointers of all ranks and its own output pointer
     def allreduce(self, sends, recv, n, dtype, op="sum", algo="direct"):

@@ -174,3 +174,64 @@ def _leaver(rank, world, port, q):
 def test_a_rank_that_leaves_makes_the_next_call_time_out():
     res, _ = _spawn(_leaver, 2, timeout=180)
     assert res == {0: "timeout", 1: "left"}, res
+
+
+def _forms(rank, world, port, q):
+    """The in-place forms a rank view accepts (the root's own Broadcast and Scatter), the ones it
+    refuses (an output over an input a peer may still read), and the schedules it does not run."""
+    try:
+        _setup(rank, world, port, 60)
+        import numpy as np
+        import torch.distributed as dist
+
+        import oracle as O
+        from collective_communication_primitives_b200 import ranks
+        from collective_communication_primitives_b200 import simcomm as SC
+        from gpu_helpers import make_inputs, to_numpy, to_torch
+        p, m = world, 1031
+        n = p * m
+        ins = make_inputs("normal", p, n, "fp32", "ranks.forms")
+        comm = ranks.RankComm()
+        buf = ranks.SharedBuffer(n * 4)
+        buf.view("fp32", n).copy_(to_torch(ins[rank], "fp32"))
+        sends = comm.register(buf)
+        root = 1
+        out = ranks.SharedBuffer(n * 4)
+        # the root broadcasts in place (its output is its input); the others receive into their own
+        recv = buf.ptr if rank == root else out.ptr
+        comm.broadcast(sends, recv, root, n, "fp32")
+        got = to_numpy((buf if rank == root else out).view("fp32", n), "fp32")
+        assert np.array_equal(got.view(np.uint32), ins[root].view(np.uint32)), "broadcast"
+        # the root scatters in place: its block stays where it is
+        recv = buf.ptr + rank * m * 4 if rank == root else out.ptr
+        comm.scatter(sends, recv, root, n, "fp32")
+        got = to_numpy((buf.view("fp32", m, offset=rank * m) if rank == root else out.view("fp32", m)), "fp32")
+        want = O.scatter(ins[root], p, "fp32", root)[rank]
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), "scatter"
+        # refused, on every rank alike: an in-place AllReduce (peers still read the input) and a
+        # ring schedule
+        codes = []
+        for call in (lambda: comm.allreduce(sends, buf.ptr, n, "fp32"),
+                     lambda: comm.allreduce(sends, out.ptr, n, "fp32", algo="ring")):
+            try:
+                call()
+                codes.append(0)
+            except SC.SimCommError as e:
+                codes.append(e.status)
+        assert codes == [SC.INVALID_ARG, SC.UNSUPPORTED], codes
+        comm.sync()
+        comm.close()
+        dist.barrier()
+        buf.close()
+        out.close()
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except Exception as e:
+        import traceback
+        q.put((rank, f"{type(e).__name__}: {e}\n{traceback.format_exc()}"))
+
+
+def test_rank_view_forms_and_refusals():
+    res, codes = _spawn(_forms, 3)
+    assert all(v == "ok" for v in res.values()), res
+    assert codes == [0, 0, 0]
