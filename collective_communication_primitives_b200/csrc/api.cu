@@ -48,6 +48,8 @@ struct sim_comm {
     int ll_ctas_max = 0;
     char* moe = nullptr;            // MoE dispatch counting and prefix scratch
     size_t moe_cap = 0;             // bytes
+    int32_t* moe_acc = nullptr;     // fused MoE dispatch: per-(rank, expert) totals, zero between calls
+    size_t moe_acc_cap = 0;         // elements
     uint32_t epoch = 0;
     long long chunk_bytes = 1 << 20;
     long long ring_ctas = 0;
@@ -272,6 +274,24 @@ coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
     cudaError_t e = cudaMalloc(&c->moe, bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(MoE scratch)");
     c->moe_cap = bytes;
+    return COLL_OK;
+}
+
+// The fused dispatch sums its per-(rank, expert) totals into this array during counting, and the
+// call's last CTA zeroes it again, so it is allocated zeroed and kept apart from the scratch whose
+// layout changes with the call's shape.
+coll_status_t ensure_moe_acc(sim_comm* c, size_t count) {
+    if (count <= c->moe_acc_cap) return COLL_OK;
+    if (c->capturing) return grow_in_capture("MoE totals");
+    release_scratch(c, c->moe_acc);
+    c->moe_acc = nullptr;
+    c->moe_acc_cap = 0;
+    cudaError_t e = cudaMalloc(&c->moe_acc, count * sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(MoE totals)");
+    e = cudaMemset(c->moe_acc, 0, count * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();  // zeroed before any stream's next kernel
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(MoE totals)");
+    c->moe_acc_cap = count;
     return COLL_OK;
 }
 
@@ -1038,6 +1058,7 @@ coll_status_t sim_comm_destroy(sim_comm_t c) {
     if (c->flags) cudaFree(c->flags);
     if (c->stage) cudaFree(c->stage);
     if (c->moe) cudaFree(c->moe);
+    if (c->moe_acc) cudaFree(c->moe_acc);
     if (c->ll) cudaFree(c->ll);
     if (c->dstate) cudaFree(c->dstate);
     if (c->host_words) cudaFreeHost(c->host_words);
@@ -1113,6 +1134,7 @@ coll_status_t sim_comm_reset(sim_comm_t c) {
     if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset: device synchronisation");
     e = cudaMemset(c->dstate, 0, sizeof(DevState));
     if (e == cudaSuccess && c->flags) e = cudaMemset(c->flags, 0, c->flags_cap * sizeof(unsigned long long));
+    if (e == cudaSuccess && c->moe_acc) e = cudaMemset(c->moe_acc, 0, c->moe_acc_cap * sizeof(int32_t));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset");
     c->epoch = 0;
@@ -1576,6 +1598,10 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     a.cnt = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank);
     a.base = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + b_pe);
     a.cmat = reinterpret_cast<int32_t*>(c->moe + b_hist + b_rank + 2 * b_pe);
+    if (c->moe_fused) {
+        if ((st = ensure_moe_acc(c, size_t(p) * experts)) != COLL_OK) return st;
+        a.acc = c->moe_acc;
+    }
     a.expert_counts_out = expert_counts_dev;
     a.recv_counts_out = recv_counts_dev;
     a.tma = int(c->moe_tma);

@@ -227,6 +227,10 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned 
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
+// Add v with release semantics and no return value (the thread does not wait for the L2 round trip).
+__device__ __forceinline__ void red_release_add_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -21,9 +21,6 @@ struct DevState {
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
     unsigned long long abort_clock;  // global time of the last read of the host abort word
     unsigned long long moe_task;     // fused MoE dispatch: next token row to claim (zero between calls)
-    // fused MoE dispatch: grid barriers done so far, set by the last CTA to arrive; a 128-byte line
-    // of its own, so that the CTAs polling it do not queue behind the arrivals' atomics on moe_ctr
-    alignas(128) uint32_t moe_gen;
 };
 
 // What a kernel needs to report errors and notice an abort.
@@ -213,10 +210,12 @@ struct MoeArgs {
     size_t cap_rows;                 // rows of every receive buffer (dispatch) / expert-output buffer (combine)
     uint32_t ntiles;                 // counting tiles per rank, ceil(A / kMoeTile)
     int32_t* tile_hist;              // [p][ntiles][E] per-tile expert counts, then exclusive prefix over tiles
+                                     // (the fused dispatch lays it out [p][E][ntiles])
     int32_t* rank_in_tile;           // [p][A] rank of an assignment among its tile's same-expert ones
     int32_t* cnt;                    // [p][E] assignments from rank i to expert e
     int32_t* base;                   // [p][E] first receive row of (rank i, expert e) at the expert's owner
     int32_t* cmat;                   // fused dispatch: [p][p] rows from rank i to rank j
+    int32_t* acc;                    // fused dispatch: [p][E] totals summed during counting (zero between calls)
     long long* expert_counts_out;    // [p][E] or null
     long long* recv_counts_out;      // [p] or null
     int tma;                         // dispatch copy: 1 bulk copies through shared memory, 0 loads/stores

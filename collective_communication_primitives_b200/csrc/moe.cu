@@ -360,18 +360,26 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
 //
 // Three kernels cost the dispatch ~23 us of launches and tiny serial phases before the copy starts
 // (8 + 16 us under ncu on 8 x 8192 tokens). Here one cooperative launch (every CTA resident) runs
-//   phase 1  counting: the k_moe_count work, a (rank, tile) per CTA pass, grid-strided;
-//   phase 2  a warp per (rank, expert) column: exclusive prefix of the tile counts over tiles, the
-//            total cnt[i][e] and c[i][j] += cnt[i][e] (integer atomics: exact in any order);
-//   phase 3  every CTA turns c into R[i][j] = Σ_{q<i} c[q][j] in shared memory and checks every
-//            destination's capacity (the same decision everywhere); base[i][e] = R[i][j] + Σ of
-//            cnt[i][·] over the block's lower experts, built by every CTA in its shared memory when
-//            the table is small, else by a warp per (rank, destination) block in global memory
-//            (with a third barrier);
+//   phase 1  counting: the k_moe_count work, a (rank, tile) per CTA pass, grid-strided; on the short
+//            path (below) each tile's counts are also added into acc[i][e] (integer reductions:
+//            exact in any order);
+//   phase 2  (long path only) a warp per (rank, expert) column: exclusive prefix of the tile counts
+//            over tiles, the total cnt[i][e] and c[i][j] += cnt[i][e];
+//   phase 3  every CTA turns c into R[i][j] = sum over q < i of c[q][j] in shared memory (on the
+//            short path after summing c[i][j] from acc) and checks every destination's capacity (the
+//            same decision everywhere); base[i][e] = R[i][j] + the sum of cnt[i][.] over the block's
+//            lower experts, built by every CTA in its shared memory when the table is small, else by
+//            a warp per (rank, destination) block in global memory (with a third barrier);
 //   phase 4  the copy: warps claim batches of consecutive token rows in order and copy each row with
-//            32/16-byte loads and one store per slot;
-// with a bounded grid barrier between phases. Data other CTAs wrote in this kernel is read through
-// L2 (ld.global.cg): L1 is not coherent between SMs.
+//            32/16-byte loads and one store per slot. An assignment's row is base[i][e] + the count
+//            of e in rank i's earlier tiles + its rank in its own tile: on the long path the middle
+//            term is phase 2's prefix; on the short path the warp sums the earlier tiles' counts
+//            itself, in the round trip that fetches the in-tile rank.
+// with a bounded grid barrier between phases. The short path (base table in shared memory, at most
+// kShortMaxTiles tiles per rank) has no phase 2 and no second barrier: the chain of dependent L2
+// round trips before the copy starts is what a small dispatch costs. Data other CTAs wrote in this
+// kernel is read through L2 (ld.global.cg): L1 is not coherent between SMs. acc is zeroed again by
+// the call's last CTA (and by a reset after a failed call).
 // Build-time knobs of the copy phase (measured on B200; the defaults are the fastest found).
 #ifndef SIMCOMM_MOE_FUSED_UNROLL
 #define SIMCOMM_MOE_FUSED_UNROLL 8   // packs in flight per lane
@@ -383,6 +391,39 @@ constexpr int kFusedThreads = kMoeTile;  // a counting tile per CTA pass
 constexpr int kFusedUnroll = SIMCOMM_MOE_FUSED_UNROLL;
 constexpr int kWarpHistMaxE = 1024;      // per-warp counting histograms up to this many experts (32 KiB)
 constexpr int kSmemBaseMax = 8192;       // every CTA keeps base[p][E] in shared memory up to this many entries
+constexpr int kShortMaxTiles = 64;       // short path: tiles per rank (a lane sums at most two per lookup)
+constexpr int kLookGroup = 4;            // short path: lookups whose earlier-tile counts load in one round trip
+
+// Short path: the count of expert le in tiles [0, ltile) of rank li, for the lookup of every lane
+// below nlook (lane = batch row x slot width + slot; lanes without a lookup pass ltile = 0). Warp-
+// collective: the whole warp loads the earlier tiles' counts of kLookGroup lookups at once (at most
+// two per lane, as ltile <= kShortMaxTiles) and reduces each.
+__device__ __forceinline__ int earlier_tiles_count(const MoeArgs& a, int li, uint32_t ltile, int le, int nlook,
+                                                   int lane) {
+    int mine = 0;
+    for (int q0 = 0; q0 < nlook; q0 += kLookGroup) {
+        int v[kLookGroup][2];
+#pragma unroll
+        for (int q = 0; q < kLookGroup; ++q) {
+            const int src = (q0 + q) & 31;
+            const int qi = __shfl_sync(0xffffffffu, li, src);
+            const uint32_t qt = q0 + q < nlook ? __shfl_sync(0xffffffffu, ltile, src) : 0u;
+            const int qe = __shfl_sync(0xffffffffu, le, src);
+            const int32_t* col = a.tile_hist + (size_t(qi) * a.E + qe) * a.ntiles;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t t = uint32_t(lane + 32 * r);
+                v[q][r] = t < qt ? __ldcg(col + t) : 0;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kLookGroup; ++q) {
+            const int sum = int(__reduce_add_sync(0xffffffffu, unsigned(v[q][0] + v[q][1])));
+            if (lane == q0 + q) mine = sum;
+        }
+    }
+    return mine;
+}
 
 static size_t fused_smem_ints(int p, int E) {
     const size_t hist = E <= kWarpHistMaxE ? size_t(kFusedThreads / 32) * E : size_t(E);
@@ -390,24 +431,48 @@ static size_t fused_smem_ints(int p, int E) {
     return size_t(p) * p + p + std::max(hist, base);
 }
 
-// The k-th grid barrier of a call (k = 1, 2, ...): a CTA arrives on moe_ctr; the last of the k-th
-// round of arrivals publishes k in moe_gen, which the others poll (a line the arrivals do not touch:
-// with every CTA polling the arrival counter itself, the arrivals queued behind the polls and one
-// barrier took tens of microseconds).
+// The k-th grid barrier of a call (k = 1, 2, ...): every CTA adds 1 to moe_ctr with a release
+// reduction (no return value, so no round trip) and polls moe_ctr until k rounds of arrivals are in,
+// with a short sleep between polls. Measured on B200 with 296 CTAs: 1.4-1.8 us per barrier, against
+// 1.8-2.3 us when each arrival is an atomic with a return and the last one releases a separate word
+// (the serial L2 round trips set the cost; the kind of fence does not).
+constexpr unsigned kBarrierPollSleepNs = 100;
 __device__ __forceinline__ bool moe_grid_barrier(const MoeArgs& a, uint32_t k) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(&a.st->moe_ctr, 1u) == k * gridDim.x - 1) st_release_gpu(&a.st->moe_gen, k);
-        s_ok = wait_counter(a.ctl, &a.st->moe_gen, k, a.timeout_ns) && !status_failed(a.ctl);
+        red_release_add_gpu(&a.st->moe_ctr, 1u);
+        const uint32_t want = k * gridDim.x;
+        bool ok = false;
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 0; it < kMaxSpin; ++it) {
+            if (ld_acquire_gpu(&a.st->moe_ctr) >= want) {
+                ok = true;
+                break;
+            }
+            __nanosleep(kBarrierPollSleepNs);
+            if ((it & 255u) == 255u) {
+                if (status_failed(a.ctl)) break;
+                const uint64_t now = globaltimer_ns();
+                if (now - t0 > a.timeout_ns) {
+                    raise_status(a.ctl, COLL_ERR_TIMEOUT);
+                    break;
+                }
+                if (abort_requested(a.ctl, now)) {
+                    raise_status(a.ctl, COLL_ERR_ABORTED);
+                    break;
+                }
+            }
+        }
+        if (!ok && !status_failed(a.ctl)) raise_status(a.ctl, COLL_ERR_TIMEOUT);
+        s_ok = ok && !status_failed(a.ctl);
     }
     __syncthreads();
     return s_ok != 0;
 }
 
 template <int W>
-__global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __grid_constant__ MoeArgs a) {
+__global__ void __launch_bounds__(kFusedThreads, 2) k_moe_dispatch_fused(const __grid_constant__ MoeArgs a) {
     // dynamic shared memory: [p][p] c -> R, [p] column totals, then a region used first for the
     // counting histograms ([8][E] per-warp counts when E <= kWarpHistMaxE, else [E]) and then, when
     // p * E <= kSmemBaseMax, for the first rows base[p][E]
@@ -423,10 +488,11 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
     const bool warp_hist = a.E <= kWarpHistMaxE;
     const int hist_ints = warp_hist ? (kFusedThreads / 32) * a.E : a.E;
     const bool smem_base = p * a.E <= kSmemBaseMax;
+    const bool short_path = smem_base && a.ntiles <= uint32_t(kShortMaxTiles) && a.acc != nullptr;
     int* s_base = s_cnt;
 
     // ---- phase 1: counting ----
-    if (blockIdx.x == 0)
+    if (blockIdx.x == 0 && !short_path)
         for (int x = threadIdx.x; x < p * p; x += kFusedThreads) a.cmat[x] = 0;
     const uint32_t ntask = uint32_t(p) * a.ntiles;
     // this thread's expert id in the CTA's g-th tile (-1 past the end); the next tile's id is loaded
@@ -455,7 +521,7 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         const int leader = __ffs(same) - 1;
         const int below = __popc(same & ((1u << lane) - 1u));  // same-expert assignments before it in the warp
         int rank = 0;
-        int32_t* hist = a.tile_hist + (size_t(i) * a.ntiles + tile) * a.E;
+        int32_t* hist = a.tile_hist + size_t(i) * a.E * a.ntiles + tile;  // expert x at hist[x * ntiles]
         if (warp_hist) {
             // every warp counts its own experts, then an assignment's rank adds the counts of the
             // warps before it: no turn-taking
@@ -469,7 +535,8 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
                 int t = 0;
 #pragma unroll
                 for (int w = 0; w < kFusedThreads / 32; ++w) t += s_cnt[w * a.E + x];
-                hist[x] = t;
+                hist[size_t(x) * a.ntiles] = t;
+                if (short_path && t != 0) atomicAdd(a.acc + size_t(i) * a.E + x, t);
             }
         } else {
             for (int w = 0; w < kFusedThreads / 32; ++w) {  // warps in order: ranks follow assignment order
@@ -483,31 +550,34 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
                 }
                 __syncthreads();
             }
-            for (int x = threadIdx.x; x < a.E; x += kFusedThreads) hist[x] = s_cnt[x];
+            for (int x = threadIdx.x; x < a.E; x += kFusedThreads) {
+                hist[size_t(x) * a.ntiles] = s_cnt[x];
+                if (short_path && s_cnt[x] != 0) atomicAdd(a.acc + size_t(i) * a.E + x, s_cnt[x]);
+            }
         }
         if (valid) a.rank_in_tile[size_t(i) * a.A + asg] = rank;
     }
     if (!moe_grid_barrier(a, 1)) return;
 
-    // ---- phase 2: per (rank, expert) column, prefix over tiles, totals ----
+    // ---- phase 2 (long path): per (rank, expert) column, prefix over tiles, totals ----
     const uint32_t nwarps = gridDim.x * (kFusedThreads / 32);
     const uint32_t gw = blockIdx.x * (kFusedThreads / 32) + uint32_t(warp);
-    for (uint32_t col = gw; col < uint32_t(p) * uint32_t(a.E); col += nwarps) {
+    for (uint32_t col = gw; !short_path && col < uint32_t(p) * uint32_t(a.E); col += nwarps) {
         const int i = int(col / uint32_t(a.E)), e = int(col % uint32_t(a.E));
-        int32_t* colp = a.tile_hist + size_t(i) * a.ntiles * a.E + e;
+        int32_t* colp = a.tile_hist + (size_t(i) * a.E + e) * a.ntiles;
         int run = 0;
         for (uint32_t t0 = 0; t0 < a.ntiles; t0 += 32 * kScanChunks) {
             int v[kScanChunks];
 #pragma unroll
             for (int c = 0; c < kScanChunks; ++c) {
                 const uint32_t t = t0 + uint32_t(c * 32 + lane);
-                v[c] = t < a.ntiles ? __ldcg(colp + size_t(t) * a.E) : 0;
+                v[c] = t < a.ntiles ? __ldcg(colp + t) : 0;
             }
 #pragma unroll
             for (int c = 0; c < kScanChunks; ++c) {
                 const uint32_t t = t0 + uint32_t(c * 32 + lane);
                 const int incl = warp_incl_scan_i(v[c], lane);
-                if (t < a.ntiles) colp[size_t(t) * a.E] = run + incl - v[c];
+                if (t < a.ntiles) colp[t] = run + incl - v[c];
                 run += __shfl_sync(0xffffffffu, incl, 31);
             }
         }
@@ -517,11 +587,28 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
             if (a.expert_counts_out) a.expert_counts_out[size_t(i) * a.E + e] = run;
         }
     }
-    if (!moe_grid_barrier(a, 2)) return;
+    if (!short_path && !moe_grid_barrier(a, 2)) return;
 
     // ---- phase 3: R = exclusive column prefix of c, capacity check, first rows ----
-    for (int x = threadIdx.x; x < p * p; x += kFusedThreads) s_c[x] = __ldcg(a.cmat + x);
-    if (threadIdx.x == 0) s_flag = 0;
+    if (short_path) {
+        // the totals from acc, then c[i][j] = the sum of cnt[i][e] over rank j's experts
+        for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) s_base[x] = __ldcg(a.acc + x);
+        if (threadIdx.x == 0) s_flag = 0;
+        __syncthreads();
+        if (blockIdx.x == 0 && a.expert_counts_out)
+            for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) a.expert_counts_out[x] = s_base[x];
+        for (int blk = threadIdx.x; blk < p * p; blk += kFusedThreads) {
+            const int i = blk / p, j = blk % p;
+            int t = 0;
+            for (int e = j * a.E_loc; e < (j + 1) * a.E_loc; ++e) t += s_base[i * a.E + e];
+            s_c[blk] = t;
+        }
+    } else {
+        for (int x = threadIdx.x; x < p * p; x += kFusedThreads) s_c[x] = __ldcg(a.cmat + x);
+        if (smem_base)  // the totals too, in the same round trip
+            for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) s_base[x] = __ldcg(a.cnt + x);
+        if (threadIdx.x == 0) s_flag = 0;
+    }
     __syncthreads();
     for (int j = threadIdx.x; j < p; j += kFusedThreads) {
         int run = 0;
@@ -541,8 +628,6 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
     }
     if (smem_base) {
         // every CTA builds the whole table in its shared memory: no third barrier
-        for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) s_base[x] = __ldcg(a.cnt + x);
-        __syncthreads();
         for (int blk = threadIdx.x; blk < p * p; blk += kFusedThreads) {  // (rank, destination) blocks
             const int i = blk / p, j = blk % p;
             int run = s_c[i * p + j];
@@ -579,16 +664,24 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         u0 = __shfl_sync(0xffffffffu, u0, 0);
         if (u0 >= rows) break;
         const unsigned long long my_u = u0 + unsigned(my_b);
+        const bool look = my_s < a.k && my_b < per_batch && my_u < rows;
+        int i = 0, e = 0, in_tile = 0;
+        uint32_t tile = 0;
+        size_t asg = 0;
+        if (look) {
+            i = int(my_u / a.T);
+            asg = size_t(my_u % a.T) * a.k + my_s;
+            e = a.idx[i][asg];
+            tile = uint32_t(asg / kMoeTile);
+            in_tile = __ldcg(a.rank_in_tile + size_t(i) * a.A + asg);
+        }
+        const int earlier = short_path ? earlier_tiles_count(a, i, tile, e, per_batch * kslot, lane)
+                            : look    ? __ldcg(a.tile_hist + (size_t(i) * a.E + e) * a.ntiles + tile)
+                                      : 0;
         bool bad = false;
-        if (my_s < a.k && my_b < per_batch && my_u < rows) {
-            const int i = int(my_u / a.T);
-            const size_t t = size_t(my_u % a.T);
-            const size_t asg = t * a.k + my_s;
-            const int e = a.idx[i][asg];
+        if (look) {
             const int first = smem_base ? s_base[i * a.E + e] : __ldcg(a.base + size_t(i) * a.E + e);
-            const long long row = (long long)first +
-                                  __ldcg(a.tile_hist + (size_t(i) * a.ntiles + asg / kMoeTile) * a.E + e) +
-                                  __ldcg(a.rank_in_tile + size_t(i) * a.A + asg);
+            const long long row = (long long)first + earlier + in_tile;
             bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
             if (bad) raise_status(a.ctl, COLL_ERR_INTERNAL);
             if (a.pos[i]) a.pos[i][asg] = bad ? -1 : int32_t(row);
@@ -627,17 +720,22 @@ __global__ void __launch_bounds__(kFusedThreads) k_moe_dispatch_fused(const __gr
         }
         __syncwarp();  // the next batch rewrites this warp's destination rows
     }
-    // the last CTA out clears the call's counters
+    // the last CTA out clears the call's counters and totals (every CTA has read them by now)
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(&a.st->done_ctr, 1u) == gridDim.x - 1) {
+        s_flag = atomicAdd(&a.st->done_ctr, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (s_flag) {
+        if (short_path)
+            for (int x = threadIdx.x; x < p * a.E; x += kFusedThreads) a.acc[x] = 0;
+        if (threadIdx.x == 0) {
             a.st->moe_task = 0;
             a.st->moe_ctr = 0;
-            a.st->moe_gen = 0;
             a.st->done_ctr = 0;
-            __threadfence();
         }
+        __threadfence();
     }
 }
 

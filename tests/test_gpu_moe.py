@@ -111,6 +111,64 @@ def test_dispatch_parity(p, T, k, E, H, dtype, kind, offset, fused, tma):
         assert r_g[j].guards_intact()
 
 
+SHAPE_SEQUENCE = [
+    # p, T, k, E, H, dtype, routes: one communicator, in this order
+    (4, 4000, 4, 16, 8, "bf16", "zipf"),     # 63 counting tiles per rank: up to two earlier-tile loads per lane
+    (4, 300, 2, 8, 16, "fp32", "skew"),      # fewer experts: the totals array is partly reused
+    (4, 5000, 4, 16, 8, "bf16", "uniform"),  # 79 tiles per rank: the long path (prefix phase)
+    (4, 1000, 2, 4096, 4, "fp32", "uniform"),  # first-row table too large for shared memory
+    (4, 4000, 4, 16, 8, "bf16", "zipf"),     # the short path again, after both long forms
+    (2, 3000, 8, 64, 4, "int32", "skew"),    # fewer ranks, 8 slots per token (16 lookups per batch)
+]
+
+
+def test_fused_dispatch_shape_sequence_on_one_communicator():
+    """The fused dispatch keeps per-(rank, expert) totals between calls only as zeros: its short path
+    (at most 64 counting tiles per rank and a first-row table in shared memory) sums them during
+    counting and its last CTA clears them. Calls of changing shape on one communicator, short and long
+    paths interleaved, each bit-exact against the oracle; then an overflow (which leaves the totals
+    uncleared), a reset, and a short-path call that must again match."""
+    comm = SC.SimComm(SHAPE_SEQUENCE[0][0])
+    try:
+        for case_no, (p, T, k, E, H, dtype, kind) in enumerate(SHAPE_SEQUENCE):
+            if p != comm.p:  # a new communicator only where the rank count changes
+                comm.close()
+                comm = SC.SimComm(p)
+            ids = make_routes(p, T, k, E, kind, seed=100 + case_no)
+            xs = make_rows(p, T, H, dtype, f"moe.seq.{case_no}")
+            ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, dtype)
+            cap = int(ref["recv_counts"].max())
+            _, r_g, _, pos_t, ec, rc = dispatch_case(comm, xs, ids, E, cap, dtype)
+            assert comm.async_error() == SC.OK, case_no
+            np.testing.assert_array_equal(rc.cpu().numpy(), ref["recv_counts"], err_msg=str(case_no))
+            np.testing.assert_array_equal(ec.cpu().numpy(), ref["expert_counts"], err_msg=str(case_no))
+            for i in range(p):
+                np.testing.assert_array_equal(pos_t[i].cpu().numpy(), ref["pos"][i], err_msg=str(case_no))
+            for j in range(p):
+                n = int(ref["recv_counts"][j])
+                np.testing.assert_array_equal(r_g[j].numpy().reshape(cap, H)[:n], ref["recv"][j][:n],
+                                              err_msg=str(case_no))
+    finally:
+        comm.close()
+    p, T, k, E, H, dtype, kind = SHAPE_SEQUENCE[0]
+    ids = make_routes(p, T, k, E, kind, seed=100)
+    xs = make_rows(p, T, H, dtype, "moe.seq.0")
+    ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, dtype)
+    with SC.SimComm(p) as comm:
+        _, r_g, _, _, _, _ = dispatch_case(comm, xs, ids, E, int(ref["recv_counts"].max()) - 1, dtype)
+        assert comm.async_error() == SC.OVERFLOW
+        comm.reset()
+        cap = int(ref["recv_counts"].max())
+        _, r_g, _, pos_t, ec, rc = dispatch_case(comm, xs, ids, E, cap, dtype)
+        assert comm.async_error() == SC.OK
+        np.testing.assert_array_equal(ec.cpu().numpy(), ref["expert_counts"])
+        for i in range(p):
+            np.testing.assert_array_equal(pos_t[i].cpu().numpy(), ref["pos"][i])
+        for j in range(p):
+            n = int(ref["recv_counts"][j])
+            np.testing.assert_array_equal(r_g[j].numpy().reshape(cap, H)[:n], ref["recv"][j][:n])
+
+
 def combine_inputs(p, T, k, cap, H, dtype, seed):
     ys = make_rows(p, cap, H, dtype, f"moe.y.{seed}")
     w = S.moe_gate_weights(p, T, k, seed)
