@@ -1537,7 +1537,8 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     coll_status_t st = check_usable(c);
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
-    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "the MoE dispatch is not built for rank views");
+    if (c->rank >= 0 && !c->moe_fused)
+        return fail(COLL_ERR_UNSUPPORTED, "a rank view's MoE dispatch runs the fused kernel only (option moe_fused 1)");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
     if (recv_cap_rows > size_t(INT32_MAX)) return fail(COLL_ERR_INVALID_ARG, "recv_cap_rows must fit in int32");
     if ((st = check_rows(recv_cap_rows, hidden, "recv_cap_rows")) != COLL_OK) return st;
@@ -1551,9 +1552,10 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     for (int r = 0; r < p; ++r) {
         if ((st = check_ptr(x[r], tokens * row, d, "token")) != COLL_OK) return st;
         if ((st = check_ptr(topk_idx[r], A * 4, 4, "expert id")) != COLL_OK) return st;
-        if ((st = check_ptr(recv[r], recv_cap_rows * row, d, "recv")) != COLL_OK) return st;
         rs.push_back({uintptr_t(x[r]), uintptr_t(x[r]) + tokens * row, false, r});
         rs.push_back({uintptr_t(topk_idx[r]), uintptr_t(topk_idx[r]) + A * 4, false, r});
+        if (c->rank >= 0 && r != c->rank) continue;  // a rank view writes only its own outputs
+        if ((st = check_ptr(recv[r], recv_cap_rows * row, d, "recv")) != COLL_OK) return st;
         rs.push_back({uintptr_t(recv[r]), uintptr_t(recv[r]) + recv_cap_rows * row, true, r});
         if (route_pos) {
             if ((st = check_ptr(route_pos[r], A * 4, 4, "route_pos")) != COLL_OK) return st;
@@ -1580,11 +1582,13 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     a.A = A;
     a.cap_rows = recv_cap_rows;
     a.ntiles = uint32_t((A + kMoeTile - 1) / kMoeTile);
+    a.view_rank = c->rank;
     for (int r = 0; r < p; ++r) {
+        const bool own = c->rank < 0 || r == c->rank;
         a.src[r] = x[r];
         a.idx[r] = topk_idx[r];
-        a.dst[r] = recv[r];
-        a.pos[r] = route_pos ? route_pos[r] : nullptr;
+        a.dst[r] = own ? recv[r] : nullptr;
+        a.pos[r] = own && route_pos ? route_pos[r] : nullptr;
     }
     // scratch: tile counts [p][ntiles][E], in-tile ranks [p][A], totals and first rows [p][E] each,
     // the count matrix [p][p]
@@ -1625,7 +1629,6 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     if (st != COLL_OK) return st;
     if (!valid_dtype(dt)) return fail(COLL_ERR_INVALID_ARG, "unknown dtype");
     if (dt == COLL_INT32) return fail(COLL_ERR_UNSUPPORTED, "the weighted combine needs fp32 or bf16 rows");
-    if (c->rank >= 0) return fail(COLL_ERR_UNSUPPORTED, "the MoE combine is not built for rank views");
     if ((st = check_moe_shape(c, tokens, k, hidden, experts)) != COLL_OK) return st;
     if ((st = check_rows(y_rows, hidden, "y_rows")) != COLL_OK) return st;
     if (!y || !topk_idx || !route_pos || !topk_weight || !out) return fail(COLL_ERR_INVALID_ARG, "null buffer array");
@@ -1635,11 +1638,12 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     std::vector<Range> rs;
     for (int r = 0; r < p; ++r) {
         if ((st = check_ptr(y[r], y_rows * row, d, "expert output")) != COLL_OK) return st;
+        rs.push_back({uintptr_t(y[r]), uintptr_t(y[r]) + y_rows * row, false, r});
+        if (c->rank >= 0 && r != c->rank) continue;  // a rank view combines only its own tokens
         if ((st = check_ptr(topk_idx[r], A * 4, 4, "expert id")) != COLL_OK) return st;
         if ((st = check_ptr(route_pos[r], A * 4, 4, "route_pos")) != COLL_OK) return st;
         if ((st = check_ptr(topk_weight[r], A * 4, 4, "gate weight")) != COLL_OK) return st;
         if ((st = check_ptr(out[r], tokens * row, d, "out")) != COLL_OK) return st;
-        rs.push_back({uintptr_t(y[r]), uintptr_t(y[r]) + y_rows * row, false, r});
         rs.push_back({uintptr_t(topk_idx[r]), uintptr_t(topk_idx[r]) + A * 4, false, r});
         rs.push_back({uintptr_t(route_pos[r]), uintptr_t(route_pos[r]) + A * 4, false, r});
         rs.push_back({uintptr_t(topk_weight[r]), uintptr_t(topk_weight[r]) + A * 4, false, r});
@@ -1650,8 +1654,10 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     // a residual may be its own rank's output (out = residual + Σ w y, element by element), and
     // must not overlap any other output
     for (int r = 0; residual && r < p; ++r) {
+        if (c->rank >= 0 && r != c->rank) continue;
         const Range res{uintptr_t(residual[r]), uintptr_t(residual[r]) + tokens * row, false, r};
         for (int q = 0; q < p; ++q) {
+            if (c->rank >= 0 && q != c->rank) continue;
             const Range o{uintptr_t(out[q]), uintptr_t(out[q]) + tokens * row, true, q};
             if (overlap(res, o) && !(q == r && res.lo == o.lo))
                 return fail(COLL_ERR_INVALID_ARG, "a residual overlaps an output other than its own rank's");
@@ -1669,8 +1675,10 @@ static coll_status_t coll_moe_combine_impl(sim_comm_t c, const void* const* y, s
     a.H = hidden;
     a.A = A;
     a.cap_rows = y_rows;
+    a.view_rank = c->rank;
     for (int r = 0; r < p; ++r) {
         a.src[r] = y[r];
+        if (c->rank >= 0 && r != c->rank) continue;
         a.idx[r] = topk_idx[r];
         a.pos[r] = const_cast<int32_t*>(route_pos[r]);
         a.w[r] = topk_weight[r];

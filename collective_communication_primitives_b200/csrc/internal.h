@@ -219,6 +219,7 @@ struct MoeArgs {
     long long* expert_counts_out;    // [p][E] or null
     long long* recv_counts_out;      // [p] or null
     int tma;                         // dispatch copy: 1 bulk copies through shared memory, 0 loads/stores
+    int view_rank;                   // a rank view: the one rank whose outputs the call writes (-1: every rank)
     int fused;                       // dispatch: 1 one cooperative kernel (counting, sums and copy), 0 three
                                      // kernels (the copy chosen by tma)
     uint64_t timeout_ns;

@@ -685,7 +685,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) k_moe_dispatch_fused(const _
             bad = row < 0 || size_t(row) >= a.cap_rows;  // cannot happen after the capacity check
             if (bad) raise_status(a.ctl, COLL_ERR_INTERNAL);
             if (a.pos[i]) a.pos[i][asg] = bad ? -1 : int32_t(row);
-            s_dst[warp][lane] = bad ? nullptr : static_cast<char*>(a.dst[e / a.E_loc]) + size_t(row) * row_bytes;
+            const int owner = e / a.E_loc;
+            const bool mine = a.view_rank < 0 || owner == a.view_rank;  // a rank view copies to itself only
+            s_dst[warp][lane] = bad || !mine ? nullptr : static_cast<char*>(a.dst[owner]) + size_t(row) * row_bytes;
         }
         __syncwarp();
         if (!__any_sync(0xffffffffu, bad)) {
@@ -694,6 +696,11 @@ __global__ void __launch_bounds__(kFusedThreads, 2) k_moe_dispatch_fused(const _
                 if (u >= rows) break;
                 const char* s_row = static_cast<const char*>(a.src[int(u / a.T)]) + size_t(u % a.T) * row_bytes;
                 char* const* d = s_dst[warp] + b * kslot;
+                if (a.view_rank >= 0) {  // a row none of whose slots goes to this rank is not read
+                    bool any = false;
+                    for (int sl = 0; sl < a.k; ++sl) any = any || d[sl] != nullptr;
+                    if (!any) continue;
+                }
                 if constexpr (W > 0) {
                     constexpr size_t kPack = size_t(W) * 4;
                     const size_t npk = row_bytes / kPack;
@@ -704,6 +711,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) k_moe_dispatch_fused(const _
                             if (c0 + q * 32 < npk) v[q] = ld_stream_words<W>(s_row + (c0 + q * 32) * kPack);
                         for (int sl = 0; sl < a.k; ++sl) {
                             char* d_row = d[sl];
+                            if (a.view_rank >= 0 && !d_row) continue;
 #pragma unroll
                             for (int q = 0; q < kFusedUnroll; ++q)
                                 if (c0 + q * 32 < npk) st_words<W>(d_row + (c0 + q * 32) * kPack, v[q]);
@@ -713,7 +721,8 @@ __global__ void __launch_bounds__(kFusedThreads, 2) k_moe_dispatch_fused(const _
                     const size_t nu = row_bytes / 2;  // 2-byte units (every row is a whole number of them)
                     for (size_t c0 = lane; c0 < nu; c0 += 32) {
                         const uint16_t v = *reinterpret_cast<const uint16_t*>(s_row + c0 * 2);
-                        for (int sl = 0; sl < a.k; ++sl) *reinterpret_cast<uint16_t*>(d[sl] + c0 * 2) = v;
+                        for (int sl = 0; sl < a.k; ++sl)
+                            if (d[sl]) *reinterpret_cast<uint16_t*>(d[sl] + c0 * 2) = v;
                     }
                 }
             }
@@ -788,7 +797,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
     __shared__ const char* s_y[kCopyThreads / 32][kMoeMaxTopk];  // per warp: the token's k expert-output rows
     __shared__ float s_w[kCopyThreads / 32][kMoeMaxTopk];        // and their gate weights
     if (cta_failed(a.ctl)) return;
-    const int i = blockIdx.y;
+    const int i = a.view_rank >= 0 ? a.view_rank : int(blockIdx.y);  // a rank view combines its own tokens
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t d = size_t(Elem<DT>::kBytes);
     const char* const* ys = s_y[warp];
@@ -916,8 +925,9 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
 static dim3 token_grid(const MoeArgs& a, int num_sms, int resident_per_sm) {
     const size_t warps_per_cta = kCopyThreads / 32;
     const size_t want = (a.T + warps_per_cta - 1) / warps_per_cta;
-    const size_t per_rank = std::max<size_t>(1, size_t(num_sms) * size_t(std::max(resident_per_sm, 1)) / size_t(a.p));
-    return dim3(unsigned(std::max<size_t>(1, std::min(want, per_rank))), unsigned(a.p), 1u);
+    const size_t ranks = a.view_rank >= 0 ? 1 : size_t(a.p);  // a rank view: its own rank's tokens only
+    const size_t per_rank = std::max<size_t>(1, size_t(num_sms) * size_t(std::max(resident_per_sm, 1)) / ranks);
+    return dim3(unsigned(std::max<size_t>(1, std::min(want, per_rank))), unsigned(ranks), 1u);
 }
 
 template <typename K>
@@ -977,6 +987,7 @@ static bool cooperative_ok() {
 
 cudaError_t launch_moe_dispatch(const MoeArgs& a, int num_sms, cudaStream_t s, int* kernels_launched) {
     *kernels_launched = 0;
+    if (a.view_rank >= 0 && !(a.fused && cooperative_ok())) return cudaErrorNotSupported;  // views: fused only
     if (a.fused && cooperative_ok()) {
         *kernels_launched = 1;
         const size_t row_bytes = a.H * size_t(a.elem_bytes);

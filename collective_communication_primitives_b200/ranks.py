@@ -160,6 +160,36 @@ class RankComm(SC.SimComm):
         self._call(super().alltoallv, sends, self._outs(recv), counts, send_cap=send_cap, recv_cap=recv_cap,
                    algo=algo, recv_counts=recv_counts, dtype=dtype)
 
+    def moe_dispatch(self, xs, topk_idx, experts, recv, tokens, topk, hidden, dtype, recv_cap, route_pos=None,
+                     expert_counts=None, recv_counts=None):
+        """xs, topk_idx: every rank's registered token rows and expert ids (pointers); recv: this rank's
+        receive buffer [recv_cap][hidden], route_pos: this rank's [tokens][topk] int32 routing map or
+        None; expert_counts / recv_counts: this process's int64 [p][E] / [p] outputs or None."""
+        L = self._L
+
+        def go():
+            self._check(L.coll_moe_dispatch(
+                self._h, self._parr(xs), self._parr(topk_idx), tokens, topk, hidden, int(experts),
+                SC.DTYPES[dtype], self._parr(self._outs(recv)), recv_cap,
+                self._parr(self._outs(route_pos)) if route_pos is not None else None,
+                ctypes.c_void_p(SC._ptr(expert_counts)) if expert_counts is not None else None,
+                ctypes.c_void_p(SC._ptr(recv_counts)) if recv_counts is not None else None, SC._stream(None)))
+        self._call(go)
+
+    def moe_combine(self, ys, y_rows, topk_idx, route_pos, topk_weight, experts, out, tokens, topk, hidden, dtype,
+                    residual=None):
+        """ys: every rank's registered expert-output rows [y_rows][hidden]; topk_idx, route_pos,
+        topk_weight, out and residual (or None): this rank's own."""
+        L = self._L
+
+        def go():
+            self._check(L.coll_moe_combine(
+                self._h, self._parr(ys), y_rows, self._parr(self._outs(topk_idx)), self._parr(self._outs(route_pos)),
+                self._parr(self._outs(topk_weight)),
+                self._parr(self._outs(residual)) if residual is not None else None, tokens, topk, hidden,
+                int(experts), SC.DTYPES[dtype], self._parr(self._outs(out)), SC._stream(None)))
+        self._call(go)
+
     def close(self):
         for ptr in getattr(self, "_opened", []):
             self._L.sim_ipc_close(ctypes.c_void_p(ptr))

@@ -144,7 +144,8 @@ sim_comm_t sim_comm_create(int p);
  * (counts_dev: this process's device copy of the whole count matrix, identical on every rank;
  * send_cap and recv_cap: every rank's capacities; only this rank's blocks are copied), Scatter,
  * Gather, COLL_ALGO_DIRECT only (the other schedules wait on other ranks inside their kernels:
- * COLL_ERR_UNSUPPORTED, as for the MoE calls). Reduce and Gather enqueue nothing
+ * COLL_ERR_UNSUPPORTED), and the MoE dispatch (fused kernel only) and combine (see there).
+ * Reduce and Gather enqueue nothing
  * on a non-root rank. No output may overlap any rank's input (a peer may still be reading it), except
  * the root's own in-place Broadcast and Scatter forms. The ranks' calls are not synchronised by the
  * library: before a call every rank's inputs must be complete, and no rank may modify its input until
@@ -357,7 +358,12 @@ coll_status_t coll_alltoallv(sim_comm_t comm, coll_bufs_t bufs, const long long*
  * overlapping outputs or an output overlapping an input. Asynchronous errors: an expert id outside
  * [0, E) -> COLL_ERR_INVALID_ARG, a rank that would receive more than recv_cap_rows rows ->
  * COLL_ERR_OVERFLOW; in both cases no row is copied. The scratch for counting is owned by the
- * communicator. T = 0 only zeroes the count outputs. */
+ * communicator. T = 0 only zeroes the count outputs.
+ * On a rank view (sim_comm_create_rank) x and topk_idx hold every rank's buffers as this process
+ * maps them, recv and route_pos only this rank's entry (the others are ignored), and the count
+ * outputs are this process's own arrays; each rank counts every rank's assignments and copies the
+ * rows destined to itself, so its outputs equal the whole communicator's for this rank bit for bit.
+ * Needs option moe_fused = 1 (else COLL_ERR_UNSUPPORTED). */
 coll_status_t coll_moe_dispatch(sim_comm_t comm, const void* const* x, const int32_t* const* topk_idx, size_t tokens,
                                 int k, size_t hidden, int experts, coll_dtype_t dtype, void* const* recv,
                                 size_t recv_cap_rows, int32_t* const* route_pos, long long* expert_counts_dev,
@@ -375,7 +381,10 @@ coll_status_t coll_moe_dispatch(sim_comm_t comm, const void* const* x, const int
  *                may equal out[i] (in place).
  *   out          HOST array of p DEVICE pointers [T][H].
  * dtype fp32 or bf16 (int32 -> COLL_ERR_UNSUPPORTED). An expert id outside [0, E) or a route_pos
- * outside [0, y_rows) is reported asynchronously as COLL_ERR_INVALID_ARG (that token is skipped). */
+ * outside [0, y_rows) is reported asynchronously as COLL_ERR_INVALID_ARG (that token is skipped).
+ * On a rank view y holds every rank's expert outputs as this process maps them, and topk_idx,
+ * route_pos, topk_weight, residual and out only this rank's entry: the call combines this rank's
+ * tokens, reading the rows they were routed to where they lie. */
 coll_status_t coll_moe_combine(sim_comm_t comm, const void* const* y, size_t y_rows, const int32_t* const* topk_idx,
                                const int32_t* const* route_pos, const float* const* topk_weight,
                                const void* const* residual, size_t tokens, int k, size_t hidden, int experts,

@@ -118,7 +118,9 @@ SHAPE_SEQUENCE = [
     (4, 5000, 4, 16, 8, "bf16", "uniform"),  # 79 tiles per rank: the long path (prefix phase)
     (4, 1000, 2, 4096, 4, "fp32", "uniform"),  # first-row table too large for shared memory
     (4, 4000, 4, 16, 8, "bf16", "zipf"),     # the short path again, after both long forms
-    (2, 3000, 8, 64, 4, "int32", "skew"),    # fewer ranks, 8 slots per token (16 lookups per batch)
+    (2, 1500, 8, 64, 4, "int32", "skew"),    # short path, 8 slots per token: 16 lookups per batch
+    (2, 600, 4, 2048, 8, "fp32", "uniform"), # short path with more experts than per-warp histograms hold
+    (2, 3000, 8, 64, 4, "int32", "skew"),    # 94 tiles per rank: long path, 8 slots per token
 ]
 
 

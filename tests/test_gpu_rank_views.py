@@ -235,3 +235,80 @@ def test_rank_view_forms_and_refusals():
     res, codes = _spawn(_forms, 3)
     assert all(v == "ok" for v in res.values()), res
     assert codes == [0, 0, 0]
+
+
+def _moe(rank, world, port, dtype, q):
+    """The MoE dispatch and combine as rank views: each rank's dispatch reads every rank's token rows
+    and expert ids where they lie (IPC mappings) and writes only its own receive rows and routing
+    map; its combine reads the expert-output rows of every rank at its own tokens' routes. Both are
+    compared bit for bit with the oracle's result for this rank."""
+    try:
+        _setup(rank, world, port, 60)
+        import numpy as np
+        import torch
+        import torch.distributed as dist
+
+        import oracle as O
+        from collective_communication_primitives_b200 import ranks
+        from collective_communication_primitives_b200 import simcomm as SC
+        from collective_communication_primitives_b200 import synth as S
+        from gpu_helpers import to_numpy, to_torch
+        p = world
+        T, k, E, H = 700, 2, 4 * p, 40  # 6 counting tiles per rank
+        d = ranks.BYTES[dtype]
+        ids = S.moe_routes(p, T, E, k, 1.1, 5 + p)
+        xs = [S.normal(f"ranks.moe.x.{i}", T * H, 1.0, dtype).reshape(T, H) for i in range(p)]
+        ref = O.moe_dispatch(xs, list(ids), E, p * T * k, dtype)
+        cap = int(ref["recv_counts"].max())
+        comm = ranks.RankComm()
+        xbuf, ibuf, ybuf = ranks.SharedBuffer(T * H * d), ranks.SharedBuffer(T * k * 4), ranks.SharedBuffer(cap * H * d)
+        xbuf.view(dtype, T * H).copy_(to_torch(xs[rank].ravel(), dtype))
+        ibuf.view("int32", T * k).copy_(torch.from_numpy(np.ascontiguousarray(ids[rank].ravel(), dtype=np.int32)))
+        xp, ip, yp = comm.register(xbuf), comm.register(ibuf), comm.register(ybuf)
+        pos = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+        ec = torch.full((p, E), -1, dtype=torch.int64, device="cuda")
+        rc = torch.full((p,), -1, dtype=torch.int64, device="cuda")
+        comm.moe_dispatch(xp, ip, E, ybuf.ptr, T, k, H, dtype, cap, route_pos=pos.data_ptr(), expert_counts=ec,
+                          recv_counts=rc)
+        assert np.array_equal(rc.cpu().numpy(), ref["recv_counts"]), "recv_counts"
+        assert np.array_equal(ec.cpu().numpy(), ref["expert_counts"]), "expert_counts"
+        assert np.array_equal(pos.cpu().numpy(), ref["pos"][rank]), "route_pos"
+        nr = int(ref["recv_counts"][rank])
+        got = to_numpy(ybuf.view(dtype, nr * H), dtype).reshape(nr, H)
+        assert np.array_equal(got, ref["recv"][rank][:nr]), f"rank {rank}: received rows differ"
+        # combine: the received rows stand for the experts' outputs
+        ws = S.moe_gate_weights(p, T, k, 9)
+        res = [S.normal(f"ranks.moe.res.{i}", T * H, 1.0, dtype).reshape(T, H) for i in range(p)]
+        w_t = to_torch(ws[rank].ravel(), "fp32").view(T, k)
+        res_t = to_torch(res[rank].ravel(), dtype)
+        out = torch.empty_like(res_t)
+        comm.moe_combine(yp, cap, ibuf.ptr, pos.data_ptr(), w_t.data_ptr(), E, out.data_ptr(), T, k, H, dtype,
+                         residual=res_t.data_ptr())
+        want = O.moe_combine([r[:cap] for r in ref["recv"]], list(ids), list(ws), dtype, E, residual=res,
+                             acc="slotfold")[rank]
+        assert np.array_equal(to_numpy(out, dtype).reshape(T, H), want), f"rank {rank}: combine differs"
+        # the three-kernel dispatch is not built for rank views: refused on every rank, in step
+        comm.set_option("moe_fused", 0)
+        try:
+            comm.moe_dispatch(xp, ip, E, ybuf.ptr, T, k, H, dtype, cap)
+            raise AssertionError("the three-kernel dispatch ran on a rank view")
+        except SC.SimCommError as e:
+            assert e.status == SC.UNSUPPORTED, e.status
+        assert comm.async_error() == 0
+        comm.sync()
+        comm.close()
+        dist.barrier()
+        for b in (xbuf, ibuf, ybuf):
+            b.close()
+        dist.destroy_process_group()
+        q.put((rank, "ok"))
+    except Exception as e:  # reported to the parent
+        import traceback
+        q.put((rank, f"{type(e).__name__}: {e}\n{traceback.format_exc()}"))
+
+
+@pytest.mark.parametrize("world,dtype", [(2, "bf16"), (3, "fp32"), (4, "bf16")])
+def test_rank_view_moe_dispatch_and_combine_match_the_oracle(world, dtype):
+    res, codes = _spawn(_moe, world, dtype)
+    assert all(v == "ok" for v in res.values()), res
+    assert codes == [0] * world
