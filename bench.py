@@ -398,6 +398,47 @@ def time_e2e(comm, wl, make_ops, steps, warmup, stream, device):
     return start.elapsed_time(end), h2d, d2h
 
 
+def pcie_ceiling(device, nbytes=512 << 20, chunks=8, reps=3):
+    """The host link's copy rates on this machine, the denominator of the e2e leg: pinned host memory to
+    the device, the device to pinned host memory, and both directions at once on two streams (as the
+    e2e pipeline runs them), each over `nbytes` in `chunks` copies, median of `reps`. GB/s per
+    direction."""
+    import torch
+    n = nbytes // 4 // chunks
+    h_in = [torch.empty(n, dtype=torch.float32).pin_memory() for _ in range(chunks)]
+    h_out = [torch.empty(n, dtype=torch.float32).pin_memory() for _ in range(chunks)]
+    d_in = [torch.empty(n, dtype=torch.float32, device=device) for _ in range(chunks)]
+    d_out = [torch.zeros(n, dtype=torch.float32, device=device) for _ in range(chunks)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    cur = torch.cuda.current_stream()
+
+    def run(h2d, d2h):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for c in range(chunks):
+            if h2d:
+                with torch.cuda.stream(s_in):
+                    d_in[c].copy_(h_in[c], non_blocking=True)
+            if d2h:
+                with torch.cuda.stream(s_out):
+                    h_out[c].copy_(d_out[c], non_blocking=True)
+        cur.wait_stream(s_in)
+        cur.wait_stream(s_out)
+        e1.record(cur)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    out = {}
+    for name, h2d, d2h in (("h2d_GBps", 1, 0), ("d2h_GBps", 0, 1), ("both_GBps_per_direction", 1, 1)):
+        run(h2d, d2h)
+        ms = statistics.median(run(h2d, d2h) for _ in range(reps))
+        out[name] = round(chunks * n * 4 / (ms / 1e3) / 1e9, 1)
+    return out
+
+
 # ---------------------------------------------------------------------------------------------
 # MoE dispatch and combine on the MoE workload
 
@@ -1081,9 +1122,13 @@ def main():
         e_ms, h2d, d2h = time_e2e(comm, wl, make_ops, e_steps, 1, stream, device)
         if world > 1:
             e_ms = reduce_max(e_ms, device)
+        link = pcie_ceiling(device)
+        # the copies alone, both directions at once at the link's measured rate: the e2e step's floor
+        floor_ms = max(h2d, d2h) / (link["both_GBps_per_direction"] * 1e9) * 1e3
         e2e = {"value": job_gbps(world, eff_per_step, e_ms / e_steps), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / e_steps, 3),
-               "steps": e_steps,
+               "steps": e_steps, "host_link": link, "copy_floor_ms_per_step": round(floor_ms, 3),
+               "frac_of_copy_floor": round(floor_ms / (e_ms / e_steps), 4),
                "pipeline": "2 buffer sets: step k+1's host-to-device copies and step k-1's device-to-host "
                            "reads overlap step k's kernels; the first step's copies in and the last step's "
                            "reads out are inside the timed region"}
