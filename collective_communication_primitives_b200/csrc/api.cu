@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "internal.h"
@@ -68,6 +69,7 @@ struct sim_comm {
     bool capturing = false;               // the current call's stream is being captured into a graph
     bool captured_any = false;            // some call was captured: graphs may hold scratch pointers
     std::vector<void*> retired;           // scratch replaced after a capture, freed at destroy
+    std::vector<std::pair<int32_t*, size_t>> retired_acc;  // MoE totals among them (zeroed by a reset too)
     long long trace = 0;                  // 1: keep a record of every call (sim_comm_trace_read)
     std::vector<TraceSlot> trace_ring;    // the last kTraceCap calls
     unsigned long long trace_seq = 0;     // calls recorded so far
@@ -283,6 +285,8 @@ coll_status_t ensure_moe(sim_comm* c, size_t bytes) {
 coll_status_t ensure_moe_acc(sim_comm* c, size_t count) {
     if (count <= c->moe_acc_cap) return COLL_OK;
     if (c->capturing) return grow_in_capture("MoE totals");
+    // a graph captured earlier keeps using the old array; a reset after a failed replay clears it too
+    if (c->moe_acc && c->captured_any) c->retired_acc.push_back({c->moe_acc, c->moe_acc_cap});
     release_scratch(c, c->moe_acc);
     c->moe_acc = nullptr;
     c->moe_acc_cap = 0;
@@ -1135,6 +1139,8 @@ coll_status_t sim_comm_reset(sim_comm_t c) {
     e = cudaMemset(c->dstate, 0, sizeof(DevState));
     if (e == cudaSuccess && c->flags) e = cudaMemset(c->flags, 0, c->flags_cap * sizeof(unsigned long long));
     if (e == cudaSuccess && c->moe_acc) e = cudaMemset(c->moe_acc, 0, c->moe_acc_cap * sizeof(int32_t));
+    for (const auto& ra : c->retired_acc)
+        if (e == cudaSuccess) e = cudaMemset(ra.first, 0, ra.second * sizeof(int32_t));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "sim_comm_reset");
     c->epoch = 0;

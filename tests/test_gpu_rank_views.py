@@ -237,7 +237,7 @@ def test_rank_view_forms_and_refusals():
     assert codes == [0, 0, 0]
 
 
-def _moe(rank, world, port, dtype, q):
+def _moe(rank, world, port, dtype, T, q):
     """The MoE dispatch and combine as rank views: each rank's dispatch reads every rank's token rows
     and expert ids where they lie (IPC mappings) and writes only its own receive rows and routing
     map; its combine reads the expert-output rows of every rank at its own tokens' routes. Both are
@@ -254,7 +254,7 @@ def _moe(rank, world, port, dtype, q):
         from collective_communication_primitives_b200 import synth as S
         from gpu_helpers import to_numpy, to_torch
         p = world
-        T, k, E, H = 700, 2, 4 * p, 40  # 6 counting tiles per rank
+        k, E, H = 2, 4 * p, 40
         d = ranks.BYTES[dtype]
         ids = S.moe_routes(p, T, E, k, 1.1, 5 + p)
         xs = [S.normal(f"ranks.moe.x.{i}", T * H, 1.0, dtype).reshape(T, H) for i in range(p)]
@@ -307,8 +307,9 @@ def _moe(rank, world, port, dtype, q):
         q.put((rank, f"{type(e).__name__}: {e}\n{traceback.format_exc()}"))
 
 
-@pytest.mark.parametrize("world,dtype", [(2, "bf16"), (3, "fp32"), (4, "bf16")])
-def test_rank_view_moe_dispatch_and_combine_match_the_oracle(world, dtype):
-    res, codes = _spawn(_moe, world, dtype)
+@pytest.mark.parametrize("world,dtype,T", [(2, "bf16", 700), (3, "fp32", 700), (4, "bf16", 700),
+                                           (2, "fp32", 9000)])  # 6 counting tiles per rank; 71 (long path)
+def test_rank_view_moe_dispatch_and_combine_match_the_oracle(world, dtype, T):
+    res, codes = _spawn(_moe, world, dtype, T)
     assert all(v == "ok" for v in res.values()), res
     assert codes == [0] * world
