@@ -1616,6 +1616,7 @@ static coll_status_t coll_moe_dispatch_impl(sim_comm_t c, const void* const* x, 
     a.recv_counts_out = recv_counts_dev;
     a.tma = int(c->moe_tma);
     a.fused = int(c->moe_fused);
+    a.skip_cta = int(c->fault_skip_rank);
     a.timeout_ns = uint64_t(c->timeout_ns);
     a.st = c->dstate;
     a.ctl = make_ctl(c);

@@ -220,6 +220,8 @@ struct MoeArgs {
     long long* recv_counts_out;      // [p] or null
     int tma;                         // dispatch copy: 1 bulk copies through shared memory, 0 loads/stores
     int view_rank;                   // a rank view: the one rank whose outputs the call writes (-1: every rank)
+    int skip_cta;                    // fault injection: this CTA of the fused dispatch never arrives at its
+                                     // first grid barrier (-1 = off)
     int fused;                       // dispatch: 1 one cooperative kernel (counting, sums and copy), 0 three
                                      // kernels (the copy chosen by tma)
     uint64_t timeout_ns;

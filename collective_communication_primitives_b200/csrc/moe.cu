@@ -441,7 +441,7 @@ __device__ __forceinline__ bool moe_grid_barrier(const MoeArgs& a, uint32_t k) {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        red_release_add_gpu(&a.st->moe_ctr, 1u);
+        if (!(k == 1 && int(blockIdx.x) == a.skip_cta)) red_release_add_gpu(&a.st->moe_ctr, 1u);
         const uint32_t want = k * gridDim.x;
         bool ok = false;
         const uint64_t t0 = globaltimer_ns();

@@ -196,8 +196,9 @@ const char* coll_status_string(coll_status_t status);
  *                  LL word, a bulk copy) before the call gives up with COLL_ERR_TIMEOUT (default 2e9)
  *   "fault_skip_rank"  debugging: this rank is silenced (the ring and tree executors never signal
  *                  its chunks, the butterfly executor never counts its tasks, the LL kernels never
- *                  send its words), so a successor times out (-1 = off, the default). Host-side
- *                  fault injection only.
+ *                  send its words, and the fused MoE dispatch's CTA of this index never arrives at
+ *                  its first grid barrier), so the waits on it time out (-1 = off, the default).
+ *                  Host-side fault injection only.
  *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v)/Scatter/Gather: -1 = the
  *                  default (Broadcast and AllGather: 9 where the buffers allow it; the others: 6,
  *                  2 stages x 32 KiB, 3 CTAs per SM); 0..7 = a bulk-copy pipeline shape (stages x

@@ -80,3 +80,46 @@ def test_abort_stops_a_waiting_schedule(algo):
     assert c.async_error() == SC.OK
     assert np.array_equal(u[3].cpu().numpy(), np.full(n, float(p), np.float32))
     c.close()
+
+
+@pytest.mark.parametrize("mode", ["timeout", "abort"])
+def test_fused_moe_dispatch_barrier_wait_is_bounded(mode):
+    """The fused MoE dispatch's grid barrier: with fault_skip_rank = 1 its CTA 1 never arrives, so
+    every other CTA's wait runs out (COLL_ERR_TIMEOUT) or ends on sim_comm_abort (COLL_ERR_ABORTED)
+    and nothing is copied. The failed call leaves its per-(rank, expert) totals uncleared; after
+    sim_comm_reset the next dispatch matches the oracle exactly."""
+    import oracle
+
+    from collective_communication_primitives_b200 import synth as S
+    p, T, k, E, H = 4, 600, 2, 8, 16
+    ids = S.moe_routes(p, T, E, k, 1.1, 3)
+    xs = [S.normal(f"faults.moe.rank{r}", T * H, 1.0, "fp32").reshape(T, H) for r in range(p)]
+    ref = oracle.moe_dispatch(xs, list(ids), E, p * T * k, "fp32")
+    cap = int(ref["recv_counts"].max())
+    x = [torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda() for a in xs]
+    idx = [torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda() for a in ids]
+    recv = [torch.zeros(cap, H, device="cuda") for _ in range(p)]
+    c = SC.SimComm(p)
+    c.set_option("timeout_ns", 100_000_000 if mode == "timeout" else 5_000_000_000)
+    c.set_option("fault_skip_rank", 1)
+    t0 = time.time()
+    c.moe_dispatch(x, idx, E, recv)
+    if mode == "abort":
+        time.sleep(0.05)
+        c.abort()
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 4.0
+    assert c.async_error() == (SC.TIMEOUT if mode == "timeout" else SC.ABORTED)
+    assert all(int(torch.count_nonzero(g)) == 0 for g in recv), "a failed dispatch copied rows"
+    c.set_option("fault_skip_rank", -1)
+    c.reset()
+    pos = [torch.empty(T, k, dtype=torch.int32, device="cuda") for _ in range(p)]
+    c.moe_dispatch(x, idx, E, recv, route_pos=pos)
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    for j in range(p):
+        n = int(ref["recv_counts"][j])
+        assert np.array_equal(recv[j][:n].cpu().numpy(), ref["recv"][j][:n]), j
+    for i in range(p):
+        assert np.array_equal(pos[i].cpu().numpy(), ref["pos"][i]), i
+    c.close()
