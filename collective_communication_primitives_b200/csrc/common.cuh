@@ -403,6 +403,10 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // Wait until every committed bulk group has completed (writes performed).
+// Wait until at most the most recent bulk group is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_but_last() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // L2 policy that evicts the touched lines first (streaming data read or written once).

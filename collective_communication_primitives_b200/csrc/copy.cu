@@ -514,33 +514,39 @@ __global__ void __launch_bounds__(kLsuThreads, 2) k_copy_lsu(const __grid_consta
     if (threadIdx.x == 0) leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
 }
 
-// ---- lean fan-out: Broadcast and AllGather on 16-byte aligned buffers -------------------------------
+// ---- lean fan-out: Broadcast, AllGather (and the equal All-to-All) on 16-byte aligned buffers -------
 // The fan-out pattern with nothing else on the critical path (the loop of the bulk fan-out probe):
-// one lane issues everything; each segment (the root's buffer, or a rank's shard) is cut into whole
-// 32 KiB tiles, the last one shorter (a multiple of 16 bytes when the segment is); task t is tile
-// t % per_seg of segment t / per_seg, claimed in order; a tile is loaded once and stored to every
-// destination except the source itself (the in-place forms). Used when every buffer is 16-byte
-// aligned and the segment a whole number of 16-byte units, so no tile needs a byte head or tail.
-constexpr int kFanStages = 4;
+// one lane issues everything; each segment (the root's buffer, or a rank's shard; for All-to-All
+// block j of rank i, segment i * p + j) is cut into whole 32 KiB tiles, the last one shorter (a
+// multiple of 16 bytes when the segment is); task t is tile t % per_seg of segment t / per_seg,
+// claimed in order; a tile is loaded once and stored to every destination except the source itself
+// (the in-place forms; All-to-All has one destination). Used when every buffer is 16-byte aligned
+// and the segment a whole number of 16-byte units, so no tile needs a byte head or tail. LAG: before
+// a stage is reloaded, wait only until the stores of the tile before the one just stored have read
+// it (the stage being reloaded is that tile's), not for the latest tile's stores too.
 constexpr uint32_t kFanTile = 32 * 1024;
 
-template <int KIND>
+template <int KIND, bool LAG, int STAGES>
 __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs a) {
-    static_assert(KIND == COPY_BCAST || KIND == COPY_ALLGATHER, "fan-out collectives only");
+    static_assert(STAGES >= 2, "a stage is reloaded only after the tile before it was stored");
+    static_assert(KIND == COPY_BCAST || KIND == COPY_ALLGATHER || KIND == COPY_ALLTOALL, "lean copy kinds only");
     extern __shared__ __align__(128) unsigned char stages[];
-    __shared__ uint64_t bars[kFanStages];
-    __shared__ uint32_t s_task[kFanStages];
+    __shared__ uint64_t bars[STAGES];
+    __shared__ uint32_t s_task[STAGES];
     if (threadIdx.x != 0) return;
     if (status_failed(a.ctl)) return;
     const int p = a.p;
     const size_t seg_bytes = a.blk_elems * size_t(a.elem_bytes);
     const uint32_t per_seg = uint32_t((seg_bytes + kFanTile - 1) / kFanTile);
-    const uint32_t total = per_seg * uint32_t(KIND == COPY_BCAST ? 1 : p);
-    for (int st = 0; st < kFanStages; ++st) mbar_init(&bars[st], 1);
+    const uint32_t total = per_seg * uint32_t(KIND == COPY_BCAST ? 1 : KIND == COPY_ALLTOALL ? p * p : p);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
     fence_barrier_init();
     const uint64_t pol = a.l2_hint ? l2_evict_first_policy() : 0;  // on the stores only
     auto source = [&](uint32_t t) -> const char* {
         const uint32_t q = t / per_seg;
+        if constexpr (KIND == COPY_ALLTOALL)
+            return static_cast<const char*>(a.ptrs.send[int(q) / p]) + size_t(q % uint32_t(p)) * seg_bytes +
+                   size_t(t % per_seg) * kFanTile;
         return static_cast<const char*>(a.ptrs.send[KIND == COPY_BCAST ? a.root : int(q)]) +
                size_t(t % per_seg) * kFanTile;
     };
@@ -556,15 +562,15 @@ __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs 
             more = false;
             return;
         }
-        const int st = int(head % kFanStages);
+        const int st = int(head % STAGES);
         s_task[st] = t;
         mbar_arrive_expect_tx(&bars[st], tile_bytes(t));
         bulk_g2s(stages + size_t(st) * kFanTile, source(t), tile_bytes(t), &bars[st]);
         ++head;
     };
-    while (more && head < kFanStages - 1) issue();
+    while (more && head < STAGES - 1) issue();
     while (tail < head) {
-        const int st = int(tail % kFanStages);
+        const int st = int(tail % STAGES);
         if (!mbar_wait_bounded(a.ctl, &bars[st], (phase >> st) & 1u, a.timeout_ns)) {
             failed = true;  // a load that never lands: stop issuing (the error is recorded)
             break;
@@ -572,19 +578,29 @@ __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs 
         phase ^= 1u << st;
         const uint32_t t = s_task[st];
         const char* src = source(t);
-        const size_t dst_off = (KIND == COPY_ALLGATHER ? size_t(t / per_seg) * seg_bytes : 0) +
-                               size_t(t % per_seg) * kFanTile;
         const uint32_t bytes = tile_bytes(t);
-        for (int r = 0; r < p; ++r) {
-            char* dst = static_cast<char*>(a.ptrs.recv[r]) + dst_off;
-            if (dst == src) continue;
+        if constexpr (KIND == COPY_ALLTOALL) {
+            const uint32_t q = t / per_seg;  // block q % p of rank q / p goes to rank q % p, block q / p
+            char* dst = static_cast<char*>(a.ptrs.recv[int(q % uint32_t(p))]) + size_t(q / uint32_t(p)) * seg_bytes +
+                        size_t(t % per_seg) * kFanTile;
             if (a.l2_hint) bulk_s2g_hint(dst, stages + size_t(st) * kFanTile, bytes, pol);
             else bulk_s2g(dst, stages + size_t(st) * kFanTile, bytes);
+        } else {
+            const size_t dst_off = (KIND == COPY_ALLGATHER ? size_t(t / per_seg) * seg_bytes : 0) +
+                                   size_t(t % per_seg) * kFanTile;
+            for (int r = 0; r < p; ++r) {
+                char* dst = static_cast<char*>(a.ptrs.recv[r]) + dst_off;
+                if (dst == src) continue;
+                if (a.l2_hint) bulk_s2g_hint(dst, stages + size_t(st) * kFanTile, bytes, pol);
+                else bulk_s2g(dst, stages + size_t(st) * kFanTile, bytes);
+            }
         }
         bulk_commit();
         ++tail;
         if (more) {
-            bulk_wait_read_all();  // the next load reuses the stage task tail-1 was stored from
+            // the next load reuses the stage task tail-1 was stored from
+            if constexpr (LAG) bulk_wait_read_but_last();
+            else bulk_wait_read_all();
             issue();
         }
     }
@@ -702,17 +718,27 @@ static cudaError_t launch_kind(const CopyArgs& a, int num_sms, int variant, cuda
 }
 
 // Per-collective defaults, the fastest measured on B200 at the DP-bucket size (p = 8, 100 MiB per
-// rank) with tasks claimed in order, each row charged with its own write-back: every collective on
+// rank) with tasks claimed in order, each row charged with its own write-back. The general engine:
 // 2 stages of 32 KiB with 3 CTAs per SM, block after block (All-to-All 0.257 ms against 0.345-0.405
-// ms for the deeper 1-2 CTA shapes; Broadcast and AllGather 0.166-0.167 ms against 0.170-0.176;
-// All-to-Allv on the Zipf counts 0.266 ms against 0.276 on the load/store path and 0.282 in the
-// interleaved order).
+// ms for the deeper 1-2 CTA shapes; All-to-Allv on the Zipf counts 0.266 ms against 0.276 on the
+// load/store path and 0.282 in the interleaved order). On aligned buffers Broadcast and AllGather
+// take the lean fan-out (0.160-0.161 ms against 0.166-0.167; lagged stage reuse 0.162-0.165), and
+// the equal All-to-All the lean copy with lagged stage reuse, 4 stages, 1 CTA per SM (0.2546 ms
+// against 0.2578 for the general engine and 0.2547-0.2556 for the other lagged shapes; on the MoE
+// All-to-All, 8 x 8 MiB bf16 blocks per rank, 0.168-0.171 ms against 0.173; without the lag the
+// lean copy takes 0.277 ms: a lane that waits for each tile's store to leave shared memory before
+// reloading keeps too little in flight for a 1:1 copy).
 constexpr int kVariantLsu = kNumCopyShapes;
 constexpr int kVariantFan1 = kNumCopyShapes + 1;  // lean fan-out, 1 CTA per SM
 constexpr int kVariantFan2 = kNumCopyShapes + 2;  // lean fan-out, 2 CTAs per SM
+constexpr int kVariantFanLag1 = kNumCopyShapes + 3;  // lean, lagged stage reuse, 4 stages, 1 CTA per SM
+constexpr int kVariantFanLag2 = kNumCopyShapes + 4;  // lean, lagged, 3 stages, 2 CTAs per SM
+constexpr int kVariantFanLag3 = kNumCopyShapes + 5;  // lean, lagged, 6 stages, 1 CTA per SM
+constexpr int kVariantFanLag4 = kNumCopyShapes + 6;  // lean, lagged, 2 stages, 3 CTAs per SM
+constexpr int kVariantFan6 = kNumCopyShapes + 7;     // lean, 6 stages, 1 CTA per SM
 
 void copy_defaults(int kind, int* variant, int* order) {
-    *variant = (kind == COPY_BCAST || kind == COPY_ALLGATHER) ? kVariantFan1 : 6;
+    *variant = (kind == COPY_BCAST || kind == COPY_ALLGATHER) ? kVariantFan1 : kind == COPY_ALLTOALL ? kVariantFanLag1 : 6;
     *order = 0;
 }
 
@@ -721,31 +747,50 @@ static bool fanout_ok(const CopyArgs& a) {
     if ((a.blk_elems * size_t(a.elem_bytes)) % 16 != 0) return false;
     for (int r = 0; r < a.p; ++r) {
         if (reinterpret_cast<uintptr_t>(a.ptrs.recv[r]) % 16 != 0) return false;
-        if ((a.kind == COPY_ALLGATHER || r == a.root) && reinterpret_cast<uintptr_t>(a.ptrs.send[r]) % 16 != 0)
+        if ((a.kind != COPY_BCAST || r == a.root) && reinterpret_cast<uintptr_t>(a.ptrs.send[r]) % 16 != 0)
             return false;
     }
     return true;
 }
 
-template <int KIND>
+template <int KIND, bool LAG, int STAGES>
 static cudaError_t launch_fanout(const CopyArgs& a, int num_sms, int ctas_per_sm, cudaStream_t s) {
     static unsigned long long attr_set = 0;  // bit d: set on device d
     const unsigned long long bit = device_bit();
-    const size_t smem = size_t(kFanStages) * kFanTile;
+    const size_t smem = size_t(STAGES) * kFanTile;
     if (!(attr_set & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(k_fanout<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(k_fanout<KIND, LAG, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
         if (e != cudaSuccess) return e;
         attr_set |= bit;
     }
-    k_fanout<KIND><<<num_sms * ctas_per_sm, 32, smem, s>>>(a);
+    k_fanout<KIND, LAG, STAGES><<<num_sms * ctas_per_sm, 32, smem, s>>>(a);
     return cudaGetLastError();
 }
 
+template <bool LAG, int STAGES>
+static cudaError_t launch_lean(const CopyArgs& a, int num_sms, int cps, cudaStream_t s) {
+    switch (a.kind) {
+        case COPY_BCAST: return launch_fanout<COPY_BCAST, LAG, STAGES>(a, num_sms, cps, s);
+        case COPY_ALLGATHER: return launch_fanout<COPY_ALLGATHER, LAG, STAGES>(a, num_sms, cps, s);
+        default: return launch_fanout<COPY_ALLTOALL, LAG, STAGES>(a, num_sms, cps, s);
+    }
+}
+
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
-    if (variant == kVariantFan1 || variant == kVariantFan2) {
-        const int cps = variant == kVariantFan1 ? 1 : 2;
-        if (a.kind == COPY_BCAST && fanout_ok(a)) return launch_fanout<COPY_BCAST>(a, num_sms, cps, s);
-        if (a.kind == COPY_ALLGATHER && fanout_ok(a)) return launch_fanout<COPY_ALLGATHER>(a, num_sms, cps, s);
+    if (variant >= kVariantFan1 && variant <= kVariantFan6) {
+        const bool lean = (a.kind == COPY_BCAST || a.kind == COPY_ALLGATHER || a.kind == COPY_ALLTOALL) && fanout_ok(a);
+        if (lean) {
+            switch (variant) {
+                case kVariantFan1: return launch_lean<false, 4>(a, num_sms, 1, s);
+                case kVariantFan2: return launch_lean<false, 4>(a, num_sms, 2, s);
+                case kVariantFanLag1: return launch_lean<true, 4>(a, num_sms, 1, s);
+                case kVariantFanLag2: return launch_lean<true, 3>(a, num_sms, 2, s);
+                case kVariantFanLag3: return launch_lean<true, 6>(a, num_sms, 1, s);
+                case kVariantFanLag4: return launch_lean<true, 2>(a, num_sms, 3, s);
+                default: return launch_lean<false, 6>(a, num_sms, 1, s);
+            }
+        }
         variant = 6;  // other collectives, or unaligned buffers: the general engine
     }
     if (variant == kVariantLsu) {
@@ -764,6 +809,6 @@ cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_
     }
 }
 
-int copy_num_variants() { return kNumCopyShapes + 3; }
+int copy_num_variants() { return kNumCopyShapes + 8; }
 
 }  // namespace simcomm

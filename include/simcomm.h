@@ -200,11 +200,13 @@ const char* coll_status_string(coll_status_t status);
  *                  its first grid barrier), so the waits on it time out (-1 = off, the default).
  *                  Host-side fault injection only.
  *   "copy_variant" copy path of the direct Broadcast/AllGather/All-to-All(v)/Scatter/Gather: -1 = the
- *                  default (Broadcast and AllGather: 9 where the buffers allow it; the others: 6,
- *                  2 stages x 32 KiB, 3 CTAs per SM); 0..7 = a bulk-copy pipeline shape (stages x
- *                  tile bytes, CTAs per SM); 8 = the 16-byte load/store path (All-to-All(v) only);
- *                  9, 10 = the lean fan-out of Broadcast and AllGather (4 stages x 32 KiB, 1 or 2
- *                  CTAs per SM; 16-byte aligned buffers and whole 16-byte segments, else 6). Every
+ *                  default (Broadcast and AllGather: 9, the equal All-to-All: 11, where the buffers
+ *                  allow it; the others: 6, 2 stages x 32 KiB, 3 CTAs per SM); 0..7 = a bulk-copy
+ *                  pipeline shape (stages x tile bytes, CTAs per SM); 8 = the 16-byte load/store path
+ *                  (All-to-All(v) only); 9..15 = the lean copy of Broadcast, AllGather and the equal
+ *                  All-to-All (32 KiB tiles; 16-byte aligned buffers and whole 16-byte blocks, else 6):
+ *                  9, 10 = 4 stages, 1 or 2 CTAs per SM; 11..14 = with lagged stage reuse, 4 stages
+ *                  and 1 CTA per SM, 3 and 2, 6 and 1, 2 and 3; 15 = 6 stages, 1 CTA per SM. Every
  *                  copy path takes its tiles in order from a shared counter.
  *   "copy_order"   tile order of the direct copy paths: -1 = the default per collective,
  *                  1 = interleaved over all blocks, 0 = block after block
