@@ -38,7 +38,7 @@ ROOT_RANK = 2
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a row's kernel, from an
 # ncu capture of the current build, and the per-rank element count it was captured at.
-NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_187_432_704 + 1_415_354_880, 26_214_400)}
+NCU_TRAFFIC = {"allreduce_avg_fp32_ring": (2_184_816_640 + 1_417_508_352, 26_214_400)}
 SPACER_CYCLES = 4_000_000  # ~2 ms of a spinning kernel ahead of a timed region
 
 
