@@ -444,6 +444,37 @@ def test_synchronous_argument_errors():
     assert c.async_error() == SC.OK
 
 
+@pytest.mark.parametrize("p", [1, 4, 6])
+def test_zero_size_calls_are_no_ops(p):
+    """n = 0 (and an All-to-Allv of all-zero counts) is accepted by every collective and schedule and
+    touches no input or output; the All-to-Allv reports zero received elements."""
+    c = comm(p)
+    t = [torch.full((64,), 3.0, device="cuda") for _ in range(p)]
+    u = [torch.full((64,), 7.0, device="cuda") for _ in range(p)]
+    pow2 = p & (p - 1) == 0
+    for algo in ("direct", "ring", "tree", "dbtree", "ll", "tree_ll", "dbtree_ll") + (("rd", "hd", "rd_ll") if pow2 else ()):
+        for op in ("sum", "max"):
+            c.allreduce(t, u, op=op, algo=algo, n=0)
+    for algo in ("direct", "ring"):
+        c.reduce(t, u, p - 1, algo=algo, n=0)
+        c.broadcast(t, u, 0, algo=algo, n=0)
+        c.reduce_scatter(t, u, algo=algo, n=0)
+        c.allgather(t, u, algo=algo, n=0)
+        c.alltoall(t, u, algo=algo, n=0)
+        rc = torch.full((p,), -1, dtype=torch.int64, device="cuda")
+        c.alltoallv(t, u, torch.zeros((p, p), dtype=torch.int64, device="cuda"), algo=algo, recv_counts=rc)
+        torch.cuda.synchronize()
+        assert torch.equal(rc, torch.zeros_like(rc)), algo
+    c.reduce_scatter(t, u, algo="ll", n=0)
+    c.allgather(t, u, algo="ll", n=0)
+    c.scatter(t, u, 0, n=0)
+    c.gather(t, u, 0, n=0)
+    torch.cuda.synchronize()
+    assert c.async_error() == SC.OK
+    assert all(torch.equal(x, torch.full_like(x, 7.0)) for x in u)
+    assert all(torch.equal(x, torch.full_like(x, 3.0)) for x in t)
+
+
 def test_alltoallv_overflow_is_reported_and_nothing_is_copied():
     p = 3
     c = comm(p)
