@@ -60,7 +60,7 @@ struct sim_comm {
     long long copy_order = -1;
     long long direct_pack = 0;
     long long direct_ctas_per_sm = 16;
-    long long l2_hint = 0;
+    long long l2_hint = -1;
     long long ring_task_bytes = 0;  // bytes of the wire type one ring / tree task moves; 0 = by message size
     long long moe_tma = 0;          // MoE dispatch copy: 0 loads and stores (faster, measured), 1 bulk copies
     long long moe_fused = 1;        // MoE dispatch: 1 one cooperative kernel, 0 three kernels
@@ -386,9 +386,9 @@ coll_status_t run_copy(sim_comm* c, const coll_bufs_t& b, int kind, size_t blk_e
     if (c->copy_variant >= 0) variant = int(c->copy_variant);
     if (c->copy_order >= 0) order = int(c->copy_order);
     a.order = order;
-    a.l2_hint = int(c->l2_hint);
     a.st = c->dstate;
     a.only_dst_plus1 = only_dst + 1;
+    a.l2_hint = c->l2_hint >= 0 ? int(c->l2_hint) : copy_path_l2_hint(a, variant);
     a.ctl = make_ctl(c);
     cudaError_t e = launch_copy(a, c->num_sms, variant, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy engine launch");
@@ -797,7 +797,7 @@ coll_status_t set_option_impl(sim_comm* c, const char* key, long long value) {
         if (value < -1 || value > 1) return fail(COLL_ERR_INVALID_ARG, "copy_order must be -1, 0 or 1");
         c->copy_order = value;
     } else if (k == "l2_hint") {
-        if (value < 0 || value > 2) return fail(COLL_ERR_INVALID_ARG, "l2_hint must be 0, 1 or 2");
+        if (value < -1 || value > 2) return fail(COLL_ERR_INVALID_ARG, "l2_hint must be -1, 0, 1 or 2");
         c->l2_hint = value;
     } else if (k == "direct_pack") {
         if (value != 0 && value != 16 && value != 32) return fail(COLL_ERR_INVALID_ARG, "direct_pack must be 0, 16 or 32");

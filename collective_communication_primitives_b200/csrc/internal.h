@@ -239,6 +239,7 @@ cudaError_t launch_direct_reduce(const DirectReduceArgs& a, int dtype, int op, i
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s);
 int copy_num_variants();
 void copy_defaults(int kind, int* variant, int* order);
+int copy_path_l2_hint(const CopyArgs& a, int variant);  // the l2_hint a copy takes by default (option -1)
 cudaError_t launch_ring(const RingArgs& a, int dtype, int op, int ctas, cudaStream_t s);
 int ring_max_ctas(int num_sms);
 cudaError_t launch_ring_ll(const LLArgs& a, int dtype, int op, cudaStream_t s);

@@ -216,7 +216,8 @@ const char* coll_status_string(coll_status_t status);
  *                  iteration's worth of positions
  *   "l2_hint"      1 = evict-first L2 policy on the streaming loads and stores of the direct
  *                  paths (data read or written once), 2 = on the stores of the bulk-copy paths
- *                  only, 0 = none (default; measured fastest)
+ *                  only, 0 = none, -1 = per path (default; measured fastest): evict-first stores
+ *                  where the lean fan-out of Broadcast or AllGather runs, none elsewhere
  *   "moe_fused"    coll_moe_dispatch as one cooperative kernel (counting, prefix sums and the copy
  *                  with grid barriers between them; 1, the default, where the device supports
  *                  cooperative launches) or as three kernels (0)

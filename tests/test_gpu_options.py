@@ -16,7 +16,7 @@ OPTIONS = {
     "fault_skip_rank": ([-1, 0, P - 1], [-2, P]),
     "copy_variant": ([-1, 0, 8, 9, 15], [-2, 16]),
     "copy_order": ([-1, 0, 1], [-2, 2]),
-    "l2_hint": ([0, 1, 2], [-1, 3]),
+    "l2_hint": ([-1, 0, 1, 2], [-2, 3]),
     "direct_pack": ([0, 16, 32], [8, 64, -1]),
     "direct_ctas_per_sm": ([0, 16, 32], [-1, 33]),
     "ring_task_bytes": ([0, 4096, 64 << 20], [256, 4095, 4096 + 128, (64 << 20) + 256]),
