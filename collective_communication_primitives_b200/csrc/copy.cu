@@ -608,6 +608,47 @@ __global__ void __launch_bounds__(32) k_fanout(const __grid_constant__ CopyArgs 
     if (!failed) leave_tasks(&a.st->task_ctr, &a.st->done_ctr);
 }
 
+// ---- one-pass copy: the equal All-to-All with 32-byte loads and stores --------------------------------
+// A CTA per 32 KiB tile of a block (block j of rank i to rank j's block i, segment i * p + j, tiles in
+// address order): the grid holds every tile and the hardware hands CTAs to SMs in order as they free
+// up, as for the fused reduction's waves; each thread keeps its 4 x 32-byte loads in flight before its
+// stores. Used when every buffer is 32-byte aligned and the block a whole number of 32-byte units.
+constexpr int kPassThreads = 256;
+
+template <int UNROLL>  // tile = 256 threads x UNROLL x 32 bytes
+__global__ void __launch_bounds__(kPassThreads) k_a2a_pass(const __grid_constant__ CopyArgs a, uint32_t per_seg) {
+    constexpr uint32_t kPassTile = uint32_t(kPassThreads) * UNROLL * 32;
+    __shared__ int s_stop;
+    if (threadIdx.x == 0) s_stop = status_failed(a.ctl);
+    __syncthreads();
+    if (s_stop) return;
+    const size_t seg_bytes = a.blk_elems * size_t(a.elem_bytes);
+    const uint32_t q = blockIdx.x / per_seg;
+    const size_t off = size_t(blockIdx.x % per_seg) * kPassTile;
+    const char* src = static_cast<const char*>(a.ptrs.send[int(q) / a.p]) + size_t(q % uint32_t(a.p)) * seg_bytes + off;
+    char* dst = static_cast<char*>(a.ptrs.recv[int(q % uint32_t(a.p))]) + size_t(q / uint32_t(a.p)) * seg_bytes + off;
+    const size_t nvec = min(size_t(kPassTile), seg_bytes - off) / 32;
+    Words<8> v[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+        const size_t k = threadIdx.x + size_t(u) * kPassThreads;
+        if (k < nvec) v[u] = ld_stream_words<8>(src + k * 32);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+        const size_t k = threadIdx.x + size_t(u) * kPassThreads;
+        if (k < nvec) st_words<8>(dst + k * 32, v[u]);
+    }
+}
+
+static bool pass_ok(const CopyArgs& a) {
+    if ((a.blk_elems * size_t(a.elem_bytes)) % 32 != 0) return false;
+    for (int r = 0; r < a.p; ++r)
+        if (reinterpret_cast<uintptr_t>(a.ptrs.send[r]) % 32 != 0 || reinterpret_cast<uintptr_t>(a.ptrs.recv[r]) % 32 != 0)
+            return false;
+    return true;
+}
+
 // The current device as one bit of a mask (0 for devices 63 and up, which set the attribute every launch).
 static unsigned long long device_bit() {
     int dev = 0;
@@ -736,6 +777,9 @@ constexpr int kVariantFanLag2 = kNumCopyShapes + 4;  // lean, lagged, 3 stages, 
 constexpr int kVariantFanLag3 = kNumCopyShapes + 5;  // lean, lagged, 6 stages, 1 CTA per SM
 constexpr int kVariantFanLag4 = kNumCopyShapes + 6;  // lean, lagged, 2 stages, 3 CTAs per SM
 constexpr int kVariantFan6 = kNumCopyShapes + 7;     // lean, 6 stages, 1 CTA per SM
+constexpr int kVariantPass = kNumCopyShapes + 8;     // one-pass 32-byte load/store, 32 KiB per CTA (equal All-to-All)
+constexpr int kVariantPass64 = kNumCopyShapes + 9;   // the same, 64 KiB per CTA
+constexpr int kVariantPass16 = kNumCopyShapes + 10;  // the same, 16 KiB per CTA
 
 void copy_defaults(int kind, int* variant, int* order) {
     *variant = (kind == COPY_BCAST || kind == COPY_ALLGATHER) ? kVariantFan1 : kind == COPY_ALLTOALL ? kVariantFanLag1 : 6;
@@ -788,6 +832,23 @@ int copy_path_l2_hint(const CopyArgs& a, int variant) {
 }
 
 cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_t s) {
+    if (variant >= kVariantPass && variant <= kVariantPass16) {
+        if (a.kind == COPY_ALLTOALL && pass_ok(a)) {
+            const int unroll = variant == kVariantPass ? 4 : variant == kVariantPass64 ? 8 : 2;
+            const size_t tile = size_t(kPassThreads) * unroll * 32;
+            const size_t seg_bytes = a.blk_elems * size_t(a.elem_bytes);
+            const size_t per_seg = (seg_bytes + tile - 1) / tile;
+            const size_t grid = per_seg * size_t(a.p) * size_t(a.p);
+            if (grid == 0) return cudaSuccess;
+            if (grid <= 0x7fffffffu) {
+                if (unroll == 4) k_a2a_pass<4><<<unsigned(grid), kPassThreads, 0, s>>>(a, uint32_t(per_seg));
+                else if (unroll == 8) k_a2a_pass<8><<<unsigned(grid), kPassThreads, 0, s>>>(a, uint32_t(per_seg));
+                else k_a2a_pass<2><<<unsigned(grid), kPassThreads, 0, s>>>(a, uint32_t(per_seg));
+                return cudaGetLastError();
+            }
+        }
+        variant = 6;  // other collectives, or unaligned buffers: the general engine
+    }
     if (variant >= kVariantFan1 && variant <= kVariantFan6) {
         const bool lean = (a.kind == COPY_BCAST || a.kind == COPY_ALLGATHER || a.kind == COPY_ALLTOALL) && fanout_ok(a);
         if (lean) {
@@ -819,6 +880,6 @@ cudaError_t launch_copy(const CopyArgs& a, int num_sms, int variant, cudaStream_
     }
 }
 
-int copy_num_variants() { return kNumCopyShapes + 8; }
+int copy_num_variants() { return kNumCopyShapes + 11; }
 
 }  // namespace simcomm

@@ -206,8 +206,11 @@ const char* coll_status_string(coll_status_t status);
  *                  (All-to-All(v) only); 9..15 = the lean copy of Broadcast, AllGather and the equal
  *                  All-to-All (32 KiB tiles; 16-byte aligned buffers and whole 16-byte blocks, else 6):
  *                  9, 10 = 4 stages, 1 or 2 CTAs per SM; 11..14 = with lagged stage reuse, 4 stages
- *                  and 1 CTA per SM, 3 and 2, 6 and 1, 2 and 3; 15 = 6 stages, 1 CTA per SM. Every
- *                  copy path takes its tiles in order from a shared counter.
+ *                  and 1 CTA per SM, 3 and 2, 6 and 1, 2 and 3; 15 = 6 stages, 1 CTA per SM;
+ *                  16..18 = the equal All-to-All in one pass of 32-byte loads and stores, a CTA per
+ *                  32, 64 or 16 KiB tile (32-byte aligned buffers and whole 32-byte blocks, else 6).
+ *                  The bulk paths take their tiles in order from a shared counter; the one-pass
+ *                  grid is handed out in order by the hardware.
  *   "copy_order"   tile order of the direct copy paths: -1 = the default per collective,
  *                  1 = interleaved over all blocks, 0 = block after block
  *   "direct_pack"  access width of the fused reduction: 0 = widest the alignment allows

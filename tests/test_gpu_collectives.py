@@ -567,18 +567,19 @@ def test_launch_count_counts_kernels():
 
 
 @pytest.mark.parametrize("order", [-1, 0, 1])
-@pytest.mark.parametrize("variant", list(range(-1, 16)))
+@pytest.mark.parametrize("variant", list(range(-1, 19)))
 @pytest.mark.parametrize("p", [3, 8])
 def test_copy_engine_variants(variant, p, order):
     """Every copy path (the per-collective default, each bulk-copy pipeline shape, the load/store
     path and the lean copies of Broadcast, AllGather and All-to-All, with and without lagged stage
     reuse) in both tile orders gives the oracle's results. The lean copies need 16-byte aligned
-    buffers and whole 16-byte blocks (the 65,540-element case); the others fall back."""
+    buffers and whole 16-byte (one-pass: 32-byte) blocks, as in the 65,544-element case with its
+    short last tile; the others fall back."""
     c = comm(p)
     c.set_option("copy_variant", variant)
     c.set_option("copy_order", order)
     try:
-        for n, off in ((p * 7, 0), (p * 40961, 1), (p * 300007, 0), (p * 65540, 0)):
+        for n, off in ((p * 7, 0), (p * 40961, 1), (p * 300007, 0), (p * 65544, 0)):
             m = n // p
             ins = make_inputs("int24", p, n, "int32", f"cv.{p}.{n}")
             src = [Guarded(n, "int32", offset=off, fill=x) for x in ins]

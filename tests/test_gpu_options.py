@@ -14,7 +14,7 @@ OPTIONS = {
     "ring_ctas": ([0, 1, 65535], [-1, 65536]),
     "timeout_ns": ([1000, 2_000_000_000], [999, 0, -5]),
     "fault_skip_rank": ([-1, 0, P - 1], [-2, P]),
-    "copy_variant": ([-1, 0, 8, 9, 15], [-2, 16]),
+    "copy_variant": ([-1, 0, 8, 9, 18], [-2, 19]),
     "copy_order": ([-1, 0, 1], [-2, 2]),
     "l2_hint": ([-1, 0, 1, 2], [-2, 3]),
     "direct_pack": ([0, 16, 32], [8, 64, -1]),
