@@ -475,6 +475,40 @@ def test_zero_size_calls_are_no_ops(p):
     assert all(torch.equal(x, torch.full_like(x, 3.0)) for x in t)
 
 
+@pytest.mark.parametrize("hint", [-1, 0, 1, 2])
+def test_l2_policies_change_no_result(hint):
+    """Every L2 policy of option l2_hint (per path, none, evict-first loads and stores on the direct
+    paths, evict-first stores on the bulk copies) gives the oracle's results on the fused reduction's
+    32-byte path and the copy paths."""
+    p, n = 8, 8 * 65544
+    c = comm(p)
+    c.set_option("l2_hint", hint)
+    try:
+        ins = make_inputs("int24", p, n, "int32", f"l2.{hint}")
+        src = [Guarded(n, "int32", fill=x) for x in ins]
+        out = [Guarded(n, "int32") for _ in ins]
+        c.allreduce([b.t for b in src], [b.t for b in out], op="sum")
+        finish(c, src + out)
+        want = O.allreduce(ins, "int32", "sum")
+        for r in range(p):
+            np.testing.assert_array_equal(out[r].numpy(), want[r])
+        c.reduce_scatter([b.t for b in src], [b.t[: n // p] for b in out], op="max")
+        finish(c, out)
+        want = O.reduce_scatter(ins, "int32", "max")
+        for r in range(p):
+            np.testing.assert_array_equal(out[r].numpy()[: n // p], want[r])
+        c.broadcast([b.t for b in src], [b.t for b in out], 3)
+        finish(c, out)
+        for r in range(p):
+            np.testing.assert_array_equal(out[r].numpy(), ins[3])
+        c.alltoall([b.t for b in src], [b.t for b in out])
+        finish(c, out)
+        for r, w in enumerate(O.alltoall(ins, "int32")):
+            np.testing.assert_array_equal(out[r].numpy(), w)
+    finally:
+        c.set_option("l2_hint", -1)
+
+
 def test_alltoallv_overflow_is_reported_and_nothing_is_copied():
     p = 3
     c = comm(p)
