@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
 #define SIMCOMM_MOE_FUSED_UNROLL 8   // packs in flight per lane
 #endif
 #ifndef SIMCOMM_MOE_FUSED_BATCH
-#define SIMCOMM_MOE_FUSED_BATCH 2    // most token rows a warp claims at once (at most 32 / k rounded up)
+#define SIMCOMM_MOE_FUSED_BATCH 1    // most token rows a warp claims at once (at most 32 / k rounded up)
 #endif
 constexpr int kFusedThreads = kMoeTile;  // a counting tile per CTA pass
 constexpr int kFusedUnroll = SIMCOMM_MOE_FUSED_UNROLL;
