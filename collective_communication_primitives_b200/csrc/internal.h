@@ -21,6 +21,8 @@ struct DevState {
     uint32_t step_ctr[32];  // butterfly executor: finished tasks per step (zero between calls)
     unsigned long long abort_clock;  // global time of the last read of the host abort word
     unsigned long long moe_task;     // fused MoE dispatch: next token row to claim (zero between calls)
+    unsigned long long comb_task;    // MoE combine: next token to claim (zero between calls)
+    uint32_t comb_done;              // MoE combine: CTAs that left the token loop (the last one resets both)
 };
 
 // What a kernel needs to report errors and notice an abort.

@@ -797,12 +797,19 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
     __shared__ const char* s_y[kCopyThreads / 32][kMoeMaxTopk];  // per warp: the token's k expert-output rows
     __shared__ float s_w[kCopyThreads / 32][kMoeMaxTopk];        // and their gate weights
     if (cta_failed(a.ctl)) return;
-    const int i = a.view_rank >= 0 ? a.view_rank : int(blockIdx.y);  // a rank view combines its own tokens
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t d = size_t(Elem<DT>::kBytes);
     const char* const* ys = s_y[warp];
     const float* ws = s_w[warp];
-    for (size_t t = size_t(blockIdx.x) * (kCopyThreads / 32) + warp; t < a.T; t += size_t(gridDim.x) * (kCopyThreads / 32)) {
+    // warps claim tokens in order (rank-major) from a counter; a rank view combines its own tokens
+    const unsigned long long total = (a.view_rank >= 0 ? 1ull : (unsigned long long)a.p) * a.T;
+    while (true) {
+        unsigned long long u = 0;
+        if (lane == 0) u = status_failed(a.ctl) ? total : atomicAdd(&a.st->comb_task, 1ull);
+        u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= total) break;
+        const int i = a.view_rank >= 0 ? a.view_rank : int(u / a.T);
+        const size_t t = size_t(u % a.T);
         bool bad = false;
         if (lane < a.k) {
             const size_t asg = t * a.k + lane;
@@ -915,6 +922,16 @@ __global__ void __launch_bounds__(kCopyThreads) k_moe_combine(const __grid_const
             }
         }
         __syncwarp();  // the next token rewrites this warp's rows and weights
+    }
+    // the last CTA out resets the counter for the next call
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&a.st->comb_done, 1u) == gridDim.x * gridDim.y - 1) {
+            a.st->comb_task = 0;
+            a.st->comb_done = 0;
+            __threadfence();
+        }
     }
 }
 
@@ -1046,8 +1063,13 @@ cudaError_t launch_moe_combine(const MoeArgs& a, int dtype, int num_sms, cudaStr
         vec = vec && reinterpret_cast<uintptr_t>(a.src[r]) % 16 == 0 && reinterpret_cast<uintptr_t>(a.dst[r]) % 16 == 0;
         if (a.has_res) vec = vec && reinterpret_cast<uintptr_t>(a.res[r]) % 16 == 0;
     }
+    // one wave of resident CTAs whose warps claim tokens in order
     auto go = [&](auto kernel) {
-        kernel<<<token_grid(a, num_sms, resident_per_sm(kernel)), kCopyThreads, 0, s>>>(a);
+        const size_t warps_per_cta = kCopyThreads / 32;
+        const size_t tokens = a.T * size_t(a.view_rank >= 0 ? 1 : a.p);
+        const size_t want = (tokens + warps_per_cta - 1) / warps_per_cta;
+        const size_t wave = size_t(num_sms) * size_t(resident_per_sm(kernel));
+        kernel<<<unsigned(std::max<size_t>(1, std::min(want, wave))), kCopyThreads, 0, s>>>(a);
     };
     if (dtype == COLL_BF16) {
         if (vec) go(k_moe_combine<COLL_BF16, true>);
