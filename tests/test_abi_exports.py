@@ -173,3 +173,18 @@ def test_rank_view_and_ipc_entries_check_their_arguments_without_a_gpu(lib):
     assert L.sim_ipc_open(ctypes.byref(h), None) == SC.INVALID_ARG
     assert L.sim_ipc_free(None) == SC.OK and L.sim_ipc_close(None) == SC.OK
     assert ctypes.sizeof(SC.IpcHandle) == 64
+
+
+def test_header_documents_every_option_the_library_accepts():
+    """The option list in include/simcomm.h names exactly the keys the library takes (the key table
+    in csrc/api.cu, which sim_comm_create also reads from the environment)."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    header = open(os.path.join(root, "include", "simcomm.h")).read()
+    start = header.index("/* Options (each also read from the environment")
+    block = header[start:header.index("*/", start)]
+    documented = set(re.findall(r'^ \*   "([a-z0-9_]+)"', block, flags=re.M))
+    src = open(os.path.join(root, "collective_communication_primitives_b200", "csrc", "api.cu")).read()
+    table = src[src.index("kOptionKeys[] = {"):]
+    table = table[:table.index("};")]
+    accepted = set(re.findall(r'"([a-z0-9_]+)"', table))
+    assert documented == accepted, (sorted(documented - accepted), sorted(accepted - documented))
