@@ -49,6 +49,12 @@ def test_byte_model_pins():
     # "8 primitives" blog §6.2: TP AllReduce of one H = 8192 fp16 activation row over N = 8 ranks
     # moves about 2 * 8192 * 2 * 0.875 bytes = 28,672 B per rank.
     assert B.ring_wire_bytes_per_rank("allreduce", 8, 8192 * 2) == 28672
+    # the same page's MoE arithmetic: 1,024 tokens of H = 8192 fp16 per card, 63/64 of them routed
+    # away (64 destinations): 1008 * 2 * 8192 bytes sent per card, about 16 MB, and eight cards'
+    # worth, about 128 MB per layer
+    per_card = B.ring_wire_bytes_per_rank("alltoall", 64, 1024 * 2 * 8192)
+    assert per_card == 1008 * 2 * 8192 == 16_515_072
+    assert 8 * per_card == 132_120_576
     # Atlas §2.5 bus-bandwidth factors
     assert B.busbw_factor("allreduce", 8) == pytest.approx(1.75)
     assert B.busbw_factor("reduce_scatter", 4) == pytest.approx(0.75)
