@@ -49,7 +49,7 @@ def test_byte_model_pins():
     # "8 primitives" blog §6.2: TP AllReduce of one H = 8192 fp16 activation row over N = 8 ranks
     # moves about 2 * 8192 * 2 * 0.875 bytes = 28,672 B per rank.
     assert B.ring_wire_bytes_per_rank("allreduce", 8, 8192 * 2) == 28672
-    # the same page's MoE arithmetic: 1,024 tokens of H = 8192 fp16 per card, 63/64 of them routed
+    # the same section's MoE example: 1,024 tokens of H = 8192 fp16 per card, 63/64 of them routed
     # away (64 destinations): 1008 * 2 * 8192 bytes sent per card, about 16 MB, and eight cards'
     # worth, about 128 MB per layer
     per_card = B.ring_wire_bytes_per_rank("alltoall", 64, 1024 * 2 * 8192)
