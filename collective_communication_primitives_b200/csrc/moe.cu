@@ -13,7 +13,9 @@
 // Because all ranks share one memory, the pack and the exchange are one copy: every token row is
 // read once and written straight into the k receive rows its assignments own; the reverse
 // exchange, the unpermute and the weighted sum are likewise one pass that reads each token's k
-// expert-output rows where the experts left them. Kernels:
+// expert-output rows where the experts left them. The dispatch runs as one cooperative kernel,
+// k_moe_dispatch_fused (below); the three kernels it fuses remain for devices without cooperative
+// launches. Kernels:
 //   k_moe_count   one CTA per (rank, tile of 256 assignments): validates expert ids, counts them per
 //                 expert, and ranks every assignment among the tile's assignments of the same expert
 //                 (warps in order; __match_any_sync groups equal experts inside a warp);
@@ -23,7 +25,8 @@
 //   k_moe_dispatch_copy  one warp per token: the k destination rows (written to the routing map and
 //                 kept in shared memory for the warp), then 16/32-byte streaming loads of the token
 //                 row and k stores;
-//   k_moe_combine one warp per token: fp32 left fold in slot order (residual first), rounded once.
+//   k_moe_combine one warp per token, tokens claimed in order: fp32 left fold in slot order
+//                 (residual first), rounded once.
 #include <algorithm>
 
 #include "common.cuh"
