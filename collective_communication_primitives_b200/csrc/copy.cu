@@ -12,7 +12,10 @@
 // shared memory (completing on an mbarrier), then one cp.async.bulk store per destination. A
 // fan-out tile is thus read from HBM once and written p times. Bytes before the first and after
 // the last 16-byte boundary, and segments whose source and destination disagree modulo 16, are
-// copied by the warp with 2-byte loads and stores.
+// copied by the warp with 2-byte loads and stores. On aligned buffers Broadcast, AllGather and the
+// equal All-to-All take a lean form of the same pipeline (k_fanout: whole 32 KiB tiles, one lane,
+// nothing else on its path), and the equal All-to-All can also run as one pass of 32-byte loads
+// and stores (k_a2a_pass); All-to-All(v) also has a 16-byte load/store path (k_copy_lsu).
 //
 // Semantics ("集合通信：原语、算法、NCCL 实现与拓扑映射", llm-infra-atlas.github.io/hpc/04_collectives):
 // §1.1 Broadcast, §1.2 AllGather (rank-ordered concatenation), §1.6 AllToAll (block transpose);
