@@ -448,7 +448,7 @@ coll_status_t sim_hbm_probe(int kind, void* dst, const void* src, size_t bytes, 
  * (about p * n * 4 < 32 MiB, e.g. n up to ~1M elements at p = 8); larger calls return
  * COLL_ERR_INVALID_ARG with the sizes in sim_comm_last_error(). Other argument errors as for
  * coll_allreduce. The first call on a device looks up the scratch's device address on that device
- * and keeps it for the life of the process (make that first call before any stream capture); after
+ * and keeps it for the life of the process; after
  * cudaDeviceReset or any other teardown of the device's primary context that address is stale, so
  * do not call this entry point again in that process. Every call shares the scratch and clears what
  * must start at zero on its own stream; calls that overlap on the GPU race on it and must be
